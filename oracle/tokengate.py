@@ -1,0 +1,339 @@
+"""Plain float64 CPU oracle of the TokenGate hot path (test infrastructure only).
+
+Sources, cited below by tag (page title, then the section or figure used):
+  [fluxbbs]    "TokenGate 长上下文预填充提速 11.3 倍，斯坦福伯克利开源门控剪枝"
+  [digest]     "TokenGate: Adapting LLMs for Fast and Memory-Efficient Prefill with
+                Learned Token Pruning" (paper digest)
+  [farwalk]    "斯坦福与 UC Berkeley 提出 TokenGate：token 门控注意力让长上下文预填充最高快 11.3 倍"
+  [aiwillknow] "TokenGate：让模型学会跳读，而不只压缩 KV 缓存"
+
+What the pages fix, and what this oracle reads into the gaps (each reading is also
+listed with its reason in the design notes of the repository):
+  * gate at layer L: RMSNorm of the post-attention residual, a small scoring MLP
+    giving one scalar per token ([fluxbbs] 门控到底插在模型的哪个位置; [digest]
+    方法关键点; [farwalk] How does TokenGate learned token pruning work?).
+    Reading: MLP 2048 -> 256 -> 1, SiLU, no biases; RMSNorm eps 1e-6.
+  * scores RMSNorm-normalised along the sequence ([fluxbbs] same section).
+    Reading: the RMS runs over all tokens of the request, no gain, eps 1e-6.
+  * top-K over prunable (document) tokens only; question tokens are always kept
+    ([farwalk] same section; [digest] 方法关键点).  Reading: order "larger score
+    first, equal scores -> lower index first", NaN below every number, -0 == +0;
+    the budget counts every kept token, question included.
+  * kept tokens keep their original positions ([aiwillknow] 图1(a)(b)).
+  * token-gated attention: the kept token's score enters the upper layers' logits as
+    a per-key bias with a learnable per-head gain, plus an SSMax-style temperature
+    that rescales by the log-ratio of kept rank to original position ([fluxbbs]
+    端到端训练的关键在 token 门控注意力; [farwalk] What is token-gated attention?;
+    [aiwillknow] 图1(c)).  The formula adopted by this library:
+        logit[r, c] = tau_r * (q_r . k_c) / sqrt(d) + gamma_h * z_c     (c <= r)
+        tau_r       = beta * ln(r + 1) / ln(p_r + 1),   tau_r = beta when p_r = 0
+    with r the query's 0-based rank in the kept list, p_r its original position and
+    z_c = 0 for non-prunable keys.
+  * upper layers keep KV only for kept tokens ([farwalk] How does TokenGate learned
+    token pruning work?; [digest] 方法关键点).
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+
+__all__ = [
+    "as_f64", "rmsnorm_rows", "gate_score", "sequence_rmsnorm", "kept_counts",
+    "select_topk", "gather_rows", "rope", "rope_angles", "temperature",
+    "gated_attention", "kv_compact", "gated_layer", "prefill", "silu",
+]
+
+
+def as_f64(x) -> np.ndarray:
+    """Any torch tensor / array (bf16 included) as a float64 NumPy array, exactly."""
+    if hasattr(x, "detach"):
+        import torch  # local: the oracle itself needs only NumPy
+        x = x.detach().to("cpu")
+        if x.dtype in (torch.bfloat16, torch.float16):
+            x = x.to(torch.float32)
+        x = x.numpy()
+    return np.asarray(x, dtype=np.float64)
+
+
+def _as_int(x) -> np.ndarray:
+    if hasattr(x, "detach"):
+        x = x.detach().to("cpu").numpy()
+    return np.asarray(x, dtype=np.int64)
+
+
+def silu(u: np.ndarray) -> np.ndarray:
+    """u * sigmoid(u), written so that large |u| neither overflows nor loses the sign."""
+    out = np.empty_like(u)
+    pos = u >= 0
+    out[pos] = u[pos] / (1.0 + np.exp(-u[pos]))
+    e = np.exp(u[~pos])
+    out[~pos] = u[~pos] * e / (1.0 + e)
+    return out
+
+
+# ------------------------------------------------------------------ gate scoring
+
+def rmsnorm_rows(x, weight=None, eps: float = 1e-6) -> np.ndarray:
+    """x_t * w / sqrt(mean(x_t^2) + eps), row by row."""
+    x = as_f64(x)
+    inv = 1.0 / np.sqrt(np.mean(x * x, axis=-1, keepdims=True) + eps)
+    y = x * inv
+    if weight is not None:
+        y = y * as_f64(weight)
+    return y
+
+
+def gate_score(h, norm_w, W1, w2, eps: float = 1e-6) -> np.ndarray:
+    """Per-token gate score s_t = w2 . SiLU(W1 RMSNorm(h_t)).
+
+    [fluxbbs] 门控到底插在模型的哪个位置: a small MLP reads each token's normalised
+    residual and gives one scalar; [digest] 方法关键点 and [farwalk] How does TokenGate
+    learned token pruning work?: the residual is the post-attention residual at L.
+    W1 is stored [F, H] (output rows), w2 is [F].
+    """
+    x = rmsnorm_rows(h, norm_w, eps)
+    u = x @ as_f64(W1).T
+    return silu(u) @ as_f64(w2)
+
+
+def sequence_rmsnorm(s, cu_seqlens, prunable, eps: float = 1e-6):
+    """z_t = s_t / sqrt(mean_{t' in request} s_t'^2 + eps); bias_t = z_t on prunable tokens, else 0.
+
+    [fluxbbs] 门控到底插在模型的哪个位置: the scores are RMSNorm-normalised along the
+    sequence.  The mean runs over every token of the request.
+    """
+    s = as_f64(s)
+    cu = _as_int(cu_seqlens)
+    pr = _as_int(prunable).astype(bool)
+    z = np.empty_like(s)
+    for b in range(len(cu) - 1):
+        lo, hi = cu[b], cu[b + 1]
+        seg = s[lo:hi]
+        rms = math.sqrt(float(np.mean(seg * seg)) + eps) if hi > lo else 1.0
+        z[lo:hi] = seg / rms
+    bias = np.where(pr, z, 0.0)
+    return z, bias
+
+
+# ------------------------------------------------------------------ selection
+
+def kept_counts(prunable, cu_seqlens, budgets) -> np.ndarray:
+    """cu_kept from per-request budgets: K_b = Q_b + min(D_b, max(0, budget_b - Q_b)).
+
+    [farwalk] How do you deploy TokenGate?: the user gives a budget of kept prefill
+    tokens; [farwalk] How does TokenGate learned token pruning work?: the question
+    is never pruned.  The budget is read as counting every kept token.
+    """
+    cu = _as_int(cu_seqlens)
+    pr = _as_int(prunable).astype(bool)
+    out = [0]
+    for b in range(len(cu) - 1):
+        seg = pr[cu[b]:cu[b + 1]]
+        d = int(seg.sum())
+        q = int(seg.size - d)
+        kd = min(d, max(0, int(budgets[b]) - q))
+        out.append(out[-1] + q + kd)
+    return np.asarray(out, dtype=np.int64)
+
+
+def _selection_order(values: np.ndarray, index: np.ndarray) -> np.ndarray:
+    """Indices of `values` sorted by: numbers before NaN, larger first, lower index first."""
+    isnan = np.isnan(values)
+    neg = np.where(isnan, 0.0, -(values.astype(np.float64) + 0.0))  # + 0.0 maps -0 to +0
+    return np.lexsort((index, neg, isnan))
+
+
+def select_topk(z, prunable, cu_seqlens, cu_kept):
+    """Prunable-only top-K with the question kept, listed in original order.
+
+    For each request: among prunable tokens keep the Kd_b = K_b - Q_b best under the
+    order of `_selection_order`, add every non-prunable token, and list the kept
+    tokens by ascending position.  Decisions are taken on the float32 values given.
+    Returns (kept_idx [packed row id], kept_pos [position in request],
+    kept_bias [z on prunable rows, 0 on question rows]) with float32 bias.
+    [fluxbbs] 门控到底插在模型的哪个位置 (top-K, question never pruned);
+    [aiwillknow] 图1(a)(b) (original positions kept).
+    """
+    z32 = np.asarray(as_f64(z), dtype=np.float32) if not (
+        isinstance(z, np.ndarray) and z.dtype == np.float32) else z
+    cu = _as_int(cu_seqlens)
+    ck = _as_int(cu_kept)
+    pr = _as_int(prunable).astype(bool)
+    idx_out, pos_out, bias_out = [], [], []
+    for b in range(len(cu) - 1):
+        lo, hi = cu[b], cu[b + 1]
+        seg_z = z32[lo:hi]
+        seg_p = pr[lo:hi]
+        cand = np.nonzero(seg_p)[0]
+        keep_q = np.nonzero(~seg_p)[0]
+        kd = int(ck[b + 1] - ck[b]) - keep_q.size
+        if kd < 0 or kd > cand.size:
+            raise ValueError(f"request {b}: kept count {ck[b + 1] - ck[b]} inconsistent with mask")
+        order = _selection_order(seg_z[cand], cand)
+        chosen = cand[order[:kd]]
+        kept = np.sort(np.concatenate([chosen, keep_q]))
+        idx_out.append(lo + kept)
+        pos_out.append(kept)
+        bias_out.append(np.where(seg_p[kept], seg_z[kept], np.float32(0.0)).astype(np.float32))
+    cat = (lambda xs, dt: np.concatenate(xs).astype(dt) if xs else np.zeros(0, dt))
+    return cat(idx_out, np.int64), cat(pos_out, np.int64), cat(bias_out, np.float32)
+
+
+def gather_rows(h, idx) -> np.ndarray:
+    """Rows of h at the kept indices: pruned rows stop at the gate
+    ([fluxbbs] 门控到底插在模型的哪个位置)."""
+    return as_f64(h)[_as_int(idx)]
+
+
+# ------------------------------------------------------------------ RoPE, temperature
+
+def rope_angles(pos, head_dim: int, theta: float) -> np.ndarray:
+    """angle[r, i] = p_r * theta^(-2 i / head_dim), i < head_dim / 2, in float64."""
+    pos = _as_int(pos).astype(np.float64)
+    i = np.arange(head_dim // 2, dtype=np.float64)
+    inv_freq = theta ** (-2.0 * i / head_dim)
+    return pos[:, None] * inv_freq[None, :]
+
+
+def rope(x, pos, theta: float = 1.0e6) -> np.ndarray:
+    """Rotate-half rotary embedding of x [rows, heads, d] at positions pos [rows].
+
+    Pairs (i, i + d/2) rotate by angle p * theta^(-2i/d).  The kept rows use their
+    original positions ([aiwillknow] 图1(a)(b))."""
+    x = as_f64(x)
+    d = x.shape[-1]
+    half = d // 2
+    ang = rope_angles(pos, d, theta)[:, None, :]
+    c, s = np.cos(ang), np.sin(ang)
+    x1, x2 = x[..., :half], x[..., half:]
+    return np.concatenate([x1 * c - x2 * s, x2 * c + x1 * s], axis=-1)
+
+
+def temperature(rank, pos, beta: float) -> np.ndarray:
+    """tau = beta * ln(r + 1) / ln(p + 1); tau = beta where p = 0 (the limit r = p).
+
+    [fluxbbs] 端到端训练的关键在 token 门控注意力: a learnable temperature scaled by the
+    log-ratio of kept count to original position, after SSMax."""
+    r = _as_int(rank).astype(np.float64)
+    p = _as_int(pos).astype(np.float64)
+    out = np.full(r.shape, float(beta))
+    nz = p > 0
+    out[nz] = beta * np.log(r[nz] + 1.0) / np.log(p[nz] + 1.0)
+    return out
+
+
+# ------------------------------------------------------------------ attention
+
+def gated_attention(Q, K, V, cu_kept, kept_pos, kept_bias, gamma, beta,
+                    rows=None, block: int = 1024):
+    """Causal GQA attention over the kept rows with key bias and temperature.
+
+    Q [Kt, Hq, d], K/V [Kt, Hkv, d]; q head h reads kv head h // (Hq/Hkv).  Within
+    each request (rows cu_kept[b]..cu_kept[b+1]) query rank r attends to key ranks
+    c <= r with logits tau_r * q.k / sqrt(d) + gamma_h * bias_c, softmax over c.
+    Returns O [Kt, Hq, d] and the natural-log LSE [Hq, Kt] (float64).  With `rows`
+    (packed query row ids) only those rows are computed, others stay NaN.
+    [fluxbbs] 端到端训练的关键在 token 门控注意力; [farwalk] What is token-gated
+    attention?; [aiwillknow] 图1(c).
+    """
+    Q, K, V = as_f64(Q), as_f64(K), as_f64(V)
+    ck = _as_int(cu_kept)
+    pos = _as_int(kept_pos)
+    bias = as_f64(kept_bias)
+    gamma = as_f64(gamma)
+    Kt, Hq, d = Q.shape
+    Hkv = K.shape[1]
+    grp = Hq // Hkv
+    O = np.full(Q.shape, np.nan)
+    lse = np.full((Hq, Kt), np.nan)
+    want = None if rows is None else np.zeros(Kt, dtype=bool)
+    if want is not None:
+        want[_as_int(rows)] = True
+    for b in range(len(ck) - 1):
+        lo, hi = ck[b], ck[b + 1]
+        n = hi - lo
+        if n == 0:
+            continue
+        rank = np.arange(n)
+        tau = temperature(rank, pos[lo:hi], beta)
+        qsel = np.arange(n) if want is None else np.nonzero(want[lo:hi])[0]
+        for start in range(0, qsel.size, block):
+            qi = qsel[start:start + block]
+            if qi.size == 0:
+                continue
+            kmax = int(qi.max()) + 1
+            causal = np.arange(kmax)[None, :] <= qi[:, None]
+            for h in range(Hq):
+                g = h // grp
+                S = Q[lo + qi, h, :] @ K[lo:lo + kmax, g, :].T
+                logit = tau[qi, None] * S / math.sqrt(d) + gamma[h] * bias[None, lo:lo + kmax]
+                logit = np.where(causal, logit, -np.inf)
+                m = logit.max(axis=1, keepdims=True)
+                e = np.exp(logit - m)
+                den = e.sum(axis=1, keepdims=True)
+                O[lo + qi, h, :] = (e / den) @ V[lo:lo + kmax, g, :]
+                lse[h, lo + qi] = (m + np.log(den))[:, 0]
+    return O, lse
+
+
+def kv_compact(K, V, row_idx=None):
+    """Compacted KV cache rows: K and V of the kept rows only ([farwalk] How does
+    TokenGate learned token pruning work?: no KV entries for pruned tokens)."""
+    K, V = as_f64(K), as_f64(V)
+    if row_idx is None:
+        return K.copy(), V.copy()
+    i = _as_int(row_idx)
+    return K[i], V[i]
+
+
+# ------------------------------------------------------------------ one gated layer
+
+def gated_layer(x, Wqkv, Wo, gamma, beta, cu_kept, kept_pos, kept_bias,
+                n_q_heads: int, n_kv_heads: int, head_dim: int,
+                theta: float = 1.0e6, eps: float = 1e-6):
+    """One upper layer on the kept rows: x + Wo . Attn(RoPE(Wq a), RoPE(Wk a), Wv a), a = RMSNorm(x).
+
+    Wqkv [(Hq + 2 Hkv) d, H] holds Wq, Wk, Wv row blocks; Wo is [H, Hq d].  RoPE uses
+    the original positions.  Returns (x_out, K_cache, V_cache, parts) with the
+    intermediates in `parts` for teacher-forced checks.
+    """
+    x = as_f64(x)
+    a = rmsnorm_rows(x, None, eps)
+    qkv = a @ as_f64(Wqkv).T
+    nq, nk = n_q_heads * head_dim, n_kv_heads * head_dim
+    Kt = x.shape[0]
+    q = qkv[:, :nq].reshape(Kt, n_q_heads, head_dim)
+    k = qkv[:, nq:nq + nk].reshape(Kt, n_kv_heads, head_dim)
+    v = qkv[:, nq + nk:].reshape(Kt, n_kv_heads, head_dim)
+    q = rope(q, kept_pos, theta)
+    k = rope(k, kept_pos, theta)
+    o, lse = gated_attention(q, k, v, cu_kept, kept_pos, kept_bias, gamma, beta)
+    x_out = x + o.reshape(Kt, nq) @ as_f64(Wo).T
+    parts = {"a": a, "qkv": qkv, "q": q, "k": k, "v": v, "o": o, "lse": lse}
+    return x_out, k, v, parts
+
+
+def prefill(h, prunable, cu_seqlens, budgets, gate, layers, n_q_heads, n_kv_heads,
+            head_dim, theta=1.0e6, norm_eps=1e-6, seq_eps=1e-6, scores=None):
+    """Gate + selection + gathered upper layers, end to end.
+
+    `gate` holds norm_w, W1, w2; `layers` is a list of dicts with Wqkv, Wo, gamma,
+    beta.  With `scores` given, selection consumes those raw scores instead of the
+    scorer's (the planted-cluster workload).
+    """
+    s = gate_score(h, gate["norm_w"], gate["W1"], gate["w2"], norm_eps) if scores is None \
+        else as_f64(scores)
+    z, bias = sequence_rmsnorm(s, cu_seqlens, prunable, seq_eps)
+    cu_kept = kept_counts(prunable, cu_seqlens, budgets)
+    kept_idx, kept_pos, kept_bias = select_topk(z.astype(np.float32), prunable,
+                                                cu_seqlens, cu_kept)
+    x = gather_rows(h, kept_idx)
+    caches = []
+    for L in layers:
+        x, k, v, _ = gated_layer(x, L["Wqkv"], L["Wo"], L["gamma"], L["beta"], cu_kept,
+                                 kept_pos, kept_bias, n_q_heads, n_kv_heads, head_dim,
+                                 theta, norm_eps)
+        caches.append((k, v))
+    return {"s": s, "z": z, "bias": bias, "cu_kept": cu_kept, "kept_idx": kept_idx,
+            "kept_pos": kept_pos, "kept_bias": kept_bias, "x": x, "caches": caches}

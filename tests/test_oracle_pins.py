@@ -1,0 +1,386 @@
+"""Pins of the CPU oracle against things other than itself (no GPU needed).
+
+Each test checks an oracle function against a hand-derived closed form, brute force
+on tiny inputs, a library routine for a special case, or an invariant the
+mathematics fixes.  The cases are chosen so that a dropped term, a wrong sign,
+a wrong index or a transposed operand in the oracle fails at least one of them.
+"""
+import itertools
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+import torch.nn.functional as F
+
+import oracle as O
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _golden(name):
+    with open(os.path.join(GOLDEN, name)) as f:
+        return json.load(f)
+
+
+# ------------------------------------------------------------------ closed form
+
+def test_closed_form_normalisation_and_selection():
+    g = _golden("closed_form_4tok.json")
+    inp, exp = g["inputs"], g["expected"]
+    s = np.array(inp["s"])
+    pr = np.array(inp["prunable"])
+    cu = np.array([0, 4])
+    z, bias = O.sequence_rmsnorm(s, cu, pr, inp["eps_seq"])
+    c = exp["c"]
+    np.testing.assert_allclose(z, s * c, rtol=0, atol=1e-15)
+    np.testing.assert_allclose(bias, np.array([1.0, -1.0, 1.4, 0.0]) * c, atol=1e-15)
+    cu_kept = O.kept_counts(pr, cu, [inp["budget"]])
+    assert list(cu_kept) == [0, 3]
+    idx, pos, kb = O.select_topk(z.astype(np.float32), pr, cu, cu_kept)
+    assert list(pos) == exp["kept_pos"] and list(idx) == exp["kept_pos"]
+    np.testing.assert_allclose(kb, np.array(exp["kept_bias_over_c"]) * c, rtol=1e-7)
+
+
+def test_closed_form_temperature():
+    g = _golden("closed_form_4tok.json")
+    tau = O.temperature([0, 1, 2], g["expected"]["kept_pos"], g["inputs"]["beta"])
+    np.testing.assert_allclose(tau, g["expected"]["tau"], rtol=0, atol=1e-15)
+
+
+def _closed_form_attention(gamma, beta):
+    g = _golden("closed_form_4tok.json")
+    inp, exp = g["inputs"], g["expected"]
+    c = exp["c"]
+    Q = np.array(inp["q_by_rank"], dtype=np.float64)[:, None, :]
+    K = np.array(inp["k_by_rank"], dtype=np.float64)[:, None, :]
+    V = np.array(inp["v_by_rank"], dtype=np.float64)[:, None, :]
+    bias = np.array(exp["kept_bias_over_c"]) * c
+    out, lse = O.gated_attention(Q, K, V, [0, 3], exp["kept_pos"], bias, [gamma], beta)
+    return out[:, 0, :3], lse, exp
+
+
+def test_closed_form_attention_weights():
+    out, _, exp = _closed_form_attention(1.0, 1.0)
+    np.testing.assert_allclose(out, np.array(exp["weights"]), rtol=0, atol=1e-14)
+
+
+def test_closed_form_plain_causal():
+    out, _, exp = _closed_form_attention(0.0, 1.0)
+    # gamma = 0 removes the bias but tau still scales rank 2 by ln3/ln4
+    assert not np.allclose(out[2], exp["weights_rank2_gamma0_beta1"], atol=1e-6)
+    # with every position equal to its rank, tau = beta = 1: plain causal softmax
+    g = _golden("closed_form_4tok.json")
+    inp = g["inputs"]
+    Q = np.array(inp["q_by_rank"], dtype=np.float64)[:, None, :]
+    K = np.array(inp["k_by_rank"], dtype=np.float64)[:, None, :]
+    V = np.array(inp["v_by_rank"], dtype=np.float64)[:, None, :]
+    o2, _ = O.gated_attention(Q, K, V, [0, 3], [0, 1, 2], np.zeros(3), [0.0], 1.0)
+    np.testing.assert_allclose(o2[2, 0, :3], exp["weights_rank2_gamma0_beta1"], atol=1e-14)
+
+
+# ------------------------------------------------------------------ selection brute force
+
+def _brute_topk(z32, prunable, kd):
+    """Enumerate every kd-subset of prunable tokens; exactly one beats every dropped token."""
+    cand = [i for i in range(len(z32)) if prunable[i]]
+
+    def better(i, j):  # token i strictly ahead of token j
+        zi, zj = float(z32[i]), float(z32[j])
+        if math.isnan(zi) or math.isnan(zj):
+            if math.isnan(zi) and math.isnan(zj):
+                return i < j
+            return math.isnan(zj)
+        if zi != zj:
+            return zi > zj
+        return i < j
+
+    winners = []
+    for sub in itertools.combinations(cand, kd):
+        rest = [j for j in cand if j not in sub]
+        if all(better(i, j) for i in sub for j in rest):
+            winners.append(sub)
+    assert len(winners) == 1
+    kept = sorted(set(winners[0]) | {i for i in range(len(z32)) if not prunable[i]})
+    return kept
+
+
+@pytest.mark.parametrize("seed", range(40))
+def test_selection_brute_force(seed):
+    rng = np.random.default_rng(seed)
+    n = int(rng.integers(1, 11))
+    z = rng.normal(size=n).astype(np.float32)
+    if seed % 3 == 0:  # heavy ties
+        z = np.round(z * 2.0).astype(np.float32) / np.float32(2.0)
+    if seed % 5 == 0 and n > 2:
+        z[0] = np.float32(-0.0)
+        z[1] = np.float32(0.0)
+    if seed % 7 == 0 and n > 3:
+        z[2] = np.float32(np.nan)
+        z[3] = np.float32(-np.inf)
+    pr = (rng.random(n) < 0.7).astype(np.uint8)
+    d = int(pr.sum())
+    q = n - d
+    budget = int(rng.integers(0, n + 2))
+    cu_kept = O.kept_counts(pr, [0, n], [budget])
+    kd = int(cu_kept[1]) - q
+    assert kd == min(d, max(0, budget - q))
+    idx, pos, kb = O.select_topk(z, pr, [0, n], cu_kept)
+    assert list(pos) == _brute_topk(z, pr, kd)
+    for i, p in enumerate(pos):
+        want = z[p] if pr[p] else np.float32(0.0)
+        assert (np.isnan(want) and np.isnan(kb[i])) or kb[i] == want
+
+
+def test_selection_packed_requests_and_offsets():
+    z = np.array([0.5, 0.1, 0.9, -1.0, 3.0, 2.0, 2.0, 1.0, 0.0], dtype=np.float32)
+    pr = np.array([1, 1, 1, 0, 1, 1, 1, 1, 0], dtype=np.uint8)
+    cu = [0, 4, 9]
+    cu_kept = O.kept_counts(pr, cu, [2, 3])
+    assert list(cu_kept) == [0, 2, 5]
+    idx, pos, kb = O.select_topk(z, pr, cu, cu_kept)
+    # request 0: question token 3 plus best doc token 2
+    # request 1: question token 8 plus tokens 0 (3.0) and 1 (2.0, lower index of the tie)
+    assert list(idx) == [2, 3, 4, 5, 8]
+    assert list(pos) == [2, 3, 0, 1, 4]
+    np.testing.assert_array_equal(kb, np.array([0.9, 0.0, 3.0, 2.0, 0.0], dtype=np.float32))
+
+
+def test_kept_counts_rules():
+    pr = np.array([1] * 6 + [0] * 2, dtype=np.uint8)
+    cu = [0, 8]
+    assert list(O.kept_counts(pr, cu, [0])) == [0, 2]      # budget below question size
+    assert list(O.kept_counts(pr, cu, [5])) == [0, 5]
+    assert list(O.kept_counts(pr, cu, [100])) == [0, 8]    # budget above request size
+
+
+def test_selection_scale_invariance():
+    rng = np.random.default_rng(3)
+    s = rng.normal(size=200)
+    pr = (rng.random(200) < 0.8).astype(np.uint8)
+    cu = [0, 200]
+    ck = O.kept_counts(pr, cu, [60])
+    z1, _ = O.sequence_rmsnorm(s, cu, pr, 0.0)
+    z2, _ = O.sequence_rmsnorm(s * 7.5, cu, pr, 0.0)
+    np.testing.assert_allclose(z1, z2, rtol=1e-13)
+    a = O.select_topk(z1.astype(np.float32), pr, cu, ck)[0]
+    b = O.select_topk(z2.astype(np.float32), pr, cu, ck)[0]
+    assert np.array_equal(a, b)
+    # every question token kept, kept positions strictly increasing
+    idx, pos, _ = O.select_topk(z1.astype(np.float32), pr, cu, ck)
+    assert set(np.nonzero(pr == 0)[0]) <= set(idx.tolist())
+    assert np.all(np.diff(pos) > 0) and len(idx) == ck[1]
+
+
+def test_sequence_rmsnorm_per_request():
+    s = np.array([3.0, 4.0, 1.0, 1.0, 1.0])
+    z, _ = O.sequence_rmsnorm(s, [0, 2, 5], np.ones(5), 0.0)
+    np.testing.assert_allclose(z, [3 / math.sqrt(12.5), 4 / math.sqrt(12.5), 1, 1, 1])
+
+
+# ------------------------------------------------------------------ scorer
+
+def test_gate_score_against_library_special_case():
+    """W1 selecting input channels turns the scorer into sum_f w2_f SiLU(RMSNorm(h)[perm_f])."""
+    H, Fw, T = 12, 5, 7
+    g = torch.Generator().manual_seed(11)
+    h = torch.randn((T, H), generator=g, dtype=torch.float64) * 3.0
+    norm_w = torch.rand((H,), generator=g, dtype=torch.float64) + 0.5
+    perm = [7, 0, 11, 3, 3]
+    W1 = torch.zeros((Fw, H), dtype=torch.float64)
+    for f, j in enumerate(perm):
+        W1[f, j] = 1.0
+    w2 = torch.tensor([0.5, -1.25, 2.0, 0.75, -0.3], dtype=torch.float64)
+    want = F.silu(F.rms_norm(h, (H,), weight=norm_w, eps=1e-6))[:, perm] @ w2
+    got = O.gate_score(h, norm_w, W1, w2, 1e-6)
+    np.testing.assert_allclose(got, want.numpy(), rtol=1e-13, atol=1e-13)
+
+
+def test_gate_score_row_scale_invariance_and_general_mlp():
+    rng = np.random.default_rng(5)
+    H, Fw = 16, 6
+    h = rng.normal(size=(9, H))
+    W1 = rng.normal(size=(Fw, H))
+    w2 = rng.normal(size=Fw)
+    s1 = O.gate_score(h, None, W1, w2, 0.0)
+    s2 = O.gate_score(h * 13.0, None, W1, w2, 0.0)
+    np.testing.assert_allclose(s1, s2, rtol=1e-12)
+    # general weights against torch's Linear + SiLU + RMSNorm stack
+    ht = torch.tensor(h)
+    want = F.linear(F.silu(F.linear(F.rms_norm(ht, (H,), eps=1e-6), torch.tensor(W1))),
+                    torch.tensor(w2)[None, :])[:, 0]
+    np.testing.assert_allclose(O.gate_score(h, None, W1, w2, 1e-6), want.numpy(), rtol=1e-12)
+
+
+# ------------------------------------------------------------------ RoPE
+
+def test_rope_matches_complex_rotation():
+    rng = np.random.default_rng(9)
+    d, theta = 16, 1.0e6
+    x = rng.normal(size=(5, 3, d))
+    pos = np.array([0, 1, 17, 4095, 131071])
+    got = O.rope(x, pos, theta)
+    half = d // 2
+    zc = x[..., :half] + 1j * x[..., half:]
+    freq = theta ** (-np.arange(half) * 2.0 / d)
+    rot = zc * np.exp(1j * pos[:, None, None] * freq[None, None, :])
+    want = np.concatenate([rot.real, rot.imag], axis=-1)
+    np.testing.assert_allclose(got, want, atol=1e-12)
+    np.testing.assert_allclose(got[0], x[0], atol=0)       # position 0 is the identity
+
+
+def test_rope_relative_position():
+    rng = np.random.default_rng(10)
+    d = 32
+    q = rng.normal(size=(1, 1, d))
+    k = rng.normal(size=(1, 1, d))
+    a = np.sum(O.rope(q, [100], 1e4) * O.rope(k, [60], 1e4))
+    b = np.sum(O.rope(q, [1040], 1e4) * O.rope(k, [1000], 1e4))
+    c = np.sum(O.rope(q, [60], 1e4) * O.rope(k, [100], 1e4))
+    assert abs(a - b) < 1e-10 and abs(a - c) > 1e-3
+
+
+# ------------------------------------------------------------------ attention
+
+def _attn_loops(Q, K, V, cu, pos, bias, gamma, beta):
+    """Explicit per-(request, head, query, key) loops; tiny sizes only."""
+    Kt, Hq, d = Q.shape
+    grp = Hq // K.shape[1]
+    out = np.zeros_like(Q)
+    for b in range(len(cu) - 1):
+        for h in range(Hq):
+            for r in range(cu[b + 1] - cu[b]):
+                p = pos[cu[b] + r]
+                tau = beta if p == 0 else beta * math.log(r + 1) / math.log(p + 1)
+                ls = []
+                for c in range(r + 1):
+                    dot = sum(Q[cu[b] + r, h, i] * K[cu[b] + c, h // grp, i] for i in range(d))
+                    ls.append(tau * dot / math.sqrt(d) + gamma[h] * bias[cu[b] + c])
+                m = max(ls)
+                w = [math.exp(x - m) for x in ls]
+                tot = sum(w)
+                for c in range(r + 1):
+                    out[cu[b] + r, h] += w[c] / tot * V[cu[b] + c, h // grp]
+    return out
+
+
+def _rand_attn_case(seed, lens, Hq=4, Hkv=2, d=8):
+    rng = np.random.default_rng(seed)
+    cu = np.concatenate([[0], np.cumsum(lens)])
+    Kt = int(cu[-1])
+    Q = rng.normal(size=(Kt, Hq, d))
+    K = rng.normal(size=(Kt, Hkv, d))
+    V = rng.normal(size=(Kt, Hkv, d))
+    pos = np.concatenate([np.sort(rng.choice(4 * n + 3, size=n, replace=False)) for n in lens])
+    bias = rng.normal(size=Kt) * (rng.random(Kt) < 0.8)
+    gamma = rng.uniform(0.5, 2.0, size=Hq)
+    return Q, K, V, cu, pos, bias, gamma
+
+
+@pytest.mark.parametrize("seed", range(4))
+def test_attention_brute_force_loops(seed):
+    Q, K, V, cu, pos, bias, gamma = _rand_attn_case(seed, [5, 1, 7])
+    beta = 0.8 + 0.1 * seed
+    got, _ = O.gated_attention(Q, K, V, cu, pos, bias, gamma, beta, block=3)
+    want = _attn_loops(Q, K, V, cu, pos, bias, gamma, beta)
+    np.testing.assert_allclose(got, want, atol=1e-12)
+
+
+def test_attention_reduces_to_library_causal_gqa():
+    """K = N, gamma = 0, positions = ranks (tau = 1): plain causal GQA attention."""
+    Q, K, V, cu, _, bias, gamma = _rand_attn_case(21, [33], Hq=8, Hkv=2, d=16)
+    pos = np.arange(33)
+    got, lse = O.gated_attention(Q, K, V, cu, pos, bias, np.zeros(8), 1.0)
+    q = torch.tensor(Q).permute(1, 0, 2)[None]
+    k = torch.tensor(K).permute(1, 0, 2).repeat_interleave(4, dim=0)[None]
+    v = torch.tensor(V).permute(1, 0, 2).repeat_interleave(4, dim=0)[None]
+    want = F.scaled_dot_product_attention(q, k, v, is_causal=True)[0].permute(1, 0, 2)
+    np.testing.assert_allclose(got, want.numpy(), atol=1e-12)
+    # LSE against logsumexp of the causal logits
+    s = torch.einsum("hqd,hkd->hqk", q[0], k[0]) / 4.0
+    s = s.masked_fill(torch.triu(torch.ones(33, 33, dtype=torch.bool), 1), float("-inf"))
+    np.testing.assert_allclose(lse, torch.logsumexp(s, -1).numpy(), atol=1e-12)
+
+
+def test_attention_invariants():
+    Q, K, V, cu, pos, bias, gamma = _rand_attn_case(4, [40, 9])
+    ones = np.ones_like(V)
+    o1, _ = O.gated_attention(Q, K, ones, cu, pos, bias, gamma, 1.0)
+    np.testing.assert_allclose(o1, 1.0, atol=1e-13)                   # rows sum to 1
+    o, _ = O.gated_attention(Q, K, V, cu, pos, bias, gamma, 1.0)
+    for b in range(2):
+        for h in range(4):
+            np.testing.assert_allclose(o[cu[b], h], V[cu[b], h // 2], atol=1e-14)  # rank 0
+    # a bias constant over a request (all keys prunable) cancels in the softmax
+    const = np.full_like(bias, 0.7)
+    oa, _ = O.gated_attention(Q, K, V, cu, pos, const, gamma, 1.0)
+    ob, _ = O.gated_attention(Q, K, V, cu, pos, const, np.zeros(4), 1.0)
+    np.testing.assert_allclose(oa, ob, atol=1e-13)
+    # but a non-constant bias with gamma > 0 does matter, and in the sign's direction
+    hi = np.zeros_like(bias)
+    hi[cu[0] + 3] = 5.0
+    oc, _ = O.gated_attention(Q, K, ones * np.arange(1, 1 + V.shape[0])[:, None, None],
+                              cu, pos, hi, gamma, 1.0)
+    od, _ = O.gated_attention(Q, K, ones * np.arange(1, 1 + V.shape[0])[:, None, None],
+                              cu, pos, -hi, gamma, 1.0)
+    r = cu[0] + 10
+    assert abs(oc[r, 0, 0] - 4.0) < abs(od[r, 0, 0] - 4.0)
+
+
+def test_attention_kv_head_mapping():
+    """q head h must read kv head h // (Hq/Hkv): zero all but one kv head's values."""
+    Q, K, V, cu, pos, bias, gamma = _rand_attn_case(8, [12], Hq=4, Hkv=2)
+    V2 = np.zeros_like(V)
+    V2[:, 1] = 1.0
+    o, _ = O.gated_attention(Q, K, V2, cu, pos, bias, gamma, 1.0)
+    np.testing.assert_allclose(o[:, :2], 0.0, atol=0)
+    np.testing.assert_allclose(o[:, 2:], 1.0, atol=1e-13)
+
+
+def test_attention_sampled_rows_match_full():
+    Q, K, V, cu, pos, bias, gamma = _rand_attn_case(13, [30, 25])
+    full, lf = O.gated_attention(Q, K, V, cu, pos, bias, gamma, 1.1)
+    rows = [0, 7, 29, 30, 54]
+    part, lp = O.gated_attention(Q, K, V, cu, pos, bias, gamma, 1.1, rows=rows, block=2)
+    np.testing.assert_allclose(part[rows], full[rows], atol=1e-13)
+    np.testing.assert_allclose(lp[:, rows], lf[:, rows], atol=1e-13)
+    assert np.isnan(part[1]).all()
+
+
+# ------------------------------------------------------------------ layer / pipeline
+
+def test_layer_zero_output_projection_keeps_residual():
+    rng = np.random.default_rng(2)
+    Hq, Hkv, d, H = 2, 1, 8, 16
+    x = rng.normal(size=(6, H))
+    Wqkv = rng.normal(size=((Hq + 2 * Hkv) * d, H)) * 0.3
+    Wo = np.zeros((H, Hq * d))
+    pos = np.array([0, 3, 4, 8, 9, 11])
+    x2, k, v, parts = O.gated_layer(x, Wqkv, Wo, [1.0, 1.5], 1.0, [0, 6], pos,
+                                    np.zeros(6), Hq, Hkv, d, 1e4)
+    np.testing.assert_allclose(x2, x, atol=0)
+    a = x / np.sqrt(np.mean(x * x, 1, keepdims=True) + 1e-6)
+    kk = (a @ Wqkv.T)[:, Hq * d:(Hq + Hkv) * d].reshape(6, Hkv, d)
+    np.testing.assert_allclose(k, O.rope(kk, pos, 1e4), atol=1e-12)
+    vv = (a @ Wqkv.T)[:, (Hq + Hkv) * d:].reshape(6, Hkv, d)
+    np.testing.assert_allclose(v, vv, atol=1e-12)
+
+
+def test_prefill_tiny_pipeline_consistency():
+    import synthetic_inputs as S
+    wl = S.custom([40, 24], [4, 6], [10, 12], n_layers=1, hidden=32, scorer_width=8,
+                  n_q_heads=4, n_kv_heads=2, head_dim=8)
+    h = S.hidden_rows(wl)
+    gate = S.gate_weights(wl)
+    layer = S.layer_weights(wl, 0)
+    pr = S.prunable_mask(wl)
+    out = O.prefill(h, pr, wl.cu_seqlens(), wl.budgets, gate, [layer], 4, 2, 8)
+    assert list(out["cu_kept"]) == [0, 10, 22]
+    assert len(out["kept_idx"]) == 22
+    # question tokens (last Q_b of each request) are all kept
+    for b, (lo, n, q) in enumerate(zip(wl.cu_seqlens()[:-1], wl.lengths, wl.questions)):
+        kept_b = set(out["kept_idx"][out["cu_kept"][b]:out["cu_kept"][b + 1]].tolist())
+        assert set(range(lo + n - q, lo + n)) <= kept_b
+    assert out["x"].shape == (22, 32)
