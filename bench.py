@@ -1,0 +1,484 @@
+#!/usr/bin/env python
+"""Gated-prefill benchmark: input tokens/s of one TokenGate prefill step on B200.
+
+A step is one pass of the whole hot path over one synthetic batch: gate scores and
+their sequence RMSNorm, prunable-only top-K with compaction, the row gather, then per
+gated layer the RMSNorm-folded QKV projection, RoPE at original positions, the
+compacted KV-cache write, token-gated attention and the output projection.
+
+Default workload: N=16384 (16320 document + 64 question tokens), budget 1638 kept,
+28 stacked gated layers, Qwen3-1.7B-sized heads (16 q / 8 kv, head_dim 128).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload n16k|n128k|...]
+  python bench.py --impl reference ...   # the CPU oracle timed on the host cores
+
+Multi-GPU (torchrun, one rank per GPU): every rank runs an independent replica on
+its own batch (no collective on the data path); value = all ranks' tokens / the
+slowest rank's time.
+
+Timing: W untimed warm-up steps; then K steps, each replayed from a CUDA graph of the
+step with timing events at every stage boundary.  L2 is flushed (a 512 MiB write)
+before every timed step, outside the events.  SM clocks and throttle reasons are
+sampled through NVML during the timed region.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "gated-prefill input tokens/s at N=16k/128k; attn TFLOP/s & select GB/s vs peak"
+UNIT = "tokens/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="n16k")
+    ap.add_argument("--launch", choices=["graph", "eager"], default="graph")
+    ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-sample-layers", type=int, default=2)
+    return ap.parse_args()
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return {k: float(d[k]) for k in FALLBACK_PEAKS}, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def workload(name):
+    import synthetic_inputs as S
+    table = S.all_workloads()
+    if name not in table:
+        raise SystemExit(f"unknown workload {name}; choose from {sorted(table)}")
+    return table[name]
+
+
+# ------------------------------------------------------------------ algorithmic work
+
+def stage_work(wl, kept_counts):
+    """Algorithmic bytes / flops per launch of each stage (see the design notes)."""
+    T = wl.total_tokens
+    Ks = [kept_counts[b + 1] - kept_counts[b] for b in range(wl.batch)]
+    K = sum(Ks)
+    H, F, hq, hkv, d = wl.hidden, wl.scorer_width, wl.n_q_heads, wl.n_kv_heads, wl.head_dim
+    nqkv = (hq + 2 * hkv) * d
+    attn_pairs = sum(k * (k + 1) // 2 for k in Ks)
+    return {
+        "gate_score": {"bound": "hbm", "bytes": T * H * 2 + F * H * 2 + T * 4 * 3 + T,
+                       "flops": 2 * T * H * F},
+        "seq_rmsnorm": {"bound": "hbm", "bytes": T * 13},
+        "topk_compact": {"bound": "hbm", "bytes": T * 5 + K * 12},
+        "gather": {"bound": "hbm", "bytes": 2 * K * H * 2 + K * 4},
+        "qkv_proj": {"bound": "tensor", "flops": 2 * K * H * nqkv,
+                     "bytes": K * H * 2 + nqkv * H * 2 + K * nqkv * 2},
+        "rope": {"bound": "hbm", "bytes": 2 * K * (hq + hkv) * d * 2 + K * 4},
+        "kv_compact": {"bound": "hbm", "bytes": 2 * 2 * K * hkv * d * 2},
+        "attention": {"bound": "tensor", "flops": 4 * d * hq * attn_pairs},
+        "out_proj": {"bound": "tensor", "flops": 2 * K * hq * d * H,
+                     "bytes": K * hq * d * 2 + H * hq * d * 2 + 2 * K * H * 2},
+    }
+
+
+# ------------------------------------------------------------------ clocks (NVML)
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons of one GPU every ~20 ms in a thread."""
+
+    def __init__(self, device_index):
+        self.samples = []
+        self.ok = False
+        self._stop = threading.Event()
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # no NVML: report that, not a guess
+            self.err = str(e)
+
+    def _run(self):
+        nv = self.nv
+        names = {
+            "hw_slowdown": getattr(nv, "nvmlClocksEventReasonHwSlowdown", 0x8),
+            "hw_thermal_slowdown": getattr(nv, "nvmlClocksEventReasonHwThermalSlowdown", 0x40),
+            "sw_thermal_slowdown": getattr(nv, "nvmlClocksEventReasonSwThermalSlowdown", 0x20),
+            "sw_power_cap": getattr(nv, "nvmlClocksEventReasonSwPowerCap", 0x4),
+            "hw_power_brake_slowdown": getattr(nv, "nvmlClocksEventReasonHwPowerBrakeSlowdown", 0x80),
+        }
+        while not self._stop.is_set():
+            try:
+                mhz = nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)
+                try:
+                    r = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                except Exception:
+                    r = nv.nvmlDeviceGetCurrentClocksThrottleReasons(self.h)
+                active = [k for k, bit in names.items() if r & bit]
+                self.samples.append((mhz, active))
+            except Exception:
+                pass
+            time.sleep(0.02)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+
+    def summary(self):
+        if not self.ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "note": "NVML unavailable"}
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0}
+        reasons = sorted({r for _, rs in self.samples for r in rs})
+        return {"sm_mhz": statistics.median(m for m, _ in self.samples),
+                "sm_max_mhz": self.max_mhz, "reasons": reasons, "samples": len(self.samples)}
+
+
+# ------------------------------------------------------------------ our arm
+
+def run_ours(args, rank, world):
+    import numpy as np
+    import torch
+
+    import learned_token_pruning_scoring_b200 as tg
+    import synthetic_inputs as S
+
+    dev = torch.device("cuda", torch.cuda.current_device())
+    wl = workload(args.workload)
+    # replicas: rank r draws its own batch (seed offset), same weights
+    if world > 1:
+        wl = S.Workload(**{**wl.__dict__, "seeds": tuple(s + 1000 * rank for s in wl.seeds)})
+    h = S.hidden_rows(wl)
+    pr = S.prunable_mask(wl)
+    gate = {k: v.to(dev) for k, v in S.gate_weights(wl).items()}
+    layers = []
+    for i in range(wl.n_layers):
+        L = S.layer_weights(wl, i)
+        layers.append({k: (v.to(dev) if torch.is_tensor(v) else v) for k, v in L.items()})
+    scores = S.drawn_scores(wl).to(dev) if wl.planted_cluster else None
+    pipe = tg.GatedPrefill(gate, layers, wl.n_q_heads, wl.n_kv_heads, wl.head_dim,
+                           wl.rope_theta, device=dev)
+    P = pipe.plan(wl.lengths, wl.questions, wl.budgets)
+    h_dev = h.to(dev)
+    pr_dev = pr.to(dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        pipe.run(h_dev, pr_dev, scores=scores)
+
+    for _ in range(max(args.warmup, 1)):
+        step()
+    torch.cuda.synchronize()
+    status = tg.tg_status_read(pipe.status)
+    if status:
+        raise SystemExit(f"device status {status:#x} after warm-up")
+
+    # stage boundary events (external: they become event nodes inside the graph)
+    marks = []
+    use_graph = args.launch == "graph"
+
+    def make_marker(evs):
+        def marker(name):
+            e = torch.cuda.Event(enable_timing=True, external=use_graph)
+            e.record(stream)
+            evs.append((name, e))
+        return marker
+
+    start_ev = torch.cuda.Event(enable_timing=True, external=use_graph)
+    graph = None
+    launches_before = tg.launch_count
+    if use_graph:
+        g = torch.cuda.CUDAGraph()
+        s_side = torch.cuda.Stream()
+        s_side.wait_stream(stream)
+        with torch.cuda.stream(s_side):
+            pipe.marker = make_marker(marks)
+            with torch.cuda.graph(g, stream=s_side):
+                start_ev.record(s_side)
+                # inside capture the current stream is s_side
+                stream_cap = torch.cuda.current_stream()
+                pipe.marker = None
+                evs = []
+
+                def marker(name, _evs=evs):
+                    e = torch.cuda.Event(enable_timing=True, external=True)
+                    e.record(stream_cap)
+                    _evs.append((name, e))
+                pipe.marker = marker
+                step()
+            pipe.marker = None
+        stream.wait_stream(s_side)
+        marks = evs
+        graph = g
+    launches_per_step = tg.launch_count - launches_before
+    torch.cuda.synchronize()
+
+    flush = torch.empty(512 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+    per_stage = {}
+    step_ms = []
+
+    def run_timed_step():
+        flush.fill_(1.0)  # evict L2 (outside the step's events)
+        if use_graph:
+            graph.replay()
+        else:
+            marks.clear()
+            start_ev.record(stream)
+            pipe.marker = make_marker(marks)
+            step()
+            pipe.marker = None
+        torch.cuda.synchronize()
+        t_prev = start_ev
+        for name, e in marks:
+            ms = t_prev.elapsed_time(e)
+            per_stage.setdefault(name, []).append(ms)
+            t_prev = e
+        step_ms.append(start_ev.elapsed_time(marks[-1][1]))
+
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    launches_timed_before = tg.launch_count
+    with ClockSampler(dev.index) as clk:
+        for _ in range(args.steps):
+            run_timed_step()
+    torch.cuda.synchronize()
+    eager_launches = tg.launch_count - launches_timed_before
+    gpu_launches = launches_per_step * args.steps if use_graph else eager_launches
+    total_ms = sum(step_ms)
+    if world > 1:
+        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        total_ms = float(t.item())
+        torch.distributed.barrier()
+    status = tg.tg_status_read(pipe.status)
+    if status:
+        raise SystemExit(f"device status {status:#x} after timed steps")
+
+    tokens_per_step = wl.total_tokens
+    value = tokens_per_step * world * args.steps / (total_ms / 1e3)
+
+    # ---- end to end through the public API: host inputs in, result out, per step
+    h_pin = h.pin_memory()
+    pr_pin = pr.pin_memory()
+    x_host = torch.empty(P["x"].shape, dtype=P["x"].dtype).pin_memory()
+    e2e_ms = []
+    for i in range(args.e2e_steps + 1):
+        flush.fill_(1.0)
+        torch.cuda.synchronize()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        h_dev.copy_(h_pin, non_blocking=True)
+        pr_dev.copy_(pr_pin, non_blocking=True)
+        if use_graph:
+            graph.replay()
+        else:
+            step()
+        x_host.copy_(P["x"], non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        if i:  # first one is a warm-up of the copy path
+            e2e_ms.append(e0.elapsed_time(e1))
+    e2e_total = sum(e2e_ms)
+    if world > 1:
+        t = torch.tensor([e2e_total], dtype=torch.float64, device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        e2e_total = float(t.item())
+    e2e_value = tokens_per_step * world * len(e2e_ms) / (e2e_total / 1e3)
+    h2d = h.numel() * h.element_size() + pr.numel() * pr.element_size()
+    d2h = x_host.numel() * x_host.element_size()
+
+    # ---- per-stage roofline
+    peaks, peak_src = load_peaks()
+    work = stage_work(wl, [int(x) for x in P["ck_h"].tolist()])
+    stages = {}
+    for name, ms_list in per_stage.items():
+        n_launch = len(ms_list)
+        avg_ms = sum(ms_list) / n_launch
+        w = work.get(name, {})
+        entry = {"launches": n_launch, "total_ms": sum(ms_list), "avg_ms": avg_ms}
+        if w.get("bound") == "tensor" and "flops" in w:
+            ach = w["flops"] / (avg_ms / 1e3) / 1e12
+            entry.update(bound="tensor", achieved=ach, unit="TFLOP/s",
+                         peak=peaks["bf16_tflops_sustained"], frac=ach / peaks["bf16_tflops_sustained"])
+        elif "bytes" in w:
+            ach = w["bytes"] / (avg_ms / 1e3) / 1e9
+            entry.update(bound="hbm", achieved=ach, unit="GB/s", peak=peaks["hbm_gbs"],
+                         frac=ach / peaks["hbm_gbs"])
+        stages[name] = entry
+    tot = sum(v["total_ms"] for v in stages.values())
+    for v in stages.values():
+        v["share"] = v["total_ms"] / tot if tot else None
+    dom = max(stages, key=lambda k: stages[k]["total_ms"])
+    d = stages[dom]
+    traffic = load_traffic(dom, wl.name)
+    roofline = {"kernel": dom, "bound": d.get("bound"), "achieved": d.get("achieved"),
+                "peak": d.get("peak"), "unit": d.get("unit"), "frac": d.get("frac"),
+                "traffic": traffic, "peak_source": f"{peak_src} (sustained for tensor, "
+                                                   f"copy bandwidth for hbm)"}
+
+    out = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": wl.name, "batch": wl.batch, "tokens_per_request": list(wl.lengths)
+                   if wl.batch <= 8 else None, "question_tokens": list(wl.questions)
+                   if wl.batch <= 8 else None, "kept": int(P["ck_h"][-1]),
+                   "gated_layers": wl.n_layers, "hidden": wl.hidden,
+                   "heads": f"{wl.n_q_heads}q/{wl.n_kv_heads}kv x {wl.head_dim}",
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                   "l2": "flushed before every timed step (512 MiB write, outside the timing)",
+                   "launch": "cuda_graph" if use_graph else "eager"},
+        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+        "gpu_launches": gpu_launches,
+        "roofline": roofline,
+        "stages": {k: {kk: (round(vv, 5) if isinstance(vv, float) else vv)
+                       for kk, vv in v.items()} for k, v in stages.items()},
+        "clocks": clk.summary(),
+    }
+    return out
+
+
+def load_traffic(kernel, workload_name):
+    """Per-launch DRAM bytes from a committed ncu summary, if one exists for this kernel."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return d.get(workload_name, {}).get(kernel)
+    except Exception:
+        return None
+
+
+# ------------------------------------------------------------------ CPU oracle arm
+
+def oracle_sample(wl, n_layers_sample):
+    """Time the oracle on a bounded sample of the workload and scale to one full step.
+
+    Sample: the whole gate (scorer + sequence RMSNorm + selection + gather) over all N
+    tokens, then `n_layers_sample` of the gated layers; the per-layer time is scaled to
+    the workload's layer count."""
+    import numpy as np
+
+    import oracle as O
+    import synthetic_inputs as S
+    h = S.hidden_rows(wl)
+    pr = S.prunable_mask(wl)
+    gate = S.gate_weights(wl)
+    t0 = time.perf_counter()
+    s = O.gate_score(h, gate["norm_w"], gate["W1"], gate["w2"])
+    if wl.planted_cluster:
+        s = O.as_f64(S.drawn_scores(wl))
+    z, _ = O.sequence_rmsnorm(s, wl.cu_seqlens(), pr)
+    ck = O.kept_counts(pr, wl.cu_seqlens(), wl.budgets)
+    idx, pos, kb = O.select_topk(z.astype(np.float32), pr, wl.cu_seqlens(), ck)
+    x = O.gather_rows(h, idx)
+    t1 = time.perf_counter()
+    nl = max(1, min(n_layers_sample, wl.n_layers))
+    for i in range(nl):
+        L = S.layer_weights(wl, i)
+        x, _, _, _ = O.gated_layer(x, L["Wqkv"], L["Wo"], L["gamma"], L["beta"], ck, pos, kb,
+                                   wl.n_q_heads, wl.n_kv_heads, wl.head_dim, wl.rope_theta)
+    t2 = time.perf_counter()
+    full_s = (t1 - t0) + (t2 - t1) / nl * wl.n_layers
+    return {"seconds_per_step": full_s, "measured_s": t2 - t0, "layers_run": nl}
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [d.get("num_threads") for d in threadpool_info() if d.get("user_api") == "blas"]
+        return max(n) if n else os.cpu_count()
+    except Exception:
+        return os.cpu_count()
+
+
+def cpu_baseline(wl, n_layers_sample):
+    r = oracle_sample(wl, n_layers_sample)
+    return {"value": wl.total_tokens / r["seconds_per_step"], "unit": UNIT,
+            "cores": blas_threads(), "kind": "oracle",
+            "sample": (f"float64 NumPy oracle: gate over all {wl.total_tokens} tokens + "
+                       f"{r['layers_run']} of {wl.n_layers} gated layers "
+                       f"({r['measured_s']:.1f} s measured), layer time scaled to "
+                       f"{wl.n_layers} layers")}
+
+
+def run_reference(args, rank, world):
+    wl = workload(args.workload)
+    for _ in range(args.warmup):
+        oracle_sample(wl, 1)
+    secs = []
+    for _ in range(args.steps):
+        secs.append(oracle_sample(wl, 1)["seconds_per_step"])
+    value = wl.total_tokens * len(secs) / sum(secs)
+    cores = blas_threads()
+    return {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * sum(secs) / len(secs),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": wl.name, "batch": wl.batch, "gated_layers": wl.n_layers},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": f"per step: gate over all {wl.total_tokens} tokens + 1 of "
+                                   f"{wl.n_layers} gated layers, layer time scaled to "
+                                   f"{wl.n_layers}"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    args = parse_args()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args, rank, world)), flush=True)
+        return
+    import torch
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    try:
+        out = run_ours(args, rank, world)
+        if rank == 0 and world == 1 and not args.no_cpu_baseline:
+            out["cpu_baseline"] = cpu_baseline(workload(args.workload), args.cpu_sample_layers)
+        if rank == 0:
+            print(json.dumps(out), flush=True)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

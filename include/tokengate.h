@@ -1,0 +1,273 @@
+/*
+ * tokengate.h -- C ABI of the TokenGate prefill hot path on NVIDIA B200 (sm_100a).
+ *
+ * The calls implement, as CUDA kernels, the gate layer and the token-gated attention
+ * described on these pages (cited below by tag, with the section used):
+ *   [fluxbbs]    "TokenGate 长上下文预填充提速 11.3 倍，斯坦福伯克利开源门控剪枝"
+ *   [digest]     "TokenGate: Adapting LLMs for Fast and Memory-Efficient Prefill with
+ *                 Learned Token Pruning" (paper digest)
+ *   [farwalk]    "斯坦福与 UC Berkeley 提出 TokenGate：token 门控注意力让长上下文预填充最高快 11.3 倍"
+ *   [aiwillknow] "TokenGate：让模型学会跳读，而不只压缩 KV 缓存"
+ *
+ * Conventions shared by every call
+ *   - Pointers are device pointers unless the name ends in `_host`.  The caller owns
+ *     every buffer; unless an entry point says otherwise, the library allocates no
+ *     device memory.  Scratch memory is passed in as `workspace`, sized by the
+ *     matching *_workspace_size() query.
+ *   - Matrices are row-major; `ld_*` is the row stride in elements.  bf16 tensors are
+ *     passed as their 16-bit patterns (tg_bf16).
+ *   - Requests are packed back to back ("varlen"): request b owns rows
+ *     cu_seqlens[b] .. cu_seqlens[b+1]-1 before the gate and kept rows
+ *     cu_kept[b] .. cu_kept[b+1]-1 after it.  Each cu array is given twice: on the
+ *     device (read by kernels) and on the host (argument checks and launch shapes);
+ *     the two copies must hold the same values.
+ *   - Every call is asynchronous on `stream` (a cudaStream_t; NULL = legacy default
+ *     stream) and never synchronises, except tg_status_read().
+ *   - Return value: TG_OK, or a negative TG_ERR_* code.  Argument errors are found on
+ *     the host before anything is launched.  Errors found on the device (a bounded
+ *     wait that ran out, a kept count that disagrees with the prunable mask) are
+ *     OR-ed into the caller's 32-bit `status` word (TG_STATUS_* bits); read it with
+ *     tg_status_read().  `status` may be NULL where a call says so.
+ *   - Device requirement: compute capability 10.0 (B200).  Other devices get
+ *     TG_ERR_UNSUPPORTED_DEVICE; there is no fallback path.
+ */
+#ifndef TOKENGATE_H
+#define TOKENGATE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef uint16_t tg_bf16;   /* bfloat16 bit pattern */
+typedef void* tg_stream_t;  /* cudaStream_t */
+
+/* Return codes. */
+#define TG_OK 0
+#define TG_ERR_INVALID_ARGUMENT (-1)   /* null pointer, bad size, inconsistent cu arrays */
+#define TG_ERR_MISALIGNED (-2)         /* pointer or row stride not 16-byte aligned */
+#define TG_ERR_UNSUPPORTED_DEVICE (-3) /* current device is not sm_100 */
+#define TG_ERR_WORKSPACE (-4)          /* workspace missing or smaller than required */
+#define TG_ERR_CUDA (-5)               /* a CUDA runtime/driver call failed; see tg_last_cuda_error */
+#define TG_ERR_UNSUPPORTED_SHAPE (-6)  /* a dimension outside what the kernels implement */
+
+/* Device status bits (OR-ed into the caller's status word by kernels). */
+#define TG_STATUS_TIMEOUT 0x1u /* a bounded wait ran out; outputs of that call are invalid */
+#define TG_STATUS_BUDGET 0x2u  /* kept count K_b inconsistent with the prunable mask */
+#define TG_STATUS_BOUNDS 0x4u  /* a row index outside the source; that row was skipped */
+
+/* ------------------------------------------------------------------ utilities */
+
+/* Short English description of a TG_* return code (static storage). */
+const char* tg_error_string(int code);
+
+/* cudaError_t value behind the most recent TG_ERR_CUDA on the calling thread. */
+int tg_last_cuda_error(void);
+
+/* 1 if `device` is a compute-capability-10.0 GPU this library runs on, else 0. */
+int tg_device_supported(int device);
+
+/* Library ABI version (major * 100 + minor). */
+int tg_version(void);
+
+/* Zero the status word (async on `stream`). */
+int tg_status_clear(uint32_t* status, tg_stream_t stream);
+
+/* Copy the status word to *out_host after synchronising `stream`. */
+int tg_status_read(const uint32_t* status, uint32_t* out_host, tg_stream_t stream);
+
+/*
+ * Rotary table for original-position RoPE ([aiwillknow] figure 1(a)(b): kept tokens
+ * keep their original position encoding).  Writes cos_sin[p][i][0] = cos(p * f_i),
+ * cos_sin[p][i][1] = sin(p * f_i) for p < max_pos, i < head_dim/2, with
+ * f_i = theta^(-2 i / head_dim).  Angles and trigonometry are evaluated in float64
+ * on the device, then rounded to float32.  cos_sin: float32 [max_pos, head_dim/2, 2].
+ */
+int tg_rope_table(float* cos_sin, int max_pos, int head_dim, double theta,
+                  tg_stream_t stream);
+
+/*
+ * Host-only planning of the kept counts from per-request budgets (no GPU work).
+ * ([farwalk] How do you deploy TokenGate?: generation takes a budget of kept prefill
+ *  tokens; [farwalk] How does TokenGate learned token pruning work?: the question is
+ *  never pruned.)  The budget counts every kept token, question included:
+ *    K_b = Q_b + min(D_b, max(0, budget_b - Q_b)),  D_b = N_b - Q_b,
+ * so a budget below Q_b keeps the question only and one above N_b keeps everything.
+ * cu_seqlens_host int32 [batch+1]; n_question_host int32 [batch] (Q_b, non-prunable
+ * tokens of request b); budgets_host int32 [batch]; writes cu_kept_host int32 [batch+1].
+ */
+int tg_plan_kept(const int32_t* cu_seqlens_host, const int32_t* n_question_host,
+                 const int32_t* budgets_host, int batch, int32_t* cu_kept_host);
+
+/* ------------------------------------------------------------------ gate scoring */
+
+/* Bytes of workspace tg_gate_score needs for `total_tokens` rows and `batch` requests. */
+size_t tg_gate_score_workspace_size(int64_t total_tokens, int hidden, int width, int batch);
+
+/*
+ * Gate scores and their sequence normalisation
+ * ([fluxbbs] 门控到底插在模型的哪个位置: a small MLP scores each token's normalised
+ *  residual and the scores are RMSNorm-normalised along the sequence;
+ *  [farwalk] How does TokenGate learned token pruning work?: the residual is the
+ *  post-attention residual at the gate layer).
+ *
+ *   x_t    = h_t * norm_w / sqrt(mean(h_t^2) + eps_norm)
+ *   s_t    = sum_f w2[f] * SiLU((W1 x_t)[f])
+ *   z_t    = s_t / sqrt(mean_{t' in request(t)} s_t'^2 + eps_seq)
+ *   bias_t = z_t if prunable[t] else 0
+ *
+ * h:        bf16 [total_tokens, hidden], row stride ld_h (multiple of 8).
+ * norm_w:   float32 [hidden] RMSNorm weight, or NULL for all ones.  When given it is
+ *           folded into W1 (rounded to bf16) inside the workspace.
+ * W1:       bf16 [width, hidden] (output rows), row stride hidden.  width must be 256.
+ * w2:       float32 [width].
+ * cu_seqlens / cu_seqlens_host: int32 [batch+1], cu_seqlens[batch] = total_tokens.
+ * prunable: uint8 [total_tokens], 1 = document (prunable), 0 = question (kept).
+ * s_out, z_out, bias_out: float32 [total_tokens] (any of them may alias nothing else).
+ * hidden must be a multiple of 64.  status may be NULL.
+ * The GEMM runs on tcgen05 tensor cores with the row RMS applied in its epilogue and
+ * per-32-row partial sums of s^2 written there; a second kernel reduces the partials
+ * of each request in a fixed order (bit-reproducible) and writes z and bias.
+ */
+int tg_gate_score(const tg_bf16* h, int64_t ld_h, int64_t total_tokens, int hidden,
+                  const float* norm_w, const tg_bf16* W1, int width, const float* w2,
+                  float eps_norm, const int32_t* cu_seqlens, const int32_t* cu_seqlens_host,
+                  int batch, float eps_seq, const uint8_t* prunable, float* s_out,
+                  float* z_out, float* bias_out, void* workspace, size_t workspace_bytes,
+                  uint32_t* status, tg_stream_t stream);
+
+/*
+ * Sequence RMSNorm of raw scores on its own ([fluxbbs] 门控到底插在模型的哪个位置):
+ *   z_t = s_t / sqrt(mean_{t' in request(t)} s_t'^2 + eps_seq),  bias_t = prunable ? z_t : 0.
+ * Same kernel and fixed reduction order as the second stage of tg_gate_score, reading
+ * s directly instead of per-chunk partial sums.  s, z_out, bias_out float32 [total];
+ * z_out and bias_out must not alias s.  No workspace.
+ */
+int tg_seq_rmsnorm(const float* s, const int32_t* cu_seqlens, const int32_t* cu_seqlens_host,
+                   int batch, const uint8_t* prunable, float eps_seq, float* z_out,
+                   float* bias_out, tg_stream_t stream);
+
+/* ------------------------------------------------------------------ selection */
+
+/*
+ * Prunable-only top-K with order-preserving compaction
+ * ([fluxbbs] 门控到底插在模型的哪个位置: keep the top-K tokens, the question is never
+ *  pruned; [farwalk] How does TokenGate learned token pruning work?: only the document
+ *  is prunable; [aiwillknow] figure 1(a)(b): kept tokens keep their positions).
+ *
+ * For request b with Q_b non-prunable tokens and K_b = cu_kept[b+1] - cu_kept[b]
+ * kept rows, the Kd_b = K_b - Q_b prunable tokens with the largest z are kept, ties
+ * going to the lower index; NaN ranks below every number and -0 equals +0.  All
+ * non-prunable tokens are kept.  Kept tokens are listed by ascending position:
+ *   kept_idx[cu_kept[b] + r]  = cu_seqlens[b] + j   (packed row id of the token)
+ *   kept_pos[cu_kept[b] + r]  = j                   (position inside the request)
+ *   kept_bias[cu_kept[b] + r] = z[cu_seqlens[b] + j] if prunable, else 0
+ * The caller derives cu_kept from its budgets, e.g. K_b = Q_b + min(D_b, max(0,
+ * budget_b - Q_b)); if some K_b does not satisfy Q_b <= K_b <= N_b on the device,
+ * that request's outputs are left unwritten and TG_STATUS_BUDGET is set.
+ * z: float32 [total_tokens]; prunable: uint8 [total_tokens];
+ * kept_idx, kept_pos: int32 [cu_kept[batch]]; kept_bias: float32 [cu_kept[batch]].
+ * One thread-block cluster per request runs a 3-pass radix select (11/11/10 bits)
+ * over order-preserving integer keys with the histograms exchanged through
+ * distributed shared memory, then compacts with warp ballots.  status may be NULL.
+ */
+int tg_topk_compact(const float* z, const uint8_t* prunable, const int32_t* cu_seqlens,
+                    const int32_t* cu_seqlens_host, const int32_t* cu_kept,
+                    const int32_t* cu_kept_host, int batch, int32_t* kept_idx,
+                    int32_t* kept_pos, float* kept_bias, uint32_t* status,
+                    tg_stream_t stream);
+
+/* ------------------------------------------------------------------ gather / RoPE */
+
+/*
+ * Row gather with optional rotary embedding at original positions
+ * ([fluxbbs] 门控到底插在模型的哪个位置: pruned rows stop at the gate, only kept rows
+ *  go up; [aiwillknow] figure 1(a)(b): kept tokens keep their original positions).
+ *
+ *   dst[r, :width] = src[row_idx[r], :width]       (row_idx NULL: src[r])
+ * then, if rope_pos is not NULL, columns [rope_col_begin, rope_col_end) -- whole
+ * heads of head_dim columns -- are rotated rotate-half style at position rope_pos[r]:
+ *   y[i] = x[i] c - x[i + d/2] s,  y[i + d/2] = x[i + d/2] c + x[i] s,
+ *   (c, s) = cos_sin[rope_pos[r]][i], i < d/2 (table from tg_rope_table).
+ * src, dst: bf16, row strides ld_src, ld_dst (multiples of 8); width multiple of 8.
+ * src has src_rows rows; an index outside [0, src_rows) skips that output row and sets
+ * TG_STATUS_BOUNDS (status may be NULL).  dst may equal src (in place) only when
+ * row_idx is NULL.  rope_pos values must lie in [0, max_pos); rows outside are copied
+ * unrotated and set TG_STATUS_BOUNDS.
+ */
+int tg_gather_rope(const tg_bf16* src, int64_t ld_src, int64_t src_rows,
+                   const int32_t* row_idx, int64_t n_rows, int width, const int32_t* rope_pos, int rope_col_begin,
+                   int rope_col_end, int head_dim, const float* cos_sin, int max_pos,
+                   tg_bf16* dst, int64_t ld_dst, uint32_t* status, tg_stream_t stream);
+
+/* ------------------------------------------------------------------ KV cache */
+
+/*
+ * Compacted KV cache write ([farwalk] How does TokenGate learned token pruning work?:
+ * the pruned forward never creates KV entries for pruned tokens; [digest] 方法关键点:
+ * the KV cache can be selectively trimmed).
+ *   cache_k[slot_offset + r, :width] = k[row_idx[r], :width]   (row_idx NULL: k[r])
+ *   cache_v[slot_offset + r, :width] = v[row_idx[r], :width]
+ * With row_idx NULL this stores the kept rows' post-RoPE K/V into their cache slots;
+ * with row_idx = kept_idx it trims a full-length lower-layer cache to the kept rows.
+ * k, v have src_rows rows (indices outside skip the row and set TG_STATUS_BOUNDS);
+ * the caches have cache_rows rows and slot_offset + n_rows must not exceed it.
+ * All bf16; strides ld_k, ld_v, ld_cache are multiples of 8; width multiple of 8.
+ */
+int tg_kv_compact(const tg_bf16* k, int64_t ld_k, const tg_bf16* v, int64_t ld_v,
+                  int64_t src_rows, const int32_t* row_idx, int64_t n_rows, int width,
+                  tg_bf16* cache_k, tg_bf16* cache_v, int64_t ld_cache, int64_t cache_rows,
+                  int64_t slot_offset, uint32_t* status, tg_stream_t stream);
+
+/* ------------------------------------------------------------------ attention */
+
+/*
+ * Token-gated causal GQA attention over the kept rows
+ * ([fluxbbs] 端到端训练的关键在 token 门控注意力: per-head gain on the importance score
+ *  added to the logits, SSMax-style temperature from the log-ratio of kept count to
+ *  original position; [farwalk] What is token-gated attention?: the score is a bias
+ *  on the attention logits; [aiwillknow] figure 1(c): key bias, positive per-head gain).
+ * For q head h (kv head g = h / (n_q_heads / n_kv_heads)), request b, query rank r and
+ * key rank c <= r (ranks inside the request):
+ *   logit = tau_r * (q_r . k_c) / sqrt(head_dim) + gamma[h] * kept_bias[c]
+ *   tau_r = beta * ln(r + 1) / ln(p_r + 1),  tau_r = beta when p_r = 0,  p_r = kept_pos[r]
+ *   o_r   = sum_c softmax_c(logit) v_c
+ * q: bf16 [K_tot, n_q_heads * head_dim] (row stride ld_q); k, v: bf16
+ * [K_tot, n_kv_heads * head_dim] (ld_k, ld_v); o: bf16 [K_tot, n_q_heads * head_dim]
+ * (ld_o).  lse: float32 [n_q_heads, K_tot] natural-log log-sum-exp, or NULL.
+ * kept_pos int32 [K_tot]; kept_bias float32 [K_tot]; gamma float32 [n_q_heads].
+ * Implemented for head_dim = 128 and an even group size n_q_heads / n_kv_heads; q, k,
+ * v, o 16-byte aligned with strides that are multiples of 8.  The kernel runs the two
+ * q heads of a kv head on tcgen05 tensor cores with S and O accumulators in tensor
+ * memory and a TMA-fed K/V ring.  status may be NULL.
+ */
+int tg_gated_attention(const tg_bf16* q, int64_t ld_q, const tg_bf16* k, int64_t ld_k,
+                       const tg_bf16* v, int64_t ld_v, const int32_t* cu_kept,
+                       const int32_t* cu_kept_host, int batch, int n_q_heads,
+                       int n_kv_heads, int head_dim, const int32_t* kept_pos,
+                       const float* kept_bias, const float* gamma, float beta, tg_bf16* o,
+                       int64_t ld_o, float* lse, uint32_t* status, tg_stream_t stream);
+
+/* ------------------------------------------------------------------ projections */
+
+/*
+ * Dense projection used by the gated layers on the kept rows (Wq/Wk/Wv/Wo):
+ *   c[m, n] = r_m * sum_k a[m, k] w[n, k]  (+ residual[m, n])
+ * with r_m = 1/sqrt(mean_k a[m,k]^2 + eps) when rmsnorm_a is 1 (a pre-attention
+ * RMSNorm of weight 1 folded into the epilogue), else r_m = 1.
+ * a: bf16 [M, K] (lda); w: bf16 [N, K] (ldw, output rows); c, residual: bf16 [M, N]
+ * (ldc, ld_res; residual may be NULL and may equal c).  K multiple of 64, N multiple
+ * of 128, strides multiples of 8.  tcgen05 GEMM, TMA-fed, fp32 accumulation in TMEM.
+ * status may be NULL.
+ */
+int tg_linear(const tg_bf16* a, int64_t lda, const tg_bf16* w, int64_t ldw, tg_bf16* c,
+              int64_t ldc, int64_t M, int N, int K, int rmsnorm_a, float eps,
+              const tg_bf16* residual, int64_t ld_res, uint32_t* status, tg_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TOKENGATE_H */

@@ -1,0 +1,387 @@
+"""TokenGate gate layer and token-gated attention on B200 (sm_100a).
+
+Thin Python binding of ``libtokengate.so`` (declared in ``include/tokengate.h``).
+Every function named ``tg_*`` here marshals torch tensors into the C call of the same
+name; all arithmetic of the path runs in the library's CUDA kernels.  PyTorch only
+provides device memory and the stream.  If the shared library is missing, importing
+this package raises: there is no fallback implementation.
+
+``GatedPrefill`` strings the calls together for one prefill step: gate scores and
+their sequence normalisation, prunable-only top-K with order-preserving compaction,
+the row gather, then per upper layer the RMSNorm-folded QKV projection, RoPE at the
+original positions, the compacted KV-cache write, token-gated attention and the
+output projection with its residual add.
+"""
+from __future__ import annotations
+
+import ctypes as C
+from dataclasses import dataclass
+
+import torch
+
+from . import _lib
+
+__all__ = [
+    "TokenGateError", "lib", "tg_version", "tg_device_supported", "tg_plan_kept",
+    "tg_rope_table", "tg_gate_score_workspace_size", "tg_gate_score", "tg_topk_compact",
+    "tg_seq_rmsnorm", "tg_gather_rope", "tg_kv_compact", "tg_gated_attention", "tg_linear",
+    "tg_status_clear", "tg_status_read", "GatedPrefill", "STATUS_TIMEOUT", "STATUS_BUDGET",
+    "STATUS_BOUNDS",
+]
+
+lib = _lib.load()
+
+STATUS_TIMEOUT = 0x1
+STATUS_BUDGET = 0x2
+STATUS_BOUNDS = 0x4
+
+# Kernel launches issued through this binding (a benchmark reads it to report how many
+# of the library's kernels ran in its timed region).
+launch_count = 0
+
+
+def _count(n: int = 1) -> None:
+    global launch_count
+    launch_count += n
+
+
+class TokenGateError(RuntimeError):
+    def __init__(self, msg, code):
+        super().__init__(msg)
+        self.code = code
+
+
+def _check(rc: int, name: str) -> None:
+    if rc != 0:
+        msg = lib.tg_error_string(rc).decode()
+        if rc == -5:
+            msg += f" (cudaError {lib.tg_last_cuda_error()})"
+        raise TokenGateError(f"{name}: {msg}", rc)
+
+
+def _ptr(t):
+    return None if t is None else C.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return C.c_void_p(stream.cuda_stream)
+
+
+def _host_i32(x) -> torch.Tensor:
+    t = torch.as_tensor(x, dtype=torch.int32, device="cpu").contiguous()
+    return t
+
+
+def _mat(t: torch.Tensor, name: str):
+    if t.dim() != 2 or t.stride(1) != 1:
+        raise ValueError(f"{name}: expected a 2-D row-major view, got shape {tuple(t.shape)} "
+                         f"stride {t.stride()}")
+    return t.stride(0)
+
+
+def tg_version() -> int:
+    return lib.tg_version()
+
+
+def tg_device_supported(device: int = 0) -> bool:
+    return bool(lib.tg_device_supported(device))
+
+
+def tg_status_clear(status: torch.Tensor, stream=None) -> None:
+    _check(lib.tg_status_clear(_ptr(status), _stream(stream)), "tg_status_clear")
+
+
+def tg_status_read(status: torch.Tensor, stream=None) -> int:
+    out = C.c_uint32(0)
+    _check(lib.tg_status_read(_ptr(status), C.byref(out), _stream(stream)), "tg_status_read")
+    return int(out.value)
+
+
+def tg_plan_kept(cu_seqlens_host, n_question_host, budgets_host) -> torch.Tensor:
+    """Host-only: cu_kept from budgets (see include/tokengate.h)."""
+    cu = _host_i32(cu_seqlens_host)
+    nq = _host_i32(n_question_host)
+    bud = _host_i32(budgets_host)
+    batch = cu.numel() - 1
+    out = torch.zeros(batch + 1, dtype=torch.int32)
+    _check(lib.tg_plan_kept(_ptr(cu), _ptr(nq), _ptr(bud), batch, _ptr(out)), "tg_plan_kept")
+    return out
+
+
+def tg_rope_table(max_pos: int, head_dim: int, theta: float, out=None, device=None,
+                  stream=None) -> torch.Tensor:
+    if out is None:
+        out = torch.empty((max_pos, head_dim // 2, 2), dtype=torch.float32,
+                          device=device or "cuda")
+    _check(lib.tg_rope_table(_ptr(out), max_pos, head_dim, float(theta), _stream(stream)),
+           "tg_rope_table")
+    _count()
+    return out
+
+
+def tg_gate_score_workspace_size(total_tokens: int, hidden: int, width: int, batch: int) -> int:
+    return int(lib.tg_gate_score_workspace_size(total_tokens, hidden, width, batch))
+
+
+def tg_gate_score(h, W1, w2, cu_seqlens, cu_seqlens_host, prunable, norm_w=None,
+                  eps_norm=1e-6, eps_seq=1e-6, s_out=None, z_out=None, bias_out=None,
+                  workspace=None, status=None, stream=None):
+    ld_h = _mat(h, "h")
+    T, hidden = h.shape
+    width = W1.shape[0]
+    cuh = _host_i32(cu_seqlens_host)
+    batch = cuh.numel() - 1
+    dev = h.device
+    s_out = torch.empty(T, dtype=torch.float32, device=dev) if s_out is None else s_out
+    z_out = torch.empty(T, dtype=torch.float32, device=dev) if z_out is None else z_out
+    bias_out = torch.empty(T, dtype=torch.float32, device=dev) if bias_out is None else bias_out
+    need = tg_gate_score_workspace_size(T, hidden, width, batch)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    rc = lib.tg_gate_score(_ptr(h), ld_h, T, hidden, _ptr(norm_w), _ptr(W1), width, _ptr(w2),
+                           float(eps_norm), _ptr(cu_seqlens), _ptr(cuh), batch, float(eps_seq),
+                           _ptr(prunable), _ptr(s_out), _ptr(z_out), _ptr(bias_out),
+                           _ptr(workspace), workspace.numel(), _ptr(status), _stream(stream))
+    _check(rc, "tg_gate_score")
+    _count(3 if norm_w is not None else 2)
+    return s_out, z_out, bias_out
+
+
+def tg_seq_rmsnorm(s, cu_seqlens, cu_seqlens_host, prunable, eps_seq=1e-6, z_out=None,
+                   bias_out=None, stream=None):
+    cuh = _host_i32(cu_seqlens_host)
+    z_out = torch.empty_like(s) if z_out is None else z_out
+    bias_out = torch.empty_like(s) if bias_out is None else bias_out
+    rc = lib.tg_seq_rmsnorm(_ptr(s), _ptr(cu_seqlens), _ptr(cuh), cuh.numel() - 1, _ptr(prunable),
+                            float(eps_seq), _ptr(z_out), _ptr(bias_out), _stream(stream))
+    _check(rc, "tg_seq_rmsnorm")
+    _count()
+    return z_out, bias_out
+
+
+def tg_topk_compact(z, prunable, cu_seqlens, cu_seqlens_host, cu_kept, cu_kept_host,
+                    kept_idx=None, kept_pos=None, kept_bias=None, status=None, stream=None):
+    cuh = _host_i32(cu_seqlens_host)
+    ckh = _host_i32(cu_kept_host)
+    batch = cuh.numel() - 1
+    K = int(ckh[-1])
+    dev = z.device
+    kept_idx = torch.empty(K, dtype=torch.int32, device=dev) if kept_idx is None else kept_idx
+    kept_pos = torch.empty(K, dtype=torch.int32, device=dev) if kept_pos is None else kept_pos
+    kept_bias = torch.empty(K, dtype=torch.float32, device=dev) if kept_bias is None else kept_bias
+    rc = lib.tg_topk_compact(_ptr(z), _ptr(prunable), _ptr(cu_seqlens), _ptr(cuh),
+                             _ptr(cu_kept), _ptr(ckh), batch, _ptr(kept_idx), _ptr(kept_pos),
+                             _ptr(kept_bias), _ptr(status), _stream(stream))
+    _check(rc, "tg_topk_compact")
+    _count()
+    return kept_idx, kept_pos, kept_bias
+
+
+def tg_gather_rope(src, dst=None, row_idx=None, n_rows=None, rope_pos=None,
+                   rope_cols=(0, 0), head_dim=128, cos_sin=None, status=None, stream=None):
+    ld_src = _mat(src, "src")
+    width = src.shape[1]
+    if n_rows is None:
+        n_rows = row_idx.numel() if row_idx is not None else src.shape[0]
+    if dst is None:
+        dst = torch.empty((n_rows, width), dtype=src.dtype, device=src.device)
+    ld_dst = _mat(dst, "dst")
+    max_pos = cos_sin.shape[0] if cos_sin is not None else 0
+    rc = lib.tg_gather_rope(_ptr(src), ld_src, src.shape[0], _ptr(row_idx), n_rows, width,
+                            _ptr(rope_pos), int(rope_cols[0]), int(rope_cols[1]), head_dim,
+                            _ptr(cos_sin), max_pos, _ptr(dst), ld_dst, _ptr(status),
+                            _stream(stream))
+    _check(rc, "tg_gather_rope")
+    _count()
+    return dst
+
+
+def tg_kv_compact(k, v, cache_k, cache_v, row_idx=None, n_rows=None, slot_offset=0,
+                  status=None, stream=None):
+    ld_k, ld_v = _mat(k, "k"), _mat(v, "v")
+    ld_c = _mat(cache_k, "cache_k")
+    if _mat(cache_v, "cache_v") != ld_c:
+        raise ValueError("cache_k and cache_v must share a row stride")
+    width = k.shape[1]
+    if n_rows is None:
+        n_rows = row_idx.numel() if row_idx is not None else k.shape[0]
+    if v.shape[0] != k.shape[0] or cache_v.shape[0] != cache_k.shape[0]:
+        raise ValueError("k/v and cache_k/cache_v must have matching row counts")
+    rc = lib.tg_kv_compact(_ptr(k), ld_k, _ptr(v), ld_v, k.shape[0], _ptr(row_idx), n_rows,
+                           width, _ptr(cache_k), _ptr(cache_v), ld_c, cache_k.shape[0],
+                           int(slot_offset), _ptr(status), _stream(stream))
+    _check(rc, "tg_kv_compact")
+    _count()
+
+
+def tg_gated_attention(q, k, v, cu_kept, cu_kept_host, n_q_heads, n_kv_heads, kept_pos,
+                       kept_bias, gamma, beta, o=None, lse=None, head_dim=128, status=None,
+                       stream=None):
+    ld_q, ld_k, ld_v = _mat(q, "q"), _mat(k, "k"), _mat(v, "v")
+    ckh = _host_i32(cu_kept_host)
+    batch = ckh.numel() - 1
+    if o is None:
+        o = torch.empty((q.shape[0], n_q_heads * head_dim), dtype=q.dtype, device=q.device)
+    ld_o = _mat(o, "o")
+    rc = lib.tg_gated_attention(_ptr(q), ld_q, _ptr(k), ld_k, _ptr(v), ld_v, _ptr(cu_kept),
+                                _ptr(ckh), batch, n_q_heads, n_kv_heads, head_dim,
+                                _ptr(kept_pos), _ptr(kept_bias), _ptr(gamma), float(beta),
+                                _ptr(o), ld_o, _ptr(lse), _ptr(status), _stream(stream))
+    _check(rc, "tg_gated_attention")
+    _count()
+    return o
+
+
+def tg_linear(a, w, c=None, rmsnorm=False, eps=1e-6, residual=None, status=None, stream=None):
+    lda, ldw = _mat(a, "a"), _mat(w, "w")
+    M, K = a.shape
+    N = w.shape[0]
+    if c is None:
+        c = torch.empty((M, N), dtype=a.dtype, device=a.device)
+    ldc = _mat(c, "c")
+    ldr = _mat(residual, "residual") if residual is not None else 0
+    rc = lib.tg_linear(_ptr(a), lda, _ptr(w), ldw, _ptr(c), ldc, M, N, K, 1 if rmsnorm else 0,
+                       float(eps), _ptr(residual), ldr, _ptr(status), _stream(stream))
+    _check(rc, "tg_linear")
+    _count()
+    return c
+
+
+# ----------------------------------------------------------------------------- pipeline
+
+@dataclass
+class LayerWeights:
+    Wqkv: torch.Tensor   # bf16 [(Hq + 2 Hkv) d, H]
+    Wo: torch.Tensor     # bf16 [H, Hq d]
+    gamma: torch.Tensor  # fp32 [Hq]
+    beta: float
+
+
+class GatedPrefill:
+    """Buffers and call sequence of one gated prefill step on one device.
+
+    ``plan`` fixes the request layout (host work: lengths, question sizes, budgets ->
+    cu_kept) and allocates the device buffers; ``run`` then only launches kernels on
+    the stream, with no host synchronisation.
+    """
+
+    def __init__(self, gate: dict, layers: list, n_q_heads=16, n_kv_heads=8, head_dim=128,
+                 rope_theta=1.0e6, norm_eps=1e-6, seq_eps=1e-6, device="cuda"):
+        self.device = torch.device(device)
+        self.gate = gate
+        self.layers = [l if isinstance(l, LayerWeights) else LayerWeights(**l) for l in layers]
+        self.hq, self.hkv, self.d = n_q_heads, n_kv_heads, head_dim
+        self.theta = rope_theta
+        self.norm_eps, self.seq_eps = norm_eps, seq_eps
+        self.hidden = gate["W1"].shape[1]
+        self.width = gate["W1"].shape[0]
+        self.cos_sin = None
+        self.status = torch.zeros(1, dtype=torch.int32, device=self.device)
+        self.planned = None
+        # optional callable(stage_name) invoked after each launch (e.g. to record events)
+        self.marker = None
+
+    def _mark(self, name):
+        if self.marker is not None:
+            self.marker(name)
+
+    def plan(self, lengths, n_question, budgets):
+        lengths = [int(x) for x in lengths]
+        cu = [0]
+        for n in lengths:
+            cu.append(cu[-1] + n)
+        cu_h = _host_i32(cu)
+        ck_h = tg_plan_kept(cu_h, n_question, budgets)
+        T, K = cu[-1], int(ck_h[-1])
+        dev = self.device
+        max_pos = max(lengths) if lengths else 1
+        if self.cos_sin is None or self.cos_sin.shape[0] < max_pos:
+            self.cos_sin = tg_rope_table(max_pos, self.d, self.theta, device=dev)
+        f32 = dict(dtype=torch.float32, device=dev)
+        bf = dict(dtype=torch.bfloat16, device=dev)
+        nqkv = (self.hq + 2 * self.hkv) * self.d
+        self.planned = dict(
+            T=T, K=K, cu_h=cu_h, ck_h=ck_h,
+            cu=cu_h.to(dev), ck=ck_h.to(dev),
+            s=torch.empty(T, **f32), z=torch.empty(T, **f32), bias=torch.empty(T, **f32),
+            ws=torch.empty(tg_gate_score_workspace_size(T, self.hidden, self.width,
+                                                        len(lengths)), dtype=torch.uint8,
+                           device=dev),
+            kept_idx=torch.empty(K, dtype=torch.int32, device=dev),
+            kept_pos=torch.empty(K, dtype=torch.int32, device=dev),
+            kept_bias=torch.empty(K, **f32),
+            x=torch.empty((K, self.hidden), **bf),
+            qkv=torch.empty((K, nqkv), **bf),
+            o=torch.empty((K, self.hq * self.d), **bf),
+            caches=[(torch.empty((K, self.hkv * self.d), **bf),
+                     torch.empty((K, self.hkv * self.d), **bf)) for _ in self.layers],
+        )
+        return self.planned
+
+    def score(self, h, prunable, stream=None):
+        P = self.planned
+        g = self.gate
+        tg_gate_score(h, g["W1"], g["w2"], P["cu"], P["cu_h"], prunable, norm_w=g.get("norm_w"),
+                      eps_norm=self.norm_eps, eps_seq=self.seq_eps, s_out=P["s"], z_out=P["z"],
+                      bias_out=P["bias"], workspace=P["ws"], status=self.status, stream=stream)
+        self._mark("gate_score")
+
+    def select(self, prunable, z=None, stream=None):
+        P = self.planned
+        tg_topk_compact(P["z"] if z is None else z, prunable, P["cu"], P["cu_h"], P["ck"],
+                        P["ck_h"], P["kept_idx"], P["kept_pos"], P["kept_bias"],
+                        status=self.status, stream=stream)
+        self._mark("topk_compact")
+
+    def gather(self, h, stream=None):
+        """x = h[kept_idx]: the kept rows go up, pruned rows stop here."""
+        P = self.planned
+        if P["K"]:
+            tg_gather_rope(h, P["x"], row_idx=P["kept_idx"], status=self.status, stream=stream)
+            self._mark("gather")
+
+    def layer(self, i, stream=None):
+        """Upper layer i on the kept rows, in place on x; K/V land in cache i."""
+        P = self.planned
+        if P["K"] == 0:
+            return
+        L = self.layers[i]
+        ck, cv = P["caches"][i]
+        nq, nk = self.hq * self.d, self.hkv * self.d
+        qkv, o, x = P["qkv"], P["o"], P["x"]
+        tg_linear(x, L.Wqkv, qkv, rmsnorm=True, eps=self.norm_eps, status=self.status,
+                  stream=stream)
+        self._mark("qkv_proj")
+        tg_gather_rope(qkv, qkv, rope_pos=P["kept_pos"], rope_cols=(0, nq + nk),
+                       head_dim=self.d, cos_sin=self.cos_sin, status=self.status, stream=stream)
+        self._mark("rope")
+        tg_kv_compact(qkv[:, nq:nq + nk], qkv[:, nq + nk:], ck, cv, status=self.status,
+                      stream=stream)
+        self._mark("kv_compact")
+        tg_gated_attention(qkv[:, :nq], ck, cv, P["ck"], P["ck_h"], self.hq, self.hkv,
+                           P["kept_pos"], P["kept_bias"], L.gamma, L.beta, o=o,
+                           head_dim=self.d, status=self.status, stream=stream)
+        self._mark("attention")
+        tg_linear(o, L.Wo, x, residual=x, status=self.status, stream=stream)
+        self._mark("out_proj")
+
+    def upper_layers(self, h, stream=None):
+        self.gather(h, stream=stream)
+        for i in range(len(self.layers)):
+            self.layer(i, stream=stream)
+
+    def run(self, h, prunable, scores=None, stream=None):
+        """One gated prefill step.  The scorer always runs on h; with `scores` (raw
+        per-token scores, fp32 [T]) selection uses the sequence-normalised `scores`
+        instead of the scorer's own (the drawn planted-cluster workload)."""
+        self.score(h, prunable, stream=stream)
+        if scores is not None:
+            P = self.planned
+            tg_seq_rmsnorm(scores, P["cu"], P["cu_h"], prunable, self.seq_eps, P["z"],
+                           P["bias"], stream=stream)
+            self._mark("seq_rmsnorm")
+        self.select(prunable, stream=stream)
+        self.upper_layers(h, stream=stream)
+        return self.planned

@@ -1,0 +1,237 @@
+// tcgen05 GEMM C[M, N] = A[M, K] * W[N, K]^T for bf16 inputs with fp32 accumulation
+// in tensor memory, fed by TMA through a STAGES-deep shared-memory ring.
+//
+// Roles (192 threads):
+//   warp 0     one thread issues the TMA loads of A and W tiles (128-byte swizzle);
+//   warp 1     allocates TMEM; one thread issues tcgen05.mma (M=128, N=BN, K=16);
+//   warps 2-5  epilogue, one TMEM lane quarter each (thread = output row).  With a
+//              folded RMSNorm they also read every A stage from shared memory during
+//              the mainloop to accumulate the row's sum of squares, so the norm costs
+//              no extra HBM pass: RMSNorm(a) W^T = r * (a W^T), r = 1/sqrt(mean a^2 + eps).
+// Epilogues: EpiStore writes bf16 rows (optionally + residual); EpiScore reduces each
+// row to one scalar s = sum_f w2[f] SiLU(r * acc[f]) and writes per-32-row partial
+// sums of s^2 for the sequence normalisation.
+#pragma once
+#include <cuda.h>
+
+#include <cstdint>
+
+#include "tg_ptx.cuh"
+
+namespace tg {
+
+enum { EpiStore = 0, EpiScore = 1 };
+
+struct GemmParams {
+  int64_t M;
+  int N, K;
+  int rmsnorm;
+  float eps;
+  // EpiStore
+  uint16_t* c;
+  int64_t ldc;
+  const uint16_t* residual;
+  int64_t ldr;
+  // EpiScore
+  const float* w2;
+  float* s_out;
+  float* partial;  // [ceil(M / 32)]
+  uint32_t* status;
+};
+
+template <int BN, int STAGES>
+struct GemmCfg {
+  static constexpr int BM = 128, BK = 64;
+  static constexpr int A_BYTES = BM * BK * 2;
+  static constexpr int B_BYTES = BN * BK * 2;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int TILE_BYTES = STAGES * STAGE_BYTES;
+  static constexpr int BAR_BYTES = 256;
+  static constexpr int W2_BYTES = BN * 4;
+  static constexpr int SMEM = 1024 + TILE_BYTES + BAR_BYTES + W2_BYTES;
+  static constexpr int THREADS = 192;
+};
+
+template <int BN, int STAGES, int EPI>
+__global__ void __launch_bounds__(192, 1)
+    gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                GemmParams p) {
+  using Cfg = GemmCfg<BN, STAGES>;
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  unsigned char* smem = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  unsigned char* tiles = smem;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + Cfg::TILE_BYTES);
+  uint64_t* empty = full + STAGES;
+  uint64_t* acc_full = empty + STAGES;
+  uint64_t* drain = acc_full + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  float* w2s = reinterpret_cast<float*>(smem + Cfg::TILE_BYTES + Cfg::BAR_BYTES);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int64_t m0 = (int64_t)blockIdx.x * Cfg::BM;
+  const int n0 = blockIdx.y * BN;
+  const int nk = p.K / Cfg::BK;
+
+  if (tid == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1 + (p.rmsnorm ? 4 : 0));
+    }
+    mbar_init(acc_full, 1);
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, BN);
+    tmem_relinquish();
+  }
+  if (EPI == EpiScore) {
+    for (int i = tid; i < BN; i += Cfg::THREADS) w2s[i] = p.w2[n0 + i];
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int issued = 0;
+      for (int kb = 0; kb < nk; ++kb) {
+        const int s = kb % STAGES;
+        const uint32_t ph = (uint32_t)(kb / STAGES) & 1u;
+        if (!mbar_wait(&empty[s], ph ^ 1u, abort_flag, p.status)) break;
+        unsigned char* a_s = tiles + s * Cfg::STAGE_BYTES;
+        mbar_arrive_expect_tx(&full[s], Cfg::STAGE_BYTES);
+        tma_load_2d(a_s, &tmA, kb * Cfg::BK, (int32_t)m0, &full[s]);
+        tma_load_2d(a_s + Cfg::A_BYTES, &tmB, kb * Cfg::BK, n0, &full[s]);
+        ++issued;
+      }
+      // Never leave the CTA with bulk copies still landing in its shared memory.
+      for (int kb = issued - STAGES < 0 ? 0 : issued - STAGES; kb < issued; ++kb)
+        mbar_wait(&full[kb % STAGES], (uint32_t)(kb / STAGES) & 1u, nullptr, p.status);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16_f32(128, BN, false, false);
+      for (int kb = 0; kb < nk; ++kb) {
+        const int s = kb % STAGES;
+        const uint32_t ph = (uint32_t)(kb / STAGES) & 1u;
+        if (!mbar_wait(&full[s], ph, abort_flag, p.status)) break;
+        tc_fence_after();
+        const uint32_t a_addr = smem_u32(tiles + s * Cfg::STAGE_BYTES);
+        const uint32_t b_addr = a_addr + Cfg::A_BYTES;
+#pragma unroll
+        for (int k = 0; k < Cfg::BK / 16; ++k) {
+          const uint64_t ad = sw128_desc(a_addr + k * 32, 16, 1024);
+          const uint64_t bd = sw128_desc(b_addr + k * 32, 16, 1024);
+          mma_ss(tmem, ad, bd, idesc, (kb | k) != 0);
+        }
+        mma_commit(&empty[s]);
+      }
+      mma_commit(acc_full);
+      mma_commit(drain);
+      mbar_wait(drain, 0, nullptr, p.status);  // all MMAs retired before TMEM is freed
+    }
+  } else {
+    const int q = warp & 3;  // TMEM lane quarter this warp may access
+    const int row = q * 32 + lane;
+    const int64_t grow = m0 + row;
+    float ss = 0.f;
+    if (p.rmsnorm) {
+      for (int kb = 0; kb < nk; ++kb) {
+        const int s = kb % STAGES;
+        const uint32_t ph = (uint32_t)(kb / STAGES) & 1u;
+        if (!warp_all(mbar_wait(&full[s], ph, abort_flag, p.status))) break;
+        const unsigned char* rowp = tiles + s * Cfg::STAGE_BYTES + row * 128;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          // the row's 16-byte chunks in any order cover the whole row; XOR-ing the
+          // chunk index with the row keeps each quarter-warp on distinct banks
+          const uint4 v = *reinterpret_cast<const uint4*>(rowp + ((j ^ (row & 7)) << 4));
+          const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float2 f = unpack_bf16x2(w[e]);
+            ss = fmaf(f.x, f.x, ss);
+            ss = fmaf(f.y, f.y, ss);
+          }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[s]);
+      }
+    }
+    const float rscale = p.rmsnorm ? rsqrtf(ss / (float)p.K + p.eps) : 1.0f;
+    const bool ok = warp_all(mbar_wait(acc_full, 0, abort_flag, p.status));
+    tc_fence_after();
+    if (ok) {
+      const uint32_t tbase = tmem + ((uint32_t)(q * 32) << 16);
+      float score = 0.f;
+#pragma unroll 1
+      for (int c = 0; c < BN / 32; ++c) {
+        uint32_t r[32];
+        tmem_ld32(tbase + c * 32, r);
+        tmem_wait_ld();
+        if (EPI == EpiStore) {
+          if (grow < p.M) {
+            const int col = n0 + c * 32;
+            float v[32];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]) * rscale;
+            if (p.residual) {
+              const uint4* rp = reinterpret_cast<const uint4*>(p.residual + grow * p.ldr + col);
+#pragma unroll
+              for (int u = 0; u < 4; ++u) {
+                const uint4 t = rp[u];
+                const uint32_t w[4] = {t.x, t.y, t.z, t.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                  const float2 f = unpack_bf16x2(w[e]);
+                  v[u * 8 + 2 * e] += f.x;
+                  v[u * 8 + 2 * e + 1] += f.y;
+                }
+              }
+            }
+            uint4* cp = reinterpret_cast<uint4*>(p.c + grow * p.ldc + col);
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              uint4 t;
+              t.x = pack_bf16x2(v[u * 8 + 0], v[u * 8 + 1]);
+              t.y = pack_bf16x2(v[u * 8 + 2], v[u * 8 + 3]);
+              t.z = pack_bf16x2(v[u * 8 + 4], v[u * 8 + 5]);
+              t.w = pack_bf16x2(v[u * 8 + 6], v[u * 8 + 7]);
+              cp[u] = t;
+            }
+          }
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const float u = __uint_as_float(r[i]) * rscale;
+            score = fmaf(w2s[c * 32 + i], u / (1.0f + __expf(-u)), score);
+          }
+        }
+      }
+      if (EPI == EpiScore) {
+        if (grow < p.M) p.s_out[grow] = score;
+        float sq = grow < p.M ? score * score : 0.f;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) sq += __shfl_xor_sync(0xFFFFFFFFu, sq, o);
+        if (lane == 0 && m0 + q * 32 < p.M) p.partial[(m0 + q * 32) >> 5] = sq;
+      }
+    }
+    tc_fence_before();
+  }
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, BN);
+  }
+}
+
+}  // namespace tg

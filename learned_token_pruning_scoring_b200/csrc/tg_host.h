@@ -1,0 +1,52 @@
+// Host-side helpers shared by the entry points: error bookkeeping, device checks,
+// alignment checks and TMA tensor-map encoding (through the driver entry point, so
+// the library needs no link-time dependency on libcuda).
+#pragma once
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cstdint>
+
+#include "tokengate.h"
+
+namespace tg {
+
+void set_cuda_error(cudaError_t e);
+
+// TG_ERR_UNSUPPORTED_DEVICE unless the current device is compute capability 10.0.
+int check_device();
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Row stride (elements) times element size must be a multiple of 16 bytes.
+inline bool stride_ok(int64_t ld, int elem_bytes) { return ld > 0 && (ld * elem_bytes) % 16 == 0; }
+
+// Returns TG_ERR_CUDA (and records the error) if the last launch failed.
+int check_launch();
+
+// 2-D bf16 row-major tensor [rows, cols] with row stride `ld` elements, tiled in boxes
+// of box_cols x box_rows with 128-byte swizzle (box_cols * 2 must be 128).  Elements
+// outside the tensor read as zero.
+int make_tmap_bf16_2d(CUtensorMap* out, const void* base, uint64_t rows, uint64_t cols,
+                      uint64_t ld, uint32_t box_cols, uint32_t box_rows);
+
+// Number of SMs of the current device (cached).
+int sm_count();
+
+}  // namespace tg
+
+#define TG_CUDA_TRY(expr)                      \
+  do {                                         \
+    cudaError_t _e = (expr);                   \
+    if (_e != cudaSuccess) {                   \
+      ::tg::set_cuda_error(_e);                \
+      return TG_ERR_CUDA;                      \
+    }                                          \
+  } while (0)
+
+#define TG_TRY(expr)             \
+  do {                           \
+    int _rc = (expr);            \
+    if (_rc != TG_OK) return _rc; \
+  } while (0)

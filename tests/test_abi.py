@@ -1,0 +1,94 @@
+"""The C ABI library loads on the host and exports every symbol the header declares;
+host-only logic (argument checks that return before any launch, kept-count planning)
+is exercised without a GPU."""
+import ctypes as C
+import os
+import re
+
+import numpy as np
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "tokengate.h")
+
+
+def _declared():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(tg_[a-z0-9_]+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from learned_token_pruning_scoring_b200 import _lib
+    return _lib.load()
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = _declared()
+    assert len(names) >= 14
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_binding_covers_header(lib):
+    from learned_token_pruning_scoring_b200 import _lib
+    assert set(_declared()) == set(_lib.SIGNATURES)
+
+
+def test_error_strings(lib):
+    for code in range(0, -7, -1):
+        s = lib.tg_error_string(code)
+        assert s and s != b"unknown error"
+
+
+def test_plan_kept_rules(lib):
+    import learned_token_pruning_scoring_b200 as tg
+    import oracle as O
+    rng = np.random.default_rng(0)
+    for _ in range(50):
+        B = int(rng.integers(1, 6))
+        lengths = rng.integers(0, 40, B)
+        cu = np.concatenate([[0], np.cumsum(lengths)]).astype(np.int32)
+        pr = (rng.random(int(cu[-1])) < 0.7).astype(np.uint8)
+        nq = [int((pr[cu[b]:cu[b + 1]] == 0).sum()) for b in range(B)]
+        budgets = rng.integers(-3, 50, B)
+        got = tg.tg_plan_kept(cu, nq, budgets).numpy()
+        assert np.array_equal(got, O.kept_counts(pr, cu, budgets))
+
+
+def test_plan_kept_rejects_bad_layout(lib):
+    import learned_token_pruning_scoring_b200 as tg
+    with pytest.raises(tg.TokenGateError):
+        tg.tg_plan_kept([0, 5, 3], [0, 0], [1, 1])        # decreasing cu_seqlens
+    with pytest.raises(tg.TokenGateError):
+        tg.tg_plan_kept([0, 5], [6], [1])                 # more questions than tokens
+
+
+def test_host_side_argument_errors(lib):
+    """Shape and argument errors return before any device work."""
+    p = C.c_void_p(0x10000)  # never dereferenced: the calls fail their checks first
+    cu = (C.c_int32 * 2)(0, 8)
+    # attention: head_dim other than 128 is not implemented
+    assert lib.tg_gated_attention(p, 2048, p, 1024, p, 1024, p, cu, 1, 16, 8, 64, p, p, p,
+                                  1.0, p, 2048, None, None, None) == -6
+    # attention: odd GQA group
+    assert lib.tg_gated_attention(p, 2048, p, 1024, p, 1024, p, cu, 1, 3, 3, 128, p, p, p,
+                                  1.0, p, 2048, None, None, None) == -6
+    # projections: N not a multiple of 128, K not a multiple of 64
+    assert lib.tg_linear(p, 64, p, 64, p, 100, 4, 100, 64, 0, 0.0, None, 0, None, None) == -6
+    assert lib.tg_linear(p, 96, p, 96, p, 128, 4, 128, 96, 0, 0.0, None, 0, None, None) == -6
+    # scorer: width other than 256
+    assert lib.tg_gate_score(p, 2048, 8, 2048, None, p, 128, p, 1e-6, p, cu, 1, 1e-6, p, p,
+                             p, p, p, 1 << 20, None, None) == -6
+    # selection: K_b > N_b
+    ck = (C.c_int32 * 2)(0, 9)
+    assert lib.tg_topk_compact(p, p, p, cu, p, ck, 1, p, p, p, None, None) == -1
+    # gather: misaligned pointer
+    assert lib.tg_gather_rope(C.c_void_p(0x10002), 64, 4, None, 4, 64, None, 0, 0, 128, None,
+                              0, p, 64, None, None) == -2
+    # KV cache: slots beyond the cache
+    assert lib.tg_kv_compact(p, 64, p, 64, 10, None, 10, 64, p, p, 64, 12, 5, None, None) == -1
+    # workspace too small
+    assert lib.tg_gate_score(p, 2048, 8, 2048, None, p, 256, p, 1e-6, p, cu, 1, 1e-6, p, p,
+                             p, p, p, 16, None, None) == -4

@@ -1,0 +1,392 @@
+"""Per-kernel parity of the CUDA path against the CPU oracle (needs a B200).
+
+Every call goes through the C ABI (the ctypes binding).  Integer and index work is
+compared bit for bit; floating point within the stated tolerances:
+  * attention output: max-abs <= 2e-2 and mean-abs <= 1e-3 (bf16 inputs, fp32 accumulation);
+  * gate z: max-abs <= 1e-2, mean-abs <= 1e-3 with the unit RMSNorm weight of the
+    workloads.  A non-unit weight is folded into W1 rounded to bf16, a relative operand
+    rounding of up to 2^-9 per product (the same order as a bf16 RMSNorm output); the
+    z error then averages about 2^-9 |z| ~ 1.5e-3, so that case uses mean-abs <= 2.5e-3;
+  * bf16 outputs of projections / RoPE: the bf16 rounding of the result plus fp32
+    accumulation error, i.e. |err| <= 2^-7 |ref| + atol (atol stated per test).
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+import synthetic_inputs as S
+
+pytestmark = [pytest.mark.gpu,
+              pytest.mark.skipif(not torch.cuda.is_available(), reason="needs a CUDA device")]
+
+ATT_MAX, ATT_MEAN = 2e-2, 1e-3
+Z_MAX, Z_MEAN = 1e-2, 1e-3
+
+
+@pytest.fixture(scope="module")
+def tg():
+    import learned_token_pruning_scoring_b200 as m
+    assert m.tg_device_supported(torch.cuda.current_device())
+    return m
+
+
+def _dev(t):
+    return t.to("cuda")
+
+
+def _f64(t):
+    return O.as_f64(t)
+
+
+def _status():
+    return torch.zeros(1, dtype=torch.int32, device="cuda")
+
+
+# ------------------------------------------------------------------ RoPE table / gather
+
+def test_rope_table(tg):
+    tab = tg.tg_rope_table(4099, 128, 1.0e6).cpu().double().numpy()
+    ang = O.rope_angles(np.arange(4099), 128, 1.0e6)
+    assert np.abs(tab[..., 0] - np.cos(ang)).max() < 1e-7
+    assert np.abs(tab[..., 1] - np.sin(ang)).max() < 1e-7
+
+
+def test_rope_table_large_positions(tg):
+    tab = tg.tg_rope_table(131072, 128, 1.0e6).cpu().double().numpy()
+    rows = np.array([0, 1, 65535, 100003, 131071])
+    ang = O.rope_angles(rows, 128, 1.0e6)
+    assert np.abs(tab[rows, :, 0] - np.cos(ang)).max() < 1e-7
+    assert np.abs(tab[rows, :, 1] - np.sin(ang)).max() < 1e-7
+
+
+@pytest.mark.parametrize("n_src,n_rows,width", [(1000, 333, 2048), (50, 50, 8), (7, 3, 264)])
+def test_gather_bit_exact(tg, n_src, n_rows, width):
+    src = _dev(S.uniform_rows(n_src, width, seed=n_rows))
+    idx = torch.randint(0, n_src, (n_rows,), generator=torch.Generator().manual_seed(1),
+                        dtype=torch.int32)
+    out = tg.tg_gather_rope(src, row_idx=_dev(idx))
+    assert torch.equal(out.cpu(), src.cpu()[idx.long()])
+
+
+def test_gather_strided_views(tg):
+    big = _dev(S.uniform_rows(300, 4096, seed=3))
+    src = big[:, 1024:3072]
+    dst_big = torch.zeros((100, 2560), dtype=torch.bfloat16, device="cuda")
+    dst = dst_big[:, 256:2304]
+    idx = torch.arange(299, 0, -3, dtype=torch.int32)[:100]
+    tg.tg_gather_rope(src, dst, row_idx=_dev(idx))
+    assert torch.equal(dst.cpu(), src.cpu()[idx.long()])
+    assert torch.count_nonzero(dst_big[:, :256]) == 0 and torch.count_nonzero(dst_big[:, 2304:]) == 0
+
+
+def test_rope_in_place_against_oracle(tg):
+    Hq, Hkv, d = 16, 8, 128
+    n = 257
+    qkv = S.uniform_rows(n, (Hq + 2 * Hkv) * d, seed=5)
+    pos = torch.sort(torch.randperm(131072, generator=torch.Generator().manual_seed(2))[:n])[0]
+    pos = pos.to(torch.int32)
+    cs = tg.tg_rope_table(131072, d, 1.0e6)
+    x = _dev(qkv.clone())
+    tg.tg_gather_rope(x, x, rope_pos=_dev(pos), rope_cols=(0, (Hq + Hkv) * d), head_dim=d,
+                      cos_sin=cs)
+    got = _f64(x.cpu())
+    src = _f64(qkv)
+    want = np.concatenate([
+        O.rope(src[:, :(Hq + Hkv) * d].reshape(n, Hq + Hkv, d), pos, 1.0e6).reshape(n, -1),
+        src[:, (Hq + Hkv) * d:]], axis=1)
+    err = np.abs(got - want)
+    assert np.all(err <= 2.0 ** -7 * np.abs(want) + 1e-5), err.max()
+    # V columns are untouched bit for bit
+    assert torch.equal(x.cpu()[:, (Hq + Hkv) * d:], qkv[:, (Hq + Hkv) * d:])
+
+
+def test_kv_compact_bit_exact(tg):
+    qkv = _dev(S.uniform_rows(200, 4096, seed=9))
+    k, v = qkv[:, 2048:3072], qkv[:, 3072:]
+    ck = torch.zeros((260, 1024), dtype=torch.bfloat16, device="cuda")
+    cv = torch.zeros_like(ck)
+    tg.tg_kv_compact(k, v, ck, cv, slot_offset=60)
+    assert torch.equal(ck[60:].cpu(), k.cpu()) and torch.equal(cv[60:].cpu(), v.cpu())
+    assert torch.count_nonzero(ck[:60]) == 0
+    idx = _dev(torch.tensor([5, 0, 199, 17], dtype=torch.int32))
+    tg.tg_kv_compact(k, v, ck, cv, row_idx=idx, slot_offset=0)
+    assert torch.equal(ck[:4].cpu(), k.cpu()[idx.long().cpu()])
+    assert torch.equal(cv[:4].cpu(), v.cpu()[idx.long().cpu()])
+
+
+# ------------------------------------------------------------------ selection
+
+def _topk_case(tg, z32, prunable, lengths, budgets):
+    cu = np.concatenate([[0], np.cumsum(lengths)]).astype(np.int32)
+    nq = [int((prunable[cu[b]:cu[b + 1]] == 0).sum()) for b in range(len(lengths))]
+    ck = tg.tg_plan_kept(cu, nq, budgets)
+    assert np.array_equal(ck.numpy(), O.kept_counts(prunable, cu, budgets))
+    st = _status()
+    idx, pos, kb = tg.tg_topk_compact(_dev(torch.from_numpy(z32)),
+                                      _dev(torch.from_numpy(prunable)),
+                                      _dev(torch.from_numpy(cu)), cu, _dev(ck), ck, status=st)
+    assert tg.tg_status_read(st) == 0
+    w_idx, w_pos, w_kb = O.select_topk(z32, prunable, cu, ck.numpy())
+    assert np.array_equal(idx.cpu().numpy(), w_idx)
+    assert np.array_equal(pos.cpu().numpy(), w_pos)
+    assert np.array_equal(kb.cpu().numpy().view(np.uint32), w_kb.view(np.uint32))
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_topk_random_ragged(tg, seed):
+    rng = np.random.default_rng(seed)
+    lengths = [1, 31, 33, 1000, 4097, 0, 257][: 3 + seed % 5]
+    T = sum(lengths)
+    z = rng.normal(size=T).astype(np.float32)
+    if seed % 2:
+        z = (np.round(z * 3) / 3).astype(np.float32)  # many ties
+    pr = (rng.random(T) < 0.85).astype(np.uint8)
+    budgets = [int(rng.integers(0, n + 3)) for n in lengths]
+    _topk_case(tg, z, pr, lengths, budgets)
+
+
+def test_topk_special_values(tg):
+    z = np.array([np.nan, -0.0, 0.0, np.inf, -np.inf, 1.0, 1.0, np.nan, -0.0, 5.0, -1e30, 1e-45],
+                 dtype=np.float32)
+    pr = np.array([1, 1, 1, 1, 1, 1, 1, 1, 1, 0, 1, 1], dtype=np.uint8)
+    for budget in range(0, 13):
+        _topk_case(tg, z, pr, [12], [budget])
+
+
+def test_topk_all_equal_and_extremes(tg):
+    z = np.full(5000, 0.25, dtype=np.float32)
+    pr = np.ones(5000, dtype=np.uint8)
+    pr[-10:] = 0
+    for budget in (0, 10, 11, 2500, 4999, 5000, 9000):
+        _topk_case(tg, z, pr, [5000], [budget])
+
+
+def test_topk_planted_cluster_full_size(tg):
+    wl = S.n128k()
+    s = S.drawn_scores(wl)
+    pr = S.prunable_mask(wl).numpy()
+    z, _ = O.sequence_rmsnorm(s, wl.cu_seqlens(), pr)
+    _topk_case(tg, z.astype(np.float32), pr, list(wl.lengths), list(wl.budgets))
+
+
+def test_topk_ragged8_full_size(tg):
+    wl = S.ragged8()
+    T = wl.total_tokens
+    rng = np.random.default_rng(8)
+    z = rng.normal(size=T).astype(np.float32)
+    _topk_case(tg, z, S.prunable_mask(wl).numpy(), list(wl.lengths), list(wl.budgets))
+
+
+def test_topk_long_request_uncached_path(tg):
+    n = 300_000  # slices exceed the per-CTA shared-memory key cache
+    rng = np.random.default_rng(4)
+    z = rng.normal(size=n).astype(np.float32)
+    pr = np.ones(n, dtype=np.uint8)
+    pr[-100:] = 0
+    _topk_case(tg, z, pr, [n], [30_000])
+
+
+def test_topk_budget_inconsistency_sets_status(tg):
+    z = torch.randn(100, device="cuda")
+    pr = torch.ones(100, dtype=torch.uint8, device="cuda")
+    pr[-20:] = 0
+    cu = np.array([0, 100], dtype=np.int32)
+    ck = np.array([0, 10], dtype=np.int32)  # fewer than the 20 question tokens
+    st = _status()
+    idx = torch.full((10,), -7, dtype=torch.int32, device="cuda")
+    tg.tg_topk_compact(z, pr, _dev(torch.from_numpy(cu)), cu, _dev(torch.from_numpy(ck)), ck,
+                       kept_idx=idx, status=st)
+    assert tg.tg_status_read(st) & tg.STATUS_BUDGET
+    assert torch.all(idx == -7)  # nothing written
+
+
+# ------------------------------------------------------------------ gate score
+
+def _gate_case(tg, lengths, questions, seed, norm_w_random=False, rows=None):
+    wl = S.custom(lengths, questions, [0] * len(lengths), seeds=[seed + i for i in range(len(lengths))])
+    h = S.hidden_rows(wl)
+    gw = S.gate_weights(wl)
+    if norm_w_random:
+        gw["norm_w"] = (0.5 + torch.rand(wl.hidden, generator=torch.Generator().manual_seed(7)))
+        gw["norm_w"] = gw["norm_w"].to(torch.float32)
+    pr = S.prunable_mask(wl)
+    cu = np.array(wl.cu_seqlens(), dtype=np.int32)
+    st = _status()
+    s, z, bias = tg.tg_gate_score(_dev(h), _dev(gw["W1"]), _dev(gw["w2"]),
+                                  _dev(torch.from_numpy(cu)), cu, _dev(pr),
+                                  norm_w=_dev(gw["norm_w"]), status=st)
+    assert tg.tg_status_read(st) == 0
+    w_s = O.gate_score(h, gw["norm_w"], gw["W1"], gw["w2"])
+    w_z, w_b = O.sequence_rmsnorm(w_s, cu, pr)
+    g_s, g_z, g_b = s.cpu().double().numpy(), z.cpu().double().numpy(), bias.cpu().double().numpy()
+    scale = np.sqrt(np.mean(w_s ** 2))
+    assert np.abs(g_s - w_s).max() <= 1e-2 * scale
+    z_mean_tol = 2.5e-3 if norm_w_random else Z_MEAN
+    assert np.abs(g_z - w_z).max() <= Z_MAX and np.abs(g_z - w_z).mean() <= z_mean_tol
+    assert np.abs(g_b - w_b).max() <= Z_MAX
+    assert np.all(g_b[pr.numpy() == 0] == 0)
+    return g_z, w_z
+
+
+def test_gate_score_n1k(tg):
+    _gate_case(tg, [1024], [64], seed=0)
+
+
+def test_gate_score_ragged_requests_and_norm_weight(tg):
+    # lengths not multiples of the 128-row tile or the 32-row partial chunks
+    _gate_case(tg, [100, 37, 900, 1, 31, 33], [5, 0, 64, 1, 3, 33], seed=3, norm_w_random=True)
+
+
+def test_gate_score_n16k_full(tg):
+    _gate_case(tg, [16384], [64], seed=0)
+
+
+def test_gate_score_deterministic(tg):
+    wl = S.custom([5000, 3000], [64, 16], [0, 0])
+    h = _dev(S.hidden_rows(wl))
+    gw = {k: _dev(v) for k, v in S.gate_weights(wl).items()}
+    pr = _dev(S.prunable_mask(wl))
+    cu = np.array(wl.cu_seqlens(), dtype=np.int32)
+    outs = [tg.tg_gate_score(h, gw["W1"], gw["w2"], _dev(torch.from_numpy(cu)), cu, pr,
+                             norm_w=gw["norm_w"]) for _ in range(2)]
+    for a, b in zip(*outs):
+        assert torch.equal(a, b)
+
+
+# ------------------------------------------------------------------ projections
+
+@pytest.mark.parametrize("M,N,K,rms,res", [(1, 128, 64, False, False), (100, 256, 2048, True, False),
+                                           (1638, 4096, 2048, True, False),
+                                           (1638, 2048, 2048, False, True),
+                                           (300, 384, 192, True, True)])
+def test_linear_against_oracle(tg, M, N, K, rms, res):
+    a = S.uniform_rows(M, K, seed=M + 1)
+    w = S.uniform_rows(N, K, seed=N + 2, scale=0.02)
+    r = S.uniform_rows(M, N, seed=3) if res else None
+    c = tg.tg_linear(_dev(a), _dev(w), rmsnorm=rms, residual=_dev(r) if res else None)
+    A = O.rmsnorm_rows(a) if rms else _f64(a)
+    want = A @ _f64(w).T + (_f64(r) if res else 0.0)
+    got = _f64(c.cpu())
+    err = np.abs(got - want)
+    assert np.all(err <= 2.0 ** -7 * np.abs(want) + 2e-3), err.max()
+
+
+def test_linear_residual_in_place(tg):
+    x = _dev(S.uniform_rows(257, 256, seed=1))
+    x0 = x.clone()
+    o = _dev(S.uniform_rows(257, 512, seed=2))
+    w = _dev(S.uniform_rows(256, 512, seed=3, scale=0.02))
+    tg.tg_linear(o, w, x, residual=x)
+    want = _f64(x0.cpu()) + _f64(o.cpu()) @ _f64(w.cpu()).T
+    err = np.abs(_f64(x.cpu()) - want)
+    assert np.all(err <= 2.0 ** -7 * np.abs(want) + 2e-3)
+
+
+# ------------------------------------------------------------------ attention
+
+def _attn_inputs(lengths, Hq, Hkv, seed, pos_spread=4, dense=False):
+    d = 128
+    g = torch.Generator().manual_seed(seed)
+    Kt = int(sum(lengths))
+    q = (torch.randn((Kt, Hq * d), generator=g)).to(torch.bfloat16)
+    k = (torch.randn((Kt, Hkv * d), generator=g)).to(torch.bfloat16)
+    v = (torch.randn((Kt, Hkv * d), generator=g)).to(torch.bfloat16)
+    pos, bias = [], []
+    for n in lengths:
+        if dense:
+            pos.append(torch.arange(n, dtype=torch.int32))
+        else:
+            pos.append(torch.sort(torch.randperm(max(1, pos_spread * n + 5), generator=g)[:n])[0]
+                       .to(torch.int32))
+        b = torch.randn((n,), generator=g) * (torch.rand((n,), generator=g) < 0.9)
+        bias.append(b.to(torch.float32))
+    pos = torch.cat(pos) if pos else torch.zeros(0, dtype=torch.int32)
+    bias = torch.cat(bias) if bias else torch.zeros(0)
+    gamma = (0.5 + 1.5 * torch.rand((Hq,), generator=g)).to(torch.float32)
+    cu = np.concatenate([[0], np.cumsum(lengths)]).astype(np.int32)
+    return q, k, v, pos, bias, gamma, cu
+
+
+def _run_attention(tg, q, k, v, pos, bias, gamma, beta, cu, Hq, Hkv, lse=True):
+    Kt = q.shape[0]
+    lse_t = torch.full((Hq, Kt), float("nan"), device="cuda") if lse else None
+    st = _status()
+    o = tg.tg_gated_attention(_dev(q), _dev(k), _dev(v), _dev(torch.from_numpy(cu)), cu, Hq, Hkv,
+                              _dev(pos), _dev(bias), _dev(gamma), beta, lse=lse_t, status=st)
+    assert tg.tg_status_read(st) == 0
+    return o.cpu(), (lse_t.cpu() if lse else None)
+
+
+def _check_attention(o_gpu, lse_gpu, q, k, v, pos, bias, gamma, beta, cu, Hq, Hkv, rows=None):
+    d = 128
+    Kt = q.shape[0]
+    Q = _f64(q).reshape(Kt, Hq, d)
+    K = _f64(k).reshape(Kt, Hkv, d)
+    V = _f64(v).reshape(Kt, Hkv, d)
+    want, wlse = O.gated_attention(Q, K, V, cu, pos, bias, gamma, beta, rows=rows)
+    got = _f64(o_gpu).reshape(Kt, Hq, d)
+    sel = slice(None) if rows is None else np.asarray(rows)
+    err = np.abs(got[sel] - want[sel])
+    assert err.max() <= ATT_MAX, err.max()
+    assert err.mean() <= ATT_MEAN, err.mean()
+    if lse_gpu is not None:
+        lerr = np.abs(_f64(lse_gpu)[:, sel] - wlse[:, sel])
+        assert lerr.max() <= 1e-3, lerr.max()
+
+
+@pytest.mark.parametrize("lengths", [[1], [5], [127], [128], [129], [300], [256, 1, 129, 77]])
+def test_attention_small_shapes(tg, lengths):
+    q, k, v, pos, bias, gamma, cu = _attn_inputs(lengths, 16, 8, seed=sum(lengths))
+    o, lse = _run_attention(tg, q, k, v, pos, bias, gamma, 1.0, cu, 16, 8)
+    _check_attention(o, lse, q, k, v, pos, bias, gamma, 1.0, cu, 16, 8)
+
+
+def test_attention_group4_and_beta(tg):
+    q, k, v, pos, bias, gamma, cu = _attn_inputs([700, 190], 8, 2, seed=11)
+    o, lse = _run_attention(tg, q, k, v, pos, bias, gamma, 0.7, cu, 8, 2)
+    _check_attention(o, lse, q, k, v, pos, bias, gamma, 0.7, cu, 8, 2)
+
+
+def test_attention_n16k_kept_1638(tg):
+    q, k, v, pos, bias, gamma, cu = _attn_inputs([1638], 16, 8, seed=1638, pos_spread=10)
+    o, lse = _run_attention(tg, q, k, v, pos, bias, gamma, 1.0, cu, 16, 8)
+    _check_attention(o, lse, q, k, v, pos, bias, gamma, 1.0, cu, 16, 8)
+
+
+def test_attention_n128k_kept_13107_sampled_rows(tg):
+    q, k, v, pos, bias, gamma, cu = _attn_inputs([13107], 16, 8, seed=13107, pos_spread=10)
+    o, lse = _run_attention(tg, q, k, v, pos, bias, gamma, 1.0, cu, 16, 8)
+    rng = np.random.default_rng(0)
+    rows = np.unique(np.concatenate([[0, 1, 127, 128, 13106], rng.integers(0, 13107, 120)]))
+    _check_attention(o, lse, q, k, v, pos, bias, gamma, 1.0, cu, 16, 8, rows=rows)
+
+
+def test_attention_dense_matches_sdpa(tg):
+    """K = N, gamma = 0, positions = ranks: plain causal GQA attention (library SDPA)."""
+    n = 1000
+    q, k, v, pos, bias, gamma, cu = _attn_inputs([n], 16, 8, seed=5, dense=True)
+    o, _ = _run_attention(tg, q, k, v, pos, bias, torch.zeros(16), 1.0, cu, 16, 8, lse=False)
+    qt = q.view(n, 16, 128).permute(1, 0, 2)[None].cuda().float()
+    kt = k.view(n, 8, 128).permute(1, 0, 2).repeat_interleave(2, 0)[None].cuda().float()
+    vt = v.view(n, 8, 128).permute(1, 0, 2).repeat_interleave(2, 0)[None].cuda().float()
+    ref = torch.nn.functional.scaled_dot_product_attention(qt, kt, vt, is_causal=True)
+    ref = ref[0].permute(1, 0, 2).reshape(n, -1).cpu().double()
+    err = (o.double() - ref).abs()
+    assert err.max() <= ATT_MAX and err.mean() <= ATT_MEAN
+
+
+def test_attention_rows_sum_to_one(tg):
+    q, k, v, pos, bias, gamma, cu = _attn_inputs([517, 300], 16, 8, seed=2)
+    ones = torch.ones_like(v)
+    o, _ = _run_attention(tg, q, k, ones, pos, bias, gamma, 1.0, cu, 16, 8, lse=False)
+    assert (o.double() - 1.0).abs().max() <= 2 ** -8
+
+
+def test_attention_deterministic(tg):
+    q, k, v, pos, bias, gamma, cu = _attn_inputs([900], 16, 8, seed=3)
+    a, la = _run_attention(tg, q, k, v, pos, bias, gamma, 1.0, cu, 16, 8)
+    b, lb = _run_attention(tg, q, k, v, pos, bias, gamma, 1.0, cu, 16, 8)
+    assert torch.equal(a, b) and torch.equal(la, lb)

@@ -1,0 +1,56 @@
+"""Tolerance derivation for the multi-layer end-to-end check (CPU only, not collected).
+
+Runs the oracle's gated layers twice from the same seeded inputs: once in float64,
+once with bf16 rounding at the points where the CUDA path rounds (q, k, v after the
+projection and after RoPE, the attention output O, the residual stream x).  The gap
+between the two is the error a correct bf16 implementation is expected to show; the
+end-to-end test's bounds are set above it.  Usage: python tests/tolerance_study.py
+"""
+import os
+import sys
+
+import numpy as np
+import torch
+
+sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
+import oracle as O  # noqa: E402
+import synthetic_inputs as S  # noqa: E402
+
+
+def bf16(x):
+    return (torch.from_numpy(np.ascontiguousarray(x)).to(torch.float32)
+            .to(torch.bfloat16).to(torch.float64).numpy())
+
+
+def layer_rounded(x, L, cu_kept, pos, bias, wl):
+    hq, hkv, d = wl.n_q_heads, wl.n_kv_heads, wl.head_dim
+    Kt = x.shape[0]
+    qkv = bf16(O.rmsnorm_rows(x) @ O.as_f64(L["Wqkv"]).T)
+    q = bf16(O.rope(qkv[:, :hq * d].reshape(Kt, hq, d), pos, wl.rope_theta))
+    k = bf16(O.rope(qkv[:, hq * d:(hq + hkv) * d].reshape(Kt, hkv, d), pos, wl.rope_theta))
+    v = qkv[:, (hq + hkv) * d:].reshape(Kt, hkv, d)
+    o, _ = O.gated_attention(q, k, v, cu_kept, pos, bias, L["gamma"], L["beta"])
+    return bf16(x + bf16(o.reshape(Kt, -1)) @ O.as_f64(L["Wo"]).T)
+
+
+def study(wl, report=(1, 2, 4, 8, 16, 28)):
+    h, pr, gate = S.hidden_rows(wl), S.prunable_mask(wl), S.gate_weights(wl)
+    ref = O.prefill(h, pr, wl.cu_seqlens(), wl.budgets, gate, [], wl.n_q_heads,
+                    wl.n_kv_heads, wl.head_dim, wl.rope_theta)
+    ck, pos, kb = ref["cu_kept"], ref["kept_pos"], ref["kept_bias"]
+    x64 = O.gather_rows(h, ref["kept_idx"])
+    xr = x64.copy()
+    for i in range(wl.n_layers):
+        L = S.layer_weights(wl, i)
+        x64, *_ = O.gated_layer(x64, L["Wqkv"], L["Wo"], L["gamma"], L["beta"], ck, pos, kb,
+                                wl.n_q_heads, wl.n_kv_heads, wl.head_dim, wl.rope_theta)
+        xr = layer_rounded(xr, L, ck, pos, kb, wl)
+        if i + 1 in report or i + 1 == wl.n_layers:
+            e = np.abs(xr - x64)
+            print(f"{wl.name} layer {i + 1}: max {e.max():.4f} mean {e.mean():.5f} "
+                  f"|x|max {np.abs(x64).max():.2f}", flush=True)
+
+
+if __name__ == "__main__":
+    study(S.custom([700, 1500, 333], [16, 64, 5], [100, 800, 300], n_layers=2, name="ragged3"))
+    study(S.n16k())
