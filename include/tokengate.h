@@ -52,6 +52,7 @@ typedef void* tg_stream_t;  /* cudaStream_t */
 #define TG_ERR_WORKSPACE (-4)          /* workspace missing or smaller than required */
 #define TG_ERR_CUDA (-5)               /* a CUDA runtime/driver call failed; see tg_last_cuda_error */
 #define TG_ERR_UNSUPPORTED_SHAPE (-6)  /* a dimension outside what the kernels implement */
+#define TG_ERR_SCRATCH_LIMIT (-7)      /* larger than the fixed scratch of tg_gate_score_noalloc */
 
 /* Device status bits (OR-ed into the caller's status word by kernels). */
 #define TG_STATUS_TIMEOUT 0x1u /* a bounded wait ran out; outputs of that call are invalid */
@@ -148,6 +149,31 @@ int tg_gate_score(const tg_bf16* h, int64_t ld_h, int64_t total_tokens, int hidd
 int tg_seq_rmsnorm(const float* s, const int32_t* cu_seqlens, const int32_t* cu_seqlens_host,
                    int batch, const uint8_t* prunable, float eps_seq, float* z_out,
                    float* bias_out, tg_stream_t stream);
+
+/*
+ * tg_gate_score without a workspace argument, for callers that cannot allocate device
+ * memory (for example a serving engine that plans all device memory ahead and forbids
+ * allocation during a request, a plug-in limited to the buffers its host framework
+ * hands it, or a path that cannot afford cudaMalloc's implicit device synchronisation).
+ * The pages have no counterpart of this call: it is a deployment convenience only.
+ * Same arguments, results and errors as tg_gate_score, minus workspace/workspace_bytes.
+ * Scratch comes from one array compiled into the library (about 2.2 MB), which every GPU
+ * that loads the library keeps until the process exits.  Limits: total_tokens <=
+ * TG_NOALLOC_MAX_TOKENS and hidden <= TG_NOALLOC_MAX_HIDDEN, else TG_ERR_SCRATCH_LIMIT
+ * and nothing is launched.  The first call on each device looks up the array's device
+ * address (cudaGetSymbolAddress); make that first call before any stream capture.  All
+ * calls share the one array: calls whose GPU work can overlap (different streams, or
+ * several host threads) race on it, so serialise them.  The library allocates nothing
+ * here (no cudaMalloc/cudaFree, no allocating library routine).
+ */
+#define TG_NOALLOC_MAX_TOKENS (1 << 20)
+#define TG_NOALLOC_MAX_HIDDEN 4096
+int tg_gate_score_noalloc(const tg_bf16* h, int64_t ld_h, int64_t total_tokens, int hidden,
+                          const float* norm_w, const tg_bf16* W1, int width, const float* w2,
+                          float eps_norm, const int32_t* cu_seqlens,
+                          const int32_t* cu_seqlens_host, int batch, float eps_seq,
+                          const uint8_t* prunable, float* s_out, float* z_out,
+                          float* bias_out, uint32_t* status, tg_stream_t stream);
 
 /* ------------------------------------------------------------------ selection */
 

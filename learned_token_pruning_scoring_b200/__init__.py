@@ -24,7 +24,7 @@ from . import _lib
 __all__ = [
     "TokenGateError", "lib", "tg_version", "tg_device_supported", "tg_plan_kept",
     "tg_rope_table", "tg_gate_score_workspace_size", "tg_gate_score", "tg_topk_compact",
-    "tg_seq_rmsnorm", "tg_gather_rope", "tg_kv_compact", "tg_gated_attention", "tg_linear",
+    "tg_gate_score_noalloc", "tg_seq_rmsnorm", "tg_gather_rope", "tg_kv_compact", "tg_gated_attention", "tg_linear",
     "tg_status_clear", "tg_status_read", "GatedPrefill", "STATUS_TIMEOUT", "STATUS_BUDGET",
     "STATUS_BOUNDS",
 ]
@@ -145,6 +145,32 @@ def tg_gate_score(h, W1, w2, cu_seqlens, cu_seqlens_host, prunable, norm_w=None,
                            _ptr(prunable), _ptr(s_out), _ptr(z_out), _ptr(bias_out),
                            _ptr(workspace), workspace.numel(), _ptr(status), _stream(stream))
     _check(rc, "tg_gate_score")
+    _count(3 if norm_w is not None else 2)
+    return s_out, z_out, bias_out
+
+
+def tg_gate_score_noalloc(h, W1, w2, cu_seqlens, cu_seqlens_host, prunable, norm_w=None,
+                          eps_norm=1e-6, eps_seq=1e-6, s_out=None, z_out=None, bias_out=None,
+                          status=None, stream=None):
+    """tg_gate_score without a workspace: for callers that may not allocate device
+    memory.  Scratch is a fixed array inside the library (limits and the one-time
+    per-device set-up are described in include/tokengate.h); calls that can overlap on
+    the GPU share that array and race, so serialise them.  This wrapper allocates the
+    outputs only when they are not passed in."""
+    ld_h = _mat(h, "h")
+    T, hidden = h.shape
+    width = W1.shape[0]
+    cuh = _host_i32(cu_seqlens_host)
+    batch = cuh.numel() - 1
+    dev = h.device
+    s_out = torch.empty(T, dtype=torch.float32, device=dev) if s_out is None else s_out
+    z_out = torch.empty(T, dtype=torch.float32, device=dev) if z_out is None else z_out
+    bias_out = torch.empty(T, dtype=torch.float32, device=dev) if bias_out is None else bias_out
+    rc = lib.tg_gate_score_noalloc(_ptr(h), ld_h, T, hidden, _ptr(norm_w), _ptr(W1), width,
+                                   _ptr(w2), float(eps_norm), _ptr(cu_seqlens), _ptr(cuh), batch,
+                                   float(eps_seq), _ptr(prunable), _ptr(s_out), _ptr(z_out),
+                                   _ptr(bias_out), _ptr(status), _stream(stream))
+    _check(rc, "tg_gate_score_noalloc")
     _count(3 if norm_w is not None else 2)
     return s_out, z_out, bias_out
 

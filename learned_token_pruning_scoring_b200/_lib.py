@@ -30,6 +30,8 @@ SIGNATURES = {
     "tg_gate_score_workspace_size": (_sz, [_i64, _i32, _i32, _i32]),
     "tg_gate_score": (_i32, [_p, _i64, _i64, _i32, _p, _p, _i32, _p, _f32, _p, _p, _i32, _f32,
                              _p, _p, _p, _p, _p, _sz, _p, _p]),
+    "tg_gate_score_noalloc": (_i32, [_p, _i64, _i64, _i32, _p, _p, _i32, _p, _f32, _p, _p, _i32,
+                                     _f32, _p, _p, _p, _p, _p, _p]),
     "tg_seq_rmsnorm": (_i32, [_p, _p, _p, _i32, _p, _f32, _p, _p, _p]),
     "tg_topk_compact": (_i32, [_p, _p, _p, _p, _p, _p, _i32, _p, _p, _p, _p, _p]),
     "tg_gather_rope": (_i32, [_p, _i64, _i64, _p, _i64, _i32, _p, _i32, _i32, _i32, _p, _i32,

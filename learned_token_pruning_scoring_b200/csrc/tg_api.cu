@@ -88,6 +88,9 @@ const char* tg_error_string(int code) {
     case TG_ERR_WORKSPACE: return "workspace missing or too small";
     case TG_ERR_CUDA: return "CUDA runtime or driver call failed";
     case TG_ERR_UNSUPPORTED_SHAPE: return "shape not implemented by the kernels";
+    case TG_ERR_SCRATCH_LIMIT:
+      return "size exceeds the fixed scratch of tg_gate_score_noalloc "
+             "(TG_NOALLOC_MAX_TOKENS / TG_NOALLOC_MAX_HIDDEN)";
     default: return "unknown error";
   }
 }

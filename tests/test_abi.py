@@ -37,7 +37,7 @@ def test_binding_covers_header(lib):
 
 
 def test_error_strings(lib):
-    for code in range(0, -7, -1):
+    for code in range(0, -8, -1):
         s = lib.tg_error_string(code)
         assert s and s != b"unknown error"
 
