@@ -51,7 +51,7 @@ def parse_args():
     ap.add_argument("--launch", choices=["graph", "eager"], default="graph")
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--cpu-sample-layers", type=int, default=2)
+    ap.add_argument("--cpu-sample-layers", type=int, default=12)
     return ap.parse_args()
 
 
@@ -369,12 +369,17 @@ def run_ours(args, rank, world):
 
 
 def load_traffic(kernel, workload_name):
-    """Per-launch DRAM bytes from a committed ncu summary, if one exists for this kernel."""
+    """Per-launch DRAM bytes from a committed ncu summary, if one exists for this kernel
+    and was taken on the kernel source as it is now (sha256 match); else None."""
+    import hashlib
     path = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(path) as f:
-            d = json.load(f)
-        return d.get(workload_name, {}).get(kernel)
+            e = json.load(f)[workload_name][kernel]
+        with open(os.path.join(ROOT, e["source"]), "rb") as f:
+            if hashlib.sha256(f.read()).hexdigest() != e["source_sha256"]:
+                return None
+        return int(e["bytes_per_launch"])
     except Exception:
         return None
 
