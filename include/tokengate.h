@@ -265,16 +265,27 @@ int tg_kv_compact(const tg_bf16* k, int64_t ld_k, const tg_bf16* v, int64_t ld_v
  * (ld_o).  lse: float32 [n_q_heads, K_tot] natural-log log-sum-exp, or NULL.
  * kept_pos int32 [K_tot]; kept_bias float32 [K_tot]; gamma float32 [n_q_heads].
  * Implemented for head_dim = 128 and an even group size n_q_heads / n_kv_heads; q, k,
- * v, o 16-byte aligned with strides that are multiples of 8.  The kernel runs the two
- * q heads of a kv head on tcgen05 tensor cores with S and O accumulators in tensor
- * memory and a TMA-fed K/V ring.  status may be NULL.
+ * v, o 16-byte aligned with strides that are multiples of 8; at most 512 requests per
+ * call.  The kernel runs the two q heads of a kv head on tcgen05 tensor cores with S and
+ * O accumulators in tensor memory and a TMA-fed K/V ring.  workspace (16-byte aligned,
+ * tg_gated_attention_workspace_size bytes) may be NULL.  status may be NULL.
  */
 int tg_gated_attention(const tg_bf16* q, int64_t ld_q, const tg_bf16* k, int64_t ld_k,
                        const tg_bf16* v, int64_t ld_v, const int32_t* cu_kept,
                        const int32_t* cu_kept_host, int batch, int n_q_heads,
                        int n_kv_heads, int head_dim, const int32_t* kept_pos,
                        const float* kept_bias, const float* gamma, float beta, tg_bf16* o,
-                       int64_t ld_o, float* lse, uint32_t* status, tg_stream_t stream);
+                       int64_t ld_o, float* lse, void* workspace, size_t workspace_bytes,
+                       uint32_t* status, tg_stream_t stream);
+
+/*
+ * Workspace bytes that let tg_gated_attention split the key range of long causal query
+ * tiles over several CTAs (balancing the triangle over all SMs; a second kernel merges
+ * the parts).  0 when the layout needs no split.  With a smaller or NULL workspace the
+ * call still runs, one CTA per query tile and kv-head pair.
+ */
+size_t tg_gated_attention_workspace_size(const int32_t* cu_kept_host, int batch,
+                                         int n_q_heads, int n_kv_heads, int head_dim);
 
 /* ------------------------------------------------------------------ projections */
 
@@ -291,6 +302,30 @@ int tg_gated_attention(const tg_bf16* q, int64_t ld_q, const tg_bf16* k, int64_t
 int tg_linear(const tg_bf16* a, int64_t lda, const tg_bf16* w, int64_t ldw, tg_bf16* c,
               int64_t ldc, int64_t M, int N, int K, int rmsnorm_a, float eps,
               const tg_bf16* residual, int64_t ld_res, uint32_t* status, tg_stream_t stream);
+
+/*
+ * One gated layer's QKV projection with RoPE and the compacted KV-cache write fused into
+ * the GEMM epilogue ([aiwillknow] figure 1(a)(b): kept tokens keep their original
+ * positions, upper layers store KV only for kept tokens; [farwalk] How does TokenGate
+ * learned token pruning work?):
+ *   a = RMSNorm(x) (weight 1, eps);  [Q | K | V] = a w_qkv^T;
+ *   q_out[r]                = RoPE(Q[r], pos[r])
+ *   cache_k[slot_offset+r]  = RoPE(K[r], pos[r]);  cache_v[slot_offset+r] = V[r]
+ * RoPE is rotate-half on every head with the table of tg_rope_table, applied to the fp32
+ * accumulators before the single rounding to bf16.  Equivalent to tg_linear (rmsnorm=1)
+ * followed by tg_gather_rope (rope mode) and tg_kv_compact, in one kernel.
+ * x: bf16 [M, hidden] (ld_x); w_qkv: bf16 [(n_q_heads + 2 n_kv_heads) * head_dim, hidden]
+ * (rows: Wq, Wk, Wv); pos: int32 [M] (values < max_pos, else TG_STATUS_BOUNDS and the
+ * row uses position 0); q_out: bf16 [M, n_q_heads * head_dim] (ld_q); cache_k/cache_v:
+ * bf16 rows of n_kv_heads * head_dim (ld_cache).  head_dim = 128, hidden multiple of 64.
+ * status may be NULL.
+ */
+int tg_qkv_rope_cache(const tg_bf16* x, int64_t ld_x, const tg_bf16* w_qkv, int64_t ld_w,
+                      int64_t M, int hidden, int n_q_heads, int n_kv_heads, int head_dim,
+                      float eps, const int32_t* pos, const float* cos_sin, int max_pos,
+                      tg_bf16* q_out, int64_t ld_q, tg_bf16* cache_k, tg_bf16* cache_v,
+                      int64_t ld_cache, int64_t slot_offset, uint32_t* status,
+                      tg_stream_t stream);
 
 #ifdef __cplusplus
 }

@@ -242,21 +242,34 @@ def tg_kv_compact(k, v, cache_k, cache_v, row_idx=None, n_rows=None, slot_offset
     _count()
 
 
+def tg_gated_attention_workspace_size(cu_kept_host, n_q_heads, n_kv_heads, head_dim=128) -> int:
+    ckh = _host_i32(cu_kept_host)
+    return int(lib.tg_gated_attention_workspace_size(_ptr(ckh), ckh.numel() - 1, n_q_heads,
+                                                     n_kv_heads, head_dim))
+
+
 def tg_gated_attention(q, k, v, cu_kept, cu_kept_host, n_q_heads, n_kv_heads, kept_pos,
-                       kept_bias, gamma, beta, o=None, lse=None, head_dim=128, status=None,
-                       stream=None):
+                       kept_bias, gamma, beta, o=None, lse=None, head_dim=128, workspace=None,
+                       status=None, stream=None):
+    """Token-gated attention.  `workspace=None` allocates the split-KV workspace the
+    layout asks for (pass a uint8 tensor to reuse one; an empty one disables splitting)."""
     ld_q, ld_k, ld_v = _mat(q, "q"), _mat(k, "k"), _mat(v, "v")
     ckh = _host_i32(cu_kept_host)
     batch = ckh.numel() - 1
     if o is None:
         o = torch.empty((q.shape[0], n_q_heads * head_dim), dtype=q.dtype, device=q.device)
     ld_o = _mat(o, "o")
+    if workspace is None:
+        need = tg_gated_attention_workspace_size(ckh, n_q_heads, n_kv_heads, head_dim)
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    ws_ptr = _ptr(workspace) if workspace.numel() else None
     rc = lib.tg_gated_attention(_ptr(q), ld_q, _ptr(k), ld_k, _ptr(v), ld_v, _ptr(cu_kept),
                                 _ptr(ckh), batch, n_q_heads, n_kv_heads, head_dim,
                                 _ptr(kept_pos), _ptr(kept_bias), _ptr(gamma), float(beta),
-                                _ptr(o), ld_o, _ptr(lse), _ptr(status), _stream(stream))
+                                _ptr(o), ld_o, _ptr(lse), ws_ptr, workspace.numel(),
+                                _ptr(status), _stream(stream))
     _check(rc, "tg_gated_attention")
-    _count()
+    _count(2 if (ws_ptr is not None and workspace.numel() > 0) else 1)
     return o
 
 
@@ -273,6 +286,27 @@ def tg_linear(a, w, c=None, rmsnorm=False, eps=1e-6, residual=None, status=None,
     _check(rc, "tg_linear")
     _count()
     return c
+
+
+def tg_qkv_rope_cache(x, w_qkv, pos, cos_sin, cache_k, cache_v, n_q_heads, n_kv_heads,
+                      q_out=None, head_dim=128, eps=1e-6, slot_offset=0, status=None,
+                      stream=None):
+    """Fused QKV projection (RMSNorm folded) + RoPE at `pos` + compacted KV-cache write."""
+    ld_x, ld_w = _mat(x, "x"), _mat(w_qkv, "w_qkv")
+    M, hidden = x.shape
+    if q_out is None:
+        q_out = torch.empty((M, n_q_heads * head_dim), dtype=x.dtype, device=x.device)
+    ld_q = _mat(q_out, "q_out")
+    ld_c = _mat(cache_k, "cache_k")
+    if _mat(cache_v, "cache_v") != ld_c:
+        raise ValueError("cache_k and cache_v must share a row stride")
+    rc = lib.tg_qkv_rope_cache(_ptr(x), ld_x, _ptr(w_qkv), ld_w, M, hidden, n_q_heads, n_kv_heads,
+                               head_dim, float(eps), _ptr(pos), _ptr(cos_sin), cos_sin.shape[0],
+                               _ptr(q_out), ld_q, _ptr(cache_k), _ptr(cache_v), ld_c,
+                               int(slot_offset), _ptr(status), _stream(stream))
+    _check(rc, "tg_qkv_rope_cache")
+    _count()
+    return q_out
 
 
 # ----------------------------------------------------------------------------- pipeline
@@ -308,6 +342,8 @@ class GatedPrefill:
         self.planned = None
         # optional callable(stage_name) invoked after each launch (e.g. to record events)
         self.marker = None
+        # QKV projection, RoPE and KV-cache write as one fused kernel (else three)
+        self.fused_qkv = True
 
     def _mark(self, name):
         if self.marker is not None:
@@ -341,6 +377,8 @@ class GatedPrefill:
             x=torch.empty((K, self.hidden), **bf),
             qkv=torch.empty((K, nqkv), **bf),
             o=torch.empty((K, self.hq * self.d), **bf),
+            attn_ws=torch.empty(tg_gated_attention_workspace_size(ck_h, self.hq, self.hkv, self.d),
+                                dtype=torch.uint8, device=dev),
             caches=[(torch.empty((K, self.hkv * self.d), **bf),
                      torch.empty((K, self.hkv * self.d), **bf)) for _ in self.layers],
         )
@@ -377,18 +415,26 @@ class GatedPrefill:
         ck, cv = P["caches"][i]
         nq, nk = self.hq * self.d, self.hkv * self.d
         qkv, o, x = P["qkv"], P["o"], P["x"]
-        tg_linear(x, L.Wqkv, qkv, rmsnorm=True, eps=self.norm_eps, status=self.status,
-                  stream=stream)
-        self._mark("qkv_proj")
-        tg_gather_rope(qkv, qkv, rope_pos=P["kept_pos"], rope_cols=(0, nq + nk),
-                       head_dim=self.d, cos_sin=self.cos_sin, status=self.status, stream=stream)
-        self._mark("rope")
-        tg_kv_compact(qkv[:, nq:nq + nk], qkv[:, nq + nk:], ck, cv, status=self.status,
+        if self.fused_qkv:
+            tg_qkv_rope_cache(x, L.Wqkv, P["kept_pos"], self.cos_sin, ck, cv, self.hq, self.hkv,
+                              q_out=qkv[:, :nq], head_dim=self.d, eps=self.norm_eps,
+                              status=self.status, stream=stream)
+            self._mark("qkv_rope_cache")
+        else:
+            tg_linear(x, L.Wqkv, qkv, rmsnorm=True, eps=self.norm_eps, status=self.status,
                       stream=stream)
-        self._mark("kv_compact")
+            self._mark("qkv_proj")
+            tg_gather_rope(qkv, qkv, rope_pos=P["kept_pos"], rope_cols=(0, nq + nk),
+                           head_dim=self.d, cos_sin=self.cos_sin, status=self.status,
+                           stream=stream)
+            self._mark("rope")
+            tg_kv_compact(qkv[:, nq:nq + nk], qkv[:, nq + nk:], ck, cv, status=self.status,
+                          stream=stream)
+            self._mark("kv_compact")
         tg_gated_attention(qkv[:, :nq], ck, cv, P["ck"], P["ck_h"], self.hq, self.hkv,
                            P["kept_pos"], P["kept_bias"], L.gamma, L.beta, o=o,
-                           head_dim=self.d, status=self.status, stream=stream)
+                           head_dim=self.d, workspace=P["attn_ws"], status=self.status,
+                           stream=stream)
         self._mark("attention")
         tg_linear(o, L.Wo, x, residual=x, status=self.status, stream=stream)
         self._mark("out_proj")

@@ -14,17 +14,25 @@
 // One CTA = one request, one tile of 128 query ranks, one kv head and the two q
 // heads (h0, h0 + 1) that read it.  Tensor memory (512 columns):
 //   S0/P0 [0,128)  S1/P1 [128,256)  O0 [256,384)  O1 [384,512)
-// Warps: 0 TMA producer (Q once, then K/V tiles + key bias through a 2-stage ring);
-// 1 MMA issuer (S = Q K^T from shared memory, O += P V with P read from TMEM);
-// 2-5 softmax of head h0, 6-9 softmax of head h1, one thread per query row (warp w
-// reads TMEM lane quarter w % 4, so each group of four covers all 128 rows).  The two
-// heads ping-pong: while one softmax runs, the tensor core works on the other head.
-// Softmax works in the log2 domain; the running max is only moved (and O rescaled in
-// TMEM) when it grows by more than 2^8, which keeps P within bf16 range.
+// Warpgroup 0 (warps 0-3, registers lowered to 120): warp 0 loads Q once and then K/V
+// tiles through a 2-stage TMA ring (a K stage is released as soon as both heads' S
+// MMAs have read it, a V stage after both PV MMAs), and with each V the tile's key bias
+// pre-scaled by gamma_h * log2(e) for each of the two heads; warp 1 issues S = Q K^T (both operands
+// in shared memory) and O += P V (P read from TMEM, V an MN-major shared operand).
+// Warpgroups 1 and 2 (registers raised to 192) are the softmax of head h0 and h0 + 1,
+// one thread per query row: the logits tau * s * log2(e) / sqrt(d) + bias come from
+// one packed fp32x2 FMA per pair, the row max from 3-input max, 2^(l - m) from the
+// MUFU unit, the row sum from packed adds, and P goes back to TMEM as bf16.  Masking
+// is only applied on the diagonal tile.  The running max moves (and O is rescaled in
+// TMEM) only when it grows by more than 2^8, which keeps P inside bf16 range.  The two
+// heads ping-pong on the tensor core: while one softmax runs the MMA works on the other.
 #include <cuda.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstdint>
+#include <functional>
+#include <vector>
 
 #include "tg_host.h"
 #include "tg_ptx.cuh"
@@ -36,7 +44,12 @@ constexpr int kD = 128;         // head_dim
 constexpr int kBM = 128;        // query rows per tile
 constexpr int kBN = 128;        // keys per KV tile
 constexpr int kStages = 2;      // K/V ring depth
-constexpr int kThreads = 320;   // 10 warps
+constexpr int kThreads = 384;   // 3 warpgroups
+constexpr int kLaunchRegs = 168;  // 65536 / 384, rounded down to a multiple of 8
+constexpr int kRegsLow = 120;     // warpgroup 0 after setmaxnreg.dec
+constexpr int kRegsHigh = 192;    // softmax warpgroups after setmaxnreg.inc
+static_assert(128 * kRegsLow + 256 * kRegsHigh <= kThreads * kLaunchRegs,
+              "register split exceeds the launch allocation");
 constexpr int kMaxBatch = 512;  // requests per call (tile table lives in the parameters)
 constexpr int kTileBytes = kBM * kD * 2;  // 32 KB: 128 rows x 128 bf16, two 64-column boxes
 constexpr float kLog2e = 1.4426950408889634f;
@@ -48,8 +61,8 @@ struct AttnSmem {
   static constexpr int Q1 = Q0 + kTileBytes;
   static constexpr int K = Q1 + kTileBytes;
   static constexpr int V = K + kStages * kTileBytes;
-  static constexpr int BIAS = V + kStages * kTileBytes;
-  static constexpr int BAR = BIAS + kStages * kBN * 4;
+  static constexpr int BIAS = V + kStages * kTileBytes;    // [stage][head][kBN] fp32
+  static constexpr int BAR = BIAS + kStages * 2 * kBN * 4;
   static constexpr int END = BAR + 256;
   static constexpr int BYTES = END + 1024;  // alignment slack
 };
@@ -70,13 +83,91 @@ struct AttnParams {
   int n_kv_heads;
   int batch;
   uint32_t* status;
-  int32_t tile_prefix[kMaxBatch + 1];  // q tiles before request b
+  int chunk;           // key tiles per work item (split-KV); >= every request's tile count = no split
+  float* part_ws;      // partial results of split query tiles (see kPartFloats), or null
+  int32_t item_prefix[kMaxBatch + 1];  // work items before request b
 };
 
-#ifndef TG_ATTN_MAXNREG
-#define TG_ATTN_MAXNREG 168  // 320 threads: the per-block limit is taken in 128-thread units
-#endif
-__global__ void __maxnreg__(TG_ATTN_MAXNREG)
+// Floats per (work item, q head) in the split-KV workspace: 128 rows x 128 unnormalised
+// O values, then 128 row maxima (log2 domain), then 128 row sums.  O is stored as 32
+// groups of 4 columns, each group row-contiguous (group f of row r at float4 index
+// f * 128 + r), so that one thread per row reads and writes coalesced.
+constexpr int kPartFloats = kBM * kD + 2 * kBM;
+
+__host__ __device__ __forceinline__ int ceil_div(int a, int b) { return (a + b - 1) / b; }
+
+// Work item t -> request b, query tile qt, part index and part count.  Within a request
+// items run over query tiles from the heaviest (last) to the lightest, the parts of a
+// tile consecutively; part i covers key tiles [i * chunk, min((i + 1) * chunk, qt + 1)).
+__device__ __forceinline__ void decode_item(const AttnParams& p, int t, int& b, int& qt,
+                                            int& part, int& nparts) {
+  int lo = 0, hi = p.batch;  // largest b with item_prefix[b] <= t
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (p.item_prefix[mid] <= t) lo = mid; else hi = mid;
+  }
+  b = lo;
+  int idx = t - p.item_prefix[b];
+  const int n_b = p.cu_kept[b + 1] - p.cu_kept[b];
+  const int ntiles = ceil_div(n_b, kBM);
+  qt = ntiles - 1;
+  if (p.chunk >= ntiles) {  // no split: one item per query tile
+    qt = ntiles - 1 - idx;
+    part = 0;
+    nparts = 1;
+    return;
+  }
+  while (true) {
+    const int np = ceil_div(qt + 1, p.chunk);
+    if (idx < np) {
+      part = idx;
+      nparts = np;
+      return;
+    }
+    idx -= np;
+    --qt;
+  }
+}
+
+// Logits of one row for one key tile: l = s * t2 + b (pairs), written back into sv.
+template <bool kDiag>
+__device__ __forceinline__ float logits_and_max(uint32_t (&sv)[kBN], const float* bsl,
+                                                float tau2, int rit) {
+  const uint64_t t2 = f2pack(tau2, tau2);
+  const float4* b4p = reinterpret_cast<const float4*>(bsl);
+  float m0 = -INFINITY, m1 = -INFINITY, m2 = -INFINITY, m3 = -INFINITY;
+#pragma unroll
+  for (int i = 0; i < kBN / 4; ++i) {
+    const float4 b4 = b4p[i];
+    const uint64_t l01 = fma2(f2pack(__uint_as_float(sv[4 * i]), __uint_as_float(sv[4 * i + 1])),
+                              t2, f2pack(b4.x, b4.y));
+    const uint64_t l23 = fma2(f2pack(__uint_as_float(sv[4 * i + 2]), __uint_as_float(sv[4 * i + 3])),
+                              t2, f2pack(b4.z, b4.w));
+    float a, b, c, d;
+    f2unpack(l01, a, b);
+    f2unpack(l23, c, d);
+    if (kDiag) {
+      if (4 * i + 0 > rit) a = -INFINITY;
+      if (4 * i + 1 > rit) b = -INFINITY;
+      if (4 * i + 2 > rit) c = -INFINITY;
+      if (4 * i + 3 > rit) d = -INFINITY;
+    }
+    sv[4 * i] = __float_as_uint(a);
+    sv[4 * i + 1] = __float_as_uint(b);
+    sv[4 * i + 2] = __float_as_uint(c);
+    sv[4 * i + 3] = __float_as_uint(d);
+    if (i & 1) {
+      m2 = max3(m2, a, b);
+      m3 = max3(m3, c, d);
+    } else {
+      m0 = max3(m0, a, b);
+      m1 = max3(m1, c, d);
+    }
+  }
+  return fmaxf(max3(m0, m1, m2), m3);
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
     gated_attention_kernel(const __grid_constant__ CUtensorMap tmQ,
                            const __grid_constant__ CUtensorMap tmK,
                            const __grid_constant__ CUtensorMap tmV,
@@ -89,8 +180,10 @@ __global__ void __maxnreg__(TG_ATTN_MAXNREG)
   uint64_t* q_full = bars + 0;
   uint64_t* k_full = bars + 1;             // [kStages]
   uint64_t* v_full = k_full + kStages;     // [kStages]
-  uint64_t* kv_empty = v_full + kStages;   // [kStages]
-  uint64_t* s_full = kv_empty + kStages;   // [2]
+  uint64_t* k_empty = v_full + kStages;    // [kStages]
+  uint64_t* v_empty = k_empty + kStages;   // [kStages]
+  uint64_t* b_full = v_empty + kStages;    // [kStages] key bias of the stage written
+  uint64_t* s_full = b_full + kStages;     // [2]
   uint64_t* p_full = s_full + 2;           // [2]
   uint64_t* pv_done = p_full + 2;          // [2]
   uint64_t* drain = pv_done + 2;
@@ -99,34 +192,29 @@ __global__ void __maxnreg__(TG_ATTN_MAXNREG)
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
-  // ---- which tile: heads vary fastest, then q tiles heaviest-first within a request
+  // ---- which work item: head groups vary fastest, then items heaviest first
   const int hg = p.n_kv_heads * p.head_pairs;
   const int head_grp = blockIdx.x % hg;
-  const int t = blockIdx.x / hg;
-  int b = 0;
-  {
-    int lo = 0, hi = p.batch;  // largest b with tile_prefix[b] <= t
-    while (hi - lo > 1) {
-      const int mid = (lo + hi) >> 1;
-      if (p.tile_prefix[mid] <= t) lo = mid; else hi = mid;
-    }
-    b = lo;
-  }
-  const int ntiles_b = p.tile_prefix[b + 1] - p.tile_prefix[b];
-  const int qt = ntiles_b - 1 - (t - p.tile_prefix[b]);
+  const int item = blockIdx.x / hg;
+  int b, qt, part, nparts;
+  decode_item(p, item, b, qt, part, nparts);
   const int g = head_grp / p.head_pairs;
   const int h0 = g * p.group + 2 * (head_grp % p.head_pairs);
   const int64_t row0 = p.cu_kept[b];
   const int n_b = p.cu_kept[b + 1] - p.cu_kept[b];
   const int q0 = qt * kBM;
-  const int nt = qt + 1;  // causal: key tiles 0..qt
+  // causal: key tiles 0..qt, this item's share [j0, j0 + nt)
+  const int j0 = part * p.chunk;
+  const int nt = min(qt + 1, j0 + p.chunk) - j0;
 
   if (tid == 0) {
     mbar_init(q_full, 1);
     for (int s = 0; s < kStages; ++s) {
-      mbar_init(&k_full[s], 2);  // TMA bytes + key-bias stores
+      mbar_init(&k_full[s], 1);
+      mbar_init(&b_full[s], 1);
       mbar_init(&v_full[s], 1);
-      mbar_init(&kv_empty[s], 1);
+      mbar_init(&k_empty[s], 1);
+      mbar_init(&v_empty[s], 1);
     }
     for (int h = 0; h < 2; ++h) {
       mbar_init(&s_full[h], 1);
@@ -151,119 +239,151 @@ __global__ void __maxnreg__(TG_ATTN_MAXNREG)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 0) {
-    // ------------------------------------------------------------ producer
-    int loaded = 0;
-    bool q_issued = false;
-    if (lane == 0) {
-      mbar_arrive_expect_tx(q_full, 2 * kTileBytes);
-      const int y = (int)(row0 + q0);
-      tma_load_2d(smem + AttnSmem::Q0, &tmQ, h0 * kD, y, q_full);
-      tma_load_2d(smem + AttnSmem::Q0 + kTileBytes / 2, &tmQ, h0 * kD + 64, y, q_full);
-      tma_load_2d(smem + AttnSmem::Q1, &tmQ, (h0 + 1) * kD, y, q_full);
-      tma_load_2d(smem + AttnSmem::Q1 + kTileBytes / 2, &tmQ, (h0 + 1) * kD + 64, y, q_full);
-      q_issued = true;
-    }
-    for (int j = 0; j < nt; ++j) {
-      const int s = j % kStages;
-      const uint32_t ph = (uint32_t)(j / kStages) & 1u;
-      if (!warp_all(mbar_wait(&kv_empty[s], ph ^ 1u, abort_flag, p.status))) break;
-      const int k0 = j * kBN;
-      const int y = (int)(row0 + k0);
-      unsigned char* kt = smem + AttnSmem::K + s * kTileBytes;
-      unsigned char* vt = smem + AttnSmem::V + s * kTileBytes;
+  if (warp < 4) {
+    regs_dec<kRegsLow>();
+    if (warp == 0) {
+      // ---------------------------------------------------------- producer
+      const float gb0 = p.gamma[h0] * kLog2e, gb1 = p.gamma[h0 + 1] * kLog2e;
+      int loaded = 0, loaded_v = 0;
+      bool q_issued = false;
       if (lane == 0) {
-        mbar_arrive_expect_tx(&k_full[s], kTileBytes);
-        tma_load_2d(kt, &tmK, g * kD, y, &k_full[s]);
-        tma_load_2d(kt + kTileBytes / 2, &tmK, g * kD + 64, y, &k_full[s]);
-        mbar_arrive_expect_tx(&v_full[s], kTileBytes);
-        tma_load_2d(vt, &tmV, g * kD, y, &v_full[s]);
-        tma_load_2d(vt + kTileBytes / 2, &tmV, g * kD + 64, y, &v_full[s]);
+        mbar_arrive_expect_tx(q_full, 2 * kTileBytes);
+        const int y = (int)(row0 + q0);
+        tma_load_2d(smem + AttnSmem::Q0, &tmQ, h0 * kD, y, q_full);
+        tma_load_2d(smem + AttnSmem::Q0 + kTileBytes / 2, &tmQ, h0 * kD + 64, y, q_full);
+        tma_load_2d(smem + AttnSmem::Q1, &tmQ, (h0 + 1) * kD, y, q_full);
+        tma_load_2d(smem + AttnSmem::Q1 + kTileBytes / 2, &tmQ, (h0 + 1) * kD + 64, y, q_full);
+        q_issued = true;
       }
-      float* bsl = bias_s + s * kBN;
+      // Key bias of tile j, loaded one tile ahead so its global latency overlaps the
+      // wait for a free stage.
+      auto load_bias = [&](int j, float (&bv)[4]) {
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int c = k0 + lane * 4 + e;
-        bsl[lane * 4 + e] = c < n_b ? p.kept_bias[row0 + c] : 0.0f;
-      }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&k_full[s]);
-      ++loaded;
-    }
-    if (lane == 0) {
-      // drain: no bulk copy may still be landing when the CTA exits
-      if (q_issued) mbar_wait(q_full, 0, nullptr, p.status);
-      for (int j = loaded - kStages < 0 ? 0 : loaded - kStages; j < loaded; ++j) {
+        for (int e = 0; e < 4; ++e) {
+          const int c = (j0 + j) * kBN + lane * 4 + e;
+          bv[e] = (j < nt && c < n_b) ? p.kept_bias[row0 + c] : 0.0f;
+        }
+      };
+      float bv[4];
+      load_bias(0, bv);
+      for (int j = 0; j < nt; ++j) {
+        const int s = j % kStages;
         const uint32_t ph = (uint32_t)(j / kStages) & 1u;
-        mbar_wait(&k_full[j % kStages], ph, nullptr, p.status);
-        mbar_wait(&v_full[j % kStages], ph, nullptr, p.status);
+        const int y = (int)(row0 + (j0 + j) * kBN);
+        // K of tile j once both heads' S MMAs of tile j - kStages are done
+        if (!warp_all(mbar_wait(&k_empty[s], ph ^ 1u, abort_flag, p.status))) break;
+        unsigned char* kt = smem + AttnSmem::K + s * kTileBytes;
+        if (lane == 0) {
+          mbar_arrive_expect_tx(&k_full[s], kTileBytes);
+          tma_load_2d(kt, &tmK, g * kD, y, &k_full[s]);
+          tma_load_2d(kt + kTileBytes / 2, &tmK, g * kD + 64, y, &k_full[s]);
+        }
+        // V and the key bias of tile j once both heads' PV MMAs of tile j - kStages are
+        // done (the PV MMAs follow both softmaxes of that tile, the bias's only readers)
+        if (!warp_all(mbar_wait(&v_empty[s], ph ^ 1u, abort_flag, p.status))) {
+          ++loaded;
+          break;
+        }
+        unsigned char* vt = smem + AttnSmem::V + s * kTileBytes;
+        if (lane == 0) {
+          mbar_arrive_expect_tx(&v_full[s], kTileBytes);
+          tma_load_2d(vt, &tmV, g * kD, y, &v_full[s]);
+          tma_load_2d(vt + kTileBytes / 2, &tmV, g * kD + 64, y, &v_full[s]);
+        }
+        float4* b0 = reinterpret_cast<float4*>(bias_s + (s * 2 + 0) * kBN) + lane;
+        float4* b1 = reinterpret_cast<float4*>(bias_s + (s * 2 + 1) * kBN) + lane;
+        *b0 = make_float4(bv[0] * gb0, bv[1] * gb0, bv[2] * gb0, bv[3] * gb0);
+        *b1 = make_float4(bv[0] * gb1, bv[1] * gb1, bv[2] * gb1, bv[3] * gb1);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&b_full[s]);
+        load_bias(j + 1, bv);
+        ++loaded;
+        ++loaded_v;
       }
-    }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t idesc_s = idesc_bf16_f32(128, kBN, false, false);
-      constexpr uint32_t idesc_o = idesc_bf16_f32(128, kD, false, true);
-      const uint32_t q_addr[2] = {smem_u32(smem + AttnSmem::Q0), smem_u32(smem + AttnSmem::Q1)};
-      const uint32_t s_col[2] = {0u, 128u};
-      const uint32_t o_col[2] = {256u, 384u};
-      auto issue_s = [&](int hh, int j) {
-        const uint32_t k_addr = smem_u32(smem + AttnSmem::K + (j % kStages) * kTileBytes);
-#pragma unroll
-        for (int kk = 0; kk < kD / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * (kTileBytes / 2) + (kk & 3) * 32;
-          mma_ss(tmem + s_col[hh], sw128_desc(q_addr[hh] + off, 16, 1024),
-                 sw128_desc(k_addr + off, 16, 1024), idesc_s, kk != 0);
-        }
-        mma_commit(&s_full[hh]);
-      };
-      auto issue_pv = [&](int hh, int j) {
-        const uint32_t v_addr = smem_u32(smem + AttnSmem::V + (j % kStages) * kTileBytes);
-#pragma unroll
-        for (int kk = 0; kk < kBN / 16; ++kk) {
-          // A = P (bf16 pairs in TMEM, 8 columns per 16 keys); B = V rows kk*16.. (MN-major)
-          mma_ts(tmem + o_col[hh], tmem + s_col[hh] + kk * 8,
-                 sw128_desc(v_addr + kk * 16 * 128, kTileBytes / 2, 1024), idesc_o,
-                 (j | kk) != 0);
-        }
-        mma_commit(&pv_done[hh]);
-      };
-      bool ok = mbar_wait(q_full, 0, abort_flag, p.status) &&
-                mbar_wait(&k_full[0], 0, abort_flag, p.status);
-      if (ok) {
-        tc_fence_after();
-        issue_s(0, 0);
-        issue_s(1, 0);
-        for (int j = 0; j < nt && ok; ++j) {
-          const int s = j % kStages;
+      if (lane == 0) {
+        // drain: no bulk copy may still be landing when the CTA exits
+        if (q_issued) mbar_wait(q_full, 0, nullptr, p.status);
+        for (int j = loaded - kStages < 0 ? 0 : loaded - kStages; j < loaded; ++j) {
           const uint32_t ph = (uint32_t)(j / kStages) & 1u;
-          const uint32_t pj = (uint32_t)j & 1u;
-          ok = mbar_wait(&v_full[s], ph, abort_flag, p.status) &&
-               mbar_wait(&p_full[0], pj, abort_flag, p.status);
-          if (!ok) break;
-          tc_fence_after();
-          issue_pv(0, j);
-          const bool more = j + 1 < nt;
-          if (more) {
-            const int s2 = (j + 1) % kStages;
-            const uint32_t ph2 = (uint32_t)((j + 1) / kStages) & 1u;
-            if (!(ok = mbar_wait(&k_full[s2], ph2, abort_flag, p.status))) break;
-            tc_fence_after();
-            issue_s(0, j + 1);
-          }
-          if (!(ok = mbar_wait(&p_full[1], pj, abort_flag, p.status))) break;
-          tc_fence_after();
-          issue_pv(1, j);
-          mma_commit(&kv_empty[s]);
-          if (more) issue_s(1, j + 1);
+          mbar_wait(&k_full[j % kStages], ph, nullptr, p.status);
+          if (j < loaded_v) mbar_wait(&v_full[j % kStages], ph, nullptr, p.status);
         }
       }
-      mma_commit(drain);
-      mbar_wait(drain, 0, nullptr, p.status);  // every MMA retired before TMEM is freed
+    } else if (warp == 1) {
+      // ---------------------------------------------------------- MMA issuer
+      if (lane == 0) {
+        constexpr uint32_t idesc_s = idesc_bf16_f32(128, kBN, false, false);
+        constexpr uint32_t idesc_o = idesc_bf16_f32(128, kD, false, true);
+        // Descriptors are built once; stepping along K only moves the start-address
+        // field (bits 0-13, address >> 4), which cannot carry for shared addresses
+        // below 256 KB.
+        const uint64_t q_desc[2] = {sw128_desc(smem_u32(smem + AttnSmem::Q0), 16, 1024),
+                                    sw128_desc(smem_u32(smem + AttnSmem::Q1), 16, 1024)};
+        const uint64_t k_desc0 = sw128_desc(smem_u32(smem + AttnSmem::K), 16, 1024);
+        const uint64_t v_desc0 = sw128_desc(smem_u32(smem + AttnSmem::V), kTileBytes / 2, 1024);
+        const uint32_t s_col[2] = {0u, 128u};
+        const uint32_t o_col[2] = {256u, 384u};
+        auto issue_s = [&](int hh, int j) {
+          const uint64_t kd = k_desc0 + (uint64_t)(((j % kStages) * kTileBytes) >> 4);
+#pragma unroll
+          for (int kk = 0; kk < kD / 16; ++kk) {
+            const uint64_t off = (uint64_t)(((kk >> 2) * (kTileBytes / 2) + (kk & 3) * 32) >> 4);
+            mma_ss(tmem + s_col[hh], q_desc[hh] + off, kd + off, idesc_s, kk != 0);
+          }
+          mma_commit(&s_full[hh]);
+        };
+        auto issue_pv = [&](int hh, int j) {
+          const uint64_t vd = v_desc0 + (uint64_t)(((j % kStages) * kTileBytes) >> 4);
+#pragma unroll
+          for (int kk = 0; kk < kBN / 16; ++kk) {
+            // A = P (bf16 pairs in TMEM, 8 columns per 16 keys); B = V rows kk*16.. (MN-major)
+            mma_ts(tmem + o_col[hh], tmem + s_col[hh] + kk * 8, vd + (uint64_t)((kk * 16 * 128) >> 4),
+                   idesc_o, (j | kk) != 0);
+          }
+          mma_commit(&pv_done[hh]);
+        };
+        bool ok = mbar_wait(q_full, 0, abort_flag, p.status) &&
+                  mbar_wait(&k_full[0], 0, abort_flag, p.status);
+        if (ok) {
+          tc_fence_after();
+          issue_s(0, 0);
+          issue_s(1, 0);
+          mma_commit(&k_empty[0]);
+          for (int j = 0; j < nt && ok; ++j) {
+            const int s = j % kStages;
+            const uint32_t ph = (uint32_t)(j / kStages) & 1u;
+            const uint32_t pj = (uint32_t)j & 1u;
+            ok = mbar_wait(&v_full[s], ph, abort_flag, p.status) &&
+                 mbar_wait(&p_full[0], pj, abort_flag, p.status);
+            if (!ok) break;
+            tc_fence_after();
+            issue_pv(0, j);
+            const bool more = j + 1 < nt;
+            if (more) {
+              const int s2 = (j + 1) % kStages;
+              const uint32_t ph2 = (uint32_t)((j + 1) / kStages) & 1u;
+              if (!(ok = mbar_wait(&k_full[s2], ph2, abort_flag, p.status))) break;
+              tc_fence_after();
+              issue_s(0, j + 1);
+            }
+            if (!(ok = mbar_wait(&p_full[1], pj, abort_flag, p.status))) break;
+            tc_fence_after();
+            issue_pv(1, j);
+            mma_commit(&v_empty[s]);
+            if (more) {
+              issue_s(1, j + 1);
+              mma_commit(&k_empty[(j + 1) % kStages]);
+            }
+          }
+        }
+        mma_commit(drain);
+        mbar_wait(drain, 0, nullptr, p.status);  // every MMA retired before TMEM is freed
+      }
     }
   } else {
+    regs_inc<kRegsHigh>();
     // ------------------------------------------------------------ softmax
-    const int wg = (warp - 2) >> 2;  // 0: head h0, 1: head h0 + 1
+    const int wg = (warp - 4) >> 2;  // 0: head h0, 1: head h0 + 1
     const int hh = h0 + wg;
     const int q = warp & 3;
     const int rit = q * 32 + lane;   // row in tile
@@ -279,7 +399,6 @@ __global__ void __maxnreg__(TG_ATTN_MAXNREG)
       if (pos > 0) tau = (double)p.beta * log((double)r + 1.0) / log((double)pos + 1.0);
     }
     const float tau2 = (float)(tau / sqrt((double)kD) * 1.4426950408889634);
-    const float gb = p.gamma[hh] * kLog2e;
 
     float m_run = -INFINITY, l_sum = 0.f;
     bool ok = true;
@@ -287,46 +406,49 @@ __global__ void __maxnreg__(TG_ATTN_MAXNREG)
       if (!(ok = warp_all(mbar_wait(&s_full[wg], (uint32_t)j & 1u, abort_flag, p.status)))) break;
       tc_fence_after();
       uint32_t sv[kBN];
-      const float* bsl = bias_s + (j % kStages) * kBN;
-      const bool diag = (j == qt);
-      float mx = -INFINITY;
-#pragma unroll
-      for (int c = 0; c < kBN / 32; ++c) {
-        // one 32-column chunk at a time keeps only 32 bias values in flight
-        tmem_ld32(s_t + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&sv[32 * c]));
-        tmem_wait_ld();
-#pragma unroll
-        for (int i = 32 * c; i < 32 * c + 32; ++i) {
-          float v = fmaf(__uint_as_float(sv[i]), tau2, gb * bsl[i]);
-          if (diag && i > rit) v = -INFINITY;
-          sv[i] = __float_as_uint(v);
-          mx = fmaxf(mx, v);
-        }
-      }
+      tmem_ld32(s_t + 0, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
+      tmem_ld32(s_t + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
+      tmem_ld32(s_t + 64, *reinterpret_cast<uint32_t(*)[32]>(&sv[64]));
+      tmem_ld32(s_t + 96, *reinterpret_cast<uint32_t(*)[32]>(&sv[96]));
+      tmem_wait_ld();
+      if (!(ok = warp_all(mbar_wait(&b_full[j % kStages], (uint32_t)(j / kStages) & 1u, abort_flag,
+                                    p.status))))
+        break;
+      const float* bsl = bias_s + ((j % kStages) * 2 + wg) * kBN;
+      const float mx = (j0 + j == qt) ? logits_and_max<true>(sv, bsl, tau2, rit)
+                                 : logits_and_max<false>(sv, bsl, tau2, rit);
       // Lazy rescale: move the running max only when it grows by more than 2^8.
       float alpha = 1.0f;
       bool rescale = false;
       if (j == 0) {
         m_run = mx;
       } else if (mx > m_run + kRescaleThreshold) {
-        alpha = exp2f(m_run - mx);
+        alpha = ex2_approx(m_run - mx);
         m_run = mx;
         rescale = true;
       }
-      float rs = 0.f;
+      const uint64_t negm = f2pack(-m_run, -m_run);
+      uint64_t acc0 = f2pack(0.f, 0.f), acc1 = acc0;
 #pragma unroll
       for (int hf = 0; hf < 2; ++hf) {
         uint32_t pk[32];
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
-          const float p0 = exp2f(__uint_as_float(sv[64 * hf + 2 * i]) - m_run);
-          const float p1 = exp2f(__uint_as_float(sv[64 * hf + 2 * i + 1]) - m_run);
-          rs += p0 + p1;
+          const int e = 64 * hf + 2 * i;
+          const uint64_t d = add2(f2pack(__uint_as_float(sv[e]), __uint_as_float(sv[e + 1])), negm);
+          float x0, x1;
+          f2unpack(d, x0, x1);
+          const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
+          if (i & 1) acc1 = add2(acc1, f2pack(p0, p1));
+          else acc0 = add2(acc0, f2pack(p0, p1));
           pk[i] = pack_bf16x2(p0, p1);
         }
         tmem_st32(s_t + 32 * hf, pk);
       }
-      l_sum = l_sum * alpha + rs;
+      float a0, a1, a2, a3;
+      f2unpack(acc0, a0, a1);
+      f2unpack(acc1, a2, a3);
+      l_sum = l_sum * alpha + ((a0 + a1) + (a2 + a3));
       // O rescale, warp-uniform (tcgen05.ld/st are warp-collective; alpha = 1 on rows
       // that keep their max).  PV(j-1) has retired: S(j) was committed after it.
       if (__any_sync(0xFFFFFFFFu, rescale)) {
@@ -350,28 +472,46 @@ __global__ void __maxnreg__(TG_ATTN_MAXNREG)
     }
     if (ok && warp_all(mbar_wait(&pv_done[wg], (uint32_t)(nt - 1) & 1u, abort_flag, p.status))) {
       tc_fence_after();
-      const float inv = 1.0f / l_sum;
-      uint16_t* orow = p.o + (row0 + r) * p.ld_o + (int64_t)hh * kD;
+      if (nparts == 1) {
+        const float inv = 1.0f / l_sum;
+        uint16_t* orow = p.o + (row0 + r) * p.ld_o + (int64_t)hh * kD;
 #pragma unroll 1
-      for (int c = 0; c < kD / 32; ++c) {
-        uint32_t ro[32];
-        tmem_ld32(o_t + c * 32, ro);
-        tmem_wait_ld();
-        if (row_valid) {
-          uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+        for (int c = 0; c < kD / 32; ++c) {
+          uint32_t ro[32];
+          tmem_ld32(o_t + c * 32, ro);
+          tmem_wait_ld();
+          if (row_valid) {
+            uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
 #pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            uint4 w;
-            w.x = pack_bf16x2(__uint_as_float(ro[u * 8 + 0]) * inv, __uint_as_float(ro[u * 8 + 1]) * inv);
-            w.y = pack_bf16x2(__uint_as_float(ro[u * 8 + 2]) * inv, __uint_as_float(ro[u * 8 + 3]) * inv);
-            w.z = pack_bf16x2(__uint_as_float(ro[u * 8 + 4]) * inv, __uint_as_float(ro[u * 8 + 5]) * inv);
-            w.w = pack_bf16x2(__uint_as_float(ro[u * 8 + 6]) * inv, __uint_as_float(ro[u * 8 + 7]) * inv);
-            dst[u] = w;
+            for (int u = 0; u < 4; ++u) {
+              uint4 w;
+              w.x = pack_bf16x2(__uint_as_float(ro[u * 8 + 0]) * inv, __uint_as_float(ro[u * 8 + 1]) * inv);
+              w.y = pack_bf16x2(__uint_as_float(ro[u * 8 + 2]) * inv, __uint_as_float(ro[u * 8 + 3]) * inv);
+              w.z = pack_bf16x2(__uint_as_float(ro[u * 8 + 4]) * inv, __uint_as_float(ro[u * 8 + 5]) * inv);
+              w.w = pack_bf16x2(__uint_as_float(ro[u * 8 + 6]) * inv, __uint_as_float(ro[u * 8 + 7]) * inv);
+              dst[u] = w;
+            }
           }
         }
+        if (row_valid && p.lse)
+          p.lse[(int64_t)hh * p.k_total + row0 + r] = (m_run + log2f(l_sum)) * 0.69314718055994531f;
+      } else {
+        // split query tile: unnormalised O, row max and row sum for the combine kernel
+        float* part_base = p.part_ws + ((int64_t)item * p.n_q_heads + hh) * kPartFloats;
+        float4* ocol = reinterpret_cast<float4*>(part_base) + rit;
+#pragma unroll 1
+        for (int c = 0; c < kD / 32; ++c) {
+          uint32_t ro[32];
+          tmem_ld32(o_t + c * 32, ro);
+          tmem_wait_ld();
+#pragma unroll
+          for (int u = 0; u < 8; ++u)
+            ocol[(c * 8 + u) * kBM] = make_float4(__uint_as_float(ro[4 * u]), __uint_as_float(ro[4 * u + 1]),
+                                                  __uint_as_float(ro[4 * u + 2]), __uint_as_float(ro[4 * u + 3]));
+        }
+        part_base[kBM * kD + rit] = m_run;
+        part_base[kBM * kD + kBM + rit] = l_sum;
       }
-      if (row_valid && p.lse)
-        p.lse[(int64_t)hh * p.k_total + row0 + r] = (m_run + log2f(l_sum)) * 0.69314718055994531f;
     }
     tc_fence_before();
   }
@@ -382,34 +522,193 @@ __global__ void __maxnreg__(TG_ATTN_MAXNREG)
   }
 }
 
+// Merge the parts of split query tiles: per row, m = max_i m_i, L = sum_i 2^(m_i - m) l_i,
+// o = sum_i 2^(m_i - m) O_i / L.  One CTA per (work item, q head) and 128 threads, one
+// per row (only the first part's CTA of a split tile works); with the column-group
+// layout above every load and store of a warp is contiguous.
+constexpr int kMaxParts = 64;
+__global__ void __launch_bounds__(128) combine_parts_kernel(const __grid_constant__ AttnParams p) {
+  const int item = blockIdx.x, hh = blockIdx.y;
+  int b, qt, part, nparts;
+  decode_item(p, item, b, qt, part, nparts);
+  if (nparts == 1 || part != 0) return;
+  const int64_t row0 = p.cu_kept[b];
+  const int n_b = p.cu_kept[b + 1] - p.cu_kept[b];
+  const int rit = threadIdx.x;
+  const int r = qt * kBM + rit;
+  if (r >= n_b) return;
+  const int np = nparts < kMaxParts ? nparts : kMaxParts;
+  const int64_t stride = (int64_t)p.n_q_heads * kPartFloats;  // floats between parts
+  const float* base0 = p.part_ws + ((int64_t)item * p.n_q_heads + hh) * kPartFloats;
+  float m = -INFINITY;
+  for (int i = 0; i < np; ++i) m = fmaxf(m, base0[i * stride + kBM * kD + rit]);
+  float L = 0.f;
+  float w[kMaxParts];
+  for (int i = 0; i < np; ++i) {
+    w[i] = exp2f(base0[i * stride + kBM * kD + rit] - m);
+    L += w[i] * base0[i * stride + kBM * kD + kBM + rit];
+  }
+  const float inv = 1.0f / L;
+  uint4* orow = reinterpret_cast<uint4*>(p.o + (row0 + r) * p.ld_o + (int64_t)hh * kD);
+#pragma unroll 1
+  for (int f = 0; f < kD / 4; f += 2) {
+    float4 a = make_float4(0.f, 0.f, 0.f, 0.f), c = a;
+    for (int i = 0; i < np; ++i) {
+      const float4* g = reinterpret_cast<const float4*>(base0 + i * stride) + rit;
+      const float4 x = g[f * kBM], y = g[(f + 1) * kBM];
+      a.x += w[i] * x.x; a.y += w[i] * x.y; a.z += w[i] * x.z; a.w += w[i] * x.w;
+      c.x += w[i] * y.x; c.y += w[i] * y.y; c.z += w[i] * y.z; c.w += w[i] * y.w;
+    }
+    uint4 out;
+    out.x = pack_bf16x2(a.x * inv, a.y * inv);
+    out.y = pack_bf16x2(a.z * inv, a.w * inv);
+    out.z = pack_bf16x2(c.x * inv, c.y * inv);
+    out.w = pack_bf16x2(c.z * inv, c.w * inv);
+    orow[f / 2] = out;
+  }
+  if (p.lse) p.lse[(int64_t)hh * p.k_total + row0 + r] = (m + log2f(L)) * 0.69314718055994531f;
+}
+
+// Work plan: the key-tile chunk per item and the item count per request, chosen to
+// minimise the estimated makespan over the SMs (one CTA per SM at a time).
+struct AttnPlan {
+  int chunk;
+  int n_items;
+  bool split;
+};
+
+// Makespan (in key-tile units) of launching the items of `chunk` in launch order on
+// `sms` SMs, one CTA per SM at a time: the block scheduler hands each CTA to the first
+// SM that frees up, which is list scheduling in launch order (heaviest first within a
+// request).  Each CTA also pays a fixed prologue/epilogue cost of kCtaOverhead tiles.
+constexpr double kCtaOverhead = 1.5;
+double simulate_makespan(const int32_t* cu_kept_host, int batch, int head_groups, int sms,
+                         int chunk) {
+  std::vector<double> busy((size_t)sms, 0.0);  // min-heap of SM finish times
+  std::make_heap(busy.begin(), busy.end(), std::greater<double>());
+  double makespan = 0.0;
+  for (int b = 0; b < batch; ++b) {
+    const int nt = ceil_div(cu_kept_host[b + 1] - cu_kept_host[b], kBM);
+    for (int qt = nt - 1; qt >= 0; --qt) {
+      const int np = ceil_div(qt + 1, chunk);
+      for (int part = 0; part < np; ++part) {
+        const int units = std::min(qt + 1, (part + 1) * chunk) - part * chunk;
+        for (int h = 0; h < head_groups; ++h) {
+          std::pop_heap(busy.begin(), busy.end(), std::greater<double>());
+          busy.back() += units + kCtaOverhead;
+          makespan = std::max(makespan, busy.back());
+          std::push_heap(busy.begin(), busy.end(), std::greater<double>());
+        }
+      }
+    }
+  }
+  return makespan;
+}
+
+int make_plan(const int32_t* cu_kept_host, int batch, int head_groups, int sms, AttnPlan& plan,
+              int32_t* item_prefix) {
+  int max_tiles = 0;
+  int64_t units = 0;
+  for (int b = 0; b < batch; ++b) {
+    const int64_t n = (int64_t)cu_kept_host[b + 1] - cu_kept_host[b];
+    if (n < 0) return TG_ERR_INVALID_ARGUMENT;
+    const int nt = ceil_div((int)n, kBM);
+    max_tiles = std::max(max_tiles, nt);
+    units += (int64_t)nt * (nt + 1) / 2;
+  }
+  // Plans are cached per layout: the gated layers of a step share one.
+  static thread_local std::vector<int32_t> cached_layout;
+  static thread_local AttnPlan cached_plan;
+  static thread_local int cached_hg = -1, cached_sms = -1;
+  std::vector<int32_t> layout(cu_kept_host, cu_kept_host + batch + 1);
+  if (layout == cached_layout && cached_hg == head_groups && cached_sms == sms) {
+    plan = cached_plan;
+  } else {
+    // Candidates: no split, and chunks near the balanced share of one SM.
+    const double share = (double)units * head_groups / sms;
+    int best = std::max(max_tiles, 1);
+    double best_cost = simulate_makespan(cu_kept_host, batch, head_groups, sms, best);
+    for (double f : {0.5, 0.75, 1.0, 1.25, 1.5, 2.0, 3.0}) {
+      const int c = (int)std::ceil(share * f);
+      if (c < 2 || c >= max_tiles) continue;
+      const double cost = simulate_makespan(cu_kept_host, batch, head_groups, sms, c) + 1.0;
+      if (cost < best_cost) {
+        best_cost = cost;
+        best = c;
+      }
+    }
+    plan.split = best < max_tiles;
+    plan.chunk = best;
+    cached_layout = layout;
+    cached_plan = plan;
+    cached_hg = head_groups;
+    cached_sms = sms;
+  }
+  int64_t items = 0;
+  item_prefix[0] = 0;
+  for (int b = 0; b < batch; ++b) {
+    const int nt = ceil_div(cu_kept_host[b + 1] - cu_kept_host[b], kBM);
+    for (int qt = 0; qt < nt; ++qt) items += ceil_div(qt + 1, plan.chunk);
+    if (items > 0x3FFFFFFF) return TG_ERR_UNSUPPORTED_SHAPE;
+    item_prefix[b + 1] = (int32_t)items;
+  }
+  plan.n_items = (int)items;
+  return TG_OK;
+}
+
+// The register split above assumes the kernel is launched with kLaunchRegs registers
+// per thread; a smaller launch allocation would leave setmaxnreg.inc waiting forever.
+int check_register_budget() {
+  static int checked_dev = -1;
+  int dev = 0;
+  TG_CUDA_TRY(cudaGetDevice(&dev));
+  if (checked_dev == dev) return TG_OK;
+  cudaFuncAttributes fa;
+  TG_CUDA_TRY(cudaFuncGetAttributes(&fa, gated_attention_kernel));
+  if (fa.numRegs * kThreads < 128 * kRegsLow + 256 * kRegsHigh ||
+      fa.maxThreadsPerBlock < kThreads)
+    return TG_ERR_UNSUPPORTED_SHAPE;
+  TG_CUDA_TRY(cudaFuncSetAttribute(gated_attention_kernel,
+                                   cudaFuncAttributeMaxDynamicSharedMemorySize, AttnSmem::BYTES));
+  checked_dev = dev;
+  return TG_OK;
+}
+
 }  // namespace
 }  // namespace tg
 
 using namespace tg;
+
+extern "C" size_t tg_gated_attention_workspace_size(const int32_t* cu_kept_host, int batch,
+                                                    int n_q_heads, int n_kv_heads, int head_dim) {
+  if (head_dim != kD || batch <= 0 || batch > kMaxBatch || !cu_kept_host || n_kv_heads <= 0 ||
+      n_q_heads <= 0 || n_q_heads % n_kv_heads || (n_q_heads / n_kv_heads) % 2)
+    return 0;
+  AttnPlan plan;
+  static thread_local int32_t prefix[kMaxBatch + 1];
+  if (make_plan(cu_kept_host, batch, n_q_heads / 2, sm_count(), plan, prefix) != TG_OK ||
+      !plan.split)
+    return 0;
+  return (size_t)plan.n_items * n_q_heads * kPartFloats * sizeof(float);
+}
 
 extern "C" int tg_gated_attention(const tg_bf16* q, int64_t ld_q, const tg_bf16* k, int64_t ld_k,
                                   const tg_bf16* v, int64_t ld_v, const int32_t* cu_kept,
                                   const int32_t* cu_kept_host, int batch, int n_q_heads,
                                   int n_kv_heads, int head_dim, const int32_t* kept_pos,
                                   const float* kept_bias, const float* gamma, float beta,
-                                  tg_bf16* o, int64_t ld_o, float* lse, uint32_t* status,
-                                  tg_stream_t stream) {
+                                  tg_bf16* o, int64_t ld_o, float* lse, void* workspace,
+                                  size_t workspace_bytes, uint32_t* status, tg_stream_t stream) {
   if (head_dim != kD) return TG_ERR_UNSUPPORTED_SHAPE;
   if (n_q_heads <= 0 || n_kv_heads <= 0 || n_q_heads % n_kv_heads) return TG_ERR_INVALID_ARGUMENT;
   const int group = n_q_heads / n_kv_heads;
   if (group % 2) return TG_ERR_UNSUPPORTED_SHAPE;
-  if (batch < 0 || batch > kMaxBatch || !cu_kept_host) return batch > kMaxBatch ? TG_ERR_UNSUPPORTED_SHAPE : TG_ERR_INVALID_ARGUMENT;
+  if (batch > kMaxBatch) return TG_ERR_UNSUPPORTED_SHAPE;
+  if (batch < 0 || !cu_kept_host) return TG_ERR_INVALID_ARGUMENT;
   if (batch == 0) return TG_OK;
   if (cu_kept_host[0] != 0) return TG_ERR_INVALID_ARGUMENT;
-  AttnParams prm{};
-  int tiles = 0;
-  prm.tile_prefix[0] = 0;
-  for (int b = 0; b < batch; ++b) {
-    const int64_t n = (int64_t)cu_kept_host[b + 1] - cu_kept_host[b];
-    if (n < 0) return TG_ERR_INVALID_ARGUMENT;
-    tiles += (int)((n + kBM - 1) / kBM);
-    prm.tile_prefix[b + 1] = tiles;
-  }
+  for (int b = 0; b < batch; ++b)
+    if (cu_kept_host[b + 1] < cu_kept_host[b]) return TG_ERR_INVALID_ARGUMENT;
   const int64_t k_total = cu_kept_host[batch];
   if (k_total == 0) return TG_OK;
   if (!q || !k || !v || !o || !cu_kept || !kept_pos || !kept_bias || !gamma)
@@ -420,8 +719,30 @@ extern "C" int tg_gated_attention(const tg_bf16* q, int64_t ld_q, const tg_bf16*
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !stride_ok(ld_q, 2) ||
       !stride_ok(ld_k, 2) || !stride_ok(ld_v, 2) || !stride_ok(ld_o, 2))
     return TG_ERR_MISALIGNED;
+  if (workspace && !aligned16(workspace)) return TG_ERR_MISALIGNED;
   if (!std::isfinite(beta)) return TG_ERR_INVALID_ARGUMENT;
   TG_TRY(check_device());
+  TG_TRY(check_register_budget());
+
+  AttnParams prm{};
+  const int head_groups = n_kv_heads * (group / 2);
+  AttnPlan plan;
+  TG_TRY(make_plan(cu_kept_host, batch, head_groups, sm_count(), plan, prm.item_prefix));
+  const size_t need = (size_t)plan.n_items * n_q_heads * kPartFloats * sizeof(float);
+  if (plan.split && (!workspace || workspace_bytes < need)) {
+    // no room for partial results: one item per query tile
+    int max_tiles = 1;
+    for (int b = 0; b < batch; ++b)
+      max_tiles = std::max(max_tiles, ceil_div(cu_kept_host[b + 1] - cu_kept_host[b], kBM));
+    plan.split = false;
+    plan.chunk = max_tiles;
+    int items = 0;
+    for (int b = 0; b < batch; ++b) {
+      items += ceil_div(cu_kept_host[b + 1] - cu_kept_host[b], kBM);
+      prm.item_prefix[b + 1] = items;
+    }
+    plan.n_items = items;
+  }
 
   CUtensorMap tq, tk, tv;
   TG_TRY(make_tmap_bf16_2d(&tq, q, (uint64_t)k_total, (uint64_t)n_q_heads * kD, (uint64_t)ld_q, 64, kBM));
@@ -442,19 +763,18 @@ extern "C" int tg_gated_attention(const tg_bf16* q, int64_t ld_q, const tg_bf16*
   prm.n_kv_heads = n_kv_heads;
   prm.batch = batch;
   prm.status = status;
+  prm.chunk = plan.chunk;
+  prm.part_ws = plan.split ? static_cast<float*>(workspace) : nullptr;
 
-  static int attr_dev = -1;
-  int dev = 0;
-  TG_CUDA_TRY(cudaGetDevice(&dev));
-  if (attr_dev != dev) {
-    TG_CUDA_TRY(cudaFuncSetAttribute(gated_attention_kernel,
-                                     cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     AttnSmem::BYTES));
-    attr_dev = dev;
-  }
-  const int64_t grid = (int64_t)tiles * n_kv_heads * (group / 2);
+  const int64_t grid = (int64_t)plan.n_items * head_groups;
   if (grid > 0x7FFFFFFF) return TG_ERR_UNSUPPORTED_SHAPE;
   gated_attention_kernel<<<(unsigned)grid, kThreads, AttnSmem::BYTES, (cudaStream_t)stream>>>(
       tq, tk, tv, prm);
-  return check_launch();
+  TG_TRY(check_launch());
+  if (plan.split) {
+    combine_parts_kernel<<<dim3((unsigned)plan.n_items, (unsigned)n_q_heads), 128, 0,
+                           (cudaStream_t)stream>>>(prm);
+    TG_TRY(check_launch());
+  }
+  return TG_OK;
 }

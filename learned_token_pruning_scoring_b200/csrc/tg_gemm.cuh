@@ -10,7 +10,10 @@
 //              no extra HBM pass: RMSNorm(a) W^T = r * (a W^T), r = 1/sqrt(mean a^2 + eps).
 // Epilogues: EpiStore writes bf16 rows (optionally + residual); EpiScore reduces each
 // row to one scalar s = sum_f w2[f] SiLU(r * acc[f]) and writes per-32-row partial
-// sums of s^2 for the sequence normalisation.
+// sums of s^2 for the sequence normalisation; EpiQKV applies rotate-half RoPE at the
+// row's position to the Q and K heads (pairs of columns 64 apart, from the TMEM chunks
+// c and c + 2) and writes Q, K and V tiles to three destinations (Q rows, and the K
+// and V rows of a compacted cache).
 #pragma once
 #include <cuda.h>
 
@@ -20,7 +23,7 @@
 
 namespace tg {
 
-enum { EpiStore = 0, EpiScore = 1 };
+enum { EpiStore = 0, EpiScore = 1, EpiQKV = 2 };
 
 struct GemmParams {
   int64_t M;
@@ -36,6 +39,14 @@ struct GemmParams {
   const float* w2;
   float* s_out;
   float* partial;  // [ceil(M / 32)]
+  // EpiQKV
+  const int32_t* pos;     // [M] rotary position of each row
+  const float* cos_sin;   // [max_pos, head_dim / 2, 2]
+  int max_pos;
+  int q_cols, k_cols;     // Q heads in [0, q_cols), K heads in [q_cols, q_cols + k_cols)
+  uint16_t* k_out;        // K rows: k_out + row * ld_kv (columns relative to q_cols)
+  uint16_t* v_out;        // V rows: v_out + row * ld_kv (columns relative to q_cols + k_cols)
+  int64_t ld_kv;
   uint32_t* status;
 };
 
@@ -173,6 +184,62 @@ __global__ void __launch_bounds__(192, 1)
     if (ok) {
       const uint32_t tbase = tmem + ((uint32_t)(q * 32) << 16);
       float score = 0.f;
+      if (EPI == EpiQKV) {
+        // destination of this tile: Q, K or V (tiles never straddle the boundaries)
+        uint16_t* dst;
+        int dcol;
+        if (n0 < p.q_cols) {
+          dst = p.c + grow * p.ldc;
+          dcol = n0;
+        } else if (n0 < p.q_cols + p.k_cols) {
+          dst = p.k_out + grow * p.ld_kv;
+          dcol = n0 - p.q_cols;
+        } else {
+          dst = p.v_out + grow * p.ld_kv;
+          dcol = n0 - p.q_cols - p.k_cols;
+        }
+        const bool rope = n0 < p.q_cols + p.k_cols;
+        int pos = (rope && grow < p.M) ? p.pos[grow] : 0;
+        if (pos < 0 || pos >= p.max_pos) {
+          if (grow < p.M && p.status) atomicOr(p.status, TG_STATUS_BOUNDS);
+          pos = 0;
+        }
+        const float4* cs_row = reinterpret_cast<const float4*>(p.cos_sin + (int64_t)pos * 128);
+#pragma unroll 1
+        for (int pr = 0; pr < BN / 64; ++pr) {
+          // chunk pairs (0,2), (1,3), (4,6), (5,7): columns i and i + 64 of one head
+          const int ca = (pr & 1) + 4 * (pr >> 1), cb = ca + 2;
+          uint32_t ra[32], rb[32];
+          tmem_ld32(tbase + ca * 32, ra);
+          tmem_ld32(tbase + cb * 32, rb);
+          tmem_wait_ld();
+          if (grow < p.M) {
+            uint4* da = reinterpret_cast<uint4*>(dst + dcol + ca * 32);
+            uint4* db = reinterpret_cast<uint4*>(dst + dcol + cb * 32);
+            const float4* cs = cs_row + (ca & 3) * 16;  // (cos, sin) pairs of i = (ca&3)*32 ..
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              uint32_t wa[4], wb[4];
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const int i = u * 8 + 2 * e;
+                float x1a = __uint_as_float(ra[i]) * rscale, x1b = __uint_as_float(ra[i + 1]) * rscale;
+                float x2a = __uint_as_float(rb[i]) * rscale, x2b = __uint_as_float(rb[i + 1]) * rscale;
+                if (rope) {
+                  const float4 t = cs[i >> 1];  // (cos_i, sin_i, cos_i+1, sin_i+1)
+                  const float y1a = x1a * t.x - x2a * t.y, y2a = x2a * t.x + x1a * t.y;
+                  const float y1b = x1b * t.z - x2b * t.w, y2b = x2b * t.z + x1b * t.w;
+                  x1a = y1a; x2a = y2a; x1b = y1b; x2b = y2b;
+                }
+                wa[e] = pack_bf16x2(x1a, x1b);
+                wb[e] = pack_bf16x2(x2a, x2b);
+              }
+              da[u] = make_uint4(wa[0], wa[1], wa[2], wa[3]);
+              db[u] = make_uint4(wb[0], wb[1], wb[2], wb[3]);
+            }
+          }
+        }
+      } else {
 #pragma unroll 1
       for (int c = 0; c < BN / 32; ++c) {
         uint32_t r[32];
@@ -216,6 +283,7 @@ __global__ void __launch_bounds__(192, 1)
             score = fmaf(w2s[c * 32 + i], u / (1.0f + __expf(-u)), score);
           }
         }
+      }
       }
       if (EPI == EpiScore) {
         if (grow < p.M) p.s_out[grow] = score;

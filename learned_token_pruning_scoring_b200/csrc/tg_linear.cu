@@ -29,6 +29,25 @@ template int launch_gemm<128, 3, EpiStore>(const CUtensorMap&, const CUtensorMap
                                            const GemmParams&, cudaStream_t);
 template int launch_gemm<256, 4, EpiScore>(const CUtensorMap&, const CUtensorMap&,
                                            const GemmParams&, cudaStream_t);
+template int launch_gemm<256, 4, EpiQKV>(const CUtensorMap&, const CUtensorMap&,
+                                         const GemmParams&, cudaStream_t);
+template int launch_gemm<128, 3, EpiQKV>(const CUtensorMap&, const CUtensorMap&,
+                                         const GemmParams&, cudaStream_t);
+
+// Tile width that wastes the fewest SM slots in the last wave: BN=256 runs one CTA
+// per SM, BN=128 two (smaller ring), so both fill all SMs per wave.
+int pick_bn(int64_t M, int N) {
+  const int64_t mt = (M + 127) / 128;
+  const int sms = sm_count();
+  auto eff = [&](int64_t tiles, int64_t slots) {
+    const int64_t waves = (tiles + slots - 1) / slots;
+    return (double)tiles / (double)(waves * slots);
+  };
+  const bool can256 = (N % 256) == 0;
+  const double e256 = can256 ? eff(mt * (N / 256), sms) : -1.0;
+  const double e128 = eff(mt * (N / 128), 2 * (int64_t)sms);
+  return (can256 && e256 >= e128) ? 256 : 128;
+}
 
 }  // namespace tg
 
@@ -49,18 +68,7 @@ extern "C" int tg_linear(const tg_bf16* a, int64_t lda, const tg_bf16* w, int64_
   if (rmsnorm_a && !(eps >= 0.f)) return TG_ERR_INVALID_ARGUMENT;
   TG_TRY(check_device());
 
-  // Tile width: the choice that wastes the fewest SM slots in the last wave.  BN=256
-  // runs one CTA per SM, BN=128 two (smaller ring), so both fill 148 SMs per wave.
-  const int64_t mt = (M + 127) / 128;
-  const int sms = sm_count();
-  auto eff = [&](int64_t tiles, int64_t slots) {
-    const int64_t waves = (tiles + slots - 1) / slots;
-    return (double)tiles / (double)(waves * slots);
-  };
-  const bool can256 = (N % 256) == 0;
-  const double e256 = can256 ? eff(mt * (N / 256), sms) : -1.0;
-  const double e128 = eff(mt * (N / 128), 2 * (int64_t)sms);
-  const int bn = (can256 && e256 >= e128) ? 256 : 128;
+  const int bn = pick_bn(M, N);
 
   CUtensorMap ta, tb;
   TG_TRY(make_tmap_bf16_2d(&ta, a, (uint64_t)M, (uint64_t)K, (uint64_t)lda, 64, 128));
@@ -78,4 +86,53 @@ extern "C" int tg_linear(const tg_bf16* a, int64_t lda, const tg_bf16* w, int64_
   p.status = status;
   if (bn == 256) return launch_gemm<256, 4, EpiStore>(ta, tb, p, (cudaStream_t)stream);
   return launch_gemm<128, 3, EpiStore>(ta, tb, p, (cudaStream_t)stream);
+}
+
+extern "C" int tg_qkv_rope_cache(const tg_bf16* x, int64_t ld_x, const tg_bf16* w_qkv, int64_t ld_w,
+                                 int64_t M, int hidden, int n_q_heads, int n_kv_heads,
+                                 int head_dim, float eps, const int32_t* pos,
+                                 const float* cos_sin, int max_pos, tg_bf16* q_out, int64_t ld_q,
+                                 tg_bf16* cache_k, tg_bf16* cache_v, int64_t ld_cache,
+                                 int64_t slot_offset, uint32_t* status, tg_stream_t stream) {
+  if (head_dim != 128 || n_q_heads <= 0 || n_kv_heads <= 0 || hidden <= 0 || (hidden % 64))
+    return TG_ERR_UNSUPPORTED_SHAPE;
+  if (M < 0 || slot_offset < 0 || max_pos <= 0) return TG_ERR_INVALID_ARGUMENT;
+  if (M == 0) return TG_OK;
+  const int q_cols = n_q_heads * head_dim, kv_cols = n_kv_heads * head_dim;
+  const int N = q_cols + 2 * kv_cols;
+  if (!x || !w_qkv || !pos || !cos_sin || !q_out || !cache_k || !cache_v)
+    return TG_ERR_INVALID_ARGUMENT;
+  if (ld_x < hidden || ld_w < hidden || ld_q < q_cols || ld_cache < kv_cols)
+    return TG_ERR_INVALID_ARGUMENT;
+  if (!aligned16(x) || !aligned16(w_qkv) || !aligned16(q_out) || !aligned16(cache_k) ||
+      !aligned16(cache_v) || !aligned16(cos_sin) || !stride_ok(ld_x, 2) || !stride_ok(ld_w, 2) ||
+      !stride_ok(ld_q, 2) || !stride_ok(ld_cache, 2))
+    return TG_ERR_MISALIGNED;
+  if (!(eps >= 0.f)) return TG_ERR_INVALID_ARGUMENT;
+  TG_TRY(check_device());
+  // BN=256 only when the Q/K/V boundaries fall on 256-column tile edges
+  int bn = pick_bn(M, N);
+  if (bn == 256 && ((q_cols % 256) || (kv_cols % 256))) bn = 128;
+  CUtensorMap ta, tb;
+  TG_TRY(make_tmap_bf16_2d(&ta, x, (uint64_t)M, (uint64_t)hidden, (uint64_t)ld_x, 64, 128));
+  TG_TRY(make_tmap_bf16_2d(&tb, w_qkv, (uint64_t)N, (uint64_t)hidden, (uint64_t)ld_w, 64, bn));
+  GemmParams p{};
+  p.M = M;
+  p.N = N;
+  p.K = hidden;
+  p.rmsnorm = 1;
+  p.eps = eps;
+  p.c = reinterpret_cast<uint16_t*>(q_out);
+  p.ldc = ld_q;
+  p.pos = pos;
+  p.cos_sin = cos_sin;
+  p.max_pos = max_pos;
+  p.q_cols = q_cols;
+  p.k_cols = kv_cols;
+  p.k_out = reinterpret_cast<uint16_t*>(cache_k) + slot_offset * ld_cache;
+  p.v_out = reinterpret_cast<uint16_t*>(cache_v) + slot_offset * ld_cache;
+  p.ld_kv = ld_cache;
+  p.status = status;
+  if (bn == 256) return launch_gemm<256, 4, EpiQKV>(ta, tb, p, (cudaStream_t)stream);
+  return launch_gemm<128, 3, EpiQKV>(ta, tb, p, (cudaStream_t)stream);
 }

@@ -71,10 +71,10 @@ def test_host_side_argument_errors(lib):
     cu = (C.c_int32 * 2)(0, 8)
     # attention: head_dim other than 128 is not implemented
     assert lib.tg_gated_attention(p, 2048, p, 1024, p, 1024, p, cu, 1, 16, 8, 64, p, p, p,
-                                  1.0, p, 2048, None, None, None) == -6
+                                  1.0, p, 2048, None, None, 0, None, None) == -6
     # attention: odd GQA group
     assert lib.tg_gated_attention(p, 2048, p, 1024, p, 1024, p, cu, 1, 3, 3, 128, p, p, p,
-                                  1.0, p, 2048, None, None, None) == -6
+                                  1.0, p, 2048, None, None, 0, None, None) == -6
     # projections: N not a multiple of 128, K not a multiple of 64
     assert lib.tg_linear(p, 64, p, 64, p, 100, 4, 100, 64, 0, 0.0, None, 0, None, None) == -6
     assert lib.tg_linear(p, 96, p, 96, p, 128, 4, 128, 96, 0, 0.0, None, 0, None, None) == -6

@@ -310,12 +310,14 @@ def _attn_inputs(lengths, Hq, Hkv, seed, pos_spread=4, dense=False):
     return q, k, v, pos, bias, gamma, cu
 
 
-def _run_attention(tg, q, k, v, pos, bias, gamma, beta, cu, Hq, Hkv, lse=True):
+def _run_attention(tg, q, k, v, pos, bias, gamma, beta, cu, Hq, Hkv, lse=True, split=True):
     Kt = q.shape[0]
     lse_t = torch.full((Hq, Kt), float("nan"), device="cuda") if lse else None
     st = _status()
+    ws = None if split else torch.empty(0, dtype=torch.uint8, device="cuda")
     o = tg.tg_gated_attention(_dev(q), _dev(k), _dev(v), _dev(torch.from_numpy(cu)), cu, Hq, Hkv,
-                              _dev(pos), _dev(bias), _dev(gamma), beta, lse=lse_t, status=st)
+                              _dev(pos), _dev(bias), _dev(gamma), beta, lse=lse_t, workspace=ws,
+                              status=st)
     assert tg.tg_status_read(st) == 0
     return o.cpu(), (lse_t.cpu() if lse else None)
 
@@ -350,10 +352,24 @@ def test_attention_group4_and_beta(tg):
     _check_attention(o, lse, q, k, v, pos, bias, gamma, 0.7, cu, 8, 2)
 
 
-def test_attention_n16k_kept_1638(tg):
+@pytest.mark.parametrize("split", [True, False])
+def test_attention_n16k_kept_1638(tg, split):
+    cu_h = np.array([0, 1638], dtype=np.int32)
+    assert tg.tg_gated_attention_workspace_size(cu_h, 16, 8) > 0  # this layout splits
     q, k, v, pos, bias, gamma, cu = _attn_inputs([1638], 16, 8, seed=1638, pos_spread=10)
-    o, lse = _run_attention(tg, q, k, v, pos, bias, gamma, 1.0, cu, 16, 8)
+    o, lse = _run_attention(tg, q, k, v, pos, bias, gamma, 1.0, cu, 16, 8, split=split)
     _check_attention(o, lse, q, k, v, pos, bias, gamma, 1.0, cu, 16, 8)
+
+
+def test_attention_split_varlen_requests(tg):
+    lengths = [2000, 60, 3, 1100]
+    q, k, v, pos, bias, gamma, cu = _attn_inputs(lengths, 16, 8, seed=77, pos_spread=6)
+    assert tg.tg_gated_attention_workspace_size(cu, 16, 8) > 0
+    o, lse = _run_attention(tg, q, k, v, pos, bias, gamma, 0.9, cu, 16, 8)
+    _check_attention(o, lse, q, k, v, pos, bias, gamma, 0.9, cu, 16, 8)
+    o2, lse2 = _run_attention(tg, q, k, v, pos, bias, gamma, 0.9, cu, 16, 8, split=False)
+    assert (o.double() - o2.double()).abs().max() <= 2 ** -7
+    assert (lse - lse2).abs().max() <= 1e-4
 
 
 def test_attention_n128k_kept_13107_sampled_rows(tg):
@@ -390,3 +406,69 @@ def test_attention_deterministic(tg):
     a, la = _run_attention(tg, q, k, v, pos, bias, gamma, 1.0, cu, 16, 8)
     b, lb = _run_attention(tg, q, k, v, pos, bias, gamma, 1.0, cu, 16, 8)
     assert torch.equal(a, b) and torch.equal(la, lb)
+
+
+# ------------------------------------------------------------------ fused QKV + RoPE + cache
+
+@pytest.mark.parametrize("M", [1, 257, 1638])
+def test_qkv_rope_cache_against_oracle(tg, M):
+    Hq, Hkv, d, H = 16, 8, 128, 2048
+    x = S.uniform_rows(M, H, seed=M)
+    w = S.uniform_rows((Hq + 2 * Hkv) * d, H, seed=M + 1, scale=0.02)
+    pos = torch.sort(torch.randperm(16384, generator=torch.Generator().manual_seed(M))[:M])[0]
+    pos = pos.to(torch.int32)
+    cs = tg.tg_rope_table(16384, d, 1.0e6)
+    slot = 5
+    ck = torch.zeros((M + slot, Hkv * d), dtype=torch.bfloat16, device="cuda")
+    cv = torch.zeros_like(ck)
+    st = _status()
+    q = tg.tg_qkv_rope_cache(_dev(x), _dev(w), _dev(pos), cs, ck, cv, Hq, Hkv, slot_offset=slot,
+                             status=st)
+    assert tg.tg_status_read(st) == 0
+    a = O.rmsnorm_rows(x)
+    qkv = a @ _f64(w).T
+    want_q = O.rope(qkv[:, :Hq * d].reshape(M, Hq, d), pos, 1.0e6).reshape(M, -1)
+    want_k = O.rope(qkv[:, Hq * d:(Hq + Hkv) * d].reshape(M, Hkv, d), pos, 1.0e6).reshape(M, -1)
+    want_v = qkv[:, (Hq + Hkv) * d:]
+    for got, want in ((q, want_q), (ck[slot:], want_k), (cv[slot:], want_v)):
+        err = np.abs(_f64(got.cpu()) - want)
+        assert np.all(err <= 2.0 ** -7 * np.abs(want) + 2e-3), err.max()
+    assert torch.count_nonzero(ck[:slot]) == 0 and torch.count_nonzero(cv[:slot]) == 0
+
+
+def test_qkv_rope_cache_matches_unfused_path(tg):
+    """The fused call equals projection -> RoPE -> KV copy up to one bf16 rounding."""
+    M, Hq, Hkv, d, H = 300, 16, 8, 128, 2048
+    x = _dev(S.uniform_rows(M, H, seed=4))
+    w = _dev(S.uniform_rows((Hq + 2 * Hkv) * d, H, seed=5, scale=0.02))
+    pos = _dev(torch.arange(0, 3 * M, 3, dtype=torch.int32))
+    cs = tg.tg_rope_table(4096, d, 1.0e6)
+    ck = torch.empty((M, Hkv * d), dtype=torch.bfloat16, device="cuda")
+    cv = torch.empty_like(ck)
+    q = tg.tg_qkv_rope_cache(x, w, pos, cs, ck, cv, Hq, Hkv)
+    qkv = tg.tg_linear(x, w, rmsnorm=True)
+    tg.tg_gather_rope(qkv, qkv, rope_pos=pos, rope_cols=(0, (Hq + Hkv) * d), head_dim=d,
+                      cos_sin=cs)
+    ref = qkv.double()
+    # The unfused path rounds to bf16 before rotating: per element its error is bounded
+    # by 2^-8 of the rotation pair's magnitude (which the rotation preserves) plus one
+    # final rounding of each path.
+    for got, want in ((q, ref[:, :Hq * d]), (ck, ref[:, Hq * d:(Hq + Hkv) * d]),
+                      (cv, ref[:, (Hq + Hkv) * d:])):
+        w = want.view(M, -1, 2, d // 2)
+        pair = torch.sqrt(w[:, :, 0] ** 2 + w[:, :, 1] ** 2).repeat(1, 1, 2).view(M, -1)
+        err = (got.double() - want).abs()
+        assert (err <= 2.0 ** -7 * pair + 2.0 ** -8 * want.abs() + 1e-3).all(), err.max()
+
+
+def test_qkv_rope_cache_position_out_of_table_sets_status(tg):
+    M, Hq, Hkv, d, H = 4, 2, 2, 128, 64
+    x = _dev(S.uniform_rows(M, H, seed=1))
+    w = _dev(S.uniform_rows((Hq + 2 * Hkv) * d, H, seed=2, scale=0.1))
+    pos = _dev(torch.tensor([0, 1, 99, 2], dtype=torch.int32))
+    cs = tg.tg_rope_table(8, d, 1.0e6)
+    ck = torch.empty((M, Hkv * d), dtype=torch.bfloat16, device="cuda")
+    cv = torch.empty_like(ck)
+    st = _status()
+    tg.tg_qkv_rope_cache(x, w, pos, cs, ck, cv, Hq, Hkv, status=st)
+    assert tg.tg_status_read(st) & tg.STATUS_BOUNDS
