@@ -16,10 +16,11 @@ Multi-GPU (torchrun, one rank per GPU): every rank runs an independent replica o
 its own batch (no collective on the data path); value = all ranks' tokens / the
 slowest rank's time.
 
-Timing: W untimed warm-up steps; then K steps, each replayed from a CUDA graph of the
-step with timing events at every stage boundary.  L2 is flushed (a 512 MiB write)
-before every timed step, outside the events.  SM clocks and throttle reasons are
-sampled through NVML during the timed region.
+Timing: W untimed warm-up steps; then K steps, each a replay of a CUDA graph of the step
+between two CUDA events; L2 is flushed (a 512 MiB write) before every timed step, outside
+the events.  SM clocks and throttle reasons are sampled through NVML during that loop.  A
+second loop of K replays of the same step captured with timing events at every stage
+boundary gives the per-stage times (and the roofline of the dominant kernel).
 """
 from __future__ import annotations
 
@@ -89,6 +90,9 @@ def stage_work(wl, kept_counts):
         "seq_rmsnorm": {"bound": "hbm", "bytes": T * 13},
         "topk_compact": {"bound": "hbm", "bytes": T * 5 + K * 12},
         "gather": {"bound": "hbm", "bytes": 2 * K * H * 2 + K * 4},
+        "qkv_rope_cache": {"bound": "tensor", "flops": 2 * K * H * nqkv,
+                           "bytes": K * H * 2 + nqkv * H * 2 + K * nqkv * 2 + K * 4
+                           + K * (H // 128) * 4},
         "qkv_proj": {"bound": "tensor", "flops": 2 * K * H * nqkv,
                      "bytes": K * H * 2 + nqkv * H * 2 + K * nqkv * 2},
         "rope": {"bound": "hbm", "bytes": 2 * K * (hq + hkv) * d * 2 + K * 4},
@@ -200,84 +204,106 @@ def run_ours(args, rank, world):
     if status:
         raise SystemExit(f"device status {status:#x} after warm-up")
 
-    # stage boundary events (external: they become event nodes inside the graph)
-    marks = []
+    # Two CUDA graphs of the same step: a plain one for the headline timing, and one with
+    # external timing events at every stage boundary for the per-stage breakdown (event
+    # nodes between kernels cost a little time, so they stay out of the headline).
     use_graph = args.launch == "graph"
+    marks = []
 
-    def make_marker(evs):
-        def marker(name):
-            e = torch.cuda.Event(enable_timing=True, external=use_graph)
-            e.record(stream)
-            evs.append((name, e))
-        return marker
+    def capture(with_marks):
+        evs = []
+        g = torch.cuda.CUDAGraph()
+        side = torch.cuda.Stream()
+        side.wait_stream(stream)
+        with torch.cuda.stream(side):
+            with torch.cuda.graph(g, stream=side):
+                cap = torch.cuda.current_stream()
+                if with_marks:
+                    e0 = torch.cuda.Event(enable_timing=True, external=True)
+                    e0.record(cap)
+                    evs.append(("start", e0))
 
-    start_ev = torch.cuda.Event(enable_timing=True, external=use_graph)
-    graph = None
+                    def marker(name):
+                        e = torch.cuda.Event(enable_timing=True, external=True)
+                        e.record(cap)
+                        evs.append((name, e))
+                    pipe.marker = marker
+                step()
+                pipe.marker = None
+        stream.wait_stream(side)
+        return g, evs
+
     launches_before = tg.launch_count
     if use_graph:
-        g = torch.cuda.CUDAGraph()
-        s_side = torch.cuda.Stream()
-        s_side.wait_stream(stream)
-        with torch.cuda.stream(s_side):
-            pipe.marker = make_marker(marks)
-            with torch.cuda.graph(g, stream=s_side):
-                start_ev.record(s_side)
-                # inside capture the current stream is s_side
-                stream_cap = torch.cuda.current_stream()
-                pipe.marker = None
-                evs = []
-
-                def marker(name, _evs=evs):
-                    e = torch.cuda.Event(enable_timing=True, external=True)
-                    e.record(stream_cap)
-                    _evs.append((name, e))
-                pipe.marker = marker
-                step()
-            pipe.marker = None
-        stream.wait_stream(s_side)
-        marks = evs
-        graph = g
-    launches_per_step = tg.launch_count - launches_before
+        graph_plain, _ = capture(False)
+        launches_per_step = tg.launch_count - launches_before
+        graph_marked, marks = capture(True)
+    else:
+        graph_plain = graph_marked = None
+        step()
+        launches_per_step = tg.launch_count - launches_before
     torch.cuda.synchronize()
 
     flush = torch.empty(512 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
     per_stage = {}
     step_ms = []
+    marked_ms = []
 
-    def run_timed_step():
+    def run_step_plain():
         flush.fill_(1.0)  # evict L2 (outside the step's events)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
         if use_graph:
-            graph.replay()
+            graph_plain.replay()
         else:
-            marks.clear()
-            start_ev.record(stream)
-            pipe.marker = make_marker(marks)
+            step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        step_ms.append(e0.elapsed_time(e1))
+
+    def run_step_marked():
+        flush.fill_(1.0)
+        if use_graph:
+            graph_marked.replay()
+            evs = marks
+        else:
+            evs = []
+            e0 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            evs.append(("start", e0))
+
+            def marker(name):
+                e = torch.cuda.Event(enable_timing=True)
+                e.record(stream)
+                evs.append((name, e))
+            pipe.marker = marker
             step()
             pipe.marker = None
         torch.cuda.synchronize()
-        t_prev = start_ev
-        for name, e in marks:
-            ms = t_prev.elapsed_time(e)
-            per_stage.setdefault(name, []).append(ms)
-            t_prev = e
-        step_ms.append(start_ev.elapsed_time(marks[-1][1]))
+        prev = evs[0][1]
+        for name, e in evs[1:]:
+            per_stage.setdefault(name, []).append(prev.elapsed_time(e))
+            prev = e
+        marked_ms.append(evs[0][1].elapsed_time(evs[-1][1]))
 
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize()
-    launches_timed_before = tg.launch_count
     with ClockSampler(dev.index) as clk:
         for _ in range(args.steps):
-            run_timed_step()
+            run_step_plain()
     torch.cuda.synchronize()
-    eager_launches = tg.launch_count - launches_timed_before
-    gpu_launches = launches_per_step * args.steps if use_graph else eager_launches
+    gpu_launches = launches_per_step * args.steps
     total_ms = sum(step_ms)
     if world > 1:
         t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
         torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
         total_ms = float(t.item())
         torch.distributed.barrier()
+    # per-stage breakdown (second timed loop, same step with stage events)
+    for _ in range(args.steps):
+        run_step_marked()
     status = tg.tg_status_read(pipe.status)
     if status:
         raise SystemExit(f"device status {status:#x} after timed steps")
@@ -299,7 +325,7 @@ def run_ours(args, rank, world):
         h_dev.copy_(h_pin, non_blocking=True)
         pr_dev.copy_(pr_pin, non_blocking=True)
         if use_graph:
-            graph.replay()
+            graph_plain.replay()
         else:
             step()
         x_host.copy_(P["x"], non_blocking=True)
@@ -360,6 +386,7 @@ def run_ours(args, rank, world):
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
         "gpu_launches": gpu_launches,
+        "ms_per_step_with_stage_events": sum(marked_ms) / max(1, len(marked_ms)),
         "roofline": roofline,
         "stages": {k: {kk: (round(vv, 5) if isinstance(vv, float) else vv)
                        for kk, vv in v.items()} for k, v in stages.items()},

@@ -221,12 +221,16 @@ int tg_topk_compact(const float* z, const uint8_t* prunable, const int32_t* cu_s
  * src has src_rows rows; an index outside [0, src_rows) skips that output row and sets
  * TG_STATUS_BOUNDS (status may be NULL).  dst may equal src (in place) only when
  * row_idx is NULL.  rope_pos values must lie in [0, max_pos); rows outside are copied
- * unrotated and set TG_STATUS_BOUNDS.
+ * unrotated and set TG_STATUS_BOUNDS.  Without rope, row_ssq_out (float32, row stride
+ * ld_ssq_out >= width / 128, width a multiple of 128; may be NULL) receives the sums of
+ * squares of each copied row per 128-column group, for a later folded RMSNorm.
  */
 int tg_gather_rope(const tg_bf16* src, int64_t ld_src, int64_t src_rows,
-                   const int32_t* row_idx, int64_t n_rows, int width, const int32_t* rope_pos, int rope_col_begin,
-                   int rope_col_end, int head_dim, const float* cos_sin, int max_pos,
-                   tg_bf16* dst, int64_t ld_dst, uint32_t* status, tg_stream_t stream);
+                   const int32_t* row_idx, int64_t n_rows, int width,
+                   const int32_t* rope_pos, int rope_col_begin, int rope_col_end,
+                   int head_dim, const float* cos_sin, int max_pos, tg_bf16* dst,
+                   int64_t ld_dst, float* row_ssq_out, int64_t ld_ssq_out, uint32_t* status,
+                   tg_stream_t stream);
 
 /* ------------------------------------------------------------------ KV cache */
 
@@ -296,12 +300,16 @@ size_t tg_gated_attention_workspace_size(const int32_t* cu_kept_host, int batch,
  * RMSNorm of weight 1 folded into the epilogue), else r_m = 1.
  * a: bf16 [M, K] (lda); w: bf16 [N, K] (ldw, output rows); c, residual: bf16 [M, N]
  * (ldc, ld_res; residual may be NULL and may equal c).  K multiple of 64, N multiple
- * of 128, strides multiples of 8.  tcgen05 GEMM, TMA-fed, fp32 accumulation in TMEM.
- * status may be NULL.
+ * of 128, strides multiples of 8.  row_ssq_out (may be NULL): float32 [M, N/128] (row
+ * stride ld_ssq_out) receiving the sums of squares of each stored bf16 output row per
+ * 128 columns (what a following folded RMSNorm needs).  tcgen05 GEMM, TMA-fed, fp32
+ * accumulation in TMEM; without rmsnorm_a and with N a multiple of 256 it runs on CTA
+ * pairs (tcgen05 cta_group::2, 256 x 256 tiles).  status may be NULL.
  */
 int tg_linear(const tg_bf16* a, int64_t lda, const tg_bf16* w, int64_t ldw, tg_bf16* c,
               int64_t ldc, int64_t M, int N, int K, int rmsnorm_a, float eps,
-              const tg_bf16* residual, int64_t ld_res, uint32_t* status, tg_stream_t stream);
+              const tg_bf16* residual, int64_t ld_res, float* row_ssq_out,
+              int64_t ld_ssq_out, uint32_t* status, tg_stream_t stream);
 
 /*
  * One gated layer's QKV projection with RoPE and the compacted KV-cache write fused into
@@ -318,14 +326,17 @@ int tg_linear(const tg_bf16* a, int64_t lda, const tg_bf16* w, int64_t ldw, tg_b
  * (rows: Wq, Wk, Wv); pos: int32 [M] (values < max_pos, else TG_STATUS_BOUNDS and the
  * row uses position 0); q_out: bf16 [M, n_q_heads * head_dim] (ld_q); cache_k/cache_v:
  * bf16 rows of n_kv_heads * head_dim (ld_cache).  head_dim = 128, hidden multiple of 64.
- * status may be NULL.
+ * row_ssq_in (may be NULL): float32 [M, hidden/128] (row stride ld_ssq_in) holding the
+ * sums of squares of x per 128 columns (from tg_gather_rope or tg_linear row_ssq_out);
+ * with it the norm needs no extra read of x and the GEMM runs on CTA pairs; without it
+ * the norm is accumulated from x inside the GEMM.  status may be NULL.
  */
 int tg_qkv_rope_cache(const tg_bf16* x, int64_t ld_x, const tg_bf16* w_qkv, int64_t ld_w,
                       int64_t M, int hidden, int n_q_heads, int n_kv_heads, int head_dim,
                       float eps, const int32_t* pos, const float* cos_sin, int max_pos,
                       tg_bf16* q_out, int64_t ld_q, tg_bf16* cache_k, tg_bf16* cache_v,
-                      int64_t ld_cache, int64_t slot_offset, uint32_t* status,
-                      tg_stream_t stream);
+                      int64_t ld_cache, int64_t slot_offset, const float* row_ssq_in,
+                      int64_t ld_ssq_in, uint32_t* status, tg_stream_t stream);
 
 #ifdef __cplusplus
 }

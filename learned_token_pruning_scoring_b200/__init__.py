@@ -206,7 +206,8 @@ def tg_topk_compact(z, prunable, cu_seqlens, cu_seqlens_host, cu_kept, cu_kept_h
 
 
 def tg_gather_rope(src, dst=None, row_idx=None, n_rows=None, rope_pos=None,
-                   rope_cols=(0, 0), head_dim=128, cos_sin=None, status=None, stream=None):
+                   rope_cols=(0, 0), head_dim=128, cos_sin=None, row_ssq=None, status=None,
+                   stream=None):
     ld_src = _mat(src, "src")
     width = src.shape[1]
     if n_rows is None:
@@ -215,10 +216,11 @@ def tg_gather_rope(src, dst=None, row_idx=None, n_rows=None, rope_pos=None,
         dst = torch.empty((n_rows, width), dtype=src.dtype, device=src.device)
     ld_dst = _mat(dst, "dst")
     max_pos = cos_sin.shape[0] if cos_sin is not None else 0
+    ld_ssq = _mat(row_ssq, "row_ssq") if row_ssq is not None else 0
     rc = lib.tg_gather_rope(_ptr(src), ld_src, src.shape[0], _ptr(row_idx), n_rows, width,
                             _ptr(rope_pos), int(rope_cols[0]), int(rope_cols[1]), head_dim,
-                            _ptr(cos_sin), max_pos, _ptr(dst), ld_dst, _ptr(status),
-                            _stream(stream))
+                            _ptr(cos_sin), max_pos, _ptr(dst), ld_dst, _ptr(row_ssq), ld_ssq,
+                            _ptr(status), _stream(stream))
     _check(rc, "tg_gather_rope")
     _count()
     return dst
@@ -273,7 +275,8 @@ def tg_gated_attention(q, k, v, cu_kept, cu_kept_host, n_q_heads, n_kv_heads, ke
     return o
 
 
-def tg_linear(a, w, c=None, rmsnorm=False, eps=1e-6, residual=None, status=None, stream=None):
+def tg_linear(a, w, c=None, rmsnorm=False, eps=1e-6, residual=None, row_ssq=None, status=None,
+              stream=None):
     lda, ldw = _mat(a, "a"), _mat(w, "w")
     M, K = a.shape
     N = w.shape[0]
@@ -281,16 +284,18 @@ def tg_linear(a, w, c=None, rmsnorm=False, eps=1e-6, residual=None, status=None,
         c = torch.empty((M, N), dtype=a.dtype, device=a.device)
     ldc = _mat(c, "c")
     ldr = _mat(residual, "residual") if residual is not None else 0
+    ld_ssq = _mat(row_ssq, "row_ssq") if row_ssq is not None else 0
     rc = lib.tg_linear(_ptr(a), lda, _ptr(w), ldw, _ptr(c), ldc, M, N, K, 1 if rmsnorm else 0,
-                       float(eps), _ptr(residual), ldr, _ptr(status), _stream(stream))
+                       float(eps), _ptr(residual), ldr, _ptr(row_ssq), ld_ssq, _ptr(status),
+                       _stream(stream))
     _check(rc, "tg_linear")
     _count()
     return c
 
 
 def tg_qkv_rope_cache(x, w_qkv, pos, cos_sin, cache_k, cache_v, n_q_heads, n_kv_heads,
-                      q_out=None, head_dim=128, eps=1e-6, slot_offset=0, status=None,
-                      stream=None):
+                      q_out=None, head_dim=128, eps=1e-6, slot_offset=0, row_ssq=None,
+                      status=None, stream=None):
     """Fused QKV projection (RMSNorm folded) + RoPE at `pos` + compacted KV-cache write."""
     ld_x, ld_w = _mat(x, "x"), _mat(w_qkv, "w_qkv")
     M, hidden = x.shape
@@ -300,10 +305,12 @@ def tg_qkv_rope_cache(x, w_qkv, pos, cos_sin, cache_k, cache_v, n_q_heads, n_kv_
     ld_c = _mat(cache_k, "cache_k")
     if _mat(cache_v, "cache_v") != ld_c:
         raise ValueError("cache_k and cache_v must share a row stride")
+    ld_ssq = _mat(row_ssq, "row_ssq") if row_ssq is not None else 0
     rc = lib.tg_qkv_rope_cache(_ptr(x), ld_x, _ptr(w_qkv), ld_w, M, hidden, n_q_heads, n_kv_heads,
                                head_dim, float(eps), _ptr(pos), _ptr(cos_sin), cos_sin.shape[0],
                                _ptr(q_out), ld_q, _ptr(cache_k), _ptr(cache_v), ld_c,
-                               int(slot_offset), _ptr(status), _stream(stream))
+                               int(slot_offset), _ptr(row_ssq), ld_ssq, _ptr(status),
+                               _stream(stream))
     _check(rc, "tg_qkv_rope_cache")
     _count()
     return q_out
@@ -375,6 +382,7 @@ class GatedPrefill:
             kept_pos=torch.empty(K, dtype=torch.int32, device=dev),
             kept_bias=torch.empty(K, **f32),
             x=torch.empty((K, self.hidden), **bf),
+            ssq=torch.empty((K, self.hidden // 128), **f32),
             qkv=torch.empty((K, nqkv), **bf),
             o=torch.empty((K, self.hq * self.d), **bf),
             attn_ws=torch.empty(tg_gated_attention_workspace_size(ck_h, self.hq, self.hkv, self.d),
@@ -403,7 +411,8 @@ class GatedPrefill:
         """x = h[kept_idx]: the kept rows go up, pruned rows stop here."""
         P = self.planned
         if P["K"]:
-            tg_gather_rope(h, P["x"], row_idx=P["kept_idx"], status=self.status, stream=stream)
+            tg_gather_rope(h, P["x"], row_idx=P["kept_idx"], row_ssq=P["ssq"], status=self.status,
+                           stream=stream)
             self._mark("gather")
 
     def layer(self, i, stream=None):
@@ -418,7 +427,7 @@ class GatedPrefill:
         if self.fused_qkv:
             tg_qkv_rope_cache(x, L.Wqkv, P["kept_pos"], self.cos_sin, ck, cv, self.hq, self.hkv,
                               q_out=qkv[:, :nq], head_dim=self.d, eps=self.norm_eps,
-                              status=self.status, stream=stream)
+                              row_ssq=P["ssq"], status=self.status, stream=stream)
             self._mark("qkv_rope_cache")
         else:
             tg_linear(x, L.Wqkv, qkv, rmsnorm=True, eps=self.norm_eps, status=self.status,
@@ -436,7 +445,7 @@ class GatedPrefill:
                            head_dim=self.d, workspace=P["attn_ws"], status=self.status,
                            stream=stream)
         self._mark("attention")
-        tg_linear(o, L.Wo, x, residual=x, status=self.status, stream=stream)
+        tg_linear(o, L.Wo, x, residual=x, row_ssq=P["ssq"], status=self.status, stream=stream)
         self._mark("out_proj")
 
     def upper_layers(self, h, stream=None):

@@ -35,16 +35,16 @@ SIGNATURES = {
     "tg_seq_rmsnorm": (_i32, [_p, _p, _p, _i32, _p, _f32, _p, _p, _p]),
     "tg_topk_compact": (_i32, [_p, _p, _p, _p, _p, _p, _i32, _p, _p, _p, _p, _p]),
     "tg_gather_rope": (_i32, [_p, _i64, _i64, _p, _i64, _i32, _p, _i32, _i32, _i32, _p, _i32,
-                              _p, _i64, _p, _p]),
+                              _p, _i64, _p, _i64, _p, _p]),
     "tg_kv_compact": (_i32, [_p, _i64, _p, _i64, _i64, _p, _i64, _i32, _p, _p, _i64, _i64, _i64,
                              _p, _p]),
     "tg_gated_attention": (_i32, [_p, _i64, _p, _i64, _p, _i64, _p, _p, _i32, _i32, _i32, _i32,
                                   _p, _p, _p, _f32, _p, _i64, _p, _p, _sz, _p, _p]),
     "tg_gated_attention_workspace_size": (_sz, [_p, _i32, _i32, _i32, _i32]),
     "tg_qkv_rope_cache": (_i32, [_p, _i64, _p, _i64, _i64, _i32, _i32, _i32, _i32, _f32, _p, _p,
-                                 _i32, _p, _i64, _p, _p, _i64, _i64, _p, _p]),
+                                 _i32, _p, _i64, _p, _p, _i64, _i64, _p, _i64, _p, _p]),
     "tg_linear": (_i32, [_p, _i64, _p, _i64, _p, _i64, _i64, _i32, _i32, _i32, _f32, _p, _i64,
-                         _p, _p]),
+                         _p, _i64, _p, _p]),
 }
 
 

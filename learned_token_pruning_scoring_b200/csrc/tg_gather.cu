@@ -84,8 +84,49 @@ struct GatherArgs {
   int max_pos;
   uint16_t* dst;
   int64_t ld_dst;
+  float* row_ssq;  // optional: sums of squares of each gathered row per 128 columns
+  int64_t ld_ssq;
   uint32_t* status;
 };
+
+// Sum of squares of the 8 bf16 values of one 16-byte vector.
+__device__ __forceinline__ float ssq8(const uint4& v) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  float s = 0.f;
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const float2 f = unpack_bf16x2(w[e]);
+    s = fmaf(f.x, f.x, s);
+    s = fmaf(f.y, f.y, s);
+  }
+  return s;
+}
+
+// Gathered copy of one row that also writes its sums of squares per 128 columns
+// (16 vectors): lane l holds vectors l, l+32, ...; groups of 16 lanes share a group.
+__device__ __forceinline__ void copy_row_ssq(const uint4* __restrict__ s, uint4* __restrict__ d,
+                                             int nvec, int lane, float* ssq_row) {
+  for (int base = 0; base < nvec; base += 32 * kVecPerBatch) {
+    uint4 buf[kVecPerBatch];
+#pragma unroll
+    for (int u = 0; u < kVecPerBatch; ++u) {
+      const int v = base + u * 32 + lane;
+      if (v < nvec) buf[u] = s[v];
+    }
+#pragma unroll
+    for (int u = 0; u < kVecPerBatch; ++u) {
+      const int v = base + u * 32 + lane;
+      float q = v < nvec ? ssq8(buf[u]) : 0.f;
+      // reduce over the 16 lanes of this half-warp (vectors of one 128-column group)
+#pragma unroll
+      for (int o = 8; o > 0; o >>= 1) q += __shfl_xor_sync(0xFFFFFFFFu, q, o);
+      if (v < nvec) {
+        d[v] = buf[u];
+        if ((lane & 15) == 0) ssq_row[v >> 4] = q;
+      }
+    }
+  }
+}
 
 __global__ void __launch_bounds__(kCopyWarps * 32) gather_rope_kernel(GatherArgs a) {
   const int lane = threadIdx.x & 31;
@@ -104,7 +145,8 @@ __global__ void __launch_bounds__(kCopyWarps * 32) gather_rope_kernel(GatherArgs
     if (a.rope_pos && (pos < 0 || pos >= a.max_pos) && lane == 0 && a.status)
       atomicOr(a.status, TG_STATUS_BOUNDS);
     if (pos < 0 || pos >= a.max_pos || a.rope_begin >= a.rope_end) {
-      copy_row(s, d, 0, nvec, lane);
+      if (a.row_ssq) copy_row_ssq(s, d, nvec, lane, a.row_ssq + r * a.ld_ssq);
+      else copy_row(s, d, 0, nvec, lane);
       continue;
     }
     const int vb = a.rope_begin >> 3, ve = a.rope_end >> 3;
@@ -191,7 +233,8 @@ extern "C" int tg_gather_rope(const tg_bf16* src, int64_t ld_src, int64_t src_ro
                               const int32_t* row_idx, int64_t n_rows, int width,
                               const int32_t* rope_pos, int rope_col_begin, int rope_col_end,
                               int head_dim, const float* cos_sin, int max_pos, tg_bf16* dst,
-                              int64_t ld_dst, uint32_t* status, tg_stream_t stream) {
+                              int64_t ld_dst, float* row_ssq_out, int64_t ld_ssq_out,
+                              uint32_t* status, tg_stream_t stream) {
   if (n_rows < 0 || width <= 0 || (width & 7) || src_rows < 0) return TG_ERR_INVALID_ARGUMENT;
   if (!row_idx && n_rows > src_rows) return TG_ERR_INVALID_ARGUMENT;
   if (n_rows == 0) return TG_OK;
@@ -200,6 +243,8 @@ extern "C" int tg_gather_rope(const tg_bf16* src, int64_t ld_src, int64_t src_ro
     return TG_ERR_MISALIGNED;
   if (ld_src < width || ld_dst < width) return TG_ERR_INVALID_ARGUMENT;
   if (row_idx && src == dst) return TG_ERR_INVALID_ARGUMENT;
+  if (row_ssq_out && (rope_pos || (width % 128) || ld_ssq_out < width / 128))
+    return TG_ERR_INVALID_ARGUMENT;
   if (rope_pos) {
     if (!cos_sin || max_pos <= 0 || head_dim < 16 || (head_dim & 15)) return TG_ERR_INVALID_ARGUMENT;
     if (rope_col_begin < 0 || rope_col_end > width || rope_col_begin > rope_col_end ||
@@ -210,7 +255,7 @@ extern "C" int tg_gather_rope(const tg_bf16* src, int64_t ld_src, int64_t src_ro
   TG_TRY(check_device());
   GatherArgs a{reinterpret_cast<const uint16_t*>(src), ld_src, src_rows, row_idx, n_rows, width,
                rope_pos, rope_col_begin, rope_col_end, head_dim, cos_sin, max_pos,
-               reinterpret_cast<uint16_t*>(dst), ld_dst, status};
+               reinterpret_cast<uint16_t*>(dst), ld_dst, row_ssq_out, ld_ssq_out, status};
   gather_rope_kernel<<<copy_grid(n_rows), kCopyWarps * 32, 0, (cudaStream_t)stream>>>(a);
   return check_launch();
 }

@@ -1,19 +1,28 @@
-// tcgen05 GEMM C[M, N] = A[M, K] * W[N, K]^T for bf16 inputs with fp32 accumulation
-// in tensor memory, fed by TMA through a STAGES-deep shared-memory ring.
+// tcgen05 GEMMs C[M, N] = A[M, K] * W[N, K]^T for bf16 inputs with fp32 accumulation
+// in tensor memory, fed by TMA through a shared-memory ring.
 //
-// Roles (192 threads):
+// gemm_kernel (one CTA per 128 x BN tile), 192 threads:
 //   warp 0     one thread issues the TMA loads of A and W tiles (128-byte swizzle);
 //   warp 1     allocates TMEM; one thread issues tcgen05.mma (M=128, N=BN, K=16);
 //   warps 2-5  epilogue, one TMEM lane quarter each (thread = output row).  With a
 //              folded RMSNorm they also read every A stage from shared memory during
 //              the mainloop to accumulate the row's sum of squares, so the norm costs
 //              no extra HBM pass: RMSNorm(a) W^T = r * (a W^T), r = 1/sqrt(mean a^2 + eps).
-// Epilogues: EpiStore writes bf16 rows (optionally + residual); EpiScore reduces each
-// row to one scalar s = sum_f w2[f] SiLU(r * acc[f]) and writes per-32-row partial
-// sums of s^2 for the sequence normalisation; EpiQKV applies rotate-half RoPE at the
-// row's position to the Q and K heads (pairs of columns 64 apart, from the TMEM chunks
-// c and c + 2) and writes Q, K and V tiles to three destinations (Q rows, and the K
-// and V rows of a compacted cache).
+// gemm_pair_kernel (a cluster of two CTAs per 256 x 256 tile), same roles: each CTA
+//   loads its 128 rows of A and its 128 rows of W; the even CTA issues the M=256 MMA
+//   (tcgen05 cta_group::2) that reads both CTAs' shared memory and writes each CTA's
+//   128 output rows into its own TMEM.  Per SM this halves the W bytes streamed per
+//   MMA, so a 6-stage ring covers the load latency.  Both CTAs' loads (cta_group::2
+//   TMA, no multicast) count their bytes on the even CTA's stage barrier, so the MMA
+//   issuer sees one barrier per stage with no forwarding hop; the even CTA's commits
+//   arrive on both CTAs' stage-free barriers.  A folded RMSNorm here
+//   takes per-row sums of squares computed by the producer of A (row_ssq_in).
+// Epilogues (per thread-row): EpiStore writes bf16 (+ residual, and optionally the
+// sums of squares of the stored bf16 values per 128 columns); EpiScore reduces the row
+// to s = sum_f w2[f] SiLU(r * acc[f]) and per-32-row partial sums of s^2; EpiQKV
+// applies rotate-half RoPE at the row's position to the Q and K heads (pairs of
+// columns 64 apart, from TMEM chunks c and c + 2) and routes Q, K and V tiles to their
+// destinations (Q rows and the K and V rows of a compacted cache).
 #pragma once
 #include <cuda.h>
 
@@ -30,11 +39,16 @@ struct GemmParams {
   int N, K;
   int rmsnorm;
   float eps;
+  // optional per-row sums of squares of A (K / 128 groups per row), used for the norm
+  const float* row_ssq_in;
+  int64_t ld_ssq_in;
   // EpiStore
   uint16_t* c;
   int64_t ldc;
   const uint16_t* residual;
   int64_t ldr;
+  float* row_ssq_out;  // optional: sums of squares of the stored row, per 128 columns
+  int64_t ld_ssq_out;
   // EpiScore
   const float* w2;
   float* s_out;
@@ -63,6 +77,140 @@ struct GemmCfg {
   static constexpr int THREADS = 192;
 };
 
+// Row scale of the folded RMSNorm from per-row partial sums of squares.
+__device__ __forceinline__ float rscale_from_ssq(const GemmParams& p, int64_t grow) {
+  const float* ss = p.row_ssq_in + grow * p.ld_ssq_in;
+  float t = 0.f;
+  for (int g = 0; g < p.K / 128; ++g) t += ss[g];
+  return rsqrtf(t / (float)p.K + p.eps);
+}
+
+// Epilogue of one output row held by this thread: BN accumulator columns at TMEM
+// address `tbase` (the warp's lane quarter), output columns n0 .. n0 + BN.  All lanes
+// of the warp must call it (tcgen05.ld is warp-collective).  Returns the row's score
+// for EpiScore.
+template <int BN, int EPI>
+__device__ __forceinline__ float epilogue_row(const GemmParams& p, uint32_t tbase, int64_t grow,
+                                              int n0, float rscale, const float* w2s) {
+  const bool live = grow < p.M;
+  float score = 0.f;
+  if (EPI == EpiQKV) {
+    // destination of this tile: Q, K or V (tiles never straddle the boundaries)
+    uint16_t* dst;
+    int dcol;
+    if (n0 < p.q_cols) {
+      dst = p.c + grow * p.ldc;
+      dcol = n0;
+    } else if (n0 < p.q_cols + p.k_cols) {
+      dst = p.k_out + grow * p.ld_kv;
+      dcol = n0 - p.q_cols;
+    } else {
+      dst = p.v_out + grow * p.ld_kv;
+      dcol = n0 - p.q_cols - p.k_cols;
+    }
+    const bool rope = n0 < p.q_cols + p.k_cols;
+    int pos = (rope && live) ? p.pos[grow] : 0;
+    if (pos < 0 || pos >= p.max_pos) {
+      if (live && p.status) atomicOr(p.status, TG_STATUS_BOUNDS);
+      pos = 0;
+    }
+    const float4* cs_row = reinterpret_cast<const float4*>(p.cos_sin + (int64_t)pos * 128);
+#pragma unroll 1
+    for (int pr = 0; pr < BN / 64; ++pr) {
+      // chunk pairs (0,2), (1,3), (4,6), (5,7): columns i and i + 64 of one head
+      const int ca = (pr & 1) + 4 * (pr >> 1), cb = ca + 2;
+      uint32_t ra[32], rb[32];
+      tmem_ld32(tbase + ca * 32, ra);
+      tmem_ld32(tbase + cb * 32, rb);
+      tmem_wait_ld();
+      if (live) {
+        uint4* da = reinterpret_cast<uint4*>(dst + dcol + ca * 32);
+        uint4* db = reinterpret_cast<uint4*>(dst + dcol + cb * 32);
+        const float4* cs = cs_row + (ca & 3) * 16;  // (cos, sin) pairs of i = (ca&3)*32 ..
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          uint32_t wa[4], wb[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int i = u * 8 + 2 * e;
+            float x1a = __uint_as_float(ra[i]) * rscale, x1b = __uint_as_float(ra[i + 1]) * rscale;
+            float x2a = __uint_as_float(rb[i]) * rscale, x2b = __uint_as_float(rb[i + 1]) * rscale;
+            if (rope) {
+              const float4 t = cs[i >> 1];  // (cos_i, sin_i, cos_i+1, sin_i+1)
+              const float y1a = x1a * t.x - x2a * t.y, y2a = x2a * t.x + x1a * t.y;
+              const float y1b = x1b * t.z - x2b * t.w, y2b = x2b * t.z + x1b * t.w;
+              x1a = y1a;
+              x2a = y2a;
+              x1b = y1b;
+              x2b = y2b;
+            }
+            wa[e] = pack_bf16x2(x1a, x1b);
+            wb[e] = pack_bf16x2(x2a, x2b);
+          }
+          da[u] = make_uint4(wa[0], wa[1], wa[2], wa[3]);
+          db[u] = make_uint4(wb[0], wb[1], wb[2], wb[3]);
+        }
+      }
+    }
+    return 0.f;
+  }
+  float ssq = 0.f;
+#pragma unroll 1
+  for (int c = 0; c < BN / 32; ++c) {
+    uint32_t r[32];
+    tmem_ld32(tbase + c * 32, r);
+    tmem_wait_ld();
+    if (EPI == EpiStore) {
+      if (live) {
+        const int col = n0 + c * 32;
+        float v[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]) * rscale;
+        if (p.residual) {
+          const uint4* rp = reinterpret_cast<const uint4*>(p.residual + grow * p.ldr + col);
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const uint4 t = rp[u];
+            const uint32_t w[4] = {t.x, t.y, t.z, t.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float2 f = unpack_bf16x2(w[e]);
+              v[u * 8 + 2 * e] += f.x;
+              v[u * 8 + 2 * e + 1] += f.y;
+            }
+          }
+        }
+        uint4* cp = reinterpret_cast<uint4*>(p.c + grow * p.ldc + col);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          uint32_t w[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            w[e] = pack_bf16x2(v[u * 8 + 2 * e], v[u * 8 + 2 * e + 1]);
+            if (p.row_ssq_out) {  // sums of squares of the values as stored (bf16)
+              const float2 f = unpack_bf16x2(w[e]);
+              ssq = fmaf(f.x, f.x, ssq);
+              ssq = fmaf(f.y, f.y, ssq);
+            }
+          }
+          cp[u] = make_uint4(w[0], w[1], w[2], w[3]);
+        }
+        if (p.row_ssq_out && (c & 3) == 3) {
+          p.row_ssq_out[grow * p.ld_ssq_out + (n0 + c * 32) / 128] = ssq;
+          ssq = 0.f;
+        }
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        const float u = __uint_as_float(r[i]) * rscale;
+        score = fmaf(w2s[c * 32 + i], u / (1.0f + __expf(-u)), score);
+      }
+    }
+  }
+  return score;
+}
+
 template <int BN, int STAGES, int EPI>
 __global__ void __launch_bounds__(192, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
@@ -84,11 +232,12 @@ __global__ void __launch_bounds__(192, 1)
   const int64_t m0 = (int64_t)blockIdx.x * Cfg::BM;
   const int n0 = blockIdx.y * BN;
   const int nk = p.K / Cfg::BK;
+  const bool norm_here = p.rmsnorm && !p.row_ssq_in;  // epilogue warps consume A stages
 
   if (tid == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 1 + (p.rmsnorm ? 4 : 0));
+      mbar_init(&empty[s], 1 + (norm_here ? 4 : 0));
     }
     mbar_init(acc_full, 1);
     mbar_init(drain, 1);
@@ -155,7 +304,7 @@ __global__ void __launch_bounds__(192, 1)
     const int row = q * 32 + lane;
     const int64_t grow = m0 + row;
     float ss = 0.f;
-    if (p.rmsnorm) {
+    if (norm_here) {
       for (int kb = 0; kb < nk; ++kb) {
         const int s = kb % STAGES;
         const uint32_t ph = (uint32_t)(kb / STAGES) & 1u;
@@ -178,113 +327,16 @@ __global__ void __launch_bounds__(192, 1)
         if (lane == 0) mbar_arrive(&empty[s]);
       }
     }
-    const float rscale = p.rmsnorm ? rsqrtf(ss / (float)p.K + p.eps) : 1.0f;
+    float rscale = 1.0f;
+    if (p.rmsnorm) {
+      if (p.row_ssq_in) rscale = grow < p.M ? rscale_from_ssq(p, grow) : 1.0f;
+      else rscale = rsqrtf(ss / (float)p.K + p.eps);
+    }
     const bool ok = warp_all(mbar_wait(acc_full, 0, abort_flag, p.status));
     tc_fence_after();
     if (ok) {
       const uint32_t tbase = tmem + ((uint32_t)(q * 32) << 16);
-      float score = 0.f;
-      if (EPI == EpiQKV) {
-        // destination of this tile: Q, K or V (tiles never straddle the boundaries)
-        uint16_t* dst;
-        int dcol;
-        if (n0 < p.q_cols) {
-          dst = p.c + grow * p.ldc;
-          dcol = n0;
-        } else if (n0 < p.q_cols + p.k_cols) {
-          dst = p.k_out + grow * p.ld_kv;
-          dcol = n0 - p.q_cols;
-        } else {
-          dst = p.v_out + grow * p.ld_kv;
-          dcol = n0 - p.q_cols - p.k_cols;
-        }
-        const bool rope = n0 < p.q_cols + p.k_cols;
-        int pos = (rope && grow < p.M) ? p.pos[grow] : 0;
-        if (pos < 0 || pos >= p.max_pos) {
-          if (grow < p.M && p.status) atomicOr(p.status, TG_STATUS_BOUNDS);
-          pos = 0;
-        }
-        const float4* cs_row = reinterpret_cast<const float4*>(p.cos_sin + (int64_t)pos * 128);
-#pragma unroll 1
-        for (int pr = 0; pr < BN / 64; ++pr) {
-          // chunk pairs (0,2), (1,3), (4,6), (5,7): columns i and i + 64 of one head
-          const int ca = (pr & 1) + 4 * (pr >> 1), cb = ca + 2;
-          uint32_t ra[32], rb[32];
-          tmem_ld32(tbase + ca * 32, ra);
-          tmem_ld32(tbase + cb * 32, rb);
-          tmem_wait_ld();
-          if (grow < p.M) {
-            uint4* da = reinterpret_cast<uint4*>(dst + dcol + ca * 32);
-            uint4* db = reinterpret_cast<uint4*>(dst + dcol + cb * 32);
-            const float4* cs = cs_row + (ca & 3) * 16;  // (cos, sin) pairs of i = (ca&3)*32 ..
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-              uint32_t wa[4], wb[4];
-#pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                const int i = u * 8 + 2 * e;
-                float x1a = __uint_as_float(ra[i]) * rscale, x1b = __uint_as_float(ra[i + 1]) * rscale;
-                float x2a = __uint_as_float(rb[i]) * rscale, x2b = __uint_as_float(rb[i + 1]) * rscale;
-                if (rope) {
-                  const float4 t = cs[i >> 1];  // (cos_i, sin_i, cos_i+1, sin_i+1)
-                  const float y1a = x1a * t.x - x2a * t.y, y2a = x2a * t.x + x1a * t.y;
-                  const float y1b = x1b * t.z - x2b * t.w, y2b = x2b * t.z + x1b * t.w;
-                  x1a = y1a; x2a = y2a; x1b = y1b; x2b = y2b;
-                }
-                wa[e] = pack_bf16x2(x1a, x1b);
-                wb[e] = pack_bf16x2(x2a, x2b);
-              }
-              da[u] = make_uint4(wa[0], wa[1], wa[2], wa[3]);
-              db[u] = make_uint4(wb[0], wb[1], wb[2], wb[3]);
-            }
-          }
-        }
-      } else {
-#pragma unroll 1
-      for (int c = 0; c < BN / 32; ++c) {
-        uint32_t r[32];
-        tmem_ld32(tbase + c * 32, r);
-        tmem_wait_ld();
-        if (EPI == EpiStore) {
-          if (grow < p.M) {
-            const int col = n0 + c * 32;
-            float v[32];
-#pragma unroll
-            for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]) * rscale;
-            if (p.residual) {
-              const uint4* rp = reinterpret_cast<const uint4*>(p.residual + grow * p.ldr + col);
-#pragma unroll
-              for (int u = 0; u < 4; ++u) {
-                const uint4 t = rp[u];
-                const uint32_t w[4] = {t.x, t.y, t.z, t.w};
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                  const float2 f = unpack_bf16x2(w[e]);
-                  v[u * 8 + 2 * e] += f.x;
-                  v[u * 8 + 2 * e + 1] += f.y;
-                }
-              }
-            }
-            uint4* cp = reinterpret_cast<uint4*>(p.c + grow * p.ldc + col);
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-              uint4 t;
-              t.x = pack_bf16x2(v[u * 8 + 0], v[u * 8 + 1]);
-              t.y = pack_bf16x2(v[u * 8 + 2], v[u * 8 + 3]);
-              t.z = pack_bf16x2(v[u * 8 + 4], v[u * 8 + 5]);
-              t.w = pack_bf16x2(v[u * 8 + 6], v[u * 8 + 7]);
-              cp[u] = t;
-            }
-          }
-        } else {
-#pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const float u = __uint_as_float(r[i]) * rscale;
-            score = fmaf(w2s[c * 32 + i], u / (1.0f + __expf(-u)), score);
-          }
-        }
-      }
-      }
+      const float score = epilogue_row<BN, EPI>(p, tbase, grow, n0, rscale, w2s);
       if (EPI == EpiScore) {
         if (grow < p.M) p.s_out[grow] = score;
         float sq = grow < p.M ? score * score : 0.f;
@@ -299,6 +351,138 @@ __global__ void __launch_bounds__(192, 1)
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, BN);
+  }
+}
+
+// ------------------------------------------------------------------ CTA-pair kernel
+
+template <int STAGES>
+struct PairCfg {
+  static constexpr int BM = 128, BN = 256, BK = 64;   // per CTA: 128 rows of A, 128 of W
+  static constexpr int A_BYTES = BM * BK * 2;
+  static constexpr int B_BYTES = (BN / 2) * BK * 2;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int TILE_BYTES = STAGES * STAGE_BYTES;
+  static constexpr int BAR_BYTES = 512;
+  static constexpr int SMEM = 1024 + TILE_BYTES + BAR_BYTES;
+  static constexpr int THREADS = 192;
+};
+
+template <int STAGES, int EPI>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
+    gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
+                     const __grid_constant__ CUtensorMap tmB, GemmParams p) {
+  using Cfg = PairCfg<STAGES>;
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  unsigned char* smem = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  unsigned char* tiles = smem;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + Cfg::TILE_BYTES);  // even CTA: both landed
+  uint64_t* empty = full + STAGES;     // stage free in this CTA (MMA done with it)
+  uint64_t* acc_full = empty + STAGES;
+  uint64_t* drain = acc_full + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const uint32_t rank = cluster_ctarank();
+  const int64_t m0 = (int64_t)(blockIdx.x >> 1) * 256 + rank * 128;
+  const int n0 = blockIdx.y * Cfg::BN;
+  const int nk = p.K / Cfg::BK;
+
+  if (tid == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(acc_full, 1);
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(tmem_slot, Cfg::BN);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  cluster_sync_all();  // barriers of both CTAs initialised before any remote arrive
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // The odd CTA's bytes may reach the even CTA's barrier before the even CTA's
+      // expect_tx: the phase cannot complete early, as it still waits for that arrive.
+      // A stage is reloaded only after the even CTA's commit freed it, which follows
+      // the completion of that barrier's previous phase.
+      const uint32_t full_lead0 = mapa_shared(smem_u32(&full[0]), 0);
+      int issued = 0;
+      for (int kb = 0; kb < nk; ++kb) {
+        const int s = kb % STAGES;
+        const uint32_t ph = (uint32_t)(kb / STAGES) & 1u;
+        if (!mbar_wait(&empty[s], ph ^ 1u, abort_flag, p.status)) break;
+        unsigned char* a_s = tiles + s * Cfg::STAGE_BYTES;
+        if (rank == 0) mbar_arrive_expect_tx(&full[s], 2 * Cfg::STAGE_BYTES);
+        tma_load_2d_pair(a_s, &tmA, kb * Cfg::BK, (int32_t)m0, full_lead0 + s * 8);
+        tma_load_2d_pair(a_s + Cfg::A_BYTES, &tmB, kb * Cfg::BK,
+                         n0 + (int)rank * (Cfg::BN / 2), full_lead0 + s * 8);
+        ++issued;
+      }
+      // The even CTA waits until the last stages' bytes (both CTAs') have landed; the odd
+      // CTA is held by the closing cluster barrier until then.
+      if (rank == 0)
+        for (int kb = issued - STAGES < 0 ? 0 : issued - STAGES; kb < issued; ++kb)
+          mbar_wait(&full[kb % STAGES], (uint32_t)(kb / STAGES) & 1u, nullptr, p.status);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      if (rank == 0) {
+        constexpr uint32_t idesc = idesc_bf16_f32(256, Cfg::BN, false, false);
+        const uint32_t empty_peer0 = mapa_shared(smem_u32(&empty[0]), 1);
+        const uint32_t acc_peer = mapa_shared(smem_u32(acc_full), 1);
+        for (int kb = 0; kb < nk; ++kb) {
+          const int s = kb % STAGES;
+          const uint32_t ph = (uint32_t)(kb / STAGES) & 1u;
+          if (!mbar_wait(&full[s], ph, abort_flag, p.status)) break;
+          tc_fence_after();
+          const uint32_t a_addr = smem_u32(tiles + s * Cfg::STAGE_BYTES);
+          const uint32_t b_addr = a_addr + Cfg::A_BYTES;
+#pragma unroll
+          for (int k = 0; k < Cfg::BK / 16; ++k)
+            mma_ss_pair(tmem, sw128_desc(a_addr + k * 32, 16, 1024),
+                        sw128_desc(b_addr + k * 32, 16, 1024), idesc, (kb | k) != 0);
+          mma_commit_pair(smem_u32(&empty[s]));
+          mma_commit_pair(empty_peer0 + s * 8);
+        }
+        mma_commit_pair(smem_u32(acc_full));
+        mma_commit_pair(acc_peer);
+        mma_commit_pair(smem_u32(drain));
+        mbar_wait(drain, 0, nullptr, p.status);  // all MMAs (and their arrives) done
+      }
+    }
+  } else {
+    const int q = warp & 3;
+    const int row = q * 32 + lane;
+    const int64_t grow = m0 + row;
+    float rscale = 1.0f;
+    if (p.rmsnorm && p.row_ssq_in && grow < p.M) rscale = rscale_from_ssq(p, grow);
+    const bool ok = warp_all(mbar_wait(acc_full, 0, abort_flag, p.status));
+    tc_fence_after();
+    if (ok) {
+      const uint32_t tbase = tmem + ((uint32_t)(q * 32) << 16);
+      epilogue_row<Cfg::BN, EPI>(p, tbase, grow, n0, rscale, nullptr);
+    }
+    tc_fence_before();
+  }
+  __syncthreads();
+  cluster_sync_all();  // no CTA leaves while the pair's MMAs or arrives may touch it
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem, Cfg::BN);
   }
 }
 

@@ -22,6 +22,23 @@ int launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const GemmParams& 
   return check_launch();
 }
 
+template <int STAGES, int EPI>
+int launch_pair(const CUtensorMap& ta, const CUtensorMap& tb, const GemmParams& p,
+                cudaStream_t stream) {
+  using Cfg = PairCfg<STAGES>;
+  static int attr_dev = -1;
+  int dev = 0;
+  TG_CUDA_TRY(cudaGetDevice(&dev));
+  if (attr_dev != dev) {
+    TG_CUDA_TRY(cudaFuncSetAttribute(gemm_pair_kernel<STAGES, EPI>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM));
+    attr_dev = dev;
+  }
+  dim3 grid((unsigned)(2 * ((p.M + 255) / 256)), (unsigned)(p.N / Cfg::BN));
+  gemm_pair_kernel<STAGES, EPI><<<grid, Cfg::THREADS, Cfg::SMEM, stream>>>(ta, tb, p);
+  return check_launch();
+}
+
 // Explicit instantiations used by the entry points.
 template int launch_gemm<256, 4, EpiStore>(const CUtensorMap&, const CUtensorMap&,
                                            const GemmParams&, cudaStream_t);
@@ -55,8 +72,8 @@ using namespace tg;
 
 extern "C" int tg_linear(const tg_bf16* a, int64_t lda, const tg_bf16* w, int64_t ldw, tg_bf16* c,
                          int64_t ldc, int64_t M, int N, int K, int rmsnorm_a, float eps,
-                         const tg_bf16* residual, int64_t ld_res, uint32_t* status,
-                         tg_stream_t stream) {
+                         const tg_bf16* residual, int64_t ld_res, float* row_ssq_out,
+                         int64_t ld_ssq_out, uint32_t* status, tg_stream_t stream) {
   if (M < 0 || N <= 0 || K <= 0 || (N % 128) || (K % 64)) return TG_ERR_UNSUPPORTED_SHAPE;
   if (M == 0) return TG_OK;
   if (!a || !w || !c) return TG_ERR_INVALID_ARGUMENT;
@@ -66,9 +83,12 @@ extern "C" int tg_linear(const tg_bf16* a, int64_t lda, const tg_bf16* w, int64_
       (residual && !stride_ok(ld_res, 2)))
     return TG_ERR_MISALIGNED;
   if (rmsnorm_a && !(eps >= 0.f)) return TG_ERR_INVALID_ARGUMENT;
+  if (row_ssq_out && ld_ssq_out < N / 128) return TG_ERR_INVALID_ARGUMENT;
   TG_TRY(check_device());
 
-  const int bn = pick_bn(M, N);
+  // CTA-pair kernel for 256-column tiles without an in-kernel norm; else one CTA per tile
+  const bool pair = !rmsnorm_a && (N % 256) == 0;
+  const int bn = pair ? 128 : pick_bn(M, N);
 
   CUtensorMap ta, tb;
   TG_TRY(make_tmap_bf16_2d(&ta, a, (uint64_t)M, (uint64_t)K, (uint64_t)lda, 64, 128));
@@ -83,7 +103,10 @@ extern "C" int tg_linear(const tg_bf16* a, int64_t lda, const tg_bf16* w, int64_
   p.ldc = ldc;
   p.residual = reinterpret_cast<const uint16_t*>(residual);
   p.ldr = ld_res;
+  p.row_ssq_out = row_ssq_out;
+  p.ld_ssq_out = ld_ssq_out;
   p.status = status;
+  if (pair) return launch_pair<6, EpiStore>(ta, tb, p, (cudaStream_t)stream);
   if (bn == 256) return launch_gemm<256, 4, EpiStore>(ta, tb, p, (cudaStream_t)stream);
   return launch_gemm<128, 3, EpiStore>(ta, tb, p, (cudaStream_t)stream);
 }
@@ -93,7 +116,8 @@ extern "C" int tg_qkv_rope_cache(const tg_bf16* x, int64_t ld_x, const tg_bf16* 
                                  int head_dim, float eps, const int32_t* pos,
                                  const float* cos_sin, int max_pos, tg_bf16* q_out, int64_t ld_q,
                                  tg_bf16* cache_k, tg_bf16* cache_v, int64_t ld_cache,
-                                 int64_t slot_offset, uint32_t* status, tg_stream_t stream) {
+                                 int64_t slot_offset, const float* row_ssq_in,
+                                 int64_t ld_ssq_in, uint32_t* status, tg_stream_t stream) {
   if (head_dim != 128 || n_q_heads <= 0 || n_kv_heads <= 0 || hidden <= 0 || (hidden % 64))
     return TG_ERR_UNSUPPORTED_SHAPE;
   if (M < 0 || slot_offset < 0 || max_pos <= 0) return TG_ERR_INVALID_ARGUMENT;
@@ -109,10 +133,14 @@ extern "C" int tg_qkv_rope_cache(const tg_bf16* x, int64_t ld_x, const tg_bf16* 
       !stride_ok(ld_q, 2) || !stride_ok(ld_cache, 2))
     return TG_ERR_MISALIGNED;
   if (!(eps >= 0.f)) return TG_ERR_INVALID_ARGUMENT;
+  if (row_ssq_in && (ld_ssq_in < hidden / 128 || (hidden % 128))) return TG_ERR_INVALID_ARGUMENT;
   TG_TRY(check_device());
-  // BN=256 only when the Q/K/V boundaries fall on 256-column tile edges
-  int bn = pick_bn(M, N);
-  if (bn == 256 && ((q_cols % 256) || (kv_cols % 256))) bn = 128;
+  // 256-column tiles only when the Q/K/V boundaries fall on their edges; the CTA-pair
+  // kernel when the row norms come precomputed
+  const bool aligned256 = (q_cols % 256) == 0 && (kv_cols % 256) == 0;
+  const bool pair = row_ssq_in && aligned256;
+  int bn = pair ? 128 : pick_bn(M, N);
+  if (!pair && bn == 256 && !aligned256) bn = 128;
   CUtensorMap ta, tb;
   TG_TRY(make_tmap_bf16_2d(&ta, x, (uint64_t)M, (uint64_t)hidden, (uint64_t)ld_x, 64, 128));
   TG_TRY(make_tmap_bf16_2d(&tb, w_qkv, (uint64_t)N, (uint64_t)hidden, (uint64_t)ld_w, 64, bn));
@@ -132,7 +160,10 @@ extern "C" int tg_qkv_rope_cache(const tg_bf16* x, int64_t ld_x, const tg_bf16* 
   p.k_out = reinterpret_cast<uint16_t*>(cache_k) + slot_offset * ld_cache;
   p.v_out = reinterpret_cast<uint16_t*>(cache_v) + slot_offset * ld_cache;
   p.ld_kv = ld_cache;
+  p.row_ssq_in = row_ssq_in;
+  p.ld_ssq_in = ld_ssq_in;
   p.status = status;
+  if (pair) return launch_pair<6, EpiQKV>(ta, tb, p, (cudaStream_t)stream);
   if (bn == 256) return launch_gemm<256, 4, EpiQKV>(ta, tb, p, (cudaStream_t)stream);
   return launch_gemm<128, 3, EpiQKV>(ta, tb, p, (cudaStream_t)stream);
 }

@@ -76,8 +76,10 @@ def test_host_side_argument_errors(lib):
     assert lib.tg_gated_attention(p, 2048, p, 1024, p, 1024, p, cu, 1, 3, 3, 128, p, p, p,
                                   1.0, p, 2048, None, None, 0, None, None) == -6
     # projections: N not a multiple of 128, K not a multiple of 64
-    assert lib.tg_linear(p, 64, p, 64, p, 100, 4, 100, 64, 0, 0.0, None, 0, None, None) == -6
-    assert lib.tg_linear(p, 96, p, 96, p, 128, 4, 128, 96, 0, 0.0, None, 0, None, None) == -6
+    assert lib.tg_linear(p, 64, p, 64, p, 100, 4, 100, 64, 0, 0.0, None, 0, None, 0, None,
+                         None) == -6
+    assert lib.tg_linear(p, 96, p, 96, p, 128, 4, 128, 96, 0, 0.0, None, 0, None, 0, None,
+                         None) == -6
     # scorer: width other than 256
     assert lib.tg_gate_score(p, 2048, 8, 2048, None, p, 128, p, 1e-6, p, cu, 1, 1e-6, p, p,
                              p, p, p, 1 << 20, None, None) == -6
@@ -86,7 +88,7 @@ def test_host_side_argument_errors(lib):
     assert lib.tg_topk_compact(p, p, p, cu, p, ck, 1, p, p, p, None, None) == -1
     # gather: misaligned pointer
     assert lib.tg_gather_rope(C.c_void_p(0x10002), 64, 4, None, 4, 64, None, 0, 0, 128, None,
-                              0, p, 64, None, None) == -2
+                              0, p, 64, None, 0, None, None) == -2
     # KV cache: slots beyond the cache
     assert lib.tg_kv_compact(p, 64, p, 64, 10, None, 10, 64, p, p, 64, 12, 5, None, None) == -1
     # workspace too small

@@ -258,10 +258,14 @@ def test_gate_score_deterministic(tg):
 
 # ------------------------------------------------------------------ projections
 
+# shapes with N % 256 == 0 and no folded norm run on CTA pairs (256 x 256 tiles)
 @pytest.mark.parametrize("M,N,K,rms,res", [(1, 128, 64, False, False), (100, 256, 2048, True, False),
                                            (1638, 4096, 2048, True, False),
                                            (1638, 2048, 2048, False, True),
-                                           (300, 384, 192, True, True)])
+                                           (300, 384, 192, True, True),
+                                           (1, 256, 64, False, False),
+                                           (257, 512, 1024, False, True),
+                                           (1638, 4096, 2048, False, False)])
 def test_linear_against_oracle(tg, M, N, K, rms, res):
     a = S.uniform_rows(M, K, seed=M + 1)
     w = S.uniform_rows(N, K, seed=N + 2, scale=0.02)
@@ -272,6 +276,18 @@ def test_linear_against_oracle(tg, M, N, K, rms, res):
     got = _f64(c.cpu())
     err = np.abs(got - want)
     assert np.all(err <= 2.0 ** -7 * np.abs(want) + 2e-3), err.max()
+
+
+@pytest.mark.parametrize("N", [384, 2048])
+def test_linear_row_sums_of_squares(tg, N):
+    M, K = 333, 512
+    a = _dev(S.uniform_rows(M, K, seed=6))
+    w = _dev(S.uniform_rows(N, K, seed=7, scale=0.05))
+    r = _dev(S.uniform_rows(M, N, seed=8))
+    ssq = torch.full((M, N // 128), float("nan"), device="cuda")
+    c = tg.tg_linear(a, w, residual=r, row_ssq=ssq)
+    want = (c.double() ** 2).view(M, N // 128, 128).sum(-1)
+    assert torch.allclose(ssq.double(), want, rtol=1e-5, atol=1e-5)
 
 
 def test_linear_residual_in_place(tg):
@@ -434,6 +450,38 @@ def test_qkv_rope_cache_against_oracle(tg, M):
         err = np.abs(_f64(got.cpu()) - want)
         assert np.all(err <= 2.0 ** -7 * np.abs(want) + 2e-3), err.max()
     assert torch.count_nonzero(ck[:slot]) == 0 and torch.count_nonzero(cv[:slot]) == 0
+
+
+@pytest.mark.parametrize("M", [1, 1638])
+def test_qkv_rope_cache_with_row_sums_against_oracle(tg, M):
+    """Precomputed row sums of squares select the CTA-pair kernel."""
+    Hq, Hkv, d, H = 16, 8, 128, 2048
+    x = S.uniform_rows(M, H, seed=M + 40)
+    w = S.uniform_rows((Hq + 2 * Hkv) * d, H, seed=M + 41, scale=0.02)
+    pos = torch.arange(0, 5 * M, 5, dtype=torch.int32)
+    cs = tg.tg_rope_table(5 * M + 1, d, 1.0e6)
+    ssq = torch.from_numpy((_f64(x) ** 2).reshape(M, H // 128, 128).sum(-1)).float()
+    ck = torch.zeros((M, Hkv * d), dtype=torch.bfloat16, device="cuda")
+    cv = torch.zeros_like(ck)
+    q = tg.tg_qkv_rope_cache(_dev(x), _dev(w), _dev(pos), cs, ck, cv, Hq, Hkv, row_ssq=_dev(ssq))
+    a = O.rmsnorm_rows(x)
+    qkv = a @ _f64(w).T
+    want_q = O.rope(qkv[:, :Hq * d].reshape(M, Hq, d), pos, 1.0e6).reshape(M, -1)
+    want_k = O.rope(qkv[:, Hq * d:(Hq + Hkv) * d].reshape(M, Hkv, d), pos, 1.0e6).reshape(M, -1)
+    want_v = qkv[:, (Hq + Hkv) * d:]
+    for got, want in ((q, want_q), (ck, want_k), (cv, want_v)):
+        err = np.abs(_f64(got.cpu()) - want)
+        assert np.all(err <= 2.0 ** -7 * np.abs(want) + 2e-3), err.max()
+
+
+def test_gather_row_sums_of_squares(tg):
+    src = _dev(S.uniform_rows(500, 2048, seed=12))
+    idx = _dev(torch.randint(0, 500, (321,), generator=torch.Generator().manual_seed(3),
+                             dtype=torch.int32))
+    ssq = torch.full((321, 16), float("nan"), device="cuda")
+    out = tg.tg_gather_rope(src, row_idx=idx, row_ssq=ssq)
+    want = (out.double() ** 2).view(321, 16, 128).sum(-1)
+    assert torch.allclose(ssq.double(), want, rtol=1e-5, atol=1e-5)
 
 
 def test_qkv_rope_cache_matches_unfused_path(tg):
