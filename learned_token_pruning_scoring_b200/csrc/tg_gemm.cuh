@@ -356,6 +356,13 @@ __global__ void __launch_bounds__(192, 1)
 
 // ------------------------------------------------------------------ CTA-pair kernel
 
+// Tensor maps of the CTA-pair kernel (boxes of 64 columns x 128 rows, 128-byte swizzle).
+struct PairMaps {
+  CUtensorMap a, b;    // operands A [M, K] and W [N, K]
+  CUtensorMap out[3];  // EpiStore: out[0] = C [M, N]; EpiQKV: Q [M, q_cols], K rows, V rows
+  CUtensorMap res;     // EpiStore with a residual: R [M, N]
+};
+
 template <int STAGES>
 struct PairCfg {
   static constexpr int BM = 128, BN = 256, BK = 64;   // per CTA: 128 rows of A, 128 of W
@@ -363,49 +370,180 @@ struct PairCfg {
   static constexpr int B_BYTES = (BN / 2) * BK * 2;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int TILE_BYTES = STAGES * STAGE_BYTES;
-  static constexpr int BAR_BYTES = 512;
-  static constexpr int SMEM = 1024 + TILE_BYTES + BAR_BYTES;
+  static constexpr int BOX_BYTES = BM * 64 * 2;        // one 64-column box of the output tile
+  static constexpr int OUT_BYTES = 4 * BOX_BYTES;      // staging of one 128 x 256 output tile
+  static constexpr int BAR_BYTES = 256;
+  static constexpr int SMEM = 1024 + TILE_BYTES + OUT_BYTES + BAR_BYTES;
   static constexpr int THREADS = 192;
+  static constexpr int TMEM_COLS = 2 * BN;             // two accumulators (double buffer)
 };
 
+// Byte offset of 16-byte chunk k (columns 8k .. 8k + 7) of row r inside a box of 64 bf16
+// columns stored with the 128-byte swizzle: the chunk index is XOR-ed with r mod 8.
+__device__ __forceinline__ uint32_t sw128_chunk(int r, int k) {
+  return (uint32_t)(r * 128 + ((k ^ (r & 7)) << 4));
+}
+
+// One 256 x 256 output tile of the pair (each CTA: 128 rows, staged in shared memory as
+// four swizzled boxes); `row` is the thread's row in the CTA's half, `tacc` the TMEM
+// address of the row's accumulator (lane quarter and buffer included).
+template <int EPI>
+__device__ __forceinline__ void pair_epilogue_tile(const GemmParams& p, unsigned char* out_s,
+                                                   uint32_t tacc, int row, int64_t grow, int n0,
+                                                   bool has_res) {
+  const bool live = grow < p.M;
+  const float rscale =
+      (p.rmsnorm && p.row_ssq_in && live) ? rscale_from_ssq(p, grow) : 1.0f;
+  if (EPI == EpiQKV) {
+    const bool rope = n0 < p.q_cols + p.k_cols;
+    int pos = (rope && live) ? p.pos[grow] : 0;
+    if (pos < 0 || pos >= p.max_pos) {
+      if (live && p.status) atomicOr(p.status, TG_STATUS_BOUNDS);
+      pos = 0;
+    }
+    const float4* cs_row = reinterpret_cast<const float4*>(p.cos_sin + (int64_t)pos * 128);
+#pragma unroll 1
+    for (int pr = 0; pr < 4; ++pr) {
+      // 32-column pieces ca and ca + 2 hold columns i and i + 64 of one 128-column head
+      const int ca = (pr & 1) + 4 * (pr >> 1), cb = ca + 2;
+      uint32_t ra[32], rb[32];
+      tmem_ld32(tacc + ca * 32, ra);
+      tmem_ld32(tacc + cb * 32, rb);
+      tmem_wait_ld();
+      unsigned char* box_a = out_s + (ca >> 1) * PairCfg<1>::BOX_BYTES;
+      unsigned char* box_b = out_s + (cb >> 1) * PairCfg<1>::BOX_BYTES;
+      const float4* cs = cs_row + (ca & 3) * 16;  // (cos, sin) pairs of i = (ca & 3) * 32 ..
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        uint32_t wa[4], wb[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int i = u * 8 + 2 * e;
+          float x1a = __uint_as_float(ra[i]) * rscale, x1b = __uint_as_float(ra[i + 1]) * rscale;
+          float x2a = __uint_as_float(rb[i]) * rscale, x2b = __uint_as_float(rb[i + 1]) * rscale;
+          if (rope) {
+            const float4 t = cs[i >> 1];  // (cos_i, sin_i, cos_i+1, sin_i+1)
+            const float y1a = x1a * t.x - x2a * t.y, y2a = x2a * t.x + x1a * t.y;
+            const float y1b = x1b * t.z - x2b * t.w, y2b = x2b * t.z + x1b * t.w;
+            x1a = y1a;
+            x2a = y2a;
+            x1b = y1b;
+            x2b = y2b;
+          }
+          wa[e] = pack_bf16x2(x1a, x1b);
+          wb[e] = pack_bf16x2(x2a, x2b);
+        }
+        const int k = (ca & 1) * 4 + u;  // chunk of the piece within its box
+        *reinterpret_cast<uint4*>(box_a + sw128_chunk(row, k)) =
+            make_uint4(wa[0], wa[1], wa[2], wa[3]);
+        *reinterpret_cast<uint4*>(box_b + sw128_chunk(row, k)) =
+            make_uint4(wb[0], wb[1], wb[2], wb[3]);
+      }
+    }
+    return;
+  }
+  float ssq = 0.f;
+#pragma unroll 1
+  for (int j = 0; j < 4; ++j) {  // box j: tile columns 64 j .. 64 j + 63
+    uint32_t ra[32], rb[32];
+    tmem_ld32(tacc + j * 64, ra);
+    tmem_ld32(tacc + j * 64 + 32, rb);
+    tmem_wait_ld();
+    unsigned char* box = out_s + j * PairCfg<1>::BOX_BYTES;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      uint4* cp = reinterpret_cast<uint4*>(box + sw128_chunk(row, k));
+      float v[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e)
+        v[e] = __uint_as_float(k < 4 ? ra[8 * k + e] : rb[8 * (k - 4) + e]) * rscale;
+      if (has_res) {
+        const uint4 t = *cp;
+        const uint32_t w[4] = {t.x, t.y, t.z, t.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 f = unpack_bf16x2(w[e]);
+          v[2 * e] += f.x;
+          v[2 * e + 1] += f.y;
+        }
+      }
+      uint32_t w[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        w[e] = pack_bf16x2(v[2 * e], v[2 * e + 1]);
+        if (p.row_ssq_out) {  // sums of squares of the values as stored (bf16)
+          const float2 f = unpack_bf16x2(w[e]);
+          ssq = fmaf(f.x, f.x, ssq);
+          ssq = fmaf(f.y, f.y, ssq);
+        }
+      }
+      *cp = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+    if (p.row_ssq_out && (j & 1)) {
+      if (live) p.row_ssq_out[grow * p.ld_ssq_out + n0 / 128 + (j >> 1)] = ssq;
+      ssq = 0.f;
+    }
+  }
+}
+
+// Persistent CTA-pair GEMM: each cluster of two CTAs walks the 256 x 256 output tiles
+// t = cluster, cluster + clusters, ...  Roles per CTA:
+//   warp 0     one thread streams A and W k-blocks of every tile through the ring;
+//   warp 1     TMEM owner; in the even CTA one thread issues the M=256 MMAs into
+//              accumulator buffer (tile index & 1);
+//   warps 2-5  epilogue of the previous tile while the next one accumulates: TMEM ->
+//              registers -> bf16 in a swizzled staging tile -> TMA stores.  For EpiStore
+//              with a residual, the staging tile is first filled with the residual rows
+//              by a TMA load issued one tile ahead.
+// Barriers: full/empty per ring stage (full lives in the even CTA and counts both CTAs'
+// bytes); acc_full[b] (the even CTA's commit, in both CTAs); acc_empty[b] (even CTA,
+// one arrive per CTA once its epilogue has read buffer b); res_full (this CTA).
 template <int STAGES, int EPI>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
-    gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
-                     const __grid_constant__ CUtensorMap tmB, GemmParams p) {
+    gemm_pair_kernel(const __grid_constant__ PairMaps maps, GemmParams p) {
   using Cfg = PairCfg<STAGES>;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   unsigned char* tiles = smem;
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + Cfg::TILE_BYTES);  // even CTA: both landed
-  uint64_t* empty = full + STAGES;     // stage free in this CTA (MMA done with it)
-  uint64_t* acc_full = empty + STAGES;
-  uint64_t* drain = acc_full + 1;
+  unsigned char* out_s = smem + Cfg::TILE_BYTES;
+  uint64_t* full = reinterpret_cast<uint64_t*>(out_s + Cfg::OUT_BYTES);
+  uint64_t* empty = full + STAGES;
+  uint64_t* acc_full = empty + STAGES;   // [2]
+  uint64_t* acc_empty = acc_full + 2;    // [2]
+  uint64_t* res_full = acc_empty + 2;
+  uint64_t* drain = res_full + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const uint32_t rank = cluster_ctarank();
-  const int64_t m0 = (int64_t)(blockIdx.x >> 1) * 256 + rank * 128;
-  const int n0 = blockIdx.y * Cfg::BN;
+  const int n_tiles_n = p.N / Cfg::BN;
+  const int n_tiles = (int)((p.M + 255) / 256) * n_tiles_n;
+  const int cluster = (int)(blockIdx.x >> 1), n_clusters = (int)(gridDim.x >> 1);
   const int nk = p.K / Cfg::BK;
+  const bool has_res = EPI == EpiStore && p.residual != nullptr;
 
   if (tid == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
-    mbar_init(acc_full, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_empty[b], 2);
+    }
+    mbar_init(res_full, 1);
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
   if (warp == 0 && lane == 0) {
-    tma_prefetch_desc(&tmA);
-    tma_prefetch_desc(&tmB);
+    tma_prefetch_desc(&maps.a);
+    tma_prefetch_desc(&maps.b);
   }
   if (warp == 1) {
-    tmem_alloc_pair(tmem_slot, Cfg::BN);
+    tmem_alloc_pair(tmem_slot, Cfg::TMEM_COLS);
     tmem_relinquish_pair();
   }
   tc_fence_before();
@@ -420,69 +558,140 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
       // A stage is reloaded only after the even CTA's commit freed it, which follows
       // the completion of that barrier's previous phase.
       const uint32_t full_lead0 = mapa_shared(smem_u32(&full[0]), 0);
-      int issued = 0;
-      for (int kb = 0; kb < nk; ++kb) {
-        const int s = kb % STAGES;
-        const uint32_t ph = (uint32_t)(kb / STAGES) & 1u;
-        if (!mbar_wait(&empty[s], ph ^ 1u, abort_flag, p.status)) break;
-        unsigned char* a_s = tiles + s * Cfg::STAGE_BYTES;
-        if (rank == 0) mbar_arrive_expect_tx(&full[s], 2 * Cfg::STAGE_BYTES);
-        tma_load_2d_pair(a_s, &tmA, kb * Cfg::BK, (int32_t)m0, full_lead0 + s * 8);
-        tma_load_2d_pair(a_s + Cfg::A_BYTES, &tmB, kb * Cfg::BK,
-                         n0 + (int)rank * (Cfg::BN / 2), full_lead0 + s * 8);
-        ++issued;
+      int kg = 0;
+      bool ok = true;
+      for (int t = cluster; ok && t < n_tiles; t += n_clusters) {
+        const int64_t m0 = (int64_t)(t / n_tiles_n) * 256 + rank * 128;
+        const int n0 = (t % n_tiles_n) * Cfg::BN + (int)rank * (Cfg::BN / 2);
+        for (int kb = 0; kb < nk; ++kb, ++kg) {
+          const int s = kg % STAGES;
+          const uint32_t ph = (uint32_t)(kg / STAGES) & 1u;
+          if (!mbar_wait(&empty[s], ph ^ 1u, abort_flag, p.status)) {
+            ok = false;
+            break;
+          }
+          unsigned char* a_s = tiles + s * Cfg::STAGE_BYTES;
+          if (rank == 0) mbar_arrive_expect_tx(&full[s], 2 * Cfg::STAGE_BYTES);
+          tma_load_2d_pair(a_s, &maps.a, kb * Cfg::BK, (int32_t)m0, full_lead0 + s * 8);
+          tma_load_2d_pair(a_s + Cfg::A_BYTES, &maps.b, kb * Cfg::BK, n0, full_lead0 + s * 8);
+        }
       }
       // The even CTA waits until the last stages' bytes (both CTAs') have landed; the odd
       // CTA is held by the closing cluster barrier until then.
       if (rank == 0)
-        for (int kb = issued - STAGES < 0 ? 0 : issued - STAGES; kb < issued; ++kb)
-          mbar_wait(&full[kb % STAGES], (uint32_t)(kb / STAGES) & 1u, nullptr, p.status);
+        for (int g = kg - STAGES < 0 ? 0 : kg - STAGES; g < kg; ++g)
+          mbar_wait(&full[g % STAGES], (uint32_t)(g / STAGES) & 1u, nullptr, p.status);
     }
   } else if (warp == 1) {
-    if (lane == 0) {
-      if (rank == 0) {
-        constexpr uint32_t idesc = idesc_bf16_f32(256, Cfg::BN, false, false);
-        const uint32_t empty_peer0 = mapa_shared(smem_u32(&empty[0]), 1);
-        const uint32_t acc_peer = mapa_shared(smem_u32(acc_full), 1);
-        for (int kb = 0; kb < nk; ++kb) {
-          const int s = kb % STAGES;
-          const uint32_t ph = (uint32_t)(kb / STAGES) & 1u;
-          if (!mbar_wait(&full[s], ph, abort_flag, p.status)) break;
+    if (lane == 0 && rank == 0) {
+      constexpr uint32_t idesc = idesc_bf16_f32(256, Cfg::BN, false, false);
+      const uint32_t empty_peer0 = mapa_shared(smem_u32(&empty[0]), 1);
+      const uint32_t acc_full_peer0 = mapa_shared(smem_u32(&acc_full[0]), 1);
+      int kg = 0, i = 0;
+      bool ok = true;
+      for (int t = cluster; ok && t < n_tiles; t += n_clusters, ++i) {
+        const int b = i & 1;
+        // both CTAs' epilogues are done with this buffer (first use passes at once)
+        if (!mbar_wait(&acc_empty[b], ((uint32_t)(i >> 1) & 1u) ^ 1u, abort_flag, p.status)) break;
+        tc_fence_after();
+        const uint32_t d = tmem + (uint32_t)(b * Cfg::BN);
+        for (int kb = 0; kb < nk; ++kb, ++kg) {
+          const int s = kg % STAGES;
+          const uint32_t ph = (uint32_t)(kg / STAGES) & 1u;
+          if (!mbar_wait(&full[s], ph, abort_flag, p.status)) {
+            ok = false;
+            break;
+          }
           tc_fence_after();
           const uint32_t a_addr = smem_u32(tiles + s * Cfg::STAGE_BYTES);
           const uint32_t b_addr = a_addr + Cfg::A_BYTES;
 #pragma unroll
           for (int k = 0; k < Cfg::BK / 16; ++k)
-            mma_ss_pair(tmem, sw128_desc(a_addr + k * 32, 16, 1024),
+            mma_ss_pair(d, sw128_desc(a_addr + k * 32, 16, 1024),
                         sw128_desc(b_addr + k * 32, 16, 1024), idesc, (kb | k) != 0);
           mma_commit_pair(smem_u32(&empty[s]));
           mma_commit_pair(empty_peer0 + s * 8);
         }
-        mma_commit_pair(smem_u32(acc_full));
-        mma_commit_pair(acc_peer);
-        mma_commit_pair(smem_u32(drain));
-        mbar_wait(drain, 0, nullptr, p.status);  // all MMAs (and their arrives) done
+        if (!ok) break;
+        mma_commit_pair(smem_u32(&acc_full[b]));
+        mma_commit_pair(acc_full_peer0 + b * 8);
       }
+      mma_commit_pair(smem_u32(drain));
+      mbar_wait(drain, 0, nullptr, p.status);  // all MMAs (and their arrives) done
     }
   } else {
-    const int q = warp & 3;
+    const int q = warp & 3;  // TMEM lane quarter this warp may access
     const int row = q * 32 + lane;
-    const int64_t grow = m0 + row;
-    float rscale = 1.0f;
-    if (p.rmsnorm && p.row_ssq_in && grow < p.M) rscale = rscale_from_ssq(p, grow);
-    const bool ok = warp_all(mbar_wait(acc_full, 0, abort_flag, p.status));
-    tc_fence_after();
-    if (ok) {
-      const uint32_t tbase = tmem + ((uint32_t)(q * 32) << 16);
-      epilogue_row<Cfg::BN, EPI>(p, tbase, grow, n0, rscale, nullptr);
+    const bool elected = warp == 2 && lane == 0;
+    const uint32_t acc_empty_lead0 = mapa_shared(smem_u32(&acc_empty[0]), 0);
+    auto dest = [&](int n0, int& mi, int& x) {
+      if (EPI == EpiQKV) {
+        if (n0 < p.q_cols) {
+          mi = 0;
+          x = n0;
+        } else if (n0 < p.q_cols + p.k_cols) {
+          mi = 1;
+          x = n0 - p.q_cols;
+        } else {
+          mi = 2;
+          x = n0 - p.q_cols - p.k_cols;
+        }
+      } else {
+        mi = 0;
+        x = n0;
+      }
+    };
+    int res_loads = 0;  // residual tiles requested by the elected thread
+    auto load_res = [&](int t) {
+      const int64_t m0 = (int64_t)(t / n_tiles_n) * 256 + rank * 128;
+      const int n0 = (t % n_tiles_n) * Cfg::BN;
+      ++res_loads;
+      mbar_arrive_expect_tx(res_full, Cfg::OUT_BYTES);
+      for (int j = 0; j < 4; ++j)
+        tma_load_2d(out_s + j * Cfg::BOX_BYTES, &maps.res, n0 + 64 * j, (int32_t)m0, res_full);
+    };
+    if (has_res && elected && cluster < n_tiles) load_res(cluster);
+    int i = 0;
+    for (int t = cluster; t < n_tiles; t += n_clusters, ++i) {
+      const int b = i & 1;
+      const int64_t m0 = (int64_t)(t / n_tiles_n) * 256 + rank * 128;
+      const int n0 = (t % n_tiles_n) * Cfg::BN;
+      bool ok = mbar_wait(&acc_full[b], (uint32_t)(i >> 1) & 1u, abort_flag, p.status);
+      if (ok && has_res) ok = mbar_wait(res_full, (uint32_t)i & 1u, abort_flag, p.status);
+      // one decision for all four warps (they meet at named barriers below)
+      if (!named_bar_and(1, 128, ok)) break;
+      tc_fence_after();
+      pair_epilogue_tile<EPI>(p, out_s, tmem + (uint32_t)(b * Cfg::BN) + ((uint32_t)(q * 32) << 16),
+                              row, m0 + row, n0, has_res);
+      tc_fence_before();
+      fence_proxy_async_smem();  // staging writes visible to the TMA stores
+      named_bar_sync(1, 128);
+      if (elected) {
+        if (rank == 0)
+          mbar_arrive(&acc_empty[b]);
+        else
+          mbar_arrive_cluster(acc_empty_lead0 + b * 8);
+        int mi, x;
+        dest(n0, mi, x);
+        for (int j = 0; j < 4; ++j)
+          tma_store_2d(&maps.out[mi], x + 64 * j, (int32_t)m0, out_s + j * Cfg::BOX_BYTES);
+        bulk_commit_group();
+        bulk_wait_read_all();  // staging may be overwritten from here on
+        if (has_res && t + n_clusters < n_tiles) load_res(t + n_clusters);
+      }
+      named_bar_sync(1, 128);
     }
-    tc_fence_before();
+    if (elected) {
+      bulk_wait_all();
+      // after an abort: a residual load may still be landing in the staging tile
+      if (res_loads > i) mbar_wait(res_full, (uint32_t)(res_loads - 1) & 1u, nullptr, p.status);
+    }
   }
   __syncthreads();
   cluster_sync_all();  // no CTA leaves while the pair's MMAs or arrives may touch it
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc_pair(tmem, Cfg::BN);
+    tmem_dealloc_pair(tmem, Cfg::TMEM_COLS);
   }
 }
 

@@ -3,6 +3,8 @@
 #include "tg_gemm.cuh"
 #include "tg_host.h"
 
+#include <algorithm>
+
 namespace tg {
 
 template <int BN, int STAGES, int EPI>
@@ -23,8 +25,7 @@ int launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const GemmParams& 
 }
 
 template <int STAGES, int EPI>
-int launch_pair(const CUtensorMap& ta, const CUtensorMap& tb, const GemmParams& p,
-                cudaStream_t stream) {
+int launch_pair(const PairMaps& maps, const GemmParams& p, cudaStream_t stream) {
   using Cfg = PairCfg<STAGES>;
   static int attr_dev = -1;
   int dev = 0;
@@ -34,10 +35,15 @@ int launch_pair(const CUtensorMap& ta, const CUtensorMap& tb, const GemmParams& 
                                      cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM));
     attr_dev = dev;
   }
-  dim3 grid((unsigned)(2 * ((p.M + 255) / 256)), (unsigned)(p.N / Cfg::BN));
-  gemm_pair_kernel<STAGES, EPI><<<grid, Cfg::THREADS, Cfg::SMEM, stream>>>(ta, tb, p);
+  // persistent: at most one cluster (two CTAs) per SM pair, each walking its tiles
+  const int64_t tiles = ((p.M + 255) / 256) * (p.N / Cfg::BN);
+  const int64_t clusters = std::min<int64_t>(tiles, std::max(1, sm_count() / 2));
+  gemm_pair_kernel<STAGES, EPI><<<dim3((unsigned)(2 * clusters)), Cfg::THREADS, Cfg::SMEM,
+                                  stream>>>(maps, p);
   return check_launch();
 }
+
+constexpr int kPairStages = 5;
 
 // Explicit instantiations used by the entry points.
 template int launch_gemm<256, 4, EpiStore>(const CUtensorMap&, const CUtensorMap&,
@@ -90,9 +96,18 @@ extern "C" int tg_linear(const tg_bf16* a, int64_t lda, const tg_bf16* w, int64_
   const bool pair = !rmsnorm_a && (N % 256) == 0;
   const int bn = pair ? 128 : pick_bn(M, N);
 
-  CUtensorMap ta, tb;
+  PairMaps maps;
+  CUtensorMap& ta = maps.a;
+  CUtensorMap& tb = maps.b;
   TG_TRY(make_tmap_bf16_2d(&ta, a, (uint64_t)M, (uint64_t)K, (uint64_t)lda, 64, 128));
   TG_TRY(make_tmap_bf16_2d(&tb, w, (uint64_t)N, (uint64_t)K, (uint64_t)ldw, 64, bn));
+  if (pair) {
+    TG_TRY(make_tmap_bf16_2d(&maps.out[0], c, (uint64_t)M, (uint64_t)N, (uint64_t)ldc, 64, 128));
+    maps.out[1] = maps.out[2] = maps.res = maps.out[0];
+    if (residual)
+      TG_TRY(make_tmap_bf16_2d(&maps.res, residual, (uint64_t)M, (uint64_t)N, (uint64_t)ld_res,
+                               64, 128));
+  }
   GemmParams p{};
   p.M = M;
   p.N = N;
@@ -106,7 +121,7 @@ extern "C" int tg_linear(const tg_bf16* a, int64_t lda, const tg_bf16* w, int64_
   p.row_ssq_out = row_ssq_out;
   p.ld_ssq_out = ld_ssq_out;
   p.status = status;
-  if (pair) return launch_pair<6, EpiStore>(ta, tb, p, (cudaStream_t)stream);
+  if (pair) return launch_pair<kPairStages, EpiStore>(maps, p, (cudaStream_t)stream);
   if (bn == 256) return launch_gemm<256, 4, EpiStore>(ta, tb, p, (cudaStream_t)stream);
   return launch_gemm<128, 3, EpiStore>(ta, tb, p, (cudaStream_t)stream);
 }
@@ -141,9 +156,22 @@ extern "C" int tg_qkv_rope_cache(const tg_bf16* x, int64_t ld_x, const tg_bf16* 
   const bool pair = row_ssq_in && aligned256;
   int bn = pair ? 128 : pick_bn(M, N);
   if (!pair && bn == 256 && !aligned256) bn = 128;
-  CUtensorMap ta, tb;
+  PairMaps maps;
+  CUtensorMap& ta = maps.a;
+  CUtensorMap& tb = maps.b;
   TG_TRY(make_tmap_bf16_2d(&ta, x, (uint64_t)M, (uint64_t)hidden, (uint64_t)ld_x, 64, 128));
   TG_TRY(make_tmap_bf16_2d(&tb, w_qkv, (uint64_t)N, (uint64_t)hidden, (uint64_t)ld_w, 64, bn));
+  if (pair) {
+    tg_bf16* k_rows = cache_k + slot_offset * ld_cache;
+    tg_bf16* v_rows = cache_v + slot_offset * ld_cache;
+    TG_TRY(make_tmap_bf16_2d(&maps.out[0], q_out, (uint64_t)M, (uint64_t)q_cols, (uint64_t)ld_q,
+                             64, 128));
+    TG_TRY(make_tmap_bf16_2d(&maps.out[1], k_rows, (uint64_t)M, (uint64_t)kv_cols,
+                             (uint64_t)ld_cache, 64, 128));
+    TG_TRY(make_tmap_bf16_2d(&maps.out[2], v_rows, (uint64_t)M, (uint64_t)kv_cols,
+                             (uint64_t)ld_cache, 64, 128));
+    maps.res = maps.out[0];
+  }
   GemmParams p{};
   p.M = M;
   p.N = N;
@@ -163,7 +191,7 @@ extern "C" int tg_qkv_rope_cache(const tg_bf16* x, int64_t ld_x, const tg_bf16* 
   p.row_ssq_in = row_ssq_in;
   p.ld_ssq_in = ld_ssq_in;
   p.status = status;
-  if (pair) return launch_pair<6, EpiQKV>(ta, tb, p, (cudaStream_t)stream);
+  if (pair) return launch_pair<kPairStages, EpiQKV>(maps, p, (cudaStream_t)stream);
   if (bn == 256) return launch_gemm<256, 4, EpiQKV>(ta, tb, p, (cudaStream_t)stream);
   return launch_gemm<128, 3, EpiQKV>(ta, tb, p, (cudaStream_t)stream);
 }
