@@ -374,7 +374,7 @@ struct PairCfg {
   static constexpr int OUT_BYTES = 4 * BOX_BYTES;      // staging of one 128 x 256 output tile
   static constexpr int BAR_BYTES = 256;
   static constexpr int SMEM = 1024 + TILE_BYTES + OUT_BYTES + BAR_BYTES;
-  static constexpr int THREADS = 192;
+  static constexpr int THREADS = 320;
   static constexpr int TMEM_COLS = 2 * BN;             // two accumulators (double buffer)
 };
 
@@ -384,13 +384,14 @@ __device__ __forceinline__ uint32_t sw128_chunk(int r, int k) {
   return (uint32_t)(r * 128 + ((k ^ (r & 7)) << 4));
 }
 
-// One 256 x 256 output tile of the pair (each CTA: 128 rows, staged in shared memory as
-// four swizzled boxes); `row` is the thread's row in the CTA's half, `tacc` the TMEM
-// address of the row's accumulator (lane quarter and buffer included).
+// Columns [128 h, 128 h + 128) of one 256 x 256 output tile of the pair (each CTA: 128
+// rows, staged in shared memory as four swizzled 64-column boxes); `row` is the thread's
+// row in the CTA's half, `tacc` the TMEM address of the row's accumulator (lane quarter
+// and buffer included).
 template <int EPI>
-__device__ __forceinline__ void pair_epilogue_tile(const GemmParams& p, unsigned char* out_s,
+__device__ __forceinline__ void pair_epilogue_half(const GemmParams& p, unsigned char* out_s,
                                                    uint32_t tacc, int row, int64_t grow, int n0,
-                                                   bool has_res) {
+                                                   int h, bool has_res) {
   const bool live = grow < p.M;
   const float rscale =
       (p.rmsnorm && p.row_ssq_in && live) ? rscale_from_ssq(p, grow) : 1.0f;
@@ -403,9 +404,9 @@ __device__ __forceinline__ void pair_epilogue_tile(const GemmParams& p, unsigned
     }
     const float4* cs_row = reinterpret_cast<const float4*>(p.cos_sin + (int64_t)pos * 128);
 #pragma unroll 1
-    for (int pr = 0; pr < 4; ++pr) {
+    for (int pr = 0; pr < 2; ++pr) {
       // 32-column pieces ca and ca + 2 hold columns i and i + 64 of one 128-column head
-      const int ca = (pr & 1) + 4 * (pr >> 1), cb = ca + 2;
+      const int ca = 4 * h + pr, cb = ca + 2;
       uint32_t ra[32], rb[32];
       tmem_ld32(tacc + ca * 32, ra);
       tmem_ld32(tacc + cb * 32, rb);
@@ -444,7 +445,7 @@ __device__ __forceinline__ void pair_epilogue_tile(const GemmParams& p, unsigned
   }
   float ssq = 0.f;
 #pragma unroll 1
-  for (int j = 0; j < 4; ++j) {  // box j: tile columns 64 j .. 64 j + 63
+  for (int j = 2 * h; j < 2 * h + 2; ++j) {  // box j: tile columns 64 j .. 64 j + 63
     uint32_t ra[32], rb[32];
     tmem_ld32(tacc + j * 64, ra);
     tmem_ld32(tacc + j * 64 + 32, rb);
@@ -479,10 +480,7 @@ __device__ __forceinline__ void pair_epilogue_tile(const GemmParams& p, unsigned
       }
       *cp = make_uint4(w[0], w[1], w[2], w[3]);
     }
-    if (p.row_ssq_out && (j & 1)) {
-      if (live) p.row_ssq_out[grow * p.ld_ssq_out + n0 / 128 + (j >> 1)] = ssq;
-      ssq = 0.f;
-    }
+    if (p.row_ssq_out && (j & 1) && live) p.row_ssq_out[grow * p.ld_ssq_out + n0 / 128 + h] = ssq;
   }
 }
 
@@ -491,15 +489,17 @@ __device__ __forceinline__ void pair_epilogue_tile(const GemmParams& p, unsigned
 //   warp 0     one thread streams A and W k-blocks of every tile through the ring;
 //   warp 1     TMEM owner; in the even CTA one thread issues the M=256 MMAs into
 //              accumulator buffer (tile index & 1);
-//   warps 2-5  epilogue of the previous tile while the next one accumulates: TMEM ->
-//              registers -> bf16 in a swizzled staging tile -> TMA stores.  For EpiStore
-//              with a residual, the staging tile is first filled with the residual rows
-//              by a TMA load issued one tile ahead.
+//   warps 2-9  epilogue of the previous tile while the next one accumulates, as two
+//              independent groups of four warps (one per TMEM lane quarter), group g
+//              owning tile columns [128 g, 128 g + 128): TMEM -> registers -> bf16 in
+//              swizzled staging boxes -> TMA stores.  For EpiStore with a residual, the
+//              group's boxes are first filled with the residual rows by a TMA load
+//              issued one tile ahead.
 // Barriers: full/empty per ring stage (full lives in the even CTA and counts both CTAs'
 // bytes); acc_full[b] (the even CTA's commit, in both CTAs); acc_empty[b] (even CTA,
-// one arrive per CTA once its epilogue has read buffer b); res_full (this CTA).
+// one arrive per epilogue group of each CTA once it has read buffer b); res_full[g].
 template <int STAGES, int EPI>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(320, 1)
     gemm_pair_kernel(const __grid_constant__ PairMaps maps, GemmParams p) {
   using Cfg = PairCfg<STAGES>;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
@@ -511,8 +511,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
   uint64_t* empty = full + STAGES;
   uint64_t* acc_full = empty + STAGES;   // [2]
   uint64_t* acc_empty = acc_full + 2;    // [2]
-  uint64_t* res_full = acc_empty + 2;
-  uint64_t* drain = res_full + 1;
+  uint64_t* res_full = acc_empty + 2;   // [2]
+  uint64_t* drain = res_full + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -531,9 +531,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&acc_full[b], 1);
-      mbar_init(&acc_empty[b], 2);
+      mbar_init(&acc_empty[b], 4);
+      mbar_init(&res_full[b], 1);
     }
-    mbar_init(res_full, 1);
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -620,35 +620,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
       mbar_wait(drain, 0, nullptr, p.status);  // all MMAs (and their arrives) done
     }
   } else {
-    const int q = warp & 3;  // TMEM lane quarter this warp may access
+    const int q = warp & 3;        // TMEM lane quarter this warp may access
+    const int g = (warp - 2) >> 2;  // epilogue group: tile columns [128 g, 128 g + 128)
     const int row = q * 32 + lane;
-    const bool elected = warp == 2 && lane == 0;
+    const bool elected = (warp & 3) == 2 && lane == 0;  // warps 2 and 6
+    const uint32_t bar_id = 1 + (uint32_t)g;
     const uint32_t acc_empty_lead0 = mapa_shared(smem_u32(&acc_empty[0]), 0);
-    auto dest = [&](int n0, int& mi, int& x) {
-      if (EPI == EpiQKV) {
-        if (n0 < p.q_cols) {
-          mi = 0;
-          x = n0;
-        } else if (n0 < p.q_cols + p.k_cols) {
-          mi = 1;
-          x = n0 - p.q_cols;
-        } else {
-          mi = 2;
-          x = n0 - p.q_cols - p.k_cols;
-        }
-      } else {
-        mi = 0;
-        x = n0;
-      }
-    };
-    int res_loads = 0;  // residual tiles requested by the elected thread
+    int res_loads = 0;  // residual half-tiles requested by this group's elected thread
     auto load_res = [&](int t) {
       const int64_t m0 = (int64_t)(t / n_tiles_n) * 256 + rank * 128;
       const int n0 = (t % n_tiles_n) * Cfg::BN;
       ++res_loads;
-      mbar_arrive_expect_tx(res_full, Cfg::OUT_BYTES);
-      for (int j = 0; j < 4; ++j)
-        tma_load_2d(out_s + j * Cfg::BOX_BYTES, &maps.res, n0 + 64 * j, (int32_t)m0, res_full);
+      mbar_arrive_expect_tx(&res_full[g], 2 * Cfg::BOX_BYTES);
+      for (int j = 2 * g; j < 2 * g + 2; ++j)
+        tma_load_2d(out_s + j * Cfg::BOX_BYTES, &maps.res, n0 + 64 * j, (int32_t)m0,
+                    &res_full[g]);
     };
     if (has_res && elected && cluster < n_tiles) load_res(cluster);
     int i = 0;
@@ -657,34 +643,44 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
       const int64_t m0 = (int64_t)(t / n_tiles_n) * 256 + rank * 128;
       const int n0 = (t % n_tiles_n) * Cfg::BN;
       bool ok = mbar_wait(&acc_full[b], (uint32_t)(i >> 1) & 1u, abort_flag, p.status);
-      if (ok && has_res) ok = mbar_wait(res_full, (uint32_t)i & 1u, abort_flag, p.status);
-      // one decision for all four warps (they meet at named barriers below)
-      if (!named_bar_and(1, 128, ok)) break;
+      if (ok && has_res) ok = mbar_wait(&res_full[g], (uint32_t)i & 1u, abort_flag, p.status);
+      // one decision for the group's four warps (they meet at named barriers below)
+      if (!named_bar_and(bar_id, 128, ok)) break;
       tc_fence_after();
-      pair_epilogue_tile<EPI>(p, out_s, tmem + (uint32_t)(b * Cfg::BN) + ((uint32_t)(q * 32) << 16),
-                              row, m0 + row, n0, has_res);
+      pair_epilogue_half<EPI>(p, out_s,
+                              tmem + (uint32_t)(b * Cfg::BN) + ((uint32_t)(q * 32) << 16), row,
+                              m0 + row, n0, g, has_res);
       tc_fence_before();
       fence_proxy_async_smem();  // staging writes visible to the TMA stores
-      named_bar_sync(1, 128);
+      named_bar_sync(bar_id, 128);
       if (elected) {
         if (rank == 0)
           mbar_arrive(&acc_empty[b]);
         else
           mbar_arrive_cluster(acc_empty_lead0 + b * 8);
-        int mi, x;
-        dest(n0, mi, x);
-        for (int j = 0; j < 4; ++j)
+        int mi = 0, x = n0;
+        if (EPI == EpiQKV) {
+          if (n0 >= p.q_cols + p.k_cols) {
+            mi = 2;
+            x = n0 - p.q_cols - p.k_cols;
+          } else if (n0 >= p.q_cols) {
+            mi = 1;
+            x = n0 - p.q_cols;
+          }
+        }
+        for (int j = 2 * g; j < 2 * g + 2; ++j)
           tma_store_2d(&maps.out[mi], x + 64 * j, (int32_t)m0, out_s + j * Cfg::BOX_BYTES);
         bulk_commit_group();
-        bulk_wait_read_all();  // staging may be overwritten from here on
+        bulk_wait_read_all();  // the group's staging boxes may be overwritten from here on
         if (has_res && t + n_clusters < n_tiles) load_res(t + n_clusters);
       }
-      named_bar_sync(1, 128);
+      named_bar_sync(bar_id, 128);
     }
     if (elected) {
       bulk_wait_all();
-      // after an abort: a residual load may still be landing in the staging tile
-      if (res_loads > i) mbar_wait(res_full, (uint32_t)(res_loads - 1) & 1u, nullptr, p.status);
+      // after an abort: a residual load may still be landing in the staging boxes
+      if (res_loads > i)
+        mbar_wait(&res_full[g], (uint32_t)(res_loads - 1) & 1u, nullptr, p.status);
     }
   }
   __syncthreads();
