@@ -25,7 +25,8 @@ __all__ = [
     "TokenGateError", "lib", "tg_version", "tg_device_supported", "tg_plan_kept",
     "tg_rope_table", "tg_gate_score_workspace_size", "tg_gate_score", "tg_topk_compact",
     "tg_gate_score_noalloc", "tg_seq_rmsnorm", "tg_gather_rope", "tg_kv_compact", "tg_gated_attention", "tg_linear",
-    "tg_status_clear", "tg_status_read", "GatedPrefill", "STATUS_TIMEOUT", "STATUS_BUDGET",
+    "tg_status_clear", "tg_status_read", "tg_set_launch_overlap", "tg_get_launch_overlap",
+    "GatedPrefill", "STATUS_TIMEOUT", "STATUS_BUDGET",
     "STATUS_BOUNDS",
 ]
 
@@ -91,6 +92,15 @@ def tg_device_supported(device: int = 0) -> bool:
 
 def tg_status_clear(status: torch.Tensor, stream=None) -> None:
     _check(lib.tg_status_clear(_ptr(status), _stream(stream)), "tg_status_clear")
+
+
+def tg_set_launch_overlap(enable: bool) -> None:
+    """Launch every kernel with programmatic stream serialisation (default off)."""
+    _check(lib.tg_set_launch_overlap(1 if enable else 0), "tg_set_launch_overlap")
+
+
+def tg_get_launch_overlap() -> bool:
+    return bool(lib.tg_get_launch_overlap())
 
 
 def tg_status_read(status: torch.Tensor, stream=None) -> int:

@@ -1,4 +1,5 @@
 // Library-wide entry points (errors, device checks, status word) and host helpers.
+#include <atomic>
 #include <cstring>
 #include <mutex>
 
@@ -61,6 +62,13 @@ int make_tmap_bf16_2d(CUtensorMap* out, const void* base, uint64_t rows, uint64_
   }
   return TG_OK;
 }
+
+namespace {
+std::atomic<int> g_launch_overlap{0};
+}
+
+bool launch_overlap() { return g_launch_overlap.load(std::memory_order_relaxed) != 0; }
+void set_launch_overlap(bool on) { g_launch_overlap.store(on ? 1 : 0, std::memory_order_relaxed); }
 
 int sm_count() {
   static int cached[64] = {0};
@@ -130,6 +138,13 @@ int tg_plan_kept(const int32_t* cu_seqlens_host, const int32_t* n_question_host,
   }
   return TG_OK;
 }
+
+int tg_set_launch_overlap(int enable) {
+  tg::set_launch_overlap(enable != 0);
+  return TG_OK;
+}
+
+int tg_get_launch_overlap(void) { return tg::launch_overlap() ? 1 : 0; }
 
 int tg_status_clear(uint32_t* status, tg_stream_t stream) {
   if (!status) return TG_ERR_INVALID_ARGUMENT;

@@ -192,21 +192,6 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
-  // ---- which work item: head groups vary fastest, then items heaviest first
-  const int hg = p.n_kv_heads * p.head_pairs;
-  const int head_grp = blockIdx.x % hg;
-  const int item = blockIdx.x / hg;
-  int b, qt, part, nparts;
-  decode_item(p, item, b, qt, part, nparts);
-  const int g = head_grp / p.head_pairs;
-  const int h0 = g * p.group + 2 * (head_grp % p.head_pairs);
-  const int64_t row0 = p.cu_kept[b];
-  const int n_b = p.cu_kept[b + 1] - p.cu_kept[b];
-  const int q0 = qt * kBM;
-  // causal: key tiles 0..qt, this item's share [j0, j0 + nt)
-  const int j0 = part * p.chunk;
-  const int nt = min(qt + 1, j0 + p.chunk) - j0;
-
   if (tid == 0) {
     mbar_init(q_full, 1);
     for (int s = 0; s < kStages; ++s) {
@@ -238,6 +223,23 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // everything below reads what earlier grids wrote
+  griddep_wait();
+
+  // ---- which work item: head groups vary fastest, then items heaviest first
+  const int hg = p.n_kv_heads * p.head_pairs;
+  const int head_grp = blockIdx.x % hg;
+  const int item = blockIdx.x / hg;
+  int b, qt, part, nparts;
+  decode_item(p, item, b, qt, part, nparts);
+  const int g = head_grp / p.head_pairs;
+  const int h0 = g * p.group + 2 * (head_grp % p.head_pairs);
+  const int64_t row0 = p.cu_kept[b];
+  const int n_b = p.cu_kept[b + 1] - p.cu_kept[b];
+  const int q0 = qt * kBM;
+  // causal: key tiles 0..qt, this item's share [j0, j0 + nt)
+  const int j0 = part * p.chunk;
+  const int nt = min(qt + 1, j0 + p.chunk) - j0;
 
   if (warp < 4) {
     regs_dec<kRegsLow>();
@@ -528,6 +530,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 // layout above every load and store of a warp is contiguous.
 constexpr int kMaxParts = 64;
 __global__ void __launch_bounds__(128) combine_parts_kernel(const __grid_constant__ AttnParams p) {
+  griddep_wait();
   const int item = blockIdx.x, hh = blockIdx.y;
   int b, qt, part, nparts;
   decode_item(p, item, b, qt, part, nparts);
@@ -768,13 +771,10 @@ extern "C" int tg_gated_attention(const tg_bf16* q, int64_t ld_q, const tg_bf16*
 
   const int64_t grid = (int64_t)plan.n_items * head_groups;
   if (grid > 0x7FFFFFFF) return TG_ERR_UNSUPPORTED_SHAPE;
-  gated_attention_kernel<<<(unsigned)grid, kThreads, AttnSmem::BYTES, (cudaStream_t)stream>>>(
-      tq, tk, tv, prm);
-  TG_TRY(check_launch());
-  if (plan.split) {
-    combine_parts_kernel<<<dim3((unsigned)plan.n_items, (unsigned)n_q_heads), 128, 0,
-                           (cudaStream_t)stream>>>(prm);
-    TG_TRY(check_launch());
-  }
+  TG_TRY(launch(gated_attention_kernel, dim3((unsigned)grid), dim3(kThreads), AttnSmem::BYTES,
+                (cudaStream_t)stream, tq, tk, tv, prm));
+  if (plan.split)
+    TG_TRY(launch(combine_parts_kernel, dim3((unsigned)plan.n_items, (unsigned)n_q_heads),
+                  dim3(128), 0, (cudaStream_t)stream, prm));
   return TG_OK;
 }

@@ -31,6 +31,7 @@ constexpr int kNormRowsPerCta = 8192;
 
 __global__ void fold_norm_kernel(const uint16_t* __restrict__ W1, const float* __restrict__ w,
                                  uint16_t* __restrict__ out, int width, int hidden) {
+  griddep_wait();
   const int64_t n = (int64_t)width * hidden;
   for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n;
        i += (int64_t)gridDim.x * blockDim.x) {
@@ -57,6 +58,7 @@ __global__ void __launch_bounds__(kNormThreads)
                     const int32_t* __restrict__ cu, const uint8_t* __restrict__ prunable,
                     float eps, float* __restrict__ z, float* __restrict__ bias) {
   __shared__ double red[kNormThreads / 32];
+  griddep_wait();
   const int b = blockIdx.y;
   const int64_t lo = cu[b], hi = cu[b + 1];
   const int64_t n = hi - lo;
@@ -137,9 +139,8 @@ extern "C" int tg_gate_score(const tg_bf16* h, int64_t ld_h, int64_t total_token
     const int64_t n = (int64_t)width * hidden;
     int grid = (int)((n + 255) / 256);
     if (grid > sm_count() * 8) grid = sm_count() * 8;
-    fold_norm_kernel<<<grid, 256, 0, st>>>(reinterpret_cast<const uint16_t*>(W1), norm_w, w1f,
-                                           width, hidden);
-    TG_TRY(check_launch());
+    TG_TRY(launch(fold_norm_kernel, dim3(grid), dim3(256), 0, st,
+                  reinterpret_cast<const uint16_t*>(W1), norm_w, w1f, width, hidden));
     wmat = w1f;
   }
   CUtensorMap ta, tb;
@@ -160,9 +161,8 @@ extern "C" int tg_gate_score(const tg_bf16* h, int64_t ld_h, int64_t total_token
   TG_TRY((launch_gemm<256, 4, EpiScore>(ta, tb, p, st)));
 
   dim3 grid((unsigned)((max_n + kNormRowsPerCta - 1) / kNormRowsPerCta), (unsigned)batch);
-  seq_norm_kernel<<<grid, kNormThreads, 0, st>>>(s_out, partial, cu_seqlens, prunable, eps_seq,
-                                                 z_out, bias_out);
-  return check_launch();
+  return launch(seq_norm_kernel, grid, dim3(kNormThreads), 0, st, (const float*)s_out,
+                (const float*)partial, cu_seqlens, prunable, eps_seq, z_out, bias_out);
 }
 
 extern "C" int tg_seq_rmsnorm(const float* s, const int32_t* cu_seqlens,
@@ -182,7 +182,7 @@ extern "C" int tg_seq_rmsnorm(const float* s, const int32_t* cu_seqlens,
   if (z_out == s || bias_out == s) return TG_ERR_INVALID_ARGUMENT;
   TG_TRY(check_device());
   dim3 grid((unsigned)((max_n + kNormRowsPerCta - 1) / kNormRowsPerCta), (unsigned)batch);
-  seq_norm_kernel<<<grid, kNormThreads, 0, (cudaStream_t)stream>>>(s, nullptr, cu_seqlens, prunable,
-                                                                   eps_seq, z_out, bias_out);
-  return check_launch();
+  TG_TRY(launch(seq_norm_kernel, grid, dim3(kNormThreads), 0, (cudaStream_t)stream, s,
+                (const float*)nullptr, cu_seqlens, prunable, eps_seq, z_out, bias_out));
+  return TG_OK;
 }

@@ -23,6 +23,7 @@ constexpr int kVecPerBatch = 8;   // 16-byte vectors in flight per lane
 
 __global__ void rope_table_kernel(float2* __restrict__ table, int max_pos, int half,
                                   double theta, int head_dim) {
+  griddep_wait();
   const int64_t n = (int64_t)max_pos * half;
   for (int64_t t = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; t < n;
        t += (int64_t)gridDim.x * blockDim.x) {
@@ -129,6 +130,7 @@ __device__ __forceinline__ void copy_row_ssq(const uint4* __restrict__ s, uint4*
 }
 
 __global__ void __launch_bounds__(kCopyWarps * 32) gather_rope_kernel(GatherArgs a) {
+  griddep_wait();
   const int lane = threadIdx.x & 31;
   const int64_t warp0 = (int64_t)blockIdx.x * kCopyWarps + (threadIdx.x >> 5);
   const int64_t nwarps = (int64_t)gridDim.x * kCopyWarps;
@@ -186,6 +188,7 @@ struct KvArgs {
 };
 
 __global__ void __launch_bounds__(kCopyWarps * 32) kv_compact_kernel(KvArgs a) {
+  griddep_wait();
   const int lane = threadIdx.x & 31;
   const int64_t warp0 = (int64_t)blockIdx.x * kCopyWarps + (threadIdx.x >> 5);
   const int64_t nwarps = (int64_t)gridDim.x * kCopyWarps;
@@ -224,9 +227,8 @@ extern "C" int tg_rope_table(float* cos_sin, int max_pos, int head_dim, double t
   const int64_t n = (int64_t)max_pos * half;
   int grid = (int)((n + 255) / 256);
   if (grid > sm_count() * 16) grid = sm_count() * 16;
-  rope_table_kernel<<<grid, 256, 0, (cudaStream_t)stream>>>(reinterpret_cast<float2*>(cos_sin),
-                                                            max_pos, half, theta, head_dim);
-  return check_launch();
+  return launch(rope_table_kernel, dim3(grid), dim3(256), 0, (cudaStream_t)stream,
+                reinterpret_cast<float2*>(cos_sin), max_pos, half, theta, head_dim);
 }
 
 extern "C" int tg_gather_rope(const tg_bf16* src, int64_t ld_src, int64_t src_rows,
@@ -256,8 +258,8 @@ extern "C" int tg_gather_rope(const tg_bf16* src, int64_t ld_src, int64_t src_ro
   GatherArgs a{reinterpret_cast<const uint16_t*>(src), ld_src, src_rows, row_idx, n_rows, width,
                rope_pos, rope_col_begin, rope_col_end, head_dim, cos_sin, max_pos,
                reinterpret_cast<uint16_t*>(dst), ld_dst, row_ssq_out, ld_ssq_out, status};
-  gather_rope_kernel<<<copy_grid(n_rows), kCopyWarps * 32, 0, (cudaStream_t)stream>>>(a);
-  return check_launch();
+  return launch(gather_rope_kernel, dim3(copy_grid(n_rows)), dim3(kCopyWarps * 32), 0,
+                (cudaStream_t)stream, a);
 }
 
 extern "C" int tg_kv_compact(const tg_bf16* k, int64_t ld_k, const tg_bf16* v, int64_t ld_v,
@@ -279,6 +281,6 @@ extern "C" int tg_kv_compact(const tg_bf16* k, int64_t ld_k, const tg_bf16* v, i
   KvArgs a{reinterpret_cast<const uint16_t*>(k), ld_k, reinterpret_cast<const uint16_t*>(v), ld_v,
            src_rows, row_idx, n_rows, width, reinterpret_cast<uint16_t*>(cache_k),
            reinterpret_cast<uint16_t*>(cache_v), ld_cache, slot_offset, status};
-  kv_compact_kernel<<<copy_grid(2 * n_rows), kCopyWarps * 32, 0, (cudaStream_t)stream>>>(a);
-  return check_launch();
+  return launch(kv_compact_kernel, dim3(copy_grid(2 * n_rows)), dim3(kCopyWarps * 32), 0,
+                (cudaStream_t)stream, a);
 }

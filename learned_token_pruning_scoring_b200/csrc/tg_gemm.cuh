@@ -252,6 +252,7 @@ __global__ void __launch_bounds__(192, 1)
     tmem_alloc(tmem_slot, BN);
     tmem_relinquish();
   }
+  griddep_wait();  // operands and outputs may belong to earlier grids
   if (EPI == EpiScore) {
     for (int i = tid; i < BN; i += Cfg::THREADS) w2s[i] = p.w2[n0 + i];
   }
@@ -558,6 +559,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(320, 1)
       // A stage is reloaded only after the even CTA's commit freed it, which follows
       // the completion of that barrier's previous phase.
       const uint32_t full_lead0 = mapa_shared(smem_u32(&full[0]), 0);
+      griddep_wait();
       int kg = 0;
       bool ok = true;
       for (int t = cluster; ok && t < n_tiles; t += n_clusters) {
@@ -626,6 +628,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(320, 1)
     const bool elected = (warp & 3) == 2 && lane == 0;  // warps 2 and 6
     const uint32_t bar_id = 1 + (uint32_t)g;
     const uint32_t acc_empty_lead0 = mapa_shared(smem_u32(&acc_empty[0]), 0);
+    griddep_wait();
     int res_loads = 0;  // residual half-tiles requested by this group's elected thread
     auto load_res = [&](int t) {
       const int64_t m0 = (int64_t)(t / n_tiles_n) * 256 + rank * 128;

@@ -34,6 +34,35 @@ int make_tmap_bf16_2d(CUtensorMap* out, const void* base, uint64_t rows, uint64_
 // Number of SMs of the current device (cached).
 int sm_count();
 
+// Library-wide switch (tg_set_launch_overlap): launch kernels with programmatic stream
+// serialisation so that a grid's launch and prologue overlap the end of the grid before it.
+bool launch_overlap();
+void set_launch_overlap(bool on);
+
+// Launch `kernel` on `stream`, with programmatic stream serialisation when the switch is
+// on.  Every kernel launched this way calls griddep_wait() before it touches global
+// memory that an earlier grid may write.  Returns TG_OK or TG_ERR_CUDA.
+template <typename... KArgs, typename... Args>
+int launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+           Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = launch_overlap() ? 1 : 0;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, static_cast<Args&&>(args)...);
+  if (e != cudaSuccess) {
+    set_cuda_error(e);
+    return TG_ERR_CUDA;
+  }
+  return TG_OK;
+}
+
 }  // namespace tg
 
 #define TG_CUDA_TRY(expr)                      \

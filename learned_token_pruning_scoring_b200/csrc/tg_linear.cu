@@ -20,8 +20,8 @@ int launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const GemmParams& 
     attr_dev = dev;
   }
   dim3 grid((unsigned)((p.M + Cfg::BM - 1) / Cfg::BM), (unsigned)(p.N / BN));
-  gemm_kernel<BN, STAGES, EPI><<<grid, Cfg::THREADS, Cfg::SMEM, stream>>>(ta, tb, p);
-  return check_launch();
+  return launch(gemm_kernel<BN, STAGES, EPI>, grid, dim3(Cfg::THREADS), Cfg::SMEM, stream, ta, tb,
+                p);
 }
 
 template <int STAGES, int EPI>
@@ -38,9 +38,8 @@ int launch_pair(const PairMaps& maps, const GemmParams& p, cudaStream_t stream) 
   // persistent: at most one cluster (two CTAs) per SM pair, each walking its tiles
   const int64_t tiles = ((p.M + 255) / 256) * (p.N / Cfg::BN);
   const int64_t clusters = std::min<int64_t>(tiles, std::max(1, sm_count() / 2));
-  gemm_pair_kernel<STAGES, EPI><<<dim3((unsigned)(2 * clusters)), Cfg::THREADS, Cfg::SMEM,
-                                  stream>>>(maps, p);
-  return check_launch();
+  return launch(gemm_pair_kernel<STAGES, EPI>, dim3((unsigned)(2 * clusters)), dim3(Cfg::THREADS),
+                Cfg::SMEM, stream, maps, p);
 }
 
 constexpr int kPairStages = 5;

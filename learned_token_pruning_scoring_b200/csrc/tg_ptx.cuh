@@ -32,6 +32,23 @@ __device__ __forceinline__ uint32_t lane_id() {
   return l;
 }
 
+// ------------------------------------------------------------------ dependent launch
+
+// Programmatic dependent launch.  A grid launched with programmatic stream serialisation
+// may start once every CTA of the grid before it in the stream has exited, before that
+// grid has completed and its writes have been flushed; griddep_wait() blocks the calling
+// thread until every grid it depends on has completed and its memory is visible (it
+// returns at once for an ordinary launch).  The wait orders those writes for this
+// thread's generic accesses; the proxy fence after it extends that to the TMA loads
+// (async proxy) the thread issues next, which a kernel boundary would otherwise order.
+// Every kernel of this library calls it before touching global memory that another
+// grid may write.  None of them signals an earlier start
+// (griddepcontrol.launch_dependents): letting the next grid's CTAs occupy SMs while this
+// grid still runs was measured to slow the attention kernels.
+__device__ __forceinline__ void griddep_wait() {
+  asm volatile("griddepcontrol.wait;\n\tfence.proxy.async.global;" ::: "memory");
+}
+
 // ------------------------------------------------------------------ mbarrier
 
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {

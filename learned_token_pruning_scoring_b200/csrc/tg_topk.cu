@@ -23,6 +23,7 @@
 
 #include "tg_host.h"
 #include "tg_ptx.cuh"
+#include "tg_ptx.cuh"
 
 namespace cg = cooperative_groups;
 
@@ -94,6 +95,7 @@ __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kThreads)
   const int b = blockIdx.x / kCluster;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const uint32_t lt_mask = (1u << lane) - 1u;
+  griddep_wait();
 
   const int64_t lo_b = a.cu_seqlens[b];
   const int64_t n_b = (int64_t)a.cu_seqlens[b + 1] - lo_b;
@@ -331,6 +333,6 @@ extern "C" int tg_topk_compact(const float* z, const uint8_t* prunable, const in
     attr_done = true;
   }
   TopkArgs a{z, prunable, cu_seqlens, cu_kept, kept_idx, kept_pos, kept_bias, status};
-  topk_kernel<<<batch * kCluster, kThreads, smem, (cudaStream_t)stream>>>(a);
-  return check_launch();
+  return launch(topk_kernel, dim3((unsigned)(batch * kCluster)), dim3(kThreads), smem,
+                (cudaStream_t)stream, a);
 }

@@ -94,3 +94,12 @@ def test_host_side_argument_errors(lib):
     # workspace too small
     assert lib.tg_gate_score(p, 2048, 8, 2048, None, p, 256, p, 1e-6, p, cu, 1, 1e-6, p, p,
                              p, p, p, 16, None, None) == -4
+
+
+def test_launch_overlap_switch(lib):
+    """The overlap switch is host state only (no device needed)."""
+    prev = lib.tg_get_launch_overlap()
+    assert prev in (0, 1)
+    assert lib.tg_set_launch_overlap(0) == 0 and lib.tg_get_launch_overlap() == 0
+    assert lib.tg_set_launch_overlap(7) == 0 and lib.tg_get_launch_overlap() == 1
+    lib.tg_set_launch_overlap(prev)

@@ -203,3 +203,48 @@ def test_pipeline_n128k_planted_cluster(tg):
     x = P["x"].float()
     assert torch.isfinite(x).all()
     assert tg.tg_status_read(pipe.status) == 0
+
+
+def test_launch_overlap_gives_identical_results(tg):
+    """Programmatic dependent launch changes only when kernels are scheduled: a step run
+    eagerly and replayed from a CUDA graph with the overlap on must match, bit for bit,
+    the same step with it off (every kernel here is deterministic)."""
+    wl = S.custom([2100, 700, 1500], [16, 64, 5], [900, 300, 600], n_layers=3,
+                  name="overlap3")
+    h, gate, layers, pr, pipe = _setup(tg, wl)
+    hd, prd = h.cuda(), pr.cuda()
+    P = pipe.planned
+    keys = ("z", "kept_idx", "x", "ssq")
+
+    def snapshot():
+        torch.cuda.synchronize()
+        out = {k: P[k].clone() for k in keys}
+        out["caches"] = [(k.clone(), v.clone()) for k, v in P["caches"]]
+        return out
+
+    prev = tg.tg_get_launch_overlap()
+    try:
+        tg.tg_set_launch_overlap(False)
+        pipe.run(hd, prd)
+        ref = snapshot()
+        tg.tg_set_launch_overlap(True)
+        assert tg.tg_get_launch_overlap()
+        pipe.run(hd, prd)
+        eager = snapshot()
+        stream = torch.cuda.Stream()
+        stream.wait_stream(torch.cuda.current_stream())
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            pipe.run(hd, prd, stream=stream)
+        for _ in range(2):
+            g.replay()
+        graphed = snapshot()
+        del g
+    finally:
+        tg.tg_set_launch_overlap(prev)
+    for got in (eager, graphed):
+        for k in keys:
+            assert torch.equal(got[k], ref[k]), k
+        for (k0, v0), (k1, v1) in zip(got["caches"], ref["caches"]):
+            assert torch.equal(k0, k1) and torch.equal(v0, v1)
+    assert tg.tg_status_read(pipe.status) == 0
