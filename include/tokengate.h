@@ -298,9 +298,13 @@ int tg_gated_attention(const tg_bf16* q, int64_t ld_q, const tg_bf16* k, int64_t
 
 /*
  * Workspace bytes that let tg_gated_attention split the key range of long causal query
- * tiles over several CTAs (balancing the triangle over all SMs; a second kernel merges
- * the parts).  0 when the layout needs no split.  With a smaller or NULL workspace the
- * call still runs, one CTA per query tile and kv-head pair.
+ * tiles over several CTAs (balancing the triangle over all SMs).  Each part writes its
+ * partial result (unnormalised O, row max, row sum) there and counts itself in; the
+ * part that completes a tile's count merges the parts and writes o.  0 when the layout
+ * needs no split.  With a smaller or NULL workspace the call still runs, one CTA per
+ * query tile and kv-head pair.  The workspace must be zero-filled before its first use
+ * (the counters); every call that completes leaves it that way.  After a call that
+ * raised TG_STATUS_TIMEOUT, zero it again before reusing it.
  */
 size_t tg_gated_attention_workspace_size(const int32_t* cu_kept_host, int batch,
                                          int n_q_heads, int n_kv_heads, int head_dim);

@@ -264,7 +264,8 @@ def tg_gated_attention(q, k, v, cu_kept, cu_kept_host, n_q_heads, n_kv_heads, ke
                        kept_bias, gamma, beta, o=None, lse=None, head_dim=128, workspace=None,
                        status=None, stream=None):
     """Token-gated attention.  `workspace=None` allocates the split-KV workspace the
-    layout asks for (pass a uint8 tensor to reuse one; an empty one disables splitting)."""
+    layout asks for (pass a zero-filled uint8 tensor to reuse one: calls leave it zeroed;
+    an empty one disables splitting)."""
     ld_q, ld_k, ld_v = _mat(q, "q"), _mat(k, "k"), _mat(v, "v")
     ckh = _host_i32(cu_kept_host)
     batch = ckh.numel() - 1
@@ -273,7 +274,7 @@ def tg_gated_attention(q, k, v, cu_kept, cu_kept_host, n_q_heads, n_kv_heads, ke
     ld_o = _mat(o, "o")
     if workspace is None:
         need = tg_gated_attention_workspace_size(ckh, n_q_heads, n_kv_heads, head_dim)
-        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+        workspace = torch.zeros(need, dtype=torch.uint8, device=q.device)
     ws_ptr = _ptr(workspace) if workspace.numel() else None
     rc = lib.tg_gated_attention(_ptr(q), ld_q, _ptr(k), ld_k, _ptr(v), ld_v, _ptr(cu_kept),
                                 _ptr(ckh), batch, n_q_heads, n_kv_heads, head_dim,
@@ -281,7 +282,7 @@ def tg_gated_attention(q, k, v, cu_kept, cu_kept_host, n_q_heads, n_kv_heads, ke
                                 _ptr(o), ld_o, _ptr(lse), ws_ptr, workspace.numel(),
                                 _ptr(status), _stream(stream))
     _check(rc, "tg_gated_attention")
-    _count(2 if (ws_ptr is not None and workspace.numel() > 0) else 1)
+    _count()
     return o
 
 
@@ -395,7 +396,7 @@ class GatedPrefill:
             ssq=torch.empty((K, self.hidden // 128), **f32),
             qkv=torch.empty((K, nqkv), **bf),
             o=torch.empty((K, self.hq * self.d), **bf),
-            attn_ws=torch.empty(tg_gated_attention_workspace_size(ck_h, self.hq, self.hkv, self.d),
+            attn_ws=torch.zeros(tg_gated_attention_workspace_size(ck_h, self.hq, self.hkv, self.d),
                                 dtype=torch.uint8, device=dev),
             caches=[(torch.empty((K, self.hkv * self.d), **bf),
                      torch.empty((K, self.hkv * self.d), **bf)) for _ in self.layers],

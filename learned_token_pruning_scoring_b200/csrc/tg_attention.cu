@@ -54,6 +54,11 @@ constexpr int kMaxBatch = 512;  // requests per call (tile table lives in the pa
 constexpr int kTileBytes = kBM * kD * 2;  // 32 KB: 128 rows x 128 bf16, two 64-column boxes
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleThreshold = 8.0f;
+constexpr int kMaxParts = 8;    // parts per split query tile
+constexpr int kBoxBytes = kBM * 64 * 2;  // one 64-column bf16 box of a 128-row tile
+// Epilogue staging (the Q/K/V/bias region is free once every MMA has retired): a split
+// part's block for both heads at 0, the bf16 output tile (2 heads x 2 boxes) after it.
+constexpr int kEpiOut = 2 * (kBM * kD + 2 * kBM) * 4;
 
 struct AttnSmem {
   // 1024-aligned tiles first
@@ -66,6 +71,9 @@ struct AttnSmem {
   static constexpr int END = BAR + 256;
   static constexpr int BYTES = END + 1024;  // alignment slack
 };
+
+static_assert(kEpiOut % 1024 == 0 && kEpiOut + 4 * kBoxBytes <= AttnSmem::BAR,
+              "epilogue staging must fit below the barriers, 1024-byte aligned");
 
 struct AttnParams {
   const int32_t* cu_kept;
@@ -85,6 +93,8 @@ struct AttnParams {
   uint32_t* status;
   int chunk;           // key tiles per work item (split-KV); >= every request's tile count = no split
   float* part_ws;      // partial results of split query tiles (see kPartFloats), or null
+  int* part_count;     // per (first item of a split tile, head group): parts arrived
+  int* part_ready;     // per (work item, head group): 1 once the part's partial is written
   int32_t item_prefix[kMaxBatch + 1];  // work items before request b
 };
 
@@ -171,6 +181,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     gated_attention_kernel(const __grid_constant__ CUtensorMap tmQ,
                            const __grid_constant__ CUtensorMap tmK,
                            const __grid_constant__ CUtensorMap tmV,
+                           const __grid_constant__ CUtensorMap tmO,
                            const __grid_constant__ AttnParams p) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>(
@@ -187,8 +198,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* p_full = s_full + 2;           // [2]
   uint64_t* pv_done = p_full + 2;          // [2]
   uint64_t* drain = pv_done + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* merge_full = drain + 1;        // a split tile's other part staged for the merge
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(merge_full + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  volatile int* last_part = reinterpret_cast<volatile int*>(tmem_slot + 2);
+  volatile int* parts_ready = reinterpret_cast<volatile int*>(tmem_slot + 3);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
@@ -207,6 +221,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&pv_done[h], 1);
     }
     mbar_init(drain, 1);
+    mbar_init(merge_full, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -472,49 +487,253 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       mbar_arrive(&p_full[wg]);
     }
-    if (ok && warp_all(mbar_wait(&pv_done[wg], (uint32_t)(nt - 1) & 1u, abort_flag, p.status))) {
-      tc_fence_after();
-      if (nparts == 1) {
-        const float inv = 1.0f / l_sum;
-        uint16_t* orow = p.o + (row0 + r) * p.ld_o + (int64_t)hh * kD;
-#pragma unroll 1
-        for (int c = 0; c < kD / 32; ++c) {
-          uint32_t ro[32];
-          tmem_ld32(o_t + c * 32, ro);
-          tmem_wait_ld();
-          if (row_valid) {
-            uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+    const bool done =
+        ok && warp_all(mbar_wait(&pv_done[wg], (uint32_t)(nt - 1) & 1u, abort_flag, p.status));
+    if (done) tc_fence_after();
+    // Both heads meet here once: after it every MMA has retired, so the Q/K/V/bias
+    // shared memory is free for staging, whatever path follows (all CTA-uniform).
+    const bool all_done = named_bar_and(1, 256, done);
+    const bool elected = warp == 4 && lane == 0;
+    // A full query tile lies inside its request: its bf16 output goes through shared
+    // memory (128-byte swizzle, two 64-column boxes per head) and TMA stores.  A
+    // request's ragged last tile stores rows directly (a full box would reach into the
+    // next request's rows).
+    const bool full_tile = q0 + kBM <= n_b;
+    unsigned char* out_head = smem + kEpiOut + wg * 2 * kBoxBytes;
+    auto put_chunk = [&](int c, const float (&acc)[32], float inv) {
+      uint32_t w[16];
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-              uint4 w;
-              w.x = pack_bf16x2(__uint_as_float(ro[u * 8 + 0]) * inv, __uint_as_float(ro[u * 8 + 1]) * inv);
-              w.y = pack_bf16x2(__uint_as_float(ro[u * 8 + 2]) * inv, __uint_as_float(ro[u * 8 + 3]) * inv);
-              w.z = pack_bf16x2(__uint_as_float(ro[u * 8 + 4]) * inv, __uint_as_float(ro[u * 8 + 5]) * inv);
-              w.w = pack_bf16x2(__uint_as_float(ro[u * 8 + 6]) * inv, __uint_as_float(ro[u * 8 + 7]) * inv);
-              dst[u] = w;
-            }
-          }
+      for (int e = 0; e < 16; ++e) w[e] = pack_bf16x2(acc[2 * e] * inv, acc[2 * e + 1] * inv);
+      if (full_tile) {
+        unsigned char* box = out_head + (c >> 1) * kBoxBytes;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int k = (c & 1) * 4 + u;  // 16-byte chunk of the row inside its box
+          *reinterpret_cast<uint4*>(box + rit * 128 + ((k ^ (rit & 7)) << 4)) =
+              make_uint4(w[4 * u], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]);
         }
-        if (row_valid && p.lse)
-          p.lse[(int64_t)hh * p.k_total + row0 + r] = (m_run + log2f(l_sum)) * 0.69314718055994531f;
-      } else {
-        // split query tile: unnormalised O, row max and row sum for the combine kernel
-        float* part_base = p.part_ws + ((int64_t)item * p.n_q_heads + hh) * kPartFloats;
-        float4* ocol = reinterpret_cast<float4*>(part_base) + rit;
+      } else if (row_valid) {
+        uint4* dst = reinterpret_cast<uint4*>(p.o + (row0 + r) * p.ld_o + (int64_t)hh * kD + c * 32);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) dst[u] = make_uint4(w[4 * u], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]);
+      }
+    };
+    auto store_lse = [&](float M, float L) {
+      if (row_valid && p.lse)
+        p.lse[(int64_t)hh * p.k_total + row0 + r] = (M + log2f(L)) * 0.69314718055994531f;
+    };
+    // after every thread has put its chunks: the staged tile goes out by TMA
+    auto flush_out = [&]() {
+      fence_proxy_async_smem();
+      named_bar_sync(1, 256);
+      if (full_tile && elected) {
+        for (int h = 0; h < 2; ++h)
+          for (int bx = 0; bx < 2; ++bx)
+            tma_store_2d(&tmO, (h0 + h) * kD + 64 * bx, (int32_t)(row0 + q0),
+                         smem + kEpiOut + (h * 2 + bx) * kBoxBytes);
+        bulk_commit_group();
+      }
+    };
+    auto own_chunk = [&](int c, float (&x)[32]) {
+      uint32_t ro[32];
+      tmem_ld32(o_t + c * 32, ro);
+      tmem_wait_ld();
+#pragma unroll
+      for (int e = 0; e < 32; ++e) x[e] = __uint_as_float(ro[e]);
+    };
+
+    if (nparts == 1) {
+      if (all_done) {
+        const float inv = 1.0f / l_sum;
 #pragma unroll 1
         for (int c = 0; c < kD / 32; ++c) {
-          uint32_t ro[32];
-          tmem_ld32(o_t + c * 32, ro);
-          tmem_wait_ld();
+          float acc[32];
+          own_chunk(c, acc);
+          put_chunk(c, acc, inv);
+        }
+        store_lse(m_run, l_sum);
+        flush_out();
+      }
+    } else if (all_done) {
+      // Split query tile.  Each part counts its arrival; every part but the last to
+      // arrive publishes its partial result (unnormalised O, row max, row sum) with bulk
+      // stores and raises its ready flag; the last one merges all parts, summing in part
+      // order whichever part it is (so every run rounds alike):
+      //   M = max_i m_i, L = sum_i 2^(m_i - M) l_i, o = sum_i 2^(m_i - M) O_i / L.
+      // It waits only for parts that have already arrived and are just storing, so the
+      // wait always ends.
+      int* cnt = p.part_count + (int64_t)(item - part) * hg + head_grp;
+      if (elected) *last_part = atomicAdd(cnt, 1) == nparts - 1 ? 1 : 0;
+      named_bar_sync(1, 256);
+      float* blk_smem = reinterpret_cast<float*>(smem) + wg * kPartFloats;  // this head's block
+      auto blk = [&](int i, int h) {
+        return p.part_ws + ((int64_t)(item - part + i) * p.n_q_heads + h) * kPartFloats;
+      };
+      if (!*last_part) {
+        float4* ocol = reinterpret_cast<float4*>(blk_smem) + rit;
+#pragma unroll 1
+        for (int c = 0; c < kD / 32; ++c) {
+          float x[32];
+          own_chunk(c, x);
 #pragma unroll
           for (int u = 0; u < 8; ++u)
-            ocol[(c * 8 + u) * kBM] = make_float4(__uint_as_float(ro[4 * u]), __uint_as_float(ro[4 * u + 1]),
-                                                  __uint_as_float(ro[4 * u + 2]), __uint_as_float(ro[4 * u + 3]));
+            ocol[(c * 8 + u) * kBM] = make_float4(x[4 * u], x[4 * u + 1], x[4 * u + 2], x[4 * u + 3]);
         }
-        part_base[kBM * kD + rit] = m_run;
-        part_base[kBM * kD + kBM + rit] = l_sum;
+        blk_smem[kBM * kD + rit] = m_run;
+        blk_smem[kBM * kD + kBM + rit] = l_sum;
+        fence_proxy_async_smem();
+        named_bar_sync(1, 256);
+        if (elected) {
+          bulk_store(blk(part, h0), smem, kPartFloats * 4);
+          bulk_store(blk(part, h0 + 1), smem + kPartFloats * 4, kPartFloats * 4);
+          bulk_commit_group();
+          bulk_wait_all();          // the partial is in global memory
+          fence_proxy_async_global();
+          st_release_gpu(p.part_ready + (int64_t)item * hg + head_grp, 1);
+        }
+      } else {
+        if (elected) {
+          bool ready = true;
+          for (int i = 0; i < nparts && ready; ++i)
+            if (i != part)
+              ready = wait_flag_gpu(p.part_ready + (int64_t)(item - part + i) * hg + head_grp,
+                                    abort_flag, p.status);
+          fence_proxy_async_global();  // the partials are read by bulk copies next
+          *parts_ready = ready ? 1 : 0;
+        }
+        named_bar_sync(1, 256);
+        const int np = nparts;
+        int copies = 0;
+        // stage part i's block (both heads) in shared memory; CTA-uniform outcome
+        auto stage = [&](int i) {
+          named_bar_sync(1, 256);  // nobody still reads the previous staged part
+          if (elected) {
+            fence_proxy_async_smem();
+            mbar_arrive_expect_tx(merge_full, 2 * kPartFloats * 4);
+            bulk_load(smem, blk(i, h0), kPartFloats * 4, merge_full);
+            bulk_load(smem + kPartFloats * 4, blk(i, h0 + 1), kPartFloats * 4, merge_full);
+          }
+          const bool got = named_bar_and(
+              1, 256, mbar_wait(merge_full, (uint32_t)copies & 1u, abort_flag, p.status));
+          ++copies;
+          return got;
+        };
+        bool ok_m = *parts_ready != 0;
+        if (ok_m && np == 2) {
+          // one other part: stage it, then a single pass
+          const int other = 1 - part;
+          ok_m = stage(other);
+          if (ok_m) {
+            const float m_o = blk_smem[kBM * kD + rit], l_o = blk_smem[kBM * kD + kBM + rit];
+            const float M = fmaxf(m_run, m_o);
+            const float w_own = ex2_approx(m_run - M), w_o = ex2_approx(m_o - M);
+            const float w0 = part == 0 ? w_own : w_o, w1 = part == 0 ? w_o : w_own;
+            const float L = fmaf(w1, part == 0 ? l_o : l_sum, w0 * (part == 0 ? l_sum : l_o));
+            const float inv = 1.0f / L;
+            const float4* g = reinterpret_cast<const float4*>(blk_smem) + rit;
+#pragma unroll 1
+            for (int c = 0; c < kD / 32; ++c) {
+              float own[32], acc[32];
+              own_chunk(c, own);
+#pragma unroll
+              for (int u = 0; u < 8; ++u) {
+                const float4 x = g[(c * 8 + u) * kBM];
+                const float xs[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                  const float a0 = part == 0 ? own[4 * u + e] : xs[e];
+                  const float a1 = part == 0 ? xs[e] : own[4 * u + e];
+                  acc[4 * u + e] = fmaf(w1, a1, w0 * a0);
+                }
+              }
+              put_chunk(c, acc, inv);
+            }
+            store_lse(M, L);
+          }
+        } else if (ok_m) {
+          // several other parts: batch-load every row max and sum, then one pass per
+          // part in part order with the running sum kept in the TMEM columns S used
+          float mi[kMaxParts], li[kMaxParts];
+#pragma unroll
+          for (int i = 0; i < kMaxParts; ++i) {
+            if (i < np) {
+              mi[i] = i == part ? m_run : __ldcg(blk(i, hh) + kBM * kD + rit);
+              li[i] = i == part ? l_sum : __ldcg(blk(i, hh) + kBM * kD + kBM + rit);
+            }
+          }
+          float M = -INFINITY;
+#pragma unroll
+          for (int i = 0; i < kMaxParts; ++i)
+            if (i < np) M = fmaxf(M, mi[i]);
+          float L = 0.f;
+#pragma unroll
+          for (int i = 0; i < kMaxParts; ++i) {
+            if (i < np) {
+              mi[i] = ex2_approx(mi[i] - M);  // from here on: the part's weight
+              L = i == 0 ? mi[i] * li[i] : fmaf(mi[i], li[i], L);
+            }
+          }
+          const float inv = 1.0f / L;
+#pragma unroll 1
+          for (int i = 0; i < np && ok_m; ++i) {
+            float w = mi[0];
+#pragma unroll
+            for (int t = 1; t < kMaxParts; ++t)
+              if (t == i) w = mi[t];
+            if (i != part && !(ok_m = stage(i))) break;
+            const float4* g = reinterpret_cast<const float4*>(blk_smem) + rit;
+#pragma unroll 1
+            for (int c = 0; c < kD / 32; ++c) {
+              float acc[32];
+              if (i > 0) {
+                uint32_t ra[32];
+                tmem_ld32(s_t + c * 32, ra);
+                tmem_wait_ld();
+#pragma unroll
+                for (int e = 0; e < 32; ++e) acc[e] = __uint_as_float(ra[e]);
+              }
+              float x[32];
+              if (i == part) {
+                own_chunk(c, x);
+              } else {
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                  const float4 v4 = g[(c * 8 + u) * kBM];
+                  x[4 * u] = v4.x;
+                  x[4 * u + 1] = v4.y;
+                  x[4 * u + 2] = v4.z;
+                  x[4 * u + 3] = v4.w;
+                }
+              }
+#pragma unroll
+              for (int e = 0; e < 32; ++e) acc[e] = i == 0 ? w * x[e] : fmaf(w, x[e], acc[e]);
+              if (i == np - 1) {
+                put_chunk(c, acc, inv);
+              } else {
+                uint32_t wa[32];
+#pragma unroll
+                for (int e = 0; e < 32; ++e) wa[e] = __float_as_uint(acc[e]);
+                tmem_st32(s_t + c * 32, wa);
+                tmem_wait_st();
+              }
+            }
+          }
+          if (ok_m) store_lse(M, L);
+        }
+        // after an abort: the last staged copy may still be landing in shared memory
+        if (!ok_m && copies > 0 && elected)
+          mbar_wait(merge_full, (uint32_t)(copies - 1) & 1u, nullptr, p.status);
+        const int ok_all = named_bar_and(1, 256, ok_m);
+        if (ok_all) flush_out();
+        named_bar_sync(1, 256);  // every read of the partials is done
+        if (elected) {  // leave the counters zeroed for the next call
+          for (int i = 0; i < nparts; ++i)
+            p.part_ready[(int64_t)(item - part + i) * hg + head_grp] = 0;
+          *cnt = 0;
+        }
       }
     }
+    if (elected) bulk_wait_all();  // TMA/bulk stores have read shared memory and landed
     tc_fence_before();
   }
   __syncthreads();
@@ -522,54 +741,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
-}
-
-// Merge the parts of split query tiles: per row, m = max_i m_i, L = sum_i 2^(m_i - m) l_i,
-// o = sum_i 2^(m_i - m) O_i / L.  One CTA per (work item, q head) and 128 threads, one
-// per row (only the first part's CTA of a split tile works); with the column-group
-// layout above every load and store of a warp is contiguous.
-constexpr int kMaxParts = 64;
-__global__ void __launch_bounds__(128) combine_parts_kernel(const __grid_constant__ AttnParams p) {
-  griddep_wait();
-  const int item = blockIdx.x, hh = blockIdx.y;
-  int b, qt, part, nparts;
-  decode_item(p, item, b, qt, part, nparts);
-  if (nparts == 1 || part != 0) return;
-  const int64_t row0 = p.cu_kept[b];
-  const int n_b = p.cu_kept[b + 1] - p.cu_kept[b];
-  const int rit = threadIdx.x;
-  const int r = qt * kBM + rit;
-  if (r >= n_b) return;
-  const int np = nparts < kMaxParts ? nparts : kMaxParts;
-  const int64_t stride = (int64_t)p.n_q_heads * kPartFloats;  // floats between parts
-  const float* base0 = p.part_ws + ((int64_t)item * p.n_q_heads + hh) * kPartFloats;
-  float m = -INFINITY;
-  for (int i = 0; i < np; ++i) m = fmaxf(m, base0[i * stride + kBM * kD + rit]);
-  float L = 0.f;
-  float w[kMaxParts];
-  for (int i = 0; i < np; ++i) {
-    w[i] = exp2f(base0[i * stride + kBM * kD + rit] - m);
-    L += w[i] * base0[i * stride + kBM * kD + kBM + rit];
-  }
-  const float inv = 1.0f / L;
-  uint4* orow = reinterpret_cast<uint4*>(p.o + (row0 + r) * p.ld_o + (int64_t)hh * kD);
-#pragma unroll 1
-  for (int f = 0; f < kD / 4; f += 2) {
-    float4 a = make_float4(0.f, 0.f, 0.f, 0.f), c = a;
-    for (int i = 0; i < np; ++i) {
-      const float4* g = reinterpret_cast<const float4*>(base0 + i * stride) + rit;
-      const float4 x = g[f * kBM], y = g[(f + 1) * kBM];
-      a.x += w[i] * x.x; a.y += w[i] * x.y; a.z += w[i] * x.z; a.w += w[i] * x.w;
-      c.x += w[i] * y.x; c.y += w[i] * y.y; c.z += w[i] * y.z; c.w += w[i] * y.w;
-    }
-    uint4 out;
-    out.x = pack_bf16x2(a.x * inv, a.y * inv);
-    out.y = pack_bf16x2(a.z * inv, a.w * inv);
-    out.z = pack_bf16x2(c.x * inv, c.y * inv);
-    out.w = pack_bf16x2(c.z * inv, c.w * inv);
-    orow[f / 2] = out;
-  }
-  if (p.lse) p.lse[(int64_t)hh * p.k_total + row0 + r] = (m + log2f(L)) * 0.69314718055994531f;
 }
 
 // Work plan: the key-tile chunk per item and the item count per request, chosen to
@@ -633,7 +804,7 @@ int make_plan(const int32_t* cu_kept_host, int batch, int head_groups, int sms, 
     double best_cost = simulate_makespan(cu_kept_host, batch, head_groups, sms, best);
     for (double f : {0.5, 0.75, 1.0, 1.25, 1.5, 2.0, 3.0}) {
       const int c = (int)std::ceil(share * f);
-      if (c < 2 || c >= max_tiles) continue;
+      if (c < 2 || c >= max_tiles || ceil_div(max_tiles, c) > kMaxParts) continue;
       const double cost = simulate_makespan(cu_kept_host, batch, head_groups, sms, c) + 1.0;
       if (cost < best_cost) {
         best_cost = cost;
@@ -657,6 +828,16 @@ int make_plan(const int32_t* cu_kept_host, int batch, int head_groups, int sms, 
   }
   plan.n_items = (int)items;
   return TG_OK;
+}
+
+// Split workspace: the parts' partial results, then at a 256-byte boundary two int32
+// arrays indexed by (work item, head group): arrival counters (used at a tile's first
+// item) and ready flags.
+size_t part_bytes(int64_t n_items, int n_q_heads) {
+  return ((size_t)n_items * n_q_heads * kPartFloats * sizeof(float) + 255) & ~size_t(255);
+}
+size_t split_workspace_bytes(int64_t n_items, int n_q_heads, int head_groups) {
+  return part_bytes(n_items, n_q_heads) + 2 * (size_t)n_items * head_groups * sizeof(int32_t);
 }
 
 // The register split above assumes the kernel is launched with kLaunchRegs registers
@@ -692,7 +873,7 @@ extern "C" size_t tg_gated_attention_workspace_size(const int32_t* cu_kept_host,
   if (make_plan(cu_kept_host, batch, n_q_heads / 2, sm_count(), plan, prefix) != TG_OK ||
       !plan.split)
     return 0;
-  return (size_t)plan.n_items * n_q_heads * kPartFloats * sizeof(float);
+  return split_workspace_bytes(plan.n_items, n_q_heads, n_q_heads / 2);
 }
 
 extern "C" int tg_gated_attention(const tg_bf16* q, int64_t ld_q, const tg_bf16* k, int64_t ld_k,
@@ -731,7 +912,7 @@ extern "C" int tg_gated_attention(const tg_bf16* q, int64_t ld_q, const tg_bf16*
   const int head_groups = n_kv_heads * (group / 2);
   AttnPlan plan;
   TG_TRY(make_plan(cu_kept_host, batch, head_groups, sm_count(), plan, prm.item_prefix));
-  const size_t need = (size_t)plan.n_items * n_q_heads * kPartFloats * sizeof(float);
+  const size_t need = split_workspace_bytes(plan.n_items, n_q_heads, head_groups);
   if (plan.split && (!workspace || workspace_bytes < need)) {
     // no room for partial results: one item per query tile
     int max_tiles = 1;
@@ -747,10 +928,11 @@ extern "C" int tg_gated_attention(const tg_bf16* q, int64_t ld_q, const tg_bf16*
     plan.n_items = items;
   }
 
-  CUtensorMap tq, tk, tv;
+  CUtensorMap tq, tk, tv, to;
   TG_TRY(make_tmap_bf16_2d(&tq, q, (uint64_t)k_total, (uint64_t)n_q_heads * kD, (uint64_t)ld_q, 64, kBM));
   TG_TRY(make_tmap_bf16_2d(&tk, k, (uint64_t)k_total, (uint64_t)n_kv_heads * kD, (uint64_t)ld_k, 64, kBN));
   TG_TRY(make_tmap_bf16_2d(&tv, v, (uint64_t)k_total, (uint64_t)n_kv_heads * kD, (uint64_t)ld_v, 64, kBN));
+  TG_TRY(make_tmap_bf16_2d(&to, o, (uint64_t)k_total, (uint64_t)n_q_heads * kD, (uint64_t)ld_o, 64, kBM));
   prm.cu_kept = cu_kept;
   prm.kept_pos = kept_pos;
   prm.kept_bias = kept_bias;
@@ -768,13 +950,14 @@ extern "C" int tg_gated_attention(const tg_bf16* q, int64_t ld_q, const tg_bf16*
   prm.status = status;
   prm.chunk = plan.chunk;
   prm.part_ws = plan.split ? static_cast<float*>(workspace) : nullptr;
+  prm.part_count = plan.split ? reinterpret_cast<int*>(static_cast<unsigned char*>(workspace) +
+                                                       part_bytes(plan.n_items, n_q_heads))
+                              : nullptr;
+  prm.part_ready = plan.split ? prm.part_count + (int64_t)plan.n_items * head_groups : nullptr;
 
   const int64_t grid = (int64_t)plan.n_items * head_groups;
   if (grid > 0x7FFFFFFF) return TG_ERR_UNSUPPORTED_SHAPE;
   TG_TRY(launch(gated_attention_kernel, dim3((unsigned)grid), dim3(kThreads), AttnSmem::BYTES,
-                (cudaStream_t)stream, tq, tk, tv, prm));
-  if (plan.split)
-    TG_TRY(launch(combine_parts_kernel, dim3((unsigned)plan.n_items, (unsigned)n_q_heads),
-                  dim3(128), 0, (cudaStream_t)stream, prm));
+                (cudaStream_t)stream, tq, tk, tv, to, prm));
   return TG_OK;
 }

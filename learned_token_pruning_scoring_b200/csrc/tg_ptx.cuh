@@ -103,6 +103,32 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
   }
 }
 
+// Release store / bounded acquire wait on a 32-bit flag in global memory (GPU scope).
+__device__ __forceinline__ void st_release_gpu(int* flag, int v) {
+  asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(flag), "r"(v) : "memory");
+}
+__device__ __forceinline__ int ld_acquire_gpu(const int* flag) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(flag) : "memory");
+  return v;
+}
+// Wait until *flag != 0; gives up like mbar_wait (abort flag raised, or the time limit).
+__device__ __forceinline__ bool wait_flag_gpu(const int* flag, volatile int* abort_flag,
+                                              uint32_t* status) {
+  if (ld_acquire_gpu(flag)) return true;
+  const uint64_t t0 = global_timer_ns();
+  while (true) {
+    __nanosleep(64);
+    if (ld_acquire_gpu(flag)) return true;
+    if (abort_flag && *abort_flag) return false;
+    if (global_timer_ns() - t0 > TG_WAIT_LIMIT_NS) {
+      if (abort_flag) *abort_flag = 1;
+      if (status) atomicOr(status, TG_STATUS_TIMEOUT);
+      return false;
+    }
+  }
+}
+
 // Warp-uniform outcome of per-thread waits: warp-collective tcgen05 instructions that
 // follow must be executed by all 32 lanes or by none.
 __device__ __forceinline__ bool warp_all(bool ok) { return __all_sync(0xFFFFFFFFu, ok); }
@@ -111,6 +137,9 @@ __device__ __forceinline__ bool warp_all(bool ok) { return __all_sync(0xFFFFFFFF
 
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
 }
 
 // ------------------------------------------------------------------ TMA
@@ -128,6 +157,26 @@ __device__ __forceinline__ void tma_load_2d(void* smem_dst, const void* tmap, in
       " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_u32(smem_dst)),
       "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y), "r"(smem_u32(bar))
       : "memory");
+}
+
+// Contiguous bulk copy of `bytes` (multiple of 16; both addresses 16-byte aligned) from
+// global to this CTA's shared memory, completing that many transaction bytes on `bar`.
+__device__ __forceinline__ void bulk_load(void* smem_dst, const void* gsrc, uint32_t bytes,
+                                          uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(smem_dst)),
+      "l"(reinterpret_cast<uint64_t>(gsrc)), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
+// Contiguous bulk copy of `bytes` from this CTA's shared memory to global memory, tracked
+// by the issuing thread's bulk groups (same size and alignment rules as bulk_load).
+__device__ __forceinline__ void bulk_store(void* gdst, const void* smem_src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(
+                   reinterpret_cast<uint64_t>(gdst)),
+               "r"(smem_u32(smem_src)), "r"(bytes)
+               : "memory");
 }
 
 // The same load for a CTA pair: the box lands in this CTA's shared memory, and its bytes
