@@ -58,6 +58,7 @@ typedef void* tg_stream_t;  /* cudaStream_t */
 #define TG_STATUS_TIMEOUT 0x1u /* a bounded wait ran out; outputs of that call are invalid */
 #define TG_STATUS_BUDGET 0x2u  /* kept count K_b inconsistent with the prunable mask */
 #define TG_STATUS_BOUNDS 0x4u  /* a row index outside the source; that row was skipped */
+#define TG_STATUS_WORKSPACE 0x8u /* a split-attention workspace was not zero-filled */
 
 /* ------------------------------------------------------------------ utilities */
 
@@ -304,7 +305,14 @@ int tg_gated_attention(const tg_bf16* q, int64_t ld_q, const tg_bf16* k, int64_t
  * needs no split.  With a smaller or NULL workspace the call still runs, one CTA per
  * query tile and kv-head pair.  The workspace must be zero-filled before its first use
  * (the counters); every call that completes leaves it that way.  After a call that
- * raised TG_STATUS_TIMEOUT, zero it again before reusing it.
+ * raised TG_STATUS_TIMEOUT or TG_STATUS_WORKSPACE, zero it again before reusing it.
+ * Layout, for n_items work items and G = n_q_heads / 2 head groups (size = n_items *
+ * (n_q_heads * 66560 + 8 * G) bytes): the partial results (66560 bytes per item and q
+ * head), then int32 arrival counters [n_items][G], then int32 ready flags [n_items][G].
+ * A counter found outside [0, parts) sets TG_STATUS_WORKSPACE; that tile's parts then
+ * neither publish nor merge, so its output rows are left unwritten (and a part that
+ * already counted itself last waits for a flag that never comes, up to the bounded
+ * wait, and sets TG_STATUS_TIMEOUT).
  */
 size_t tg_gated_attention_workspace_size(const int32_t* cu_kept_host, int batch,
                                          int n_q_heads, int n_kv_heads, int head_dim);

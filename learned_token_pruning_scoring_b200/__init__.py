@@ -27,7 +27,7 @@ __all__ = [
     "tg_gate_score_noalloc", "tg_seq_rmsnorm", "tg_gather_rope", "tg_kv_compact", "tg_gated_attention", "tg_linear",
     "tg_status_clear", "tg_status_read", "tg_set_launch_overlap", "tg_get_launch_overlap",
     "GatedPrefill", "STATUS_TIMEOUT", "STATUS_BUDGET",
-    "STATUS_BOUNDS",
+    "STATUS_BOUNDS", "STATUS_WORKSPACE",
 ]
 
 lib = _lib.load()
@@ -35,6 +35,7 @@ lib = _lib.load()
 STATUS_TIMEOUT = 0x1
 STATUS_BUDGET = 0x2
 STATUS_BOUNDS = 0x4
+STATUS_WORKSPACE = 0x8
 
 # Kernel launches issued through this binding (a benchmark reads it to report how many
 # of the library's kernels ran in its timed region).

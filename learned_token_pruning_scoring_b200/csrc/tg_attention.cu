@@ -563,13 +563,24 @@ __global__ void __launch_bounds__(kThreads, 1)
       // It waits only for parts that have already arrived and are just storing, so the
       // wait always ends.
       int* cnt = p.part_count + (int64_t)(item - part) * hg + head_grp;
-      if (elected) *last_part = atomicAdd(cnt, 1) == nparts - 1 ? 1 : 0;
+      if (elected) {
+        const int before = atomicAdd(cnt, 1);
+        if (before < 0 || before >= nparts) {
+          // the counter did not start at zero: the workspace was not zero-filled
+          if (p.status) atomicOr(p.status, TG_STATUS_WORKSPACE);
+          *last_part = 2;  // neither publish nor merge
+        } else {
+          *last_part = before == nparts - 1 ? 1 : 0;
+        }
+      }
       named_bar_sync(1, 256);
       float* blk_smem = reinterpret_cast<float*>(smem) + wg * kPartFloats;  // this head's block
       auto blk = [&](int i, int h) {
         return p.part_ws + ((int64_t)(item - part + i) * p.n_q_heads + h) * kPartFloats;
       };
-      if (!*last_part) {
+      if (*last_part == 2) {
+        // corrupt workspace: nothing to do (status set above)
+      } else if (!*last_part) {
         float4* ocol = reinterpret_cast<float4*>(blk_smem) + rit;
 #pragma unroll 1
         for (int c = 0; c < kD / 32; ++c) {

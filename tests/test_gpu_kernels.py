@@ -424,6 +424,33 @@ def test_attention_deterministic(tg):
     assert torch.equal(a, b) and torch.equal(la, lb)
 
 
+def test_attention_dirty_workspace_times_out_and_reports(tg):
+    """Failure detection without a fault: a split workspace that was not zero-filled.
+    One tile's arrival counter starts at 1, so that tile's first part counts itself last
+    and waits for a ready flag that never comes (its other part sees the counter out of
+    range and publishes nothing).  The bounded wait runs out (about 2 s); the call
+    reports TIMEOUT | WORKSPACE and returns, and the next call on a clean workspace is
+    correct."""
+    import time
+    q, k, v, pos, bias, gamma, cu = _attn_inputs([1638], 16, 8, seed=4, pos_spread=10)
+    need = tg.tg_gated_attention_workspace_size(cu, 16, 8)
+    groups = 8
+    per_item = 16 * 66560 + 8 * groups   # partials for 16 q heads, counter + flag per group
+    assert need > 0 and need % per_item == 0
+    n_items = need // per_item
+    ws = torch.zeros(need, dtype=torch.uint8, device="cuda")
+    ws[n_items * 16 * 66560:].view(torch.int32)[0] = 1  # item 0 (a split tile), group 0
+    st = _status()
+    t0 = time.time()
+    tg.tg_gated_attention(_dev(q), _dev(k), _dev(v), _dev(torch.from_numpy(cu)), cu, 16, 8,
+                          _dev(pos), _dev(bias), _dev(gamma), 1.0, workspace=ws, status=st)
+    got = tg.tg_status_read(st)
+    assert got & tg.STATUS_TIMEOUT and got & tg.STATUS_WORKSPACE, hex(got)
+    assert time.time() - t0 < 30
+    o, lse = _run_attention(tg, q, k, v, pos, bias, gamma, 1.0, cu, 16, 8)
+    _check_attention(o, lse, q, k, v, pos, bias, gamma, 1.0, cu, 16, 8)
+
+
 # ------------------------------------------------------------------ fused QKV + RoPE + cache
 
 @pytest.mark.parametrize("M", [1, 257, 1638])
