@@ -282,7 +282,11 @@ int tg_kv_compact(const tg_bf16* k, int64_t ld_k, const tg_bf16* v, int64_t ld_v
  * q: bf16 [K_tot, n_q_heads * head_dim] (row stride ld_q); k, v: bf16
  * [K_tot, n_kv_heads * head_dim] (ld_k, ld_v); o: bf16 [K_tot, n_q_heads * head_dim]
  * (ld_o).  lse: float32 [n_q_heads, K_tot] natural-log log-sum-exp, or NULL.
- * kept_pos int32 [K_tot]; kept_bias float32 [K_tot]; gamma float32 [n_q_heads].
+ * kept_pos int32 [K_tot]; kept_bias float32 [K_tot]; gamma float32 [n_q_heads]; beta
+ * finite and >= 0 (a temperature scale; otherwise TG_ERR_INVALID_ARGUMENT).
+ * The kernel adds the bias term inside the Q K^T MMA (an extra K=16 step whose columns
+ * hold gamma_h log2(e) / t_r and kept_bias, each split into two bf16 parts, t_r the
+ * row's log2-domain temperature factor), so logits keep fp32 accuracy.
  * Implemented for head_dim = 128 and an even group size n_q_heads / n_kv_heads; q, k,
  * v, o 16-byte aligned with strides that are multiples of 8; at most 512 requests per
  * call.  The kernel runs the two q heads of a kv head on tcgen05 tensor cores with S and

@@ -54,11 +54,28 @@ constexpr int kMaxBatch = 512;  // requests per call (tile table lives in the pa
 constexpr int kTileBytes = kBM * kD * 2;  // 32 KB: 128 rows x 128 bf16, two 64-column boxes
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleThreshold = 8.0f;
+
+// x ~ hi + lo with both parts bf16 (round to nearest): hi carries 8 significant bits,
+// lo the next 8.
+__device__ __forceinline__ void split_bf16(float x, uint16_t& hi, uint16_t& lo) {
+  const __nv_bfloat16 h = __float2bfloat16_rn(x);
+  const __nv_bfloat16 l = __float2bfloat16_rn(x - __bfloat162float(h));
+  hi = *reinterpret_cast<const uint16_t*>(&h);
+  lo = *reinterpret_cast<const uint16_t*>(&l);
+}
 constexpr int kMaxParts = 8;    // parts per split query tile
 constexpr int kBoxBytes = kBM * 64 * 2;  // one 64-column bf16 box of a 128-row tile
 // Epilogue staging (the Q/K/V/bias region is free once every MMA has retired): a split
 // part's block for both heads at 0, the bf16 output tile (2 heads x 2 boxes) after it.
 constexpr int kEpiOut = 2 * (kBM * kD + 2 * kBM) * 4;
+
+// Extra K columns of the S = Q K^T MMA that add the gate bias: a 128 x 16 bf16 operand
+// in the no-swizzle core-matrix layout (8-row x 16-byte core matrices; the two along K
+// 128 bytes apart, 8-row groups 256 bytes apart).
+constexpr int kExBytes = 128 * 16 * 2;
+__host__ __device__ constexpr int ex_off(int row, int chunk) {
+  return (row >> 3) * 256 + chunk * 128 + (row & 7) * 16;
+}
 
 struct AttnSmem {
   // 1024-aligned tiles first
@@ -66,8 +83,9 @@ struct AttnSmem {
   static constexpr int Q1 = Q0 + kTileBytes;
   static constexpr int K = Q1 + kTileBytes;
   static constexpr int V = K + kStages * kTileBytes;
-  static constexpr int BIAS = V + kStages * kTileBytes;    // [stage][head][kBN] fp32
-  static constexpr int BAR = BIAS + kStages * 2 * kBN * 4;
+  static constexpr int AEX = V + kStages * kTileBytes;  // [head] extra A columns (gain)
+  static constexpr int BEX = AEX + 2 * kExBytes;        // [stage] extra B columns (key bias)
+  static constexpr int BAR = BEX + kStages * kExBytes;
   static constexpr int END = BAR + 256;
   static constexpr int BYTES = END + 1024;  // alignment slack
 };
@@ -139,33 +157,25 @@ __device__ __forceinline__ void decode_item(const AttnParams& p, int t, int& b, 
   }
 }
 
-// Logits of one row for one key tile: l = s * t2 + b (pairs), written back into sv.
+// Row maximum of one key tile's logits; on the diagonal tile keys past the row are set
+// to -inf first.
 template <bool kDiag>
-__device__ __forceinline__ float logits_and_max(uint32_t (&sv)[kBN], const float* bsl,
-                                                float tau2, int rit) {
-  const uint64_t t2 = f2pack(tau2, tau2);
-  const float4* b4p = reinterpret_cast<const float4*>(bsl);
+__device__ __forceinline__ float row_max(uint32_t (&sv)[kBN], int rit) {
   float m0 = -INFINITY, m1 = -INFINITY, m2 = -INFINITY, m3 = -INFINITY;
 #pragma unroll
   for (int i = 0; i < kBN / 4; ++i) {
-    const float4 b4 = b4p[i];
-    const uint64_t l01 = fma2(f2pack(__uint_as_float(sv[4 * i]), __uint_as_float(sv[4 * i + 1])),
-                              t2, f2pack(b4.x, b4.y));
-    const uint64_t l23 = fma2(f2pack(__uint_as_float(sv[4 * i + 2]), __uint_as_float(sv[4 * i + 3])),
-                              t2, f2pack(b4.z, b4.w));
-    float a, b, c, d;
-    f2unpack(l01, a, b);
-    f2unpack(l23, c, d);
+    float a = __uint_as_float(sv[4 * i]), b = __uint_as_float(sv[4 * i + 1]);
+    float c = __uint_as_float(sv[4 * i + 2]), d = __uint_as_float(sv[4 * i + 3]);
     if (kDiag) {
       if (4 * i + 0 > rit) a = -INFINITY;
       if (4 * i + 1 > rit) b = -INFINITY;
       if (4 * i + 2 > rit) c = -INFINITY;
       if (4 * i + 3 > rit) d = -INFINITY;
+      sv[4 * i] = __float_as_uint(a);
+      sv[4 * i + 1] = __float_as_uint(b);
+      sv[4 * i + 2] = __float_as_uint(c);
+      sv[4 * i + 3] = __float_as_uint(d);
     }
-    sv[4 * i] = __float_as_uint(a);
-    sv[4 * i + 1] = __float_as_uint(b);
-    sv[4 * i + 2] = __float_as_uint(c);
-    sv[4 * i + 3] = __float_as_uint(d);
     if (i & 1) {
       m2 = max3(m2, a, b);
       m3 = max3(m3, c, d);
@@ -186,15 +196,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  float* bias_s = reinterpret_cast<float*>(smem + AttnSmem::BIAS);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + AttnSmem::BAR);
   uint64_t* q_full = bars + 0;
   uint64_t* k_full = bars + 1;             // [kStages]
   uint64_t* v_full = k_full + kStages;     // [kStages]
   uint64_t* k_empty = v_full + kStages;    // [kStages]
   uint64_t* v_empty = k_empty + kStages;   // [kStages]
-  uint64_t* b_full = v_empty + kStages;    // [kStages] key bias of the stage written
-  uint64_t* s_full = b_full + kStages;     // [2]
+  uint64_t* bx_full = v_empty + kStages;   // [kStages] extra bias columns of the stage written
+  uint64_t* ax_ready = bx_full + kStages;  // [2] the head's extra A columns written (per row)
+  uint64_t* s_full = ax_ready + 2;         // [2]
   uint64_t* p_full = s_full + 2;           // [2]
   uint64_t* pv_done = p_full + 2;          // [2]
   uint64_t* drain = pv_done + 2;
@@ -210,12 +220,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(q_full, 1);
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&k_full[s], 1);
-      mbar_init(&b_full[s], 1);
+      mbar_init(&bx_full[s], 1);
       mbar_init(&v_full[s], 1);
       mbar_init(&k_empty[s], 1);
       mbar_init(&v_empty[s], 1);
     }
     for (int h = 0; h < 2; ++h) {
+      mbar_init(&ax_ready[h], 128);
       mbar_init(&s_full[h], 1);
       mbar_init(&p_full[h], 128);
       mbar_init(&pv_done[h], 1);
@@ -260,7 +271,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     regs_dec<kRegsLow>();
     if (warp == 0) {
       // ---------------------------------------------------------- producer
-      const float gb0 = p.gamma[h0] * kLog2e, gb1 = p.gamma[h0 + 1] * kLog2e;
       int loaded = 0, loaded_v = 0;
       bool q_issued = false;
       if (lane == 0) {
@@ -295,8 +305,25 @@ __global__ void __launch_bounds__(kThreads, 1)
           tma_load_2d(kt, &tmK, g * kD, y, &k_full[s]);
           tma_load_2d(kt + kTileBytes / 2, &tmK, g * kD + 64, y, &k_full[s]);
         }
-        // V and the key bias of tile j once both heads' PV MMAs of tile j - kStages are
-        // done (the PV MMAs follow both softmaxes of that tile, the bias's only readers)
+        // Extra B columns of the tile's keys: (b_hi, b_lo, b_hi, 0, ...); with a row's
+        // (g_hi, g_hi, g_lo, 0, ...) the MMA adds g_hi b_hi + g_hi b_lo + g_lo b_hi, i.e.
+        // g * b to ~2^-16 relative
+        {
+          unsigned char* bx = smem + AttnSmem::BEX + s * kExBytes;
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            uint16_t b_hi, b_lo;
+            split_bf16(bv[e], b_hi, b_lo);
+            const int key = lane * 4 + e;
+            *reinterpret_cast<uint4*>(bx + ex_off(key, 0)) =
+                make_uint4((uint32_t)b_hi | ((uint32_t)b_lo << 16), b_hi, 0u, 0u);
+            *reinterpret_cast<uint4*>(bx + ex_off(key, 1)) = make_uint4(0u, 0u, 0u, 0u);
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&bx_full[s]);
+        }
+        // V of tile j once both heads' PV MMAs of tile j - kStages are done
         if (!warp_all(mbar_wait(&v_empty[s], ph ^ 1u, abort_flag, p.status))) {
           ++loaded;
           break;
@@ -307,12 +334,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           tma_load_2d(vt, &tmV, g * kD, y, &v_full[s]);
           tma_load_2d(vt + kTileBytes / 2, &tmV, g * kD + 64, y, &v_full[s]);
         }
-        float4* b0 = reinterpret_cast<float4*>(bias_s + (s * 2 + 0) * kBN) + lane;
-        float4* b1 = reinterpret_cast<float4*>(bias_s + (s * 2 + 1) * kBN) + lane;
-        *b0 = make_float4(bv[0] * gb0, bv[1] * gb0, bv[2] * gb0, bv[3] * gb0);
-        *b1 = make_float4(bv[0] * gb1, bv[1] * gb1, bv[2] * gb1, bv[3] * gb1);
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&b_full[s]);
         load_bias(j + 1, bv);
         ++loaded;
         ++loaded_v;
@@ -338,6 +359,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                                     sw128_desc(smem_u32(smem + AttnSmem::Q1), 16, 1024)};
         const uint64_t k_desc0 = sw128_desc(smem_u32(smem + AttnSmem::K), 16, 1024);
         const uint64_t v_desc0 = sw128_desc(smem_u32(smem + AttnSmem::V), kTileBytes / 2, 1024);
+        // extra K columns (gate bias): core matrices 128 bytes apart along K, 8-row groups
+        // 256 bytes apart
+        const uint64_t ax_desc[2] = {
+            interleave_desc(smem_u32(smem + AttnSmem::AEX), 128, 256),
+            interleave_desc(smem_u32(smem + AttnSmem::AEX + kExBytes), 128, 256)};
+        const uint64_t bx_desc0 = interleave_desc(smem_u32(smem + AttnSmem::BEX), 128, 256);
         const uint32_t s_col[2] = {0u, 128u};
         const uint32_t o_col[2] = {256u, 384u};
         auto issue_s = [&](int hh, int j) {
@@ -347,6 +374,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint64_t off = (uint64_t)(((kk >> 2) * (kTileBytes / 2) + (kk & 3) * 32) >> 4);
             mma_ss(tmem + s_col[hh], q_desc[hh] + off, kd + off, idesc_s, kk != 0);
           }
+          // + (gamma_h * log2(e) / t_r) * bias_c, one more K=16 step on the extra columns
+          mma_ss(tmem + s_col[hh], ax_desc[hh],
+                 bx_desc0 + (uint64_t)(((j % kStages) * kExBytes) >> 4), idesc_s, 1u);
           mma_commit(&s_full[hh]);
         };
         auto issue_pv = [&](int hh, int j) {
@@ -360,7 +390,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           mma_commit(&pv_done[hh]);
         };
         bool ok = mbar_wait(q_full, 0, abort_flag, p.status) &&
-                  mbar_wait(&k_full[0], 0, abort_flag, p.status);
+                  mbar_wait(&ax_ready[0], 0, abort_flag, p.status) &&
+                  mbar_wait(&ax_ready[1], 0, abort_flag, p.status) &&
+                  mbar_wait(&k_full[0], 0, abort_flag, p.status) &&
+                  mbar_wait(&bx_full[0], 0, abort_flag, p.status);
         if (ok) {
           tc_fence_after();
           issue_s(0, 0);
@@ -379,7 +412,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (more) {
               const int s2 = (j + 1) % kStages;
               const uint32_t ph2 = (uint32_t)((j + 1) / kStages) & 1u;
-              if (!(ok = mbar_wait(&k_full[s2], ph2, abort_flag, p.status))) break;
+              if (!(ok = mbar_wait(&k_full[s2], ph2, abort_flag, p.status) &&
+                         mbar_wait(&bx_full[s2], ph2, abort_flag, p.status)))
+                break;
               tc_fence_after();
               issue_s(0, j + 1);
             }
@@ -417,6 +452,24 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     const float tau2 = (float)(tau / sqrt((double)kD) * 1.4426950408889634);
 
+    // The logit in the log2 domain is t * S with t = tau_r * log2(e) / sqrt(d) and
+    // S = q.k + (gamma_h * log2(e) / t) * bias_c: the tensor core adds the bias term
+    // through one extra K=16 step whose A columns, per row, hold g = gamma_h log2(e) / t
+    // split into bf16 parts (g_hi, g_hi, g_lo).  t >= 0 (beta >= 0); t = 0 (first kept
+    // token of a request whose position is not 0) is taken as 2^-66, which leaves
+    // t * S = gamma_h log2(e) bias_c.
+    const float t2 = fmaxf(tau2, 0x1p-66f);
+    {
+      uint16_t g_hi, g_lo;
+      split_bf16(p.gamma[hh] * kLog2e / t2, g_hi, g_lo);
+      unsigned char* ax = smem + AttnSmem::AEX + wg * kExBytes;
+      *reinterpret_cast<uint4*>(ax + ex_off(rit, 0)) =
+          make_uint4((uint32_t)g_hi | ((uint32_t)g_hi << 16), g_lo, 0u, 0u);
+      *reinterpret_cast<uint4*>(ax + ex_off(rit, 1)) = make_uint4(0u, 0u, 0u, 0u);
+      fence_proxy_async_smem();  // read by the tensor core
+      mbar_arrive(&ax_ready[wg]);
+    }
+
     float m_run = -INFINITY, l_sum = 0.f;
     bool ok = true;
     for (int j = 0; j < nt; ++j) {
@@ -428,12 +481,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tmem_ld32(s_t + 64, *reinterpret_cast<uint32_t(*)[32]>(&sv[64]));
       tmem_ld32(s_t + 96, *reinterpret_cast<uint32_t(*)[32]>(&sv[96]));
       tmem_wait_ld();
-      if (!(ok = warp_all(mbar_wait(&b_full[j % kStages], (uint32_t)(j / kStages) & 1u, abort_flag,
-                                    p.status))))
-        break;
-      const float* bsl = bias_s + ((j % kStages) * 2 + wg) * kBN;
-      const float mx = (j0 + j == qt) ? logits_and_max<true>(sv, bsl, tau2, rit)
-                                 : logits_and_max<false>(sv, bsl, tau2, rit);
+      const float mx = t2 * ((j0 + j == qt) ? row_max<true>(sv, rit) : row_max<false>(sv, rit));
       // Lazy rescale: move the running max only when it grows by more than 2^8.
       float alpha = 1.0f;
       bool rescale = false;
@@ -445,6 +493,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         rescale = true;
       }
       const uint64_t negm = f2pack(-m_run, -m_run);
+      const uint64_t t2p = f2pack(t2, t2);
       uint64_t acc0 = f2pack(0.f, 0.f), acc1 = acc0;
 #pragma unroll
       for (int hf = 0; hf < 2; ++hf) {
@@ -452,7 +501,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
           const int e = 64 * hf + 2 * i;
-          const uint64_t d = add2(f2pack(__uint_as_float(sv[e]), __uint_as_float(sv[e + 1])), negm);
+          const uint64_t d = fma2(f2pack(__uint_as_float(sv[e]), __uint_as_float(sv[e + 1])), t2p, negm);
           float x0, x1;
           f2unpack(d, x0, x1);
           const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
@@ -915,7 +964,7 @@ extern "C" int tg_gated_attention(const tg_bf16* q, int64_t ld_q, const tg_bf16*
       !stride_ok(ld_k, 2) || !stride_ok(ld_v, 2) || !stride_ok(ld_o, 2))
     return TG_ERR_MISALIGNED;
   if (workspace && !aligned16(workspace)) return TG_ERR_MISALIGNED;
-  if (!std::isfinite(beta)) return TG_ERR_INVALID_ARGUMENT;
+  if (!std::isfinite(beta) || beta < 0.f) return TG_ERR_INVALID_ARGUMENT;
   TG_TRY(check_device());
   TG_TRY(check_register_budget());
 

@@ -413,6 +413,19 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t smem_addr, uint32_t lbo_
   return d;
 }
 
+// Shared-memory matrix descriptor without swizzle: 8-row x 16-byte core matrices,
+// `lbo_bytes` between core matrices adjacent along K, `sbo_bytes` between adjacent
+// 8-row groups (K-major operand).
+__device__ __forceinline__ uint64_t interleave_desc(uint32_t smem_addr, uint32_t lbo_bytes,
+                                                    uint32_t sbo_bytes) {
+  uint64_t d = 0;
+  d |= (uint64_t)((smem_addr & 0x3FFFFu) >> 4);
+  d |= (uint64_t)((lbo_bytes >> 4) & 0x3FFFu) << 16;
+  d |= (uint64_t)((sbo_bytes >> 4) & 0x3FFFu) << 32;
+  d |= (uint64_t)1 << 46;  // descriptor version for tcgen05; layout 0 = no swizzle
+  return d;
+}
+
 // Instruction descriptor: bf16 x bf16 -> f32, shape M x N, operand majors.
 __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool a_mn_major,
                                                       bool b_mn_major) {

@@ -75,6 +75,10 @@ def test_host_side_argument_errors(lib):
     # attention: odd GQA group
     assert lib.tg_gated_attention(p, 2048, p, 1024, p, 1024, p, cu, 1, 3, 3, 128, p, p, p,
                                   1.0, p, 2048, None, None, 0, None, None) == -6
+    # attention: the temperature scale beta must be finite and non-negative
+    for beta in (-0.5, float("nan"), float("inf")):
+        assert lib.tg_gated_attention(p, 2048, p, 1024, p, 1024, p, cu, 1, 16, 8, 128, p, p, p,
+                                      beta, p, 2048, None, None, 0, None, None) == -1
     # projections: N not a multiple of 128, K not a multiple of 64
     assert lib.tg_linear(p, 64, p, 64, p, 100, 4, 100, 64, 0, 0.0, None, 0, None, 0, None,
                          None) == -6
