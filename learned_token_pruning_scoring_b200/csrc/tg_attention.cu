@@ -11,21 +11,24 @@
 //   logit[r, c] = tau_r * q_r.k_c / sqrt(d) + gamma_h * bias_c   (c <= r, same request)
 //   tau_r = beta * ln(r + 1) / ln(p_r + 1), tau_r = beta when p_r = 0.
 //
-// One CTA = one request, one tile of 128 query ranks, one kv head and the two q
-// heads (h0, h0 + 1) that read it.  Tensor memory (512 columns):
+// One CTA = one request, one tile of 128 query ranks, one share of its causal key range
+// (split-KV, see the plan below), one kv head and the two q heads (h0, h0 + 1) that read
+// it.  Tensor memory (512 columns):
 //   S0/P0 [0,128)  S1/P1 [128,256)  O0 [256,384)  O1 [384,512)
 // Warpgroup 0 (warps 0-3, registers lowered to 120): warp 0 loads Q once and then K/V
-// tiles through a 2-stage TMA ring (a K stage is released as soon as both heads' S
-// MMAs have read it, a V stage after both PV MMAs), and with each V the tile's key bias
-// pre-scaled by gamma_h * log2(e) for each of the two heads; warp 1 issues S = Q K^T (both operands
-// in shared memory) and O += P V (P read from TMEM, V an MN-major shared operand).
+// tiles through a 2-stage TMA ring (a K stage is released once both heads' S MMAs have
+// read it, a V stage after both PV MMAs) and writes each tile's key bias as two extra
+// bf16 K columns; warp 1 issues S = Q K^T + (one more K=16 step) gain x bias, both
+// operands in shared memory, and O += P V (P read from TMEM, V an MN-major shared
+// operand).
 // Warpgroups 1 and 2 (registers raised to 192) are the softmax of head h0 and h0 + 1,
-// one thread per query row: the logits tau * s * log2(e) / sqrt(d) + bias come from
-// one packed fp32x2 FMA per pair, the row max from 3-input max, 2^(l - m) from the
-// MUFU unit, the row sum from packed adds, and P goes back to TMEM as bf16.  Masking
-// is only applied on the diagonal tile.  The running max moves (and O is rescaled in
-// TMEM) only when it grows by more than 2^8, which keeps P inside bf16 range.  The two
-// heads ping-pong on the tensor core: while one softmax runs the MMA works on the other.
+// one thread per query row.  S from TMEM is the row's logit divided by its temperature
+// factor t = tau * log2(e) / sqrt(d) (the extra MMA step adds gamma * log2(e) / t times
+// the bias), so the softmax takes the row max of S, forms t * S - m with one packed
+// fp32x2 FMA per two keys, exponentiates on the MUFU unit, sums in packed pairs and
+// stores P to TMEM as bf16.  Masking is only applied on the diagonal tile.  The running
+// max moves (and O is rescaled in TMEM) only when it grows by more than 2^8, which keeps
+// P inside bf16 range.  The two heads ping-pong on the tensor core.
 #include <cuda.h>
 
 #include <algorithm>
