@@ -94,6 +94,13 @@ int tg_status_read(const uint32_t* status, uint32_t* out_host, tg_stream_t strea
 int tg_set_launch_overlap(int enable);
 int tg_get_launch_overlap(void);
 
+/* L2 prefetch hint (not part of the method): issue bulk prefetches that bring
+ * [ptr, ptr + bytes) into the L2 cache ahead of a later kernel that reads it (the
+ * next layer's weights while attention runs, for instance).  Nothing waits for the
+ * data and results never depend on it.  ptr 16-byte aligned; bytes is rounded down to a
+ * multiple of 16 (0 does nothing).  Asynchronous on `stream`; one small kernel launch. */
+int tg_prefetch_l2(const void* ptr, size_t bytes, tg_stream_t stream);
+
 /*
  * Rotary table for original-position RoPE ([aiwillknow] figure 1(a)(b): kept tokens
  * keep their original position encoding).  Writes cos_sin[p][i][0] = cos(p * f_i),

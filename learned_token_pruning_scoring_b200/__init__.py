@@ -26,6 +26,7 @@ __all__ = [
     "tg_rope_table", "tg_gate_score_workspace_size", "tg_gate_score", "tg_topk_compact",
     "tg_gate_score_noalloc", "tg_seq_rmsnorm", "tg_gather_rope", "tg_kv_compact", "tg_gated_attention", "tg_linear",
     "tg_status_clear", "tg_status_read", "tg_set_launch_overlap", "tg_get_launch_overlap",
+    "tg_prefetch_l2",
     "GatedPrefill", "STATUS_TIMEOUT", "STATUS_BUDGET",
     "STATUS_BOUNDS", "STATUS_WORKSPACE",
 ]
@@ -102,6 +103,15 @@ def tg_set_launch_overlap(enable: bool) -> None:
 
 def tg_get_launch_overlap() -> bool:
     return bool(lib.tg_get_launch_overlap())
+
+
+def tg_prefetch_l2(t: torch.Tensor, stream=None) -> None:
+    """Bring a contiguous device tensor into L2 ahead of its use (a hint)."""
+    if not t.is_contiguous():
+        raise ValueError("tg_prefetch_l2 needs a contiguous tensor")
+    _check(lib.tg_prefetch_l2(_ptr(t), t.numel() * t.element_size(), _stream(stream)),
+           "tg_prefetch_l2")
+    _count()
 
 
 def tg_status_read(status: torch.Tensor, stream=None) -> int:
@@ -363,6 +373,11 @@ class GatedPrefill:
         self.marker = None
         # QKV projection, RoPE and KV-cache write as one fused kernel (else three)
         self.fused_qkv = True
+        # optional: while layer i's attention runs, a side stream pulls that layer's Wo
+        # and the next layer's Wqkv into L2 (measured slower on the 16k and 128k steps:
+        # off by default)
+        self.prefetch_weights = False
+        self._side = None
 
     def _mark(self, name):
         if self.marker is not None:
@@ -452,6 +467,14 @@ class GatedPrefill:
             tg_kv_compact(qkv[:, nq:nq + nk], qkv[:, nq + nk:], ck, cv, status=self.status,
                           stream=stream)
             self._mark("kv_compact")
+        if self.prefetch_weights:
+            main = stream if stream is not None else torch.cuda.current_stream(self.device)
+            if self._side is None:
+                self._side = torch.cuda.Stream(device=self.device)
+            self._side.wait_stream(main)
+            tg_prefetch_l2(L.Wo, stream=self._side)
+            if i + 1 < len(self.layers):
+                tg_prefetch_l2(self.layers[i + 1].Wqkv, stream=self._side)
         tg_gated_attention(qkv[:, :nq], ck, cv, P["ck"], P["ck_h"], self.hq, self.hkv,
                            P["kept_pos"], P["kept_bias"], L.gamma, L.beta, o=o,
                            head_dim=self.d, workspace=P["attn_ws"], status=self.status,
@@ -464,6 +487,9 @@ class GatedPrefill:
         self.gather(h, stream=stream)
         for i in range(len(self.layers)):
             self.layer(i, stream=stream)
+        if self._side is not None:  # join the prefetch stream (a captured graph needs it)
+            main = stream if stream is not None else torch.cuda.current_stream(self.device)
+            main.wait_stream(self._side)
 
     def run(self, h, prunable, scores=None, stream=None):
         """One gated prefill step.  The scorer always runs on h; with `scores` (raw

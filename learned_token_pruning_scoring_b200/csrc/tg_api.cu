@@ -161,3 +161,42 @@ int tg_status_read(const uint32_t* status, uint32_t* out_host, tg_stream_t strea
 }
 
 }  // extern "C"
+
+// ------------------------------------------------------------------ L2 prefetch
+
+namespace tg {
+namespace {
+
+constexpr uint32_t kPrefetchChunk = 32768;
+
+// One thread per 32 KB chunk: a bulk L2 prefetch (a hint with no completion to wait for).
+__global__ void prefetch_l2_kernel(const unsigned char* base, uint64_t bytes) {
+  const uint64_t chunk = (uint64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const uint64_t off = chunk * kPrefetchChunk;
+  if (off >= bytes) return;
+  const uint64_t left = bytes - off;
+  const uint32_t n = left < kPrefetchChunk ? (uint32_t)left : kPrefetchChunk;
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(
+                   reinterpret_cast<uint64_t>(base + off)),
+               "r"(n)
+               : "memory");
+}
+
+}  // namespace
+}  // namespace tg
+
+extern "C" int tg_prefetch_l2(const void* ptr, size_t bytes, tg_stream_t stream) {
+  using namespace tg;
+  if (bytes == 0) return TG_OK;
+  if (!ptr) return TG_ERR_INVALID_ARGUMENT;
+  if (!aligned16(ptr)) return TG_ERR_MISALIGNED;
+  const uint64_t n = (uint64_t)bytes & ~uint64_t(15);  // the bulk unit is 16 bytes
+  if (n == 0) return TG_OK;
+  TG_TRY(check_device());
+  const uint64_t chunks = (n + kPrefetchChunk - 1) / kPrefetchChunk;
+  const uint64_t blocks = (chunks + 127) / 128;
+  if (blocks > 0x7FFFFFFFull) return TG_ERR_UNSUPPORTED_SHAPE;
+  prefetch_l2_kernel<<<(unsigned)blocks, 128, 0, (cudaStream_t)stream>>>(
+      static_cast<const unsigned char*>(ptr), n);
+  return check_launch();
+}

@@ -27,7 +27,12 @@ namespace {
 
 constexpr int kWidth = 256;
 constexpr int kNormThreads = 256;
-constexpr int kNormRowsPerCta = 8192;
+// Rows written per CTA.  Every CTA of a request recomputes the request's sum of squares
+// (in a fixed order, so all agree bit for bit): from the 32-row chunk sums that is cheap
+// and small CTAs spread the work; without chunk sums each CTA rereads the whole request,
+// so there the CTAs stay large.
+constexpr int kNormRowsPerCta = 512;
+constexpr int kNormRowsPerCtaNoPartials = 8192;
 
 __global__ void fold_norm_kernel(const uint16_t* __restrict__ W1, const float* __restrict__ w,
                                  uint16_t* __restrict__ out, int width, int hidden) {
@@ -56,13 +61,14 @@ __device__ double block_sum_fixed(double v, double* red) {
 __global__ void __launch_bounds__(kNormThreads)
     seq_norm_kernel(const float* __restrict__ s, const float* __restrict__ partial,
                     const int32_t* __restrict__ cu, const uint8_t* __restrict__ prunable,
-                    float eps, float* __restrict__ z, float* __restrict__ bias) {
+                    float eps, float* __restrict__ z, float* __restrict__ bias,
+                    int rows_per_cta) {
   __shared__ double red[kNormThreads / 32];
   griddep_wait();
   const int b = blockIdx.y;
   const int64_t lo = cu[b], hi = cu[b + 1];
   const int64_t n = hi - lo;
-  const int64_t my_lo = lo + (int64_t)blockIdx.x * kNormRowsPerCta;
+  const int64_t my_lo = lo + (int64_t)blockIdx.x * rows_per_cta;
   if (n <= 0 || my_lo >= hi) return;
   const int tid = threadIdx.x;
   const int64_t c_first = (lo + 31) >> 5, c_last = hi >> 5;  // whole chunks [c_first, c_last)
@@ -76,7 +82,7 @@ __global__ void __launch_bounds__(kNormThreads)
   }
   const double total = block_sum_fixed(acc, red);
   const float rms = (float)sqrt(total / (double)n + (double)eps);
-  int64_t my_hi = my_lo + kNormRowsPerCta;
+  int64_t my_hi = my_lo + rows_per_cta;
   if (my_hi > hi) my_hi = hi;
   for (int64_t j = my_lo + tid; j < my_hi; j += kNormThreads) {
     const float zz = s[j] / rms;
@@ -162,7 +168,8 @@ extern "C" int tg_gate_score(const tg_bf16* h, int64_t ld_h, int64_t total_token
 
   dim3 grid((unsigned)((max_n + kNormRowsPerCta - 1) / kNormRowsPerCta), (unsigned)batch);
   return launch(seq_norm_kernel, grid, dim3(kNormThreads), 0, st, (const float*)s_out,
-                (const float*)partial, cu_seqlens, prunable, eps_seq, z_out, bias_out);
+                (const float*)partial, cu_seqlens, prunable, eps_seq, z_out, bias_out,
+                kNormRowsPerCta);
 }
 
 extern "C" int tg_seq_rmsnorm(const float* s, const int32_t* cu_seqlens,
@@ -181,8 +188,10 @@ extern "C" int tg_seq_rmsnorm(const float* s, const int32_t* cu_seqlens,
   if (!s || !cu_seqlens || !prunable || !z_out || !bias_out) return TG_ERR_INVALID_ARGUMENT;
   if (z_out == s || bias_out == s) return TG_ERR_INVALID_ARGUMENT;
   TG_TRY(check_device());
-  dim3 grid((unsigned)((max_n + kNormRowsPerCta - 1) / kNormRowsPerCta), (unsigned)batch);
+  dim3 grid((unsigned)((max_n + kNormRowsPerCtaNoPartials - 1) / kNormRowsPerCtaNoPartials),
+            (unsigned)batch);
   TG_TRY(launch(seq_norm_kernel, grid, dim3(kNormThreads), 0, (cudaStream_t)stream, s,
-                (const float*)nullptr, cu_seqlens, prunable, eps_seq, z_out, bias_out));
+                (const float*)nullptr, cu_seqlens, prunable, eps_seq, z_out, bias_out,
+                kNormRowsPerCtaNoPartials));
   return TG_OK;
 }

@@ -107,3 +107,11 @@ def test_launch_overlap_switch(lib):
     assert lib.tg_set_launch_overlap(0) == 0 and lib.tg_get_launch_overlap() == 0
     assert lib.tg_set_launch_overlap(7) == 0 and lib.tg_get_launch_overlap() == 1
     lib.tg_set_launch_overlap(prev)
+
+
+def test_prefetch_argument_checks(lib):
+    """tg_prefetch_l2 rejects bad pointers on the host; zero bytes is a no-op."""
+    assert lib.tg_prefetch_l2(None, 0, None) == 0
+    assert lib.tg_prefetch_l2(C.c_void_p(0x10000), 0, None) == 0
+    assert lib.tg_prefetch_l2(None, 4096, None) == -1
+    assert lib.tg_prefetch_l2(C.c_void_p(0x10004), 4096, None) == -2
