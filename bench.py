@@ -93,6 +93,7 @@ def stage_work(wl, kept_counts):
         "qkv_rope_cache": {"bound": "tensor", "flops": 2 * K * H * nqkv,
                            "bytes": K * H * 2 + nqkv * H * 2 + K * nqkv * 2 + K * 4
                            + K * (H // 128) * 4},
+        "out_proj_qkv": {"bound": "tensor", "flops": 2 * K * hq * d * H + 2 * K * H * nqkv},
         "qkv_proj": {"bound": "tensor", "flops": 2 * K * H * nqkv,
                      "bytes": K * H * 2 + nqkv * H * 2 + K * nqkv * 2},
         "rope": {"bound": "hbm", "bytes": 2 * K * (hq + hkv) * d * 2 + K * 4},

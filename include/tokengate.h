@@ -375,6 +375,37 @@ int tg_qkv_rope_cache(const tg_bf16* x, int64_t ld_x, const tg_bf16* w_qkv, int6
                       int64_t ld_cache, int64_t slot_offset, const float* row_ssq_in,
                       int64_t ld_ssq_in, uint32_t* status, tg_stream_t stream);
 
+/*
+ * One layer boundary in one launch: the output projection of gated layer l followed by
+ * gated layer l+1's QKV projection, RoPE and KV-cache write, with identical results to
+ *   tg_linear(o, W_o, x, residual = x, row_ssq)            (x <- x + o W_o^T)
+ *   tg_qkv_rope_cache(x, W_qkv, ..., row_ssq_in = row_ssq)
+ * Both run on the CTA-pair kernel over 256 x 256 tiles: the projection's tiles first,
+ * then the QKV tiles, each of which starts once every projection tile of its 256 rows
+ * has stored them (counted in `workspace`), so the QKV work fills the SMs the projection
+ * leaves idle instead of waiting for a second launch.
+ * o: bf16 [M, o_cols] (ld_o); w_o: bf16 [hidden, o_cols] (ld_wo); x: bf16 [M, hidden]
+ * (ld_x, updated in place); row_ssq: float32 [M, hidden/128] (ld_ssq) receives the new
+ * rows' sums of squares per 128 columns and feeds the folded RMSNorm of the QKV part;
+ * the remaining arguments are those of tg_qkv_rope_cache.  hidden, n_q_heads*head_dim
+ * and n_kv_heads*head_dim must be multiples of 256; head_dim 128; o_cols multiple of 64.
+ * workspace: tg_out_proj_qkv_workspace_size(M) bytes, 4-byte aligned, zero-filled before
+ * its first use; every completed call leaves it zeroed (after TG_STATUS_TIMEOUT, zero it
+ * again).  The launch is cooperative (all its CTAs resident at once); a device that
+ * cannot hold them returns TG_ERR_CUDA.
+ */
+int tg_out_proj_qkv_next(const tg_bf16* o, int64_t ld_o, const tg_bf16* w_o, int64_t ld_wo,
+                         tg_bf16* x, int64_t ld_x, float* row_ssq, int64_t ld_ssq, int64_t M,
+                         int hidden, int o_cols, const tg_bf16* w_qkv, int64_t ld_wqkv,
+                         int n_q_heads, int n_kv_heads, int head_dim, float eps,
+                         const int32_t* pos, const float* cos_sin, int max_pos, tg_bf16* q_out,
+                         int64_t ld_q, tg_bf16* cache_k, tg_bf16* cache_v, int64_t ld_cache,
+                         int64_t slot_offset, void* workspace, size_t workspace_bytes,
+                         uint32_t* status, tg_stream_t stream);
+
+/* Workspace bytes of tg_out_proj_qkv_next for M rows (two int32 counters per 256 rows). */
+size_t tg_out_proj_qkv_workspace_size(int64_t M);
+
 #ifdef __cplusplus
 }
 #endif

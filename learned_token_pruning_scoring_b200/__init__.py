@@ -26,7 +26,7 @@ __all__ = [
     "tg_rope_table", "tg_gate_score_workspace_size", "tg_gate_score", "tg_topk_compact",
     "tg_gate_score_noalloc", "tg_seq_rmsnorm", "tg_gather_rope", "tg_kv_compact", "tg_gated_attention", "tg_linear",
     "tg_status_clear", "tg_status_read", "tg_set_launch_overlap", "tg_get_launch_overlap",
-    "tg_prefetch_l2",
+    "tg_prefetch_l2", "tg_out_proj_qkv_next", "tg_out_proj_qkv_workspace_size",
     "GatedPrefill", "STATUS_TIMEOUT", "STATUS_BUDGET",
     "STATUS_BOUNDS", "STATUS_WORKSPACE",
 ]
@@ -338,6 +338,33 @@ def tg_qkv_rope_cache(x, w_qkv, pos, cos_sin, cache_k, cache_v, n_q_heads, n_kv_
     return q_out
 
 
+def tg_out_proj_qkv_workspace_size(M: int) -> int:
+    return int(lib.tg_out_proj_qkv_workspace_size(int(M)))
+
+
+def tg_out_proj_qkv_next(o, w_o, x, row_ssq, w_qkv, pos, cos_sin, cache_k, cache_v, n_q_heads,
+                         n_kv_heads, q_out, workspace, head_dim=128, eps=1e-6, slot_offset=0,
+                         status=None, stream=None):
+    """x <- x + o w_o^T (row sums of squares into row_ssq), then the next layer's fused
+    QKV + RoPE + KV-cache write from the new x, in one launch.  `workspace` is a
+    zero-filled uint8 tensor of tg_out_proj_qkv_workspace_size(M) bytes (left zeroed)."""
+    ld_o, ld_wo, ld_x = _mat(o, "o"), _mat(w_o, "w_o"), _mat(x, "x")
+    ld_ssq, ld_wqkv, ld_q = _mat(row_ssq, "row_ssq"), _mat(w_qkv, "w_qkv"), _mat(q_out, "q_out")
+    ld_c = _mat(cache_k, "cache_k")
+    if _mat(cache_v, "cache_v") != ld_c:
+        raise ValueError("cache_k and cache_v must share a row stride")
+    M, hidden = x.shape
+    rc = lib.tg_out_proj_qkv_next(_ptr(o), ld_o, _ptr(w_o), ld_wo, _ptr(x), ld_x, _ptr(row_ssq),
+                                  ld_ssq, M, hidden, o.shape[1], _ptr(w_qkv), ld_wqkv, n_q_heads,
+                                  n_kv_heads, head_dim, float(eps), _ptr(pos), _ptr(cos_sin),
+                                  cos_sin.shape[0], _ptr(q_out), ld_q, _ptr(cache_k),
+                                  _ptr(cache_v), ld_c, int(slot_offset), _ptr(workspace),
+                                  workspace.numel(), _ptr(status), _stream(stream))
+    _check(rc, "tg_out_proj_qkv_next")
+    _count()
+    return x
+
+
 # ----------------------------------------------------------------------------- pipeline
 
 @dataclass
@@ -378,6 +405,12 @@ class GatedPrefill:
         # off by default)
         self.prefetch_weights = False
         self._side = None
+        # optional: one launch per layer boundary, layer i's output projection and layer
+        # i+1's QKV (tg_out_proj_qkv_next).  At K = 1638 every projection tile finishes
+        # in the first round, so the QKV tiles gain nothing by starting in the same
+        # launch (measured equal to two launches); off by default.
+        self.fuse_boundaries = False
+        self._qkv_done = -1  # index of the layer whose QKV already ran in a fused launch
 
     def _mark(self, name):
         if self.marker is not None:
@@ -416,6 +449,8 @@ class GatedPrefill:
                                 dtype=torch.uint8, device=dev),
             caches=[(torch.empty((K, self.hkv * self.d), **bf),
                      torch.empty((K, self.hkv * self.d), **bf)) for _ in self.layers],
+            chain_ws=torch.zeros(max(16, tg_out_proj_qkv_workspace_size(K)), dtype=torch.uint8,
+                                 device=dev),
         )
         return self.planned
 
@@ -442,8 +477,15 @@ class GatedPrefill:
                            stream=stream)
             self._mark("gather")
 
-    def layer(self, i, stream=None):
-        """Upper layer i on the kept rows, in place on x; K/V land in cache i."""
+    def _fusable(self):
+        nq, nkv = self.hq * self.d, self.hkv * self.d
+        return (self.fused_qkv and self.hidden % 256 == 0 and nq % 256 == 0 and nkv % 256 == 0
+                and self.d == 128)
+
+    def layer(self, i, stream=None, fuse_next=False):
+        """Upper layer i on the kept rows, in place on x; K/V land in cache i.  With
+        `fuse_next`, layer i's output projection and layer i+1's QKV run as one launch
+        (then layer i+1 skips its QKV)."""
         P = self.planned
         if P["K"] == 0:
             return
@@ -451,7 +493,9 @@ class GatedPrefill:
         ck, cv = P["caches"][i]
         nq, nk = self.hq * self.d, self.hkv * self.d
         qkv, o, x = P["qkv"], P["o"], P["x"]
-        if self.fused_qkv:
+        if self._qkv_done == i:
+            pass  # ran with the previous layer's output projection
+        elif self.fused_qkv:
             tg_qkv_rope_cache(x, L.Wqkv, P["kept_pos"], self.cos_sin, ck, cv, self.hq, self.hkv,
                               q_out=qkv[:, :nq], head_dim=self.d, eps=self.norm_eps,
                               row_ssq=P["ssq"], status=self.status, stream=stream)
@@ -480,13 +524,25 @@ class GatedPrefill:
                            head_dim=self.d, workspace=P["attn_ws"], status=self.status,
                            stream=stream)
         self._mark("attention")
-        tg_linear(o, L.Wo, x, residual=x, row_ssq=P["ssq"], status=self.status, stream=stream)
-        self._mark("out_proj")
+        if fuse_next and i + 1 < len(self.layers) and self._fusable():
+            Ln = self.layers[i + 1]
+            ckn, cvn = P["caches"][i + 1]
+            tg_out_proj_qkv_next(o, L.Wo, x, P["ssq"], Ln.Wqkv, P["kept_pos"], self.cos_sin, ckn,
+                                 cvn, self.hq, self.hkv, qkv[:, :nq], P["chain_ws"],
+                                 head_dim=self.d, eps=self.norm_eps, status=self.status,
+                                 stream=stream)
+            self._qkv_done = i + 1
+            self._mark("out_proj_qkv")
+        else:
+            tg_linear(o, L.Wo, x, residual=x, row_ssq=P["ssq"], status=self.status, stream=stream)
+            self._mark("out_proj")
 
     def upper_layers(self, h, stream=None):
         self.gather(h, stream=stream)
+        self._qkv_done = -1
         for i in range(len(self.layers)):
-            self.layer(i, stream=stream)
+            self.layer(i, stream=stream, fuse_next=self.fuse_boundaries)
+        self._qkv_done = -1
         if self._side is not None:  # join the prefetch stream (a captured graph needs it)
             main = stream if stream is not None else torch.cuda.current_stream(self.device)
             main.wait_stream(self._side)

@@ -46,6 +46,10 @@ SIGNATURES = {
     "tg_gated_attention_workspace_size": (_sz, [_p, _i32, _i32, _i32, _i32]),
     "tg_qkv_rope_cache": (_i32, [_p, _i64, _p, _i64, _i64, _i32, _i32, _i32, _i32, _f32, _p, _p,
                                  _i32, _p, _i64, _p, _p, _i64, _i64, _p, _i64, _p, _p]),
+    "tg_out_proj_qkv_next": (_i32, [_p, _i64, _p, _i64, _p, _i64, _p, _i64, _i64, _i32, _i32,
+                                     _p, _i64, _i32, _i32, _i32, _f32, _p, _p, _i32, _p, _i64,
+                                     _p, _p, _i64, _i64, _p, _sz, _p, _p]),
+    "tg_out_proj_qkv_workspace_size": (_sz, [_i64]),
     "tg_linear": (_i32, [_p, _i64, _p, _i64, _p, _i64, _i64, _i32, _i32, _i32, _f32, _p, _i64,
                          _p, _i64, _p, _p]),
 }

@@ -485,8 +485,28 @@ __device__ __forceinline__ void pair_epilogue_half(const GemmParams& p, unsigned
   }
 }
 
+// One GEMM for the CTA-pair kernel: tensor maps and parameters.
+struct PairJob {
+  PairMaps maps;
+  GemmParams p;
+};
+
+// Optional ordering between the two jobs of one launch: job 1 reads (as A and through
+// row_ssq_in) the rows job 0 writes.  ready[rp] counts job 0's finished epilogue groups
+// of row pair rp (each 256 x 256 tile contributes 4: two groups in each CTA); a job-1
+// tile of rp starts loading once ready[rp] == target.  consumed[rp] counts job-1
+// producers that passed that wait; the last one resets both, so the counters start and
+// end every launch at zero (the caller zero-fills them once).
+struct PairChain {
+  int* ready;
+  int* consumed;
+  int target;
+};
+
 // Persistent CTA-pair GEMM: each cluster of two CTAs walks the 256 x 256 output tiles
-// t = cluster, cluster + clusters, ...  Roles per CTA:
+// t = cluster, cluster + clusters, ... of job 0 and then of job 1 (tiles of job 1 follow
+// all of job 0's in that order, so a job-1 tile only ever waits for job-0 tiles that
+// are already running or done).  Roles per CTA:
 //   warp 0     one thread streams A and W k-blocks of every tile through the ring;
 //   warp 1     TMEM owner; in the even CTA one thread issues the M=256 MMAs into
 //              accumulator buffer (tile index & 1);
@@ -499,9 +519,10 @@ __device__ __forceinline__ void pair_epilogue_half(const GemmParams& p, unsigned
 // Barriers: full/empty per ring stage (full lives in the even CTA and counts both CTAs'
 // bytes); acc_full[b] (the even CTA's commit, in both CTAs); acc_empty[b] (even CTA,
 // one arrive per epilogue group of each CTA once it has read buffer b); res_full[g].
-template <int STAGES, int EPI>
+template <int STAGES, int EPI0, int EPI1>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(320, 1)
-    gemm_pair_kernel(const __grid_constant__ PairMaps maps, GemmParams p) {
+    gemm_pair_kernel(const __grid_constant__ PairJob job0, const __grid_constant__ PairJob job1,
+                     PairChain chain) {
   using Cfg = PairCfg<STAGES>;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>(
@@ -519,11 +540,24 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(320, 1)
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const uint32_t rank = cluster_ctarank();
-  const int n_tiles_n = p.N / Cfg::BN;
-  const int n_tiles = (int)((p.M + 255) / 256) * n_tiles_n;
   const int cluster = (int)(blockIdx.x >> 1), n_clusters = (int)(gridDim.x >> 1);
-  const int nk = p.K / Cfg::BK;
-  const bool has_res = EPI == EpiStore && p.residual != nullptr;
+  const int tn0 = job0.p.N / Cfg::BN, tn1 = job1.p.M > 0 ? job1.p.N / Cfg::BN : 1;
+  const int n_tiles0 = (int)((job0.p.M + 255) / 256) * tn0;
+  const int n_tiles1 = job1.p.M > 0 ? (int)((job1.p.M + 255) / 256) * tn1 : 0;
+  const int n_tiles = n_tiles0 + n_tiles1;
+  uint32_t* status = job0.p.status;
+  // tile t -> job, row pair and first column of the tile
+  auto decode = [&](int t, int& job, int& rp, int& n0) {
+    job = t >= n_tiles0;
+    const int u = job ? t - n_tiles0 : t;
+    const int tn = job ? tn1 : tn0;
+    rp = u / tn;
+    n0 = (u % tn) * Cfg::BN;
+  };
+  auto has_res = [&](int job) {
+    return job ? (EPI1 == EpiStore && job1.p.residual != nullptr)
+               : (EPI0 == EpiStore && job0.p.residual != nullptr);
+  };
 
   if (tid == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -540,8 +574,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(320, 1)
     fence_mbar_init();
   }
   if (warp == 0 && lane == 0) {
-    tma_prefetch_desc(&maps.a);
-    tma_prefetch_desc(&maps.b);
+    tma_prefetch_desc(&job0.maps.a);
+    tma_prefetch_desc(&job0.maps.b);
   }
   if (warp == 1) {
     tmem_alloc_pair(tmem_slot, Cfg::TMEM_COLS);
@@ -563,26 +597,39 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(320, 1)
       int kg = 0;
       bool ok = true;
       for (int t = cluster; ok && t < n_tiles; t += n_clusters) {
-        const int64_t m0 = (int64_t)(t / n_tiles_n) * 256 + rank * 128;
-        const int n0 = (t % n_tiles_n) * Cfg::BN + (int)rank * (Cfg::BN / 2);
+        int job, rp, n0;
+        decode(t, job, rp, n0);
+        const PairJob& jb = job ? job1 : job0;
+        if (job && chain.ready) {
+          // job 0 must have finished every column of these rows
+          if (!wait_count_gpu(chain.ready + rp, chain.target, abort_flag, status)) break;
+          fence_proxy_async_global();  // the rows are read by TMA next
+          if (atomicAdd(chain.consumed + rp, 1) == 2 * tn1 - 1) {
+            chain.ready[rp] = 0;  // every producer of these rows has passed its wait
+            chain.consumed[rp] = 0;
+          }
+        }
+        const int64_t m0 = (int64_t)rp * 256 + rank * 128;
+        const int nb = n0 + (int)rank * (Cfg::BN / 2);
+        const int nk = jb.p.K / Cfg::BK;
         for (int kb = 0; kb < nk; ++kb, ++kg) {
           const int s = kg % STAGES;
           const uint32_t ph = (uint32_t)(kg / STAGES) & 1u;
-          if (!mbar_wait(&empty[s], ph ^ 1u, abort_flag, p.status)) {
+          if (!mbar_wait(&empty[s], ph ^ 1u, abort_flag, status)) {
             ok = false;
             break;
           }
           unsigned char* a_s = tiles + s * Cfg::STAGE_BYTES;
           if (rank == 0) mbar_arrive_expect_tx(&full[s], 2 * Cfg::STAGE_BYTES);
-          tma_load_2d_pair(a_s, &maps.a, kb * Cfg::BK, (int32_t)m0, full_lead0 + s * 8);
-          tma_load_2d_pair(a_s + Cfg::A_BYTES, &maps.b, kb * Cfg::BK, n0, full_lead0 + s * 8);
+          tma_load_2d_pair(a_s, &jb.maps.a, kb * Cfg::BK, (int32_t)m0, full_lead0 + s * 8);
+          tma_load_2d_pair(a_s + Cfg::A_BYTES, &jb.maps.b, kb * Cfg::BK, nb, full_lead0 + s * 8);
         }
       }
       // The even CTA waits until the last stages' bytes (both CTAs') have landed; the odd
       // CTA is held by the closing cluster barrier until then.
       if (rank == 0)
         for (int g = kg - STAGES < 0 ? 0 : kg - STAGES; g < kg; ++g)
-          mbar_wait(&full[g % STAGES], (uint32_t)(g / STAGES) & 1u, nullptr, p.status);
+          mbar_wait(&full[g % STAGES], (uint32_t)(g / STAGES) & 1u, nullptr, status);
     }
   } else if (warp == 1) {
     if (lane == 0 && rank == 0) {
@@ -593,14 +640,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(320, 1)
       bool ok = true;
       for (int t = cluster; ok && t < n_tiles; t += n_clusters, ++i) {
         const int b = i & 1;
+        const int nk = (t >= n_tiles0 ? job1.p.K : job0.p.K) / Cfg::BK;
         // both CTAs' epilogues are done with this buffer (first use passes at once)
-        if (!mbar_wait(&acc_empty[b], ((uint32_t)(i >> 1) & 1u) ^ 1u, abort_flag, p.status)) break;
+        if (!mbar_wait(&acc_empty[b], ((uint32_t)(i >> 1) & 1u) ^ 1u, abort_flag, status)) break;
         tc_fence_after();
         const uint32_t d = tmem + (uint32_t)(b * Cfg::BN);
         for (int kb = 0; kb < nk; ++kb, ++kg) {
           const int s = kg % STAGES;
           const uint32_t ph = (uint32_t)(kg / STAGES) & 1u;
-          if (!mbar_wait(&full[s], ph, abort_flag, p.status)) {
+          if (!mbar_wait(&full[s], ph, abort_flag, status)) {
             ok = false;
             break;
           }
@@ -619,7 +667,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(320, 1)
         mma_commit_pair(acc_full_peer0 + b * 8);
       }
       mma_commit_pair(smem_u32(drain));
-      mbar_wait(drain, 0, nullptr, p.status);  // all MMAs (and their arrives) done
+      mbar_wait(drain, 0, nullptr, status);  // all MMAs (and their arrives) done
     }
   } else {
     const int q = warp & 3;        // TMEM lane quarter this warp may access
@@ -631,28 +679,47 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(320, 1)
     griddep_wait();
     int res_loads = 0;  // residual half-tiles requested by this group's elected thread
     auto load_res = [&](int t) {
-      const int64_t m0 = (int64_t)(t / n_tiles_n) * 256 + rank * 128;
-      const int n0 = (t % n_tiles_n) * Cfg::BN;
+      int job, rp, n0;
+      decode(t, job, rp, n0);
+      const PairJob& jb = job ? job1 : job0;
+      const int64_t m0 = (int64_t)rp * 256 + rank * 128;
       ++res_loads;
       mbar_arrive_expect_tx(&res_full[g], 2 * Cfg::BOX_BYTES);
       for (int j = 2 * g; j < 2 * g + 2; ++j)
-        tma_load_2d(out_s + j * Cfg::BOX_BYTES, &maps.res, n0 + 64 * j, (int32_t)m0,
+        tma_load_2d(out_s + j * Cfg::BOX_BYTES, &jb.maps.res, n0 + 64 * j, (int32_t)m0,
                     &res_full[g]);
     };
-    if (has_res && elected && cluster < n_tiles) load_res(cluster);
-    int i = 0;
+    auto res_of = [&](int t) {
+      int job, rp, n0;
+      decode(t, job, rp, n0);
+      return has_res(job);
+    };
+    if (elected && cluster < n_tiles && res_of(cluster)) load_res(cluster);
+    int i = 0, res_used = 0;
     for (int t = cluster; t < n_tiles; t += n_clusters, ++i) {
       const int b = i & 1;
-      const int64_t m0 = (int64_t)(t / n_tiles_n) * 256 + rank * 128;
-      const int n0 = (t % n_tiles_n) * Cfg::BN;
-      bool ok = mbar_wait(&acc_full[b], (uint32_t)(i >> 1) & 1u, abort_flag, p.status);
-      if (ok && has_res) ok = mbar_wait(&res_full[g], (uint32_t)i & 1u, abort_flag, p.status);
+      int job, rp, n0;
+      decode(t, job, rp, n0);
+      const PairJob& jb = job ? job1 : job0;
+      const bool with_res = has_res(job);
+      const int64_t m0 = (int64_t)rp * 256 + rank * 128;
+      bool ok = mbar_wait(&acc_full[b], (uint32_t)(i >> 1) & 1u, abort_flag, status);
+      if (ok && with_res) ok = mbar_wait(&res_full[g], (uint32_t)res_used & 1u, abort_flag, status);
+      if (with_res) ++res_used;
+      // job 1 reads job 0's row sums of squares: its producer acquired job 0's release
+      // before the loads behind this accumulator; a device fence orders this thread's
+      // reads after it too (the counter itself may already be reset by then)
+      if (job && chain.ready) __threadfence();
       // one decision for the group's four warps (they meet at named barriers below)
       if (!named_bar_and(bar_id, 128, ok)) break;
       tc_fence_after();
-      pair_epilogue_half<EPI>(p, out_s,
-                              tmem + (uint32_t)(b * Cfg::BN) + ((uint32_t)(q * 32) << 16), row,
-                              m0 + row, n0, g, has_res);
+      const uint32_t tacc = tmem + (uint32_t)(b * Cfg::BN) + ((uint32_t)(q * 32) << 16);
+      if (job)
+        pair_epilogue_half<EPI1>(jb.p, out_s, tacc, row, m0 + row, n0, g, with_res);
+      else
+        pair_epilogue_half<EPI0>(jb.p, out_s, tacc, row, m0 + row, n0, g, with_res);
+      const bool publish = !job && chain.ready;  // job 1 waits for these rows
+      if (publish) __threadfence();  // row sums of squares visible before the count
       tc_fence_before();
       fence_proxy_async_smem();  // staging writes visible to the TMA stores
       named_bar_sync(bar_id, 128);
@@ -662,28 +729,34 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(320, 1)
         else
           mbar_arrive_cluster(acc_empty_lead0 + b * 8);
         int mi = 0, x = n0;
-        if (EPI == EpiQKV) {
-          if (n0 >= p.q_cols + p.k_cols) {
+        if ((job ? EPI1 : EPI0) == EpiQKV) {
+          if (n0 >= jb.p.q_cols + jb.p.k_cols) {
             mi = 2;
-            x = n0 - p.q_cols - p.k_cols;
-          } else if (n0 >= p.q_cols) {
+            x = n0 - jb.p.q_cols - jb.p.k_cols;
+          } else if (n0 >= jb.p.q_cols) {
             mi = 1;
-            x = n0 - p.q_cols;
+            x = n0 - jb.p.q_cols;
           }
         }
         for (int j = 2 * g; j < 2 * g + 2; ++j)
-          tma_store_2d(&maps.out[mi], x + 64 * j, (int32_t)m0, out_s + j * Cfg::BOX_BYTES);
+          tma_store_2d(&jb.maps.out[mi], x + 64 * j, (int32_t)m0, out_s + j * Cfg::BOX_BYTES);
         bulk_commit_group();
-        bulk_wait_read_all();  // the group's staging boxes may be overwritten from here on
-        if (has_res && t + n_clusters < n_tiles) load_res(t + n_clusters);
+        if (publish) {
+          bulk_wait_all();             // the rows are in global memory
+          fence_proxy_async_global();  // ... and ordered before the release below
+          atomicAdd_release_gpu(chain.ready + rp, 1);
+        } else {
+          bulk_wait_read_all();  // the group's staging boxes may be overwritten from here on
+        }
+        if (t + n_clusters < n_tiles && res_of(t + n_clusters)) load_res(t + n_clusters);
       }
       named_bar_sync(bar_id, 128);
     }
     if (elected) {
       bulk_wait_all();
       // after an abort: a residual load may still be landing in the staging boxes
-      if (res_loads > i)
-        mbar_wait(&res_full[g], (uint32_t)(res_loads - 1) & 1u, nullptr, p.status);
+      if (res_loads > res_used)
+        mbar_wait(&res_full[g], (uint32_t)(res_loads - 1) & 1u, nullptr, status);
     }
   }
   __syncthreads();

@@ -27,19 +27,55 @@ int launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const GemmParams& 
 template <int STAGES, int EPI>
 int launch_pair(const PairMaps& maps, const GemmParams& p, cudaStream_t stream) {
   using Cfg = PairCfg<STAGES>;
+  auto kern = gemm_pair_kernel<STAGES, EPI, EPI>;
   static int attr_dev = -1;
   int dev = 0;
   TG_CUDA_TRY(cudaGetDevice(&dev));
   if (attr_dev != dev) {
-    TG_CUDA_TRY(cudaFuncSetAttribute(gemm_pair_kernel<STAGES, EPI>,
-                                     cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM));
+    TG_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM));
     attr_dev = dev;
   }
+  PairJob j0{maps, p}, j1{};
+  j1.p.M = 0;  // no second job
   // persistent: at most one cluster (two CTAs) per SM pair, each walking its tiles
   const int64_t tiles = ((p.M + 255) / 256) * (p.N / Cfg::BN);
   const int64_t clusters = std::min<int64_t>(tiles, std::max(1, sm_count() / 2));
-  return launch(gemm_pair_kernel<STAGES, EPI>, dim3((unsigned)(2 * clusters)), dim3(Cfg::THREADS),
-                Cfg::SMEM, stream, maps, p);
+  return launch(kern, dim3((unsigned)(2 * clusters)), dim3(Cfg::THREADS), Cfg::SMEM, stream, j0,
+                j1, PairChain{nullptr, nullptr, 0});
+}
+
+// Two chained jobs in one persistent launch (job 1 reads rows job 0 writes).  Every
+// cluster must be resident at once, because a job-1 tile can wait for a job-0 tile of
+// another cluster: the launch is cooperative, which guarantees that or fails.
+template <int STAGES, int EPI0, int EPI1>
+int launch_pair_chain(const PairJob& j0, const PairJob& j1, const PairChain& chain,
+                      cudaStream_t stream) {
+  using Cfg = PairCfg<STAGES>;
+  auto kern = gemm_pair_kernel<STAGES, EPI0, EPI1>;
+  static int attr_dev = -1;
+  int dev = 0;
+  TG_CUDA_TRY(cudaGetDevice(&dev));
+  if (attr_dev != dev) {
+    TG_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM));
+    attr_dev = dev;
+  }
+  const int64_t tiles = ((j0.p.M + 255) / 256) * (j0.p.N / Cfg::BN) +
+                        ((j1.p.M + 255) / 256) * (j1.p.N / Cfg::BN);
+  const int64_t clusters = std::min<int64_t>(tiles, std::max(1, sm_count() / 2));
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(2 * clusters));
+  cfg.blockDim = dim3(Cfg::THREADS);
+  cfg.dynamicSmemBytes = Cfg::SMEM;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = launch_overlap() ? 1 : 0;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  TG_CUDA_TRY(cudaLaunchKernelEx(&cfg, kern, j0, j1, chain));
+  return TG_OK;
 }
 
 constexpr int kPairStages = 5;
@@ -71,6 +107,73 @@ int pick_bn(int64_t M, int N) {
   return (can256 && e256 >= e128) ? 256 : 128;
 }
 
+// Output projection as a pair-kernel job: c = a w^T (+ residual), row sums of squares.
+int out_proj_job(PairJob& j, const tg_bf16* a, int64_t lda, const tg_bf16* w, int64_t ldw,
+                 tg_bf16* c, int64_t ldc, int64_t M, int N, int K, const tg_bf16* residual,
+                 int64_t ld_res, float* row_ssq_out, int64_t ld_ssq_out, uint32_t* status) {
+  TG_TRY(make_tmap_bf16_2d(&j.maps.a, a, (uint64_t)M, (uint64_t)K, (uint64_t)lda, 64, 128));
+  TG_TRY(make_tmap_bf16_2d(&j.maps.b, w, (uint64_t)N, (uint64_t)K, (uint64_t)ldw, 64, 128));
+  TG_TRY(make_tmap_bf16_2d(&j.maps.out[0], c, (uint64_t)M, (uint64_t)N, (uint64_t)ldc, 64, 128));
+  j.maps.out[1] = j.maps.out[2] = j.maps.res = j.maps.out[0];
+  if (residual)
+    TG_TRY(make_tmap_bf16_2d(&j.maps.res, residual, (uint64_t)M, (uint64_t)N, (uint64_t)ld_res,
+                             64, 128));
+  j.p = GemmParams{};
+  j.p.M = M;
+  j.p.N = N;
+  j.p.K = K;
+  j.p.c = reinterpret_cast<uint16_t*>(c);
+  j.p.ldc = ldc;
+  j.p.residual = reinterpret_cast<const uint16_t*>(residual);
+  j.p.ldr = ld_res;
+  j.p.row_ssq_out = row_ssq_out;
+  j.p.ld_ssq_out = ld_ssq_out;
+  j.p.status = status;
+  return TG_OK;
+}
+
+// QKV projection with the folded RMSNorm (row sums of squares given), RoPE and the
+// KV-cache write, as a pair-kernel job.
+int qkv_job(PairJob& j, const tg_bf16* x, int64_t ld_x, const tg_bf16* w_qkv, int64_t ld_w,
+            int64_t M, int hidden, int q_cols, int kv_cols, float eps, const int32_t* pos,
+            const float* cos_sin, int max_pos, tg_bf16* q_out, int64_t ld_q, tg_bf16* cache_k,
+            tg_bf16* cache_v, int64_t ld_cache, int64_t slot_offset, const float* row_ssq_in,
+            int64_t ld_ssq_in, uint32_t* status) {
+  const int N = q_cols + 2 * kv_cols;
+  tg_bf16* k_rows = cache_k + slot_offset * ld_cache;
+  tg_bf16* v_rows = cache_v + slot_offset * ld_cache;
+  TG_TRY(make_tmap_bf16_2d(&j.maps.a, x, (uint64_t)M, (uint64_t)hidden, (uint64_t)ld_x, 64, 128));
+  TG_TRY(make_tmap_bf16_2d(&j.maps.b, w_qkv, (uint64_t)N, (uint64_t)hidden, (uint64_t)ld_w, 64,
+                           128));
+  TG_TRY(make_tmap_bf16_2d(&j.maps.out[0], q_out, (uint64_t)M, (uint64_t)q_cols, (uint64_t)ld_q,
+                           64, 128));
+  TG_TRY(make_tmap_bf16_2d(&j.maps.out[1], k_rows, (uint64_t)M, (uint64_t)kv_cols,
+                           (uint64_t)ld_cache, 64, 128));
+  TG_TRY(make_tmap_bf16_2d(&j.maps.out[2], v_rows, (uint64_t)M, (uint64_t)kv_cols,
+                           (uint64_t)ld_cache, 64, 128));
+  j.maps.res = j.maps.out[0];
+  j.p = GemmParams{};
+  j.p.M = M;
+  j.p.N = N;
+  j.p.K = hidden;
+  j.p.rmsnorm = 1;
+  j.p.eps = eps;
+  j.p.c = reinterpret_cast<uint16_t*>(q_out);
+  j.p.ldc = ld_q;
+  j.p.pos = pos;
+  j.p.cos_sin = cos_sin;
+  j.p.max_pos = max_pos;
+  j.p.q_cols = q_cols;
+  j.p.k_cols = kv_cols;
+  j.p.k_out = reinterpret_cast<uint16_t*>(k_rows);
+  j.p.v_out = reinterpret_cast<uint16_t*>(v_rows);
+  j.p.ld_kv = ld_cache;
+  j.p.row_ssq_in = row_ssq_in;
+  j.p.ld_ssq_in = ld_ssq_in;
+  j.p.status = status;
+  return TG_OK;
+}
+
 }  // namespace tg
 
 using namespace tg;
@@ -93,20 +196,16 @@ extern "C" int tg_linear(const tg_bf16* a, int64_t lda, const tg_bf16* w, int64_
 
   // CTA-pair kernel for 256-column tiles without an in-kernel norm; else one CTA per tile
   const bool pair = !rmsnorm_a && (N % 256) == 0;
-  const int bn = pair ? 128 : pick_bn(M, N);
-
-  PairMaps maps;
-  CUtensorMap& ta = maps.a;
-  CUtensorMap& tb = maps.b;
+  if (pair) {
+    PairJob j;
+    TG_TRY(out_proj_job(j, a, lda, w, ldw, c, ldc, M, N, K, residual, ld_res, row_ssq_out,
+                        ld_ssq_out, status));
+    return launch_pair<kPairStages, EpiStore>(j.maps, j.p, (cudaStream_t)stream);
+  }
+  const int bn = pick_bn(M, N);
+  CUtensorMap ta, tb;
   TG_TRY(make_tmap_bf16_2d(&ta, a, (uint64_t)M, (uint64_t)K, (uint64_t)lda, 64, 128));
   TG_TRY(make_tmap_bf16_2d(&tb, w, (uint64_t)N, (uint64_t)K, (uint64_t)ldw, 64, bn));
-  if (pair) {
-    TG_TRY(make_tmap_bf16_2d(&maps.out[0], c, (uint64_t)M, (uint64_t)N, (uint64_t)ldc, 64, 128));
-    maps.out[1] = maps.out[2] = maps.res = maps.out[0];
-    if (residual)
-      TG_TRY(make_tmap_bf16_2d(&maps.res, residual, (uint64_t)M, (uint64_t)N, (uint64_t)ld_res,
-                               64, 128));
-  }
   GemmParams p{};
   p.M = M;
   p.N = N;
@@ -120,7 +219,6 @@ extern "C" int tg_linear(const tg_bf16* a, int64_t lda, const tg_bf16* w, int64_
   p.row_ssq_out = row_ssq_out;
   p.ld_ssq_out = ld_ssq_out;
   p.status = status;
-  if (pair) return launch_pair<kPairStages, EpiStore>(maps, p, (cudaStream_t)stream);
   if (bn == 256) return launch_gemm<256, 4, EpiStore>(ta, tb, p, (cudaStream_t)stream);
   return launch_gemm<128, 3, EpiStore>(ta, tb, p, (cudaStream_t)stream);
 }
@@ -153,24 +251,18 @@ extern "C" int tg_qkv_rope_cache(const tg_bf16* x, int64_t ld_x, const tg_bf16* 
   // kernel when the row norms come precomputed
   const bool aligned256 = (q_cols % 256) == 0 && (kv_cols % 256) == 0;
   const bool pair = row_ssq_in && aligned256;
-  int bn = pair ? 128 : pick_bn(M, N);
-  if (!pair && bn == 256 && !aligned256) bn = 128;
-  PairMaps maps;
-  CUtensorMap& ta = maps.a;
-  CUtensorMap& tb = maps.b;
+  if (pair) {
+    PairJob j;
+    TG_TRY(qkv_job(j, x, ld_x, w_qkv, ld_w, M, hidden, q_cols, kv_cols, eps, pos, cos_sin, max_pos,
+                   q_out, ld_q, cache_k, cache_v, ld_cache, slot_offset, row_ssq_in, ld_ssq_in,
+                   status));
+    return launch_pair<kPairStages, EpiQKV>(j.maps, j.p, (cudaStream_t)stream);
+  }
+  int bn = pick_bn(M, N);
+  if (bn == 256 && !aligned256) bn = 128;
+  CUtensorMap ta, tb;
   TG_TRY(make_tmap_bf16_2d(&ta, x, (uint64_t)M, (uint64_t)hidden, (uint64_t)ld_x, 64, 128));
   TG_TRY(make_tmap_bf16_2d(&tb, w_qkv, (uint64_t)N, (uint64_t)hidden, (uint64_t)ld_w, 64, bn));
-  if (pair) {
-    tg_bf16* k_rows = cache_k + slot_offset * ld_cache;
-    tg_bf16* v_rows = cache_v + slot_offset * ld_cache;
-    TG_TRY(make_tmap_bf16_2d(&maps.out[0], q_out, (uint64_t)M, (uint64_t)q_cols, (uint64_t)ld_q,
-                             64, 128));
-    TG_TRY(make_tmap_bf16_2d(&maps.out[1], k_rows, (uint64_t)M, (uint64_t)kv_cols,
-                             (uint64_t)ld_cache, 64, 128));
-    TG_TRY(make_tmap_bf16_2d(&maps.out[2], v_rows, (uint64_t)M, (uint64_t)kv_cols,
-                             (uint64_t)ld_cache, 64, 128));
-    maps.res = maps.out[0];
-  }
   GemmParams p{};
   p.M = M;
   p.N = N;
@@ -190,7 +282,53 @@ extern "C" int tg_qkv_rope_cache(const tg_bf16* x, int64_t ld_x, const tg_bf16* 
   p.row_ssq_in = row_ssq_in;
   p.ld_ssq_in = ld_ssq_in;
   p.status = status;
-  if (pair) return launch_pair<kPairStages, EpiQKV>(maps, p, (cudaStream_t)stream);
   if (bn == 256) return launch_gemm<256, 4, EpiQKV>(ta, tb, p, (cudaStream_t)stream);
   return launch_gemm<128, 3, EpiQKV>(ta, tb, p, (cudaStream_t)stream);
+}
+
+extern "C" size_t tg_out_proj_qkv_workspace_size(int64_t M) {
+  if (M <= 0) return 0;
+  return (size_t)(2 * ((M + 255) / 256)) * sizeof(int32_t);
+}
+
+extern "C" int tg_out_proj_qkv_next(
+    const tg_bf16* o, int64_t ld_o, const tg_bf16* w_o, int64_t ld_wo, tg_bf16* x, int64_t ld_x,
+    float* row_ssq, int64_t ld_ssq, int64_t M, int hidden, int o_cols, const tg_bf16* w_qkv,
+    int64_t ld_wqkv, int n_q_heads, int n_kv_heads, int head_dim, float eps, const int32_t* pos,
+    const float* cos_sin, int max_pos, tg_bf16* q_out, int64_t ld_q, tg_bf16* cache_k,
+    tg_bf16* cache_v, int64_t ld_cache, int64_t slot_offset, void* workspace,
+    size_t workspace_bytes, uint32_t* status, tg_stream_t stream) {
+  if (head_dim != 128 || n_q_heads <= 0 || n_kv_heads <= 0 || hidden <= 0 || (hidden % 256) ||
+      o_cols <= 0 || (o_cols % 64))
+    return TG_ERR_UNSUPPORTED_SHAPE;
+  const int q_cols = n_q_heads * head_dim, kv_cols = n_kv_heads * head_dim;
+  if ((q_cols % 256) || (kv_cols % 256)) return TG_ERR_UNSUPPORTED_SHAPE;
+  if (M < 0 || slot_offset < 0 || max_pos <= 0 || !(eps >= 0.f)) return TG_ERR_INVALID_ARGUMENT;
+  if (M == 0) return TG_OK;
+  if (!o || !w_o || !x || !row_ssq || !w_qkv || !pos || !cos_sin || !q_out || !cache_k ||
+      !cache_v)
+    return TG_ERR_INVALID_ARGUMENT;
+  if (ld_o < o_cols || ld_wo < o_cols || ld_x < hidden || ld_ssq < hidden / 128 ||
+      ld_wqkv < hidden || ld_q < q_cols || ld_cache < kv_cols)
+    return TG_ERR_INVALID_ARGUMENT;
+  if (!aligned16(o) || !aligned16(w_o) || !aligned16(x) || !aligned16(w_qkv) ||
+      !aligned16(q_out) || !aligned16(cache_k) || !aligned16(cache_v) || !aligned16(cos_sin) ||
+      !stride_ok(ld_o, 2) || !stride_ok(ld_wo, 2) || !stride_ok(ld_x, 2) ||
+      !stride_ok(ld_wqkv, 2) || !stride_ok(ld_q, 2) || !stride_ok(ld_cache, 2))
+    return TG_ERR_MISALIGNED;
+  if (!workspace || workspace_bytes < tg_out_proj_qkv_workspace_size(M) ||
+      (reinterpret_cast<uintptr_t>(workspace) & 3))
+    return TG_ERR_WORKSPACE;
+  TG_TRY(check_device());
+  PairJob j0, j1;
+  TG_TRY(out_proj_job(j0, o, ld_o, w_o, ld_wo, x, ld_x, M, hidden, o_cols, x, ld_x, row_ssq,
+                      ld_ssq, status));
+  TG_TRY(qkv_job(j1, x, ld_x, w_qkv, ld_wqkv, M, hidden, q_cols, kv_cols, eps, pos, cos_sin,
+                 max_pos, q_out, ld_q, cache_k, cache_v, ld_cache, slot_offset, row_ssq, ld_ssq,
+                 status));
+  const int64_t rps = (M + 255) / 256;
+  int* ready = static_cast<int*>(workspace);
+  // each output-projection tile of a row pair counts 4 (two epilogue groups per CTA)
+  const PairChain chain{ready, ready + rps, 4 * (hidden / 256)};
+  return launch_pair_chain<kPairStages, EpiStore, EpiQKV>(j0, j1, chain, (cudaStream_t)stream);
 }

@@ -129,6 +129,27 @@ __device__ __forceinline__ bool wait_flag_gpu(const int* flag, volatile int* abo
   }
 }
 
+// Wait until *counter >= target (acquire); gives up like mbar_wait.
+__device__ __forceinline__ bool wait_count_gpu(const int* counter, int target,
+                                               volatile int* abort_flag, uint32_t* status) {
+  if (ld_acquire_gpu(counter) >= target) return true;
+  const uint64_t t0 = global_timer_ns();
+  while (true) {
+    __nanosleep(32);
+    if (ld_acquire_gpu(counter) >= target) return true;
+    if (abort_flag && *abort_flag) return false;
+    if (global_timer_ns() - t0 > TG_WAIT_LIMIT_NS) {
+      if (abort_flag) *abort_flag = 1;
+      if (status) atomicOr(status, TG_STATUS_TIMEOUT);
+      return false;
+    }
+  }
+}
+// Atomic add with release semantics at GPU scope (no return value).
+__device__ __forceinline__ void atomicAdd_release_gpu(int* counter, int v) {
+  asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(counter), "r"(v) : "memory");
+}
+
 // Warp-uniform outcome of per-thread waits: warp-collective tcgen05 instructions that
 // follow must be executed by all 32 lanes or by none.
 __device__ __forceinline__ bool warp_all(bool ok) { return __all_sync(0xFFFFFFFFu, ok); }

@@ -115,3 +115,18 @@ def test_prefetch_argument_checks(lib):
     assert lib.tg_prefetch_l2(C.c_void_p(0x10000), 0, None) == 0
     assert lib.tg_prefetch_l2(None, 4096, None) == -1
     assert lib.tg_prefetch_l2(C.c_void_p(0x10004), 4096, None) == -2
+
+
+def test_out_proj_qkv_argument_checks(lib):
+    """The layer-boundary launch needs 256-multiple widths and its counter workspace."""
+    p = C.c_void_p(0x10000)
+
+    def call(hidden, ws, ws_bytes):
+        return lib.tg_out_proj_qkv_next(p, 2048, p, 2048, p, hidden, p, 16, 8, hidden, 2048, p,
+                                        hidden, 16, 8, 128, 1e-6, p, p, 100, p, 2048, p, p,
+                                        1024, 0, ws, ws_bytes, None, None)
+    assert call(1920, p, 64) == -6
+    assert call(2048, None, 0) == -4
+    assert call(2048, p, 4) == -4
+    assert lib.tg_out_proj_qkv_workspace_size(0) == 0
+    assert lib.tg_out_proj_qkv_workspace_size(257) == 16

@@ -547,3 +547,38 @@ def test_qkv_rope_cache_position_out_of_table_sets_status(tg):
     st = _status()
     tg.tg_qkv_rope_cache(x, w, pos, cs, ck, cv, Hq, Hkv, status=st)
     assert tg.tg_status_read(st) & tg.STATUS_BOUNDS
+
+
+@pytest.mark.parametrize("M", [300, 1638, 4000])
+def test_out_proj_qkv_chain_equals_the_two_calls(tg, M):
+    """One layer boundary in one launch gives, bit for bit, what the two separate calls
+    give (same tiles, same epilogues; only the scheduling differs).  M = 4000 has more
+    output-projection tiles than clusters, so QKV tiles also wait for tiles that other
+    clusters start later.  The counters come back zero."""
+    Hq, Hkv, d, H = 16, 8, 128, 2048
+    o = _dev(S.uniform_rows(M, Hq * d, seed=M + 1))
+    x0 = _dev(S.uniform_rows(M, H, seed=M + 2, scale=3.0))
+    wo = _dev(S.uniform_rows(H, Hq * d, seed=M + 3, scale=0.02))
+    wqkv = _dev(S.uniform_rows((Hq + 2 * Hkv) * d, H, seed=M + 4, scale=0.02))
+    pos = _dev(torch.arange(0, 7 * M, 7, dtype=torch.int32))
+    cs = tg.tg_rope_table(7 * M + 1, d, 1.0e6)
+
+    def fresh():
+        return (x0.clone(), torch.full((M, H // 128), float("nan"), device="cuda"),
+                torch.empty((M, Hq * d), dtype=torch.bfloat16, device="cuda"),
+                torch.empty((M, Hkv * d), dtype=torch.bfloat16, device="cuda"),
+                torch.empty((M, Hkv * d), dtype=torch.bfloat16, device="cuda"))
+
+    x1, ssq1, q1, k1, v1 = fresh()
+    tg.tg_linear(o, wo, x1, residual=x1, row_ssq=ssq1)
+    tg.tg_qkv_rope_cache(x1, wqkv, pos, cs, k1, v1, Hq, Hkv, q_out=q1, row_ssq=ssq1)
+    x2, ssq2, q2, k2, v2 = fresh()
+    ws = torch.zeros(tg.tg_out_proj_qkv_workspace_size(M), dtype=torch.uint8, device="cuda")
+    st = _status()
+    for _ in range(2):  # the second call reuses the workspace the first left zeroed
+        x2.copy_(x0)
+        tg.tg_out_proj_qkv_next(o, wo, x2, ssq2, wqkv, pos, cs, k2, v2, Hq, Hkv, q2, ws, status=st)
+    assert tg.tg_status_read(st) == 0
+    assert torch.equal(x1, x2) and torch.equal(ssq1, ssq2)
+    assert torch.equal(q1, q2) and torch.equal(k1, k2) and torch.equal(v1, v2)
+    assert int(ws.count_nonzero()) == 0
