@@ -31,6 +31,9 @@ listed with its reason in the design notes of the repository):
     z_c = 0 for non-prunable keys.
   * upper layers keep KV only for kept tokens ([farwalk] How does TokenGate learned
     token pruning work?; [digest] 方法关键点).
+  * layers below the gate see every token with ordinary causal attention; their KV
+    may optionally be trimmed to the kept tokens as well ([digest] 方法关键点;
+    [aiwillknow] 图1(a)(b)).  Reading: trimming keeps exactly the gate's kept rows.
 """
 from __future__ import annotations
 
@@ -42,6 +45,7 @@ __all__ = [
     "as_f64", "rmsnorm_rows", "gate_score", "sequence_rmsnorm", "kept_counts",
     "select_topk", "gather_rows", "rope", "rope_angles", "temperature",
     "gated_attention", "kv_compact", "gated_layer", "prefill", "silu",
+    "request_positions", "causal_attention", "full_context_layer",
 ]
 
 
@@ -314,14 +318,81 @@ def gated_layer(x, Wqkv, Wo, gamma, beta, cu_kept, kept_pos, kept_bias,
     return x_out, k, v, parts
 
 
-def prefill(h, prunable, cu_seqlens, budgets, gate, layers, n_q_heads, n_kv_heads,
-            head_dim, theta=1.0e6, norm_eps=1e-6, seq_eps=1e-6, scores=None):
-    """Gate + selection + gathered upper layers, end to end.
+# ------------------------------------------------------------------ layers below the gate
 
-    `gate` holds norm_w, W1, w2; `layers` is a list of dicts with Wqkv, Wo, gamma,
-    beta.  With `scores` given, selection consumes those raw scores instead of the
-    scorer's (the planted-cluster workload).
+def request_positions(cu_seqlens) -> np.ndarray:
+    """Position of every packed token within its own request: 0 .. N_b - 1 per request."""
+    cu = _as_int(cu_seqlens)
+    return np.concatenate([np.arange(cu[b + 1] - cu[b]) for b in range(len(cu) - 1)]
+                          + [np.zeros(0, dtype=np.int64)])
+
+
+def causal_attention(Q, K, V, cu_seqlens, block: int = 1024):
+    """Ordinary causal GQA softmax attention inside each request.
+
+    o_i = sum_{j <= i} softmax_j(q_i . k_j / sqrt(d)) v_j, q head h reading kv head
+    h // (Hq / Hkv).  This is what every layer below the gate computes: all tokens
+    are still present there and no gate term exists yet ([fluxbbs] 门控到底插在模型的
+    哪个位置).  Written from the definition, independently of `gated_attention`.
+    Returns O [T, Hq, d] (float64).
     """
+    Q, K, V = as_f64(Q), as_f64(K), as_f64(V)
+    cu = _as_int(cu_seqlens)
+    T, Hq, d = Q.shape
+    grp = Hq // K.shape[1]
+    O = np.zeros(Q.shape)
+    for b in range(len(cu) - 1):
+        lo, hi = cu[b], cu[b + 1]
+        for i0 in range(lo, hi, block):
+            i1 = min(hi, i0 + block)
+            # query i (absolute) may read keys lo .. i
+            allowed = np.arange(lo, i1)[None, :] <= np.arange(i0, i1)[:, None]
+            for h in range(Hq):
+                g = h // grp
+                logit = (Q[i0:i1, h, :] @ K[lo:i1, g, :].T) / math.sqrt(d)
+                logit[~allowed] = -np.inf
+                w = np.exp(logit - logit.max(axis=1, keepdims=True))
+                w /= w.sum(axis=1, keepdims=True)
+                O[i0:i1, h, :] = w @ V[lo:i1, g, :]
+    return O
+
+
+def full_context_layer(x, Wqkv, Wo, cu_seqlens, n_q_heads: int, n_kv_heads: int,
+                       head_dim: int, theta: float = 1.0e6, eps: float = 1e-6):
+    """One layer below the gate on all tokens: x + Wo . Attn(RoPE(Wq a), RoPE(Wk a), Wv a)
+    with a = RMSNorm(x), RoPE at each token's position in its request and ordinary
+    causal attention.  Returns (x_out, K_cache, V_cache): the full-length post-RoPE
+    K and V of this layer, [T, Hkv, d]."""
+    x = as_f64(x)
+    a = rmsnorm_rows(x, None, eps)
+    qkv = a @ as_f64(Wqkv).T
+    nq, nk = n_q_heads * head_dim, n_kv_heads * head_dim
+    T = x.shape[0]
+    pos = request_positions(cu_seqlens)
+    q = rope(qkv[:, :nq].reshape(T, n_q_heads, head_dim), pos, theta)
+    k = rope(qkv[:, nq:nq + nk].reshape(T, n_kv_heads, head_dim), pos, theta)
+    v = qkv[:, nq + nk:].reshape(T, n_kv_heads, head_dim)
+    o = causal_attention(q, k, v, cu_seqlens)
+    return x + o.reshape(T, nq) @ as_f64(Wo).T, k, v
+
+
+def prefill(h, prunable, cu_seqlens, budgets, gate, layers, n_q_heads, n_kv_heads,
+            head_dim, theta=1.0e6, norm_eps=1e-6, seq_eps=1e-6, scores=None,
+            lower_layers=()):
+    """Lower layers + gate + selection + gathered upper layers, end to end.
+
+    `gate` holds norm_w, W1, w2; `layers` (above the gate) and `lower_layers` (below
+    it) are lists of dicts with Wqkv and Wo (plus gamma, beta above the gate).  The
+    lower layers run on every token; the gate reads their output, the residual at
+    the gate layer.  Their K/V caches come back both full-length and trimmed to the
+    kept rows.  With `scores` given, selection consumes those raw scores instead of
+    the scorer's (the planted-cluster workload).
+    """
+    lower_full = []
+    for L in lower_layers:
+        h, k, v = full_context_layer(h, L["Wqkv"], L["Wo"], cu_seqlens, n_q_heads,
+                                     n_kv_heads, head_dim, theta, norm_eps)
+        lower_full.append((k, v))
     s = gate_score(h, gate["norm_w"], gate["W1"], gate["w2"], norm_eps) if scores is None \
         else as_f64(scores)
     z, bias = sequence_rmsnorm(s, cu_seqlens, prunable, seq_eps)
@@ -336,4 +407,6 @@ def prefill(h, prunable, cu_seqlens, budgets, gate, layers, n_q_heads, n_kv_head
                                  theta, norm_eps)
         caches.append((k, v))
     return {"s": s, "z": z, "bias": bias, "cu_kept": cu_kept, "kept_idx": kept_idx,
-            "kept_pos": kept_pos, "kept_bias": kept_bias, "x": x, "caches": caches}
+            "kept_pos": kept_pos, "kept_bias": kept_bias, "x": x, "caches": caches,
+            "h_gate": as_f64(h), "lower_caches_full": lower_full,
+            "lower_caches": [kv_compact(k, v, kept_idx) for k, v in lower_full]}

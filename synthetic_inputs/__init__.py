@@ -16,6 +16,8 @@ Recipe (all draws on the CPU with ``torch.Generator``):
   * gate weights: RMSNorm weight = 1, W1 [F, H] ~ N(0, 0.02) bf16, w2 [F] ~ N(0, 0.02) fp32;
   * layer l weights: Wqkv [Hq*d + 2*Hkv*d, H] ~ N(0, 0.02) bf16 (rows: Wq, then Wk,
     then Wv), Wo [H, Hq*d] ~ N(0, 0.02) bf16, gamma [Hq] ~ U(0.5, 2) fp32, beta = 1;
+  * layers below the gate (full context): Wqkv and Wo drawn the same way from their
+    own stream, no gamma or beta;
   * prunable mask: the first D_b tokens of each request are the document (prunable),
     the last Q_b tokens are the question (never pruned);
   * drawn scores (planted-cluster workload): s ~ N(0, 1) fp32 with +4 added on 64
@@ -43,6 +45,7 @@ _GATE_STREAM = 1_000_001
 _LAYER_STREAM = 2_000_003
 _LAYOUT_STREAM = 3_000_017
 _SCORE_STREAM = 4_000_037
+_LOWER_STREAM = 5_000_011
 
 
 @dataclass(frozen=True)
@@ -170,6 +173,18 @@ def layer_weights(wl: Workload, layer: int) -> dict:
     if wl.dense:
         gamma = torch.zeros_like(gamma)
     return {"Wqkv": Wqkv, "Wo": Wo, "gamma": gamma, "beta": beta}
+
+
+def lower_layer_weights(wl: Workload, n_layers: int) -> list:
+    """Weights of `n_layers` full-context layers below the gate: Wqkv, Wo only."""
+    hq, hkv, d, H = wl.n_q_heads, wl.n_kv_heads, wl.head_dim, wl.hidden
+    out = []
+    for layer in range(n_layers):
+        g = torch.Generator().manual_seed(_LOWER_STREAM + 7919 * wl.weight_seed + layer)
+        Wqkv = (torch.randn(((hq + 2 * hkv) * d, H), generator=g) * 0.02).to(torch.bfloat16)
+        Wo = (torch.randn((H, hq * d), generator=g) * 0.02).to(torch.bfloat16)
+        out.append({"Wqkv": Wqkv, "Wo": Wo})
+    return out
 
 
 def prunable_mask(wl: Workload) -> torch.Tensor:

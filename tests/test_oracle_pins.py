@@ -384,3 +384,103 @@ def test_prefill_tiny_pipeline_consistency():
         kept_b = set(out["kept_idx"][out["cu_kept"][b]:out["cu_kept"][b + 1]].tolist())
         assert set(range(lo + n - q, lo + n)) <= kept_b
     assert out["x"].shape == (22, 32)
+
+
+# ------------------------------------------------------------------ layers below the gate
+
+def test_request_positions_restart_per_request():
+    np.testing.assert_array_equal(O.request_positions([0, 3, 3, 5]), [0, 1, 2, 0, 1])
+    assert O.request_positions([0]).size == 0
+
+
+def test_causal_attention_against_library_per_request():
+    """Ordinary causal GQA attention of each request against torch's SDPA (float64)."""
+    Q, K, V, cu, _, _, _ = _rand_attn_case(31, [17, 1, 9], Hq=8, Hkv=2, d=16)
+    got = O.causal_attention(Q, K, V, cu, block=5)
+    for b in range(3):
+        lo, hi = cu[b], cu[b + 1]
+        q = torch.tensor(Q[lo:hi]).permute(1, 0, 2)[None]
+        k = torch.tensor(K[lo:hi]).permute(1, 0, 2).repeat_interleave(4, dim=0)[None]
+        v = torch.tensor(V[lo:hi]).permute(1, 0, 2).repeat_interleave(4, dim=0)[None]
+        want = F.scaled_dot_product_attention(q, k, v, is_causal=True)[0].permute(1, 0, 2)
+        np.testing.assert_allclose(got[lo:hi], want.numpy(), atol=1e-12)
+
+
+def test_causal_attention_brute_force_and_gated_special_case():
+    """Explicit loops with gamma = 0, tau = 1 (positions = ranks), and the gated
+    oracle with every token kept, gamma = 0 and beta = 1: all three agree."""
+    Q, K, V, cu, _, bias, _ = _rand_attn_case(5, [6, 4])
+    pos = O.request_positions(cu)
+    want = _attn_loops(Q, K, V, cu, pos, bias, np.zeros(4), 1.0)
+    got = O.causal_attention(Q, K, V, cu, block=4)
+    np.testing.assert_allclose(got, want, atol=1e-12)
+    gated, _ = O.gated_attention(Q, K, V, cu, pos, bias, np.zeros(4), 1.0)
+    np.testing.assert_allclose(got, gated, atol=1e-12)
+
+
+def _lower_case(seed, lens, Hq=4, Hkv=2, d=8, H=32):
+    rng = np.random.default_rng(seed)
+    cu = np.concatenate([[0], np.cumsum(lens)])
+    x = rng.normal(size=(int(cu[-1]), H))
+    Wqkv = rng.normal(size=((Hq + 2 * Hkv) * d, H)) * 0.2
+    Wo = rng.normal(size=(H, Hq * d)) * 0.2
+    return x, Wqkv, Wo, cu
+
+
+def test_full_context_layer_requests_are_independent():
+    """Packing requests side by side must not change any of them: positions restart
+    at 0 and attention stays inside the request (a packed-index position or a
+    cross-request key would break this)."""
+    x, Wqkv, Wo, cu = _lower_case(3, [11, 7])
+    xo, k, v = O.full_context_layer(x, Wqkv, Wo, cu, 4, 2, 8, 1e4)
+    for b in range(2):
+        lo, hi = cu[b], cu[b + 1]
+        xb, kb, vb = O.full_context_layer(x[lo:hi], Wqkv, Wo, [0, hi - lo], 4, 2, 8, 1e4)
+        np.testing.assert_allclose(xo[lo:hi], xb, atol=1e-12)
+        np.testing.assert_allclose(k[lo:hi], kb, atol=1e-12)
+        np.testing.assert_allclose(v[lo:hi], vb, atol=1e-12)
+
+
+def test_full_context_layer_is_the_gated_layer_with_nothing_pruned():
+    x, Wqkv, Wo, cu = _lower_case(4, [9, 5])
+    pos = O.request_positions(cu)
+    xo, k, v = O.full_context_layer(x, Wqkv, Wo, cu, 4, 2, 8, 1e4)
+    xg, kg, vg, _ = O.gated_layer(x, Wqkv, Wo, np.zeros(4), 1.0, cu, pos,
+                                  np.ones(len(pos)), 4, 2, 8, 1e4)
+    np.testing.assert_allclose(xo, xg, atol=1e-12)
+    np.testing.assert_allclose(k, kg, atol=1e-12)
+    np.testing.assert_allclose(v, vg, atol=1e-12)
+    # zero output projection: the residual passes unchanged, K carries RoPE at the
+    # in-request positions
+    x0, k0, _ = O.full_context_layer(x, Wqkv, np.zeros_like(Wo), cu, 4, 2, 8, 1e4)
+    np.testing.assert_allclose(x0, x, atol=0)
+    a = x / np.sqrt(np.mean(x * x, 1, keepdims=True) + 1e-6)
+    kk = (a @ Wqkv.T)[:, 32:48].reshape(-1, 2, 8)
+    np.testing.assert_allclose(k0, O.rope(kk, pos, 1e4), atol=1e-12)
+
+
+def test_prefill_with_lower_layers_composes_and_trims():
+    """The gate reads the lower layers' output; trimmed lower caches are exactly the
+    kept rows of the full-length ones."""
+    import synthetic_inputs as S
+    wl = S.custom([40, 24], [4, 6], [10, 12], n_layers=1, hidden=32, scorer_width=8,
+                  n_q_heads=4, n_kv_heads=2, head_dim=8)
+    h = S.hidden_rows(wl)
+    gate = S.gate_weights(wl)
+    upper = [S.layer_weights(wl, 0)]
+    lower = S.lower_layer_weights(wl, 2)
+    pr = S.prunable_mask(wl)
+    cu = wl.cu_seqlens()
+    out = O.prefill(h, pr, cu, wl.budgets, gate, upper, 4, 2, 8, lower_layers=lower)
+    hg = O.as_f64(h)
+    for L in lower:
+        hg, _, _ = O.full_context_layer(hg, L["Wqkv"], L["Wo"], cu, 4, 2, 8)
+    np.testing.assert_allclose(out["h_gate"], hg, atol=1e-12)
+    direct = O.prefill(hg, pr, cu, wl.budgets, gate, upper, 4, 2, 8)
+    np.testing.assert_array_equal(out["kept_idx"], direct["kept_idx"])
+    np.testing.assert_allclose(out["x"], direct["x"], atol=1e-12)
+    assert len(out["lower_caches"]) == 2
+    for (kf, vf), (kt, vt) in zip(out["lower_caches_full"], out["lower_caches"]):
+        assert kf.shape[0] == wl.total_tokens and kt.shape[0] == len(out["kept_idx"])
+        np.testing.assert_array_equal(kt, kf[out["kept_idx"]])
+        np.testing.assert_array_equal(vt, vf[out["kept_idx"]])
