@@ -21,6 +21,12 @@ between two CUDA events; L2 is flushed (a 512 MiB write) before every timed step
 the events.  SM clocks and throttle reasons are sampled through NVML during that loop.  A
 second loop of K replays of the same step captured with timing events at every stage
 boundary gives the per-stage times (and the roofline of the dominant kernel).
+
+Alongside (`--dense-steps`, default 3): the same layer stack over every token with no
+gate (K = N, gamma = 0, tau = 1) on the same kernels, the GPU's own full-context
+prefill, reported under "dense_reference" with the gated step's speedup over it.
+`--lower-layers L` puts L full-context layers below the gate (the gate then scores
+their output and their caches are trimmed to the kept rows).
 """
 from __future__ import annotations
 
@@ -53,6 +59,11 @@ def parse_args():
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-sample-layers", type=int, default=12)
+    ap.add_argument("--lower-layers", type=int, default=0,
+                    help="full-context layers below the gate (their caches trimmed to the "
+                         "kept rows); 0 = the gate reads the input rows directly")
+    ap.add_argument("--dense-steps", type=int, default=3,
+                    help="timed steps of the full-context reference (0 skips it)")
     return ap.parse_args()
 
 
@@ -101,6 +112,13 @@ def stage_work(wl, kept_counts):
         "attention": {"bound": "tensor", "flops": 4 * d * hq * attn_pairs},
         "out_proj": {"bound": "tensor", "flops": 2 * K * hq * d * H,
                      "bytes": K * hq * d * 2 + H * hq * d * 2 + 2 * K * H * 2},
+        # layers below the gate: the same kernels over all T tokens, and the trim of
+        # their caches to the kept rows (one launch per lower layer)
+        "lower_qkv_rope_cache": {"bound": "tensor", "flops": 2 * T * H * nqkv},
+        "lower_attention": {"bound": "tensor",
+                            "flops": 4 * d * hq * sum(n * (n + 1) // 2 for n in wl.lengths)},
+        "lower_out_proj": {"bound": "tensor", "flops": 2 * T * hq * d * H},
+        "lower_kv_trim": {"bound": "hbm", "bytes": 2 * 2 * K * hkv * d * 2 + K * 4},
     }
 
 
@@ -188,8 +206,14 @@ def run_ours(args, rank, world):
         L = S.layer_weights(wl, i)
         layers.append({k: (v.to(dev) if torch.is_tensor(v) else v) for k, v in L.items()})
     scores = S.drawn_scores(wl).to(dev) if wl.planted_cluster else None
+    lower = None
+    if args.lower_layers:
+        lower = tg.FullContextLayers([{k: v.to(dev) for k, v in L.items()}
+                                      for L in S.lower_layer_weights(wl, args.lower_layers)],
+                                     wl.n_q_heads, wl.n_kv_heads, wl.head_dim, wl.rope_theta,
+                                     device=dev)
     pipe = tg.GatedPrefill(gate, layers, wl.n_q_heads, wl.n_kv_heads, wl.head_dim,
-                           wl.rope_theta, device=dev)
+                           wl.rope_theta, device=dev, lower=lower)
     P = pipe.plan(wl.lengths, wl.questions, wl.budgets)
     h_dev = h.to(dev)
     pr_dev = pr.to(dev)
@@ -379,7 +403,8 @@ def run_ours(args, rank, world):
         "config": {"workload": wl.name, "batch": wl.batch, "tokens_per_request": list(wl.lengths)
                    if wl.batch <= 8 else None, "question_tokens": list(wl.questions)
                    if wl.batch <= 8 else None, "kept": int(P["ck_h"][-1]),
-                   "gated_layers": wl.n_layers, "hidden": wl.hidden,
+                   "gated_layers": wl.n_layers, "lower_layers": args.lower_layers,
+                   "hidden": wl.hidden,
                    "heads": f"{wl.n_q_heads}q/{wl.n_kv_heads}kv x {wl.head_dim}",
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                    "l2": "flushed before every timed step (512 MiB write, outside the timing)",
@@ -393,7 +418,64 @@ def run_ours(args, rank, world):
                        for kk, vv in v.items()} for k, v in stages.items()},
         "clocks": clk.summary(),
     }
+    if args.dense_steps > 0:
+        out["dense_reference"] = dense_reference(tg, wl, layers, h_dev, flush, stream,
+                                                 args.dense_steps, peaks,
+                                                 total_ms / args.steps)
     return out
+
+
+def dense_reference(tg, wl, layers, h_dev, flush, stream, steps, peaks, gated_ms):
+    """The same layer stack over every token (K = N, gamma = 0, tau = 1, no gate): the
+    GPU's own full-context prefill on the same kernels, timed like the gated step
+    (L2 flushed before each step, CUDA events on the stream, eager launches)."""
+    import torch
+    full = tg.FullContextLayers(layers, wl.n_q_heads, wl.n_kv_heads, wl.head_dim,
+                                wl.rope_theta, device=h_dev.device)
+    full.plan(wl.lengths, wl.hidden)
+    for _ in range(2):
+        full.run(h_dev)
+    torch.cuda.synchronize()
+    ms = []
+    for _ in range(steps):
+        flush.fill_(1.0)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        full.run(h_dev)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ms.append(e0.elapsed_time(e1))
+    # one step with an event after every launch, for the attention kernel's own time
+    evs = []
+    flush.fill_(1.0)
+    e = torch.cuda.Event(enable_timing=True)
+    e.record(stream)
+    evs.append(("start", e))
+
+    def marker(name):
+        ev = torch.cuda.Event(enable_timing=True)
+        ev.record(stream)
+        evs.append((name, ev))
+    full.marker = marker
+    full.run(h_dev)
+    full.marker = None
+    torch.cuda.synchronize()
+    status = tg.tg_status_read(full.status)
+    if status:
+        raise SystemExit(f"device status {status:#x} in the full-context reference")
+    attn = [p[1].elapsed_time(c[1]) for p, c in zip(evs, evs[1:]) if c[0] == "attention"]
+    d_ms = sum(ms) / len(ms)
+    pairs = sum(n * (n + 1) // 2 for n in wl.lengths)
+    attn_ms = sum(attn) / len(attn) if attn else None
+    tf = 4 * wl.head_dim * wl.n_q_heads * pairs / (attn_ms / 1e3) / 1e12 if attn else None
+    peak = peaks["bf16_tflops_sustained"]
+    return {"what": "same layers over all tokens: K = N, gamma = 0, tau = 1, no gate",
+            "kept": wl.total_tokens, "layers": len(layers), "steps": steps,
+            "ms_per_step": d_ms, "tokens_per_s": wl.total_tokens / (d_ms / 1e3),
+            "gated_speedup": d_ms / gated_ms,
+            "attention": {"avg_ms": attn_ms, "achieved": tf, "unit": "TFLOP/s",
+                          "peak": peak, "frac": tf / peak if tf else None}}
 
 
 def load_traffic(kernel, workload_name):

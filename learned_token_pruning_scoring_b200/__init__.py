@@ -27,7 +27,7 @@ __all__ = [
     "tg_gate_score_noalloc", "tg_seq_rmsnorm", "tg_gather_rope", "tg_kv_compact", "tg_gated_attention", "tg_linear",
     "tg_status_clear", "tg_status_read", "tg_set_launch_overlap", "tg_get_launch_overlap",
     "tg_prefetch_l2", "tg_out_proj_qkv_next", "tg_out_proj_qkv_workspace_size",
-    "GatedPrefill", "STATUS_TIMEOUT", "STATUS_BUDGET",
+    "GatedPrefill", "FullContextLayers", "LayerWeights", "STATUS_TIMEOUT", "STATUS_BUDGET",
     "STATUS_BOUNDS", "STATUS_WORKSPACE",
 ]
 
@@ -375,6 +375,105 @@ class LayerWeights:
     beta: float
 
 
+class FullContextLayers:
+    """Layers below the gate: every token of every request, ordinary causal GQA
+    attention on the same kernels as the gated layers (gamma = 0, every token kept,
+    so tau = beta = 1 and no key bias).  Also the full-context reference of a gated
+    stack: the same weights without pruning.
+
+    ``plan`` allocates full-length buffers and caches; ``run`` leaves the residual
+    stream after the last layer in ``planned["x"]`` (the gate's input) and each
+    layer's post-RoPE K/V in ``planned["caches"]``; ``trim`` copies the kept rows of
+    those caches into compacted ones.
+    """
+
+    def __init__(self, layers: list, n_q_heads=16, n_kv_heads=8, head_dim=128,
+                 rope_theta=1.0e6, norm_eps=1e-6, device="cuda"):
+        self.device = torch.device(device)
+        self.layers = [(l["Wqkv"], l["Wo"]) if isinstance(l, dict) else (l.Wqkv, l.Wo)
+                       for l in layers]
+        self.hq, self.hkv, self.d = n_q_heads, n_kv_heads, head_dim
+        self.theta, self.norm_eps = rope_theta, norm_eps
+        self.status = torch.zeros(1, dtype=torch.int32, device=self.device)
+        self.cos_sin = None
+        self.planned = None
+        self.marker = None
+        self.stage_prefix = ""
+
+    def _mark(self, name):
+        if self.marker is not None:
+            self.marker(self.stage_prefix + name)
+
+    def plan(self, lengths, hidden):
+        lengths = [int(x) for x in lengths]
+        cu = [0]
+        for n in lengths:
+            cu.append(cu[-1] + n)
+        cu_h = _host_i32(cu)
+        T = cu[-1]
+        dev = self.device
+        max_pos = max(lengths) if lengths else 1
+        if self.cos_sin is None or self.cos_sin.shape[0] < max_pos:
+            self.cos_sin = tg_rope_table(max_pos, self.d, self.theta, device=dev)
+        pos = torch.cat([torch.arange(n, dtype=torch.int32) for n in lengths]) if T else \
+            torch.zeros(0, dtype=torch.int32)
+        bf = dict(dtype=torch.bfloat16, device=dev)
+        nqkv = (self.hq + 2 * self.hkv) * self.d
+        self.planned = dict(
+            T=T, cu_h=cu_h, cu=cu_h.to(dev), pos=pos.to(dev),
+            bias=torch.zeros(T, dtype=torch.float32, device=dev),
+            gamma=torch.zeros(self.hq, dtype=torch.float32, device=dev),
+            x=torch.empty((T, hidden), **bf),
+            ssq=torch.empty((T, hidden // 128), dtype=torch.float32, device=dev),
+            qkv=torch.empty((T, nqkv), **bf),
+            o=torch.empty((T, self.hq * self.d), **bf),
+            attn_ws=torch.zeros(tg_gated_attention_workspace_size(cu_h, self.hq, self.hkv,
+                                                                  self.d),
+                                dtype=torch.uint8, device=dev),
+            caches=[(torch.empty((T, self.hkv * self.d), **bf),
+                     torch.empty((T, self.hkv * self.d), **bf)) for _ in self.layers],
+        )
+        return self.planned
+
+    def run(self, h, stream=None):
+        """All layers on all rows of h (left untouched); returns the final residual."""
+        P = self.planned
+        if P["T"] == 0:
+            return P["x"]
+        nq = self.hq * self.d
+        qkv, o, x = P["qkv"], P["o"], P["x"]
+        tg_gather_rope(h, x, row_ssq=P["ssq"], status=self.status, stream=stream)
+        for (Wqkv, Wo), (ck, cv) in zip(self.layers, P["caches"]):
+            tg_qkv_rope_cache(x, Wqkv, P["pos"], self.cos_sin, ck, cv, self.hq, self.hkv,
+                              q_out=qkv[:, :nq], head_dim=self.d, eps=self.norm_eps,
+                              row_ssq=P["ssq"], status=self.status, stream=stream)
+            self._mark("qkv_rope_cache")
+            tg_gated_attention(qkv[:, :nq], ck, cv, P["cu"], P["cu_h"], self.hq, self.hkv,
+                               P["pos"], P["bias"], P["gamma"], 1.0, o=o, head_dim=self.d,
+                               workspace=P["attn_ws"], status=self.status, stream=stream)
+            self._mark("attention")
+            tg_linear(o, Wo, x, residual=x, row_ssq=P["ssq"], status=self.status,
+                      stream=stream)
+            self._mark("out_proj")
+        return x
+
+    def trim(self, kept_idx, out=None, stream=None):
+        """Keep only the kept rows of every layer's cache (lower-layer KV trimming).
+        `out`: list of (k, v) [K, Hkv d] bf16 pairs to fill, else allocated."""
+        P = self.planned
+        K = kept_idx.numel()
+        if out is None:
+            out = [(torch.empty((K, self.hkv * self.d), dtype=torch.bfloat16,
+                                device=self.device),
+                    torch.empty((K, self.hkv * self.d), dtype=torch.bfloat16,
+                                device=self.device)) for _ in self.layers]
+        if K:
+            for (ck, cv), (tk, tv) in zip(P["caches"], out):
+                tg_kv_compact(ck, cv, tk, tv, row_idx=kept_idx, status=self.status,
+                              stream=stream)
+        return out
+
+
 class GatedPrefill:
     """Buffers and call sequence of one gated prefill step on one device.
 
@@ -384,8 +483,14 @@ class GatedPrefill:
     """
 
     def __init__(self, gate: dict, layers: list, n_q_heads=16, n_kv_heads=8, head_dim=128,
-                 rope_theta=1.0e6, norm_eps=1e-6, seq_eps=1e-6, device="cuda"):
+                 rope_theta=1.0e6, norm_eps=1e-6, seq_eps=1e-6, device="cuda", lower=None,
+                 trim_lower_kv=True):
+        """`lower`: optional FullContextLayers below the gate.  The gate then scores
+        their output (the residual at the gate layer), the kept rows of that output go
+        up, and with `trim_lower_kv` their caches are trimmed to the kept rows."""
         self.device = torch.device(device)
+        self.lower = lower
+        self.trim_lower_kv = trim_lower_kv
         self.gate = gate
         self.layers = [l if isinstance(l, LayerWeights) else LayerWeights(**l) for l in layers]
         self.hq, self.hkv, self.d = n_q_heads, n_kv_heads, head_dim
@@ -395,6 +500,9 @@ class GatedPrefill:
         self.width = gate["W1"].shape[0]
         self.cos_sin = None
         self.status = torch.zeros(1, dtype=torch.int32, device=self.device)
+        if lower is not None:
+            lower.status = self.status  # one status word for the whole step
+            lower.stage_prefix = "lower_"
         self.planned = None
         # optional callable(stage_name) invoked after each launch (e.g. to record events)
         self.marker = None
@@ -452,6 +560,12 @@ class GatedPrefill:
             chain_ws=torch.zeros(max(16, tg_out_proj_qkv_workspace_size(K)), dtype=torch.uint8,
                                  device=dev),
         )
+        if self.lower is not None:
+            self.lower.plan(lengths, self.hidden)
+            if self.trim_lower_kv:
+                self.planned["lower_caches"] = [
+                    (torch.empty((K, self.hkv * self.d), **bf),
+                     torch.empty((K, self.hkv * self.d), **bf)) for _ in self.lower.layers]
         return self.planned
 
     def score(self, h, prunable, stream=None):
@@ -548,9 +662,15 @@ class GatedPrefill:
             main.wait_stream(self._side)
 
     def run(self, h, prunable, scores=None, stream=None):
-        """One gated prefill step.  The scorer always runs on h; with `scores` (raw
-        per-token scores, fp32 [T]) selection uses the sequence-normalised `scores`
-        instead of the scorer's own (the drawn planted-cluster workload)."""
+        """One gated prefill step.  With lower layers, h is the model's input rows and
+        the lower layers run first on all of them.  The scorer always runs on the
+        gate layer's residual; with `scores` (raw per-token scores, fp32 [T]) selection
+        uses the sequence-normalised `scores` instead of the scorer's own (the drawn
+        planted-cluster workload)."""
+        if self.lower is not None:
+            self.lower.marker = self.marker
+            h = self.lower.run(h, stream=stream)
+            self.lower.marker = None
         self.score(h, prunable, stream=stream)
         if scores is not None:
             P = self.planned
@@ -558,5 +678,9 @@ class GatedPrefill:
                            P["bias"], stream=stream)
             self._mark("seq_rmsnorm")
         self.select(prunable, stream=stream)
+        if self.lower is not None and self.trim_lower_kv:
+            P = self.planned
+            self.lower.trim(P["kept_idx"], out=P["lower_caches"], stream=stream)
+            self._mark("lower_kv_trim")
         self.upper_layers(h, stream=stream)
         return self.planned

@@ -248,3 +248,96 @@ def test_launch_overlap_gives_identical_results(tg):
         for (k0, v0), (k1, v1) in zip(got["caches"], ref["caches"]):
             assert torch.equal(k0, k1) and torch.equal(v0, v1)
     assert tg.tg_status_read(pipe.status) == 0
+
+
+# ------------------------------------------------------------------ layers below the gate
+#
+# Tolerances for the full-context layers, derived by `tests/tolerance_study.py lower`
+# (oracle run in float64 and with bf16 rounding where the CUDA path rounds): after two
+# lower layers x moves by max 0.029 / mean 0.0016, the K cache by 0.0054 max|k| in both
+# layers, the scorer's s by max 0.0014 / mean 0.0003 and z by max 0.0089 / mean 0.0020.
+# The bounds below sit 2-3x above those.
+
+def _lower_setup(tg, wl, n_lower):
+    lower = S.lower_layer_weights(wl, n_lower)
+    full = tg.FullContextLayers([_dev_dict(l) for l in lower], wl.n_q_heads, wl.n_kv_heads,
+                                wl.head_dim, wl.rope_theta)
+    return lower, full
+
+
+@pytest.mark.parametrize("lengths", [[300], [700, 1500, 333]])
+def test_full_context_layers_against_oracle(tg, lengths):
+    wl = S.custom(lengths, [8] * len(lengths), [64] * len(lengths), n_layers=0,
+                  name="lower")
+    h = S.hidden_rows(wl)
+    lower, full = _lower_setup(tg, wl, 2)
+    P = full.plan(wl.lengths, wl.hidden)
+    hd = h.cuda()
+    x = full.run(hd)
+    torch.cuda.synchronize()
+    assert torch.equal(hd.cpu(), h)  # the input rows are left alone
+    cu = wl.cu_seqlens()
+    xr = O.as_f64(h)
+    for i, L in enumerate(lower):
+        xr, k, v = O.full_context_layer(xr, L["Wqkv"], L["Wo"], cu, wl.n_q_heads,
+                                        wl.n_kv_heads, wl.head_dim, wl.rope_theta)
+        kc = O.as_f64(P["caches"][i][0].cpu()).reshape(k.shape)
+        vc = O.as_f64(P["caches"][i][1].cpu()).reshape(v.shape)
+        assert np.abs(kc - k).max() <= 2.0 ** -6 * np.abs(k).max()
+        assert np.abs(vc - v).max() <= 2.0 ** -6 * np.abs(v).max()
+    err = np.abs(O.as_f64(x.cpu()) - xr)
+    tol, tol_mean = _x_tol(xr, 2)
+    assert np.all(err <= tol), err.max()
+    assert err.mean() <= tol_mean, err.mean()
+    assert tg.tg_status_read(full.status) == 0
+
+
+def test_pipeline_with_lower_layers_and_kv_trim(tg):
+    """Two full-context layers, the gate on their output, selection on drawn scores
+    (so that the kept set does not hinge on rounding), one gated layer above; the
+    lower caches trimmed to the kept rows."""
+    wl = S.custom([700, 1500, 333], [16, 64, 5], [100, 800, 300], n_layers=1,
+                  planted_cluster=True, name="ragged3_lower")
+    h = S.hidden_rows(wl)
+    gate = S.gate_weights(wl)
+    upper = [S.layer_weights(wl, 0)]
+    pr = S.prunable_mask(wl)
+    drawn = S.drawn_scores(wl)
+    lower, full = _lower_setup(tg, wl, 2)
+    pipe = tg.GatedPrefill(_dev_dict(gate), [_dev_dict(l) for l in upper], wl.n_q_heads,
+                           wl.n_kv_heads, wl.head_dim, wl.rope_theta, lower=full)
+    P = pipe.plan(wl.lengths, wl.questions, wl.budgets)
+    hd = h.cuda()
+    pipe.run(hd, pr.cuda(), scores=drawn.cuda())
+    torch.cuda.synchronize()
+    cu = wl.cu_seqlens()
+    ref = O.prefill(h, pr, cu, wl.budgets, gate, upper, wl.n_q_heads, wl.n_kv_heads,
+                    wl.head_dim, wl.rope_theta, scores=drawn, lower_layers=lower)
+    # the residual at the gate layer
+    xg = O.as_f64(full.planned["x"].cpu())
+    err = np.abs(xg - ref["h_gate"])
+    tol, tol_mean = _x_tol(ref["h_gate"], 2)
+    assert np.all(err <= tol) and err.mean() <= tol_mean, (err.max(), err.mean())
+    # the scorer reads that residual
+    s_ref = O.gate_score(ref["h_gate"], gate["norm_w"], gate["W1"], gate["w2"])
+    s_err = np.abs(P["s"].cpu().double().numpy() - s_ref)
+    assert s_err.max() <= 5e-3 and s_err.mean() <= 1e-3, (s_err.max(), s_err.mean())
+    # selection on the drawn scores
+    same = _check_selection(wl, pr.numpy(), ref["z"], ref["cu_kept"],
+                            P["kept_idx"].cpu().numpy(), P["ck_h"].numpy())
+    assert same
+    kept = P["kept_idx"].cpu().numpy()
+    assert np.array_equal(P["kept_pos"].cpu().numpy(), ref["kept_pos"])
+    # trimmed lower caches: exactly the kept rows of the full-length ones, and those
+    # against the oracle's trimmed caches
+    for i, ((tk, tv), (fk, fv)) in enumerate(zip(P["lower_caches"], full.planned["caches"])):
+        assert torch.equal(tk.cpu(), fk.cpu()[kept]) and torch.equal(tv.cpu(), fv.cpu()[kept])
+        k_ref, v_ref = ref["lower_caches"][i]
+        kc = O.as_f64(tk.cpu()).reshape(k_ref.shape)
+        assert np.abs(kc - k_ref).max() <= 2.0 ** -6 * np.abs(k_ref).max()
+    # one gated layer above: three layers of rounding in the residual stream
+    x = O.as_f64(P["x"].cpu())
+    err = np.abs(x - ref["x"])
+    tol, tol_mean = _x_tol(ref["x"], 3)
+    assert np.all(err <= tol) and err.mean() <= tol_mean, (err.max(), err.mean())
+    assert tg.tg_status_read(pipe.status) == 0

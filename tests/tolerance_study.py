@@ -51,6 +51,34 @@ def study(wl, report=(1, 2, 4, 8, 16, 28)):
                   f"|x|max {np.abs(x64).max():.2f}", flush=True)
 
 
+def study_lower(wl, n_lower):
+    """Layers below the gate, float64 against bf16-rounded, and what that does to the
+    gate's scores s and z read from their output."""
+    h, pr, gate = S.hidden_rows(wl), S.prunable_mask(wl), S.gate_weights(wl)
+    cu = wl.cu_seqlens()
+    pos = O.request_positions(cu)
+    zero_bias = np.zeros(wl.total_tokens)
+    x64 = O.as_f64(h)
+    xr = x64.copy()
+    for L in S.lower_layer_weights(wl, n_lower):
+        x64, _, _ = O.full_context_layer(x64, L["Wqkv"], L["Wo"], cu, wl.n_q_heads,
+                                         wl.n_kv_heads, wl.head_dim, wl.rope_theta)
+        Lg = dict(L, gamma=np.zeros(wl.n_q_heads), beta=1.0)
+        xr = layer_rounded(xr, Lg, cu, pos, zero_bias, wl)
+    e = np.abs(xr - x64)
+    s64 = O.gate_score(x64, gate["norm_w"], gate["W1"], gate["w2"])
+    sr = O.gate_score(xr, gate["norm_w"], gate["W1"], gate["w2"])
+    z64, _ = O.sequence_rmsnorm(s64, cu, pr)
+    zr, _ = O.sequence_rmsnorm(sr, cu, pr)
+    print(f"{wl.name} {n_lower} lower layers: x max {e.max():.4f} mean {e.mean():.5f}; "
+          f"s max {np.abs(sr - s64).max():.5f} mean {np.abs(sr - s64).mean():.6f}; "
+          f"z max {np.abs(zr - z64).max():.5f} mean {np.abs(zr - z64).mean():.6f}", flush=True)
+
+
 if __name__ == "__main__":
+    if len(sys.argv) > 1 and sys.argv[1] == "lower":
+        study_lower(S.custom([700, 1500, 333], [16, 64, 5], [100, 800, 300], n_layers=1,
+                             name="ragged3"), 2)
+        sys.exit(0)
     study(S.custom([700, 1500, 333], [16, 64, 5], [100, 800, 300], n_layers=2, name="ragged3"))
     study(S.n16k())
