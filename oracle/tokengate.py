@@ -31,6 +31,12 @@ listed with its reason in the design notes of the repository):
     z_c = 0 for non-prunable keys.
   * upper layers keep KV only for kept tokens ([farwalk] How does TokenGate learned
     token pruning work?; [digest] 方法关键点).
+  * a full transformer layer body (optional, both below and above the gate): the
+    Qwen3-shaped layer the pages evaluate on adds a weighted pre-attention RMSNorm,
+    per-head RMSNorm of q and k before RoPE (QK-norm) and a SwiGLU MLP behind its own
+    weighted RMSNorm; the pages say pruned tokens skip the upper MLPs too ([fluxbbs]
+    门控到底插在模型的哪个位置).  Reading: eps 1e-6 everywhere, QK-norm weight shared by
+    the heads, MLP x + W_down (SiLU(W_gate b) * W_up b) with b the normalised x.
   * layers below the gate see every token with ordinary causal attention; their KV
     may optionally be trimmed to the kept tokens as well ([digest] 方法关键点;
     [aiwillknow] 图1(a)(b)).  Reading: trimming keeps exactly the gate's kept rows.
@@ -46,6 +52,7 @@ __all__ = [
     "select_topk", "gather_rows", "rope", "rope_angles", "temperature",
     "gated_attention", "kv_compact", "gated_layer", "prefill", "silu",
     "request_positions", "causal_attention", "full_context_layer",
+    "rmsnorm_heads", "swiglu_mlp",
 ]
 
 
@@ -291,30 +298,68 @@ def kv_compact(K, V, row_idx=None):
     return K[i], V[i]
 
 
+# ------------------------------------------------------------------ layer body parts
+
+def rmsnorm_heads(x, weight, eps: float = 1e-6) -> np.ndarray:
+    """RMSNorm of each head's d values (the last axis) times a weight [d] shared by
+    the heads: the QK-norm of a Qwen3-shaped layer, applied to q and k before RoPE."""
+    x = as_f64(x)
+    return x / np.sqrt(np.mean(x * x, axis=-1, keepdims=True) + eps) * as_f64(weight)
+
+
+def swiglu_mlp(x, norm_w, W_gate, W_up, W_down, eps: float = 1e-6) -> np.ndarray:
+    """Residual SwiGLU MLP: x + W_down (SiLU(W_gate b) * (W_up b)), b = RMSNorm(x) * norm_w.
+    W_gate and W_up are [F, H], W_down is [H, F].  Pruned tokens never reach it above
+    the gate ([fluxbbs] 门控到底插在模型的哪个位置)."""
+    x = as_f64(x)
+    b = rmsnorm_rows(x, norm_w, eps)
+    g = b @ as_f64(W_gate).T
+    u = b @ as_f64(W_up).T
+    return x + (silu(g) * u) @ as_f64(W_down).T
+
+
+def _attention_inputs(x, Wqkv, pos, n_q_heads, n_kv_heads, head_dim, theta, eps,
+                      attn_norm=None, q_norm=None, k_norm=None):
+    """a = RMSNorm(x) (times attn_norm), [q, k, v] = a Wqkv^T, optional QK-norm, then
+    RoPE of q and k at `pos`."""
+    a = rmsnorm_rows(x, attn_norm, eps)
+    qkv = a @ as_f64(Wqkv).T
+    nq, nk = n_q_heads * head_dim, n_kv_heads * head_dim
+    rows = x.shape[0]
+    q = qkv[:, :nq].reshape(rows, n_q_heads, head_dim)
+    k = qkv[:, nq:nq + nk].reshape(rows, n_kv_heads, head_dim)
+    v = qkv[:, nq + nk:].reshape(rows, n_kv_heads, head_dim)
+    if q_norm is not None:
+        q = rmsnorm_heads(q, q_norm, eps)
+    if k_norm is not None:
+        k = rmsnorm_heads(k, k_norm, eps)
+    return a, qkv, rope(q, pos, theta), rope(k, pos, theta), v
+
+
 # ------------------------------------------------------------------ one gated layer
 
 def gated_layer(x, Wqkv, Wo, gamma, beta, cu_kept, kept_pos, kept_bias,
                 n_q_heads: int, n_kv_heads: int, head_dim: int,
-                theta: float = 1.0e6, eps: float = 1e-6):
+                theta: float = 1.0e6, eps: float = 1e-6,
+                attn_norm=None, q_norm=None, k_norm=None, mlp=None):
     """One upper layer on the kept rows: x + Wo . Attn(RoPE(Wq a), RoPE(Wk a), Wv a), a = RMSNorm(x).
 
     Wqkv [(Hq + 2 Hkv) d, H] holds Wq, Wk, Wv row blocks; Wo is [H, Hq d].  RoPE uses
-    the original positions.  Returns (x_out, K_cache, V_cache, parts) with the
-    intermediates in `parts` for teacher-forced checks.
+    the original positions.  Optional full-layer parts: `attn_norm` [H] weights the
+    pre-attention RMSNorm, `q_norm` / `k_norm` [d] turn on QK-norm, `mlp` (a dict with
+    norm_w, W_gate, W_up, W_down) appends the SwiGLU MLP.  Returns (x_out, K_cache,
+    V_cache, parts) with the intermediates in `parts` for teacher-forced checks.
     """
     x = as_f64(x)
-    a = rmsnorm_rows(x, None, eps)
-    qkv = a @ as_f64(Wqkv).T
-    nq, nk = n_q_heads * head_dim, n_kv_heads * head_dim
+    a, qkv, q, k, v = _attention_inputs(x, Wqkv, kept_pos, n_q_heads, n_kv_heads, head_dim,
+                                        theta, eps, attn_norm, q_norm, k_norm)
     Kt = x.shape[0]
-    q = qkv[:, :nq].reshape(Kt, n_q_heads, head_dim)
-    k = qkv[:, nq:nq + nk].reshape(Kt, n_kv_heads, head_dim)
-    v = qkv[:, nq + nk:].reshape(Kt, n_kv_heads, head_dim)
-    q = rope(q, kept_pos, theta)
-    k = rope(k, kept_pos, theta)
     o, lse = gated_attention(q, k, v, cu_kept, kept_pos, kept_bias, gamma, beta)
-    x_out = x + o.reshape(Kt, nq) @ as_f64(Wo).T
-    parts = {"a": a, "qkv": qkv, "q": q, "k": k, "v": v, "o": o, "lse": lse}
+    x_out = x + o.reshape(Kt, n_q_heads * head_dim) @ as_f64(Wo).T
+    parts = {"a": a, "qkv": qkv, "q": q, "k": k, "v": v, "o": o, "lse": lse,
+             "x_attn": x_out}
+    if mlp is not None:
+        x_out = swiglu_mlp(x_out, mlp["norm_w"], mlp["W_gate"], mlp["W_up"], mlp["W_down"], eps)
     return x_out, k, v, parts
 
 
@@ -358,22 +403,27 @@ def causal_attention(Q, K, V, cu_seqlens, block: int = 1024):
 
 
 def full_context_layer(x, Wqkv, Wo, cu_seqlens, n_q_heads: int, n_kv_heads: int,
-                       head_dim: int, theta: float = 1.0e6, eps: float = 1e-6):
+                       head_dim: int, theta: float = 1.0e6, eps: float = 1e-6,
+                       attn_norm=None, q_norm=None, k_norm=None, mlp=None):
     """One layer below the gate on all tokens: x + Wo . Attn(RoPE(Wq a), RoPE(Wk a), Wv a)
     with a = RMSNorm(x), RoPE at each token's position in its request and ordinary
-    causal attention.  Returns (x_out, K_cache, V_cache): the full-length post-RoPE
-    K and V of this layer, [T, Hkv, d]."""
+    causal attention; the optional full-layer parts as in `gated_layer`.  Returns
+    (x_out, K_cache, V_cache): the full-length post-RoPE K and V, [T, Hkv, d]."""
     x = as_f64(x)
-    a = rmsnorm_rows(x, None, eps)
-    qkv = a @ as_f64(Wqkv).T
-    nq, nk = n_q_heads * head_dim, n_kv_heads * head_dim
     T = x.shape[0]
     pos = request_positions(cu_seqlens)
-    q = rope(qkv[:, :nq].reshape(T, n_q_heads, head_dim), pos, theta)
-    k = rope(qkv[:, nq:nq + nk].reshape(T, n_kv_heads, head_dim), pos, theta)
-    v = qkv[:, nq + nk:].reshape(T, n_kv_heads, head_dim)
+    _, _, q, k, v = _attention_inputs(x, Wqkv, pos, n_q_heads, n_kv_heads, head_dim, theta,
+                                      eps, attn_norm, q_norm, k_norm)
     o = causal_attention(q, k, v, cu_seqlens)
-    return x + o.reshape(T, nq) @ as_f64(Wo).T, k, v
+    x = x + o.reshape(T, n_q_heads * head_dim) @ as_f64(Wo).T
+    if mlp is not None:
+        x = swiglu_mlp(x, mlp["norm_w"], mlp["W_gate"], mlp["W_up"], mlp["W_down"], eps)
+    return x, k, v
+
+
+def _body_parts(L) -> dict:
+    """The optional full-layer parts present in a layer's weight dict."""
+    return {k: L[k] for k in ("attn_norm", "q_norm", "k_norm", "mlp") if L.get(k) is not None}
 
 
 def prefill(h, prunable, cu_seqlens, budgets, gate, layers, n_q_heads, n_kv_heads,
@@ -382,7 +432,8 @@ def prefill(h, prunable, cu_seqlens, budgets, gate, layers, n_q_heads, n_kv_head
     """Lower layers + gate + selection + gathered upper layers, end to end.
 
     `gate` holds norm_w, W1, w2; `layers` (above the gate) and `lower_layers` (below
-    it) are lists of dicts with Wqkv and Wo (plus gamma, beta above the gate).  The
+    it) are lists of dicts with Wqkv and Wo (plus gamma, beta above the gate, and
+    optionally attn_norm, q_norm, k_norm and mlp for a full layer body).  The
     lower layers run on every token; the gate reads their output, the residual at
     the gate layer.  Their K/V caches come back both full-length and trimmed to the
     kept rows.  With `scores` given, selection consumes those raw scores instead of
@@ -391,7 +442,8 @@ def prefill(h, prunable, cu_seqlens, budgets, gate, layers, n_q_heads, n_kv_head
     lower_full = []
     for L in lower_layers:
         h, k, v = full_context_layer(h, L["Wqkv"], L["Wo"], cu_seqlens, n_q_heads,
-                                     n_kv_heads, head_dim, theta, norm_eps)
+                                     n_kv_heads, head_dim, theta, norm_eps,
+                                     **_body_parts(L))
         lower_full.append((k, v))
     s = gate_score(h, gate["norm_w"], gate["W1"], gate["w2"], norm_eps) if scores is None \
         else as_f64(scores)
@@ -404,7 +456,7 @@ def prefill(h, prunable, cu_seqlens, budgets, gate, layers, n_q_heads, n_kv_head
     for L in layers:
         x, k, v, _ = gated_layer(x, L["Wqkv"], L["Wo"], L["gamma"], L["beta"], cu_kept,
                                  kept_pos, kept_bias, n_q_heads, n_kv_heads, head_dim,
-                                 theta, norm_eps)
+                                 theta, norm_eps, **_body_parts(L))
         caches.append((k, v))
     return {"s": s, "z": z, "bias": bias, "cu_kept": cu_kept, "kept_idx": kept_idx,
             "kept_pos": kept_pos, "kept_bias": kept_bias, "x": x, "caches": caches,

@@ -18,6 +18,9 @@ Recipe (all draws on the CPU with ``torch.Generator``):
     then Wv), Wo [H, Hq*d] ~ N(0, 0.02) bf16, gamma [Hq] ~ U(0.5, 2) fp32, beta = 1;
   * layers below the gate (full context): Wqkv and Wo drawn the same way from their
     own stream, no gamma or beta;
+  * full layer body (optional): attention-norm weight [H], QK-norm weights [d] and the
+    MLP norm weight [H] ~ U(0.8, 1.2) fp32; W_gate, W_up [F, H] and W_down [H, F]
+    ~ N(0, 0.02) bf16 with F = 6144, from their own stream;
   * prunable mask: the first D_b tokens of each request are the document (prunable),
     the last Q_b tokens are the question (never pruned);
   * drawn scores (planted-cluster workload): s ~ N(0, 1) fp32 with +4 added on 64
@@ -46,6 +49,8 @@ _LAYER_STREAM = 2_000_003
 _LAYOUT_STREAM = 3_000_017
 _SCORE_STREAM = 4_000_037
 _LOWER_STREAM = 5_000_011
+_BODY_STREAM = 6_000_023
+FFN = 6144  # SwiGLU width of the Qwen3-1.7B-shaped layer
 
 
 @dataclass(frozen=True)
@@ -185,6 +190,26 @@ def lower_layer_weights(wl: Workload, n_layers: int) -> list:
         Wo = (torch.randn((H, hq * d), generator=g) * 0.02).to(torch.bfloat16)
         out.append({"Wqkv": Wqkv, "Wo": Wo})
     return out
+
+
+def layer_body_parts(wl: Workload, layer: int, lower: bool = False, ffn: int = FFN) -> dict:
+    """The optional parts of a full layer body for layer `layer` (above the gate, or
+    below it with `lower`): attn_norm, q_norm, k_norm and mlp (norm_w, W_gate, W_up,
+    W_down)."""
+    H, d = wl.hidden, wl.head_dim
+    g = torch.Generator().manual_seed(_BODY_STREAM + 7919 * wl.weight_seed + 104729 * int(lower)
+                                      + layer)
+
+    def gain(n):
+        return (0.8 + 0.4 * torch.rand((n,), generator=g)).to(torch.float32)
+
+    attn_norm, q_norm, k_norm = gain(H), gain(d), gain(d)
+    mlp_norm = gain(H)
+    W_gate = (torch.randn((ffn, H), generator=g) * 0.02).to(torch.bfloat16)
+    W_up = (torch.randn((ffn, H), generator=g) * 0.02).to(torch.bfloat16)
+    W_down = (torch.randn((H, ffn), generator=g) * 0.02).to(torch.bfloat16)
+    return {"attn_norm": attn_norm, "q_norm": q_norm, "k_norm": k_norm,
+            "mlp": {"norm_w": mlp_norm, "W_gate": W_gate, "W_up": W_up, "W_down": W_down}}
 
 
 def prunable_mask(wl: Workload) -> torch.Tensor:

@@ -484,3 +484,94 @@ def test_prefill_with_lower_layers_composes_and_trims():
         assert kf.shape[0] == wl.total_tokens and kt.shape[0] == len(out["kept_idx"])
         np.testing.assert_array_equal(kt, kf[out["kept_idx"]])
         np.testing.assert_array_equal(vt, vf[out["kept_idx"]])
+
+
+# ------------------------------------------------------------------ full layer body
+
+def test_rmsnorm_heads_against_library():
+    rng = np.random.default_rng(40)
+    x = rng.normal(size=(5, 3, 16)) * 2.0
+    w = rng.uniform(0.8, 1.2, size=16)
+    want = F.rms_norm(torch.tensor(x), (16,), torch.tensor(w), eps=1e-6).numpy()
+    np.testing.assert_allclose(O.rmsnorm_heads(x, w), want, atol=1e-12)
+
+
+def test_swiglu_mlp_against_library():
+    rng = np.random.default_rng(41)
+    H, Fw = 24, 40
+    x = rng.normal(size=(7, H))
+    nw = rng.uniform(0.8, 1.2, size=H)
+    Wg, Wu, Wd = (rng.normal(size=s) * 0.3 for s in ((Fw, H), (Fw, H), (H, Fw)))
+    xt = torch.tensor(x)
+    b = F.rms_norm(xt, (H,), torch.tensor(nw), eps=1e-6)
+    want = xt + F.linear(F.silu(F.linear(b, torch.tensor(Wg))) * F.linear(b, torch.tensor(Wu)),
+                         torch.tensor(Wd))
+    np.testing.assert_allclose(O.swiglu_mlp(x, nw, Wg, Wu, Wd), want.numpy(), atol=1e-12)
+    np.testing.assert_allclose(O.swiglu_mlp(x, nw, Wg, Wu, np.zeros_like(Wd)), x, atol=0)
+
+
+def _body_case(seed, Hq=4, Hkv=2, d=8, H=32, Fw=48, n=11):
+    rng = np.random.default_rng(seed)
+    x = rng.normal(size=(n, H))
+    Wqkv = rng.normal(size=((Hq + 2 * Hkv) * d, H)) * 0.2
+    Wo = rng.normal(size=(H, Hq * d)) * 0.2
+    parts = {"attn_norm": rng.uniform(0.8, 1.2, H), "q_norm": rng.uniform(0.8, 1.2, d),
+             "k_norm": rng.uniform(0.8, 1.2, d),
+             "mlp": {"norm_w": rng.uniform(0.8, 1.2, H),
+                     "W_gate": rng.normal(size=(Fw, H)) * 0.2,
+                     "W_up": rng.normal(size=(Fw, H)) * 0.2,
+                     "W_down": rng.normal(size=(H, Fw)) * 0.2}}
+    pos = np.sort(rng.choice(4 * n, size=n, replace=False))
+    bias = rng.normal(size=n)
+    gamma = rng.uniform(0.5, 2.0, Hq)
+    return x, Wqkv, Wo, parts, pos, bias, gamma
+
+
+def test_full_layer_cache_is_qk_normed_before_rope():
+    """K cache = RoPE(RMSNorm_head(W_k RMSNorm(x; attn_norm); k_norm)), built here from
+    torch's rms_norm and linear (RoPE itself is pinned above)."""
+    x, Wqkv, Wo, parts, pos, bias, gamma = _body_case(42)
+    _, k, v, _ = O.gated_layer(x, Wqkv, Wo, gamma, 1.0, [0, 11], pos, bias, 4, 2, 8, 1e4,
+                               **parts)
+    a = F.rms_norm(torch.tensor(x), (32,), torch.tensor(parts["attn_norm"]), eps=1e-6)
+    kk = F.linear(a, torch.tensor(Wqkv[32:48])).view(11, 2, 8)
+    kn = F.rms_norm(kk, (8,), torch.tensor(parts["k_norm"]), eps=1e-6).numpy()
+    np.testing.assert_allclose(k, O.rope(kn, pos, 1e4), atol=1e-12)
+    vv = F.linear(a, torch.tensor(Wqkv[48:])).view(11, 2, 8).numpy()
+    np.testing.assert_allclose(v, vv, atol=1e-12)
+
+
+def test_qk_norm_removes_the_scale_of_q_and_k():
+    """With QK-norm, scaling W_q and W_k by 3 changes nothing (eps aside); without it the
+    logits scale by 9 and the output moves."""
+    x, Wqkv, Wo, parts, pos, bias, gamma = _body_case(43)
+    W2 = Wqkv.copy()
+    W2[:48] *= 3.0
+    a1, *_ = O.gated_layer(x, Wqkv, Wo, gamma, 1.0, [0, 11], pos, bias, 4, 2, 8, 1e4, **parts)
+    a2, *_ = O.gated_layer(x, W2, Wo, gamma, 1.0, [0, 11], pos, bias, 4, 2, 8, 1e4, **parts)
+    np.testing.assert_allclose(a1, a2, atol=1e-5)
+    no_qk = {k: v for k, v in parts.items() if k not in ("q_norm", "k_norm")}
+    b1, *_ = O.gated_layer(x, Wqkv, Wo, gamma, 1.0, [0, 11], pos, bias, 4, 2, 8, 1e4, **no_qk)
+    b2, *_ = O.gated_layer(x, W2, Wo, gamma, 1.0, [0, 11], pos, bias, 4, 2, 8, 1e4, **no_qk)
+    assert np.abs(b1 - b2).max() > 1e-2
+
+
+def test_full_layer_mlp_follows_attention():
+    x, Wqkv, Wo, parts, pos, bias, gamma = _body_case(44)
+    m = parts["mlp"]
+    xo, _, _, pp = O.gated_layer(x, Wqkv, Wo, gamma, 1.0, [0, 11], pos, bias, 4, 2, 8, 1e4,
+                                 **parts)
+    no_mlp = {k: v for k, v in parts.items() if k != "mlp"}
+    xa, _, _, _ = O.gated_layer(x, Wqkv, Wo, gamma, 1.0, [0, 11], pos, bias, 4, 2, 8, 1e4,
+                                **no_mlp)
+    np.testing.assert_allclose(pp["x_attn"], xa, atol=1e-13)
+    np.testing.assert_allclose(xo, O.swiglu_mlp(xa, m["norm_w"], m["W_gate"], m["W_up"],
+                                                m["W_down"]), atol=1e-13)
+    # the same body below the gate: full context layer = gated layer with nothing pruned
+    cu = [0, 6, 11]
+    rp = O.request_positions(cu)
+    f, kf, _ = O.full_context_layer(x, Wqkv, Wo, cu, 4, 2, 8, 1e4, **parts)
+    g, kg, _, _ = O.gated_layer(x, Wqkv, Wo, np.zeros(4), 1.0, cu, rp, bias, 4, 2, 8, 1e4,
+                                **parts)
+    np.testing.assert_allclose(f, g, atol=1e-12)
+    np.testing.assert_allclose(kf, kg, atol=1e-12)
