@@ -376,6 +376,60 @@ int tg_qkv_rope_cache(const tg_bf16* x, int64_t ld_x, const tg_bf16* w_qkv, int6
                       int64_t ld_ssq_in, uint32_t* status, tg_stream_t stream);
 
 /*
+ * tg_qkv_rope_cache with QK-norm, for a full (Qwen3-shaped) layer body: each Q and K
+ * head of a row is RMS-normalised over its head_dim values and multiplied by q_norm_w
+ * or k_norm_w (float32 [head_dim], shared by the heads) before RoPE:
+ *   Q_h <- Q_h / sqrt(mean(Q_h^2) + eps) * q_norm_w  (K likewise with k_norm_w)
+ * in fp32 from the accumulators, then RoPE and the single rounding to bf16.  The layer
+ * body comes from the page [fluxbbs] (门控到底插在模型的哪个位置) evaluating a Qwen3 model;
+ * the QK-norm itself is that model's, not the pages'.  Requires row_ssq_in and Q/K/V
+ * widths that are multiples of 256 (CTA-pair kernel): else TG_ERR_INVALID_ARGUMENT /
+ * TG_ERR_UNSUPPORTED_SHAPE.  A weighted pre-attention RMSNorm is folded into w_qkv
+ * beforehand with tg_fold_norm_weight.  Other arguments as tg_qkv_rope_cache.
+ */
+int tg_qkv_qknorm_rope_cache(const tg_bf16* x, int64_t ld_x, const tg_bf16* w_qkv,
+                             int64_t ld_w, int64_t M, int hidden, int n_q_heads, int n_kv_heads,
+                             int head_dim, float eps, const float* q_norm_w,
+                             const float* k_norm_w, const int32_t* pos, const float* cos_sin,
+                             int max_pos, tg_bf16* q_out, int64_t ld_q, tg_bf16* cache_k,
+                             tg_bf16* cache_v, int64_t ld_cache, int64_t slot_offset,
+                             const float* row_ssq_in, int64_t ld_ssq_in, uint32_t* status,
+                             tg_stream_t stream);
+
+/*
+ * Up half of the SwiGLU MLP of a full layer body (pruned tokens skip the upper MLPs as
+ * well: [fluxbbs] 门控到底插在模型的哪个位置):
+ *   b = RMSNorm(x) (eps; the norm weight folded into w_gu by tg_pack_gate_up),
+ *   h_out[m, f] = SiLU(b . W_gate[f]) * (b . W_up[f]),  SiLU(v) = v / (1 + e^-v)
+ * evaluated in fp32 from the two accumulators, one rounding to bf16.
+ * x: bf16 [M, hidden] (ld_x); row_ssq_in: float32 [M, hidden/128] (ld_ssq_in, required:
+ * the row sums of squares tg_linear's row_ssq_out gives); w_gu: bf16 [2 ffn, hidden]
+ * (ld_w) in the layout tg_pack_gate_up writes; h_out: bf16 [M, ffn] (ld_h).  hidden and
+ * ffn multiples of 128, strides multiples of 8, 16-byte aligned bases.  CTA-pair
+ * tcgen05 GEMM over 256 x 256 tiles of the interleaved weight.  The down projection is
+ * tg_linear(h_out, W_down, x, residual = x).  status may be NULL.
+ */
+int tg_swiglu(const tg_bf16* x, int64_t ld_x, const tg_bf16* w_gu, int64_t ld_w, int64_t M,
+              int hidden, int ffn, float eps, const float* row_ssq_in, int64_t ld_ssq_in,
+              tg_bf16* h_out, int64_t ld_h, uint32_t* status, tg_stream_t stream);
+
+/*
+ * Weight preparation, once per model load (not per step).
+ * tg_fold_norm_weight: out[r, c] = bf16(w[r, c] * norm_w[c]) for an RMSNorm weight that
+ *   multiplies the input of w (w: bf16 [rows, cols], ld_w; out may equal w).
+ * tg_pack_gate_up: out = bf16 [2 ffn, hidden] with rows 128 j .. 128 j + 63 = W_gate rows
+ *   64 j .. 64 j + 63 and rows 128 j + 64 .. 128 j + 127 = the same W_up rows, every
+ *   column c multiplied by norm_w[c] (norm_w may be NULL: no scaling).  ffn multiple of
+ *   64.  w_gate, w_up: bf16 [ffn, hidden] (ld_gate, ld_up); out must not alias them.
+ * Both are asynchronous on `stream`.
+ */
+int tg_fold_norm_weight(const tg_bf16* w, int64_t ld_w, int64_t rows, int cols,
+                        const float* norm_w, tg_bf16* out, int64_t ld_out, tg_stream_t stream);
+int tg_pack_gate_up(const tg_bf16* w_gate, int64_t ld_gate, const tg_bf16* w_up, int64_t ld_up,
+                    int ffn, int hidden, const float* norm_w, tg_bf16* out, int64_t ld_out,
+                    tg_stream_t stream);
+
+/*
  * One layer boundary in one launch: the output projection of gated layer l followed by
  * gated layer l+1's QKV projection, RoPE and KV-cache write, with identical results to
  *   tg_linear(o, W_o, x, residual = x, row_ssq)            (x <- x + o W_o^T)

@@ -27,6 +27,7 @@ __all__ = [
     "tg_gate_score_noalloc", "tg_seq_rmsnorm", "tg_gather_rope", "tg_kv_compact", "tg_gated_attention", "tg_linear",
     "tg_status_clear", "tg_status_read", "tg_set_launch_overlap", "tg_get_launch_overlap",
     "tg_prefetch_l2", "tg_out_proj_qkv_next", "tg_out_proj_qkv_workspace_size",
+    "tg_swiglu", "tg_fold_norm_weight", "tg_pack_gate_up", "prepare_layer",
     "GatedPrefill", "FullContextLayers", "LayerWeights", "STATUS_TIMEOUT", "STATUS_BUDGET",
     "STATUS_BOUNDS", "STATUS_WORKSPACE",
 ]
@@ -317,8 +318,10 @@ def tg_linear(a, w, c=None, rmsnorm=False, eps=1e-6, residual=None, row_ssq=None
 
 def tg_qkv_rope_cache(x, w_qkv, pos, cos_sin, cache_k, cache_v, n_q_heads, n_kv_heads,
                       q_out=None, head_dim=128, eps=1e-6, slot_offset=0, row_ssq=None,
-                      status=None, stream=None):
-    """Fused QKV projection (RMSNorm folded) + RoPE at `pos` + compacted KV-cache write."""
+                      status=None, stream=None, q_norm_w=None, k_norm_w=None):
+    """Fused QKV projection (RMSNorm folded) + RoPE at `pos` + compacted KV-cache write;
+    with q_norm_w / k_norm_w (float32 [head_dim]) also QK-norm before RoPE
+    (tg_qkv_qknorm_rope_cache)."""
     ld_x, ld_w = _mat(x, "x"), _mat(w_qkv, "w_qkv")
     M, hidden = x.shape
     if q_out is None:
@@ -328,14 +331,65 @@ def tg_qkv_rope_cache(x, w_qkv, pos, cos_sin, cache_k, cache_v, n_q_heads, n_kv_
     if _mat(cache_v, "cache_v") != ld_c:
         raise ValueError("cache_k and cache_v must share a row stride")
     ld_ssq = _mat(row_ssq, "row_ssq") if row_ssq is not None else 0
-    rc = lib.tg_qkv_rope_cache(_ptr(x), ld_x, _ptr(w_qkv), ld_w, M, hidden, n_q_heads, n_kv_heads,
-                               head_dim, float(eps), _ptr(pos), _ptr(cos_sin), cos_sin.shape[0],
-                               _ptr(q_out), ld_q, _ptr(cache_k), _ptr(cache_v), ld_c,
-                               int(slot_offset), _ptr(row_ssq), ld_ssq, _ptr(status),
-                               _stream(stream))
-    _check(rc, "tg_qkv_rope_cache")
+    if q_norm_w is not None or k_norm_w is not None:
+        rc = lib.tg_qkv_qknorm_rope_cache(_ptr(x), ld_x, _ptr(w_qkv), ld_w, M, hidden, n_q_heads,
+                                          n_kv_heads, head_dim, float(eps), _ptr(q_norm_w),
+                                          _ptr(k_norm_w), _ptr(pos), _ptr(cos_sin),
+                                          cos_sin.shape[0], _ptr(q_out), ld_q, _ptr(cache_k),
+                                          _ptr(cache_v), ld_c, int(slot_offset), _ptr(row_ssq),
+                                          ld_ssq, _ptr(status), _stream(stream))
+        _check(rc, "tg_qkv_qknorm_rope_cache")
+    else:
+        rc = lib.tg_qkv_rope_cache(_ptr(x), ld_x, _ptr(w_qkv), ld_w, M, hidden, n_q_heads,
+                                   n_kv_heads, head_dim, float(eps), _ptr(pos), _ptr(cos_sin),
+                                   cos_sin.shape[0], _ptr(q_out), ld_q, _ptr(cache_k),
+                                   _ptr(cache_v), ld_c, int(slot_offset), _ptr(row_ssq), ld_ssq,
+                                   _ptr(status), _stream(stream))
+        _check(rc, "tg_qkv_rope_cache")
     _count()
     return q_out
+
+
+def tg_swiglu(x, w_gu, row_ssq, h_out=None, eps=1e-6, status=None, stream=None):
+    """h = SiLU(b W_gate^T) * (b W_up^T), b = RMSNorm(x) from its row sums of squares;
+    w_gu from tg_pack_gate_up (norm weight folded, rows interleaved)."""
+    ld_x, ld_w, ld_ssq = _mat(x, "x"), _mat(w_gu, "w_gu"), _mat(row_ssq, "row_ssq")
+    M, hidden = x.shape
+    ffn = w_gu.shape[0] // 2
+    if h_out is None:
+        h_out = torch.empty((M, ffn), dtype=x.dtype, device=x.device)
+    ld_h = _mat(h_out, "h_out")
+    rc = lib.tg_swiglu(_ptr(x), ld_x, _ptr(w_gu), ld_w, M, hidden, ffn, float(eps),
+                       _ptr(row_ssq), ld_ssq, _ptr(h_out), ld_h, _ptr(status), _stream(stream))
+    _check(rc, "tg_swiglu")
+    _count()
+    return h_out
+
+
+def tg_fold_norm_weight(w, norm_w, out=None, stream=None):
+    """out[r, c] = bf16(w[r, c] * norm_w[c]): an RMSNorm weight folded into the projection."""
+    ld_w = _mat(w, "w")
+    if out is None:
+        out = torch.empty_like(w)
+    rc = lib.tg_fold_norm_weight(_ptr(w), ld_w, w.shape[0], w.shape[1], _ptr(norm_w), _ptr(out),
+                                 _mat(out, "out"), _stream(stream))
+    _check(rc, "tg_fold_norm_weight")
+    _count()
+    return out
+
+
+def tg_pack_gate_up(w_gate, w_up, norm_w=None, out=None, stream=None):
+    """[2 F, H] weight for tg_swiglu: gate and up rows interleaved in blocks of 64, columns
+    scaled by the MLP's RMSNorm weight."""
+    ffn, hidden = w_gate.shape
+    if out is None:
+        out = torch.empty((2 * ffn, hidden), dtype=w_gate.dtype, device=w_gate.device)
+    rc = lib.tg_pack_gate_up(_ptr(w_gate), _mat(w_gate, "w_gate"), _ptr(w_up), _mat(w_up, "w_up"),
+                             ffn, hidden, _ptr(norm_w), _ptr(out), _mat(out, "out"),
+                             _stream(stream))
+    _check(rc, "tg_pack_gate_up")
+    _count()
+    return out
 
 
 def tg_out_proj_qkv_workspace_size(M: int) -> int:
@@ -369,10 +423,50 @@ def tg_out_proj_qkv_next(o, w_o, x, row_ssq, w_qkv, pos, cos_sin, cache_k, cache
 
 @dataclass
 class LayerWeights:
-    Wqkv: torch.Tensor   # bf16 [(Hq + 2 Hkv) d, H]
+    Wqkv: torch.Tensor   # bf16 [(Hq + 2 Hkv) d, H] (a weighted attention norm folded in)
     Wo: torch.Tensor     # bf16 [H, Hq d]
-    gamma: torch.Tensor  # fp32 [Hq]
-    beta: float
+    gamma: torch.Tensor = None  # fp32 [Hq] (layers above the gate)
+    beta: float = 1.0
+    q_norm: torch.Tensor = None  # fp32 [d]: QK-norm weights (full layer body)
+    k_norm: torch.Tensor = None
+    W_gu: torch.Tensor = None    # bf16 [2 F, H]: packed SwiGLU gate/up (tg_pack_gate_up)
+    W_down: torch.Tensor = None  # bf16 [H, F]
+
+    @property
+    def ffn(self):
+        return 0 if self.W_gu is None else self.W_gu.shape[0] // 2
+
+
+def prepare_layer(layer) -> LayerWeights:
+    """LayerWeights from a weight dict: Wqkv, Wo (+ gamma, beta above the gate), and for
+    a full layer body attn_norm, q_norm, k_norm and mlp = {norm_w, W_gate, W_up, W_down}.
+    The norm weights that multiply a projection's input are folded into it here, once
+    (tg_fold_norm_weight, tg_pack_gate_up)."""
+    if isinstance(layer, LayerWeights):
+        return layer
+    d = dict(layer)
+    Wqkv = d["Wqkv"]
+    if d.get("attn_norm") is not None:
+        Wqkv = tg_fold_norm_weight(Wqkv, d["attn_norm"])
+    W_gu = W_down = None
+    mlp = d.get("mlp")
+    if mlp is not None:
+        W_gu = tg_pack_gate_up(mlp["W_gate"], mlp["W_up"], mlp.get("norm_w"))
+        W_down = mlp["W_down"]
+    return LayerWeights(Wqkv=Wqkv, Wo=d["Wo"], gamma=d.get("gamma"), beta=d.get("beta", 1.0),
+                        q_norm=d.get("q_norm"), k_norm=d.get("k_norm"), W_gu=W_gu,
+                        W_down=W_down)
+
+
+def _mlp(L, x, P, eps, status, stream, mark):
+    """The SwiGLU MLP of a full layer body, in place on x (nothing without one)."""
+    if L.W_gu is None:
+        return
+    h = P["ffn"][:, :L.ffn]
+    tg_swiglu(x, L.W_gu, P["ssq"], h_out=h, eps=eps, status=status, stream=stream)
+    mark("mlp_gate_up")
+    tg_linear(h, L.W_down, x, residual=x, row_ssq=P["ssq"], status=status, stream=stream)
+    mark("mlp_down")
 
 
 class FullContextLayers:
@@ -390,8 +484,7 @@ class FullContextLayers:
     def __init__(self, layers: list, n_q_heads=16, n_kv_heads=8, head_dim=128,
                  rope_theta=1.0e6, norm_eps=1e-6, device="cuda"):
         self.device = torch.device(device)
-        self.layers = [(l["Wqkv"], l["Wo"]) if isinstance(l, dict) else (l.Wqkv, l.Wo)
-                       for l in layers]
+        self.layers = [prepare_layer(l) for l in layers]
         self.hq, self.hkv, self.d = n_q_heads, n_kv_heads, head_dim
         self.theta, self.norm_eps = rope_theta, norm_eps
         self.status = torch.zeros(1, dtype=torch.int32, device=self.device)
@@ -432,6 +525,7 @@ class FullContextLayers:
                                 dtype=torch.uint8, device=dev),
             caches=[(torch.empty((T, self.hkv * self.d), **bf),
                      torch.empty((T, self.hkv * self.d), **bf)) for _ in self.layers],
+            ffn=torch.empty((T, max([L.ffn for L in self.layers] + [0])), **bf),
         )
         return self.planned
 
@@ -443,18 +537,20 @@ class FullContextLayers:
         nq = self.hq * self.d
         qkv, o, x = P["qkv"], P["o"], P["x"]
         tg_gather_rope(h, x, row_ssq=P["ssq"], status=self.status, stream=stream)
-        for (Wqkv, Wo), (ck, cv) in zip(self.layers, P["caches"]):
-            tg_qkv_rope_cache(x, Wqkv, P["pos"], self.cos_sin, ck, cv, self.hq, self.hkv,
+        for L, (ck, cv) in zip(self.layers, P["caches"]):
+            tg_qkv_rope_cache(x, L.Wqkv, P["pos"], self.cos_sin, ck, cv, self.hq, self.hkv,
                               q_out=qkv[:, :nq], head_dim=self.d, eps=self.norm_eps,
-                              row_ssq=P["ssq"], status=self.status, stream=stream)
+                              row_ssq=P["ssq"], status=self.status, stream=stream,
+                              q_norm_w=L.q_norm, k_norm_w=L.k_norm)
             self._mark("qkv_rope_cache")
             tg_gated_attention(qkv[:, :nq], ck, cv, P["cu"], P["cu_h"], self.hq, self.hkv,
                                P["pos"], P["bias"], P["gamma"], 1.0, o=o, head_dim=self.d,
                                workspace=P["attn_ws"], status=self.status, stream=stream)
             self._mark("attention")
-            tg_linear(o, Wo, x, residual=x, row_ssq=P["ssq"], status=self.status,
+            tg_linear(o, L.Wo, x, residual=x, row_ssq=P["ssq"], status=self.status,
                       stream=stream)
             self._mark("out_proj")
+            _mlp(L, x, P, self.norm_eps, self.status, stream, self._mark)
         return x
 
     def trim(self, kept_idx, out=None, stream=None):
@@ -492,7 +588,7 @@ class GatedPrefill:
         self.lower = lower
         self.trim_lower_kv = trim_lower_kv
         self.gate = gate
-        self.layers = [l if isinstance(l, LayerWeights) else LayerWeights(**l) for l in layers]
+        self.layers = [prepare_layer(l) for l in layers]
         self.hq, self.hkv, self.d = n_q_heads, n_kv_heads, head_dim
         self.theta = rope_theta
         self.norm_eps, self.seq_eps = norm_eps, seq_eps
@@ -559,6 +655,7 @@ class GatedPrefill:
                      torch.empty((K, self.hkv * self.d), **bf)) for _ in self.layers],
             chain_ws=torch.zeros(max(16, tg_out_proj_qkv_workspace_size(K)), dtype=torch.uint8,
                                  device=dev),
+            ffn=torch.empty((K, max([L.ffn for L in self.layers] + [0])), **bf),
         )
         if self.lower is not None:
             self.lower.plan(lengths, self.hidden)
@@ -593,8 +690,9 @@ class GatedPrefill:
 
     def _fusable(self):
         nq, nkv = self.hq * self.d, self.hkv * self.d
+        plain = all(L.q_norm is None and L.W_gu is None for L in self.layers)
         return (self.fused_qkv and self.hidden % 256 == 0 and nq % 256 == 0 and nkv % 256 == 0
-                and self.d == 128)
+                and self.d == 128 and plain)
 
     def layer(self, i, stream=None, fuse_next=False):
         """Upper layer i on the kept rows, in place on x; K/V land in cache i.  With
@@ -609,10 +707,11 @@ class GatedPrefill:
         qkv, o, x = P["qkv"], P["o"], P["x"]
         if self._qkv_done == i:
             pass  # ran with the previous layer's output projection
-        elif self.fused_qkv:
+        elif self.fused_qkv or L.q_norm is not None:
             tg_qkv_rope_cache(x, L.Wqkv, P["kept_pos"], self.cos_sin, ck, cv, self.hq, self.hkv,
                               q_out=qkv[:, :nq], head_dim=self.d, eps=self.norm_eps,
-                              row_ssq=P["ssq"], status=self.status, stream=stream)
+                              row_ssq=P["ssq"], status=self.status, stream=stream,
+                              q_norm_w=L.q_norm, k_norm_w=L.k_norm)
             self._mark("qkv_rope_cache")
         else:
             tg_linear(x, L.Wqkv, qkv, rmsnorm=True, eps=self.norm_eps, status=self.status,
@@ -650,6 +749,7 @@ class GatedPrefill:
         else:
             tg_linear(o, L.Wo, x, residual=x, row_ssq=P["ssq"], status=self.status, stream=stream)
             self._mark("out_proj")
+        _mlp(L, x, P, self.norm_eps, self.status, stream, self._mark)
 
     def upper_layers(self, h, stream=None):
         self.gather(h, stream=stream)

@@ -46,6 +46,13 @@ SIGNATURES = {
     "tg_gated_attention_workspace_size": (_sz, [_p, _i32, _i32, _i32, _i32]),
     "tg_qkv_rope_cache": (_i32, [_p, _i64, _p, _i64, _i64, _i32, _i32, _i32, _i32, _f32, _p, _p,
                                  _i32, _p, _i64, _p, _p, _i64, _i64, _p, _i64, _p, _p]),
+    "tg_qkv_qknorm_rope_cache": (_i32, [_p, _i64, _p, _i64, _i64, _i32, _i32, _i32, _i32, _f32,
+                                        _p, _p, _p, _p, _i32, _p, _i64, _p, _p, _i64, _i64,
+                                        _p, _i64, _p, _p]),
+    "tg_swiglu": (_i32, [_p, _i64, _p, _i64, _i64, _i32, _i32, _f32, _p, _i64, _p, _i64, _p,
+                         _p]),
+    "tg_fold_norm_weight": (_i32, [_p, _i64, _i64, _i32, _p, _p, _i64, _p]),
+    "tg_pack_gate_up": (_i32, [_p, _i64, _p, _i64, _i32, _i32, _p, _p, _i64, _p]),
     "tg_out_proj_qkv_next": (_i32, [_p, _i64, _p, _i64, _p, _i64, _p, _i64, _i64, _i32, _i32,
                                      _p, _i64, _i32, _i32, _i32, _f32, _p, _p, _i32, _p, _i64,
                                      _p, _p, _i64, _i64, _p, _sz, _p, _p]),

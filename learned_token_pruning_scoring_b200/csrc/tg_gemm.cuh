@@ -32,7 +32,7 @@
 
 namespace tg {
 
-enum { EpiStore = 0, EpiScore = 1, EpiQKV = 2 };
+enum { EpiStore = 0, EpiScore = 1, EpiQKV = 2, EpiSwiGLU = 3 };
 
 struct GemmParams {
   int64_t M;
@@ -61,6 +61,11 @@ struct GemmParams {
   uint16_t* k_out;        // K rows: k_out + row * ld_kv (columns relative to q_cols)
   uint16_t* v_out;        // V rows: v_out + row * ld_kv (columns relative to q_cols + k_cols)
   int64_t ld_kv;
+  // EpiQKV, CTA-pair kernel only: optional QK-norm (per-head RMSNorm of the Q and K
+  // heads before RoPE, weights [128] shared by the heads)
+  const float* q_norm_w;
+  const float* k_norm_w;
+  float qk_eps;
   uint32_t* status;
 };
 
@@ -404,6 +409,27 @@ __device__ __forceinline__ void pair_epilogue_half(const GemmParams& p, unsigned
       pos = 0;
     }
     const float4* cs_row = reinterpret_cast<const float4*>(p.cos_sin + (int64_t)pos * 128);
+    // QK-norm: this group's 128 columns are one Q or K head of the row; a first pass
+    // over them gives the head's RMS
+    float qk = 1.f;
+    const float* nw = nullptr;
+    if (rope && p.q_norm_w) {
+      nw = n0 < p.q_cols ? p.q_norm_w : p.k_norm_w;
+      float ss = 0.f;
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {
+        uint32_t r[32];
+        tmem_ld32(tacc + (4 * h + c) * 32, r);
+        tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const float v = __uint_as_float(r[i]);
+          ss = fmaf(v, v, ss);
+        }
+      }
+      qk = rsqrtf(ss * rscale * rscale * (1.0f / 128.0f) + p.qk_eps);
+    }
+    const float scale = rscale * qk;
 #pragma unroll 1
     for (int pr = 0; pr < 2; ++pr) {
       // 32-column pieces ca and ca + 2 hold columns i and i + 64 of one 128-column head
@@ -421,8 +447,15 @@ __device__ __forceinline__ void pair_epilogue_half(const GemmParams& p, unsigned
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const int i = u * 8 + 2 * e;
-          float x1a = __uint_as_float(ra[i]) * rscale, x1b = __uint_as_float(ra[i + 1]) * rscale;
-          float x2a = __uint_as_float(rb[i]) * rscale, x2b = __uint_as_float(rb[i + 1]) * rscale;
+          float x1a = __uint_as_float(ra[i]) * scale, x1b = __uint_as_float(ra[i + 1]) * scale;
+          float x2a = __uint_as_float(rb[i]) * scale, x2b = __uint_as_float(rb[i + 1]) * scale;
+          if (nw) {  // head columns c and c + 64, c = 32 pr + i
+            const int c = 32 * pr + i;
+            x1a *= __ldg(nw + c);
+            x1b *= __ldg(nw + c + 1);
+            x2a *= __ldg(nw + c + 64);
+            x2b *= __ldg(nw + c + 65);
+          }
           if (rope) {
             const float4 t = cs[i >> 1];  // (cos_i, sin_i, cos_i+1, sin_i+1)
             const float y1a = x1a * t.x - x2a * t.y, y2a = x2a * t.x + x1a * t.y;
@@ -440,6 +473,33 @@ __device__ __forceinline__ void pair_epilogue_half(const GemmParams& p, unsigned
             make_uint4(wa[0], wa[1], wa[2], wa[3]);
         *reinterpret_cast<uint4*>(box_b + sw128_chunk(row, k)) =
             make_uint4(wb[0], wb[1], wb[2], wb[3]);
+      }
+    }
+    return;
+  }
+  if (EPI == EpiSwiGLU) {
+    // Group h's 128 tile columns are 64 gate features then the same 64 up features
+    // (weight rows interleaved in blocks of 64); out = SiLU(gate) * up, 64 bf16 columns
+    // staged in box h.
+    unsigned char* box = out_s + h * PairCfg<1>::BOX_BYTES;
+#pragma unroll 1
+    for (int c = 0; c < 2; ++c) {
+      uint32_t rg[32], ru[32];
+      tmem_ld32(tacc + 128 * h + 32 * c, rg);
+      tmem_ld32(tacc + 128 * h + 64 + 32 * c, ru);
+      tmem_wait_ld();
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        uint32_t w[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int i = u * 8 + 2 * e;
+          const float ga = __uint_as_float(rg[i]) * rscale, gb = __uint_as_float(rg[i + 1]) * rscale;
+          const float ua = __uint_as_float(ru[i]) * rscale, ub = __uint_as_float(ru[i + 1]) * rscale;
+          w[e] = pack_bf16x2(ga / (1.0f + __expf(-ga)) * ua, gb / (1.0f + __expf(-gb)) * ub);
+        }
+        *reinterpret_cast<uint4*>(box + sw128_chunk(row, 4 * c + u)) =
+            make_uint4(w[0], w[1], w[2], w[3]);
       }
     }
     return;
@@ -729,7 +789,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(320, 1)
         else
           mbar_arrive_cluster(acc_empty_lead0 + b * 8);
         int mi = 0, x = n0;
-        if ((job ? EPI1 : EPI0) == EpiQKV) {
+        const int epi = job ? EPI1 : EPI0;
+        if (epi == EpiQKV) {
           if (n0 >= jb.p.q_cols + jb.p.k_cols) {
             mi = 2;
             x = n0 - jb.p.q_cols - jb.p.k_cols;
@@ -738,8 +799,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(320, 1)
             x = n0 - jb.p.q_cols;
           }
         }
-        for (int j = 2 * g; j < 2 * g + 2; ++j)
-          tma_store_2d(&jb.maps.out[mi], x + 64 * j, (int32_t)m0, out_s + j * Cfg::BOX_BYTES);
+        if (epi == EpiSwiGLU)  // 64 output columns per group: features n0 / 2 + 64 g ..
+          tma_store_2d(&jb.maps.out[0], n0 / 2 + 64 * g, (int32_t)m0, out_s + g * Cfg::BOX_BYTES);
+        else
+          for (int j = 2 * g; j < 2 * g + 2; ++j)
+            tma_store_2d(&jb.maps.out[mi], x + 64 * j, (int32_t)m0, out_s + j * Cfg::BOX_BYTES);
         bulk_commit_group();
         if (publish) {
           bulk_wait_all();             // the rows are in global memory

@@ -1,5 +1,7 @@
 // Dense projections of the gated layers on the kept rows (Wq/Wk/Wv with a folded
-// pre-attention RMSNorm, Wo with a fused residual add), on the tcgen05 GEMM.
+// pre-attention RMSNorm and optional QK-norm, Wo with a fused residual add, the SwiGLU
+// MLP of a full layer body), on the tcgen05 GEMM, plus the one-time weight packing
+// those projections read.
 #include "tg_gemm.cuh"
 #include "tg_host.h"
 
@@ -138,7 +140,8 @@ int qkv_job(PairJob& j, const tg_bf16* x, int64_t ld_x, const tg_bf16* w_qkv, in
             int64_t M, int hidden, int q_cols, int kv_cols, float eps, const int32_t* pos,
             const float* cos_sin, int max_pos, tg_bf16* q_out, int64_t ld_q, tg_bf16* cache_k,
             tg_bf16* cache_v, int64_t ld_cache, int64_t slot_offset, const float* row_ssq_in,
-            int64_t ld_ssq_in, uint32_t* status) {
+            int64_t ld_ssq_in, uint32_t* status, const float* q_norm_w = nullptr,
+            const float* k_norm_w = nullptr) {
   const int N = q_cols + 2 * kv_cols;
   tg_bf16* k_rows = cache_k + slot_offset * ld_cache;
   tg_bf16* v_rows = cache_v + slot_offset * ld_cache;
@@ -170,8 +173,73 @@ int qkv_job(PairJob& j, const tg_bf16* x, int64_t ld_x, const tg_bf16* w_qkv, in
   j.p.ld_kv = ld_cache;
   j.p.row_ssq_in = row_ssq_in;
   j.p.ld_ssq_in = ld_ssq_in;
+  j.p.q_norm_w = q_norm_w;
+  j.p.k_norm_w = k_norm_w;
+  j.p.qk_eps = eps;
   j.p.status = status;
   return TG_OK;
+}
+
+// SwiGLU up-projection as a pair-kernel job: h = SiLU(a Wg^T) * (a Wu^T), a = RMSNorm(x)
+// from the row sums of squares, W rows interleaved in blocks of 64 (gate, up).
+int swiglu_job(PairJob& j, const tg_bf16* x, int64_t ld_x, const tg_bf16* w_gu, int64_t ld_w,
+               int64_t M, int hidden, int ffn, float eps, const float* row_ssq_in,
+               int64_t ld_ssq_in, tg_bf16* h_out, int64_t ld_h, uint32_t* status) {
+  TG_TRY(make_tmap_bf16_2d(&j.maps.a, x, (uint64_t)M, (uint64_t)hidden, (uint64_t)ld_x, 64, 128));
+  TG_TRY(make_tmap_bf16_2d(&j.maps.b, w_gu, (uint64_t)(2 * ffn), (uint64_t)hidden, (uint64_t)ld_w,
+                           64, 128));
+  TG_TRY(make_tmap_bf16_2d(&j.maps.out[0], h_out, (uint64_t)M, (uint64_t)ffn, (uint64_t)ld_h, 64,
+                           128));
+  j.maps.out[1] = j.maps.out[2] = j.maps.res = j.maps.out[0];
+  j.p = GemmParams{};
+  j.p.M = M;
+  j.p.N = 2 * ffn;
+  j.p.K = hidden;
+  j.p.rmsnorm = 1;
+  j.p.eps = eps;
+  j.p.c = reinterpret_cast<uint16_t*>(h_out);
+  j.p.ldc = ld_h;
+  j.p.row_ssq_in = row_ssq_in;
+  j.p.ld_ssq_in = ld_ssq_in;
+  j.p.status = status;
+  return TG_OK;
+}
+
+// out[r, c] = bf16(src(r)[c] * norm_w[c]) (norm_w optional).  src(r) is row r of a, or
+// with `interleave` row 64 (r / 128) + r % 64 of a (r % 128 < 64) or of b (otherwise).
+__global__ void pack_rows_kernel(const uint16_t* __restrict__ a, int64_t lda,
+                                 const uint16_t* __restrict__ b, int64_t ldb, int64_t rows,
+                                 int cols, const float* __restrict__ norm_w,
+                                 uint16_t* __restrict__ out, int64_t ld_out, int interleave) {
+  const int64_t n = rows * cols;
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t r = i / cols;
+    const int c = (int)(i % cols);
+    uint16_t v;
+    if (interleave) {
+      const int64_t src = (r >> 7) * 64 + (r & 63);
+      v = (r & 64) ? b[src * ldb + c] : a[src * lda + c];
+    } else {
+      v = a[r * lda + c];
+    }
+    if (norm_w) {
+      const __nv_bfloat16 t = __float2bfloat16_rn(__uint_as_float((uint32_t)v << 16) * norm_w[c]);
+      v = *reinterpret_cast<const uint16_t*>(&t);
+    }
+    out[r * ld_out + c] = v;
+  }
+}
+
+int launch_pack_rows(const tg_bf16* a, int64_t lda, const tg_bf16* b, int64_t ldb, int64_t rows,
+                     int cols, const float* norm_w, tg_bf16* out, int64_t ld_out, int interleave,
+                     cudaStream_t stream) {
+  const int64_t n = rows * cols;
+  int64_t grid = (n + 255) / 256;
+  if (grid > 8 * (int64_t)sm_count()) grid = 8 * (int64_t)sm_count();
+  return launch(pack_rows_kernel, dim3((unsigned)grid), dim3(256), 0, stream,
+                reinterpret_cast<const uint16_t*>(a), lda, reinterpret_cast<const uint16_t*>(b),
+                ldb, rows, cols, norm_w, reinterpret_cast<uint16_t*>(out), ld_out, interleave);
 }
 
 }  // namespace tg
@@ -223,13 +291,14 @@ extern "C" int tg_linear(const tg_bf16* a, int64_t lda, const tg_bf16* w, int64_
   return launch_gemm<128, 3, EpiStore>(ta, tb, p, (cudaStream_t)stream);
 }
 
-extern "C" int tg_qkv_rope_cache(const tg_bf16* x, int64_t ld_x, const tg_bf16* w_qkv, int64_t ld_w,
-                                 int64_t M, int hidden, int n_q_heads, int n_kv_heads,
-                                 int head_dim, float eps, const int32_t* pos,
-                                 const float* cos_sin, int max_pos, tg_bf16* q_out, int64_t ld_q,
-                                 tg_bf16* cache_k, tg_bf16* cache_v, int64_t ld_cache,
-                                 int64_t slot_offset, const float* row_ssq_in,
-                                 int64_t ld_ssq_in, uint32_t* status, tg_stream_t stream) {
+static int qkv_rope_cache_impl(const tg_bf16* x, int64_t ld_x, const tg_bf16* w_qkv,
+                               int64_t ld_w, int64_t M, int hidden, int n_q_heads,
+                               int n_kv_heads, int head_dim, float eps, const int32_t* pos,
+                               const float* cos_sin, int max_pos, tg_bf16* q_out, int64_t ld_q,
+                               tg_bf16* cache_k, tg_bf16* cache_v, int64_t ld_cache,
+                               int64_t slot_offset, const float* row_ssq_in, int64_t ld_ssq_in,
+                               const float* q_norm_w, const float* k_norm_w, uint32_t* status,
+                               tg_stream_t stream) {
   if (head_dim != 128 || n_q_heads <= 0 || n_kv_heads <= 0 || hidden <= 0 || (hidden % 64))
     return TG_ERR_UNSUPPORTED_SHAPE;
   if (M < 0 || slot_offset < 0 || max_pos <= 0) return TG_ERR_INVALID_ARGUMENT;
@@ -251,11 +320,15 @@ extern "C" int tg_qkv_rope_cache(const tg_bf16* x, int64_t ld_x, const tg_bf16* 
   // kernel when the row norms come precomputed
   const bool aligned256 = (q_cols % 256) == 0 && (kv_cols % 256) == 0;
   const bool pair = row_ssq_in && aligned256;
+  if (q_norm_w || k_norm_w) {  // QK-norm lives in the CTA-pair kernel's epilogue only
+    if (!q_norm_w || !k_norm_w || !row_ssq_in) return TG_ERR_INVALID_ARGUMENT;
+    if (!aligned256) return TG_ERR_UNSUPPORTED_SHAPE;
+  }
   if (pair) {
     PairJob j;
     TG_TRY(qkv_job(j, x, ld_x, w_qkv, ld_w, M, hidden, q_cols, kv_cols, eps, pos, cos_sin, max_pos,
                    q_out, ld_q, cache_k, cache_v, ld_cache, slot_offset, row_ssq_in, ld_ssq_in,
-                   status));
+                   status, q_norm_w, k_norm_w));
     return launch_pair<kPairStages, EpiQKV>(j.maps, j.p, (cudaStream_t)stream);
   }
   int bn = pick_bn(M, N);
@@ -284,6 +357,74 @@ extern "C" int tg_qkv_rope_cache(const tg_bf16* x, int64_t ld_x, const tg_bf16* 
   p.status = status;
   if (bn == 256) return launch_gemm<256, 4, EpiQKV>(ta, tb, p, (cudaStream_t)stream);
   return launch_gemm<128, 3, EpiQKV>(ta, tb, p, (cudaStream_t)stream);
+}
+
+extern "C" int tg_qkv_rope_cache(const tg_bf16* x, int64_t ld_x, const tg_bf16* w_qkv, int64_t ld_w,
+                                 int64_t M, int hidden, int n_q_heads, int n_kv_heads,
+                                 int head_dim, float eps, const int32_t* pos,
+                                 const float* cos_sin, int max_pos, tg_bf16* q_out, int64_t ld_q,
+                                 tg_bf16* cache_k, tg_bf16* cache_v, int64_t ld_cache,
+                                 int64_t slot_offset, const float* row_ssq_in,
+                                 int64_t ld_ssq_in, uint32_t* status, tg_stream_t stream) {
+  return qkv_rope_cache_impl(x, ld_x, w_qkv, ld_w, M, hidden, n_q_heads, n_kv_heads, head_dim,
+                             eps, pos, cos_sin, max_pos, q_out, ld_q, cache_k, cache_v, ld_cache,
+                             slot_offset, row_ssq_in, ld_ssq_in, nullptr, nullptr, status, stream);
+}
+
+extern "C" int tg_qkv_qknorm_rope_cache(
+    const tg_bf16* x, int64_t ld_x, const tg_bf16* w_qkv, int64_t ld_w, int64_t M, int hidden,
+    int n_q_heads, int n_kv_heads, int head_dim, float eps, const float* q_norm_w,
+    const float* k_norm_w, const int32_t* pos, const float* cos_sin, int max_pos, tg_bf16* q_out,
+    int64_t ld_q, tg_bf16* cache_k, tg_bf16* cache_v, int64_t ld_cache, int64_t slot_offset,
+    const float* row_ssq_in, int64_t ld_ssq_in, uint32_t* status, tg_stream_t stream) {
+  if (!q_norm_w || !k_norm_w || !row_ssq_in) return TG_ERR_INVALID_ARGUMENT;
+  return qkv_rope_cache_impl(x, ld_x, w_qkv, ld_w, M, hidden, n_q_heads, n_kv_heads, head_dim,
+                             eps, pos, cos_sin, max_pos, q_out, ld_q, cache_k, cache_v, ld_cache,
+                             slot_offset, row_ssq_in, ld_ssq_in, q_norm_w, k_norm_w, status,
+                             stream);
+}
+
+extern "C" int tg_swiglu(const tg_bf16* x, int64_t ld_x, const tg_bf16* w_gu, int64_t ld_w,
+                         int64_t M, int hidden, int ffn, float eps, const float* row_ssq_in,
+                         int64_t ld_ssq_in, tg_bf16* h_out, int64_t ld_h, uint32_t* status,
+                         tg_stream_t stream) {
+  if (hidden <= 0 || (hidden % 128) || ffn <= 0 || (ffn % 128)) return TG_ERR_UNSUPPORTED_SHAPE;
+  if (M < 0) return TG_ERR_INVALID_ARGUMENT;
+  if (M == 0) return TG_OK;
+  if (!x || !w_gu || !row_ssq_in || !h_out) return TG_ERR_INVALID_ARGUMENT;
+  if (ld_x < hidden || ld_w < hidden || ld_h < ffn || ld_ssq_in < hidden / 128)
+    return TG_ERR_INVALID_ARGUMENT;
+  if (!aligned16(x) || !aligned16(w_gu) || !aligned16(h_out) || !stride_ok(ld_x, 2) ||
+      !stride_ok(ld_w, 2) || !stride_ok(ld_h, 2))
+    return TG_ERR_MISALIGNED;
+  if (!(eps >= 0.f)) return TG_ERR_INVALID_ARGUMENT;
+  TG_TRY(check_device());
+  PairJob j;
+  TG_TRY(swiglu_job(j, x, ld_x, w_gu, ld_w, M, hidden, ffn, eps, row_ssq_in, ld_ssq_in, h_out,
+                    ld_h, status));
+  return launch_pair<kPairStages, EpiSwiGLU>(j.maps, j.p, (cudaStream_t)stream);
+}
+
+extern "C" int tg_fold_norm_weight(const tg_bf16* w, int64_t ld_w, int64_t rows, int cols,
+                                   const float* norm_w, tg_bf16* out, int64_t ld_out,
+                                   tg_stream_t stream) {
+  if (rows < 0 || cols <= 0) return TG_ERR_INVALID_ARGUMENT;
+  if (rows == 0) return TG_OK;
+  if (!w || !norm_w || !out || ld_w < cols || ld_out < cols) return TG_ERR_INVALID_ARGUMENT;
+  TG_TRY(check_device());
+  return launch_pack_rows(w, ld_w, nullptr, 0, rows, cols, norm_w, out, ld_out, 0,
+                          (cudaStream_t)stream);
+}
+
+extern "C" int tg_pack_gate_up(const tg_bf16* w_gate, int64_t ld_gate, const tg_bf16* w_up,
+                               int64_t ld_up, int ffn, int hidden, const float* norm_w,
+                               tg_bf16* out, int64_t ld_out, tg_stream_t stream) {
+  if (ffn <= 0 || (ffn % 64) || hidden <= 0) return TG_ERR_UNSUPPORTED_SHAPE;
+  if (!w_gate || !w_up || !out || ld_gate < hidden || ld_up < hidden || ld_out < hidden)
+    return TG_ERR_INVALID_ARGUMENT;
+  TG_TRY(check_device());
+  return launch_pack_rows(w_gate, ld_gate, w_up, ld_up, 2 * (int64_t)ffn, hidden, norm_w, out,
+                          ld_out, 1, (cudaStream_t)stream);
 }
 
 extern "C" size_t tg_out_proj_qkv_workspace_size(int64_t M) {

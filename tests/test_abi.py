@@ -130,3 +130,31 @@ def test_out_proj_qkv_argument_checks(lib):
     assert call(2048, p, 4) == -4
     assert lib.tg_out_proj_qkv_workspace_size(0) == 0
     assert lib.tg_out_proj_qkv_workspace_size(257) == 16
+
+
+def test_full_body_argument_checks(lib):
+    """QK-norm needs both weights and the row sums of squares; the SwiGLU GEMM needs
+    128-multiple widths and the row sums of squares; the weight packers check shapes."""
+    p = C.c_void_p(0x10000)
+
+    def qkn(qw, kw, ssq):
+        return lib.tg_qkv_qknorm_rope_cache(p, 2048, p, 2048, 16, 2048, 16, 8, 128, 1e-6, qw,
+                                            kw, p, p, 100, p, 2048, p, p, 1024, 0, ssq, 16,
+                                            None, None)
+    assert qkn(None, p, p) == -1
+    assert qkn(p, None, p) == -1
+    assert qkn(p, p, None) == -1
+
+    def swi(hidden, ffn, ssq, ld_ssq=16):
+        return lib.tg_swiglu(p, hidden, p, hidden, 16, hidden, ffn, 1e-6, ssq, ld_ssq, p, ffn,
+                             None, None)
+    assert swi(2048, 6000, p) == -6   # ffn not a multiple of 128
+    assert swi(2000, 6144, p) == -6   # hidden not a multiple of 128
+    assert swi(2048, 6144, None) == -1
+    assert swi(2048, 6144, p, ld_ssq=8) == -1
+    assert lib.tg_swiglu(p, 2048, p, 2048, 0, 2048, 6144, 1e-6, p, 16, p, 6144, None,
+                         None) == 0  # nothing to do
+    assert lib.tg_pack_gate_up(p, 2048, p, 2048, 100, 2048, None, p, 2048, None) == -6
+    assert lib.tg_pack_gate_up(p, 2048, None, 2048, 128, 2048, None, p, 2048, None) == -1
+    assert lib.tg_fold_norm_weight(p, 2048, 16, 2048, None, p, 2048, None) == -1
+    assert lib.tg_fold_norm_weight(p, 2048, 0, 2048, p, p, 2048, None) == 0

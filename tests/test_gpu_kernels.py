@@ -582,3 +582,75 @@ def test_out_proj_qkv_chain_equals_the_two_calls(tg, M):
     assert torch.equal(x1, x2) and torch.equal(ssq1, ssq2)
     assert torch.equal(q1, q2) and torch.equal(k1, k2) and torch.equal(v1, v2)
     assert int(ws.count_nonzero()) == 0
+
+
+# ------------------------------------------------------------------ full layer body parts
+
+def test_weight_packing_bit_exact(tg):
+    """tg_fold_norm_weight / tg_pack_gate_up against the same products rounded by torch."""
+    F_, H = 256, 2048
+    wg = S.uniform_rows(F_, H, seed=70, scale=0.02)
+    wu = S.uniform_rows(F_, H, seed=71, scale=0.02)
+    nw = (0.8 + 0.4 * torch.rand(H, generator=torch.Generator().manual_seed(72))).float()
+    folded = tg.tg_fold_norm_weight(_dev(wg), _dev(nw)).cpu()
+    assert torch.equal(folded, (wg.float() * nw).to(torch.bfloat16))
+    packed = tg.tg_pack_gate_up(_dev(wg), _dev(wu), _dev(nw)).cpu()
+    want = torch.empty((2 * F_, H), dtype=torch.bfloat16)
+    for j in range(F_ // 64):
+        want[128 * j:128 * j + 64] = (wg[64 * j:64 * j + 64].float() * nw).to(torch.bfloat16)
+        want[128 * j + 64:128 * j + 128] = (wu[64 * j:64 * j + 64].float() * nw).to(torch.bfloat16)
+    assert torch.equal(packed, want)
+    plain = tg.tg_pack_gate_up(_dev(wg), _dev(wu)).cpu()
+    assert torch.equal(plain[64:128], wu[:64]) and torch.equal(plain[128:192], wg[64:128])
+
+
+def _ssq_rows(x, H):
+    return torch.from_numpy((_f64(x) ** 2).reshape(x.shape[0], H // 128, 128).sum(-1)).float()
+
+
+@pytest.mark.parametrize("M", [1, 300, 1638])
+def test_qkv_qknorm_rope_cache_against_oracle(tg, M):
+    """Weighted attention norm folded into Wqkv, QK-norm and RoPE in the epilogue."""
+    Hq, Hkv, d, H = 16, 8, 128, 2048
+    x = S.uniform_rows(M, H, seed=M + 80)
+    w = S.uniform_rows((Hq + 2 * Hkv) * d, H, seed=M + 81, scale=0.02)
+    g = torch.Generator().manual_seed(M + 82)
+    attn_norm = (0.8 + 0.4 * torch.rand(H, generator=g)).float()
+    qn = (0.8 + 0.4 * torch.rand(d, generator=g)).float()
+    kn = (0.8 + 0.4 * torch.rand(d, generator=g)).float()
+    pos = torch.arange(0, 3 * M, 3, dtype=torch.int32)
+    cs = tg.tg_rope_table(3 * M + 1, d, 1.0e6)
+    ck = torch.zeros((M, Hkv * d), dtype=torch.bfloat16, device="cuda")
+    cv = torch.zeros_like(ck)
+    L = tg.prepare_layer({"Wqkv": _dev(w), "Wo": _dev(w[:H, :H]), "attn_norm": _dev(attn_norm),
+                          "q_norm": _dev(qn), "k_norm": _dev(kn)})
+    st = _status()
+    q = tg.tg_qkv_rope_cache(_dev(x), L.Wqkv, _dev(pos), cs, ck, cv, Hq, Hkv,
+                             row_ssq=_dev(_ssq_rows(x, H)), q_norm_w=L.q_norm, k_norm_w=L.k_norm,
+                             status=st)
+    assert tg.tg_status_read(st) == 0
+    _, _, _, parts = O.gated_layer(x, w, w[:H, :H], np.zeros(Hq), 1.0, [0, M], pos, np.zeros(M),
+                                   Hq, Hkv, d, 1.0e6, attn_norm=attn_norm, q_norm=qn, k_norm=kn)
+    for got, want in ((q, parts["q"]), (ck, parts["k"]), (cv, parts["v"])):
+        want = want.reshape(M, -1)
+        err = np.abs(_f64(got.cpu()) - want)
+        assert np.all(err <= 2.0 ** -7 * np.abs(want) + 2e-3), err.max()
+
+
+@pytest.mark.parametrize("M", [1, 300, 1638, 4000])
+def test_swiglu_against_oracle(tg, M):
+    H, F_ = 2048, 6144
+    x = S.uniform_rows(M, H, seed=M + 90)
+    g = torch.Generator().manual_seed(M + 91)
+    nw = (0.8 + 0.4 * torch.rand(H, generator=g)).float()
+    wg = (torch.randn((F_, H), generator=g) * 0.02).to(torch.bfloat16)
+    wu = (torch.randn((F_, H), generator=g) * 0.02).to(torch.bfloat16)
+    w_gu = tg.tg_pack_gate_up(_dev(wg), _dev(wu), _dev(nw))
+    st = _status()
+    h = tg.tg_swiglu(_dev(x), w_gu, _dev(_ssq_rows(x, H)), status=st)
+    assert tg.tg_status_read(st) == 0
+    b = O.rmsnorm_rows(x, nw)
+    want = O.silu(b @ _f64(wg).T) * (b @ _f64(wu).T)
+    err = np.abs(_f64(h.cpu()) - want)
+    assert np.all(err <= 2.0 ** -7 * np.abs(want) + 2e-3), err.max()
+    assert err.mean() <= 1e-3

@@ -341,3 +341,59 @@ def test_pipeline_with_lower_layers_and_kv_trim(tg):
     tol, tol_mean = _x_tol(ref["x"], 3)
     assert np.all(err <= tol) and err.mean() <= tol_mean, (err.max(), err.mean())
     assert tg.tg_status_read(pipe.status) == 0
+
+
+# ------------------------------------------------------------------ full layer bodies
+#
+# `tests/tolerance_study.py full`: two full layer bodies (weighted norms folded into
+# bf16 weights, QK-norm, SwiGLU MLP) rounded where the CUDA path rounds move x by
+# max 0.030 / 0.051 and mean 0.0032 / 0.0056 after 1 / 2 layers; in the chain tested
+# below (one lower, two upper full layers) x moves by max 0.073 / mean 0.0079 and every
+# layer's K cache by at most 0.005 max|k|.  Bound for n full layers: |err| <= 2^-7 |ref|
+# + 0.06 n, mean <= 0.007 n (2-2.5x the study); caches 2^-6 max|k|.
+
+def _full_tol(want, n):
+    return 2.0 ** -7 * np.abs(want) + 0.06 * n, 0.007 * n
+
+
+def test_pipeline_full_layer_bodies(tg):
+    """One full-context full layer below the gate, two gated full layers above it (QK-norm,
+    weighted norms, SwiGLU MLP on the kept rows only), lower caches trimmed."""
+    wl = S.custom([700, 1500, 333], [16, 64, 5], [100, 800, 300], n_layers=2,
+                  planted_cluster=True, name="ragged3_full")
+    h = S.hidden_rows(wl)
+    gate = S.gate_weights(wl)
+    upper = [dict(S.layer_weights(wl, i), **S.layer_body_parts(wl, i)) for i in range(2)]
+    lower = [dict(L, **S.layer_body_parts(wl, 0, lower=True))
+             for L in S.lower_layer_weights(wl, 1)]
+    pr = S.prunable_mask(wl)
+    drawn = S.drawn_scores(wl)
+
+    def dev(d):
+        return {k: (dev(v) if isinstance(v, dict) else v.cuda() if torch.is_tensor(v) else v)
+                for k, v in d.items()}
+    full = tg.FullContextLayers([dev(L) for L in lower], wl.n_q_heads, wl.n_kv_heads,
+                                wl.head_dim, wl.rope_theta)
+    pipe = tg.GatedPrefill(_dev_dict(gate), [dev(L) for L in upper], wl.n_q_heads,
+                           wl.n_kv_heads, wl.head_dim, wl.rope_theta, lower=full)
+    P = pipe.plan(wl.lengths, wl.questions, wl.budgets)
+    pipe.run(h.cuda(), pr.cuda(), scores=drawn.cuda())
+    torch.cuda.synchronize()
+    assert tg.tg_status_read(pipe.status) == 0
+    ref = O.prefill(h, pr, wl.cu_seqlens(), wl.budgets, gate, upper, wl.n_q_heads,
+                    wl.n_kv_heads, wl.head_dim, wl.rope_theta, scores=drawn, lower_layers=lower)
+    err = np.abs(O.as_f64(full.planned["x"].cpu()) - ref["h_gate"])
+    tol, tol_mean = _full_tol(ref["h_gate"], 1)
+    assert np.all(err <= tol) and err.mean() <= tol_mean, (err.max(), err.mean())
+    assert _check_selection(wl, pr.numpy(), ref["z"], ref["cu_kept"],
+                            P["kept_idx"].cpu().numpy(), P["ck_h"].numpy())
+    k_ref, _ = ref["lower_caches"][0]
+    kc = O.as_f64(P["lower_caches"][0][0].cpu()).reshape(k_ref.shape)
+    assert np.abs(kc - k_ref).max() <= 2.0 ** -6 * np.abs(k_ref).max()
+    for i in range(2):  # the upper caches carry QK-normed keys
+        k_up = ref["caches"][i][0]
+        kc = O.as_f64(P["caches"][i][0].cpu()).reshape(k_up.shape)
+        assert np.abs(kc - k_up).max() <= 2.0 ** -6 * np.abs(k_up).max()
+    err = np.abs(O.as_f64(P["x"].cpu()) - ref["x"])
+    tol, tol_mean = _full_tol(ref["x"], 3)
+    assert np.all(err <= tol) and err.mean() <= tol_mean, (err.max(), err.mean())

@@ -75,7 +75,54 @@ def study_lower(wl, n_lower):
           f"z max {np.abs(zr - z64).max():.5f} mean {np.abs(zr - z64).mean():.6f}", flush=True)
 
 
+def layer_rounded_full(x, L, body, cu_kept, pos, bias, wl):
+    """A full layer body with bf16 rounding where the CUDA path rounds: the folded norm
+    weights (Wqkv * attn_norm, W_gate/W_up * mlp norm), q/k after QK-norm and RoPE, v,
+    O, the residual after attention, the SwiGLU output and the residual after the MLP."""
+    hq, hkv, d = wl.n_q_heads, wl.n_kv_heads, wl.head_dim
+    Kt = x.shape[0]
+    m = body["mlp"]
+    wqkv = bf16(O.as_f64(L["Wqkv"]) * O.as_f64(body["attn_norm"])[None, :])
+    qkv = O.rmsnorm_rows(x) @ wqkv.T
+    q = O.rmsnorm_heads(qkv[:, :hq * d].reshape(Kt, hq, d), body["q_norm"])
+    k = O.rmsnorm_heads(qkv[:, hq * d:(hq + hkv) * d].reshape(Kt, hkv, d), body["k_norm"])
+    q = bf16(O.rope(q, pos, wl.rope_theta))
+    k = bf16(O.rope(k, pos, wl.rope_theta))
+    v = bf16(qkv[:, (hq + hkv) * d:].reshape(Kt, hkv, d))
+    o, _ = O.gated_attention(q, k, v, cu_kept, pos, bias, L["gamma"], L["beta"])
+    x = bf16(x + bf16(o.reshape(Kt, -1)) @ O.as_f64(L["Wo"]).T)
+    nw = O.as_f64(m["norm_w"])[None, :]
+    b = O.rmsnorm_rows(x)
+    hmid = bf16(O.silu(b @ bf16(O.as_f64(m["W_gate"]) * nw).T)
+                * (b @ bf16(O.as_f64(m["W_up"]) * nw).T))
+    return bf16(x + hmid @ O.as_f64(m["W_down"]).T)
+
+
+def study_full(wl, n_layers):
+    """Full layer bodies above the gate (QK-norm, weighted norms, SwiGLU MLP)."""
+    h, pr, gate = S.hidden_rows(wl), S.prunable_mask(wl), S.gate_weights(wl)
+    ref = O.prefill(h, pr, wl.cu_seqlens(), wl.budgets, gate, [], wl.n_q_heads,
+                    wl.n_kv_heads, wl.head_dim, wl.rope_theta)
+    ck, pos, kb = ref["cu_kept"], ref["kept_pos"], ref["kept_bias"]
+    x64 = O.gather_rows(h, ref["kept_idx"])
+    xr = x64.copy()
+    for i in range(n_layers):
+        L = S.layer_weights(wl, i)
+        body = S.layer_body_parts(wl, i)
+        x64, *_ = O.gated_layer(x64, L["Wqkv"], L["Wo"], L["gamma"], L["beta"], ck, pos, kb,
+                                wl.n_q_heads, wl.n_kv_heads, wl.head_dim, wl.rope_theta,
+                                **body)
+        xr = layer_rounded_full(xr, L, body, ck, pos, kb, wl)
+        e = np.abs(xr - x64)
+        print(f"{wl.name} full layer {i + 1}: max {e.max():.4f} mean {e.mean():.5f} "
+              f"|x|max {np.abs(x64).max():.2f}", flush=True)
+
+
 if __name__ == "__main__":
+    if len(sys.argv) > 1 and sys.argv[1] == "full":
+        study_full(S.custom([700, 1500, 333], [16, 64, 5], [100, 800, 300], n_layers=2,
+                            name="ragged3"), 2)
+        sys.exit(0)
     if len(sys.argv) > 1 and sys.argv[1] == "lower":
         study_lower(S.custom([700, 1500, 333], [16, 64, 5], [100, 800, 300], n_layers=1,
                              name="ragged3"), 2)
