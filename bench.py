@@ -62,6 +62,9 @@ def parse_args():
     ap.add_argument("--lower-layers", type=int, default=0,
                     help="full-context layers below the gate (their caches trimmed to the "
                          "kept rows); 0 = the gate reads the input rows directly")
+    ap.add_argument("--full-layers", action="store_true",
+                    help="full layer bodies (weighted norms, QK-norm, SwiGLU MLP of width "
+                         "6144) instead of attention-only layers")
     ap.add_argument("--dense-steps", type=int, default=3,
                     help="timed steps of the full-context reference (0 skips it)")
     return ap.parse_args()
@@ -87,7 +90,7 @@ def workload(name):
 
 # ------------------------------------------------------------------ algorithmic work
 
-def stage_work(wl, kept_counts):
+def stage_work(wl, kept_counts, ffn=0):
     """Algorithmic bytes / flops per launch of each stage (see the design notes)."""
     T = wl.total_tokens
     Ks = [kept_counts[b + 1] - kept_counts[b] for b in range(wl.batch)]
@@ -119,6 +122,12 @@ def stage_work(wl, kept_counts):
                             "flops": 4 * d * hq * sum(n * (n + 1) // 2 for n in wl.lengths)},
         "lower_out_proj": {"bound": "tensor", "flops": 2 * T * hq * d * H},
         "lower_kv_trim": {"bound": "hbm", "bytes": 2 * 2 * K * hkv * d * 2 + K * 4},
+        # full layer body: the SwiGLU MLP (gate/up GEMM with the SiLU product, down
+        # projection with the residual)
+        "mlp_gate_up": {"bound": "tensor", "flops": 2 * K * H * 2 * ffn},
+        "mlp_down": {"bound": "tensor", "flops": 2 * K * ffn * H},
+        "lower_mlp_gate_up": {"bound": "tensor", "flops": 2 * T * H * 2 * ffn},
+        "lower_mlp_down": {"bound": "tensor", "flops": 2 * T * ffn * H},
     }
 
 
@@ -201,15 +210,24 @@ def run_ours(args, rank, world):
     h = S.hidden_rows(wl)
     pr = S.prunable_mask(wl)
     gate = {k: v.to(dev) for k, v in S.gate_weights(wl).items()}
+    def to_dev(d):
+        return {k: (to_dev(v) if isinstance(v, dict) else v.to(dev) if torch.is_tensor(v) else v)
+                for k, v in d.items()}
+
     layers = []
     for i in range(wl.n_layers):
         L = S.layer_weights(wl, i)
-        layers.append({k: (v.to(dev) if torch.is_tensor(v) else v) for k, v in L.items()})
+        if args.full_layers:
+            L = dict(L, **S.layer_body_parts(wl, i))
+        layers.append(to_dev(L))
     scores = S.drawn_scores(wl).to(dev) if wl.planted_cluster else None
     lower = None
     if args.lower_layers:
-        lower = tg.FullContextLayers([{k: v.to(dev) for k, v in L.items()}
-                                      for L in S.lower_layer_weights(wl, args.lower_layers)],
+        lower_w = S.lower_layer_weights(wl, args.lower_layers)
+        if args.full_layers:
+            lower_w = [dict(L, **S.layer_body_parts(wl, i, lower=True))
+                       for i, L in enumerate(lower_w)]
+        lower = tg.FullContextLayers([to_dev(L) for L in lower_w],
                                      wl.n_q_heads, wl.n_kv_heads, wl.head_dim, wl.rope_theta,
                                      device=dev)
     pipe = tg.GatedPrefill(gate, layers, wl.n_q_heads, wl.n_kv_heads, wl.head_dim,
@@ -369,7 +387,8 @@ def run_ours(args, rank, world):
 
     # ---- per-stage roofline
     peaks, peak_src = load_peaks()
-    work = stage_work(wl, [int(x) for x in P["ck_h"].tolist()])
+    work = stage_work(wl, [int(x) for x in P["ck_h"].tolist()],
+                      S.FFN if args.full_layers else 0)
     stages = {}
     for name, ms_list in per_stage.items():
         n_launch = len(ms_list)
@@ -404,6 +423,8 @@ def run_ours(args, rank, world):
                    if wl.batch <= 8 else None, "question_tokens": list(wl.questions)
                    if wl.batch <= 8 else None, "kept": int(P["ck_h"][-1]),
                    "gated_layers": wl.n_layers, "lower_layers": args.lower_layers,
+                   "layer_body": "full (QK-norm, SwiGLU 6144)" if args.full_layers
+                   else "attention only",
                    "hidden": wl.hidden,
                    "heads": f"{wl.n_q_heads}q/{wl.n_kv_heads}kv x {wl.head_dim}",
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
