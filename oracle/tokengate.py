@@ -52,7 +52,7 @@ __all__ = [
     "select_topk", "gather_rows", "rope", "rope_angles", "temperature",
     "gated_attention", "kv_compact", "gated_layer", "prefill", "silu",
     "request_positions", "causal_attention", "full_context_layer",
-    "rmsnorm_heads", "swiglu_mlp",
+    "rmsnorm_heads", "swiglu_mlp", "gated_attention_bias_grad",
 ]
 
 
@@ -286,6 +286,54 @@ def gated_attention(Q, K, V, cu_kept, kept_pos, kept_bias, gamma, beta,
                 O[lo + qi, h, :] = (e / den) @ V[lo:lo + kmax, g, :]
                 lse[h, lo + qi] = (m + np.log(den))[:, 0]
     return O, lse
+
+
+def gated_attention_bias_grad(Q, K, V, dO, cu_kept, kept_pos, kept_bias, gamma, beta):
+    """Gradients of a loss L through token-gated attention, given dL/dO, with respect to
+    the key bias, the per-head gains and the temperature scale: what training the gate
+    end to end needs ([fluxbbs] 端到端训练的关键在 token 门控注意力: the gate is trained
+    through the attention it biases; [digest] 方法关键点).
+
+    With l[r, c] = tau_r s[r, c] + gamma_h b_c, s = q.k / sqrt(d), P = softmax_c(l),
+    O_r = sum_c P[r, c] v_c, the softmax Jacobian gives
+        dl[r, c] = P[r, c] (dO_r.v_c - dO_r.O_r),
+    and l is linear in b_c (slope gamma_h), gamma_h (slope b_c) and beta (slope
+    (tau_r / beta) s[r, c], with tau_r / beta = ln(r + 1) / ln(p_r + 1), 1 at p_r = 0).
+    Returns (d_bias [Kt], d_gamma [Hq], d_beta) in float64.
+    """
+    Q, K, V, dO = as_f64(Q), as_f64(K), as_f64(V), as_f64(dO)
+    ck = _as_int(cu_kept)
+    pos = _as_int(kept_pos)
+    bias = as_f64(kept_bias)
+    gamma = as_f64(gamma)
+    Kt, Hq, d = Q.shape
+    grp = Hq // K.shape[1]
+    d_bias = np.zeros(Kt)
+    d_gamma = np.zeros(Hq)
+    d_beta = 0.0
+    for b in range(len(ck) - 1):
+        lo, hi = ck[b], ck[b + 1]
+        n = hi - lo
+        if n == 0:
+            continue
+        rank = np.arange(n)
+        rho = temperature(rank, pos[lo:hi], 1.0)  # tau / beta
+        causal = np.arange(n)[None, :] <= np.arange(n)[:, None]
+        for h in range(Hq):
+            g = h // grp
+            s = Q[lo:hi, h, :] @ K[lo:hi, g, :].T / math.sqrt(d)
+            logit = np.where(causal, beta * rho[:, None] * s + gamma[h] * bias[None, lo:hi],
+                             -np.inf)
+            P = np.exp(logit - logit.max(axis=1, keepdims=True))
+            P /= P.sum(axis=1, keepdims=True)
+            O = P @ V[lo:hi, g, :]
+            dP = dO[lo:hi, h, :] @ V[lo:hi, g, :].T
+            delta = np.sum(dO[lo:hi, h, :] * O, axis=1)
+            dl = np.where(causal, P * (dP - delta[:, None]), 0.0)
+            d_bias[lo:hi] += gamma[h] * dl.sum(axis=0)
+            d_gamma[h] += np.sum(dl * bias[None, lo:hi])
+            d_beta += np.sum(dl * rho[:, None] * s)
+    return d_bias, d_gamma, d_beta
 
 
 def kv_compact(K, V, row_idx=None):

@@ -575,3 +575,74 @@ def test_full_layer_mlp_follows_attention():
                                 **parts)
     np.testing.assert_allclose(f, g, atol=1e-12)
     np.testing.assert_allclose(kf, kg, atol=1e-12)
+
+
+# ------------------------------------------------------------------ attention gradients
+
+def _torch_gated_attention(Q, K, V, cu, pos, bias, gamma, beta):
+    """The gated attention written directly in torch (float64), for autograd."""
+    Kt, Hq, d = Q.shape
+    grp = Hq // K.shape[1]
+    outs = []
+    for b in range(len(cu) - 1):
+        lo, hi = int(cu[b]), int(cu[b + 1])
+        n = hi - lo
+        r = torch.arange(n, dtype=torch.float64)
+        p = torch.tensor(np.asarray(pos[lo:hi]), dtype=torch.float64)
+        ratio = torch.where(p > 0, torch.log(r + 1) / torch.log(p.clamp(min=1) + 1),
+                            torch.ones_like(r))
+        tau = beta * ratio
+        mask = torch.triu(torch.ones(n, n, dtype=torch.bool), 1)
+        heads = []
+        for h in range(Hq):
+            s = Q[lo:hi, h] @ K[lo:hi, h // grp].T / math.sqrt(d)
+            logit = tau[:, None] * s + gamma[h] * bias[None, lo:hi]
+            w = torch.softmax(logit.masked_fill(mask, float("-inf")), dim=1)
+            heads.append(w @ V[lo:hi, h // grp])
+        outs.append(torch.stack(heads, 1))
+    return torch.cat(outs, 0)
+
+
+@pytest.mark.parametrize("seed", range(3))
+def test_bias_grad_against_autograd(seed):
+    """d_bias, d_gamma, d_beta against torch.autograd through the forward written in torch."""
+    Q, K, V, cu, pos, bias, gamma = _rand_attn_case(60 + seed, [9, 1, 14])
+    beta = 0.7 + 0.2 * seed
+    dO = np.random.default_rng(70 + seed).normal(size=Q.shape)
+    tb = torch.tensor(bias, requires_grad=True)
+    tg_ = torch.tensor(gamma, requires_grad=True)
+    tbeta = torch.tensor(beta, dtype=torch.float64, requires_grad=True)
+    out = _torch_gated_attention(torch.tensor(Q), torch.tensor(K), torch.tensor(V), cu, pos,
+                                 tb, tg_, tbeta)
+    (out * torch.tensor(dO)).sum().backward()
+    db, dg, dbeta = O.gated_attention_bias_grad(Q, K, V, dO, cu, pos, bias, gamma, beta)
+    np.testing.assert_allclose(db, tb.grad.numpy(), atol=1e-11)
+    np.testing.assert_allclose(dg, tg_.grad.numpy(), atol=1e-11)
+    np.testing.assert_allclose(dbeta, tbeta.grad.item(), atol=1e-11)
+
+
+def test_bias_grad_finite_differences_and_invariants():
+    Q, K, V, cu, pos, bias, gamma = _rand_attn_case(80, [7, 5])
+    dO = np.random.default_rng(81).normal(size=Q.shape)
+    db, dg, dbeta = O.gated_attention_bias_grad(Q, K, V, dO, cu, pos, bias, gamma, 0.9)
+
+    def loss(bias_=bias, gamma_=gamma, beta_=0.9):
+        o, _ = O.gated_attention(Q, K, V, cu, pos, bias_, gamma_, beta_)
+        return float(np.sum(o * dO))
+    eps = 1e-6
+    for c in (0, 3, 8, 11):
+        e = np.zeros_like(bias)
+        e[c] = eps
+        fd = (loss(bias_=bias + e) - loss(bias_=bias - e)) / (2 * eps)
+        assert abs(fd - db[c]) < 1e-7
+    fd = (loss(beta_=0.9 + eps) - loss(beta_=0.9 - eps)) / (2 * eps)
+    assert abs(fd - dbeta) < 1e-7
+    e = np.zeros_like(gamma)
+    e[2] = eps
+    assert abs((loss(gamma_=gamma + e) - loss(gamma_=gamma - e)) / (2 * eps) - dg[2]) < 1e-7
+    # softmax shift invariance: a bias constant over a request has zero total gradient
+    for b in range(2):
+        assert abs(db[cu[b]:cu[b + 1]].sum()) < 1e-10
+    # gamma = 0 leaves the bias gradient zero; the first row of a request (one key) has none
+    db0, _, _ = O.gated_attention_bias_grad(Q, K, V, dO, cu, pos, bias, np.zeros(4), 0.9)
+    np.testing.assert_allclose(db0, 0.0, atol=0)
