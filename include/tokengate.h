@@ -328,6 +328,38 @@ int tg_gated_attention(const tg_bf16* q, int64_t ld_q, const tg_bf16* k, int64_t
 size_t tg_gated_attention_workspace_size(const int32_t* cu_kept_host, int batch,
                                          int n_q_heads, int n_kv_heads, int head_dim);
 
+/*
+ * Backward of tg_gated_attention with respect to the gate, what training it end to end
+ * needs ([fluxbbs] 端到端训练的关键在 token 门控注意力; [digest] 方法关键点).  Given the
+ * forward's inputs, its output o and natural-log lse, and dO = dL/do:
+ *   dl[r, c]   = P[r, c] (dO_r . v_c - dO_r . o_r)        (c <= r, same request)
+ *   d_bias[c]  = sum_h gamma_h sum_r dl[r, c]              float32 [K_tot], required
+ *   d_gamma[h] = sum_{r,c} dl[r, c] kept_bias[c]           float32 [n_q_heads], or NULL
+ *   d_beta     = sum_{h,r,c} dl[r, c] (tau_r / beta) q_r.k_c / sqrt(head_dim)   float32 [1], or NULL
+ * with P recomputed from q, k, the bias and lse exactly as the forward formed the logits.
+ * d_bias is the gradient for kept_bias; the gradient of a prunable token's gate score z is
+ * d_bias of its kept row (a question token has none).  Layouts, shapes and limits as
+ * tg_gated_attention; d_o: bf16 [K_tot, n_q_heads * head_dim] (ld_do); lse: float32
+ * [n_q_heads, K_tot] from that forward call.  workspace: at least
+ * tg_gated_attention_bias_grad_workspace_size(...) bytes (no zero-fill needed; 16-byte
+ * aligned).  tcgen05 kernel, one CTA per (request, 128-key tile, chunk of query tiles,
+ * kv head): S^T = K Q^T (+ the bias step) and dP^T = V dO^T in TMEM, one thread per key;
+ * partial sums reduced by two small kernels in a fixed order, so the results are
+ * deterministic.  Bounded waits as the forward (TG_STATUS_TIMEOUT).  status may be NULL.
+ */
+int tg_gated_attention_bias_grad(const tg_bf16* q, int64_t ld_q, const tg_bf16* k,
+                                 int64_t ld_k, const tg_bf16* v, int64_t ld_v, const tg_bf16* o,
+                                 int64_t ld_o, const tg_bf16* d_o, int64_t ld_do,
+                                 const float* lse, const int32_t* cu_kept,
+                                 const int32_t* cu_kept_host, int batch, int n_q_heads,
+                                 int n_kv_heads, int head_dim, const int32_t* kept_pos,
+                                 const float* kept_bias, const float* gamma, float beta,
+                                 float* d_bias, float* d_gamma, float* d_beta, void* workspace,
+                                 size_t workspace_bytes, uint32_t* status, tg_stream_t stream);
+size_t tg_gated_attention_bias_grad_workspace_size(const int32_t* cu_kept_host, int batch,
+                                                   int n_q_heads, int n_kv_heads,
+                                                   int head_dim);
+
 /* ------------------------------------------------------------------ projections */
 
 /*

@@ -28,6 +28,7 @@ __all__ = [
     "tg_status_clear", "tg_status_read", "tg_set_launch_overlap", "tg_get_launch_overlap",
     "tg_prefetch_l2", "tg_out_proj_qkv_next", "tg_out_proj_qkv_workspace_size",
     "tg_swiglu", "tg_fold_norm_weight", "tg_pack_gate_up", "prepare_layer",
+    "tg_gated_attention_bias_grad", "tg_gated_attention_bias_grad_workspace_size",
     "GatedPrefill", "FullContextLayers", "LayerWeights", "STATUS_TIMEOUT", "STATUS_BUDGET",
     "STATUS_BOUNDS", "STATUS_WORKSPACE",
 ]
@@ -296,6 +297,37 @@ def tg_gated_attention(q, k, v, cu_kept, cu_kept_host, n_q_heads, n_kv_heads, ke
     _check(rc, "tg_gated_attention")
     _count()
     return o
+
+
+def tg_gated_attention_bias_grad_workspace_size(cu_kept_host, n_q_heads, n_kv_heads,
+                                                head_dim=128) -> int:
+    ckh = _host_i32(cu_kept_host)
+    return int(lib.tg_gated_attention_bias_grad_workspace_size(_ptr(ckh), ckh.numel() - 1,
+                                                               n_q_heads, n_kv_heads, head_dim))
+
+
+def tg_gated_attention_bias_grad(q, k, v, o, d_o, lse, cu_kept, cu_kept_host, n_q_heads,
+                                 n_kv_heads, kept_pos, kept_bias, gamma, beta, d_bias=None,
+                                 d_gamma=None, d_beta=None, head_dim=128, workspace=None,
+                                 status=None, stream=None):
+    """Gradients of token-gated attention w.r.t. the key bias (returned), and into
+    d_gamma [Hq] / d_beta [1] when given, from the forward's o and lse and dO."""
+    ckh = _host_i32(cu_kept_host)
+    batch = ckh.numel() - 1
+    if d_bias is None:
+        d_bias = torch.empty(q.shape[0], dtype=torch.float32, device=q.device)
+    if workspace is None:
+        need = tg_gated_attention_bias_grad_workspace_size(ckh, n_q_heads, n_kv_heads, head_dim)
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    rc = lib.tg_gated_attention_bias_grad(
+        _ptr(q), _mat(q, "q"), _ptr(k), _mat(k, "k"), _ptr(v), _mat(v, "v"), _ptr(o),
+        _mat(o, "o"), _ptr(d_o), _mat(d_o, "d_o"), _ptr(lse), _ptr(cu_kept), _ptr(ckh), batch,
+        n_q_heads, n_kv_heads, head_dim, _ptr(kept_pos), _ptr(kept_bias), _ptr(gamma),
+        float(beta), _ptr(d_bias), _ptr(d_gamma), _ptr(d_beta), _ptr(workspace),
+        workspace.numel(), _ptr(status), _stream(stream))
+    _check(rc, "tg_gated_attention_bias_grad")
+    _count(4 if int(ckh[-1]) > 0 else 1)
+    return d_bias
 
 
 def tg_linear(a, w, c=None, rmsnorm=False, eps=1e-6, residual=None, row_ssq=None, status=None,

@@ -37,6 +37,7 @@
 #include <functional>
 #include <vector>
 
+#include "tg_attn_common.cuh"
 #include "tg_host.h"
 #include "tg_ptx.cuh"
 
@@ -55,30 +56,18 @@ static_assert(128 * kRegsLow + 256 * kRegsHigh <= kThreads * kLaunchRegs,
               "register split exceeds the launch allocation");
 constexpr int kMaxBatch = 512;  // requests per call (tile table lives in the parameters)
 constexpr int kTileBytes = kBM * kD * 2;  // 32 KB: 128 rows x 128 bf16, two 64-column boxes
-constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLog2e = kAttnLog2e;
 constexpr float kRescaleThreshold = 8.0f;
 
-// x ~ hi + lo with both parts bf16 (round to nearest): hi carries 8 significant bits,
-// lo the next 8.
-__device__ __forceinline__ void split_bf16(float x, uint16_t& hi, uint16_t& lo) {
-  const __nv_bfloat16 h = __float2bfloat16_rn(x);
-  const __nv_bfloat16 l = __float2bfloat16_rn(x - __bfloat162float(h));
-  hi = *reinterpret_cast<const uint16_t*>(&h);
-  lo = *reinterpret_cast<const uint16_t*>(&l);
-}
 constexpr int kMaxParts = 8;    // parts per split query tile
 constexpr int kBoxBytes = kBM * 64 * 2;  // one 64-column bf16 box of a 128-row tile
 // Epilogue staging (the Q/K/V/bias region is free once every MMA has retired): a split
 // part's block for both heads at 0, the bf16 output tile (2 heads x 2 boxes) after it.
 constexpr int kEpiOut = 2 * (kBM * kD + 2 * kBM) * 4;
 
-// Extra K columns of the S = Q K^T MMA that add the gate bias: a 128 x 16 bf16 operand
-// in the no-swizzle core-matrix layout (8-row x 16-byte core matrices; the two along K
-// 128 bytes apart, 8-row groups 256 bytes apart).
-constexpr int kExBytes = 128 * 16 * 2;
-__host__ __device__ constexpr int ex_off(int row, int chunk) {
-  return (row >> 3) * 256 + chunk * 128 + (row & 7) * 16;
-}
+// Extra K columns of the S = Q K^T MMA that add the gate bias (layout in
+// tg_attn_common.cuh).
+constexpr int kExBytes = kAttnExBytes;
 
 struct AttnSmem {
   // 1024-aligned tiles first
@@ -314,14 +303,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         {
           unsigned char* bx = smem + AttnSmem::BEX + s * kExBytes;
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            uint16_t b_hi, b_lo;
-            split_bf16(bv[e], b_hi, b_lo);
-            const int key = lane * 4 + e;
-            *reinterpret_cast<uint4*>(bx + ex_off(key, 0)) =
-                make_uint4((uint32_t)b_hi | ((uint32_t)b_lo << 16), b_hi, 0u, 0u);
-            *reinterpret_cast<uint4*>(bx + ex_off(key, 1)) = make_uint4(0u, 0u, 0u, 0u);
-          }
+          for (int e = 0; e < 4; ++e) attn_put_key_bias(bx, lane * 4 + e, bv[e]);
           fence_proxy_async_smem();
           __syncwarp();
           if (lane == 0) mbar_arrive(&bx_full[s]);
@@ -448,12 +430,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t s_t = tmem + lane_off + (wg ? 128u : 0u);
     const uint32_t o_t = tmem + lane_off + (wg ? 384u : 256u);
 
-    double tau = (double)p.beta;
-    if (row_valid) {
-      const int pos = p.kept_pos[row0 + r];
-      if (pos > 0) tau = (double)p.beta * log((double)r + 1.0) / log((double)pos + 1.0);
-    }
-    const float tau2 = (float)(tau / sqrt((double)kD) * 1.4426950408889634);
+    const double tau = attn_tau(p.beta, r, row_valid ? p.kept_pos[row0 + r] : 0);
 
     // The logit in the log2 domain is t * S with t = tau_r * log2(e) / sqrt(d) and
     // S = q.k + (gamma_h * log2(e) / t) * bias_c: the tensor core adds the bias term
@@ -461,14 +438,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     // split into bf16 parts (g_hi, g_hi, g_lo).  t >= 0 (beta >= 0); t = 0 (first kept
     // token of a request whose position is not 0) is taken as 2^-66, which leaves
     // t * S = gamma_h log2(e) bias_c.
-    const float t2 = fmaxf(tau2, 0x1p-66f);
+    const float t2 = attn_logit_scale(tau, kD);
     {
-      uint16_t g_hi, g_lo;
-      split_bf16(p.gamma[hh] * kLog2e / t2, g_hi, g_lo);
-      unsigned char* ax = smem + AttnSmem::AEX + wg * kExBytes;
-      *reinterpret_cast<uint4*>(ax + ex_off(rit, 0)) =
-          make_uint4((uint32_t)g_hi | ((uint32_t)g_hi << 16), g_lo, 0u, 0u);
-      *reinterpret_cast<uint4*>(ax + ex_off(rit, 1)) = make_uint4(0u, 0u, 0u, 0u);
+      attn_put_query_gain(smem + AttnSmem::AEX + wg * kExBytes, rit, p.gamma[hh] * kLog2e / t2);
       fence_proxy_async_smem();  // read by the tensor core
       mbar_arrive(&ax_ready[wg]);
     }

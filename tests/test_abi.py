@@ -158,3 +158,19 @@ def test_full_body_argument_checks(lib):
     assert lib.tg_pack_gate_up(p, 2048, None, 2048, 128, 2048, None, p, 2048, None) == -1
     assert lib.tg_fold_norm_weight(p, 2048, 16, 2048, None, p, 2048, None) == -1
     assert lib.tg_fold_norm_weight(p, 2048, 0, 2048, p, p, 2048, None) == 0
+
+
+def test_bias_grad_argument_checks(lib):
+    p = C.c_void_p(0x10000)
+    ck = (C.c_int32 * 2)(0, 300)
+
+    def call(beta=1.0, ws=p, ws_bytes=1 << 30, d_bias=p, head_dim=128, hq=16):
+        return lib.tg_gated_attention_bias_grad(p, 2048, p, 1024, p, 1024, p, 2048, p, 2048, p, p,
+                                                ck, 1, hq, 8, head_dim, p, p, p, beta, d_bias,
+                                                None, None, ws, ws_bytes, None, None)
+    assert call(head_dim=64) == -6
+    assert call(hq=24) == -6          # odd group of q heads per kv head
+    assert call(hq=12) == -1          # not a multiple of the kv heads
+    assert call(beta=-1.0) == -1
+    assert call(d_bias=None) == -1
+    assert lib.tg_gated_attention_bias_grad_workspace_size(ck, 1, 16, 8, 64) == 0

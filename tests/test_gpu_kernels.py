@@ -660,3 +660,71 @@ def test_swiglu_against_oracle(tg, M):
     err = np.abs(_f64(h.cpu()) - want)
     assert np.all(err <= 2.0 ** -7 * np.abs(want) + 2e-3), err.max()
     assert err.mean() <= 1e-3
+
+
+# ------------------------------------------------------------------ attention backward
+#
+# The backward forms delta_r = dO_r . O_r from the forward's bf16 output O, the one
+# rounding on its path that the float64 oracle does not make.  An oracle-only study
+# (delta from bf16(O) against exact O, lengths [300], [1, 129, 700], [1638], 16 q / 8 kv
+# heads, N(0, 1) inputs) moves d_bias by at most 0.0026 max|d_bias| (rms 0.0015 of its
+# rms), d_gamma by 0.0045 max|d_gamma| and d_beta by 0.001 of its size.  Bounds: 3-4x.
+
+def _bias_grad_case(tg, lengths, seed, beta=1.0, gamma_zero=False, with_beta=True):
+    Hq, Hkv, d = 16, 8, 128
+    q, k, v, pos, bias, gamma, cu = _attn_inputs(lengths, Hq, Hkv, seed)
+    if gamma_zero:
+        gamma = torch.zeros_like(gamma)
+    d_o = (torch.randn(q.shape, generator=torch.Generator().manual_seed(seed + 1))
+           ).to(torch.bfloat16)
+    o, lse = _run_attention(tg, q, k, v, pos, bias, gamma, beta, cu, Hq, Hkv)
+    st = _status()
+    dg = torch.full((Hq,), float("nan"), device="cuda")
+    dbeta = torch.full((1,), float("nan"), device="cuda") if with_beta else None
+    db = tg.tg_gated_attention_bias_grad(_dev(q), _dev(k), _dev(v), _dev(o), _dev(d_o), _dev(lse),
+                                         _dev(torch.from_numpy(cu)), cu, Hq, Hkv, _dev(pos),
+                                         _dev(bias), _dev(gamma), beta, d_gamma=dg, d_beta=dbeta,
+                                         status=st)
+    assert tg.tg_status_read(st) == 0
+    return (q, k, v, d_o, pos, bias, gamma, cu), db.cpu(), dg.cpu(), (
+        dbeta.cpu() if with_beta else None)
+
+
+def _check_bias_grad(inputs, db, dg, dbeta, beta):
+    q, k, v, d_o, pos, bias, gamma, cu = inputs
+    Kt = q.shape[0]
+    want_b, want_g, want_beta = O.gated_attention_bias_grad(
+        _f64(q).reshape(Kt, 16, 128), _f64(k).reshape(Kt, 8, 128), _f64(v).reshape(Kt, 8, 128),
+        _f64(d_o).reshape(Kt, 16, 128), cu, pos, bias, gamma, beta)
+    err = np.abs(_f64(db) - want_b)
+    scale = np.abs(want_b).max()
+    # absolute floor 1e-3: fp32 accumulation where the exact gradient vanishes (a
+    # one-key row has P = 1 and dl = dP - delta = 0); the gradients here are O(10-100)
+    assert err.max() <= 0.01 * scale + 1e-3, (err.max(), scale)
+    assert err.mean() <= 0.004 * np.sqrt(np.mean(want_b ** 2)) + 1e-3, err.mean()
+    eg = np.abs(_f64(dg) - want_g)
+    assert eg.max() <= 0.015 * np.abs(want_g).max() + 1e-3, (eg.max(), np.abs(want_g).max())
+    if dbeta is not None:
+        assert abs(float(dbeta[0]) - want_beta) <= 0.01 * max(abs(want_beta),
+                                                                np.abs(want_g).max()) + 1e-3, \
+            (float(dbeta[0]), want_beta)
+
+
+@pytest.mark.parametrize("lengths", [[1], [300], [1, 129, 700, 0, 257]])
+def test_bias_grad_against_oracle(tg, lengths):
+    inputs, db, dg, dbeta = _bias_grad_case(tg, lengths, seed=len(lengths) * 7 + lengths[0])
+    _check_bias_grad(inputs, db, dg, dbeta, 1.0)
+
+
+def test_bias_grad_kept_1638_and_beta(tg):
+    """One request at the 16k workload's kept count, a non-unit temperature scale."""
+    inputs, db, dg, dbeta = _bias_grad_case(tg, [1638], seed=5, beta=0.8)
+    _check_bias_grad(inputs, db, dg, dbeta, 0.8)
+
+
+def test_bias_grad_deterministic_and_gamma_zero(tg):
+    _, db1, dg1, dbeta1 = _bias_grad_case(tg, [700, 333], seed=9)
+    _, db2, dg2, dbeta2 = _bias_grad_case(tg, [700, 333], seed=9)
+    assert torch.equal(db1, db2) and torch.equal(dg1, dg2) and torch.equal(dbeta1, dbeta2)
+    _, db0, _, _ = _bias_grad_case(tg, [700, 333], seed=9, gamma_zero=True, with_beta=False)
+    assert torch.count_nonzero(db0) == 0
