@@ -65,6 +65,8 @@ def parse_args():
     ap.add_argument("--full-layers", action="store_true",
                     help="full layer bodies (weighted norms, QK-norm, SwiGLU MLP of width "
                          "6144) instead of attention-only layers")
+    ap.add_argument("--bias-grad-steps", type=int, default=10,
+                    help="timed calls of the attention backward w.r.t. the gate (0 skips it)")
     ap.add_argument("--dense-steps", type=int, default=3,
                     help="timed steps of the full-context reference (0 skips it)")
     return ap.parse_args()
@@ -439,11 +441,70 @@ def run_ours(args, rank, world):
                        for kk, vv in v.items()} for k, v in stages.items()},
         "clocks": clk.summary(),
     }
+    if args.bias_grad_steps > 0 and int(P["K"]) > 0:
+        out["bias_grad"] = bias_grad_timing(tg, wl, P, pipe, flush, stream,
+                                            args.bias_grad_steps, peaks)
     if args.dense_steps > 0:
         out["dense_reference"] = dense_reference(tg, wl, layers, h_dev, flush, stream,
                                                  args.dense_steps, peaks,
                                                  total_ms / args.steps)
     return out
+
+
+def bias_grad_timing(tg, wl, P, pipe, flush, stream, steps, peaks):
+    """The attention backward w.r.t. the gate (key bias, gains, temperature scale) on the
+    last gated layer's Q and compacted K/V of the step just run, with a seeded dO: CUDA
+    events around each call (its four launches), L2 flushed before each."""
+    import torch
+    nq = wl.n_q_heads * wl.head_dim
+    L = pipe.layers[-1]
+    q = P["qkv"][:, :nq]
+    ck, cv = P["caches"][-1]
+    K = int(P["K"])
+    dev = q.device
+    lse = torch.empty((wl.n_q_heads, K), dtype=torch.float32, device=dev)
+    o = tg.tg_gated_attention(q, ck, cv, P["ck"], P["ck_h"], wl.n_q_heads, wl.n_kv_heads,
+                              P["kept_pos"], P["kept_bias"], L.gamma, L.beta, lse=lse)
+    g = torch.Generator(device="cpu").manual_seed(17)
+    d_o = torch.randn((K, nq), generator=g).to(torch.bfloat16).to(dev)
+    d_bias = torch.empty(K, dtype=torch.float32, device=dev)
+    d_gamma = torch.empty(wl.n_q_heads, dtype=torch.float32, device=dev)
+    d_beta = torch.empty(1, dtype=torch.float32, device=dev)
+    ws = torch.empty(max(16, tg.tg_gated_attention_bias_grad_workspace_size(
+        P["ck_h"], wl.n_q_heads, wl.n_kv_heads)), dtype=torch.uint8, device=dev)
+
+    def call():
+        tg.tg_gated_attention_bias_grad(q, ck, cv, o, d_o, lse, P["ck"], P["ck_h"],
+                                        wl.n_q_heads, wl.n_kv_heads, P["kept_pos"],
+                                        P["kept_bias"], L.gamma, L.beta, d_bias=d_bias,
+                                        d_gamma=d_gamma, d_beta=d_beta, workspace=ws,
+                                        status=pipe.status)
+    for _ in range(3):
+        call()
+    torch.cuda.synchronize()
+    ms = []
+    for _ in range(steps):
+        flush.fill_(1.0)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        call()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ms.append(e0.elapsed_time(e1))
+    status = tg.tg_status_read(pipe.status)
+    if status:
+        raise SystemExit(f"device status {status:#x} in the attention backward")
+    avg = sum(ms) / len(ms)
+    Ks = [int(P["ck_h"][b + 1] - P["ck_h"][b]) for b in range(wl.batch)]
+    flops = 4 * wl.head_dim * wl.n_q_heads * sum(k * (k + 1) // 2 for k in Ks)
+    tf = flops / (avg / 1e3) / 1e12
+    peak = peaks["bf16_tflops"]
+    return {"what": "d kept_bias, d gamma, d beta of the last gated layer's attention, "
+                    "seeded dO (preparation + tcgen05 kernel + two reductions)",
+            "kept": K, "calls": steps, "avg_ms": avg, "achieved": tf, "unit": "TFLOP/s",
+            "peak": peak, "frac": tf / peak,
+            "flops_counted": "S^T = K Q^T and dP^T = V dO^T over the causal pairs"}
 
 
 def dense_reference(tg, wl, layers, h_dev, flush, stream, steps, peaks, gated_ms):

@@ -18,10 +18,12 @@
 //   S^T  = K Q^T (+ one K=16 step adding g_r b_c, as in the forward)  -> TMEM [0,128)/[128,256)
 //   dP^T = V dO^T                                                     -> TMEM [256,384)/[384,512)
 // and the compute warps form P = 2^(t_r S - lse2_r) from the forward's log-sum-exp, then
-// dl = P (dP - delta_r).  Per-query scalars (t_r, lse2_r, delta_r = dO_r.O_r, and the
-// temperature-gradient factors) come from a preparation kernel and sit in shared memory
-// next to each head's Q and dO tiles; rows past the request get lse2 = +inf, so they
-// contribute nothing.  Partial sums per (work item, head, key) go to the workspace and
+// dl = P (dP - delta_r).  A preparation kernel lays out, per q head and query tile, one
+// contiguous block: the gain operand of the bias step and the per-query scalars (t_r,
+// lse2_r, delta_r = dO_r.O_r, and the temperature-gradient factors), with lse2 = +inf
+// on rows past the request so that they contribute nothing; one bulk copy brings it in.
+// Q and dO stages are freed by the MMAs that read them (so the next tile's loads overlap
+// the compute warps), the blocks by the compute warps through a deeper ring.  Partial sums per (work item, head, key) go to the workspace and
 // two small kernels reduce them in a fixed order (deterministic results).
 // Warps: 0 producer (K, V once; per query tile and head Q, dO by TMA plus the scalars and
 // the gain operand), 1 MMA issuer, 2-5 head h0, 6-9 head h0 + 1.
@@ -44,33 +46,36 @@ constexpr int kTk = 128;      // keys per tile
 constexpr int kThreads = 320;
 constexpr int kMaxBatch = 512;
 constexpr int kTileBytes = 128 * kD * 2;  // 128 rows x 128 bf16 as two 64-column boxes
-constexpr int kColBytes = kTq * 16;       // one float4 per query row
+// Per (q head, query tile) block written by the preparation kernel: the gain operand
+// (kAttnExBytes), float4 {t, lse2, delta, rho_s} per row, float u = rho_s g per row.
+constexpr int kBlkGX = 0;
+constexpr int kBlkA = kBlkGX + kAttnExBytes;
+constexpr int kBlkU = kBlkA + kTq * 16;
+constexpr int kBlockBytes = kBlkU + kTq * 4;
+static_assert(kBlockBytes % 16 == 0, "bulk copies move multiples of 16 bytes");
 
+// Work units u = 2 j + s: query tile j of the item, head s of the pair.  Q and dO stages
+// follow the head (stage s), blocks a ring of four.
+constexpr int kBlkStages = 4;
 struct BwdSmem {
   static constexpr int K = 0;
   static constexpr int V = K + kTileBytes;
-  static constexpr int UNIT = V + kTileBytes;  // [2] one per head of the pair
-  static constexpr int U_Q = 0;
-  static constexpr int U_DO = U_Q + kTileBytes;
-  static constexpr int U_GX = U_DO + kTileBytes;      // gain operand of the bias step
-  static constexpr int U_COLA = U_GX + kAttnExBytes;  // float4 {t, lse2, delta, rho_s}
-  static constexpr int U_COLB = U_COLA + kColBytes;   // float4 {u, g, 0, 0}
-  static constexpr int UNIT_BYTES = U_COLB + kColBytes;
-  static constexpr int BX = UNIT + 2 * UNIT_BYTES;    // key-bias operand of the bias step
+  static constexpr int Q = V + kTileBytes;               // [2]
+  static constexpr int DO = Q + 2 * kTileBytes;          // [2]
+  static constexpr int BLK = DO + 2 * kTileBytes;        // [kBlkStages]
+  static constexpr int BX = BLK + kBlkStages * kBlockBytes;  // key-bias operand
   static constexpr int BAR = BX + kAttnExBytes;
   static constexpr int END = BAR + 256;
   static constexpr int BYTES = END + 1024;  // alignment slack
 };
-static_assert(BwdSmem::UNIT_BYTES % 1024 == 0, "unit tiles must stay 1024-byte aligned");
 static_assert(BwdSmem::BYTES <= 227 * 1024, "shared memory budget");
 
 struct BwdParams {
   const int32_t* cu_kept;
   const float* kept_bias;
-  const float4* col_a;  // [n_q_heads, k_total]
-  const float4* col_b;
+  const unsigned char* blocks;  // [n_q_heads][n_tiles] blocks of kBlockBytes
   float* part;          // [item * head_groups + head group][2][2][128]
-  int64_t k_total;
+  int n_tiles;          // query tiles over all requests
   int group;            // n_q_heads / n_kv_heads
   int head_pairs;       // group / 2
   int n_kv_heads;
@@ -78,6 +83,7 @@ struct BwdParams {
   int chunk;            // query tiles per work item
   uint32_t* status;
   int32_t item_prefix[kMaxBatch + 1];
+  int32_t tile_prefix[kMaxBatch + 1];  // query (= key) tiles before request b
 };
 
 __host__ __device__ __forceinline__ int cdiv(int a, int b) { return (a + b - 1) / b; }
@@ -100,50 +106,70 @@ __device__ __forceinline__ int find_request(const int32_t* prefix, int batch, in
 }
 
 // ---------------------------------------------------------------- preparation
-// Per (q head, kept row): the scalars the main kernel reads per query column.
-__global__ void bwd_prep_kernel(const uint16_t* __restrict__ o, int64_t ld_o,
-                                const uint16_t* __restrict__ d_o, int64_t ld_do,
-                                const float* __restrict__ lse, const int32_t* __restrict__ cu_kept,
-                                int batch, const int32_t* __restrict__ kept_pos,
-                                const float* __restrict__ gamma, float beta, int n_q_heads,
-                                int64_t k_total, float4* __restrict__ col_a,
-                                float4* __restrict__ col_b) {
+struct PrepParams {
+  const uint16_t* o;
+  int64_t ld_o;
+  const uint16_t* d_o;
+  int64_t ld_do;
+  const float* lse;        // [n_q_heads, k_total], natural log
+  const int32_t* cu_kept;
+  const int32_t* kept_pos;
+  const float* gamma;
+  float beta;
+  int n_q_heads;
+  int64_t k_total;
+  int batch;
+  int n_tiles;
+  unsigned char* blocks;
+  int32_t tile_prefix[kMaxBatch + 1];
+};
+
+// One thread per (q head, query tile, row of the tile): that row's entries of the block.
+__global__ void bwd_prep_kernel(const __grid_constant__ PrepParams p) {
   griddep_wait();
-  const int64_t n = k_total * n_q_heads;
+  const int64_t n = (int64_t)p.n_q_heads * p.n_tiles * kTq;
   for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n;
        i += (int64_t)gridDim.x * blockDim.x) {
-    const int h = (int)(i / k_total);
-    const int64_t row = i - (int64_t)h * k_total;
-    int lo = 0, hi = batch;
-    while (hi - lo > 1) {
-      const int mid = (lo + hi) >> 1;
-      if (cu_kept[mid] <= row) lo = mid; else hi = mid;
-    }
-    const int r = (int)(row - cu_kept[lo]);
-    const int pos = kept_pos[row];
-    // delta = dO_r . O_r over the head's 128 values
-    const uint4* a = reinterpret_cast<const uint4*>(d_o + row * ld_do + (int64_t)h * kD);
-    const uint4* b = reinterpret_cast<const uint4*>(o + row * ld_o + (int64_t)h * kD);
-    float delta = 0.f;
+    const int rr = (int)(i % kTq);
+    const int64_t ht = i / kTq;  // h * n_tiles + tile
+    const int h = (int)(ht / p.n_tiles);
+    const int tile = (int)(ht - (int64_t)h * p.n_tiles);
+    const int b = find_request(p.tile_prefix, p.batch, tile);
+    const int r = (tile - p.tile_prefix[b]) * kTq + rr;
+    const int n_b = p.cu_kept[b + 1] - p.cu_kept[b];
+    unsigned char* blk = p.blocks + ht * kBlockBytes;
+    float4 a = make_float4(0.f, INFINITY, 0.f, 0.f);
+    float u = 0.f, g = 0.f;
+    if (r < n_b) {
+      const int64_t row = p.cu_kept[b] + r;
+      const int pos = p.kept_pos[row];
+      // delta = dO_r . O_r over the head's 128 values
+      const uint4* x = reinterpret_cast<const uint4*>(p.d_o + row * p.ld_do + (int64_t)h * kD);
+      const uint4* y = reinterpret_cast<const uint4*>(p.o + row * p.ld_o + (int64_t)h * kD);
+      float delta = 0.f;
 #pragma unroll 4
-    for (int k = 0; k < kD / 8; ++k) {
-      const uint4 x = a[k], y = b[k];
-      const uint32_t xs[4] = {x.x, x.y, x.z, x.w}, ys[4] = {y.x, y.y, y.z, y.w};
+      for (int k = 0; k < kD / 8; ++k) {
+        const uint4 xv = x[k], yv = y[k];
+        const uint32_t xs[4] = {xv.x, xv.y, xv.z, xv.w}, ys[4] = {yv.x, yv.y, yv.z, yv.w};
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float2 fx = unpack_bf16x2(xs[e]), fy = unpack_bf16x2(ys[e]);
-        delta = fmaf(fx.x, fy.x, delta);
-        delta = fmaf(fx.y, fy.y, delta);
+        for (int e = 0; e < 4; ++e) {
+          const float2 fx = unpack_bf16x2(xs[e]), fy = unpack_bf16x2(ys[e]);
+          delta = fmaf(fx.x, fy.x, delta);
+          delta = fmaf(fx.y, fy.y, delta);
+        }
       }
+      const double tau = attn_tau(p.beta, r, pos);
+      const float t = attn_logit_scale(tau, kD);
+      g = p.gamma[h] * kAttnLog2e / t;
+      // d l / d beta = (tau / beta) q.k / sqrt(d); tau / beta = 1 at pos = 0
+      const double ratio = pos > 0 ? log((double)r + 1.0) / log((double)pos + 1.0) : 1.0;
+      const float rho_s = (float)(ratio / sqrt((double)kD));
+      a = make_float4(t, p.lse[(int64_t)h * p.k_total + row] * kAttnLog2e, delta, rho_s);
+      u = rho_s * g;
     }
-    const double tau = attn_tau(beta, r, pos);
-    const float t = attn_logit_scale(tau, kD);
-    const float g = gamma[h] * kAttnLog2e / t;
-    // d l / d beta = (tau / beta) q.k / sqrt(d); tau / beta = 1 at pos = 0
-    const double ratio = pos > 0 ? log((double)r + 1.0) / log((double)pos + 1.0) : 1.0;
-    const float rho_s = (float)(ratio / sqrt((double)kD));
-    col_a[i] = make_float4(t, lse[i] * kAttnLog2e, delta, rho_s);
-    col_b[i] = make_float4(rho_s * g, g, 0.f, 0.f);
+    attn_put_query_gain(blk + kBlkGX, rr, g);
+    reinterpret_cast<float4*>(blk + kBlkA)[rr] = a;
+    reinterpret_cast<float*>(blk + kBlkU)[rr] = u;
   }
 }
 
@@ -161,12 +187,16 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + BwdSmem::BAR);
   uint64_t* kv_full = bars + 0;
   uint64_t* bx_full = bars + 1;
-  uint64_t* unit_full = bars + 2;    // [2] Q, dO (bytes) + scalars and gain operand (arrive)
-  uint64_t* unit_empty = bars + 4;   // [2] MMAs done + the head's 4 compute warps done
-  uint64_t* s_full = bars + 6;       // [2] S^T and dP^T of the head in TMEM
-  uint64_t* tmem_free = bars + 8;    // [2] the head's compute threads read them
-  uint64_t* drain = bars + 10;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 11);
+  uint64_t* q_full = bars + 2;       // [2]
+  uint64_t* q_empty = bars + 4;      // [2] the S MMAs that read the stage are done
+  uint64_t* do_full = bars + 6;      // [2]
+  uint64_t* do_empty = bars + 8;     // [2] the dP MMAs that read the stage are done
+  uint64_t* blk_full = bars + 10;    // [kBlkStages]
+  uint64_t* blk_empty = bars + 14;   // [kBlkStages] MMAs + the head's 4 compute warps done
+  uint64_t* s_full = bars + 18;      // [2] S^T and dP^T of the head in TMEM
+  uint64_t* tmem_free = bars + 20;   // [2] the head's compute threads read them
+  uint64_t* drain = bars + 22;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 23);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -174,10 +204,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(kv_full, 1);
     mbar_init(bx_full, 1);
     for (int s = 0; s < 2; ++s) {
-      mbar_init(&unit_full[s], 2);
-      mbar_init(&unit_empty[s], 5);
+      mbar_init(&q_full[s], 1);
+      mbar_init(&q_empty[s], 1);
+      mbar_init(&do_full[s], 1);
+      mbar_init(&do_empty[s], 1);
       mbar_init(&s_full[s], 1);
       mbar_init(&tmem_free[s], 128);
+    }
+    for (int s = 0; s < kBlkStages; ++s) {
+      mbar_init(&blk_full[s], 1);
+      mbar_init(&blk_empty[s], 5);
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -238,48 +274,49 @@ __global__ void __launch_bounds__(kThreads, 1)
     fence_proxy_async_smem();
     __syncwarp();
     if (lane == 0) mbar_arrive(bx_full);
-    int issued = 0;
-    for (int u = 0; u < 2 * nq; ++u, ++issued) {
-      const int s = u & 1;  // unit stage = head of the pair
-      const int j = u >> 1;
-      if (!warp_all(mbar_wait(&unit_empty[s], ((uint32_t)j & 1u) ^ 1u, abort_flag, p.status)))
-        break;
-      unsigned char* un = smem + BwdSmem::UNIT + s * BwdSmem::UNIT_BYTES;
-      const int qt = qt_begin + j;
+    int n_q = 0, n_do = 0, n_blk = 0;  // loads issued into each ring
+    for (int u = 0; u < 2 * nq; ++u) {
+      const int s = u & 1;  // Q / dO stage = head of the pair
+      const int bs = u % kBlkStages;
+      const uint32_t ph2 = (uint32_t)(u >> 1) & 1u, ph4 = (uint32_t)(u / kBlkStages) & 1u;
+      const int qt = qt_begin + (u >> 1);
       const int qy = (int)(row0 + (int64_t)qt * kTq);
       const int hh = h0 + s;
+      if (!warp_all(mbar_wait(&q_empty[s], ph2 ^ 1u, abort_flag, p.status))) break;
+      unsigned char* qs = smem + BwdSmem::Q + s * kTileBytes;
       if (lane == 0) {
-        mbar_arrive_expect_tx(&unit_full[s], 2 * kTileBytes);
-        tma_load_2d(un + BwdSmem::U_Q, &tmQ, hh * kD, qy, &unit_full[s]);
-        tma_load_2d(un + BwdSmem::U_Q + kTileBytes / 2, &tmQ, hh * kD + 64, qy, &unit_full[s]);
-        tma_load_2d(un + BwdSmem::U_DO, &tmDO, hh * kD, qy, &unit_full[s]);
-        tma_load_2d(un + BwdSmem::U_DO + kTileBytes / 2, &tmDO, hh * kD + 64, qy, &unit_full[s]);
+        mbar_arrive_expect_tx(&q_full[s], kTileBytes);
+        tma_load_2d(qs, &tmQ, hh * kD, qy, &q_full[s]);
+        tma_load_2d(qs + kTileBytes / 2, &tmQ, hh * kD + 64, qy, &q_full[s]);
       }
-      float4* ca = reinterpret_cast<float4*>(un + BwdSmem::U_COLA);
-      float4* cb = reinterpret_cast<float4*>(un + BwdSmem::U_COLB);
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int rr = lane * 4 + e;
-        const int r = qt * kTq + rr;
-        float4 a = make_float4(0.f, INFINITY, 0.f, 0.f), bb = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (r < n_b) {
-          const int64_t gi = (int64_t)hh * p.k_total + row0 + r;
-          a = p.col_a[gi];
-          bb = p.col_b[gi];
-        }
-        ca[rr] = a;
-        cb[rr] = bb;
-        attn_put_query_gain(un + BwdSmem::U_GX, rr, bb.y);
+      ++n_q;
+      if (!warp_all(mbar_wait(&blk_empty[bs], ph4 ^ 1u, abort_flag, p.status))) break;
+      if (lane == 0) {
+        mbar_arrive_expect_tx(&blk_full[bs], kBlockBytes);
+        const int64_t blk = (int64_t)hh * p.n_tiles + p.tile_prefix[b] + qt;
+        bulk_load(smem + BwdSmem::BLK + bs * kBlockBytes, p.blocks + blk * kBlockBytes,
+                  kBlockBytes, &blk_full[bs]);
       }
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&unit_full[s]);
+      ++n_blk;
+      if (!warp_all(mbar_wait(&do_empty[s], ph2 ^ 1u, abort_flag, p.status))) break;
+      unsigned char* ds = smem + BwdSmem::DO + s * kTileBytes;
+      if (lane == 0) {
+        mbar_arrive_expect_tx(&do_full[s], kTileBytes);
+        tma_load_2d(ds, &tmDO, hh * kD, qy, &do_full[s]);
+        tma_load_2d(ds + kTileBytes / 2, &tmDO, hh * kD + 64, qy, &do_full[s]);
+      }
+      ++n_do;
     }
     if (lane == 0) {
       // no bulk copy may still be landing when the CTA exits
       mbar_wait(kv_full, 0, nullptr, p.status);
-      for (int u = issued - 2 < 0 ? 0 : issued - 2; u < issued; ++u)
-        mbar_wait(&unit_full[u & 1], (uint32_t)(u >> 1) & 1u, nullptr, p.status);
+      for (int u = n_q - 2 < 0 ? 0 : n_q - 2; u < n_q; ++u)
+        mbar_wait(&q_full[u & 1], (uint32_t)(u >> 1) & 1u, nullptr, p.status);
+      for (int u = n_do - 2 < 0 ? 0 : n_do - 2; u < n_do; ++u)
+        mbar_wait(&do_full[u & 1], (uint32_t)(u >> 1) & 1u, nullptr, p.status);
+      for (int u = n_blk - kBlkStages < 0 ? 0 : n_blk - kBlkStages; u < n_blk; ++u)
+        mbar_wait(&blk_full[u % kBlkStages], (uint32_t)(u / kBlkStages) & 1u, nullptr,
+                  p.status);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
@@ -293,14 +330,20 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int u = 0; ok && u < 2 * nq; ++u) {
         const int s = u & 1;
         const int j = u >> 1;
-        if (!(ok = mbar_wait(&unit_full[s], (uint32_t)j & 1u, abort_flag, p.status))) break;
+        const int bs = u % kBlkStages;
+        const uint32_t ph2 = (uint32_t)j & 1u, ph4 = (uint32_t)(u / kBlkStages) & 1u;
+        if (!(ok = mbar_wait(&q_full[s], ph2, abort_flag, p.status) &&
+                   mbar_wait(&blk_full[bs], ph4, abort_flag, p.status)))
+          break;
         if (j > 0 && !(ok = mbar_wait(&tmem_free[s], (uint32_t)(j - 1) & 1u, abort_flag, p.status)))
           break;
         tc_fence_after();
-        const uint32_t un = smem_u32(smem + BwdSmem::UNIT + s * BwdSmem::UNIT_BYTES);
-        const uint64_t q_desc = sw128_desc(un + BwdSmem::U_Q, 16, 1024);
-        const uint64_t do_desc = sw128_desc(un + BwdSmem::U_DO, 16, 1024);
-        const uint64_t gx_desc = interleave_desc(un + BwdSmem::U_GX, 128, 256);
+        const uint32_t qs = smem_u32(smem + BwdSmem::Q + s * kTileBytes);
+        const uint32_t ds = smem_u32(smem + BwdSmem::DO + s * kTileBytes);
+        const uint64_t q_desc = sw128_desc(qs, 16, 1024);
+        const uint64_t do_desc = sw128_desc(ds, 16, 1024);
+        const uint64_t gx_desc =
+            interleave_desc(smem_u32(smem + BwdSmem::BLK + bs * kBlockBytes + kBlkGX), 128, 256);
         const uint32_t s_col = tmem + (uint32_t)(s * 128);
         const uint32_t d_col = tmem + 256u + (uint32_t)(s * 128);
 #pragma unroll
@@ -309,13 +352,17 @@ __global__ void __launch_bounds__(kThreads, 1)
           mma_ss(s_col, k_desc + off, q_desc + off, idesc, kk != 0);
         }
         mma_ss(s_col, bx_desc, gx_desc, idesc, 1u);  // + g_r b_c
+        mma_commit(&q_empty[s]);
+        if (!(ok = mbar_wait(&do_full[s], ph2, abort_flag, p.status))) break;
+        tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < kD / 16; ++kk) {
           const uint64_t off = (uint64_t)(((kk >> 2) * (kTileBytes / 2) + (kk & 3) * 32) >> 4);
           mma_ss(d_col, v_desc + off, do_desc + off, idesc, kk != 0);
         }
+        mma_commit(&do_empty[s]);
         mma_commit(&s_full[s]);
-        mma_commit(&unit_empty[s]);
+        mma_commit(&blk_empty[bs]);
       }
       mma_commit(drain);
       mbar_wait(drain, 0, nullptr, p.status);  // every MMA retired before TMEM is freed
@@ -330,13 +377,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t lane_off = (uint32_t)(q * 32) << 16;
     const uint32_t s_t = tmem + lane_off + (uint32_t)(wg * 128);
     const uint32_t d_t = tmem + lane_off + 256u + (uint32_t)(wg * 128);
-    const unsigned char* un = smem + BwdSmem::UNIT + wg * BwdSmem::UNIT_BYTES;
-    const float4* ca = reinterpret_cast<const float4*>(un + BwdSmem::U_COLA);
-    const float4* cb = reinterpret_cast<const float4*>(un + BwdSmem::U_COLB);
     float acc = 0.f, accb = 0.f;
     for (int j = 0; j < nq; ++j) {
       if (!warp_all(mbar_wait(&s_full[wg], (uint32_t)j & 1u, abort_flag, p.status))) break;
       tc_fence_after();
+      const int bs = (2 * j + wg) % kBlkStages;
+      // the block's bulk copy has landed (already true: the MMAs waited for it); waiting
+      // on its barrier makes the copied scalars visible to this thread
+      if (!warp_all(mbar_wait(&blk_full[bs], (uint32_t)((2 * j + wg) / kBlkStages) & 1u,
+                              abort_flag, p.status)))
+        break;
+      const unsigned char* blk = smem + BwdSmem::BLK + bs * kBlockBytes;
+      const float4* ca = reinterpret_cast<const float4*>(blk + kBlkA);
+      const float* cu = reinterpret_cast<const float*>(blk + kBlkU);
       const bool diag = qt_begin + j == kt;  // queries before this key are masked
 #pragma unroll 1
       for (int cc = 0; cc < kTq / 32; ++cc) {
@@ -357,11 +410,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (diag && col < key) pr = 0.f;
           const float dl = pr * (__uint_as_float(dv[i]) - a.z);
           acc += dl;
-          if (kBeta) accb = fmaf(dl, fmaf(a.w, s, -cb[col].x * b_c), accb);
+          if (kBeta) accb = fmaf(dl, fmaf(a.w, s, -cu[col] * b_c), accb);
         }
       }
       __syncwarp();
-      if (lane == 0) mbar_arrive(&unit_empty[wg]);  // done with the unit's scalars
+      if (lane == 0) mbar_arrive(&blk_empty[bs]);  // done with the block's scalars
     }
     const int64_t slot = (int64_t)item * hg + head_grp;
     p.part[((slot * 2 + 0) * 2 + wg) * 128 + key] = acc;
@@ -495,14 +548,13 @@ int make_bwd_plan(const int32_t* cu_kept_host, int batch, int head_groups, int s
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 struct BwdLayout {
-  size_t col_a, col_b, part, tile_out, total;
+  size_t blocks, part, tile_out, total;
 };
 
-BwdLayout bwd_layout(int64_t k_total, int n_q_heads, int head_groups, const BwdPlan& plan) {
+BwdLayout bwd_layout(int n_q_heads, int head_groups, const BwdPlan& plan) {
   BwdLayout l;
-  l.col_a = 0;
-  l.col_b = align256((size_t)k_total * n_q_heads * 16);
-  l.part = l.col_b + align256((size_t)k_total * n_q_heads * 16);
+  l.blocks = 0;
+  l.part = align256((size_t)n_q_heads * plan.n_tiles * kBlockBytes);
   l.tile_out = l.part + align256((size_t)plan.n_items * head_groups * 4 * 128 * sizeof(float));
   l.total = l.tile_out + align256((size_t)plan.n_tiles * (n_q_heads + 1) * sizeof(float));
   return l;
@@ -549,7 +601,7 @@ extern "C" size_t tg_gated_attention_bias_grad_workspace_size(const int32_t* cu_
   static thread_local int32_t ip[kMaxBatch + 1], tp[kMaxBatch + 1];
   if (make_bwd_plan(cu_kept_host, batch, head_groups, sm_count(), plan, ip, tp) != TG_OK)
     return 0;
-  return bwd_layout(cu_kept_host[batch], n_q_heads, head_groups, plan).total;
+  return bwd_layout(n_q_heads, head_groups, plan).total;
 }
 
 extern "C" int tg_gated_attention_bias_grad(
@@ -584,7 +636,7 @@ extern "C" int tg_gated_attention_bias_grad(
   ReduceParams rp{};
   TG_TRY(make_bwd_plan(cu_kept_host, batch, head_groups, sm_count(), plan, rp.item_prefix,
                        rp.tile_prefix));
-  const BwdLayout lay = bwd_layout(k_total, n_q_heads, head_groups, plan);
+  const BwdLayout lay = bwd_layout(n_q_heads, head_groups, plan);
   if (lay.total > 0 && (!workspace || workspace_bytes < lay.total)) return TG_ERR_WORKSPACE;
   if (workspace && !aligned16(workspace)) return TG_ERR_MISALIGNED;
   unsigned char* ws = static_cast<unsigned char*>(workspace);
@@ -592,15 +644,27 @@ extern "C" int tg_gated_attention_bias_grad(
   float* tile_out = reinterpret_cast<float*>(ws + lay.tile_out);
 
   if (k_total > 0) {
-    float4* col_a = reinterpret_cast<float4*>(ws + lay.col_a);
-    float4* col_b = reinterpret_cast<float4*>(ws + lay.col_b);
-    const int64_t n = k_total * n_q_heads;
+    unsigned char* blocks = ws + lay.blocks;
+    PrepParams pp{};
+    pp.o = reinterpret_cast<const uint16_t*>(o);
+    pp.ld_o = ld_o;
+    pp.d_o = reinterpret_cast<const uint16_t*>(d_o);
+    pp.ld_do = ld_do;
+    pp.lse = lse;
+    pp.cu_kept = cu_kept;
+    pp.kept_pos = kept_pos;
+    pp.gamma = gamma;
+    pp.beta = beta;
+    pp.n_q_heads = n_q_heads;
+    pp.k_total = k_total;
+    pp.batch = batch;
+    pp.n_tiles = plan.n_tiles;
+    pp.blocks = blocks;
+    std::copy(rp.tile_prefix, rp.tile_prefix + kMaxBatch + 1, pp.tile_prefix);
+    const int64_t n = (int64_t)n_q_heads * plan.n_tiles * kTq;
     int64_t grid = (n + 255) / 256;
-    if (grid > 8 * (int64_t)sm_count()) grid = 8 * (int64_t)sm_count();
-    TG_TRY(launch(bwd_prep_kernel, dim3((unsigned)grid), dim3(256), 0, st,
-                  reinterpret_cast<const uint16_t*>(o), ld_o,
-                  reinterpret_cast<const uint16_t*>(d_o), ld_do, lse, cu_kept, batch, kept_pos,
-                  gamma, beta, n_q_heads, k_total, col_a, col_b));
+    if (grid > 16 * (int64_t)sm_count()) grid = 16 * (int64_t)sm_count();
+    TG_TRY(launch(bwd_prep_kernel, dim3((unsigned)grid), dim3(256), 0, st, pp));
 
     CUtensorMap tq, tk, tv, tdo;
     TG_TRY(make_tmap_bf16_2d(&tq, q, (uint64_t)k_total, (uint64_t)n_q_heads * kD, (uint64_t)ld_q,
@@ -614,10 +678,9 @@ extern "C" int tg_gated_attention_bias_grad(
     BwdParams bp{};
     bp.cu_kept = cu_kept;
     bp.kept_bias = kept_bias;
-    bp.col_a = col_a;
-    bp.col_b = col_b;
+    bp.blocks = blocks;
     bp.part = reinterpret_cast<float*>(ws + lay.part);
-    bp.k_total = k_total;
+    bp.n_tiles = plan.n_tiles;
     bp.group = group;
     bp.head_pairs = group / 2;
     bp.n_kv_heads = n_kv_heads;
@@ -625,6 +688,7 @@ extern "C" int tg_gated_attention_bias_grad(
     bp.chunk = plan.chunk;
     bp.status = status;
     std::copy(rp.item_prefix, rp.item_prefix + kMaxBatch + 1, bp.item_prefix);
+    std::copy(rp.tile_prefix, rp.tile_prefix + kMaxBatch + 1, bp.tile_prefix);
     const int64_t cta = (int64_t)plan.n_items * head_groups;
     if (cta > 0) {
       if (d_beta) {

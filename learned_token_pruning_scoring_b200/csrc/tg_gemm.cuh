@@ -32,7 +32,7 @@
 
 namespace tg {
 
-enum { EpiStore = 0, EpiScore = 1, EpiQKV = 2, EpiSwiGLU = 3 };
+enum { EpiStore = 0, EpiScore = 1, EpiQKV = 2, EpiSwiGLU = 3, EpiQKVNorm = 4 };
 
 struct GemmParams {
   int64_t M;
@@ -61,8 +61,8 @@ struct GemmParams {
   uint16_t* k_out;        // K rows: k_out + row * ld_kv (columns relative to q_cols)
   uint16_t* v_out;        // V rows: v_out + row * ld_kv (columns relative to q_cols + k_cols)
   int64_t ld_kv;
-  // EpiQKV, CTA-pair kernel only: optional QK-norm (per-head RMSNorm of the Q and K
-  // heads before RoPE, weights [128] shared by the heads)
+  // EpiQKVNorm (EpiQKV plus QK-norm, CTA-pair kernel only): per-head RMSNorm of the Q
+  // and K heads before RoPE, weights [128] shared by the heads
   const float* q_norm_w;
   const float* k_norm_w;
   float qk_eps;
@@ -401,7 +401,7 @@ __device__ __forceinline__ void pair_epilogue_half(const GemmParams& p, unsigned
   const bool live = grow < p.M;
   const float rscale =
       (p.rmsnorm && p.row_ssq_in && live) ? rscale_from_ssq(p, grow) : 1.0f;
-  if (EPI == EpiQKV) {
+  if (EPI == EpiQKV || EPI == EpiQKVNorm) {
     const bool rope = n0 < p.q_cols + p.k_cols;
     int pos = (rope && live) ? p.pos[grow] : 0;
     if (pos < 0 || pos >= p.max_pos) {
@@ -413,7 +413,7 @@ __device__ __forceinline__ void pair_epilogue_half(const GemmParams& p, unsigned
     // over them gives the head's RMS
     float qk = 1.f;
     const float* nw = nullptr;
-    if (rope && p.q_norm_w) {
+    if (EPI == EpiQKVNorm && rope) {
       nw = n0 < p.q_cols ? p.q_norm_w : p.k_norm_w;
       float ss = 0.f;
 #pragma unroll 1
@@ -449,7 +449,7 @@ __device__ __forceinline__ void pair_epilogue_half(const GemmParams& p, unsigned
           const int i = u * 8 + 2 * e;
           float x1a = __uint_as_float(ra[i]) * scale, x1b = __uint_as_float(ra[i + 1]) * scale;
           float x2a = __uint_as_float(rb[i]) * scale, x2b = __uint_as_float(rb[i + 1]) * scale;
-          if (nw) {  // head columns c and c + 64, c = 32 pr + i
+          if (EPI == EpiQKVNorm && nw) {  // head columns c and c + 64, c = 32 pr + i
             const int c = 32 * pr + i;
             x1a *= __ldg(nw + c);
             x1b *= __ldg(nw + c + 1);
@@ -790,7 +790,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(320, 1)
           mbar_arrive_cluster(acc_empty_lead0 + b * 8);
         int mi = 0, x = n0;
         const int epi = job ? EPI1 : EPI0;
-        if (epi == EpiQKV) {
+        if (epi == EpiQKV || epi == EpiQKVNorm) {
           if (n0 >= jb.p.q_cols + jb.p.k_cols) {
             mi = 2;
             x = n0 - jb.p.q_cols - jb.p.k_cols;

@@ -329,6 +329,7 @@ static int qkv_rope_cache_impl(const tg_bf16* x, int64_t ld_x, const tg_bf16* w_
     TG_TRY(qkv_job(j, x, ld_x, w_qkv, ld_w, M, hidden, q_cols, kv_cols, eps, pos, cos_sin, max_pos,
                    q_out, ld_q, cache_k, cache_v, ld_cache, slot_offset, row_ssq_in, ld_ssq_in,
                    status, q_norm_w, k_norm_w));
+    if (q_norm_w) return launch_pair<kPairStages, EpiQKVNorm>(j.maps, j.p, (cudaStream_t)stream);
     return launch_pair<kPairStages, EpiQKV>(j.maps, j.p, (cudaStream_t)stream);
   }
   int bn = pick_bn(M, N);
