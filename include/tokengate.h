@@ -339,7 +339,7 @@ size_t tg_gated_attention_workspace_size(const int32_t* cu_kept_host, int batch,
  * with P recomputed from q, k, the bias and lse exactly as the forward formed the logits.
  * d_bias is the gradient for kept_bias; the gradient of a prunable token's gate score z is
  * d_bias of its kept row (a question token has none).  Layouts, shapes and limits as
- * tg_gated_attention; d_o: bf16 [K_tot, n_q_heads * head_dim] (ld_do); lse: float32
+ * tg_gated_attention, and n_q_heads <= 64; d_o: bf16 [K_tot, n_q_heads * head_dim] (ld_do); lse: float32
  * [n_q_heads, K_tot] from that forward call.  workspace: at least
  * tg_gated_attention_bias_grad_workspace_size(...) bytes (no zero-fill needed; 16-byte
  * aligned).  tcgen05 kernel, one CTA per (request, 128-key tile, chunk of query tiles,

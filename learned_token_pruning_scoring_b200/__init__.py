@@ -620,6 +620,10 @@ class GatedPrefill:
         self.lower = lower
         self.trim_lower_kv = trim_lower_kv
         self.gate = gate
+        # the scorer's RMSNorm weight, folded into W1 once (the same bf16 products
+        # tg_gate_score would form on every call)
+        self._w1 = (tg_fold_norm_weight(gate["W1"], gate["norm_w"])
+                    if gate.get("norm_w") is not None else gate["W1"])
         self.layers = [prepare_layer(l) for l in layers]
         self.hq, self.hkv, self.d = n_q_heads, n_kv_heads, head_dim
         self.theta = rope_theta
@@ -700,7 +704,7 @@ class GatedPrefill:
     def score(self, h, prunable, stream=None):
         P = self.planned
         g = self.gate
-        tg_gate_score(h, g["W1"], g["w2"], P["cu"], P["cu_h"], prunable, norm_w=g.get("norm_w"),
+        tg_gate_score(h, self._w1, g["w2"], P["cu"], P["cu_h"], prunable, norm_w=None,
                       eps_norm=self.norm_eps, eps_seq=self.seq_eps, s_out=P["s"], z_out=P["z"],
                       bias_out=P["bias"], workspace=P["ws"], status=self.status, stream=stream)
         self._mark("gate_score")

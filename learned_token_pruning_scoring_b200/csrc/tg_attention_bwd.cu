@@ -88,12 +88,17 @@ struct BwdParams {
 
 __host__ __device__ __forceinline__ int cdiv(int a, int b) { return (a + b - 1) / b; }
 
-// Work items of a request are (key tile kt, query chunk ci) in kt-major order; key tile
-// kt has the chunks ci = kt / C .. n_chunks - 1.  Items before key tile kt:
-//   sum_{x < kt} (n_chunks - x / C) = kt n_chunks - (C q (q - 1) / 2 + q (kt mod C)), q = kt / C.
-__host__ __device__ __forceinline__ int items_before_tile(int kt, int n_chunks, int C) {
-  const int q = kt / C;
-  return kt * n_chunks - (C * q * (q - 1) / 2 + q * (kt % C));
+// Work items of a request are (query chunk ci, key tile kt) in ci-major order, so that
+// the CTAs running together read the same Q and dO tiles (L2 reuse).  Chunk ci covers
+// query tiles [ci C, (ci + 1) C) and pairs with the key tiles kt < min(nt, (ci + 1) C);
+// every chunk but the last is full, so the items before chunk ci number C ci (ci + 1) / 2.
+constexpr int kMaxChunk = 16;  // query tiles per item at most (Q/dO working set in L2)
+__host__ __device__ __forceinline__ int items_before_chunk(int ci, int C) {
+  return C * ci * (ci + 1) / 2;
+}
+__host__ __device__ __forceinline__ int items_in_request(int nt, int C) {
+  const int nch = (nt + C - 1) / C;
+  return nch ? items_before_chunk(nch - 1, C) + nt : 0;
 }
 
 __device__ __forceinline__ int find_request(const int32_t* prefix, int batch, int t) {
@@ -124,12 +129,16 @@ struct PrepParams {
   int32_t tile_prefix[kMaxBatch + 1];
 };
 
-// One thread per (q head, query tile, row of the tile): that row's entries of the block.
+// Four threads per (q head, query tile, row of the tile): each loads a quarter of the
+// row's dO and O (one batch of loads in flight), the quad sums delta, and its first
+// thread writes the row's entries of the block.
 __global__ void bwd_prep_kernel(const __grid_constant__ PrepParams p) {
   griddep_wait();
   const int64_t n = (int64_t)p.n_q_heads * p.n_tiles * kTq;
-  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n;
-       i += (int64_t)gridDim.x * blockDim.x) {
+  const int quad = threadIdx.x & 3;
+  const unsigned qmask = 0xFu << ((threadIdx.x & 31) & ~3u);
+  for (int64_t i = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 2; i < n;
+       i += ((int64_t)gridDim.x * blockDim.x) >> 2) {
     const int rr = (int)(i % kTq);
     const int64_t ht = i / kTq;  // h * n_tiles + tile
     const int h = (int)(ht / p.n_tiles);
@@ -137,20 +146,24 @@ __global__ void bwd_prep_kernel(const __grid_constant__ PrepParams p) {
     const int b = find_request(p.tile_prefix, p.batch, tile);
     const int r = (tile - p.tile_prefix[b]) * kTq + rr;
     const int n_b = p.cu_kept[b + 1] - p.cu_kept[b];
-    unsigned char* blk = p.blocks + ht * kBlockBytes;
-    float4 a = make_float4(0.f, INFINITY, 0.f, 0.f);
-    float u = 0.f, g = 0.f;
-    if (r < n_b) {
-      const int64_t row = p.cu_kept[b] + r;
-      const int pos = p.kept_pos[row];
-      // delta = dO_r . O_r over the head's 128 values
-      const uint4* x = reinterpret_cast<const uint4*>(p.d_o + row * p.ld_do + (int64_t)h * kD);
-      const uint4* y = reinterpret_cast<const uint4*>(p.o + row * p.ld_o + (int64_t)h * kD);
-      float delta = 0.f;
-#pragma unroll 4
-      for (int k = 0; k < kD / 8; ++k) {
-        const uint4 xv = x[k], yv = y[k];
-        const uint32_t xs[4] = {xv.x, xv.y, xv.z, xv.w}, ys[4] = {yv.x, yv.y, yv.z, yv.w};
+    const bool valid = r < n_b;  // the same for the four threads
+    const int64_t row = p.cu_kept[b] + r;
+    float delta = 0.f;
+    if (valid) {  // delta = dO_r . O_r over the head's 128 values, 32 per thread
+      const uint4* x = reinterpret_cast<const uint4*>(p.d_o + row * p.ld_do + (int64_t)h * kD) +
+                       quad * 4;
+      const uint4* y = reinterpret_cast<const uint4*>(p.o + row * p.ld_o + (int64_t)h * kD) +
+                       quad * 4;
+      uint4 xv[4], yv[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        xv[k] = x[k];
+        yv[k] = y[k];
+      }
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const uint32_t xs[4] = {xv[k].x, xv[k].y, xv[k].z, xv[k].w};
+        const uint32_t ys[4] = {yv[k].x, yv[k].y, yv[k].z, yv[k].w};
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const float2 fx = unpack_bf16x2(xs[e]), fy = unpack_bf16x2(ys[e]);
@@ -158,6 +171,15 @@ __global__ void bwd_prep_kernel(const __grid_constant__ PrepParams p) {
           delta = fmaf(fx.y, fy.y, delta);
         }
       }
+      delta += __shfl_xor_sync(qmask, delta, 1);
+      delta += __shfl_xor_sync(qmask, delta, 2);
+    }
+    if (quad != 0) continue;
+    unsigned char* blk = p.blocks + ht * kBlockBytes;
+    float4 a = make_float4(0.f, INFINITY, 0.f, 0.f);
+    float u = 0.f, g = 0.f;
+    if (valid) {
+      const int pos = p.kept_pos[row];
       const double tau = attn_tau(p.beta, r, pos);
       const float t = attn_logit_scale(tau, kD);
       g = p.gamma[h] * kAttnLog2e / t;
@@ -243,13 +265,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int64_t row0 = p.cu_kept[b];
   const int n_b = p.cu_kept[b + 1] - p.cu_kept[b];
   const int nt = cdiv(n_b, kTq);
-  const int n_chunks = cdiv(nt, p.chunk);
-  int idx = item - p.item_prefix[b], kt = 0;
-  while (idx >= n_chunks - kt / p.chunk) {
-    idx -= n_chunks - kt / p.chunk;
-    ++kt;
-  }
-  const int ci = kt / p.chunk + idx;
+  const int idx = item - p.item_prefix[b];
+  int ci = 0;
+  while (items_before_chunk(ci + 1, p.chunk) <= idx) ++ci;
+  const int kt = idx - items_before_chunk(ci, p.chunk);
   const int qt_begin = max(kt, ci * p.chunk);
   const int nq = min(nt, (ci + 1) * p.chunk) - qt_begin;  // query tiles of this item (>= 1)
   const int g = head_grp / p.head_pairs;
@@ -446,11 +465,15 @@ struct ReduceParams {
   int32_t tile_prefix[kMaxBatch + 1];
 };
 
-// One block of 128 threads per key tile: d_bias of its keys, and per head the tile's
-// sum of b_c * (sum over queries of dl), plus the tile's d_beta share, in fixed order.
-__global__ void __launch_bounds__(128)
+// One block per key tile, threads (key, head group): each thread sums its key's partials
+// of the two heads of its group over the tile's items (all these loads are independent),
+// then the block forms d_bias of its keys and, per head, the tile's sum of b_c * (sum
+// over queries of dl), plus the tile's d_beta share, all in a fixed order.
+constexpr int kReduceGroups = 8;  // blockDim.y
+__global__ void __launch_bounds__(128 * kReduceGroups)
     bias_grad_reduce_kernel(const __grid_constant__ ReduceParams p) {
-  extern __shared__ float red[];  // [n_q_heads + 1][128]
+  extern __shared__ float red[];  // [n_q_heads][128] sums per head, [kReduceGroups][128] d_beta
+  float* red_beta = red + p.n_q_heads * 128;
   griddep_wait();
   const int t = blockIdx.x;
   const int b = find_request(p.tile_prefix, p.batch, t);
@@ -458,34 +481,46 @@ __global__ void __launch_bounds__(128)
   const int64_t row0 = p.cu_kept[b];
   const int n_b = p.cu_kept[b + 1] - p.cu_kept[b];
   const int n_chunks = cdiv(cdiv(n_b, kTq), p.chunk);
-  const int first = p.item_prefix[b] + items_before_tile(kt, n_chunks, p.chunk);
-  const int n_items = n_chunks - kt / p.chunk;
   const int hg = p.n_kv_heads * p.head_pairs;
   const int key = threadIdx.x;
   const int c = kt * kTk + key;
   const bool valid = c < n_b;
-  const float b_c = valid ? p.kept_bias[row0 + c] : 0.f;
-  float db = 0.f, dbeta = 0.f;
-  for (int grp = 0; grp < hg; ++grp) {
+  float dbeta = 0.f;
+  for (int grp = threadIdx.y; grp < hg; grp += kReduceGroups) {
     const int h0 = (grp / p.head_pairs) * p.group + 2 * (grp % p.head_pairs);
-    for (int w = 0; w < 2; ++w) {
-      float a = 0.f, ab = 0.f;
-      for (int i = 0; i < n_items; ++i) {
-        const int64_t slot = (int64_t)(first + i) * hg + grp;
-        a += p.part[((slot * 2 + 0) * 2 + w) * 128 + key];
-        ab += p.part[((slot * 2 + 1) * 2 + w) * 128 + key];
-      }
-      db = fmaf(p.gamma[h0 + w], a, db);
-      dbeta += ab;
-      red[(h0 + w) * 128 + key] = valid ? b_c * a : 0.f;
+    float a0 = 0.f, a1 = 0.f;
+    for (int ci = kt / p.chunk; ci < n_chunks; ++ci) {  // the items of this key tile
+      const int item = p.item_prefix[b] + items_before_chunk(ci, p.chunk) + kt;
+      const float* pp = p.part + ((int64_t)item * hg + grp) * 512 + key;
+      a0 += pp[0];          // acc, head h0
+      a1 += pp[128];        // acc, head h0 + 1
+      dbeta += pp[256] + pp[384];
     }
+    red[h0 * 128 + key] = a0;
+    red[(h0 + 1) * 128 + key] = a1;
   }
-  red[p.n_q_heads * 128 + key] = valid ? dbeta : 0.f;
-  if (valid) p.d_bias[row0 + c] = db;
+  red_beta[threadIdx.y * 128 + key] = valid ? dbeta : 0.f;
   __syncthreads();
-  for (int h = threadIdx.x; h <= p.n_q_heads; h += blockDim.x) {
+  if (threadIdx.y == 0) {
+    const float b_c = valid ? p.kept_bias[row0 + c] : 0.f;
+    float db = 0.f;
+    for (int h = 0; h < p.n_q_heads; ++h) {
+      const float a = red[h * 128 + key];
+      db = fmaf(p.gamma[h], a, db);
+      red[h * 128 + key] = valid ? b_c * a : 0.f;
+    }
+    if (valid) p.d_bias[row0 + c] = db;
+  }
+  __syncthreads();
+  const int lin = threadIdx.y * 128 + threadIdx.x;
+  for (int h = lin; h <= p.n_q_heads; h += 128 * kReduceGroups) {
     float sum = 0.f;
-    for (int k = 0; k < 128; ++k) sum += red[h * 128 + k];
+    if (h < p.n_q_heads) {
+      for (int k = 0; k < 128; ++k) sum += red[h * 128 + k];
+    } else {
+      for (int y = 0; y < kReduceGroups; ++y)
+        for (int k = 0; k < 128; ++k) sum += red_beta[y * 128 + k];
+    }
     p.tile_out[(int64_t)t * (p.n_q_heads + 1) + h] = sum;
   }
 }
@@ -512,7 +547,8 @@ struct BwdPlan {
   int n_tiles = 0;
 };
 
-// Query tiles per work item: the largest chunk that still gives about two waves of CTAs.
+// Query tiles per work item: the largest chunk (at most kMaxChunk) that still gives
+// about two waves of CTAs.
 int make_bwd_plan(const int32_t* cu_kept_host, int batch, int head_groups, int sms,
                   BwdPlan& plan, int32_t* item_prefix, int32_t* tile_prefix) {
   int max_nt = 1;
@@ -524,20 +560,18 @@ int make_bwd_plan(const int32_t* cu_kept_host, int batch, int head_groups, int s
   }
   auto count = [&](int C) {
     int64_t items = 0;
-    for (int b = 0; b < batch; ++b) {
-      const int nt = cdiv(cu_kept_host[b + 1] - cu_kept_host[b], kTq);
-      if (nt) items += items_before_tile(nt, cdiv(nt, C), C);
-    }
+    for (int b = 0; b < batch; ++b)
+      items += items_in_request(cdiv(cu_kept_host[b + 1] - cu_kept_host[b], kTq), C);
     return items;
   };
-  int C = max_nt;
+  int C = std::min(max_nt, kMaxChunk);
   while (C > 1 && count(C) * head_groups < 2 * (int64_t)sms) --C;
   const int64_t items = count(C);
   if (items * head_groups > 0x7FFFFFFF) return TG_ERR_UNSUPPORTED_SHAPE;
   item_prefix[0] = 0;
   for (int b = 0; b < batch; ++b) {
     const int nt = cdiv(cu_kept_host[b + 1] - cu_kept_host[b], kTq);
-    item_prefix[b + 1] = item_prefix[b] + (nt ? items_before_tile(nt, cdiv(nt, C), C) : 0);
+    item_prefix[b + 1] = item_prefix[b] + items_in_request(nt, C);
   }
   plan.chunk = C;
   plan.n_items = (int)items;
@@ -564,7 +598,8 @@ int validate(const int32_t* cu_kept_host, int batch, int n_q_heads, int n_kv_hea
              int head_dim) {
   if (head_dim != kD) return TG_ERR_UNSUPPORTED_SHAPE;
   if (n_q_heads <= 0 || n_kv_heads <= 0 || n_q_heads % n_kv_heads) return TG_ERR_INVALID_ARGUMENT;
-  if ((n_q_heads / n_kv_heads) % 2 || n_q_heads > 1023) return TG_ERR_UNSUPPORTED_SHAPE;
+  // the reduction keeps one 128-key row per q head in shared memory (<= 36 KB)
+  if ((n_q_heads / n_kv_heads) % 2 || n_q_heads > 64) return TG_ERR_UNSUPPORTED_SHAPE;
   if (batch > kMaxBatch) return TG_ERR_UNSUPPORTED_SHAPE;
   if (batch < 0 || !cu_kept_host) return TG_ERR_INVALID_ARGUMENT;
   if (batch > 0 && cu_kept_host[0] != 0) return TG_ERR_INVALID_ARGUMENT;
@@ -661,7 +696,7 @@ extern "C" int tg_gated_attention_bias_grad(
     pp.n_tiles = plan.n_tiles;
     pp.blocks = blocks;
     std::copy(rp.tile_prefix, rp.tile_prefix + kMaxBatch + 1, pp.tile_prefix);
-    const int64_t n = (int64_t)n_q_heads * plan.n_tiles * kTq;
+    const int64_t n = (int64_t)n_q_heads * plan.n_tiles * kTq * 4;  // threads: four per row
     int64_t grid = (n + 255) / 256;
     if (grid > 16 * (int64_t)sm_count()) grid = 16 * (int64_t)sm_count();
     TG_TRY(launch(bwd_prep_kernel, dim3((unsigned)grid), dim3(256), 0, st, pp));
@@ -712,8 +747,9 @@ extern "C" int tg_gated_attention_bias_grad(
       rp.n_kv_heads = n_kv_heads;
       rp.batch = batch;
       rp.chunk = plan.chunk;
-      TG_TRY(launch(bias_grad_reduce_kernel, dim3((unsigned)plan.n_tiles), dim3(128),
-                    (size_t)(n_q_heads + 1) * 128 * sizeof(float), st, rp));
+      TG_TRY(launch(bias_grad_reduce_kernel, dim3((unsigned)plan.n_tiles),
+                    dim3(128, kReduceGroups),
+                    (size_t)(n_q_heads + kReduceGroups) * 128 * sizeof(float), st, rp));
     }
   }
   return launch(bias_grad_finish_kernel, dim3(1), dim3(std::min(1024, n_q_heads + 1)), 0, st,

@@ -1,6 +1,7 @@
 // Row gather with original-position RoPE, compacted KV-cache writes, and the rotary
 // table.  These are HBM-bound copies: one warp moves one row with 16-byte accesses,
-// all loads of a row issued before its stores, grid sized to fill every SM.
+// all loads of a row issued before its stores, as many warps resident per SM as the
+// kernel's registers allow.
 //
 // Sources: "TokenGate 长上下文预填充提速 11.3 倍，斯坦福伯克利开源门控剪枝", section
 // 门控到底插在模型的哪个位置 (pruned rows stop at the gate; only kept rows go up);
@@ -129,6 +130,30 @@ __device__ __forceinline__ void copy_row_ssq(const uint4* __restrict__ s, uint4*
   }
 }
 
+// Plain gather (no RoPE): one warp per row, optional per-128-column sums of squares.
+// Kept apart from the RoPE kernel so that its registers stay within 64 per thread and
+// four blocks (32 warps, 4 KB in flight each) fit on every SM.
+constexpr int kCopyBlocksPerSm = 4;
+__global__ void __launch_bounds__(kCopyWarps * 32, kCopyBlocksPerSm)
+    gather_copy_kernel(GatherArgs a) {
+  griddep_wait();
+  const int lane = threadIdx.x & 31;
+  const int64_t warp0 = (int64_t)blockIdx.x * kCopyWarps + (threadIdx.x >> 5);
+  const int64_t nwarps = (int64_t)gridDim.x * kCopyWarps;
+  const int nvec = a.width >> 3;
+  for (int64_t r = warp0; r < a.n_rows; r += nwarps) {
+    const int64_t sr = a.row_idx ? (int64_t)a.row_idx[r] : r;
+    if (sr < 0 || sr >= a.src_rows) {
+      if (lane == 0 && a.status) atomicOr(a.status, TG_STATUS_BOUNDS);
+      continue;
+    }
+    const uint4* s = reinterpret_cast<const uint4*>(a.src + sr * a.ld_src);
+    uint4* d = reinterpret_cast<uint4*>(a.dst + r * a.ld_dst);
+    if (a.row_ssq) copy_row_ssq(s, d, nvec, lane, a.row_ssq + r * a.ld_ssq);
+    else copy_row(s, d, 0, nvec, lane);
+  }
+}
+
 __global__ void __launch_bounds__(kCopyWarps * 32) gather_rope_kernel(GatherArgs a) {
   griddep_wait();
   const int lane = threadIdx.x & 31;
@@ -187,7 +212,7 @@ struct KvArgs {
   uint32_t* status;
 };
 
-__global__ void __launch_bounds__(kCopyWarps * 32) kv_compact_kernel(KvArgs a) {
+__global__ void __launch_bounds__(kCopyWarps * 32, kCopyBlocksPerSm) kv_compact_kernel(KvArgs a) {
   griddep_wait();
   const int lane = threadIdx.x & 31;
   const int64_t warp0 = (int64_t)blockIdx.x * kCopyWarps + (threadIdx.x >> 5);
@@ -207,9 +232,11 @@ __global__ void __launch_bounds__(kCopyWarps * 32) kv_compact_kernel(KvArgs a) {
   }
 }
 
-int copy_grid(int64_t rows) {
+// One warp per row, at most the blocks that are resident at once (the kernels stride
+// over the rest).
+int copy_grid(int64_t rows, int blocks_per_sm) {
   const int64_t want = (rows + kCopyWarps - 1) / kCopyWarps;
-  const int64_t cap = (int64_t)sm_count() * 8;  // 8 blocks x 8 warps = 64 warps per SM
+  const int64_t cap = (int64_t)sm_count() * blocks_per_sm;
   return (int)(want < cap ? (want < 1 ? 1 : want) : cap);
 }
 
@@ -258,7 +285,11 @@ extern "C" int tg_gather_rope(const tg_bf16* src, int64_t ld_src, int64_t src_ro
   GatherArgs a{reinterpret_cast<const uint16_t*>(src), ld_src, src_rows, row_idx, n_rows, width,
                rope_pos, rope_col_begin, rope_col_end, head_dim, cos_sin, max_pos,
                reinterpret_cast<uint16_t*>(dst), ld_dst, row_ssq_out, ld_ssq_out, status};
-  return launch(gather_rope_kernel, dim3(copy_grid(n_rows)), dim3(kCopyWarps * 32), 0,
+  if (!rope_pos || rope_col_begin >= rope_col_end)
+    return launch(gather_copy_kernel, dim3(copy_grid(n_rows, kCopyBlocksPerSm)),
+                  dim3(kCopyWarps * 32), 0, (cudaStream_t)stream, a);
+  // the RoPE kernel is register-heavy (one block per SM); it serves the unfused path
+  return launch(gather_rope_kernel, dim3(copy_grid(n_rows, 1)), dim3(kCopyWarps * 32), 0,
                 (cudaStream_t)stream, a);
 }
 
@@ -281,6 +312,6 @@ extern "C" int tg_kv_compact(const tg_bf16* k, int64_t ld_k, const tg_bf16* v, i
   KvArgs a{reinterpret_cast<const uint16_t*>(k), ld_k, reinterpret_cast<const uint16_t*>(v), ld_v,
            src_rows, row_idx, n_rows, width, reinterpret_cast<uint16_t*>(cache_k),
            reinterpret_cast<uint16_t*>(cache_v), ld_cache, slot_offset, status};
-  return launch(kv_compact_kernel, dim3(copy_grid(2 * n_rows)), dim3(kCopyWarps * 32), 0,
-                (cudaStream_t)stream, a);
+  return launch(kv_compact_kernel, dim3(copy_grid(2 * n_rows, kCopyBlocksPerSm)),
+                dim3(kCopyWarps * 32), 0, (cudaStream_t)stream, a);
 }
