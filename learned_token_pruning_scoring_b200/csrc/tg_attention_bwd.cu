@@ -23,10 +23,11 @@
 // lse2_r, delta_r = dO_r.O_r, and the temperature-gradient factors), with lse2 = +inf
 // on rows past the request so that they contribute nothing; one bulk copy brings it in.
 // Q and dO stages are freed by the MMAs that read them (so the next tile's loads overlap
-// the compute warps), the blocks by the compute warps through a deeper ring.  Partial sums per (work item, head, key) go to the workspace and
-// two small kernels reduce them in a fixed order (deterministic results).
-// Warps: 0 producer (K, V once; per query tile and head Q, dO by TMA plus the scalars and
-// the gain operand), 1 MMA issuer, 2-5 head h0, 6-9 head h0 + 1.
+// the compute warps), the blocks by the compute warps through a deeper ring.  Partial
+// sums per (work item, head, key) go to the workspace and two small kernels reduce them
+// in a fixed order (deterministic results).
+// Warps: 0 producer (K, V and the key-bias operand once; per query tile and head Q and
+// dO by TMA and the block by a bulk copy), 1 MMA issuer, 2-5 head h0, 6-9 head h0 + 1.
 #include <cuda.h>
 
 #include <algorithm>
