@@ -90,6 +90,32 @@ def workload(name):
     return table[name]
 
 
+# ------------------------------------------------------------------ replicas (N > 1)
+
+def replica_workload(wl, rank, world):
+    """Rank r's own batch: the same shapes and weights, request seeds offset by 1000 r (no
+    data is shared between ranks: the path shards by request, replicas only)."""
+    if world <= 1:
+        return wl
+    import synthetic_inputs as S
+    return S.Workload(**{**wl.__dict__, "seeds": tuple(s + 1000 * rank for s in wl.seeds)})
+
+
+def max_over_ranks(ms, world, device):
+    """The slowest rank's time (every rank takes this collective step, in the same order)."""
+    if world <= 1:
+        return ms
+    import torch
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(tokens_per_step, world, steps, total_ms):
+    """Tokens/s of the whole job: every rank's tokens over the slowest rank's time."""
+    return tokens_per_step * world * steps / (total_ms / 1e3)
+
+
 # ------------------------------------------------------------------ algorithmic work
 
 def stage_work(wl, kept_counts, ffn=0):
@@ -207,8 +233,7 @@ def run_ours(args, rank, world):
     dev = torch.device("cuda", torch.cuda.current_device())
     wl = workload(args.workload)
     # replicas: rank r draws its own batch (seed offset), same weights
-    if world > 1:
-        wl = S.Workload(**{**wl.__dict__, "seeds": tuple(s + 1000 * rank for s in wl.seeds)})
+    wl = replica_workload(wl, rank, world)
     h = S.hidden_rows(wl)
     pr = S.prunable_mask(wl)
     gate = {k: v.to(dev) for k, v in S.gate_weights(wl).items()}
@@ -340,11 +365,8 @@ def run_ours(args, rank, world):
             run_step_plain()
     torch.cuda.synchronize()
     gpu_launches = launches_per_step * args.steps
-    total_ms = sum(step_ms)
+    total_ms = max_over_ranks(sum(step_ms), world, dev)
     if world > 1:
-        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        total_ms = float(t.item())
         torch.distributed.barrier()
     # per-stage breakdown (second timed loop, same step with stage events)
     for _ in range(args.steps):
@@ -354,7 +376,7 @@ def run_ours(args, rank, world):
         raise SystemExit(f"device status {status:#x} after timed steps")
 
     tokens_per_step = wl.total_tokens
-    value = tokens_per_step * world * args.steps / (total_ms / 1e3)
+    value = whole_job_rate(tokens_per_step, world, args.steps, total_ms)
 
     # ---- end to end through the public API: host inputs in, result out, per step
     h_pin = h.pin_memory()
@@ -378,12 +400,8 @@ def run_ours(args, rank, world):
         torch.cuda.synchronize()
         if i:  # first one is a warm-up of the copy path
             e2e_ms.append(e0.elapsed_time(e1))
-    e2e_total = sum(e2e_ms)
-    if world > 1:
-        t = torch.tensor([e2e_total], dtype=torch.float64, device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        e2e_total = float(t.item())
-    e2e_value = tokens_per_step * world * len(e2e_ms) / (e2e_total / 1e3)
+    e2e_total = max_over_ranks(sum(e2e_ms), world, dev)
+    e2e_value = whole_job_rate(tokens_per_step, world, len(e2e_ms), e2e_total)
     h2d = h.numel() * h.element_size() + pr.numel() * pr.element_size()
     d2h = x_host.numel() * x_host.element_size()
 
