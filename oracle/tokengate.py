@@ -52,7 +52,7 @@ __all__ = [
     "select_topk", "gather_rows", "rope", "rope_angles", "temperature",
     "gated_attention", "kv_compact", "gated_layer", "prefill", "silu",
     "request_positions", "causal_attention", "full_context_layer",
-    "rmsnorm_heads", "swiglu_mlp", "gated_attention_bias_grad",
+    "rmsnorm_heads", "swiglu_mlp", "gated_attention_bias_grad", "gate_score_backward",
 ]
 
 
@@ -334,6 +334,49 @@ def gated_attention_bias_grad(Q, K, V, dO, cu_kept, kept_pos, kept_bias, gamma, 
             d_gamma[h] += np.sum(dl * bias[None, lo:hi])
             d_beta += np.sum(dl * rho[:, None] * s)
     return d_bias, d_gamma, d_beta
+
+
+def gate_score_backward(h, norm_w, W1, w2, cu_seqlens, prunable, kept_idx, d_kept_bias,
+                        eps_norm: float = 1e-6, eps_seq: float = 1e-6):
+    """Gradients of the gate's parameters from dL/d(kept_bias), the other half of training
+    the gate end to end ([fluxbbs] 端到端训练的关键在 token 门控注意力).
+
+    kept_bias[r] = z[kept_idx[r]] on prunable rows (0 on question rows); the top-K choice
+    itself is piecewise constant and passes no gradient.  With z = s / rms_b over the
+    request, s_t = sum_f w2_f SiLU(u_tf), u_t = W1 (n_t * norm_w), n_t = h_t / rms(h_t):
+        ds_t = (dz_t - z_t mean_b(dz z)) / rms_b
+        dw2_f = sum_t ds_t SiLU(u_tf);  du_tf = ds_t w2_f SiLU'(u_tf)
+        dW1 = sum_t du_t (n_t * norm_w)^T;  d norm_w_k = sum_t n_tk sum_f du_tf W1_fk
+    with SiLU'(u) = sig(u) (1 + u (1 - sig(u))).  Returns a dict of dz, ds, dw2, dW1,
+    dnorm_w (float64)."""
+    h = as_f64(h)
+    W1 = as_f64(W1)
+    w2 = as_f64(w2)
+    w = np.ones(h.shape[1]) if norm_w is None else as_f64(norm_w)
+    cu = _as_int(cu_seqlens)
+    pr = _as_int(prunable)
+    n = h / np.sqrt(np.mean(h * h, axis=1, keepdims=True) + eps_norm)
+    xh = n * w[None, :]
+    u = xh @ W1.T
+    sig = 1.0 / (1.0 + np.exp(-u))
+    s = (u * sig) @ w2
+    dz = np.zeros(h.shape[0])
+    idx = _as_int(kept_idx)
+    dz[idx] = as_f64(d_kept_bias) * (pr[idx] != 0)
+    ds = np.zeros_like(dz)
+    for b in range(len(cu) - 1):
+        lo, hi = cu[b], cu[b + 1]
+        if hi == lo:
+            continue
+        rms = math.sqrt(float(np.mean(s[lo:hi] ** 2)) + eps_seq)
+        z = s[lo:hi] / rms
+        ds[lo:hi] = (dz[lo:hi] - z * np.mean(dz[lo:hi] * z)) / rms
+    dsilu = sig * (1.0 + u * (1.0 - sig))
+    dw2 = (u * sig).T @ ds
+    du = ds[:, None] * w2[None, :] * dsilu
+    dW1 = du.T @ xh
+    dnorm_w = np.sum(n * (du @ W1), axis=0)
+    return {"dz": dz, "ds": ds, "dw2": dw2, "dW1": dW1, "dnorm_w": dnorm_w}
 
 
 def kv_compact(K, V, row_idx=None):

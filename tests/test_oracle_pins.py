@@ -646,3 +646,40 @@ def test_bias_grad_finite_differences_and_invariants():
     # gamma = 0 leaves the bias gradient zero; the first row of a request (one key) has none
     db0, _, _ = O.gated_attention_bias_grad(Q, K, V, dO, cu, pos, bias, np.zeros(4), 0.9)
     np.testing.assert_allclose(db0, 0.0, atol=0)
+
+
+def test_gate_score_backward_against_autograd():
+    """Scorer parameter gradients from dL/d(kept_bias), against torch.autograd through
+    RMSNorm -> MLP -> sequence RMSNorm -> kept bias written directly in torch."""
+    rng = np.random.default_rng(90)
+    lens = [13, 1, 9]
+    cu = np.concatenate([[0], np.cumsum(lens)])
+    T, H, Fw = int(cu[-1]), 16, 6
+    h = rng.normal(size=(T, H))
+    W1 = rng.normal(size=(Fw, H)) * 0.5
+    w2 = rng.normal(size=Fw)
+    nw = rng.uniform(0.8, 1.2, size=H)
+    pr = (rng.random(T) < 0.7).astype(np.uint8)
+    kept = np.sort(rng.choice(T, size=12, replace=False))
+    g = rng.normal(size=len(kept))
+    th, tW1 = torch.tensor(h), torch.tensor(W1, requires_grad=True)
+    tw2, tnw = torch.tensor(w2, requires_grad=True), torch.tensor(nw, requires_grad=True)
+    x = F.rms_norm(th, (H,), tnw, eps=1e-6)
+    s = F.silu(x @ tW1.T) @ tw2
+    z = torch.cat([s[cu[b]:cu[b + 1]] / torch.sqrt(torch.mean(s[cu[b]:cu[b + 1]] ** 2) + 1e-6)
+                   for b in range(3)])
+    bias = z * torch.tensor(pr, dtype=torch.float64)
+    (bias[torch.tensor(kept)] * torch.tensor(g)).sum().backward()
+    out = O.gate_score_backward(h, nw, W1, w2, cu, pr, kept, g)
+    np.testing.assert_allclose(out["dW1"], tW1.grad.numpy(), atol=1e-10)
+    np.testing.assert_allclose(out["dw2"], tw2.grad.numpy(), atol=1e-10)
+    np.testing.assert_allclose(out["dnorm_w"], tnw.grad.numpy(), atol=1e-10)
+    # question tokens and pruned tokens receive no dz
+    dz = out["dz"]
+    assert np.all(dz[pr == 0] == 0)
+    assert np.all(dz[np.setdiff1d(np.arange(T), kept)] == 0)
+    # the sequence norm makes z scale-free: ds is orthogonal to s within each request
+    s_np = O.gate_score(h, nw, W1, w2)
+    for b in range(3):
+        lo, hi = cu[b], cu[b + 1]
+        assert abs(np.dot(out["ds"][lo:hi], s_np[lo:hi])) < 1e-6 * (1 + np.abs(s_np[lo:hi]).sum())
