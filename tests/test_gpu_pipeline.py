@@ -205,6 +205,63 @@ def test_pipeline_n128k_planted_cluster(tg):
     assert tg.tg_status_read(pipe.status) == 0
 
 
+@pytest.mark.parametrize("make", [(lambda r=r: S.n32k_sweep(r)) for r in S.N32K_RATIOS]
+                         + [S.ragged8],
+                         ids=[f"n32k_r{r:g}" for r in S.N32K_RATIOS] + ["ragged8"])
+def test_pipeline_keep_ratio_sweep_and_ragged8(tg, make):
+    """N=32768 at keep ratios 1%, 5%, 25% and 100% (the dense point: gamma 0, beta 1, every
+    token kept, so tau is exactly 1), and 8 packed requests of 4k-32k tokens with their own
+    budgets: scores, selection, and the first layer's attention output and residual on
+    sampled query rows (the first and last row of every request among them)."""
+    wl = make()
+    h, gate, layers, pr, pipe = _setup(tg, wl)
+    hd, prd = h.cuda(), pr.cuda()
+    pipe.score(hd, prd)
+    pipe.select(prd)
+    pipe.gather(hd)
+    pipe.layer(0)
+    torch.cuda.synchronize()
+    P = pipe.planned
+    cu = wl.cu_seqlens()
+    s_ref = O.gate_score(h, gate["norm_w"], gate["W1"], gate["w2"])
+    z_ref, _ = O.sequence_rmsnorm(s_ref, cu, pr)
+    z = P["z"].cpu().double().numpy()
+    assert np.abs(z - z_ref).max() <= 1e-2 and np.abs(z - z_ref).mean() <= 1e-3
+    ck = O.kept_counts(pr, cu, wl.budgets)
+    same = _check_selection(wl, pr.numpy(), z_ref, ck, P["kept_idx"].cpu().numpy(),
+                            P["ck_h"].numpy())
+    if same:
+        idx_ref, pos_ref, bias_ref = O.select_topk(z_ref.astype(np.float32), pr, cu, ck)
+        assert np.array_equal(P["kept_pos"].cpu().numpy(), pos_ref)
+        x0 = O.gather_rows(h, idx_ref)
+        L = layers[0]
+        a = O.rmsnorm_rows(x0)
+        qkv = a @ O.as_f64(L["Wqkv"]).T
+        Kt = x0.shape[0]
+        hq, hkv, d = wl.n_q_heads, wl.n_kv_heads, wl.head_dim
+        q = O.rope(qkv[:, :hq * d].reshape(Kt, hq, d), pos_ref, wl.rope_theta)
+        k = O.rope(qkv[:, hq * d:(hq + hkv) * d].reshape(Kt, hkv, d), pos_ref, wl.rope_theta)
+        v = qkv[:, (hq + hkv) * d:].reshape(Kt, hkv, d)
+        rng = np.random.default_rng(5)
+        rows = []
+        for b in range(wl.batch):
+            lo, hi = int(ck[b]), int(ck[b + 1])
+            if hi > lo:
+                rows += [lo, hi - 1] + rng.integers(lo, hi, 24).tolist()
+        qrows = np.unique(np.array(rows, dtype=np.int64))
+        o_ref, _ = O.gated_attention(q, k, v, ck, pos_ref, bias_ref, L["gamma"], L["beta"],
+                                     rows=qrows)
+        o_gpu = O.as_f64(P["o"].cpu()).reshape(Kt, hq, d)
+        err = np.abs(o_gpu[qrows] - o_ref[qrows])
+        assert err.max() <= 2e-2 and err.mean() <= 1e-3, (err.max(), err.mean())
+        # the residual after the output projection, on the same rows
+        x_ref = x0[qrows] + o_ref[qrows].reshape(len(qrows), hq * d) @ O.as_f64(L["Wo"]).T
+        x_err = np.abs(O.as_f64(P["x"].cpu())[qrows] - x_ref)
+        tol, tol_mean = _x_tol(x_ref, 1)
+        assert np.all(x_err <= tol) and x_err.mean() <= tol_mean, (x_err.max(), x_err.mean())
+    assert tg.tg_status_read(pipe.status) == 0
+
+
 def test_launch_overlap_gives_identical_results(tg):
     """Programmatic dependent launch changes only when kernels are scheduled: a step run
     eagerly and replayed from a CUDA graph with the overlap on must match, bit for bit,
