@@ -360,6 +360,44 @@ size_t tg_gated_attention_bias_grad_workspace_size(const int32_t* cu_kept_host, 
                                                    int n_q_heads, int n_kv_heads,
                                                    int head_dim);
 
+/*
+ * Backward of the gate's scorer: its parameter gradients from dL/d(kept_bias), the
+ * gradient tg_gated_attention_bias_grad returns ([fluxbbs] 端到端训练的关键在 token 门控注意力:
+ * the gate is trained end to end through the gated attention; [fluxbbs] 门控到底插在模型的
+ * 哪个位置: the scorer and the sequence RMSNorm it differentiates).  The top-K choice is
+ * piecewise constant and passes no gradient.  With r_t = 1/sqrt(mean(h_t^2) + eps_norm),
+ * u_t = W1 (r_t h_t * norm_w), z_t = s_t / rms_b over request b:
+ *   dz_t   = d_kept_bias[r] where t = kept_idx[r] is prunable, else 0
+ *   ds_t   = (dz_t - z_t m_b) / rms_b,  m_b = mean over the request of dz z
+ *   dw2_f  = sum_t ds_t SiLU(u_tf)
+ *   dW1[f, i]  = norm_w_i sum_t ds_t w2_f SiLU'(u_tf) r_t h_ti
+ *   dnorm_w_i  = sum_f W1[f, i] sum_t ds_t w2_f SiLU'(u_tf) r_t h_ti
+ * h, ld_h, total_tokens, hidden, norm_w (NULL = ones), W1, width, w2, eps_norm,
+ * cu_seqlens(_host), batch, eps_seq, prunable: as tg_gate_score (hidden a multiple of
+ * 128, width 256).  s: float32 [total_tokens], the s_out of tg_gate_score on the same
+ * inputs.  cu_kept / cu_kept_host: int32 [batch+1] (K_b <= N_b); kept_idx: int32
+ * [K_tot] distinct rows of their request, as tg_topk_compact writes them;
+ * d_kept_bias: float32 [K_tot].  Outputs (float32, overwritten): ds_out [total_tokens],
+ * dW1 [width, hidden] (row stride hidden), dw2 [width], dnorm_w [hidden] (may be NULL).
+ * workspace: tg_gate_score_backward_workspace_size(...) bytes, 16-byte aligned, no
+ * zero-fill needed.  The scorer GEMM runs again on tcgen05 with a gradient epilogue
+ * (bf16 r_t du_t); the weight gradient h^T (r du) runs on tcgen05 with both operands
+ * MN-major, split over tokens; every reduction has a fixed order (bit-reproducible).
+ * A kept index outside its request sets TG_STATUS_BOUNDS and is skipped; bounded waits
+ * set TG_STATUS_TIMEOUT.  total_tokens = 0 writes zero gradients.  status may be NULL.
+ */
+int tg_gate_score_backward(const tg_bf16* h, int64_t ld_h, int64_t total_tokens, int hidden,
+                           const float* norm_w, const tg_bf16* W1, int width, const float* w2,
+                           float eps_norm, const float* s, const int32_t* cu_seqlens,
+                           const int32_t* cu_seqlens_host, int batch, float eps_seq,
+                           const uint8_t* prunable, const int32_t* cu_kept,
+                           const int32_t* cu_kept_host, const int32_t* kept_idx,
+                           const float* d_kept_bias, float* ds_out, float* dW1,
+                           float* dnorm_w, float* dw2, void* workspace,
+                           size_t workspace_bytes, uint32_t* status, tg_stream_t stream);
+size_t tg_gate_score_backward_workspace_size(int64_t total_tokens, int hidden, int width,
+                                             int batch);
+
 /* ------------------------------------------------------------------ projections */
 
 /*

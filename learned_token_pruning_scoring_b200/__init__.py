@@ -29,6 +29,7 @@ __all__ = [
     "tg_prefetch_l2", "tg_out_proj_qkv_next", "tg_out_proj_qkv_workspace_size",
     "tg_swiglu", "tg_fold_norm_weight", "tg_pack_gate_up", "prepare_layer",
     "tg_gated_attention_bias_grad", "tg_gated_attention_bias_grad_workspace_size",
+    "tg_gate_score_backward", "tg_gate_score_backward_workspace_size",
     "GatedPrefill", "FullContextLayers", "LayerWeights", "STATUS_TIMEOUT", "STATUS_BUDGET",
     "STATUS_BOUNDS", "STATUS_WORKSPACE",
 ]
@@ -329,6 +330,44 @@ def tg_gated_attention_bias_grad(q, k, v, o, d_o, lse, cu_kept, cu_kept_host, n_
     _count(4 if int(ckh[-1]) > 0 else 1)
     return d_bias
 
+
+
+def tg_gate_score_backward_workspace_size(total_tokens, hidden, width, batch):
+    return int(lib.tg_gate_score_backward_workspace_size(int(total_tokens), int(hidden),
+                                                         int(width), int(batch)))
+
+
+def tg_gate_score_backward(h, W1, w2, s, cu_seqlens, cu_seqlens_host, prunable, cu_kept,
+                           cu_kept_host, kept_idx, d_kept_bias, norm_w=None, eps_norm=1e-6,
+                           eps_seq=1e-6, ds_out=None, dW1=None, dnorm_w=None, dw2=None,
+                           workspace=None, status=None, stream=None):
+    """Scorer parameter gradients from dL/d(kept_bias): returns (ds, dW1, dw2, dnorm_w);
+    dnorm_w is computed when norm_w is given or dnorm_w is passed in.  `s` is the s_out
+    of tg_gate_score on the same inputs."""
+    ld_h = _mat(h, "h")
+    T, hidden = h.shape
+    width = W1.shape[0]
+    cuh, ckh = _host_i32(cu_seqlens_host), _host_i32(cu_kept_host)
+    batch = cuh.numel() - 1
+    dev = h.device
+    ds_out = torch.empty(T, dtype=torch.float32, device=dev) if ds_out is None else ds_out
+    dW1 = torch.empty((width, hidden), dtype=torch.float32, device=dev) if dW1 is None else dW1
+    dw2 = torch.empty(width, dtype=torch.float32, device=dev) if dw2 is None else dw2
+    if dnorm_w is None and norm_w is not None:
+        dnorm_w = torch.empty(hidden, dtype=torch.float32, device=dev)
+    if workspace is None:
+        need = tg_gate_score_backward_workspace_size(T, hidden, width, batch)
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+    rc = lib.tg_gate_score_backward(
+        _ptr(h), ld_h, T, hidden, _ptr(norm_w), _ptr(W1), width, _ptr(w2), float(eps_norm),
+        _ptr(s), _ptr(cu_seqlens), _ptr(cuh), batch, float(eps_seq), _ptr(prunable),
+        _ptr(cu_kept), _ptr(ckh), _ptr(kept_idx), _ptr(d_kept_bias), _ptr(ds_out), _ptr(dW1),
+        _ptr(dnorm_w), _ptr(dw2), _ptr(workspace), workspace.numel(), _ptr(status),
+        _stream(stream))
+    _check(rc, "tg_gate_score_backward")
+    if T > 0:
+        _count(6 + (1 if int(ckh[-1]) > 0 else 0) + (1 if norm_w is not None else 0))
+    return ds_out, dW1, dw2, dnorm_w
 
 def tg_linear(a, w, c=None, rmsnorm=False, eps=1e-6, residual=None, row_ssq=None, status=None,
               stream=None):

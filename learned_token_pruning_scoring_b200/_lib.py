@@ -53,6 +53,10 @@ SIGNATURES = {
                                             _p, _p, _p, _i32, _i32, _i32, _i32, _p, _p, _p,
                                             _f32, _p, _p, _p, _p, _sz, _p, _p]),
     "tg_gated_attention_bias_grad_workspace_size": (_sz, [_p, _i32, _i32, _i32, _i32]),
+    "tg_gate_score_backward": (_i32, [_p, _i64, _i64, _i32, _p, _p, _i32, _p, _f32, _p, _p, _p,
+                                      _i32, _f32, _p, _p, _p, _p, _p, _p, _p, _p, _p, _p, _sz,
+                                      _p, _p]),
+    "tg_gate_score_backward_workspace_size": (_sz, [_i64, _i32, _i32, _i32]),
     "tg_swiglu": (_i32, [_p, _i64, _p, _i64, _i64, _i32, _i32, _f32, _p, _i64, _p, _i64, _p,
                          _p]),
     "tg_fold_norm_weight": (_i32, [_p, _i64, _i64, _i32, _p, _p, _i64, _p]),

@@ -174,3 +174,29 @@ def test_bias_grad_argument_checks(lib):
     assert call(beta=-1.0) == -1
     assert call(d_bias=None) == -1
     assert lib.tg_gated_attention_bias_grad_workspace_size(ck, 1, 16, 8, 64) == 0
+
+
+def test_scorer_backward_argument_checks(lib):
+    p = C.c_void_p(0x10000)
+    cu = (C.c_int32 * 3)(0, 300, 500)
+    ck = (C.c_int32 * 3)(0, 30, 50)
+
+    def call(hidden=2048, width=256, cu_h=cu, ck_h=ck, batch=2, T=500, dW1=p, dw2=p,
+             eps=1e-6):
+        return lib.tg_gate_score_backward(p, hidden, T, hidden, None, p, width, p, eps, p, p,
+                                          cu_h, batch, 1e-6, p, p, ck_h, p, p, p, dW1, None,
+                                          dw2, p, 1 << 30, None, None)
+    assert call(width=128) == -6
+    assert call(hidden=2112) == -6                          # not a multiple of 128
+    assert call(T=499) == -1                                # cu_seqlens[batch] != T
+    assert call(ck_h=(C.c_int32 * 3)(0, 301, 320)) == -1    # K_0 > N_0
+    assert call(ck_h=(C.c_int32 * 3)(0, 30, 20)) == -1      # decreasing
+    assert call(cu_h=None) == -1
+    assert call(eps=-1.0) == -1
+    assert call(dW1=None) == -1 and call(dw2=None) == -1
+    assert call(batch=0, T=5) == -1
+    assert lib.tg_gate_score_backward_workspace_size(500, 2048, 128, 2) == 0
+    small = lib.tg_gate_score_backward_workspace_size(500, 2048, 256, 2)
+    big = lib.tg_gate_score_backward_workspace_size(50000, 2048, 256, 2)
+    # du' alone is 512 bytes per token
+    assert small > 500 * 512 and big - small >= (50000 - 500) * 512

@@ -118,10 +118,45 @@ def study_full(wl, n_layers):
               f"|x|max {np.abs(x64).max():.2f}", flush=True)
 
 
+def study_scorer_backward(wl, seed=91):
+    """Scorer parameter gradients, float64 against the CUDA path's rounding: W1 folded
+    with the norm weight and rounded to bf16 for the recomputed u, and the row-scaled
+    du rounded to bf16 before it meets h in the weight-gradient GEMM."""
+    h, pr, gate = S.hidden_rows(wl), S.prunable_mask(wl), S.gate_weights(wl)
+    g = torch.Generator().manual_seed(seed)
+    nw = (0.8 + 0.4 * torch.rand(wl.hidden, generator=g, dtype=torch.float64)).numpy()
+    cu = wl.cu_seqlens()
+    W1, w2 = O.as_f64(gate["W1"]), O.as_f64(gate["w2"])
+    s = O.gate_score(h, nw, W1, w2)
+    z, _ = O.sequence_rmsnorm(s, cu, pr)
+    ck = O.kept_counts(pr, cu, wl.budgets)
+    kept, _, _ = O.select_topk(z.astype(np.float32), pr, cu, ck)
+    dkb = torch.randn(len(kept), generator=g, dtype=torch.float64).numpy()
+    ref = O.gate_score_backward(h, nw, W1, w2, cu, pr, kept, dkb)
+    hh = O.as_f64(h)
+    r = 1.0 / np.sqrt(np.mean(hh * hh, axis=1) + 1e-6)
+    u = (hh @ bf16(W1 * nw[None, :]).T) * r[:, None]
+    sig = 1.0 / (1.0 + np.exp(-u))
+    du = bf16(r[:, None] * ref["ds"][:, None] * w2[None, :] * sig * (1.0 + u * (1.0 - sig)))
+    M = hh.T @ du                                   # [H, F]
+    got = {"dW1": (M * nw[:, None]).T, "dnorm_w": np.sum(W1.T * M, axis=1),
+           "dw2": (u * sig).T @ ref["ds"]}
+    for k, v in got.items():
+        e = np.abs(v - ref[k])
+        scale = np.abs(ref[k]).max()
+        print(f"{wl.name} {k}: max {e.max():.3e} mean {e.mean():.3e} |ref|max {scale:.3e} "
+              f"max/|ref|max {e.max() / scale:.3e}", flush=True)
+
+
 if __name__ == "__main__":
     if len(sys.argv) > 1 and sys.argv[1] == "full":
         study_full(S.custom([700, 1500, 333], [16, 64, 5], [100, 800, 300], n_layers=2,
                             name="ragged3"), 2)
+        sys.exit(0)
+    if len(sys.argv) > 1 and sys.argv[1] == "scorer_bwd":
+        study_scorer_backward(S.custom([700, 1500, 333], [16, 64, 5], [100, 800, 300],
+                                       name="ragged3"))
+        study_scorer_backward(S.n16k())
         sys.exit(0)
     if len(sys.argv) > 1 and sys.argv[1] == "lower":
         study_lower(S.custom([700, 1500, 333], [16, 64, 5], [100, 800, 300], n_layers=1,
