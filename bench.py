@@ -67,6 +67,9 @@ def parse_args():
                          "6144) instead of attention-only layers")
     ap.add_argument("--bias-grad-steps", type=int, default=10,
                     help="timed calls of the attention backward w.r.t. the gate (0 skips it)")
+    ap.add_argument("--scorer-bwd-steps", type=int, default=0,
+                    help="timed calls of the scorer backward (parameter gradients from a "
+                         "seeded d kept_bias; 0 skips it)")
     ap.add_argument("--dense-steps", type=int, default=3,
                     help="timed steps of the full-context reference (0 skips it)")
     return ap.parse_args()
@@ -514,6 +517,9 @@ def run_ours(args, rank, world):
     if args.bias_grad_steps > 0 and int(P["K"]) > 0:
         out["bias_grad"] = bias_grad_timing(tg, wl, P, pipe, flush, stream,
                                             args.bias_grad_steps, peaks)
+    if args.scorer_bwd_steps > 0 and int(P["K"]) > 0:
+        out["scorer_bwd"] = scorer_bwd_timing(tg, wl, P, pipe, h_dev, pr_dev, flush, stream,
+                                              args.scorer_bwd_steps, peaks)
     if args.dense_steps > 0:
         out["dense_reference"] = dense_reference(tg, wl, layers, h_dev, flush, stream,
                                                  args.dense_steps, peaks,
@@ -575,6 +581,60 @@ def bias_grad_timing(tg, wl, P, pipe, flush, stream, steps, peaks):
             "kept": K, "calls": steps, "avg_ms": avg, "achieved": tf, "unit": "TFLOP/s",
             "peak": peak, "frac": tf / peak,
             "flops_counted": "S^T = K Q^T and dP^T = V dO^T over the causal pairs"}
+
+
+def scorer_bwd_timing(tg, wl, P, pipe, h_dev, pr_dev, flush, stream, steps, peaks):
+    """The scorer's backward (ds, dW1, dw2, d norm_w) from a seeded d kept_bias on the kept
+    set of the step just run: CUDA events around each call, L2 flushed before each.  Its
+    work is the scorer GEMM twice (the recompute and the weight gradient, 2THF flops
+    each) with h streamed twice and r*du written and read once."""
+    import torch
+    dev = h_dev.device
+    K = int(P["K"])
+    g = torch.Generator(device="cpu").manual_seed(19)
+    dkb = torch.randn(K, generator=g).to(dev)
+    W1, w2, nw = pipe.gate["W1"], pipe.gate["w2"], pipe.gate.get("norm_w")
+    T, H = h_dev.shape
+    F = W1.shape[0]
+    ds = torch.empty(T, dtype=torch.float32, device=dev)
+    dW1 = torch.empty((F, H), dtype=torch.float32, device=dev)
+    dw2 = torch.empty(F, dtype=torch.float32, device=dev)
+    dnw = torch.empty(H, dtype=torch.float32, device=dev)
+    ws = torch.empty(max(16, tg.tg_gate_score_backward_workspace_size(T, H, F, wl.batch)),
+                     dtype=torch.uint8, device=dev)
+
+    def call():
+        tg.tg_gate_score_backward(h_dev, W1, w2, P["s"], P["cu"], P["cu_h"], pr_dev, P["ck"],
+                                  P["ck_h"], P["kept_idx"], dkb, norm_w=nw, ds_out=ds, dW1=dW1,
+                                  dnorm_w=dnw, dw2=dw2, workspace=ws, status=pipe.status)
+    for _ in range(3):
+        call()
+    torch.cuda.synchronize()
+    ms = []
+    for _ in range(steps):
+        flush.fill_(1.0)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        call()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ms.append(e0.elapsed_time(e1))
+    status = tg.tg_status_read(pipe.status)
+    if status:
+        raise SystemExit(f"device status {status:#x} in the scorer backward")
+    avg = sum(ms) / len(ms)
+    flops = 4 * T * H * F
+    nbytes = 2 * (2 * T * H) + 2 * (2 * T * F) + 2 * F * H
+    tf = flops / (avg / 1e3) / 1e12
+    gbs = nbytes / (avg / 1e3) / 1e9
+    floor_ms = max(flops / (peaks["bf16_tflops"] * 1e12), nbytes / (peaks["hbm_gbs"] * 1e9)) * 1e3
+    return {"what": "ds, dW1, dw2, d norm_w of the scorer from a seeded d kept_bias "
+                    "(ds kernels + scorer GEMM with gradient epilogue + weight-gradient "
+                    "GEMM + reductions)",
+            "tokens": T, "calls": steps, "avg_ms": avg, "tflops": tf, "gbs": gbs,
+            "floor_ms": floor_ms, "frac_of_floor": floor_ms / avg,
+            "counted": "4THF flops; h read twice, r*du written and read, W1 once"}
 
 
 def dense_reference(tg, wl, layers, h_dev, flush, stream, steps, peaks, gated_ms):
