@@ -20,7 +20,7 @@
 //      in every CTA of the request), then ds_t = -z_t m_b / rms_b on every row;
 //   2. scatter: ds_t += dz_t / rms_b on the kept prunable rows (distinct rows);
 //   3. the scorer GEMM again (tcgen05, the row RMS from the A stages as in the forward)
-//      with the EpiScoreGrad epilogue: du'_t = r_t du_t as bf16 [T, 256] and per-32-row
+//      with a gradient epilogue: du'_t = r_t du_t as bf16 [T, 256] and per-32-row
 //      column sums of ds_t SiLU(u_tf);
 //   4. weight gradient M = h^T du' on tcgen05, both operands MN-major (the tokens, the
 //      contraction index, are the rows of h and du'), one 128-feature tile of M per CTA
@@ -33,21 +33,27 @@
 // Every reduction runs in a fixed order, so the results are bit-reproducible.
 #include <cstdint>
 
-#include "tg_gemm.cuh"
 #include "tg_host.h"
+#include "tg_ptx.cuh"
 
 namespace tg {
-
-template <int BN, int STAGES, int EPI>
-int launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const GemmParams& p,
-                cudaStream_t stream);
-
 namespace {
 
 constexpr int kWidth = 256;
 constexpr int kPrepThreads = 256;
 constexpr int kPrepRowsPerCta = 8192;
 constexpr int kScatterThreads = 256;
+
+// recompute GEMM (u = W1' h_t per 128-row tile, all 256 scorer features)
+constexpr int kGgBM = 128;
+constexpr int kGgBK = 64;
+constexpr int kGgStages = 4;
+constexpr int kGgABytes = kGgBM * kGgBK * 2;             // 16 KB
+constexpr int kGgBBytes = kWidth * kGgBK * 2;            // 32 KB
+constexpr int kGgStageBytes = kGgABytes + kGgBBytes;
+constexpr int kGgBarBytes = 256;
+constexpr int kGgSmem = 1024 + kGgStages * kGgStageBytes + kGgBarBytes + kWidth * 4;
+constexpr int kGgThreads = 192;
 
 // weight-gradient GEMM tiles
 constexpr int kWgBM = 128;                          // hidden features per CTA (MMA M)
@@ -128,6 +134,196 @@ __global__ void __launch_bounds__(kScatterThreads)
   const int64_t t = kept_idx[r];
   if (t < cu[b] || t >= cu[b + 1]) return;  // reported by the prep kernel
   if (prunable[t]) ds[t] += d_kept_bias[r] / rms[b];
+}
+
+struct GradGemmParams {
+  int64_t M;          // tokens
+  int K;              // hidden
+  float eps;          // of the row RMSNorm
+  const float* w2;    // [256]
+  const float* ds;    // [M]
+  uint16_t* du;       // [M, 256] bf16: r_t ds_t w2_f SiLU'(u_tf)
+  float* chunks;      // [ceil(M / 32), 256]: sum over each 32-row chunk of ds_t SiLU(u_tf)
+  uint32_t* status;
+};
+
+// Sum over the warp's 32 lanes of each of 32 per-lane values, by recursive halving:
+// at offset o every lane keeps half of its values and adds the partner's copy of that
+// half, so after offsets 16, 8, 4, 2, 1 lane l holds the total of value l.  31 shuffles,
+// and the order of the additions is fixed.
+__device__ __forceinline__ float warp_transpose_sum(float (&v)[32], int lane) {
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) {
+    const bool upper = (lane & o) != 0;
+#pragma unroll
+    for (int i = 0; i < o; ++i) {
+      const float send = upper ? v[i] : v[i + o];
+      const float keep = upper ? v[i + o] : v[i];
+      v[i] = keep + __shfl_xor_sync(0xFFFFFFFFu, send, o);
+    }
+  }
+  return v[0];
+}
+
+// The scorer GEMM of the forward (one CTA per 128 token rows, N = 256, K = hidden in
+// 64-column k-blocks through a 4-stage TMA ring, 128-byte swizzle, K-major operands)
+// with its gradient epilogue.  Roles: warp 0 lane 0 loads the h and W1' k-blocks;
+// warp 1 owns TMEM and lane 0 issues the MMAs (M = 128, N = 256, K = 16); warps 2-5
+// read every A stage for the row sums of squares (a stage is released by the MMA
+// commit plus these four warps), then each thread takes one row of the accumulator:
+// u = r acc, du' = r ds w2 SiLU'(u) stored as bf16, and the warp's column sums of
+// ds SiLU(u) over its 32 rows.  Rows past M come from the TMA's zero fill with ds = 0.
+__global__ void __launch_bounds__(kGgThreads, 1)
+    score_grad_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
+                           const __grid_constant__ CUtensorMap tmB, GradGemmParams p) {
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  unsigned char* smem = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  unsigned char* tiles = smem;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kGgStages * kGgStageBytes);
+  uint64_t* empty = full + kGgStages;
+  uint64_t* acc_full = empty + kGgStages;
+  uint64_t* drain = acc_full + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  float* w2s = reinterpret_cast<float*>(smem + kGgStages * kGgStageBytes + kGgBarBytes);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int64_t m0 = (int64_t)blockIdx.x * kGgBM;
+  const int nk = p.K / kGgBK;
+
+  if (tid == 0) {
+    for (int s = 0; s < kGgStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1 + 4);  // the MMA commit and the four norm warps
+    }
+    mbar_init(acc_full, 1);
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, kWidth);
+    tmem_relinquish();
+  }
+  griddep_wait();  // ds comes from the grid before this one
+  for (int i = tid; i < kWidth; i += kGgThreads) w2s[i] = p.w2[i];
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int issued = 0;
+      for (int kb = 0; kb < nk; ++kb) {
+        const int s = kb % kGgStages;
+        const uint32_t ph = (uint32_t)(kb / kGgStages) & 1u;
+        if (!mbar_wait(&empty[s], ph ^ 1u, abort_flag, p.status)) break;
+        unsigned char* a_s = tiles + s * kGgStageBytes;
+        mbar_arrive_expect_tx(&full[s], kGgStageBytes);
+        tma_load_2d(a_s, &tmA, kb * kGgBK, (int32_t)m0, &full[s]);
+        tma_load_2d(a_s + kGgABytes, &tmB, kb * kGgBK, 0, &full[s]);
+        ++issued;
+      }
+      // never leave the CTA with bulk copies still landing in its shared memory
+      for (int kb = issued - kGgStages < 0 ? 0 : issued - kGgStages; kb < issued; ++kb)
+        mbar_wait(&full[kb % kGgStages], (uint32_t)(kb / kGgStages) & 1u, nullptr, p.status);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16_f32(kGgBM, kWidth, false, false);
+      for (int kb = 0; kb < nk; ++kb) {
+        const int s = kb % kGgStages;
+        const uint32_t ph = (uint32_t)(kb / kGgStages) & 1u;
+        if (!mbar_wait(&full[s], ph, abort_flag, p.status)) break;
+        tc_fence_after();
+        const uint32_t a_addr = smem_u32(tiles + s * kGgStageBytes);
+        const uint32_t b_addr = a_addr + kGgABytes;
+#pragma unroll
+        for (int k = 0; k < kGgBK / 16; ++k)
+          mma_ss(tmem, sw128_desc(a_addr + k * 32, 16, 1024),
+                 sw128_desc(b_addr + k * 32, 16, 1024), idesc, (kb | k) != 0);
+        mma_commit(&empty[s]);
+      }
+      mma_commit(acc_full);
+      mma_commit(drain);
+      mbar_wait(drain, 0, nullptr, p.status);  // all MMAs retired before TMEM is freed
+    }
+  } else {
+    const int q = warp & 3;  // TMEM lane quarter this warp may access
+    const int row = q * 32 + lane;
+    const int64_t grow = m0 + row;
+    const bool live = grow < p.M;
+    float ss = 0.f;
+    for (int kb = 0; kb < nk; ++kb) {
+      const int s = kb % kGgStages;
+      const uint32_t ph = (uint32_t)(kb / kGgStages) & 1u;
+      if (!warp_all(mbar_wait(&full[s], ph, abort_flag, p.status))) break;
+      const unsigned char* rowp = tiles + s * kGgStageBytes + row * 128;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        // the row's eight 16-byte chunks, XOR-ordered so a quarter-warp hits distinct banks
+        const uint4 v = *reinterpret_cast<const uint4*>(rowp + ((j ^ (row & 7)) << 4));
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 f = unpack_bf16x2(w[e]);
+          ss = fmaf(f.x, f.x, ss);
+          ss = fmaf(f.y, f.y, ss);
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[s]);
+    }
+    const float rscale = rsqrtf(ss / (float)p.K + p.eps);
+    const bool ok = warp_all(mbar_wait(acc_full, 0, abort_flag, p.status));
+    tc_fence_after();
+    if (ok) {
+      const uint32_t tbase = tmem + ((uint32_t)(q * 32) << 16);
+      const int64_t chunk_row = m0 + q * 32;  // first row of this warp's 32-row chunk
+      const float dsr = live ? p.ds[grow] : 0.f;
+      const float g = dsr * rscale;
+#pragma unroll 1
+      for (int c = 0; c < kWidth / 32; ++c) {
+        uint32_t r[32];
+        tmem_ld32(tbase + c * 32, r);
+        tmem_wait_ld();
+        float a[32];
+        uint32_t w[16];
+#pragma unroll
+        for (int i = 0; i < 32; i += 2) {
+          float d2[2];
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const float u = __uint_as_float(r[i + e]) * rscale;
+            const float sg = 1.0f / (1.0f + __expf(-u));
+            a[i + e] = dsr * (u * sg);
+            d2[e] = g * w2s[c * 32 + i + e] * (sg * (1.0f + u * (1.0f - sg)));
+          }
+          w[i >> 1] = pack_bf16x2(d2[0], d2[1]);
+        }
+        if (live) {
+          uint4* dp = reinterpret_cast<uint4*>(p.du + grow * kWidth + c * 32);
+#pragma unroll
+          for (int u = 0; u < 4; ++u)
+            dp[u] = make_uint4(w[4 * u], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]);
+        }
+        const float col = warp_transpose_sum(a, lane);
+        if (chunk_row < p.M) p.chunks[(chunk_row >> 5) * (int64_t)kWidth + c * 32 + lane] = col;
+      }
+    }
+    tc_fence_before();
+  }
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kWidth);
+  }
 }
 
 // M partials: CTA (x, y) accumulates features i0 = 128 x .. i0 + 127 against all 256
@@ -426,19 +622,27 @@ extern "C" int tg_gate_score_backward(
                            128));
   TG_TRY(make_tmap_bf16_2d(&tb, wmat, (uint64_t)kWidth, (uint64_t)hidden, (uint64_t)hidden, 64,
                            256));
-  GemmParams p{};
-  p.M = total_tokens;
-  p.N = kWidth;
-  p.K = hidden;
-  p.rmsnorm = 1;
-  p.eps = eps_norm;
-  p.w2 = w2;
-  p.c = du;
-  p.ldc = kWidth;
-  p.ds_in = ds_out;
-  p.partial = chunks;
-  p.status = status;
-  TG_TRY((launch_gemm<256, 4, EpiScoreGrad>(ta, tb, p, st)));
+  GradGemmParams gp{};
+  gp.M = total_tokens;
+  gp.K = hidden;
+  gp.eps = eps_norm;
+  gp.w2 = w2;
+  gp.ds = ds_out;
+  gp.du = du;
+  gp.chunks = chunks;
+  gp.status = status;
+  int dev = 0;
+  TG_CUDA_TRY(cudaGetDevice(&dev));
+  static int attr_dev = -1;
+  if (attr_dev != dev) {
+    TG_CUDA_TRY(cudaFuncSetAttribute(score_grad_gemm_kernel,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, kGgSmem));
+    TG_CUDA_TRY(cudaFuncSetAttribute(score_wgrad_kernel,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, kWgSmem));
+    attr_dev = dev;
+  }
+  TG_TRY(launch(score_grad_gemm_kernel, dim3((unsigned)((total_tokens + kGgBM - 1) / kGgBM)),
+                dim3(kGgThreads), kGgSmem, st, ta, tb, gp));
 
   // 4: M = h^T du' in token slices
   int steps = 0, per = 0, slices = 0;
@@ -448,14 +652,6 @@ extern "C" int tg_gate_score_backward(
                            kWgBK));
   TG_TRY(make_tmap_bf16_2d(&tu, du, (uint64_t)total_tokens, (uint64_t)kWidth, (uint64_t)kWidth,
                            64, kWgBK));
-  static int attr_dev = -1;
-  int dev = 0;
-  TG_CUDA_TRY(cudaGetDevice(&dev));
-  if (attr_dev != dev) {
-    TG_CUDA_TRY(cudaFuncSetAttribute(score_wgrad_kernel,
-                                     cudaFuncAttributeMaxDynamicSharedMemorySize, kWgSmem));
-    attr_dev = dev;
-  }
   TG_TRY(launch(score_wgrad_kernel, dim3((unsigned)(hidden / kWgBM), (unsigned)slices),
                 dim3(kWgThreads), kWgSmem, st, th, tu, per, steps, hidden, partial, status));
 

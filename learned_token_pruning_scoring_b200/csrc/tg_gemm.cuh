@@ -22,10 +22,7 @@
 // to s = sum_f w2[f] SiLU(r * acc[f]) and per-32-row partial sums of s^2; EpiQKV
 // applies rotate-half RoPE at the row's position to the Q and K heads (pairs of
 // columns 64 apart, from TMEM chunks c and c + 2) and routes Q, K and V tiles to their
-// destinations (Q rows and the K and V rows of a compacted cache); EpiScoreGrad is the
-// scorer's backward on the recomputed pre-activation u = r * acc: it stores
-// du'[f] = r * ds * w2[f] * SiLU'(u[f]) as bf16 (the row scale r folded in for the weight
-// gradient that follows) and per-32-row column sums of ds * SiLU(u[f]) for dw2.
+// destinations (Q rows and the K and V rows of a compacted cache).
 #pragma once
 #include <cuda.h>
 
@@ -35,7 +32,7 @@
 
 namespace tg {
 
-enum { EpiStore = 0, EpiScore = 1, EpiQKV = 2, EpiSwiGLU = 3, EpiQKVNorm = 4, EpiScoreGrad = 5 };
+enum { EpiStore = 0, EpiScore = 1, EpiQKV = 2, EpiSwiGLU = 3, EpiQKVNorm = 4 };
 
 struct GemmParams {
   int64_t M;
@@ -55,9 +52,7 @@ struct GemmParams {
   // EpiScore
   const float* w2;
   float* s_out;
-  float* partial;  // [ceil(M / 32)]; EpiScoreGrad: [ceil(M / 32), BN] column sums
-  // EpiScoreGrad (du' goes to c / ldc)
-  const float* ds_in;  // [M] dL/ds
+  float* partial;  // [ceil(M / 32)]
   // EpiQKV
   const int32_t* pos;     // [M] rotary position of each row
   const float* cos_sin;   // [max_pos, head_dim / 2, 2]
@@ -95,24 +90,6 @@ __device__ __forceinline__ float rscale_from_ssq(const GemmParams& p, int64_t gr
   return rsqrtf(t / (float)p.K + p.eps);
 }
 
-// Sum over the warp's 32 lanes of each of 32 per-lane values, by recursive halving:
-// at offset o every lane keeps half of its values and adds the partner's copy of that
-// half, so after offsets 16, 8, 4, 2, 1 lane l holds the total of value l.  31 shuffles,
-// and the order of the additions is fixed.
-__device__ __forceinline__ float warp_transpose_sum(float (&v)[32], int lane) {
-#pragma unroll
-  for (int o = 16; o >= 1; o >>= 1) {
-    const bool upper = (lane & o) != 0;
-#pragma unroll
-    for (int i = 0; i < o; ++i) {
-      const float send = upper ? v[i] : v[i + o];
-      const float keep = upper ? v[i + o] : v[i];
-      v[i] = keep + __shfl_xor_sync(0xFFFFFFFFu, send, o);
-    }
-  }
-  return v[0];
-}
-
 // Epilogue of one output row held by this thread: BN accumulator columns at TMEM
 // address `tbase` (the warp's lane quarter), output columns n0 .. n0 + BN.  All lanes
 // of the warp must call it (tcgen05.ld is warp-collective).  Returns the row's score
@@ -122,41 +99,6 @@ __device__ __forceinline__ float epilogue_row(const GemmParams& p, uint32_t tbas
                                               int n0, float rscale, const float* w2s) {
   const bool live = grow < p.M;
   float score = 0.f;
-  if (EPI == EpiScoreGrad) {
-    // rows past M come from the TMA's zero fill and carry ds = 0: they add nothing
-    const int lane = (int)(threadIdx.x & 31);
-    const int64_t chunk_row = grow - lane;  // first row of this warp's 32-row chunk
-    const float dsr = live ? p.ds_in[grow] : 0.f;
-    const float g = dsr * rscale;
-#pragma unroll 1
-    for (int c = 0; c < BN / 32; ++c) {
-      uint32_t r[32];
-      tmem_ld32(tbase + c * 32, r);
-      tmem_wait_ld();
-      float a[32];
-      uint32_t w[16];
-#pragma unroll
-      for (int i = 0; i < 32; i += 2) {
-        float d2[2];
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const float u = __uint_as_float(r[i + e]) * rscale;
-          const float sg = 1.0f / (1.0f + __expf(-u));
-          a[i + e] = dsr * (u * sg);
-          d2[e] = g * w2s[c * 32 + i + e] * (sg * (1.0f + u * (1.0f - sg)));
-        }
-        w[i >> 1] = pack_bf16x2(d2[0], d2[1]);
-      }
-      if (live) {
-        uint4* dp = reinterpret_cast<uint4*>(p.c + grow * p.ldc + n0 + c * 32);
-#pragma unroll
-        for (int u = 0; u < 4; ++u) dp[u] = make_uint4(w[4 * u], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]);
-      }
-      const float col = warp_transpose_sum(a, lane);
-      if (chunk_row < p.M) p.partial[(chunk_row >> 5) * (int64_t)BN + c * 32 + lane] = col;
-    }
-    return 0.f;
-  }
   if (EPI == EpiQKV) {
     // destination of this tile: Q, K or V (tiles never straddle the boundaries)
     uint16_t* dst;
@@ -316,7 +258,7 @@ __global__ void __launch_bounds__(192, 1)
     tmem_relinquish();
   }
   griddep_wait();  // operands and outputs may belong to earlier grids
-  if (EPI == EpiScore || EPI == EpiScoreGrad) {
+  if (EPI == EpiScore) {
     for (int i = tid; i < BN; i += Cfg::THREADS) w2s[i] = p.w2[n0 + i];
   }
   tc_fence_before();

@@ -89,8 +89,6 @@ template int launch_gemm<128, 3, EpiStore>(const CUtensorMap&, const CUtensorMap
                                            const GemmParams&, cudaStream_t);
 template int launch_gemm<256, 4, EpiScore>(const CUtensorMap&, const CUtensorMap&,
                                            const GemmParams&, cudaStream_t);
-template int launch_gemm<256, 4, EpiScoreGrad>(const CUtensorMap&, const CUtensorMap&,
-                                               const GemmParams&, cudaStream_t);
 template int launch_gemm<256, 4, EpiQKV>(const CUtensorMap&, const CUtensorMap&,
                                          const GemmParams&, cudaStream_t);
 template int launch_gemm<128, 3, EpiQKV>(const CUtensorMap&, const CUtensorMap&,
