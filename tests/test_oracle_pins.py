@@ -683,3 +683,45 @@ def test_gate_score_backward_against_autograd():
     for b in range(3):
         lo, hi = cu[b], cu[b + 1]
         assert abs(np.dot(out["ds"][lo:hi], s_np[lo:hi])) < 1e-6 * (1 + np.abs(s_np[lo:hi]).sum())
+
+
+def test_gate_score_backward_finite_differences_and_scale_invariance():
+    """Central differences of the oracle's own forward (scores -> sequence RMSNorm ->
+    kept bias) for entries of W1, w2 and the norm weight; and, as z does not change when
+    w2 is scaled (eps aside), the w2 gradient is orthogonal to w2."""
+    rng = np.random.default_rng(92)
+    lens = [11, 6]
+    cu = np.concatenate([[0], np.cumsum(lens)])
+    T, H, Fw = int(cu[-1]), 12, 5
+    h = rng.normal(size=(T, H))
+    W1 = rng.normal(size=(Fw, H)) * 0.6
+    w2 = rng.normal(size=Fw)
+    nw = rng.uniform(0.8, 1.2, size=H)
+    pr = np.ones(T, dtype=np.uint8)
+    pr[[4, 10, 16]] = 0
+    kept = np.array([0, 2, 4, 7, 9, 10, 12, 13, 16])
+    g = rng.normal(size=len(kept))
+
+    def loss(W1_=W1, w2_=w2, nw_=nw):
+        s = O.gate_score(h, nw_, W1_, w2_)
+        _, bias = O.sequence_rmsnorm(s, cu, pr)
+        return float(np.dot(bias[kept], g))
+    out = O.gate_score_backward(h, nw, W1, w2, cu, pr, kept, g)
+    eps = 1e-6
+    for f, i in ((0, 0), (2, 7), (4, 11)):
+        e = np.zeros_like(W1)
+        e[f, i] = eps
+        fd = (loss(W1_=W1 + e) - loss(W1_=W1 - e)) / (2 * eps)
+        assert abs(fd - out["dW1"][f, i]) < 1e-7 * (1 + abs(fd))
+    for f in (1, 3):
+        e = np.zeros_like(w2)
+        e[f] = eps
+        fd = (loss(w2_=w2 + e) - loss(w2_=w2 - e)) / (2 * eps)
+        assert abs(fd - out["dw2"][f]) < 1e-7 * (1 + abs(fd))
+    for i in (0, 5):
+        e = np.zeros_like(nw)
+        e[i] = eps
+        fd = (loss(nw_=nw + e) - loss(nw_=nw - e)) / (2 * eps)
+        assert abs(fd - out["dnorm_w"][i]) < 1e-7 * (1 + abs(fd))
+    # z(c w2) = z(w2) up to eps_seq: d/dc L(c w2) at c = 1 is w2 . dw2 ~ 0
+    assert abs(np.dot(w2, out["dw2"])) < 1e-4 * np.abs(w2).dot(np.abs(out["dw2"]))
