@@ -57,6 +57,8 @@ extern "C" int tg_gate_score_noalloc(const tg_bf16* h, int64_t ld_h, int64_t tot
                                      int batch, float eps_seq, const uint8_t* prunable,
                                      float* s_out, float* z_out, float* bias_out,
                                      uint32_t* status, tg_stream_t stream) {
+  // shapes tg_gate_score rejects get its error code, not the scratch limit
+  if (width != 256 || hidden <= 0 || (hidden % 64)) return TG_ERR_UNSUPPORTED_SHAPE;
   if (total_tokens > TG_NOALLOC_MAX_TOKENS || hidden > TG_NOALLOC_MAX_HIDDEN)
     return TG_ERR_SCRATCH_LIMIT;
   const size_t need = tg_gate_score_workspace_size(total_tokens, hidden, width, batch);

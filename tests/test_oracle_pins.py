@@ -368,6 +368,35 @@ def test_layer_zero_output_projection_keeps_residual():
     np.testing.assert_allclose(v, vv, atol=1e-12)
 
 
+def test_layer_output_projection_against_torch():
+    """x + Wo . O with H != Hq d and a non-zero Wo: with gamma = 0, beta = 1 and positions
+    equal to ranks the layer is a plain pre-norm causal GQA layer, written here with
+    torch's rms_norm, linear and scaled_dot_product_attention (heads concatenated in head
+    order before Wo, the usual layout).  A transposed or wrongly reshaped O, or Wo used
+    transposed, fails this."""
+    import torch
+    import torch.nn.functional as F
+    rng = np.random.default_rng(7)
+    Hq, Hkv, d, H, T = 2, 1, 12, 16, 9
+    x = rng.normal(size=(T, H))
+    Wqkv = rng.normal(size=((Hq + 2 * Hkv) * d, H)) * 0.3
+    Wo = rng.normal(size=(H, Hq * d)) * 0.3
+    pos = np.arange(T)
+    x2, _, _, _ = O.gated_layer(x, Wqkv, Wo, np.zeros(Hq), 1.0, [0, T], pos, np.zeros(T),
+                                Hq, Hkv, d, 1e4)
+    xt = torch.from_numpy(x)
+    qkv = F.linear(F.rms_norm(xt, (H,), eps=1e-6), torch.from_numpy(Wqkv))
+    q = torch.from_numpy(O.rope(qkv[:, :Hq * d].reshape(T, Hq, d).numpy(), pos, 1e4))
+    k = torch.from_numpy(O.rope(qkv[:, Hq * d:(Hq + Hkv) * d].reshape(T, Hkv, d).numpy(),
+                                pos, 1e4))
+    v = qkv[:, (Hq + Hkv) * d:].reshape(T, Hkv, d)
+    heads = lambda t, rep: t.permute(1, 0, 2).repeat_interleave(rep, 0)[None]
+    o = F.scaled_dot_product_attention(heads(q, 1), heads(k, Hq // Hkv), heads(v, Hq // Hkv),
+                                       is_causal=True)[0]
+    want = xt + F.linear(o.permute(1, 0, 2).reshape(T, Hq * d), torch.from_numpy(Wo))
+    np.testing.assert_allclose(x2, want.numpy(), atol=1e-10)
+
+
 def test_prefill_tiny_pipeline_consistency():
     import synthetic_inputs as S
     wl = S.custom([40, 24], [4, 6], [10, 12], n_layers=1, hidden=32, scorer_width=8,
