@@ -21,6 +21,8 @@ between two CUDA events; L2 is flushed (a 512 MiB write) before every timed step
 the events.  SM clocks and throttle reasons are sampled through NVML during that loop.  A
 second loop of K replays of the same step captured with timing events at every stage
 boundary gives the per-stage times (and the roofline of the dominant kernel).
+Workloads named by `--also` (default: the 128k one) are measured the same way after
+the main one and reported under "workloads" in the same line.
 
 Alongside (`--dense-steps`, default 3): the same layer stack over every token with no
 gate (K = N, gamma = 0, tau = 1) on the same kernels, the GPU's own full-context
@@ -67,9 +69,12 @@ def parse_args():
                          "6144) instead of attention-only layers")
     ap.add_argument("--bias-grad-steps", type=int, default=10,
                     help="timed calls of the attention backward w.r.t. the gate (0 skips it)")
-    ap.add_argument("--scorer-bwd-steps", type=int, default=0,
+    ap.add_argument("--scorer-bwd-steps", type=int, default=5,
                     help="timed calls of the scorer backward (parameter gradients from a "
                          "seeded d kept_bias; 0 skips it)")
+    ap.add_argument("--also", default="n128k",
+                    help="comma-separated workloads measured after the main one and "
+                         "reported as sub-records of the same line ('' for none)")
     ap.add_argument("--dense-steps", type=int, default=3,
                     help="timed steps of the full-context reference (0 skips it)")
     return ap.parse_args()
@@ -162,6 +167,62 @@ def stage_work(wl, kept_counts, ffn=0):
     }
 
 
+def kept_total(wl):
+    """Total kept rows from the budgets (the same host rule as the library's planner:
+    K_b = Q_b + min(D_b, max(0, budget_b - Q_b)))."""
+    k = 0
+    for n, q, b in zip(wl.lengths, wl.questions, wl.budgets):
+        k += q + min(n - q, max(0, b - q))
+    return k
+
+
+def config_dict(wl, args, world):
+    """The `config` of the JSON line, the same for both arms."""
+    return {"workload": wl.name, "batch": wl.batch,
+            "tokens_per_request": list(wl.lengths) if wl.batch <= 8 else None,
+            "question_tokens": list(wl.questions) if wl.batch <= 8 else None,
+            "kept": kept_total(wl), "gated_layers": wl.n_layers,
+            "lower_layers": args.lower_layers,
+            "layer_body": "full (QK-norm, SwiGLU 6144)" if args.full_layers
+            else "attention only",
+            "hidden": wl.hidden, "heads": f"{wl.n_q_heads}q/{wl.n_kv_heads}kv x {wl.head_dim}",
+            "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+            "l2": "flushed before every timed step (512 MiB write, outside the timing)",
+            "launch": "cuda_graph" if args.launch == "graph" else "eager"}
+
+
+def topk_latency_floor(tg, dev, stream, flush, reps=20):
+    """Average time of one tg_topk_compact call on a single 64-token request (32 prunable,
+    32 kept): the select's fixed dependent chain (cluster launch, three radix passes and
+    the compaction, each with a cluster-wide exchange) with almost no keys to count."""
+    import torch
+    z = torch.linspace(-1, 1, 64, device=dev)
+    pr = torch.ones(64, dtype=torch.uint8, device=dev)
+    pr[32:] = 0
+    cu_h = torch.tensor([0, 64], dtype=torch.int32)
+    ck_h = torch.tensor([0, 48], dtype=torch.int32)
+    cu, ck = cu_h.to(dev), ck_h.to(dev)
+    idx = torch.empty(48, dtype=torch.int32, device=dev)
+    pos = torch.empty_like(idx)
+    bias = torch.empty(48, dtype=torch.float32, device=dev)
+
+    def call():
+        tg.tg_topk_compact(z, pr, cu, cu_h, ck, ck_h, idx, pos, bias, stream=stream)
+    for _ in range(3):
+        call()
+    ms = []
+    for _ in range(reps):
+        flush.fill_(1.0)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        call()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ms.append(e0.elapsed_time(e1))
+    return sorted(ms)[len(ms) // 2]
+
+
 # ------------------------------------------------------------------ clocks (NVML)
 
 class ClockSampler:
@@ -227,6 +288,23 @@ class ClockSampler:
 # ------------------------------------------------------------------ our arm
 
 def run_ours(args, rank, world):
+    import torch
+    out = measure(args, args.workload, rank, world, extras=True)
+    subs = {}
+    for name in [w for w in args.also.split(",") if w and w != args.workload]:
+        torch.cuda.empty_cache()
+        sub = measure(args, name, rank, world, extras=False)
+        subs[sub["config"]["workload"]] = {k: sub[k] for k in (
+            "value", "unit", "ms_per_step", "steps", "warmup", "config", "e2e", "gpu_launches",
+            "roofline", "rooflines", "stages", "clocks")}
+    if subs:
+        out["workloads"] = subs
+    return out
+
+
+def measure(args, wl_name, rank, world, extras):
+    """One workload, timed as described at the top of this file.  With `extras`, also the
+    gate backward kernels and the dense full-context reference."""
     import numpy as np
     import torch
 
@@ -234,7 +312,7 @@ def run_ours(args, rank, world):
     import synthetic_inputs as S
 
     dev = torch.device("cuda", torch.cuda.current_device())
-    wl = workload(args.workload)
+    wl = workload(wl_name)
     # replicas: rank r draws its own batch (seed offset), same weights
     wl = replica_workload(wl, rank, world)
     h = S.hidden_rows(wl)
@@ -459,8 +537,10 @@ def run_ours(args, rank, world):
 
     # ---- per-stage roofline
     peaks, peak_src = load_peaks()
+    clocks = clk.summary()
     work = stage_work(wl, [int(x) for x in P["ck_h"].tolist()],
                       S.FFN if args.full_layers else 0)
+    topk_floor_ms = topk_latency_floor(tg, dev, stream, flush)
     stages = {}
     for name, ms_list in per_stage.items():
         n_launch = len(ms_list)
@@ -468,9 +548,21 @@ def run_ours(args, rank, world):
         w = work.get(name, {})
         entry = {"launches": n_launch, "total_ms": sum(ms_list), "avg_ms": avg_ms}
         if w.get("bound") == "tensor" and "flops" in w:
+            # kernels of a step of a few ms: the burst peak applies (the sustained figure
+            # is a seconds-long loop under the power cap), reported beside it
             ach = w["flops"] / (avg_ms / 1e3) / 1e12
             entry.update(bound="tensor", achieved=ach, unit="TFLOP/s",
-                         peak=peaks["bf16_tflops_sustained"], frac=ach / peaks["bf16_tflops_sustained"])
+                         peak=peaks["bf16_tflops"], frac=ach / peaks["bf16_tflops"],
+                         frac_of_sustained=ach / peaks["bf16_tflops_sustained"])
+        elif name in ("topk_compact",) and "bytes" in w:
+            # a few hundred KB: bound by the dependent chain of the select (three radix
+            # passes and the compaction, each a cluster-wide exchange), not by HBM
+            ach = w["bytes"] / (avg_ms / 1e3) / 1e9
+            entry.update(bound="latency", achieved_gbs=ach, floor_ms=topk_floor_ms,
+                         frac=topk_floor_ms / avg_ms if topk_floor_ms else None,
+                         hbm_frac=ach / peaks["hbm_gbs"],
+                         floor="the same kernel on one 64-token request: its fixed chain of "
+                               "three radix passes and the compaction")
         elif "bytes" in w:
             ach = w["bytes"] / (avg_ms / 1e3) / 1e9
             entry.update(bound="hbm", achieved=ach, unit="GB/s", peak=peaks["hbm_gbs"],
@@ -479,29 +571,25 @@ def run_ours(args, rank, world):
     tot = sum(v["total_ms"] for v in stages.values())
     for v in stages.values():
         v["share"] = v["total_ms"] / tot if tot else None
-    dom = max(stages, key=lambda k: stages[k]["total_ms"])
-    d = stages[dom]
-    traffic = load_traffic(dom, wl.name)
-    roofline = {"kernel": dom, "bound": d.get("bound"), "achieved": d.get("achieved"),
+
+    def roof(kernel):
+        d = stages[kernel]
+        return {"kernel": kernel, "bound": d.get("bound"), "achieved": d.get("achieved"),
                 "peak": d.get("peak"), "unit": d.get("unit"), "frac": d.get("frac"),
-                "traffic": traffic, "peak_source": f"{peak_src} (sustained for tensor, "
-                                                   f"copy bandwidth for hbm)"}
+                "traffic": load_traffic(kernel, wl.name),
+                "peak_source": f"{peak_src}: burst bf16 for tensor-bound kernels (timed "
+                               f"inside a step of a few ms), copy bandwidth for hbm",
+                "sm_mhz": clocks.get("sm_mhz")}
+    dom = max(stages, key=lambda k: stages[k]["total_ms"])
+    roofline = roof(dom)
+    rooflines = {k: roof(k) for k in ("attention", "gather", "gate_score", "qkv_rope_cache",
+                                      "out_proj") if k in stages and k != dom}
 
     out = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": wl.name, "batch": wl.batch, "tokens_per_request": list(wl.lengths)
-                   if wl.batch <= 8 else None, "question_tokens": list(wl.questions)
-                   if wl.batch <= 8 else None, "kept": int(P["ck_h"][-1]),
-                   "gated_layers": wl.n_layers, "lower_layers": args.lower_layers,
-                   "layer_body": "full (QK-norm, SwiGLU 6144)" if args.full_layers
-                   else "attention only",
-                   "hidden": wl.hidden,
-                   "heads": f"{wl.n_q_heads}q/{wl.n_kv_heads}kv x {wl.head_dim}",
-                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-                   "l2": "flushed before every timed step (512 MiB write, outside the timing)",
-                   "launch": "cuda_graph" if use_graph else "eager"},
+        "config": config_dict(wl, args, world),
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "steps": e2e_steps_done,
                 "copies": "double-buffered: next step's H2D and this step's D2H overlap the "
@@ -510,10 +598,13 @@ def run_ours(args, rank, world):
         "gpu_launches": gpu_launches,
         "ms_per_step_with_stage_events": sum(marked_ms) / max(1, len(marked_ms)),
         "roofline": roofline,
+        "rooflines": rooflines,
         "stages": {k: {kk: (round(vv, 5) if isinstance(vv, float) else vv)
                        for kk, vv in v.items()} for k, v in stages.items()},
-        "clocks": clk.summary(),
+        "clocks": clocks,
     }
+    if not extras:
+        return out
     if args.bias_grad_steps > 0 and int(P["K"]) > 0:
         out["bias_grad"] = bias_grad_timing(tg, wl, P, pipe, flush, stream,
                                             args.bias_grad_steps, peaks)
@@ -681,13 +772,15 @@ def dense_reference(tg, wl, layers, h_dev, flush, stream, steps, peaks, gated_ms
     pairs = sum(n * (n + 1) // 2 for n in wl.lengths)
     attn_ms = sum(attn) / len(attn) if attn else None
     tf = 4 * wl.head_dim * wl.n_q_heads * pairs / (attn_ms / 1e3) / 1e12 if attn else None
-    peak = peaks["bf16_tflops_sustained"]
+    peak = peaks["bf16_tflops"]
     return {"what": "same layers over all tokens: K = N, gamma = 0, tau = 1, no gate",
             "kept": wl.total_tokens, "layers": len(layers), "steps": steps,
             "ms_per_step": d_ms, "tokens_per_s": wl.total_tokens / (d_ms / 1e3),
             "gated_speedup": d_ms / gated_ms,
             "attention": {"avg_ms": attn_ms, "achieved": tf, "unit": "TFLOP/s",
-                          "peak": peak, "frac": tf / peak if tf else None}}
+                          "peak": peak, "frac": tf / peak if tf else None,
+                          "frac_of_sustained": (tf / peaks["bf16_tflops_sustained"]
+                                                if tf else None)}}
 
 
 def load_traffic(kernel, workload_name):
@@ -760,24 +853,34 @@ def cpu_baseline(wl, n_layers_sample):
 
 
 def run_reference(args, rank, world):
+    """The oracle on the host cores.  Each timed step is a bounded sample of the workload's
+    step: the whole gate over all N tokens plus ONE of the gated layers.  `steps` and
+    `ms_per_step` are the samples actually timed and their measured time; `value` is the
+    workload's tokens over the full step's time extrapolated from the sample (the gate's
+    time plus the one layer's time times the layer count), marked as such."""
     wl = workload(args.workload)
     for _ in range(args.warmup):
         oracle_sample(wl, 1)
-    secs = []
+    full, measured = [], []
     for _ in range(args.steps):
-        secs.append(oracle_sample(wl, 1)["seconds_per_step"])
-    value = wl.total_tokens * len(secs) / sum(secs)
+        r = oracle_sample(wl, 1)
+        full.append(r["seconds_per_step"])
+        measured.append(r["measured_s"])
+    value = wl.total_tokens * len(full) / sum(full)
     cores = blas_threads()
+    sample = (f"per step: gate over all {wl.total_tokens} tokens + 1 of {wl.n_layers} gated "
+              f"layers (measured), the full step's time extrapolated from that one layer")
     return {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * sum(secs) / len(secs),
+        "steps": len(measured), "warmup": args.warmup,
+        "ms_per_step": 1e3 * sum(measured) / len(measured),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic",
-        "config": {"workload": wl.name, "batch": wl.batch, "gated_layers": wl.n_layers},
+        "config": config_dict(wl, args, world),
+        "extrapolated_from_layers": 1,
+        "ms_per_full_step_extrapolated": 1e3 * sum(full) / len(full),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
-                         "sample": f"per step: gate over all {wl.total_tokens} tokens + 1 of "
-                                   f"{wl.n_layers} gated layers, layer time scaled to "
-                                   f"{wl.n_layers}"},
+                         "sample": sample},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
 
