@@ -94,6 +94,17 @@ int tg_status_read(const uint32_t* status, uint32_t* out_host, tg_stream_t strea
 int tg_set_launch_overlap(int enable);
 int tg_get_launch_overlap(void);
 
+/* Which kernel serves the gather mode of tg_gather_rope (no RoPE).  On (the default):
+ * the TMA row gather (tile::gather4 loads of four kept rows at a time, tiled TMA stores
+ * of four consecutive destination rows), used when width is a multiple of 64 and at
+ * most 8192 and the row counts fit in int32; off, or for other shapes: one warp per row
+ * with 16-byte loads and stores.  Both write the same bytes and report out-of-range
+ * indices the same way.  The setting is read at each call.
+ * tg_set_gather_tma: enable = 0 selects the warp-per-row copy; returns TG_OK.
+ * tg_get_gather_tma: the current setting (0 or 1). */
+int tg_set_gather_tma(int enable);
+int tg_get_gather_tma(void);
+
 /* L2 prefetch hint (not part of the method): issue bulk prefetches that bring
  * [ptr, ptr + bytes) into the L2 cache ahead of a later kernel that reads it (the
  * next layer's weights while attention runs, for instance).  Nothing waits for the

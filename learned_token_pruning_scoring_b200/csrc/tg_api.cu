@@ -42,6 +42,11 @@ static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 
 int make_tmap_bf16_2d(CUtensorMap* out, const void* base, uint64_t rows, uint64_t cols,
                       uint64_t ld, uint32_t box_cols, uint32_t box_rows) {
+  return make_tmap_bf16_2d_swz(out, base, rows, cols, ld, box_cols, box_rows, true);
+}
+
+int make_tmap_bf16_2d_swz(CUtensorMap* out, const void* base, uint64_t rows, uint64_t cols,
+                          uint64_t ld, uint32_t box_cols, uint32_t box_rows, bool swizzle128) {
   auto fn = encode_fn();
   if (!fn) {
     set_cuda_error(cudaErrorNotSupported);
@@ -54,7 +59,8 @@ int make_tmap_bf16_2d(CUtensorMap* out, const void* base, uint64_t rows, uint64_
   cuuint32_t estr[2] = {1, 1};
   CUresult r = fn(out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
                   strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) {
     set_cuda_error(cudaErrorInvalidValue);
@@ -65,7 +71,10 @@ int make_tmap_bf16_2d(CUtensorMap* out, const void* base, uint64_t rows, uint64_
 
 namespace {
 std::atomic<int> g_launch_overlap{0};
+std::atomic<int> g_gather_tma{1};
 }
+
+bool gather_use_tma() { return g_gather_tma.load(std::memory_order_relaxed) != 0; }
 
 bool launch_overlap() { return g_launch_overlap.load(std::memory_order_relaxed) != 0; }
 void set_launch_overlap(bool on) { g_launch_overlap.store(on ? 1 : 0, std::memory_order_relaxed); }
@@ -145,6 +154,13 @@ int tg_set_launch_overlap(int enable) {
 }
 
 int tg_get_launch_overlap(void) { return tg::launch_overlap() ? 1 : 0; }
+
+int tg_set_gather_tma(int enable) {
+  tg::g_gather_tma.store(enable ? 1 : 0);
+  return TG_OK;
+}
+
+int tg_get_gather_tma(void) { return tg::gather_use_tma() ? 1 : 0; }
 
 int tg_status_clear(uint32_t* status, tg_stream_t stream) {
   if (!status) return TG_ERR_INVALID_ARGUMENT;

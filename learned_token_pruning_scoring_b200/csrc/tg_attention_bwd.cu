@@ -215,7 +215,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* do_full = bars + 6;      // [2]
   uint64_t* do_empty = bars + 8;     // [2] the dP MMAs that read the stage are done
   uint64_t* blk_full = bars + 10;    // [kBlkStages]
-  uint64_t* blk_empty = bars + 14;   // [kBlkStages] MMAs + the head's 4 compute warps done
+  uint64_t* blk_empty = bars + 14;   // [kBlkStages] MMAs + the head's 128 compute threads done
   uint64_t* s_full = bars + 18;      // [2] S^T and dP^T of the head in TMEM
   uint64_t* tmem_free = bars + 20;   // [2] the head's compute threads read them
   uint64_t* drain = bars + 22;
@@ -236,7 +236,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int s = 0; s < kBlkStages; ++s) {
       mbar_init(&blk_full[s], 1);
-      mbar_init(&blk_empty[s], 5);
+      mbar_init(&blk_empty[s], 1 + 128);  // the MMA commit + each compute thread
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -433,8 +433,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (kBeta) accb = fmaf(dl, fmaf(a.w, s, -cu[col] * b_c), accb);
         }
       }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&blk_empty[bs]);  // done with the block's scalars
+      // done with the block's scalars: every reading thread releases it itself, its
+      // reads ordered (release, proxy fence) before the bulk copy that refills it
+      fence_proxy_async_smem();
+      mbar_arrive(&blk_empty[bs]);
     }
     const int64_t slot = (int64_t)item * hg + head_grp;
     p.part[((slot * 2 + 0) * 2 + wg) * 128 + key] = acc;

@@ -170,7 +170,7 @@ __device__ __forceinline__ float warp_transpose_sum(float (&v)[32], int lane) {
 // with its gradient epilogue.  Roles: warp 0 lane 0 loads the h and W1' k-blocks;
 // warp 1 owns TMEM and lane 0 issues the MMAs (M = 128, N = 256, K = 16); warps 2-5
 // read every A stage for the row sums of squares (a stage is released by the MMA
-// commit plus these four warps), then each thread takes one row of the accumulator:
+// commit plus each of these 128 threads), then each thread takes one row of the accumulator:
 // u = r acc, du' = r ds w2 SiLU'(u) stored as bf16, and the warp's column sums of
 // ds SiLU(u) over its 32 rows.  Rows past M come from the TMA's zero fill with ds = 0.
 __global__ void __launch_bounds__(kGgThreads, 1)
@@ -195,7 +195,7 @@ __global__ void __launch_bounds__(kGgThreads, 1)
   if (tid == 0) {
     for (int s = 0; s < kGgStages; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 1 + 4);  // the MMA commit and the four norm warps
+      mbar_init(&empty[s], 1 + 128);  // the MMA commit and each of the 128 norm readers
     }
     mbar_init(acc_full, 1);
     mbar_init(drain, 1);
@@ -277,8 +277,9 @@ __global__ void __launch_bounds__(kGgThreads, 1)
           ss = fmaf(f.y, f.y, ss);
         }
       }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&empty[s]);
+      // each reader releases the stage itself (its reads ordered before the refill)
+      fence_proxy_async_smem();
+      mbar_arrive(&empty[s]);
     }
     const float rscale = rsqrtf(ss / (float)p.K + p.eps);
     const bool ok = warp_all(mbar_wait(acc_full, 0, abort_flag, p.status));

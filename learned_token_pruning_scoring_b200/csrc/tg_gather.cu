@@ -196,6 +196,161 @@ __global__ void __launch_bounds__(kCopyWarps * 32) gather_rope_kernel(GatherArgs
   }
 }
 
+// ------------------------------------------------------------------ TMA row gather
+//
+// Gather mode through the tensor memory accelerator: groups of four kept rows come in
+// with tile::gather4 loads (four row indices, box_cols columns per load, no swizzle) and
+// leave with tiled TMA stores of four consecutive destination rows.  One CTA per SM
+// walks a contiguous range of groups through a ring of stages (a stage is one group:
+// width / box_cols chunks of 4 x box_cols elements, chunk j holding columns
+// [j box_cols, (j + 1) box_cols) of the four rows).  Thread 0 issues the loads and the
+// stores; a stage is refilled once its store has read it (bulk read groups) and, when
+// row sums of squares are asked for, once the four warps (one per row) have read it.
+// A group whose index is out of range loads row 0 in its place, stores only its valid
+// rows (a one-row store map) and sets TG_STATUS_BOUNDS, as the copy kernel skips such
+// rows; rows past n_rows of the last group are clipped by the store map.
+constexpr int kTgThreads = 128;
+constexpr int kTgMaxStages = 16;
+constexpr int kTgSmemBudget = 192 * 1024;
+constexpr int kTgRefillLag = 2;  // stores allowed to be still reading when a stage refills
+
+struct TmaGatherArgs {
+  const int32_t* row_idx;
+  int64_t n_rows;
+  int64_t src_rows;
+  int width;
+  int box_cols;
+  int stages;
+  int64_t n_groups;
+  float* row_ssq;
+  int64_t ld_ssq;
+  uint32_t* status;
+};
+
+__global__ void __launch_bounds__(kTgThreads, 1)
+    gather_tma_kernel(const __grid_constant__ CUtensorMap tm_src,
+                      const __grid_constant__ CUtensorMap tm_dst4,
+                      const __grid_constant__ CUtensorMap tm_dst1, TmaGatherArgs a) {
+  extern __shared__ __align__(128) unsigned char smem_raw[];
+  const int stage_bytes = 4 * a.width * 2;
+  unsigned char* ring = smem_raw;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem_raw + a.stages * stage_bytes);
+  uint32_t* valid = reinterpret_cast<uint32_t*>(full + kTgMaxStages);  // [stage] rows to store
+  uint32_t* bad = valid + kTgMaxStages;                               // [stage] an index was bad
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int64_t g0 = a.n_groups * blockIdx.x / gridDim.x;
+  const int64_t g1 = a.n_groups * (blockIdx.x + 1) / gridDim.x;
+  const int n_my = (int)(g1 - g0);
+  const int chunks = a.width / a.box_cols;
+  const int chunk_bytes = 4 * a.box_cols * 2;
+
+  if (tid == 0) {
+    for (int s = 0; s < a.stages; ++s) mbar_init(&full[s], 1);
+    fence_mbar_init();
+  }
+  if (tid == 0) {
+    tma_prefetch_desc(&tm_src);
+    tma_prefetch_desc(&tm_dst4);
+  }
+  __syncthreads();
+  griddep_wait();  // the indices and the source rows may come from the grid before
+
+  auto issue = [&](int li) {  // thread 0: load group g0 + li into stage li % stages
+    const int s = li % a.stages;
+    const int64_t row0 = (g0 + li) * 4;
+    int32_t r[4];
+    uint32_t ok = 0, err = 0;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int64_t row = row0 + e;
+      int64_t idx = 0;
+      if (row < a.n_rows) {
+        idx = a.row_idx ? (int64_t)a.row_idx[row] : row;
+        if (idx < 0 || idx >= a.src_rows) {
+          err = 1;
+          idx = 0;
+        } else {
+          ok |= 1u << e;
+        }
+      }
+      r[e] = (int32_t)idx;
+    }
+    if (err && a.status) atomicOr(a.status, TG_STATUS_BOUNDS);
+    valid[s] = ok;
+    bad[s] = err;
+    unsigned char* st = ring + s * stage_bytes;
+    mbar_arrive_expect_tx(&full[s], (uint32_t)stage_bytes);
+    for (int j = 0; j < chunks; ++j)
+      tma_gather4(st + j * chunk_bytes, &tm_src, j * a.box_cols, r[0], r[1], r[2], r[3],
+                  &full[s]);
+  };
+  auto store = [&](int li) {  // thread 0: store group g0 + li from its stage
+    const int s = li % a.stages;
+    const int64_t row0 = (g0 + li) * 4;
+    const unsigned char* st = ring + s * stage_bytes;
+    if (!bad[s]) {
+      for (int j = 0; j < chunks; ++j)
+        tma_store_2d(&tm_dst4, j * a.box_cols, (int32_t)row0, st + j * chunk_bytes);
+    } else {
+      for (int e = 0; e < 4; ++e)
+        if (valid[s] >> e & 1u)
+          for (int j = 0; j < chunks; ++j)
+            tma_store_2d(&tm_dst1, j * a.box_cols, (int32_t)(row0 + e),
+                         st + j * chunk_bytes + e * a.box_cols * 2);
+    }
+    bulk_commit_group();
+  };
+
+  const bool ssq = a.row_ssq != nullptr;
+  if (tid == 0)
+    for (int li = 0; li < n_my && li < a.stages; ++li) issue(li);
+  if (ssq || tid == 0) {
+    const int nvec = a.width >> 3;
+    for (int li = 0; li < n_my; ++li) {
+      const int s = li % a.stages;
+      const uint32_t ph = (uint32_t)(li / a.stages) & 1u;
+      bool ok = mbar_wait(&full[s], ph, nullptr, a.status);
+      if (ssq) ok = __syncthreads_and(ok) != 0;
+      if (!ok) break;  // a load that never landed (status has TIMEOUT): give up
+      if (ssq) {
+        // warp w: row w of the group; lane l sums vectors l, l + 32, ... (16 vectors =
+        // one 128-column group, so each half-warp holds one group per step)
+        const int64_t row = (g0 + li) * 4 + warp;
+        const bool mine = (valid[s] >> warp & 1u) != 0;
+        const unsigned char* st = ring + s * stage_bytes;
+        for (int base = 0; base < nvec; base += 32) {
+          const int v = base + lane;
+          float q = 0.f;
+          if (mine && v < nvec) {
+            const int col = v * 8;
+            const int j = col / a.box_cols;
+            q = ssq8(*reinterpret_cast<const uint4*>(st + j * chunk_bytes +
+                                                     (warp * a.box_cols + col - j * a.box_cols) * 2));
+          }
+#pragma unroll
+          for (int o = 8; o > 0; o >>= 1) q += __shfl_xor_sync(0xFFFFFFFFu, q, o);
+          if (mine && v < nvec && (lane & 15) == 0) a.row_ssq[row * a.ld_ssq + (v >> 4)] = q;
+        }
+        fence_proxy_async_smem();  // these reads before the refill's TMA write
+        __syncthreads();
+      }
+      if (tid == 0) {
+        store(li);
+        // refill the stage whose store is now at least kTgRefillLag groups old
+        const int lr = li - kTgRefillLag;
+        if (lr >= 0 && lr + a.stages < n_my) {
+          bulk_wait_read<kTgRefillLag>();
+          issue(lr + a.stages);
+        }
+      }
+    }
+    // the last kTgRefillLag stages were never refilled; nothing is left in flight but
+    // stores, which must finish before the CTA exits
+    if (tid == 0) bulk_wait_all();
+  }
+}
+
 struct KvArgs {
   const uint16_t* k;
   int64_t ld_k;
@@ -238,6 +393,37 @@ int copy_grid(int64_t rows, int blocks_per_sm) {
   const int64_t want = (rows + kCopyWarps - 1) / kCopyWarps;
   const int64_t cap = (int64_t)sm_count() * blocks_per_sm;
   return (int)(want < cap ? (want < 1 ? 1 : want) : cap);
+}
+
+// The TMA row gather for one call of the gather mode (width a multiple of 64).
+int gather_tma(const GatherArgs& g, cudaStream_t stream) {
+  const int box = (g.width % 256) == 0 ? 256 : (g.width % 128) == 0 ? 128 : 64;
+  const int stage_bytes = 4 * g.width * 2;
+  int stages = kTgSmemBudget / stage_bytes;
+  if (stages > kTgMaxStages) stages = kTgMaxStages;
+  const int64_t n_groups = (g.n_rows + 3) / 4;
+  CUtensorMap ts, t4, t1;
+  TG_TRY(make_tmap_bf16_2d_swz(&ts, g.src, (uint64_t)g.src_rows, (uint64_t)g.width,
+                               (uint64_t)g.ld_src, (uint32_t)box, 1, false));
+  TG_TRY(make_tmap_bf16_2d_swz(&t4, g.dst, (uint64_t)g.n_rows, (uint64_t)g.width,
+                               (uint64_t)g.ld_dst, (uint32_t)box, 4, false));
+  TG_TRY(make_tmap_bf16_2d_swz(&t1, g.dst, (uint64_t)g.n_rows, (uint64_t)g.width,
+                               (uint64_t)g.ld_dst, (uint32_t)box, 1, false));
+  const size_t smem = (size_t)stages * stage_bytes + kTgMaxStages * (8 + 4 + 4);
+  static int attr_dev = -1;
+  int dev = 0;
+  TG_CUDA_TRY(cudaGetDevice(&dev));
+  if (attr_dev != dev) {
+    TG_CUDA_TRY(cudaFuncSetAttribute(gather_tma_kernel,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     kTgSmemBudget + kTgMaxStages * 16));
+    attr_dev = dev;
+  }
+  TmaGatherArgs a{g.row_idx, g.n_rows, g.src_rows, g.width, box, stages, n_groups,
+                  g.row_ssq, g.ld_ssq, g.status};
+  const int64_t ctas = n_groups < sm_count() ? n_groups : sm_count();
+  return launch(gather_tma_kernel, dim3((unsigned)ctas), dim3(kTgThreads), smem, stream, ts, t4,
+                t1, a);
 }
 
 }  // namespace
@@ -285,9 +471,13 @@ extern "C" int tg_gather_rope(const tg_bf16* src, int64_t ld_src, int64_t src_ro
   GatherArgs a{reinterpret_cast<const uint16_t*>(src), ld_src, src_rows, row_idx, n_rows, width,
                rope_pos, rope_col_begin, rope_col_end, head_dim, cos_sin, max_pos,
                reinterpret_cast<uint16_t*>(dst), ld_dst, row_ssq_out, ld_ssq_out, status};
-  if (!rope_pos || rope_col_begin >= rope_col_end)
+  if (!rope_pos || rope_col_begin >= rope_col_end) {
+    if (gather_use_tma() && (width % 64) == 0 && width * 8 * (kTgRefillLag + 1) <= kTgSmemBudget &&
+        src_rows < (int64_t)0x7FFFFFFF && n_rows < (int64_t)0x7FFFFFFF)
+      return gather_tma(a, (cudaStream_t)stream);
     return launch(gather_copy_kernel, dim3(copy_grid(n_rows, kCopyBlocksPerSm)),
                   dim3(kCopyWarps * 32), 0, (cudaStream_t)stream, a);
+  }
   // the RoPE kernel is register-heavy (one block per SM); it serves the unfused path
   return launch(gather_rope_kernel, dim3(copy_grid(n_rows, 1)), dim3(kCopyWarps * 32), 0,
                 (cudaStream_t)stream, a);

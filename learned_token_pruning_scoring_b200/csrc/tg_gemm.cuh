@@ -242,7 +242,7 @@ __global__ void __launch_bounds__(192, 1)
   if (tid == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 1 + (norm_here ? 4 : 0));
+      mbar_init(&empty[s], 1 + (norm_here ? 128 : 0));  // MMA commit + each norm reader
     }
     mbar_init(acc_full, 1);
     mbar_init(drain, 1);
@@ -329,8 +329,13 @@ __global__ void __launch_bounds__(192, 1)
             ss = fmaf(f.y, f.y, ss);
           }
         }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&empty[s]);
+        // Every reading thread releases the stage itself: its arrive (release) orders
+        // its own shared-memory reads before the stage is handed back, and the proxy
+        // fence orders them before the TMA write that refills it.  A single arrive by
+        // lane 0 after __syncwarp did not order the other lanes' reads, and refills
+        // were seen to overwrite rows still being read (rows with a wrong RMS).
+        fence_proxy_async_smem();
+        mbar_arrive(&empty[s]);
       }
     }
     float rscale = 1.0f;

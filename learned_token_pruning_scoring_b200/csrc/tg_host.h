@@ -31,12 +31,20 @@ int check_launch();
 int make_tmap_bf16_2d(CUtensorMap* out, const void* base, uint64_t rows, uint64_t cols,
                       uint64_t ld, uint32_t box_cols, uint32_t box_rows);
 
+// The same with the swizzle chosen: swizzle128 = false lays a box out plainly, row after
+// row (box_cols * 2 a multiple of 16, box_cols <= 256).
+int make_tmap_bf16_2d_swz(CUtensorMap* out, const void* base, uint64_t rows, uint64_t cols,
+                          uint64_t ld, uint32_t box_cols, uint32_t box_rows, bool swizzle128);
+
 // Number of SMs of the current device (cached).
 int sm_count();
 
 // Library-wide switch (tg_set_launch_overlap): launch kernels with programmatic stream
 // serialisation so that a grid's launch and prologue overlap the end of the grid before it.
 bool launch_overlap();
+// Library-wide switch (tg_set_gather_tma): the gather mode of tg_gather_rope uses the TMA
+// row-gather kernel where the shape allows it (the default), else the warp-per-row copy.
+bool gather_use_tma();
 void set_launch_overlap(bool on);
 
 // Launch `kernel` on `stream`, with programmatic stream serialisation when the switch is

@@ -180,6 +180,28 @@ __device__ __forceinline__ void tma_load_2d(void* smem_dst, const void* tmap, in
       : "memory");
 }
 
+// Row gather: rows r0..r3 of a 2-D tensor (a tensor map whose box is box_cols x 1, no
+// swizzle), columns [x, x + box_cols), land in shared memory one after another (4 rows x
+// box_cols elements), completing 4 * box_cols * elem_size bytes on `bar`.  Rows outside
+// the tensor read as zero.  x * elem_size must be a multiple of 16.
+__device__ __forceinline__ void tma_gather4(void* smem_dst, const void* tmap, int32_t x,
+                                            int32_t r0, int32_t r1, int32_t r2, int32_t r3,
+                                            uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4, %5, %6}], [%7];" ::"r"(smem_u32(smem_dst)),
+      "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(r0), "r"(r1), "r"(r2), "r"(r3),
+      "r"(smem_u32(bar))
+      : "memory");
+}
+
+// Wait until at most N of this thread's committed bulk store groups are still reading
+// shared memory.
+template <int N>
+__device__ __forceinline__ void bulk_wait_read() {
+  asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
+
 // Contiguous bulk copy of `bytes` (multiple of 16; both addresses 16-byte aligned) from
 // global to this CTA's shared memory, completing that many transaction bytes on `bar`.
 __device__ __forceinline__ void bulk_load(void* smem_dst, const void* gsrc, uint32_t bytes,

@@ -71,6 +71,59 @@ def test_gather_bit_exact(tg, n_src, n_rows, width):
     assert torch.equal(out.cpu(), src.cpu()[idx.long()])
 
 
+@pytest.mark.parametrize("n_src,n_rows,width,ssq", [
+    (1000, 1, 2048, True), (1000, 3, 2048, False), (1000, 5, 2048, True),
+    (20000, 1638, 2048, True), (131072, 13107, 2048, True),   # kept rows of the 16k / 128k steps
+    (5000, 4000, 8192, False),                                  # three stages: refills at lag 2
+    (300, 299, 64, False), (300, 77, 192, False), (300, 257, 4096, True)])
+@pytest.mark.parametrize("tma", [True, False])
+def test_gather_tma_and_copy_kernels(tg, n_src, n_rows, width, ssq, tma):
+    """The gather mode's two kernels (TMA row gather, warp-per-row copy) move the same
+    bytes, tail groups of fewer than four rows and ring refills included, and write the
+    same row sums of squares."""
+    src = _dev(S.uniform_rows(n_src, width, seed=n_rows + width))
+    idx = torch.randint(0, n_src, (n_rows,), generator=torch.Generator().manual_seed(n_rows),
+                        dtype=torch.int32)
+    prev = tg.tg_get_gather_tma()
+    try:
+        tg.tg_set_gather_tma(tma)
+        st = _status()
+        q = torch.full((n_rows, width // 128), float("nan"), device="cuda") if ssq else None
+        out = tg.tg_gather_rope(src, row_idx=_dev(idx), row_ssq=q, status=st)
+        assert tg.tg_status_read(st) == 0
+    finally:
+        tg.tg_set_gather_tma(prev)
+    want = src.cpu()[idx.long()]
+    assert torch.equal(out.cpu(), want)
+    if ssq:
+        ref = (want.double() ** 2).view(n_rows, width // 128, 128).sum(-1)
+        assert torch.allclose(q.cpu().double(), ref, rtol=1e-5, atol=1e-5)
+
+
+@pytest.mark.parametrize("tma", [True, False])
+def test_gather_out_of_range_rows_are_skipped(tg, tma):
+    """Indices outside the source set TG_STATUS_BOUNDS and leave their destination rows
+    as they were; the other rows of the same group of four are still copied."""
+    n_src, width = 100, 2048
+    src = _dev(S.uniform_rows(n_src, width, seed=4))
+    idx = torch.tensor([3, -1, 7, 9, 100, 11, 12, 13, 50], dtype=torch.int32)
+    dst = torch.full((len(idx), width), 7.0, dtype=torch.bfloat16, device="cuda")
+    prev = tg.tg_get_gather_tma()
+    try:
+        tg.tg_set_gather_tma(tma)
+        st = _status()
+        tg.tg_gather_rope(src, dst, row_idx=_dev(idx), status=st)
+        assert tg.tg_status_read(st) & tg.STATUS_BOUNDS
+    finally:
+        tg.tg_set_gather_tma(prev)
+    got = dst.cpu()
+    for r, i in enumerate(idx.tolist()):
+        if 0 <= i < n_src:
+            assert torch.equal(got[r], src.cpu()[i]), r
+        else:
+            assert torch.all(got[r] == 7.0), r
+
+
 def test_gather_strided_views(tg):
     big = _dev(S.uniform_rows(300, 4096, seed=3))
     src = big[:, 1024:3072]
