@@ -94,16 +94,27 @@ int tg_status_read(const uint32_t* status, uint32_t* out_host, tg_stream_t strea
 int tg_set_launch_overlap(int enable);
 int tg_get_launch_overlap(void);
 
-/* Which kernel serves the gather mode of tg_gather_rope (no RoPE).  On (the default):
- * the TMA row gather (tile::gather4 loads of four kept rows at a time, tiled TMA stores
- * of four consecutive destination rows), used when width is a multiple of 64 and at
- * most 8192 and the row counts fit in int32; off, or for other shapes: one warp per row
- * with 16-byte loads and stores.  Both write the same bytes and report out-of-range
- * indices the same way.  The setting is read at each call.
+/* Which kernel serves the gather mode of tg_gather_rope (no RoPE).  Off (the default):
+ * one warp per row with 16-byte loads and stores, every row of a batch loaded before it
+ * is stored.  On: the TMA row gather (tile::gather4 loads of four kept rows at a time,
+ * tiled TMA stores of four consecutive destination rows), used when width is a multiple
+ * of 64 and at most 8192 and the row counts fit in int32.  Both write the same bytes and
+ * report out-of-range indices the same way; on B200 the warp-per-row copy measured
+ * faster at the kept-row counts of the 16k and 128k steps.  Read at each call.
  * tg_set_gather_tma: enable = 0 selects the warp-per-row copy; returns TG_OK.
  * tg_get_gather_tma: the current setting (0 or 1). */
 int tg_set_gather_tma(int enable);
 int tg_get_gather_tma(void);
+
+/* Which kernel runs the scorer GEMM of tg_gate_score (and tg_gate_score_noalloc).  On
+ * (the default): persistent CTA pairs over 256-row tiles (tcgen05 cta_group::2, each CTA
+ * streaming half of W1 per k-block, two accumulators so a tile's epilogue overlaps the
+ * next tile's loads); off: one CTA per 128-row tile.  Both form the same products in the
+ * same order, so s, z and bias are identical.  Read at each call.
+ * tg_set_scorer_pair: enable = 0 selects the one-CTA kernel; returns TG_OK.
+ * tg_get_scorer_pair: the current setting (0 or 1). */
+int tg_set_scorer_pair(int enable);
+int tg_get_scorer_pair(void);
 
 /* L2 prefetch hint (not part of the method): issue bulk prefetches that bring
  * [ptr, ptr + bytes) into the L2 cache ahead of a later kernel that reads it (the

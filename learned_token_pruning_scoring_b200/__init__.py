@@ -26,7 +26,7 @@ __all__ = [
     "tg_rope_table", "tg_gate_score_workspace_size", "tg_gate_score", "tg_topk_compact",
     "tg_gate_score_noalloc", "tg_seq_rmsnorm", "tg_gather_rope", "tg_kv_compact", "tg_gated_attention", "tg_linear",
     "tg_status_clear", "tg_status_read", "tg_set_launch_overlap", "tg_get_launch_overlap",
-    "tg_set_gather_tma", "tg_get_gather_tma",
+    "tg_set_gather_tma", "tg_get_gather_tma", "tg_set_scorer_pair", "tg_get_scorer_pair",
     "tg_prefetch_l2", "tg_out_proj_qkv_next", "tg_out_proj_qkv_workspace_size",
     "tg_swiglu", "tg_fold_norm_weight", "tg_pack_gate_up", "prepare_layer",
     "tg_gated_attention_bias_grad", "tg_gated_attention_bias_grad_workspace_size",
@@ -110,13 +110,22 @@ def tg_get_launch_overlap() -> bool:
 
 
 def tg_set_gather_tma(enable: bool) -> None:
-    """Gather mode of tg_gather_rope: the TMA row gather (True, default) or the
-    warp-per-row copy (False)."""
+    """Gather mode of tg_gather_rope: the TMA row gather (True) or the warp-per-row
+    copy (False, default)."""
     _check(lib.tg_set_gather_tma(1 if enable else 0), "tg_set_gather_tma")
 
 
 def tg_get_gather_tma() -> bool:
     return bool(lib.tg_get_gather_tma())
+
+
+def tg_set_scorer_pair(enable: bool) -> None:
+    """Scorer GEMM of tg_gate_score: CTA pairs (True, default) or one CTA per tile."""
+    _check(lib.tg_set_scorer_pair(1 if enable else 0), "tg_set_scorer_pair")
+
+
+def tg_get_scorer_pair() -> bool:
+    return bool(lib.tg_get_scorer_pair())
 
 
 def tg_prefetch_l2(t: torch.Tensor, stream=None) -> None:

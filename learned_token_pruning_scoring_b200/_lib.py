@@ -29,6 +29,8 @@ SIGNATURES = {
     "tg_get_launch_overlap": (_i32, []),
     "tg_set_gather_tma": (_i32, [_i32]),
     "tg_get_gather_tma": (_i32, []),
+    "tg_set_scorer_pair": (_i32, [_i32]),
+    "tg_get_scorer_pair": (_i32, []),
     "tg_prefetch_l2": (_i32, [_p, _sz, _p]),
     "tg_rope_table": (_i32, [_p, _i32, _i32, _f64, _p]),
     "tg_plan_kept": (_i32, [_p, _p, _p, _i32, _p]),

@@ -71,10 +71,12 @@ int make_tmap_bf16_2d_swz(CUtensorMap* out, const void* base, uint64_t rows, uin
 
 namespace {
 std::atomic<int> g_launch_overlap{0};
-std::atomic<int> g_gather_tma{1};
+std::atomic<int> g_gather_tma{0};
+std::atomic<int> g_scorer_pair{1};
 }
 
 bool gather_use_tma() { return g_gather_tma.load(std::memory_order_relaxed) != 0; }
+bool scorer_use_pair() { return g_scorer_pair.load(std::memory_order_relaxed) != 0; }
 
 bool launch_overlap() { return g_launch_overlap.load(std::memory_order_relaxed) != 0; }
 void set_launch_overlap(bool on) { g_launch_overlap.store(on ? 1 : 0, std::memory_order_relaxed); }
@@ -161,6 +163,13 @@ int tg_set_gather_tma(int enable) {
 }
 
 int tg_get_gather_tma(void) { return tg::gather_use_tma() ? 1 : 0; }
+
+int tg_set_scorer_pair(int enable) {
+  tg::g_scorer_pair.store(enable ? 1 : 0);
+  return TG_OK;
+}
+
+int tg_get_scorer_pair(void) { return tg::scorer_use_pair() ? 1 : 0; }
 
 int tg_status_clear(uint32_t* status, tg_stream_t stream) {
   if (!status) return TG_ERR_INVALID_ARGUMENT;

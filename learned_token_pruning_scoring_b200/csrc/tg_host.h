@@ -43,8 +43,11 @@ int sm_count();
 // serialisation so that a grid's launch and prologue overlap the end of the grid before it.
 bool launch_overlap();
 // Library-wide switch (tg_set_gather_tma): the gather mode of tg_gather_rope uses the TMA
-// row-gather kernel where the shape allows it (the default), else the warp-per-row copy.
+// row-gather kernel where the shape allows it, else (the default) the warp-per-row copy.
 bool gather_use_tma();
+// Library-wide switch (tg_set_scorer_pair): the scorer GEMM of tg_gate_score runs on CTA
+// pairs (the default) or on one CTA per 128-row tile.
+bool scorer_use_pair();
 void set_launch_overlap(bool on);
 
 // Launch `kernel` on `stream`, with programmatic stream serialisation when the switch is

@@ -297,6 +297,33 @@ def test_gate_score_n16k_full(tg):
     _gate_case(tg, [16384], [64], seed=0)
 
 
+@pytest.mark.parametrize("lengths", [[1], [200], [256], [257], [5000, 3000], [16384],
+                                     [700, 37, 900, 1], [40000]])
+def test_scorer_pair_matches_one_cta_kernel(tg, lengths):
+    """The CTA-pair scorer and the one-CTA scorer form the same products and reduce them
+    in the same order: s, z and bias agree bit for bit (tails of a 256-row pair tile,
+    requests shorter than a tile, several tiles per cluster at 40k)."""
+    wl = S.custom(lengths, [min(64, n) for n in lengths], [0] * len(lengths))
+    h = _dev(S.hidden_rows(wl))
+    gw = {k: _dev(v) for k, v in S.gate_weights(wl).items()}
+    nw = _dev(0.8 + 0.4 * torch.rand(wl.hidden, generator=torch.Generator().manual_seed(5)))
+    pr = _dev(S.prunable_mask(wl))
+    cu = np.array(wl.cu_seqlens(), dtype=np.int32)
+    cud = _dev(torch.from_numpy(cu))
+    prev = tg.tg_get_scorer_pair()
+    outs = []
+    try:
+        for pair in (True, False):
+            tg.tg_set_scorer_pair(pair)
+            st = _status()
+            outs.append(tg.tg_gate_score(h, gw["W1"], gw["w2"], cud, cu, pr, norm_w=nw, status=st))
+            assert tg.tg_status_read(st) == 0
+    finally:
+        tg.tg_set_scorer_pair(prev)
+    for name, a, b in zip(("s", "z", "bias"), *outs):
+        assert torch.equal(a, b), (name, (a - b).abs().max().item())
+
+
 def test_gate_score_deterministic(tg):
     wl = S.custom([5000, 3000], [64, 16], [0, 0])
     h = _dev(S.hidden_rows(wl))
