@@ -300,9 +300,10 @@ def test_gate_score_n16k_full(tg):
 @pytest.mark.parametrize("lengths", [[1], [200], [256], [257], [5000, 3000], [16384],
                                      [700, 37, 900, 1], [40000]])
 def test_scorer_pair_matches_one_cta_kernel(tg, lengths):
-    """The CTA-pair scorer and the one-CTA scorer form the same products and reduce them
-    in the same order: s, z and bias agree bit for bit (tails of a 256-row pair tile,
-    requests shorter than a tile, several tiles per cluster at 40k)."""
+    """The CTA-pair scorer and the one-CTA scorer form the same products; the pair kernel
+    sums the k-blocks of each tile from a rotated start, so the two agree to fp32
+    rounding: s within 1e-5 of its RMS, z and bias within 2e-5 (tails of a 256-row pair
+    tile, requests shorter than a tile, several tiles per cluster at 40k)."""
     wl = S.custom(lengths, [min(64, n) for n in lengths], [0] * len(lengths))
     h = _dev(S.hidden_rows(wl))
     gw = {k: _dev(v) for k, v in S.gate_weights(wl).items()}
@@ -320,8 +321,11 @@ def test_scorer_pair_matches_one_cta_kernel(tg, lengths):
             assert tg.tg_status_read(st) == 0
     finally:
         tg.tg_set_scorer_pair(prev)
-    for name, a, b in zip(("s", "z", "bias"), *outs):
-        assert torch.equal(a, b), (name, (a - b).abs().max().item())
+    s_rms = outs[1][0].double().pow(2).mean().sqrt().item()
+    for name, a, b, tol in zip(("s", "z", "bias"), *outs, (1e-5 * s_rms, 2e-5, 2e-5)):
+        err = (a.double() - b.double()).abs().max().item()
+        assert err <= tol, (name, err, tol)
+    assert torch.all(outs[0][2][pr == 0] == 0)
 
 
 def test_gate_score_deterministic(tg):
