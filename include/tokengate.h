@@ -109,10 +109,8 @@ int tg_get_gather_tma(void);
 /* Which kernel runs the scorer GEMM of tg_gate_score (and tg_gate_score_noalloc).  On
  * (the default): persistent CTA pairs over 256-row tiles (tcgen05 cta_group::2, each CTA
  * streaming half of W1 per k-block, two accumulators so a tile's epilogue overlaps the
- * next tile's loads, each tile starting at a rotated k-block so that concurrent tiles
- * read different columns of their rows); off: one CTA per 128-row tile.  Both form the
- * same products; the pair kernel sums them in a rotated order, so s, z and bias agree to
- * fp32 rounding (each kernel is deterministic).  Read at each call.
+ * next tile's loads); off: one CTA per 128-row tile.  Both form the same products in the
+ * same order, so s, z and bias are identical.  Read at each call.
  * tg_set_scorer_pair: enable = 0 selects the one-CTA kernel; returns TG_OK.
  * tg_get_scorer_pair: the current setting (0 or 1). */
 int tg_set_scorer_pair(int enable);

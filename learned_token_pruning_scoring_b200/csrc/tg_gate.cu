@@ -10,8 +10,7 @@
 //   the row RMS, SiLU and the dot with w2, writes s[T] and the sum of s^2 over each
 //   32-row chunk.  Two kernels compute it: the CTA-pair scorer below (the default) and
 //   the one-CTA GEMM with its score epilogue (tg_gemm.cuh), selected by
-//   tg_set_scorer_pair.  The pair kernel starts each tile at a rotated k-block, so its
-//   fp32 sums run in another order than the one-CTA kernel's: the two agree to rounding.
+//   tg_set_scorer_pair; both give the same s bit for bit (same products, same order).
 // Kernel 2: per request, the chunk sums inside the request plus the ragged edge rows
 //   are reduced in a fixed order (every CTA of the request computes the identical
 //   total), then z = s / rms and bias = z on prunable tokens.
@@ -127,12 +126,6 @@ constexpr int kSpSS = kSpW2 + 1024;         // [2][128] row sums of squares
 constexpr int kSpBar = kSpSS + 1024;
 constexpr int kSpSmem = kSpBar + 256 + 1024;  // + alignment slack
 
-// First k-block of tile t: the tiles that run at the same time start at different
-// column offsets of their rows (7 is odd, so co-prime with the power-of-two block
-// counts), so that their h reads do not all fall on the same 128-byte slice of every
-// row at once; each tile still sums all k-blocks, in its own fixed order.
-__device__ __forceinline__ int k_rotation(int t, int nk) { return (int)(((int64_t)t * 7) % nk); }
-
 struct ScorerArgs {
   int64_t M;
   int K;
@@ -207,7 +200,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kSpThreads, 1)
       bool ok = true;
       for (int t = cluster; ok && t < n_tiles; t += n_clusters) {
         const int32_t m0 = (int32_t)((int64_t)t * 256 + rank * 128);
-        const int rot = k_rotation(t, nk);
         for (int kb = 0; kb < nk; ++kb, ++kg) {
           const int s = kg % kSpStages;
           const uint32_t ph = (uint32_t)(kg / kSpStages) & 1u;
@@ -216,10 +208,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kSpThreads, 1)
             break;
           }
           unsigned char* st = ring + s * kSpStageBytes;
-          const int kx = ((kb + rot) % nk) * kSpBK;
           if (rank == 0) mbar_arrive_expect_tx(&full[s], 2 * kSpStageBytes);
-          tma_load_2d_pair(st, &tmA, kx, m0, full_lead0 + s * 8);
-          tma_load_2d_pair(st + kSpABytes, &tmB, kx, (int32_t)rank * 128, full_lead0 + s * 8);
+          tma_load_2d_pair(st, &tmA, kb * kSpBK, m0, full_lead0 + s * 8);
+          tma_load_2d_pair(st + kSpABytes, &tmB, kb * kSpBK, (int32_t)rank * 128,
+                           full_lead0 + s * 8);
         }
       }
       // the even CTA waits until the last stages' bytes (both CTAs') have landed; the
