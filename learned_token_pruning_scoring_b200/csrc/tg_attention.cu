@@ -712,21 +712,26 @@ __global__ void __launch_bounds__(kThreads, 1)
               L = i == 0 ? wi * l_of(i) : fmaf(wi, l_of(i), L);
             }
             const float inv = 1.0f / L;
-            // column chunk by column chunk, the parts in order
+            // 16 columns at a time, the parts in order (small enough to keep the merge
+            // from taking registers the softmax loop needs)
 #pragma unroll 1
-            for (int c = 0; c < kD / 32; ++c) {
-              float acc[32];
+            for (int c = 0; c < kD / 16; ++c) {
+              float acc[16];
 #pragma unroll 1
               for (int i = 0; i < np; ++i) {
                 const float wgt = ex2_approx(m_of(i) - M);
-                float x[32];
+                float x[16];
                 if (i == it.part) {
-                  own_chunk(c, x);
+                  uint32_t ro[16];
+                  tmem_ld16(o_t + c * 16, ro);
+                  tmem_wait_ld();
+#pragma unroll
+                  for (int e = 0; e < 16; ++e) x[e] = __uint_as_float(ro[e]);
                 } else {
                   const float4* g4 = reinterpret_cast<const float4*>(blk(i, hh)) + rit;
 #pragma unroll
-                  for (int u = 0; u < 8; ++u) {
-                    const float4 v4 = __ldcg(g4 + (c * 8 + u) * kBM);
+                  for (int u = 0; u < 4; ++u) {
+                    const float4 v4 = __ldcg(g4 + (c * 4 + u) * kBM);
                     x[4 * u] = v4.x;
                     x[4 * u + 1] = v4.y;
                     x[4 * u + 2] = v4.z;
@@ -734,9 +739,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                   }
                 }
 #pragma unroll
-                for (int e = 0; e < 32; ++e) acc[e] = i == 0 ? wgt * x[e] : fmaf(wgt, x[e], acc[e]);
+                for (int e = 0; e < 16; ++e) acc[e] = i == 0 ? wgt * x[e] : fmaf(wgt, x[e], acc[e]);
               }
-              put_chunk(c, acc, inv);
+              if (row_valid) {
+                uint32_t wv[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) wv[e] = pack_bf16x2(acc[2 * e] * inv, acc[2 * e + 1] * inv);
+                uint4* dst = reinterpret_cast<uint4*>(p.o + (it.row0 + r) * p.ld_o + (int64_t)hh * kD + c * 16);
+                dst[0] = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+                dst[1] = make_uint4(wv[4], wv[5], wv[6], wv[7]);
+              }
             }
             store_lse(M, L);
           }
@@ -840,12 +852,14 @@ int make_plan(const int32_t* cu_kept_host, int batch, int head_groups, int sms, 
     // CTA (at most kMaxParts parts per tile).
     const double share = (double)units * head_groups / sms;
     int best = std::max(max_tiles, 1);
-    double best_cost = simulate_makespan(cu_kept_host, batch, head_groups, sms, best);
+    const double unsplit = simulate_makespan(cu_kept_host, batch, head_groups, sms, best);
+    // a split must shorten the estimate by a tenth to pay for its partials' traffic
+    double best_cost = 0.9 * unsplit;
     const int c_hi = std::min(max_tiles - 1, (int)std::ceil(3.0 * share) + 1);
     for (int c = 2; c <= c_hi; ++c) {
       if (ceil_div(max_tiles, c) > kMaxParts) continue;
       const double cost = simulate_makespan(cu_kept_host, batch, head_groups, sms, c);
-      if (cost < best_cost - 0.25) {  // a split must pay for its workspace traffic
+      if (cost < best_cost) {
         best_cost = cost;
         best = c;
       }
