@@ -444,7 +444,23 @@ size_t tg_gate_score_backward_workspace_size(int64_t total_tokens, int hidden, i
 int tg_linear(const tg_bf16* a, int64_t lda, const tg_bf16* w, int64_t ldw, tg_bf16* c,
               int64_t ldc, int64_t M, int N, int K, int rmsnorm_a, float eps,
               const tg_bf16* residual, int64_t ld_res, float* row_ssq_out,
-              int64_t ld_ssq_out, uint32_t* status, tg_stream_t stream);
+              int64_t ld_ssq_out, void* workspace, size_t workspace_bytes, uint32_t* status,
+              tg_stream_t stream);
+
+/*
+ * Workspace bytes that let the CTA-pair GEMM behind tg_linear, tg_qkv_rope_cache and
+ * tg_qkv_qknorm_rope_cache share its last round of 256 x 256 tiles along K over all
+ * clusters (stream-K tail): when the tiles leave that round partly idle, every cluster
+ * takes an equal run of the remaining k-blocks; the piece holding a tile's first k-block
+ * adds the others' fp32 partial sums in k order before its epilogue (so the result is
+ * deterministic; it differs from the unsplit call only by fp32 summation order), and the
+ * launch is cooperative.  Those calls take (workspace, workspace_bytes): NULL or fewer
+ * bytes runs unsplit.  Zero-fill the workspace once before its first use (its ready
+ * flags); every completed call leaves it so; calls whose GPU work can overlap must not
+ * share one.  The size depends only on the device (its number of SM pairs: partial sums
+ * of 256 KB per cluster plus the flags).  Not part of the method: a scheduling device.
+ */
+size_t tg_gemm_workspace_size(void);
 
 /*
  * One gated layer's QKV projection with RoPE and the compacted KV-cache write fused into
@@ -471,7 +487,8 @@ int tg_qkv_rope_cache(const tg_bf16* x, int64_t ld_x, const tg_bf16* w_qkv, int6
                       float eps, const int32_t* pos, const float* cos_sin, int max_pos,
                       tg_bf16* q_out, int64_t ld_q, tg_bf16* cache_k, tg_bf16* cache_v,
                       int64_t ld_cache, int64_t slot_offset, const float* row_ssq_in,
-                      int64_t ld_ssq_in, uint32_t* status, tg_stream_t stream);
+                      int64_t ld_ssq_in, void* workspace, size_t workspace_bytes,
+                      uint32_t* status, tg_stream_t stream);
 
 /*
  * tg_qkv_rope_cache with QK-norm, for a full (Qwen3-shaped) layer body: each Q and K
@@ -491,8 +508,8 @@ int tg_qkv_qknorm_rope_cache(const tg_bf16* x, int64_t ld_x, const tg_bf16* w_qk
                              const float* k_norm_w, const int32_t* pos, const float* cos_sin,
                              int max_pos, tg_bf16* q_out, int64_t ld_q, tg_bf16* cache_k,
                              tg_bf16* cache_v, int64_t ld_cache, int64_t slot_offset,
-                             const float* row_ssq_in, int64_t ld_ssq_in, uint32_t* status,
-                             tg_stream_t stream);
+                             const float* row_ssq_in, int64_t ld_ssq_in, void* workspace,
+                             size_t workspace_bytes, uint32_t* status, tg_stream_t stream);
 
 /*
  * Up half of the SwiGLU MLP of a full layer body (pruned tokens skip the upper MLPs as

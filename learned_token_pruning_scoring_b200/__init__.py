@@ -27,6 +27,7 @@ __all__ = [
     "tg_gate_score_noalloc", "tg_seq_rmsnorm", "tg_gather_rope", "tg_kv_compact", "tg_gated_attention", "tg_linear",
     "tg_status_clear", "tg_status_read", "tg_set_launch_overlap", "tg_get_launch_overlap",
     "tg_set_gather_tma", "tg_get_gather_tma", "tg_set_scorer_pair", "tg_get_scorer_pair",
+    "tg_gemm_workspace_size",
     "tg_prefetch_l2", "tg_out_proj_qkv_next", "tg_out_proj_qkv_workspace_size",
     "tg_swiglu", "tg_fold_norm_weight", "tg_pack_gate_up", "prepare_layer",
     "tg_gated_attention_bias_grad", "tg_gated_attention_bias_grad_workspace_size",
@@ -390,8 +391,22 @@ def tg_gate_score_backward(h, W1, w2, s, cu_seqlens, cu_seqlens_host, prunable, 
         _count(6 + (1 if int(ckh[-1]) > 0 else 0) + (1 if norm_w is not None else 0))
     return ds_out, dW1, dw2, dnorm_w
 
+def tg_gemm_workspace_size() -> int:
+    """Bytes of the stream-K workspace the CTA-pair GEMMs may use (see the header)."""
+    return int(lib.tg_gemm_workspace_size())
+
+
+def _ws(workspace):
+    if workspace is None or workspace.numel() == 0:
+        return None, 0
+    return _ptr(workspace), workspace.numel() * workspace.element_size()
+
+
 def tg_linear(a, w, c=None, rmsnorm=False, eps=1e-6, residual=None, row_ssq=None, status=None,
-              stream=None):
+              stream=None, workspace=None):
+    """c = (RMSNorm(a)) w^T (+ residual).  `workspace`: a zero-filled uint8 tensor of
+    tg_gemm_workspace_size() bytes lets the CTA-pair GEMM split its last round of tiles
+    along K (left zeroed by every call)."""
     lda, ldw = _mat(a, "a"), _mat(w, "w")
     M, K = a.shape
     N = w.shape[0]
@@ -400,9 +415,10 @@ def tg_linear(a, w, c=None, rmsnorm=False, eps=1e-6, residual=None, row_ssq=None
     ldc = _mat(c, "c")
     ldr = _mat(residual, "residual") if residual is not None else 0
     ld_ssq = _mat(row_ssq, "row_ssq") if row_ssq is not None else 0
+    ws_ptr, ws_bytes = _ws(workspace)
     rc = lib.tg_linear(_ptr(a), lda, _ptr(w), ldw, _ptr(c), ldc, M, N, K, 1 if rmsnorm else 0,
-                       float(eps), _ptr(residual), ldr, _ptr(row_ssq), ld_ssq, _ptr(status),
-                       _stream(stream))
+                       float(eps), _ptr(residual), ldr, _ptr(row_ssq), ld_ssq, ws_ptr, ws_bytes,
+                       _ptr(status), _stream(stream))
     _check(rc, "tg_linear")
     _count()
     return c
@@ -410,7 +426,7 @@ def tg_linear(a, w, c=None, rmsnorm=False, eps=1e-6, residual=None, row_ssq=None
 
 def tg_qkv_rope_cache(x, w_qkv, pos, cos_sin, cache_k, cache_v, n_q_heads, n_kv_heads,
                       q_out=None, head_dim=128, eps=1e-6, slot_offset=0, row_ssq=None,
-                      status=None, stream=None, q_norm_w=None, k_norm_w=None):
+                      status=None, stream=None, q_norm_w=None, k_norm_w=None, workspace=None):
     """Fused QKV projection (RMSNorm folded) + RoPE at `pos` + compacted KV-cache write;
     with q_norm_w / k_norm_w (float32 [head_dim]) also QK-norm before RoPE
     (tg_qkv_qknorm_rope_cache)."""
@@ -423,20 +439,22 @@ def tg_qkv_rope_cache(x, w_qkv, pos, cos_sin, cache_k, cache_v, n_q_heads, n_kv_
     if _mat(cache_v, "cache_v") != ld_c:
         raise ValueError("cache_k and cache_v must share a row stride")
     ld_ssq = _mat(row_ssq, "row_ssq") if row_ssq is not None else 0
+    ws_ptr, ws_bytes = _ws(workspace)
     if q_norm_w is not None or k_norm_w is not None:
         rc = lib.tg_qkv_qknorm_rope_cache(_ptr(x), ld_x, _ptr(w_qkv), ld_w, M, hidden, n_q_heads,
                                           n_kv_heads, head_dim, float(eps), _ptr(q_norm_w),
                                           _ptr(k_norm_w), _ptr(pos), _ptr(cos_sin),
                                           cos_sin.shape[0], _ptr(q_out), ld_q, _ptr(cache_k),
                                           _ptr(cache_v), ld_c, int(slot_offset), _ptr(row_ssq),
-                                          ld_ssq, _ptr(status), _stream(stream))
+                                          ld_ssq, ws_ptr, ws_bytes, _ptr(status),
+                                          _stream(stream))
         _check(rc, "tg_qkv_qknorm_rope_cache")
     else:
         rc = lib.tg_qkv_rope_cache(_ptr(x), ld_x, _ptr(w_qkv), ld_w, M, hidden, n_q_heads,
                                    n_kv_heads, head_dim, float(eps), _ptr(pos), _ptr(cos_sin),
                                    cos_sin.shape[0], _ptr(q_out), ld_q, _ptr(cache_k),
                                    _ptr(cache_v), ld_c, int(slot_offset), _ptr(row_ssq), ld_ssq,
-                                   _ptr(status), _stream(stream))
+                                   ws_ptr, ws_bytes, _ptr(status), _stream(stream))
         _check(rc, "tg_qkv_rope_cache")
     _count()
     return q_out
@@ -557,7 +575,8 @@ def _mlp(L, x, P, eps, status, stream, mark):
     h = P["ffn"][:, :L.ffn]
     tg_swiglu(x, L.W_gu, P["ssq"], h_out=h, eps=eps, status=status, stream=stream)
     mark("mlp_gate_up")
-    tg_linear(h, L.W_down, x, residual=x, row_ssq=P["ssq"], status=status, stream=stream)
+    tg_linear(h, L.W_down, x, residual=x, row_ssq=P["ssq"], status=status, stream=stream,
+              workspace=P.get("gemm_ws"))
     mark("mlp_down")
 
 
@@ -618,6 +637,7 @@ class FullContextLayers:
             caches=[(torch.empty((T, self.hkv * self.d), **bf),
                      torch.empty((T, self.hkv * self.d), **bf)) for _ in self.layers],
             ffn=torch.empty((T, max([L.ffn for L in self.layers] + [0])), **bf),
+            gemm_ws=torch.zeros(tg_gemm_workspace_size(), dtype=torch.uint8, device=dev),
         )
         return self.planned
 
@@ -633,14 +653,15 @@ class FullContextLayers:
             tg_qkv_rope_cache(x, L.Wqkv, P["pos"], self.cos_sin, ck, cv, self.hq, self.hkv,
                               q_out=qkv[:, :nq], head_dim=self.d, eps=self.norm_eps,
                               row_ssq=P["ssq"], status=self.status, stream=stream,
-                              q_norm_w=L.q_norm, k_norm_w=L.k_norm)
+                              q_norm_w=L.q_norm, k_norm_w=L.k_norm, workspace=P["gemm_ws"])
             self._mark("qkv_rope_cache")
             tg_gated_attention(qkv[:, :nq], ck, cv, P["cu"], P["cu_h"], self.hq, self.hkv,
                                P["pos"], P["bias"], P["gamma"], 1.0, o=o, head_dim=self.d,
                                workspace=P["attn_ws"], status=self.status, stream=stream)
             self._mark("attention")
             tg_linear(o, L.Wo, x, residual=x, row_ssq=P["ssq"], status=self.status,
-                      stream=stream)
+                      stream=stream,
+                      workspace=P["gemm_ws"])
             self._mark("out_proj")
             _mlp(L, x, P, self.norm_eps, self.status, stream, self._mark)
         return x
@@ -710,6 +731,8 @@ class GatedPrefill:
         # in the first round, so the QKV tiles gain nothing by starting in the same
         # launch (measured equal to two launches); off by default.
         self.fuse_boundaries = False
+        # share the projections' last round of tiles along K over all CTA pairs (stream-K)
+        self.split_gemm = True
         self._qkv_done = -1  # index of the layer whose QKV already ran in a fused launch
 
     def _mark(self, name):
@@ -751,6 +774,9 @@ class GatedPrefill:
                      torch.empty((K, self.hkv * self.d), **bf)) for _ in self.layers],
             chain_ws=torch.zeros(max(16, tg_out_proj_qkv_workspace_size(K)), dtype=torch.uint8,
                                  device=dev),
+            # stream-K tail of the projections (zero-filled; empty = unsplit)
+            gemm_ws=torch.zeros(tg_gemm_workspace_size() if self.split_gemm else 0,
+                                dtype=torch.uint8, device=dev),
             ffn=torch.empty((K, max([L.ffn for L in self.layers] + [0])), **bf),
         )
         if self.lower is not None:
@@ -807,7 +833,7 @@ class GatedPrefill:
             tg_qkv_rope_cache(x, L.Wqkv, P["kept_pos"], self.cos_sin, ck, cv, self.hq, self.hkv,
                               q_out=qkv[:, :nq], head_dim=self.d, eps=self.norm_eps,
                               row_ssq=P["ssq"], status=self.status, stream=stream,
-                              q_norm_w=L.q_norm, k_norm_w=L.k_norm)
+                              q_norm_w=L.q_norm, k_norm_w=L.k_norm, workspace=P["gemm_ws"])
             self._mark("qkv_rope_cache")
         else:
             tg_linear(x, L.Wqkv, qkv, rmsnorm=True, eps=self.norm_eps, status=self.status,
@@ -843,7 +869,8 @@ class GatedPrefill:
             self._qkv_done = i + 1
             self._mark("out_proj_qkv")
         else:
-            tg_linear(o, L.Wo, x, residual=x, row_ssq=P["ssq"], status=self.status, stream=stream)
+            tg_linear(o, L.Wo, x, residual=x, row_ssq=P["ssq"], status=self.status, stream=stream,
+                      workspace=P["gemm_ws"])
             self._mark("out_proj")
         _mlp(L, x, P, self.norm_eps, self.status, stream, self._mark)
 

@@ -49,10 +49,11 @@ SIGNATURES = {
                                   _p, _p, _p, _f32, _p, _i64, _p, _p, _sz, _p, _p]),
     "tg_gated_attention_workspace_size": (_sz, [_p, _i32, _i32, _i32, _i32]),
     "tg_qkv_rope_cache": (_i32, [_p, _i64, _p, _i64, _i64, _i32, _i32, _i32, _i32, _f32, _p, _p,
-                                 _i32, _p, _i64, _p, _p, _i64, _i64, _p, _i64, _p, _p]),
+                                 _i32, _p, _i64, _p, _p, _i64, _i64, _p, _i64, _p, _sz, _p, _p]),
     "tg_qkv_qknorm_rope_cache": (_i32, [_p, _i64, _p, _i64, _i64, _i32, _i32, _i32, _i32, _f32,
                                         _p, _p, _p, _p, _i32, _p, _i64, _p, _p, _i64, _i64,
-                                        _p, _i64, _p, _p]),
+                                        _p, _i64, _p, _sz, _p, _p]),
+    "tg_gemm_workspace_size": (_sz, []),
     "tg_gated_attention_bias_grad": (_i32, [_p, _i64, _p, _i64, _p, _i64, _p, _i64, _p, _i64,
                                             _p, _p, _p, _i32, _i32, _i32, _i32, _p, _p, _p,
                                             _f32, _p, _p, _p, _p, _sz, _p, _p]),
@@ -70,7 +71,7 @@ SIGNATURES = {
                                      _p, _p, _i64, _i64, _p, _sz, _p, _p]),
     "tg_out_proj_qkv_workspace_size": (_sz, [_i64]),
     "tg_linear": (_i32, [_p, _i64, _p, _i64, _p, _i64, _i64, _i32, _i32, _i32, _f32, _p, _i64,
-                         _p, _i64, _p, _p]),
+                         _p, _i64, _p, _sz, _p, _p]),
 }
 
 

@@ -395,14 +395,38 @@ __device__ __forceinline__ uint32_t sw128_chunk(int r, int k) {
   return (uint32_t)(r * 128 + ((k ^ (r & 7)) << 4));
 }
 
+// Stream-K fixup: add the other pieces' fp32 partial sums (in k order) to 32 accumulator
+// columns just read from TMEM; `chunk` is the 32-column piece within the epilogue group's
+// 128 columns, adds[k] already points at this thread's row.
+template <int MAXADD>
+__device__ __forceinline__ void add_partials(uint32_t (&r)[32], int chunk,
+                                             const float4* const (&adds)[MAXADD], int n_add) {
+#pragma unroll
+  for (int k = 0; k < MAXADD; ++k) {
+    if (k < n_add) {
+      const float4* pp = adds[k] + chunk * 8 * 128;
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const float4 v = __ldcg(pp + u * 128);
+        r[4 * u] = __float_as_uint(__uint_as_float(r[4 * u]) + v.x);
+        r[4 * u + 1] = __float_as_uint(__uint_as_float(r[4 * u + 1]) + v.y);
+        r[4 * u + 2] = __float_as_uint(__uint_as_float(r[4 * u + 2]) + v.z);
+        r[4 * u + 3] = __float_as_uint(__uint_as_float(r[4 * u + 3]) + v.w);
+      }
+    }
+  }
+}
+
 // Columns [128 h, 128 h + 128) of one 256 x 256 output tile of the pair (each CTA: 128
 // rows, staged in shared memory as four swizzled 64-column boxes); `row` is the thread's
 // row in the CTA's half, `tacc` the TMEM address of the row's accumulator (lane quarter
 // and buffer included).
-template <int EPI>
+template <int EPI, int MAXADD>
 __device__ __forceinline__ void pair_epilogue_half(const GemmParams& p, unsigned char* out_s,
                                                    uint32_t tacc, int row, int64_t grow, int n0,
-                                                   int h, bool has_res) {
+                                                   int h, bool has_res,
+                                                   const float4* const (&adds)[MAXADD],
+                                                   int n_add) {
   const bool live = grow < p.M;
   const float rscale =
       (p.rmsnorm && p.row_ssq_in && live) ? rscale_from_ssq(p, grow) : 1.0f;
@@ -426,6 +450,7 @@ __device__ __forceinline__ void pair_epilogue_half(const GemmParams& p, unsigned
         uint32_t r[32];
         tmem_ld32(tacc + (4 * h + c) * 32, r);
         tmem_wait_ld();
+        add_partials(r, c, adds, n_add);
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
           const float v = __uint_as_float(r[i]);
@@ -443,6 +468,8 @@ __device__ __forceinline__ void pair_epilogue_half(const GemmParams& p, unsigned
       tmem_ld32(tacc + ca * 32, ra);
       tmem_ld32(tacc + cb * 32, rb);
       tmem_wait_ld();
+      add_partials(ra, pr, adds, n_add);
+      add_partials(rb, pr + 2, adds, n_add);
       unsigned char* box_a = out_s + (ca >> 1) * PairCfg<1>::BOX_BYTES;
       unsigned char* box_b = out_s + (cb >> 1) * PairCfg<1>::BOX_BYTES;
       const float4* cs = cs_row + (ca & 3) * 16;  // (cos, sin) pairs of i = (ca & 3) * 32 ..
@@ -493,6 +520,8 @@ __device__ __forceinline__ void pair_epilogue_half(const GemmParams& p, unsigned
       tmem_ld32(tacc + 128 * h + 32 * c, rg);
       tmem_ld32(tacc + 128 * h + 64 + 32 * c, ru);
       tmem_wait_ld();
+      add_partials(rg, c, adds, n_add);
+      add_partials(ru, c + 2, adds, n_add);
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
         uint32_t w[4];
@@ -516,6 +545,8 @@ __device__ __forceinline__ void pair_epilogue_half(const GemmParams& p, unsigned
     tmem_ld32(tacc + j * 64, ra);
     tmem_ld32(tacc + j * 64 + 32, rb);
     tmem_wait_ld();
+    add_partials(ra, 2 * (j - 2 * h), adds, n_add);
+    add_partials(rb, 2 * (j - 2 * h) + 1, adds, n_add);
     unsigned char* box = out_s + j * PairCfg<1>::BOX_BYTES;
 #pragma unroll
     for (int k = 0; k < 8; ++k) {
@@ -568,6 +599,64 @@ struct PairChain {
   int target;
 };
 
+// Stream-K tail of a single-job launch.  The first dp_tiles tiles (whole rounds of the
+// clusters) run whole, tile t on cluster t mod C; the k-blocks of the remaining tiles are
+// shared out evenly, in tile order, as one contiguous range of tail_units per cluster
+// ("pieces").  A piece holding a tile's first k-block finishes that tile: it runs last
+// in its cluster, waits for the tile's other pieces (each the first piece of a later
+// cluster, run first there), adds their fp32 partial sums in k order to its own
+// accumulator and runs the epilogue; the other pieces only publish their partial sums.
+// A cluster has at most one such contributing piece, so partials and ready flags are
+// indexed by cluster: part[((c * 2 + rank) * 2 + group) * 32 * 128 + f * 128 + row]
+// (float4, f = 4-column group within the epilogue group's 128 columns) and
+// flag[(c * 2 + rank) * 2 + group].  Every cluster must be resident at once: the launch
+// is cooperative.  part == nullptr: no split.
+struct PairSplit {
+  float4* part;
+  int* flag;
+  int dp_tiles;
+  int64_t tail_units;
+};
+constexpr int kMaxPieces = 8;  // pieces per split tile (the host keeps ranges long enough)
+
+struct Piece {
+  int t, kb0, kb1;
+  int kind;  // 0: whole tile, 1: finisher (first k-blocks), 2: contributor
+};
+
+// The pieces of cluster c in the order the cluster runs them.
+struct PieceIter {
+  int c, C, n_tiles, nk, dp_tiles;
+  int64_t u, u1;
+  int i;
+  bool split;
+  __device__ PieceIter(int c_, int C_, int n_tiles_, int nk_, const PairSplit& sp)
+      : c(c_), C(C_), n_tiles(n_tiles_), nk(nk_), dp_tiles(0), u(0), u1(0), i(0),
+        split(sp.part != nullptr) {
+    if (split) {
+      dp_tiles = sp.dp_tiles;
+      u = sp.tail_units * c / C;
+      u1 = sp.tail_units * (c + 1) / C;
+    }
+  }
+  __device__ bool next(Piece& pc) {
+    const int t = c + i * C;
+    if (!split ? t < n_tiles : t < dp_tiles) {
+      pc = {t, 0, nk, 0};
+      ++i;
+      return true;
+    }
+    if (!split || u >= u1) return false;
+    const int tt = (int)(u / nk);
+    const int kb0 = (int)(u % nk);
+    const int64_t left = u1 - u;
+    const int kb1 = left < (int64_t)(nk - kb0) ? kb0 + (int)left : nk;
+    pc = {dp_tiles + tt, kb0, kb1, kb0 == 0 ? (kb1 == nk ? 0 : 1) : 2};
+    u += kb1 - kb0;
+    return true;
+  }
+};
+
 // Persistent CTA-pair GEMM: each cluster of two CTAs walks the 256 x 256 output tiles
 // t = cluster, cluster + clusters, ... of job 0 and then of job 1 (tiles of job 1 follow
 // all of job 0's in that order, so a job-1 tile only ever waits for job-0 tiles that
@@ -587,7 +676,7 @@ struct PairChain {
 template <int STAGES, int EPI0, int EPI1>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(320, 1)
     gemm_pair_kernel(const __grid_constant__ PairJob job0, const __grid_constant__ PairJob job1,
-                     PairChain chain) {
+                     PairChain chain, PairSplit split) {
   using Cfg = PairCfg<STAGES>;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>(
@@ -661,7 +750,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(320, 1)
       griddep_wait();
       int kg = 0;
       bool ok = true;
-      for (int t = cluster; ok && t < n_tiles; t += n_clusters) {
+      PieceIter pit(cluster, n_clusters, n_tiles, job0.p.K / Cfg::BK, split);
+      Piece pc;
+      while (ok && pit.next(pc)) {
+        const int t = pc.t;
         int job, rp, n0;
         decode(t, job, rp, n0);
         const PairJob& jb = job ? job1 : job0;
@@ -677,7 +769,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(320, 1)
         const int64_t m0 = (int64_t)rp * 256 + rank * 128;
         const int nb = n0 + (int)rank * (Cfg::BN / 2);
         const int nk = jb.p.K / Cfg::BK;
-        for (int kb = 0; kb < nk; ++kb, ++kg) {
+        const int kb_end = job ? nk : pc.kb1;
+        for (int kb = job ? 0 : pc.kb0; kb < kb_end; ++kb, ++kg) {
           const int s = kg % STAGES;
           const uint32_t ph = (uint32_t)(kg / STAGES) & 1u;
           if (!mbar_wait(&empty[s], ph ^ 1u, abort_flag, status)) {
@@ -703,14 +796,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(320, 1)
       const uint32_t acc_full_peer0 = mapa_shared(smem_u32(&acc_full[0]), 1);
       int kg = 0, i = 0;
       bool ok = true;
-      for (int t = cluster; ok && t < n_tiles; t += n_clusters, ++i) {
+      PieceIter pit(cluster, n_clusters, n_tiles, job0.p.K / Cfg::BK, split);
+      Piece pc;
+      for (; ok && pit.next(pc); ++i) {
+        const int t = pc.t;
         const int b = i & 1;
-        const int nk = (t >= n_tiles0 ? job1.p.K : job0.p.K) / Cfg::BK;
+        const bool j1 = t >= n_tiles0;
+        const int kb_begin = j1 ? 0 : pc.kb0;
+        const int kb_end = j1 ? job1.p.K / Cfg::BK : pc.kb1;
         // both CTAs' epilogues are done with this buffer (first use passes at once)
         if (!mbar_wait(&acc_empty[b], ((uint32_t)(i >> 1) & 1u) ^ 1u, abort_flag, status)) break;
         tc_fence_after();
         const uint32_t d = tmem + (uint32_t)(b * Cfg::BN);
-        for (int kb = 0; kb < nk; ++kb, ++kg) {
+        for (int kb = kb_begin; kb < kb_end; ++kb, ++kg) {
           const int s = kg % STAGES;
           const uint32_t ph = (uint32_t)(kg / STAGES) & 1u;
           if (!mbar_wait(&full[s], ph, abort_flag, status)) {
@@ -723,7 +821,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(320, 1)
 #pragma unroll
           for (int k = 0; k < Cfg::BK / 16; ++k)
             mma_ss_pair(d, sw128_desc(a_addr + k * 32, 16, 1024),
-                        sw128_desc(b_addr + k * 32, 16, 1024), idesc, (kb | k) != 0);
+                        sw128_desc(b_addr + k * 32, 16, 1024), idesc,
+                        (kb != kb_begin || k != 0) ? 1u : 0u);
           mma_commit_pair(smem_u32(&empty[s]));
           mma_commit_pair(empty_peer0 + s * 8);
         }
@@ -759,18 +858,45 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(320, 1)
       decode(t, job, rp, n0);
       return has_res(job);
     };
-    if (elected && cluster < n_tiles && res_of(cluster)) load_res(cluster);
+    PieceIter pit(cluster, n_clusters, n_tiles, job0.p.K / Cfg::BK, split);
+    PieceIter peek = pit;  // one piece ahead: the residual of the next piece loads early
+    Piece pc, nx;
+    bool has_next = peek.next(nx);
+    auto needs_res = [&](const Piece& q) { return q.kind != 2 && res_of(q.t); };
+    if (elected && has_next && needs_res(nx)) load_res(nx.t);
+    const int nk0 = job0.p.K / Cfg::BK;
     int i = 0, res_used = 0;
-    for (int t = cluster; t < n_tiles; t += n_clusters, ++i) {
+    for (; pit.next(pc); ++i) {
+      has_next = peek.next(nx);  // nx: the piece after pc
+      const int t = pc.t;
       const int b = i & 1;
       int job, rp, n0;
       decode(t, job, rp, n0);
       const PairJob& jb = job ? job1 : job0;
-      const bool with_res = has_res(job);
+      const bool with_res = pc.kind != 2 && has_res(job);
       const int64_t m0 = (int64_t)rp * 256 + rank * 128;
       bool ok = mbar_wait(&acc_full[b], (uint32_t)(i >> 1) & 1u, abort_flag, status);
       if (ok && with_res) ok = mbar_wait(&res_full[g], (uint32_t)res_used & 1u, abort_flag, status);
       if (with_res) ++res_used;
+      // a finisher adds the partial sums of the tile's other pieces: the clusters whose
+      // tail ranges start inside this tile, in k order
+      const float4* adds[kMaxPieces];
+      int add_cl[kMaxPieces];
+      int n_add = 0;
+      if (pc.kind == 1) {
+        const int64_t lo = (int64_t)(t - split.dp_tiles) * nk0, hi = lo + nk0;
+        for (int c2 = cluster + 1; c2 < n_clusters && n_add < kMaxPieces; ++c2) {
+          const int64_t b2 = split.tail_units * c2 / n_clusters;
+          if (b2 >= hi) break;
+          if (b2 > lo) {
+            add_cl[n_add] = c2;
+            adds[n_add++] = split.part + (int64_t)((c2 * 2 + (int)rank) * 2 + g) * 32 * 128 + row;
+          }
+        }
+        if (elected)
+          for (int k = 0; k < n_add && ok; ++k)
+            ok = wait_flag_gpu(split.flag + (add_cl[k] * 2 + (int)rank) * 2 + g, abort_flag, status);
+      }
       // job 1 reads job 0's row sums of squares: its producer acquired job 0's release
       // before the loads behind this accumulator; a device fence orders this thread's
       // reads after it too (the counter itself may already be reset by then)
@@ -779,10 +905,41 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(320, 1)
       if (!named_bar_and(bar_id, 128, ok)) break;
       tc_fence_after();
       const uint32_t tacc = tmem + (uint32_t)(b * Cfg::BN) + ((uint32_t)(q * 32) << 16);
+      if (pc.kind == 2) {
+        // contributor: the group's 128 raw accumulator columns go to this cluster's
+        // partial block (float4 per 4 columns, row-contiguous: coalesced)
+        float4* dst = split.part + (int64_t)((cluster * 2 + (int)rank) * 2 + g) * 32 * 128 + row;
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          uint32_t r[32];
+          tmem_ld32(tacc + (4 * g + c) * 32, r);
+          tmem_wait_ld();
+#pragma unroll
+          for (int u = 0; u < 8; ++u)
+            dst[(c * 8 + u) * 128] =
+                make_float4(__uint_as_float(r[4 * u]), __uint_as_float(r[4 * u + 1]),
+                            __uint_as_float(r[4 * u + 2]), __uint_as_float(r[4 * u + 3]));
+        }
+        __threadfence();  // this thread's part is visible GPU-wide before the flag
+        tc_fence_before();
+        named_bar_sync(bar_id, 128);
+        if (elected) {
+          if (rank == 0)
+            mbar_arrive(&acc_empty[b]);
+          else
+            mbar_arrive_cluster(acc_empty_lead0 + b * 8);
+          st_release_gpu(split.flag + (cluster * 2 + (int)rank) * 2 + g, 1);
+          if (has_next && needs_res(nx)) load_res(nx.t);
+        }
+        named_bar_sync(bar_id, 128);
+        continue;
+      }
       if (job)
-        pair_epilogue_half<EPI1>(jb.p, out_s, tacc, row, m0 + row, n0, g, with_res);
+        pair_epilogue_half<EPI1, kMaxPieces>(jb.p, out_s, tacc, row, m0 + row, n0, g, with_res,
+                                             adds, n_add);
       else
-        pair_epilogue_half<EPI0>(jb.p, out_s, tacc, row, m0 + row, n0, g, with_res);
+        pair_epilogue_half<EPI0, kMaxPieces>(jb.p, out_s, tacc, row, m0 + row, n0, g, with_res,
+                                             adds, n_add);
       const bool publish = !job && chain.ready;  // job 1 waits for these rows
       if (publish) __threadfence();  // row sums of squares visible before the count
       tc_fence_before();
@@ -793,6 +950,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(320, 1)
           mbar_arrive(&acc_empty[b]);
         else
           mbar_arrive_cluster(acc_empty_lead0 + b * 8);
+        // every thread of the group has read the partials: leave the flags at zero
+        for (int k = 0; k < n_add; ++k) split.flag[(add_cl[k] * 2 + (int)rank) * 2 + g] = 0;
         int mi = 0, x = n0;
         const int epi = job ? EPI1 : EPI0;
         if (epi == EpiQKV || epi == EpiQKVNorm) {
@@ -817,7 +976,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(320, 1)
         } else {
           bulk_wait_read_all();  // the group's staging boxes may be overwritten from here on
         }
-        if (t + n_clusters < n_tiles && res_of(t + n_clusters)) load_res(t + n_clusters);
+        if (has_next && needs_res(nx)) load_res(nx.t);
       }
       named_bar_sync(bar_id, 128);
     }

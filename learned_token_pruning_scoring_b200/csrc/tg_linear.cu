@@ -26,8 +26,43 @@ int launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const GemmParams& 
                 p);
 }
 
+// Stream-K workspace: the partial sums of one contributing piece per cluster (two CTAs x
+// two epilogue groups x 128 rows x 128 fp32 columns) and its ready flags.
+size_t split_part_bytes(int clusters) { return (size_t)clusters * 4 * 32 * 128 * sizeof(float4); }
+size_t split_workspace_bytes(int clusters) {
+  return split_part_bytes(clusters) + (((size_t)clusters * 4 * sizeof(int) + 255) & ~size_t(255));
+}
+
+// Whether to share the last round's tiles along K (stream-K tail), and how.  The plain
+// persistent launch runs ceil(tiles / C) rounds of nk k-blocks; the split one runs the
+// whole rounds and then tail_units / C k-blocks per cluster plus the fixup (estimated at
+// kSplitFixup k-blocks).  Split when that saves at least 7%, no tile has more than
+// kMaxPieces pieces, and the caller gave a large enough workspace.
+constexpr double kSplitFixup = 3.0;
+PairSplit plan_split(int64_t tiles, int nk, int clusters, void* ws, size_t ws_bytes) {
+  PairSplit sp{nullptr, nullptr, 0, 0};
+  if (!ws || ws_bytes < split_workspace_bytes(clusters) || clusters < 2) return sp;
+  const int64_t rounds = tiles / clusters;
+  const int64_t tail = tiles - rounds * clusters;
+  if (tail == 0) return sp;
+  const int64_t tail_units = tail * nk;
+  const int64_t per = tail_units / clusters;
+  if (per < 1 || per * (kMaxPieces - 1) < nk) return sp;
+  const double plain = (double)((tiles + clusters - 1) / clusters) * nk;
+  const double split = (double)rounds * nk + (double)(tail_units + clusters - 1) / clusters +
+                       kSplitFixup;
+  if (split > 0.93 * plain) return sp;
+  unsigned char* w = static_cast<unsigned char*>(ws);
+  sp.part = reinterpret_cast<float4*>(w);
+  sp.flag = reinterpret_cast<int*>(w + split_part_bytes(clusters));
+  sp.dp_tiles = (int)(rounds * clusters);
+  sp.tail_units = tail_units;
+  return sp;
+}
+
 template <int STAGES, int EPI>
-int launch_pair(const PairMaps& maps, const GemmParams& p, cudaStream_t stream) {
+int launch_pair(const PairMaps& maps, const GemmParams& p, cudaStream_t stream,
+                void* ws = nullptr, size_t ws_bytes = 0) {
   using Cfg = PairCfg<STAGES>;
   auto kern = gemm_pair_kernel<STAGES, EPI, EPI>;
   static int attr_dev = -1;
@@ -41,9 +76,33 @@ int launch_pair(const PairMaps& maps, const GemmParams& p, cudaStream_t stream) 
   j1.p.M = 0;  // no second job
   // persistent: at most one cluster (two CTAs) per SM pair, each walking its tiles
   const int64_t tiles = ((p.M + 255) / 256) * (p.N / Cfg::BN);
-  const int64_t clusters = std::min<int64_t>(tiles, std::max(1, sm_count() / 2));
-  return launch(kern, dim3((unsigned)(2 * clusters)), dim3(Cfg::THREADS), Cfg::SMEM, stream, j0,
-                j1, PairChain{nullptr, nullptr, 0});
+  const int all_clusters = std::max(1, sm_count() / 2);
+  const PairSplit sp = plan_split(tiles, p.K / Cfg::BK, all_clusters, ws, ws_bytes);
+  if (!sp.part) {
+    const int64_t clusters = std::min<int64_t>(tiles, all_clusters);
+    return launch(kern, dim3((unsigned)(2 * clusters)), dim3(Cfg::THREADS), Cfg::SMEM, stream,
+                  j0, j1, PairChain{nullptr, nullptr, 0}, sp);
+  }
+  // a finishing piece waits for pieces of other clusters: all must be resident at once
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(2 * all_clusters));
+  cfg.blockDim = dim3(Cfg::THREADS);
+  cfg.dynamicSmemBytes = Cfg::SMEM;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = launch_overlap() ? 1 : 0;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  const cudaError_t e =
+      cudaLaunchKernelEx(&cfg, kern, j0, j1, PairChain{nullptr, nullptr, 0}, sp);
+  if (e != cudaSuccess) {
+    set_cuda_error(e);
+    return TG_ERR_CUDA;
+  }
+  return TG_OK;
 }
 
 // Two chained jobs in one persistent launch (job 1 reads rows job 0 writes).  Every
@@ -76,7 +135,7 @@ int launch_pair_chain(const PairJob& j0, const PairJob& j1, const PairChain& cha
   attr[1].val.programmaticStreamSerializationAllowed = launch_overlap() ? 1 : 0;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
-  TG_CUDA_TRY(cudaLaunchKernelEx(&cfg, kern, j0, j1, chain));
+  TG_CUDA_TRY(cudaLaunchKernelEx(&cfg, kern, j0, j1, chain, PairSplit{nullptr, nullptr, 0, 0}));
   return TG_OK;
 }
 
@@ -249,7 +308,8 @@ using namespace tg;
 extern "C" int tg_linear(const tg_bf16* a, int64_t lda, const tg_bf16* w, int64_t ldw, tg_bf16* c,
                          int64_t ldc, int64_t M, int N, int K, int rmsnorm_a, float eps,
                          const tg_bf16* residual, int64_t ld_res, float* row_ssq_out,
-                         int64_t ld_ssq_out, uint32_t* status, tg_stream_t stream) {
+                         int64_t ld_ssq_out, void* workspace, size_t workspace_bytes,
+                         uint32_t* status, tg_stream_t stream) {
   if (M < 0 || N <= 0 || K <= 0 || (N % 128) || (K % 64)) return TG_ERR_UNSUPPORTED_SHAPE;
   if (M == 0) return TG_OK;
   if (!a || !w || !c) return TG_ERR_INVALID_ARGUMENT;
@@ -268,7 +328,8 @@ extern "C" int tg_linear(const tg_bf16* a, int64_t lda, const tg_bf16* w, int64_
     PairJob j;
     TG_TRY(out_proj_job(j, a, lda, w, ldw, c, ldc, M, N, K, residual, ld_res, row_ssq_out,
                         ld_ssq_out, status));
-    return launch_pair<kPairStages, EpiStore>(j.maps, j.p, (cudaStream_t)stream);
+    return launch_pair<kPairStages, EpiStore>(j.maps, j.p, (cudaStream_t)stream, workspace,
+                                              workspace_bytes);
   }
   const int bn = pick_bn(M, N);
   CUtensorMap ta, tb;
@@ -297,8 +358,8 @@ static int qkv_rope_cache_impl(const tg_bf16* x, int64_t ld_x, const tg_bf16* w_
                                const float* cos_sin, int max_pos, tg_bf16* q_out, int64_t ld_q,
                                tg_bf16* cache_k, tg_bf16* cache_v, int64_t ld_cache,
                                int64_t slot_offset, const float* row_ssq_in, int64_t ld_ssq_in,
-                               const float* q_norm_w, const float* k_norm_w, uint32_t* status,
-                               tg_stream_t stream) {
+                               const float* q_norm_w, const float* k_norm_w, void* workspace,
+                               size_t workspace_bytes, uint32_t* status, tg_stream_t stream) {
   if (head_dim != 128 || n_q_heads <= 0 || n_kv_heads <= 0 || hidden <= 0 || (hidden % 64))
     return TG_ERR_UNSUPPORTED_SHAPE;
   if (M < 0 || slot_offset < 0 || max_pos <= 0) return TG_ERR_INVALID_ARGUMENT;
@@ -329,8 +390,11 @@ static int qkv_rope_cache_impl(const tg_bf16* x, int64_t ld_x, const tg_bf16* w_
     TG_TRY(qkv_job(j, x, ld_x, w_qkv, ld_w, M, hidden, q_cols, kv_cols, eps, pos, cos_sin, max_pos,
                    q_out, ld_q, cache_k, cache_v, ld_cache, slot_offset, row_ssq_in, ld_ssq_in,
                    status, q_norm_w, k_norm_w));
-    if (q_norm_w) return launch_pair<kPairStages, EpiQKVNorm>(j.maps, j.p, (cudaStream_t)stream);
-    return launch_pair<kPairStages, EpiQKV>(j.maps, j.p, (cudaStream_t)stream);
+    if (q_norm_w)
+      return launch_pair<kPairStages, EpiQKVNorm>(j.maps, j.p, (cudaStream_t)stream, workspace,
+                                                  workspace_bytes);
+    return launch_pair<kPairStages, EpiQKV>(j.maps, j.p, (cudaStream_t)stream, workspace,
+                                            workspace_bytes);
   }
   int bn = pick_bn(M, N);
   if (bn == 256 && !aligned256) bn = 128;
@@ -366,10 +430,12 @@ extern "C" int tg_qkv_rope_cache(const tg_bf16* x, int64_t ld_x, const tg_bf16* 
                                  const float* cos_sin, int max_pos, tg_bf16* q_out, int64_t ld_q,
                                  tg_bf16* cache_k, tg_bf16* cache_v, int64_t ld_cache,
                                  int64_t slot_offset, const float* row_ssq_in,
-                                 int64_t ld_ssq_in, uint32_t* status, tg_stream_t stream) {
+                                 int64_t ld_ssq_in, void* workspace, size_t workspace_bytes,
+                                 uint32_t* status, tg_stream_t stream) {
   return qkv_rope_cache_impl(x, ld_x, w_qkv, ld_w, M, hidden, n_q_heads, n_kv_heads, head_dim,
                              eps, pos, cos_sin, max_pos, q_out, ld_q, cache_k, cache_v, ld_cache,
-                             slot_offset, row_ssq_in, ld_ssq_in, nullptr, nullptr, status, stream);
+                             slot_offset, row_ssq_in, ld_ssq_in, nullptr, nullptr, workspace,
+                             workspace_bytes, status, stream);
 }
 
 extern "C" int tg_qkv_qknorm_rope_cache(
@@ -377,12 +443,17 @@ extern "C" int tg_qkv_qknorm_rope_cache(
     int n_q_heads, int n_kv_heads, int head_dim, float eps, const float* q_norm_w,
     const float* k_norm_w, const int32_t* pos, const float* cos_sin, int max_pos, tg_bf16* q_out,
     int64_t ld_q, tg_bf16* cache_k, tg_bf16* cache_v, int64_t ld_cache, int64_t slot_offset,
-    const float* row_ssq_in, int64_t ld_ssq_in, uint32_t* status, tg_stream_t stream) {
+    const float* row_ssq_in, int64_t ld_ssq_in, void* workspace, size_t workspace_bytes,
+    uint32_t* status, tg_stream_t stream) {
   if (!q_norm_w || !k_norm_w || !row_ssq_in) return TG_ERR_INVALID_ARGUMENT;
   return qkv_rope_cache_impl(x, ld_x, w_qkv, ld_w, M, hidden, n_q_heads, n_kv_heads, head_dim,
                              eps, pos, cos_sin, max_pos, q_out, ld_q, cache_k, cache_v, ld_cache,
-                             slot_offset, row_ssq_in, ld_ssq_in, q_norm_w, k_norm_w, status,
-                             stream);
+                             slot_offset, row_ssq_in, ld_ssq_in, q_norm_w, k_norm_w, workspace,
+                             workspace_bytes, status, stream);
+}
+
+extern "C" size_t tg_gemm_workspace_size(void) {
+  return split_workspace_bytes(std::max(1, sm_count() / 2));
 }
 
 extern "C" int tg_swiglu(const tg_bf16* x, int64_t ld_x, const tg_bf16* w_gu, int64_t ld_w,

@@ -80,10 +80,10 @@ def test_host_side_argument_errors(lib):
         assert lib.tg_gated_attention(p, 2048, p, 1024, p, 1024, p, cu, 1, 16, 8, 128, p, p, p,
                                       beta, p, 2048, None, None, 0, None, None) == -1
     # projections: N not a multiple of 128, K not a multiple of 64
-    assert lib.tg_linear(p, 64, p, 64, p, 100, 4, 100, 64, 0, 0.0, None, 0, None, 0, None,
-                         None) == -6
-    assert lib.tg_linear(p, 96, p, 96, p, 128, 4, 128, 96, 0, 0.0, None, 0, None, 0, None,
-                         None) == -6
+    assert lib.tg_linear(p, 64, p, 64, p, 100, 4, 100, 64, 0, 0.0, None, 0, None, 0, None, 0,
+                         None, None) == -6
+    assert lib.tg_linear(p, 96, p, 96, p, 128, 4, 128, 96, 0, 0.0, None, 0, None, 0, None, 0,
+                         None, None) == -6
     # scorer: width other than 256
     assert lib.tg_gate_score(p, 2048, 8, 2048, None, p, 128, p, 1e-6, p, cu, 1, 1e-6, p, p,
                              p, p, p, 1 << 20, None, None) == -6
@@ -140,7 +140,7 @@ def test_full_body_argument_checks(lib):
     def qkn(qw, kw, ssq):
         return lib.tg_qkv_qknorm_rope_cache(p, 2048, p, 2048, 16, 2048, 16, 8, 128, 1e-6, qw,
                                             kw, p, p, 100, p, 2048, p, p, 1024, 0, ssq, 16,
-                                            None, None)
+                                            None, 0, None, None)
     assert qkn(None, p, p) == -1
     assert qkn(p, None, p) == -1
     assert qkn(p, p, None) == -1

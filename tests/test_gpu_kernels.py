@@ -408,6 +408,42 @@ def test_linear_row_sums_of_squares(tg, N):
     assert torch.allclose(ssq.double(), want, rtol=1e-5, atol=1e-5)
 
 
+def _gemm_flags(ws):
+    """The ready flags of a stream-K workspace: they follow the partial sums (256 KB per
+    cluster) and must be zero again after every call."""
+    part = ws.numel() // 262144 * 262144
+    return ws[part:]
+
+
+@pytest.mark.parametrize("M,N", [(1638, 2048), (1638, 4096), (300, 2048), (7000, 2048)])
+def test_linear_stream_k_against_oracle(tg, M, N):
+    """Residual + row sums of squares on the CTA-pair kernel with the stream-K tail: the
+    output projection's shape at 16k (56 tiles on 74 clusters: every tile split), a QKV
+    width, a small M, and a shape whose tail is too short to split; results within the
+    GEMM tolerance of the oracle and bit-reproducible."""
+    K = 2048
+    a = _dev(S.uniform_rows(M, K, seed=M + 11))
+    w = _dev(S.uniform_rows(N, K, seed=N + 12, scale=0.02))
+    r = _dev(S.uniform_rows(M, N, seed=13))
+    ws = torch.zeros(tg.tg_gemm_workspace_size(), dtype=torch.uint8, device="cuda")
+    outs = []
+    for _ in range(2):
+        ssq = torch.full((M, N // 128), float("nan"), device="cuda")
+        st = _status()
+        c = tg.tg_linear(a, w, residual=r, row_ssq=ssq, status=st, workspace=ws)
+        assert tg.tg_status_read(st) == 0
+        outs.append((c, ssq))
+    assert torch.equal(outs[0][0], outs[1][0]) and torch.equal(outs[0][1], outs[1][1])
+    assert torch.count_nonzero(_gemm_flags(ws)) == 0
+    c, ssq = outs[0]
+    want = _f64(a.cpu()) @ _f64(w.cpu()).T + _f64(r.cpu())
+    err = np.abs(_f64(c.cpu()) - want)
+    bad = np.argwhere(err > 2.0 ** -7 * np.abs(want) + 2e-3)
+    assert bad.size == 0, (err.max(), len(bad), bad[:8].tolist())
+    want_ssq = (c.double() ** 2).view(M, N // 128, 128).sum(-1)
+    assert torch.allclose(ssq.double(), want_ssq, rtol=1e-5, atol=1e-5)
+
+
 def test_linear_residual_in_place(tg):
     x = _dev(S.uniform_rows(257, 256, seed=1))
     x0 = x.clone()
@@ -630,9 +666,12 @@ def test_qkv_rope_cache_against_oracle(tg, M):
     assert torch.count_nonzero(ck[:slot]) == 0 and torch.count_nonzero(cv[:slot]) == 0
 
 
-@pytest.mark.parametrize("M", [1, 1638])
-def test_qkv_rope_cache_with_row_sums_against_oracle(tg, M):
-    """Precomputed row sums of squares select the CTA-pair kernel."""
+@pytest.mark.parametrize("split", [False, True])
+@pytest.mark.parametrize("M", [1, 300, 1638, 4000])
+def test_qkv_rope_cache_with_row_sums_against_oracle(tg, M, split):
+    """Precomputed row sums of squares select the CTA-pair kernel; with a GEMM workspace its
+    last round of tiles is shared along K (stream-K; M = 1638: 112 tiles on 74 clusters,
+    one whole round and 16-17 k-blocks of the rest per cluster)."""
     Hq, Hkv, d, H = 16, 8, 128, 2048
     x = S.uniform_rows(M, H, seed=M + 40)
     w = S.uniform_rows((Hq + 2 * Hkv) * d, H, seed=M + 41, scale=0.02)
@@ -641,7 +680,17 @@ def test_qkv_rope_cache_with_row_sums_against_oracle(tg, M):
     ssq = torch.from_numpy((_f64(x) ** 2).reshape(M, H // 128, 128).sum(-1)).float()
     ck = torch.zeros((M, Hkv * d), dtype=torch.bfloat16, device="cuda")
     cv = torch.zeros_like(ck)
-    q = tg.tg_qkv_rope_cache(_dev(x), _dev(w), _dev(pos), cs, ck, cv, Hq, Hkv, row_ssq=_dev(ssq))
+    ws = (torch.zeros(tg.tg_gemm_workspace_size(), dtype=torch.uint8, device="cuda") if split
+          else None)
+    st = _status()
+    q = tg.tg_qkv_rope_cache(_dev(x), _dev(w), _dev(pos), cs, ck, cv, Hq, Hkv, row_ssq=_dev(ssq),
+                             status=st, workspace=ws)
+    assert tg.tg_status_read(st) == 0
+    if split:  # the flags are left at zero, and a second call gives the same bits
+        assert torch.count_nonzero(_gemm_flags(ws)) == 0
+        q2 = tg.tg_qkv_rope_cache(_dev(x), _dev(w), _dev(pos), cs, ck.clone(), cv.clone(), Hq,
+                                  Hkv, row_ssq=_dev(ssq), workspace=ws)
+        assert torch.equal(q, q2)
     a = O.rmsnorm_rows(x)
     qkv = a @ _f64(w).T
     want_q = O.rope(qkv[:, :Hq * d].reshape(M, Hq, d), pos, 1.0e6).reshape(M, -1)
