@@ -74,7 +74,8 @@ struct AttnSmem {
   static constexpr int AEX = V + kStages * kTileBytes;  // [head] extra A columns (gain)
   static constexpr int BEX = AEX + 2 * kExBytes;        // [stage] extra B columns (key bias)
   static constexpr int BAR = BEX + kStages * kExBytes;
-  static constexpr int END = BAR + 512;
+  static constexpr int WTS = BAR + 512;   // [kMaxParts][256] merge weights, one per row
+  static constexpr int END = WTS + kMaxParts * 256 * 4;
   static constexpr int BYTES = END + 1024;  // alignment slack
 };
 
@@ -694,8 +695,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           named_bar_sync(1, 256);
           if (*parts_ready) {
             const int np = it.nparts;
-            // part i's row max and sum (its own from registers, the others' from their
-            // published blocks); read again where needed rather than kept in registers
+            // the parts' row maxima and sums (its own from registers, the others' from
+            // their published blocks; unrolled so the loads of a round are independent);
+            // the weights go to shared memory for the column loop
             auto m_of = [&](int i) {
               return i == it.part ? m_run : __ldcg(blk(i, hh) + kBM * kD + rit);
             };
@@ -703,13 +705,18 @@ __global__ void __launch_bounds__(kThreads, 1)
               return i == it.part ? l_sum : __ldcg(blk(i, hh) + kBM * kD + kBM + rit);
             };
             float M = -INFINITY;
-#pragma unroll 1
-            for (int i = 0; i < np; ++i) M = fmaxf(M, m_of(i));
+#pragma unroll
+            for (int i = 0; i < kMaxParts; ++i)
+              if (i < np) M = fmaxf(M, m_of(i));
+            float* wts = reinterpret_cast<float*>(smem + AttnSmem::WTS) + wg * 128 + rit;
             float L = 0.f;
-#pragma unroll 1
-            for (int i = 0; i < np; ++i) {
-              const float wi = ex2_approx(m_of(i) - M);  // the part's weight
-              L = i == 0 ? wi * l_of(i) : fmaf(wi, l_of(i), L);
+#pragma unroll
+            for (int i = 0; i < kMaxParts; ++i) {
+              if (i < np) {
+                const float wi = ex2_approx(m_of(i) - M);  // the part's weight
+                wts[i * 256] = wi;
+                L = i == 0 ? wi * l_of(i) : fmaf(wi, l_of(i), L);
+              }
             }
             const float inv = 1.0f / L;
             // 16 columns at a time, the parts in order (small enough to keep the merge
@@ -719,7 +726,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               float acc[16];
 #pragma unroll 1
               for (int i = 0; i < np; ++i) {
-                const float wgt = ex2_approx(m_of(i) - M);
+                const float wgt = wts[i * 256];
                 float x[16];
                 if (i == it.part) {
                   uint32_t ro[16];
