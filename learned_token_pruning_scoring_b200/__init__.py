@@ -731,8 +731,10 @@ class GatedPrefill:
         # in the first round, so the QKV tiles gain nothing by starting in the same
         # launch (measured equal to two launches); off by default.
         self.fuse_boundaries = False
-        # share the projections' last round of tiles along K over all CTA pairs (stream-K)
-        self.split_gemm = True
+        # share the projections' last round of tiles along K over all CTA pairs (stream-K):
+        # measured slower at the 16k kept count (QKV 45 -> 53 us, output projection 29 ->
+        # 39 us), so off by default
+        self.split_gemm = False
         self._qkv_done = -1  # index of the layer whose QKV already ran in a fused launch
 
     def _mark(self, name):
