@@ -319,11 +319,8 @@ int tg_kv_compact(const tg_bf16* k, int64_t ld_k, const tg_bf16* v, int64_t ld_v
  * Implemented for head_dim = 128 and an even group size n_q_heads / n_kv_heads; q, k,
  * v, o 16-byte aligned with strides that are multiples of 8; at most 512 requests per
  * call.  The kernel runs the two q heads of a kv head on tcgen05 tensor cores with S and
- * O accumulators in tensor memory and a TMA-fed K/V ring.  With a workspace of at least
- * 256 bytes the CTAs are persistent (one per SM, work items taken from a counter in the
- * workspace, heaviest first); with NULL or a smaller one every CTA runs one work item.
- * workspace (16-byte aligned, tg_gated_attention_workspace_size bytes) may be NULL.
- * status may be NULL.
+ * O accumulators in tensor memory and a TMA-fed K/V ring.  workspace (16-byte aligned,
+ * tg_gated_attention_workspace_size bytes) may be NULL.  status may be NULL.
  */
 int tg_gated_attention(const tg_bf16* q, int64_t ld_q, const tg_bf16* k, int64_t ld_k,
                        const tg_bf16* v, int64_t ld_v, const int32_t* cu_kept,
@@ -334,24 +331,21 @@ int tg_gated_attention(const tg_bf16* q, int64_t ld_q, const tg_bf16* k, int64_t
                        uint32_t* status, tg_stream_t stream);
 
 /*
- * Workspace bytes for tg_gated_attention: 256 bytes of work counters for the persistent
- * CTAs, plus, when the layout's plan splits the key range of long causal query tiles over
- * several work items (balancing the triangle over all SMs), room for the parts' partial
- * results.  Each part writes its partial result (unnormalised O, row max, row sum) there
- * and counts itself in; the part that completes a tile's count merges the parts and
- * writes o.  With at least 256 bytes but less than this size the call runs persistent
- * and unsplit; with NULL or fewer bytes, one CTA per query tile and kv-head pair.  The
- * workspace must be zero-filled before its first use (the counters); every call that
- * completes leaves it that way.  After a call that raised TG_STATUS_TIMEOUT or
- * TG_STATUS_WORKSPACE, zero it again before reusing it.
- * Layout, for n_items work items and G = n_q_heads / 2 head groups (size = 256 +
- * n_items * (n_q_heads * 66560 + 8 * G) bytes when split, else 256): int32 counters
- * (items handed out, CTAs finished), then the partial results (66560 bytes per item and
- * q head), then int32 arrival counters [n_items][G], then int32 ready flags
- * [n_items][G].  A counter found outside [0, parts) sets TG_STATUS_WORKSPACE; that
- * tile's parts then neither publish nor merge, so its output rows are left unwritten
- * (and a part that already counted itself last waits for a flag that never comes, up to
- * the bounded wait, and sets TG_STATUS_TIMEOUT).
+ * Workspace bytes that let tg_gated_attention split the key range of long causal query
+ * tiles over several CTAs (balancing the triangle over all SMs).  Each part writes its
+ * partial result (unnormalised O, row max, row sum) there and counts itself in; the
+ * part that completes a tile's count merges the parts and writes o.  0 when the layout
+ * needs no split.  With a smaller or NULL workspace the call still runs, one CTA per
+ * query tile and kv-head pair.  The workspace must be zero-filled before its first use
+ * (the counters); every call that completes leaves it that way.  After a call that
+ * raised TG_STATUS_TIMEOUT or TG_STATUS_WORKSPACE, zero it again before reusing it.
+ * Layout, for n_items work items and G = n_q_heads / 2 head groups (size = n_items *
+ * (n_q_heads * 66560 + 8 * G) bytes): the partial results (66560 bytes per item and q
+ * head), then int32 arrival counters [n_items][G], then int32 ready flags [n_items][G].
+ * A counter found outside [0, parts) sets TG_STATUS_WORKSPACE; that tile's parts then
+ * neither publish nor merge, so its output rows are left unwritten (and a part that
+ * already counted itself last waits for a flag that never comes, up to the bounded
+ * wait, and sets TG_STATUS_TIMEOUT).
  */
 size_t tg_gated_attention_workspace_size(const int32_t* cu_kept_host, int batch,
                                          int n_q_heads, int n_kv_heads, int head_dim);

@@ -298,10 +298,9 @@ def tg_gated_attention_workspace_size(cu_kept_host, n_q_heads, n_kv_heads, head_
 def tg_gated_attention(q, k, v, cu_kept, cu_kept_host, n_q_heads, n_kv_heads, kept_pos,
                        kept_bias, gamma, beta, o=None, lse=None, head_dim=128, workspace=None,
                        status=None, stream=None):
-    """Token-gated attention.  `workspace=None` allocates the workspace the layout asks
-    for (work counters of the persistent kernel and, when the plan splits, the split-KV
-    partials); pass a zero-filled uint8 tensor to reuse one (calls leave it zeroed); an
-    empty one runs one work item per CTA, unsplit."""
+    """Token-gated attention.  `workspace=None` allocates the split-KV workspace the
+    layout asks for (pass a zero-filled uint8 tensor to reuse one: calls leave it zeroed;
+    an empty one disables splitting)."""
     ld_q, ld_k, ld_v = _mat(q, "q"), _mat(k, "k"), _mat(v, "v")
     ckh = _host_i32(cu_kept_host)
     batch = ckh.numel() - 1

@@ -60,6 +60,10 @@ constexpr float kLog2e = kAttnLog2e;
 constexpr float kRescaleThreshold = 8.0f;
 
 constexpr int kMaxParts = 8;    // parts per split query tile
+constexpr int kBoxBytes = kBM * 64 * 2;  // one 64-column bf16 box of a 128-row tile
+// Epilogue staging (the Q/K/V/bias region is free once every MMA has retired): a split
+// part's block for both heads at 0, the bf16 output tile (2 heads x 2 boxes) after it.
+constexpr int kEpiOut = 2 * (kBM * kD + 2 * kBM) * 4;
 
 // Extra K columns of the S = Q K^T MMA that add the gate bias (layout in
 // tg_attn_common.cuh).
@@ -74,12 +78,12 @@ struct AttnSmem {
   static constexpr int AEX = V + kStages * kTileBytes;  // [head] extra A columns (gain)
   static constexpr int BEX = AEX + 2 * kExBytes;        // [stage] extra B columns (key bias)
   static constexpr int BAR = BEX + kStages * kExBytes;
-  static constexpr int WTS = BAR + 512;   // [kMaxParts][256] merge weights, one per row
-  static constexpr int END = WTS + kMaxParts * 256 * 4;
+  static constexpr int END = BAR + 256;
   static constexpr int BYTES = END + 1024;  // alignment slack
 };
 
-static_assert(AttnSmem::BYTES <= 227 * 1024, "shared memory");
+static_assert(kEpiOut % 1024 == 0 && kEpiOut + 4 * kBoxBytes <= AttnSmem::BAR,
+              "epilogue staging must fit below the barriers, 1024-byte aligned");
 
 struct AttnParams {
   const int32_t* cu_kept;
@@ -101,9 +105,6 @@ struct AttnParams {
   float* part_ws;      // partial results of split query tiles (see kPartFloats), or null
   int* part_count;     // per (first item of a split tile, head group): parts arrived
   int* part_ready;     // per (work item, head group): 1 once the part's partial is written
-  int n_work;          // work items x head groups
-  int* sched;          // [2]: work items handed out past the first wave, CTAs finished; or
-                       // null (one work item per CTA)
   int32_t item_prefix[kMaxBatch + 1];  // work items before request b
 };
 
@@ -178,56 +179,18 @@ __device__ __forceinline__ float row_max(uint32_t (&sv)[kBN], int rit) {
   return fmaxf(max3(m0, m1, m2), m3);
 }
 
-// Persistent form: each CTA runs a sequence of work items (request, query tile, key-range
-// part, head group).  The first item of CTA c is item c; later ones come from an atomic
-// counter in the workspace (heaviest items first, so this is list scheduling without a
-// new CTA per item), or, without a workspace, every CTA runs exactly one item.  Across
-// items the roles keep running: the producer loads the next item's Q as soon as the
-// current item's last S MMAs have read Q, and the next item's S MMAs run while the
-// softmax warps write the current item's output.  Barrier phases follow item and key-tile
-// counters that run on across items.
-__device__ __forceinline__ int next_work(const AttnParams& p, int ic) {
-  if (ic == 0) return (int)blockIdx.x < p.n_work ? (int)blockIdx.x : -1;
-  if (!p.sched) return -1;
-  const int w = (int)gridDim.x + atomicAdd(p.sched, 1);
-  return w < p.n_work ? w : -1;
-}
-
-// Work item w -> request, query tile, part, head group and the quantities every role
-// derives from them.
-struct AttnItem {
-  int b, qt, part, nparts, head_grp, item;
-  int g, h0, n_b, q0, j0, nt;
-  int64_t row0;
-};
-__device__ __forceinline__ AttnItem decode_work(const AttnParams& p, int w) {
-  AttnItem it;
-  const int hg = p.n_kv_heads * p.head_pairs;
-  it.head_grp = w % hg;
-  it.item = w / hg;
-  decode_item(p, it.item, it.b, it.qt, it.part, it.nparts);
-  it.g = it.head_grp / p.head_pairs;
-  it.h0 = it.g * p.group + 2 * (it.head_grp % p.head_pairs);
-  it.row0 = p.cu_kept[it.b];
-  it.n_b = p.cu_kept[it.b + 1] - p.cu_kept[it.b];
-  it.q0 = it.qt * kBM;
-  it.j0 = it.part * p.chunk;
-  it.nt = min(it.qt + 1, it.j0 + p.chunk) - it.j0;
-  return it;
-}
-
 __global__ void __launch_bounds__(kThreads, 1)
     gated_attention_kernel(const __grid_constant__ CUtensorMap tmQ,
                            const __grid_constant__ CUtensorMap tmK,
                            const __grid_constant__ CUtensorMap tmV,
+                           const __grid_constant__ CUtensorMap tmO,
                            const __grid_constant__ AttnParams p) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + AttnSmem::BAR);
   uint64_t* q_full = bars + 0;
-  uint64_t* q_empty = bars + 1;            // the item's last S MMAs have read Q and the gains
-  uint64_t* k_full = bars + 2;             // [kStages]
+  uint64_t* k_full = bars + 1;             // [kStages]
   uint64_t* v_full = k_full + kStages;     // [kStages]
   uint64_t* k_empty = v_full + kStages;    // [kStages]
   uint64_t* v_empty = k_empty + kStages;   // [kStages]
@@ -236,21 +199,17 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* s_full = ax_ready + 2;         // [2]
   uint64_t* p_full = s_full + 2;           // [2]
   uint64_t* pv_done = p_full + 2;          // [2]
-  uint64_t* o_empty = pv_done + 2;         // [2] the head's output has been read from TMEM
-  uint64_t* item_full = o_empty + 2;       // [2] work slot written
-  uint64_t* item_empty = item_full + 2;    // [2] work slot read by the MMA and softmax roles
-  uint64_t* drain = item_empty + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* drain = pv_done + 2;
+  uint64_t* merge_full = drain + 1;        // a split tile's other part staged for the merge
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(merge_full + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   volatile int* last_part = reinterpret_cast<volatile int*>(tmem_slot + 2);
   volatile int* parts_ready = reinterpret_cast<volatile int*>(tmem_slot + 3);
-  volatile int* work_slot = reinterpret_cast<volatile int*>(tmem_slot + 4);  // [2]
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
   if (tid == 0) {
     mbar_init(q_full, 1);
-    mbar_init(q_empty, 1);
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&k_full[s], 1);
       mbar_init(&bx_full[s], 1);
@@ -263,11 +222,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&s_full[h], 1);
       mbar_init(&p_full[h], 128);
       mbar_init(&pv_done[h], 1);
-      mbar_init(&o_empty[h], 128);
-      mbar_init(&item_full[h], 1);
-      mbar_init(&item_empty[h], 1 + 256);
     }
     mbar_init(drain, 1);
+    mbar_init(merge_full, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -286,100 +243,94 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = *tmem_slot;
   // everything below reads what earlier grids wrote
   griddep_wait();
+
+  // ---- which work item: head groups vary fastest, then items heaviest first
   const int hg = p.n_kv_heads * p.head_pairs;
+  const int head_grp = blockIdx.x % hg;
+  const int item = blockIdx.x / hg;
+  int b, qt, part, nparts;
+  decode_item(p, item, b, qt, part, nparts);
+  const int g = head_grp / p.head_pairs;
+  const int h0 = g * p.group + 2 * (head_grp % p.head_pairs);
+  const int64_t row0 = p.cu_kept[b];
+  const int n_b = p.cu_kept[b + 1] - p.cu_kept[b];
+  const int q0 = qt * kBM;
+  // causal: key tiles 0..qt, this item's share [j0, j0 + nt)
+  const int j0 = part * p.chunk;
+  const int nt = min(qt + 1, j0 + p.chunk) - j0;
 
   if (warp < 4) {
     regs_dec<kRegsLow>();
     if (warp == 0) {
       // ---------------------------------------------------------- producer
-      int ic = 0, jt = 0, q_loads = 0, k_cnt = 0, v_cnt = 0;
-      while (true) {
-        int w = 0;
-        if (lane == 0) w = next_work(p, ic);
-        w = __shfl_sync(0xFFFFFFFFu, w, 0);
-        const int slot = ic & 1;
-        if (!warp_all(mbar_wait(&item_empty[slot], (((uint32_t)ic >> 1) & 1u) ^ 1u, abort_flag,
-                                p.status)))
+      int loaded = 0, loaded_v = 0;
+      bool q_issued = false;
+      if (lane == 0) {
+        mbar_arrive_expect_tx(q_full, 2 * kTileBytes);
+        const int y = (int)(row0 + q0);
+        tma_load_2d(smem + AttnSmem::Q0, &tmQ, h0 * kD, y, q_full);
+        tma_load_2d(smem + AttnSmem::Q0 + kTileBytes / 2, &tmQ, h0 * kD + 64, y, q_full);
+        tma_load_2d(smem + AttnSmem::Q1, &tmQ, (h0 + 1) * kD, y, q_full);
+        tma_load_2d(smem + AttnSmem::Q1 + kTileBytes / 2, &tmQ, (h0 + 1) * kD + 64, y, q_full);
+        q_issued = true;
+      }
+      // Key bias of tile j, loaded one tile ahead so its global latency overlaps the
+      // wait for a free stage.
+      auto load_bias = [&](int j, float (&bv)[4]) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int c = (j0 + j) * kBN + lane * 4 + e;
+          bv[e] = (j < nt && c < n_b) ? p.kept_bias[row0 + c] : 0.0f;
+        }
+      };
+      float bv[4];
+      load_bias(0, bv);
+      for (int j = 0; j < nt; ++j) {
+        const int s = j % kStages;
+        const uint32_t ph = (uint32_t)(j / kStages) & 1u;
+        const int y = (int)(row0 + (j0 + j) * kBN);
+        // K of tile j once both heads' S MMAs of tile j - kStages are done
+        if (!warp_all(mbar_wait(&k_empty[s], ph ^ 1u, abort_flag, p.status))) break;
+        unsigned char* kt = smem + AttnSmem::K + s * kTileBytes;
+        if (lane == 0) {
+          mbar_arrive_expect_tx(&k_full[s], kTileBytes);
+          tma_load_2d(kt, &tmK, g * kD, y, &k_full[s]);
+          tma_load_2d(kt + kTileBytes / 2, &tmK, g * kD + 64, y, &k_full[s]);
+        }
+        // Extra B columns of the tile's keys: (b_hi, b_lo, b_hi, 0, ...); with a row's
+        // (g_hi, g_hi, g_lo, 0, ...) the MMA adds g_hi b_hi + g_hi b_lo + g_lo b_hi, i.e.
+        // g * b to ~2^-16 relative
+        {
+          unsigned char* bx = smem + AttnSmem::BEX + s * kExBytes;
+#pragma unroll
+          for (int e = 0; e < 4; ++e) attn_put_key_bias(bx, lane * 4 + e, bv[e]);
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&bx_full[s]);
+        }
+        // V of tile j once both heads' PV MMAs of tile j - kStages are done
+        if (!warp_all(mbar_wait(&v_empty[s], ph ^ 1u, abort_flag, p.status))) {
+          ++loaded;
           break;
+        }
+        unsigned char* vt = smem + AttnSmem::V + s * kTileBytes;
         if (lane == 0) {
-          work_slot[slot] = w;
-          mbar_arrive(&item_full[slot]);
+          mbar_arrive_expect_tx(&v_full[s], kTileBytes);
+          tma_load_2d(vt, &tmV, g * kD, y, &v_full[s]);
+          tma_load_2d(vt + kTileBytes / 2, &tmV, g * kD + 64, y, &v_full[s]);
         }
-        if (w < 0) break;
-        const AttnItem it = decode_work(p, w);
-        // Q of this item once the previous item's S MMAs are done with the Q buffers
-        if (!warp_all(mbar_wait(q_empty, ((uint32_t)ic & 1u) ^ 1u, abort_flag, p.status))) break;
-        if (lane == 0) {
-          mbar_arrive_expect_tx(q_full, 2 * kTileBytes);
-          const int y = (int)(it.row0 + it.q0);
-          tma_load_2d(smem + AttnSmem::Q0, &tmQ, it.h0 * kD, y, q_full);
-          tma_load_2d(smem + AttnSmem::Q0 + kTileBytes / 2, &tmQ, it.h0 * kD + 64, y, q_full);
-          tma_load_2d(smem + AttnSmem::Q1, &tmQ, (it.h0 + 1) * kD, y, q_full);
-          tma_load_2d(smem + AttnSmem::Q1 + kTileBytes / 2, &tmQ, (it.h0 + 1) * kD + 64, y,
-                      q_full);
-        }
-        ++q_loads;
-        // Key bias of tile j, loaded one tile ahead so its global latency overlaps the
-        // wait for a free stage.
-        auto load_bias = [&](int j, float (&bv)[4]) {
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int c = (it.j0 + j) * kBN + lane * 4 + e;
-            bv[e] = (j < it.nt && c < it.n_b) ? p.kept_bias[it.row0 + c] : 0.0f;
-          }
-        };
-        float bv[4];
-        load_bias(0, bv);
-        bool ok = true;
-        for (int j = 0; j < it.nt; ++j) {
-          const int gt = jt + j;
-          const int s = gt % kStages;
-          const uint32_t ph = (uint32_t)(gt / kStages) & 1u;
-          const int y = (int)(it.row0 + (it.j0 + j) * kBN);
-          // K of tile gt once both heads' S MMAs of tile gt - kStages are done
-          if (!(ok = warp_all(mbar_wait(&k_empty[s], ph ^ 1u, abort_flag, p.status)))) break;
-          unsigned char* kt = smem + AttnSmem::K + s * kTileBytes;
-          if (lane == 0) {
-            mbar_arrive_expect_tx(&k_full[s], kTileBytes);
-            tma_load_2d(kt, &tmK, it.g * kD, y, &k_full[s]);
-            tma_load_2d(kt + kTileBytes / 2, &tmK, it.g * kD + 64, y, &k_full[s]);
-          }
-          k_cnt = gt + 1;
-          // Extra B columns of the tile's keys: (b_hi, b_lo, b_hi, 0, ...); with a row's
-          // (g_hi, g_hi, g_lo, 0, ...) the MMA adds g_hi b_hi + g_hi b_lo + g_lo b_hi, i.e.
-          // g * b to ~2^-16 relative
-          {
-            unsigned char* bx = smem + AttnSmem::BEX + s * kExBytes;
-#pragma unroll
-            for (int e = 0; e < 4; ++e) attn_put_key_bias(bx, lane * 4 + e, bv[e]);
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&bx_full[s]);
-          }
-          // V of tile gt once both heads' PV MMAs of tile gt - kStages are done
-          if (!(ok = warp_all(mbar_wait(&v_empty[s], ph ^ 1u, abort_flag, p.status)))) break;
-          unsigned char* vt = smem + AttnSmem::V + s * kTileBytes;
-          if (lane == 0) {
-            mbar_arrive_expect_tx(&v_full[s], kTileBytes);
-            tma_load_2d(vt, &tmV, it.g * kD, y, &v_full[s]);
-            tma_load_2d(vt + kTileBytes / 2, &tmV, it.g * kD + 64, y, &v_full[s]);
-          }
-          v_cnt = gt + 1;
-          load_bias(j + 1, bv);
-        }
-        if (!ok) break;
-        jt += it.nt;
-        ++ic;
+        load_bias(j + 1, bv);
+        ++loaded;
+        ++loaded_v;
       }
       if (lane == 0) {
-        // Drain: no bulk copy may still be landing when the CTA exits.  On the normal path
-        // the MMA role has waited for every one of them; after an abort this waits (each
-        // bounded) for the last Q and the last key tiles' K and V loads.
-        if (q_loads > 0) mbar_wait(q_full, (uint32_t)(q_loads - 1) & 1u, nullptr, p.status);
-        for (int gt = k_cnt - kStages < 0 ? 0 : k_cnt - kStages; gt < k_cnt; ++gt)
-          mbar_wait(&k_full[gt % kStages], (uint32_t)(gt / kStages) & 1u, nullptr, p.status);
-        for (int gt = v_cnt - kStages < 0 ? 0 : v_cnt - kStages; gt < v_cnt; ++gt)
-          mbar_wait(&v_full[gt % kStages], (uint32_t)(gt / kStages) & 1u, nullptr, p.status);
+        // drain: no bulk copy may still be landing when the CTA exits
+        if (q_issued) mbar_wait(q_full, 0, nullptr, p.status);
+        for (int j = loaded - kStages < 0 ? 0 : loaded - kStages; j < loaded; ++j) {
+          const uint32_t ph = (uint32_t)(j / kStages) & 1u;
+          mbar_wait(&k_full[j % kStages], ph, nullptr, p.status);
+          if (j < loaded_v) mbar_wait(&v_full[j % kStages], ph, nullptr, p.status);
+        }
       }
     } else if (warp == 1) {
       // ---------------------------------------------------------- MMA issuer
@@ -401,8 +352,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint64_t bx_desc0 = interleave_desc(smem_u32(smem + AttnSmem::BEX), 128, 256);
         const uint32_t s_col[2] = {0u, 128u};
         const uint32_t o_col[2] = {256u, 384u};
-        auto issue_s = [&](int hh, int gt) {
-          const uint64_t kd = k_desc0 + (uint64_t)(((gt % kStages) * kTileBytes) >> 4);
+        auto issue_s = [&](int hh, int j) {
+          const uint64_t kd = k_desc0 + (uint64_t)(((j % kStages) * kTileBytes) >> 4);
 #pragma unroll
           for (int kk = 0; kk < kD / 16; ++kk) {
             const uint64_t off = (uint64_t)(((kk >> 2) * (kTileBytes / 2) + (kk & 3) * 32) >> 4);
@@ -410,11 +361,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           // + (gamma_h * log2(e) / t_r) * bias_c, one more K=16 step on the extra columns
           mma_ss(tmem + s_col[hh], ax_desc[hh],
-                 bx_desc0 + (uint64_t)(((gt % kStages) * kExBytes) >> 4), idesc_s, 1u);
+                 bx_desc0 + (uint64_t)(((j % kStages) * kExBytes) >> 4), idesc_s, 1u);
           mma_commit(&s_full[hh]);
         };
-        auto issue_pv = [&](int hh, int j, int gt) {
-          const uint64_t vd = v_desc0 + (uint64_t)(((gt % kStages) * kTileBytes) >> 4);
+        auto issue_pv = [&](int hh, int j) {
+          const uint64_t vd = v_desc0 + (uint64_t)(((j % kStages) * kTileBytes) >> 4);
 #pragma unroll
           for (int kk = 0; kk < kBN / 16; ++kk) {
             // A = P (bf16 pairs in TMEM, 8 columns per 16 keys); B = V rows kk*16.. (MN-major)
@@ -423,65 +374,44 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           mma_commit(&pv_done[hh]);
         };
-        int ic = 0, jt = 0;
-        bool ok = true;
-        while (ok) {
-          const int slot = ic & 1;
-          if (!mbar_wait(&item_full[slot], ((uint32_t)ic >> 1) & 1u, abort_flag, p.status)) break;
-          const int w = work_slot[slot];
-          mbar_arrive(&item_empty[slot]);
-          if (w < 0) break;
-          const AttnItem it = decode_work(p, w);
-          const uint32_t pi = (uint32_t)ic & 1u;
-          const int s0 = jt % kStages;
-          const uint32_t ph0 = (uint32_t)(jt / kStages) & 1u;
-          ok = mbar_wait(q_full, pi, abort_flag, p.status) &&
-               mbar_wait(&ax_ready[0], pi, abort_flag, p.status) &&
-               mbar_wait(&ax_ready[1], pi, abort_flag, p.status) &&
-               mbar_wait(&k_full[s0], ph0, abort_flag, p.status) &&
-               mbar_wait(&bx_full[s0], ph0, abort_flag, p.status);
-          if (!ok) break;
+        bool ok = mbar_wait(q_full, 0, abort_flag, p.status) &&
+                  mbar_wait(&ax_ready[0], 0, abort_flag, p.status) &&
+                  mbar_wait(&ax_ready[1], 0, abort_flag, p.status) &&
+                  mbar_wait(&k_full[0], 0, abort_flag, p.status) &&
+                  mbar_wait(&bx_full[0], 0, abort_flag, p.status);
+        if (ok) {
           tc_fence_after();
-          issue_s(0, jt);
-          issue_s(1, jt);
-          mma_commit(&k_empty[s0]);
-          if (it.nt == 1) mma_commit(q_empty);
-          for (int j = 0; j < it.nt && ok; ++j) {
-            const int gt = jt + j;
-            const int s = gt % kStages;
-            const uint32_t ph = (uint32_t)(gt / kStages) & 1u;
-            const uint32_t pj = (uint32_t)gt & 1u;
+          issue_s(0, 0);
+          issue_s(1, 0);
+          mma_commit(&k_empty[0]);
+          for (int j = 0; j < nt && ok; ++j) {
+            const int s = j % kStages;
+            const uint32_t ph = (uint32_t)(j / kStages) & 1u;
+            const uint32_t pj = (uint32_t)j & 1u;
             ok = mbar_wait(&v_full[s], ph, abort_flag, p.status) &&
                  mbar_wait(&p_full[0], pj, abort_flag, p.status);
-            // the first PV overwrites O: the previous item's output must have been read
-            if (ok && j == 0) ok = mbar_wait(&o_empty[0], pi ^ 1u, abort_flag, p.status);
             if (!ok) break;
             tc_fence_after();
-            issue_pv(0, j, gt);
-            const bool more = j + 1 < it.nt;
+            issue_pv(0, j);
+            const bool more = j + 1 < nt;
             if (more) {
-              const int s2 = (gt + 1) % kStages;
-              const uint32_t ph2 = (uint32_t)((gt + 1) / kStages) & 1u;
+              const int s2 = (j + 1) % kStages;
+              const uint32_t ph2 = (uint32_t)((j + 1) / kStages) & 1u;
               if (!(ok = mbar_wait(&k_full[s2], ph2, abort_flag, p.status) &&
                          mbar_wait(&bx_full[s2], ph2, abort_flag, p.status)))
                 break;
               tc_fence_after();
-              issue_s(0, gt + 1);
+              issue_s(0, j + 1);
             }
-            ok = mbar_wait(&p_full[1], pj, abort_flag, p.status);
-            if (ok && j == 0) ok = mbar_wait(&o_empty[1], pi ^ 1u, abort_flag, p.status);
-            if (!ok) break;
+            if (!(ok = mbar_wait(&p_full[1], pj, abort_flag, p.status))) break;
             tc_fence_after();
-            issue_pv(1, j, gt);
+            issue_pv(1, j);
             mma_commit(&v_empty[s]);
             if (more) {
-              issue_s(1, gt + 1);
-              mma_commit(&k_empty[(gt + 1) % kStages]);
-              if (j + 2 == it.nt) mma_commit(q_empty);  // the item's last S MMAs
+              issue_s(1, j + 1);
+              mma_commit(&k_empty[(j + 1) % kStages]);
             }
           }
-          jt += it.nt;
-          ++ic;
         }
         mma_commit(drain);
         mbar_wait(drain, 0, nullptr, p.status);  // every MMA retired before TMEM is freed
@@ -489,150 +419,155 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     regs_inc<kRegsHigh>();
-    // ------------------------------------------------------------ softmax + epilogue
+    // ------------------------------------------------------------ softmax
     const int wg = (warp - 4) >> 2;  // 0: head h0, 1: head h0 + 1
+    const int hh = h0 + wg;
     const int q = warp & 3;
     const int rit = q * 32 + lane;   // row in tile
+    const int r = q0 + rit;          // rank inside the request
+    const bool row_valid = r < n_b;
     const uint32_t lane_off = (uint32_t)(q * 32) << 16;
     const uint32_t s_t = tmem + lane_off + (wg ? 128u : 0u);
     const uint32_t o_t = tmem + lane_off + (wg ? 384u : 256u);
-    const bool elected = warp == 4 && lane == 0;
-    int ic = 0, jt = 0;
-    while (true) {
-      const int slot = ic & 1;
-      if (!warp_all(mbar_wait(&item_full[slot], ((uint32_t)ic >> 1) & 1u, abort_flag, p.status)))
-        break;
-      const int w = work_slot[slot];
-      mbar_arrive(&item_empty[slot]);
-      if (w < 0) break;
-      float t2;
-      int j0, qt, nt;
-      {
-        const AttnItem it = decode_work(p, w);
-        const int r = it.q0 + rit;  // rank inside the request
-        const double tau = attn_tau(p.beta, r, r < it.n_b ? p.kept_pos[it.row0 + r] : 0);
-        t2 = attn_logit_scale(tau, kD);
-        j0 = it.j0;
-        qt = it.qt;
-        nt = it.nt;
-        // the gain columns are read by the S MMAs: the previous item's must be done
-        if (!warp_all(mbar_wait(q_empty, ((uint32_t)ic & 1u) ^ 1u, abort_flag, p.status))) break;
-        attn_put_query_gain(smem + AttnSmem::AEX + wg * kExBytes, rit,
-                            p.gamma[it.h0 + wg] * kLog2e / t2);
-        fence_proxy_async_smem();  // read by the tensor core
-        mbar_arrive(&ax_ready[wg]);
+
+    const double tau = attn_tau(p.beta, r, row_valid ? p.kept_pos[row0 + r] : 0);
+
+    // The logit in the log2 domain is t * S with t = tau_r * log2(e) / sqrt(d) and
+    // S = q.k + (gamma_h * log2(e) / t) * bias_c: the tensor core adds the bias term
+    // through one extra K=16 step whose A columns, per row, hold g = gamma_h log2(e) / t
+    // split into bf16 parts (g_hi, g_hi, g_lo).  t >= 0 (beta >= 0); t = 0 (first kept
+    // token of a request whose position is not 0) is taken as 2^-66, which leaves
+    // t * S = gamma_h log2(e) bias_c.
+    const float t2 = attn_logit_scale(tau, kD);
+    {
+      attn_put_query_gain(smem + AttnSmem::AEX + wg * kExBytes, rit, p.gamma[hh] * kLog2e / t2);
+      fence_proxy_async_smem();  // read by the tensor core
+      mbar_arrive(&ax_ready[wg]);
+    }
+
+    float m_run = -INFINITY, l_sum = 0.f;
+    bool ok = true;
+    for (int j = 0; j < nt; ++j) {
+      if (!(ok = warp_all(mbar_wait(&s_full[wg], (uint32_t)j & 1u, abort_flag, p.status)))) break;
+      tc_fence_after();
+      uint32_t sv[kBN];
+      tmem_ld32(s_t + 0, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
+      tmem_ld32(s_t + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
+      tmem_ld32(s_t + 64, *reinterpret_cast<uint32_t(*)[32]>(&sv[64]));
+      tmem_ld32(s_t + 96, *reinterpret_cast<uint32_t(*)[32]>(&sv[96]));
+      tmem_wait_ld();
+      const float mx = t2 * ((j0 + j == qt) ? row_max<true>(sv, rit) : row_max<false>(sv, rit));
+      // Lazy rescale: move the running max only when it grows by more than 2^8.
+      float alpha = 1.0f;
+      bool rescale = false;
+      if (j == 0) {
+        m_run = mx;
+      } else if (mx > m_run + kRescaleThreshold) {
+        alpha = ex2_approx(m_run - mx);
+        m_run = mx;
+        rescale = true;
       }
-
-      // The logit in the log2 domain is t * S with t = tau_r * log2(e) / sqrt(d) and
-      // S = q.k + (gamma_h * log2(e) / t) * bias_c: the tensor core adds the bias term
-      // through one extra K=16 step whose A columns, per row, hold g = gamma_h log2(e) / t
-      // split into bf16 parts (g_hi, g_hi, g_lo).  t >= 0 (beta >= 0); t = 0 (first kept
-      // token of a request whose position is not 0) is taken as 2^-66, which leaves
-      // t * S = gamma_h log2(e) bias_c.
-
-      float m_run = -INFINITY, l_sum = 0.f;
-      bool ok = true;
-      for (int j = 0; j < nt; ++j) {
-        const int gt = jt + j;
-        if (!(ok = warp_all(mbar_wait(&s_full[wg], (uint32_t)gt & 1u, abort_flag, p.status))))
+      const uint64_t negm = f2pack(-m_run, -m_run);
+      const uint64_t t2p = f2pack(t2, t2);
+      uint64_t acc0 = f2pack(0.f, 0.f), acc1 = acc0;
+#pragma unroll
+      for (int hf = 0; hf < 2; ++hf) {
+        uint32_t pk[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const int e = 64 * hf + 2 * i;
+          const uint64_t d = fma2(f2pack(__uint_as_float(sv[e]), __uint_as_float(sv[e + 1])), t2p, negm);
+          float x0, x1;
+          f2unpack(d, x0, x1);
+          const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
+          if (i & 1) acc1 = add2(acc1, f2pack(p0, p1));
+          else acc0 = add2(acc0, f2pack(p0, p1));
+          pk[i] = pack_bf16x2(p0, p1);
+        }
+        tmem_st32(s_t + 32 * hf, pk);
+      }
+      float a0, a1, a2, a3;
+      f2unpack(acc0, a0, a1);
+      f2unpack(acc1, a2, a3);
+      l_sum = l_sum * alpha + ((a0 + a1) + (a2 + a3));
+      // O rescale, warp-uniform (tcgen05.ld/st are warp-collective; alpha = 1 on rows
+      // that keep their max).  PV(j-1) has retired: S(j) was committed after it.
+      if (__any_sync(0xFFFFFFFFu, rescale)) {
+        if (!(ok = warp_all(mbar_wait(&pv_done[wg], (uint32_t)(j - 1) & 1u, abort_flag,
+                                      p.status))))
           break;
         tc_fence_after();
-        uint32_t sv[kBN];
-        tmem_ld32(s_t + 0, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
-        tmem_ld32(s_t + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
-        tmem_ld32(s_t + 64, *reinterpret_cast<uint32_t(*)[32]>(&sv[64]));
-        tmem_ld32(s_t + 96, *reinterpret_cast<uint32_t(*)[32]>(&sv[96]));
-        tmem_wait_ld();
-        const float mx = t2 * ((j0 + j == qt) ? row_max<true>(sv, rit) : row_max<false>(sv, rit));
-        // Lazy rescale: move the running max only when it grows by more than 2^8.
-        float alpha = 1.0f;
-        bool rescale = false;
-        if (j == 0) {
-          m_run = mx;
-        } else if (mx > m_run + kRescaleThreshold) {
-          alpha = ex2_approx(m_run - mx);
-          m_run = mx;
-          rescale = true;
-        }
-        const uint64_t negm = f2pack(-m_run, -m_run);
-        const uint64_t t2p = f2pack(t2, t2);
-        uint64_t acc0 = f2pack(0.f, 0.f), acc1 = acc0;
-#pragma unroll
-        for (int hf = 0; hf < 2; ++hf) {
-          uint32_t pk[32];
-#pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const int e = 64 * hf + 2 * i;
-            const uint64_t d = fma2(f2pack(__uint_as_float(sv[e]), __uint_as_float(sv[e + 1])), t2p, negm);
-            float x0, x1;
-            f2unpack(d, x0, x1);
-            const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
-            if (i & 1) acc1 = add2(acc1, f2pack(p0, p1));
-            else acc0 = add2(acc0, f2pack(p0, p1));
-            pk[i] = pack_bf16x2(p0, p1);
-          }
-          tmem_st32(s_t + 32 * hf, pk);
-        }
-        float a0, a1, a2, a3;
-        f2unpack(acc0, a0, a1);
-        f2unpack(acc1, a2, a3);
-        l_sum = l_sum * alpha + ((a0 + a1) + (a2 + a3));
-        // O rescale, warp-uniform (tcgen05.ld/st are warp-collective; alpha = 1 on rows
-        // that keep their max).  PV(j-1) has retired: S(j) was committed after it.
-        if (__any_sync(0xFFFFFFFFu, rescale)) {
-          if (!(ok = warp_all(mbar_wait(&pv_done[wg], (uint32_t)(gt - 1) & 1u, abort_flag,
-                                        p.status))))
-            break;
-          tc_fence_after();
 #pragma unroll 1
-          for (int c = 0; c < kD / 32; ++c) {
-            uint32_t ro[32];
-            tmem_ld32(o_t + c * 32, ro);
-            tmem_wait_ld();
+        for (int c = 0; c < kD / 32; ++c) {
+          uint32_t ro[32];
+          tmem_ld32(o_t + c * 32, ro);
+          tmem_wait_ld();
 #pragma unroll
-            for (int i = 0; i < 32; ++i) ro[i] = __float_as_uint(__uint_as_float(ro[i]) * alpha);
-            tmem_st32(o_t + c * 32, ro);
-          }
+          for (int i = 0; i < 32; ++i) ro[i] = __float_as_uint(__uint_as_float(ro[i]) * alpha);
+          tmem_st32(o_t + c * 32, ro);
         }
-        tmem_wait_st();
-        tc_fence_before();
-        mbar_arrive(&p_full[wg]);
       }
-      const bool done = ok && warp_all(mbar_wait(&pv_done[wg], (uint32_t)(jt + nt - 1) & 1u,
-                                                 abort_flag, p.status));
-      if (done) tc_fence_after();
-      // Both heads meet here once per item (all outcomes CTA-uniform from here on).
-      const bool all_done = named_bar_and(1, 256, done);
-      if (!all_done) break;
-      const AttnItem it = decode_work(p, w);  // again: nothing of it stays live in the loop
-      const int hh = it.h0 + wg;
-      const int r = it.q0 + rit;  // rank inside the request
-      const bool row_valid = r < it.n_b;
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(&p_full[wg]);
+    }
+    const bool done =
+        ok && warp_all(mbar_wait(&pv_done[wg], (uint32_t)(nt - 1) & 1u, abort_flag, p.status));
+    if (done) tc_fence_after();
+    // Both heads meet here once: after it every MMA has retired, so the Q/K/V/bias
+    // shared memory is free for staging, whatever path follows (all CTA-uniform).
+    const bool all_done = named_bar_and(1, 256, done);
+    const bool elected = warp == 4 && lane == 0;
+    // A full query tile lies inside its request: its bf16 output goes through shared
+    // memory (128-byte swizzle, two 64-column boxes per head) and TMA stores.  A
+    // request's ragged last tile stores rows directly (a full box would reach into the
+    // next request's rows).
+    const bool full_tile = q0 + kBM <= n_b;
+    unsigned char* out_head = smem + kEpiOut + wg * 2 * kBoxBytes;
+    auto put_chunk = [&](int c, const float (&acc)[32], float inv) {
+      uint32_t w[16];
+#pragma unroll
+      for (int e = 0; e < 16; ++e) w[e] = pack_bf16x2(acc[2 * e] * inv, acc[2 * e + 1] * inv);
+      if (full_tile) {
+        unsigned char* box = out_head + (c >> 1) * kBoxBytes;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int k = (c & 1) * 4 + u;  // 16-byte chunk of the row inside its box
+          *reinterpret_cast<uint4*>(box + rit * 128 + ((k ^ (rit & 7)) << 4)) =
+              make_uint4(w[4 * u], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]);
+        }
+      } else if (row_valid) {
+        uint4* dst = reinterpret_cast<uint4*>(p.o + (row0 + r) * p.ld_o + (int64_t)hh * kD + c * 32);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) dst[u] = make_uint4(w[4 * u], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]);
+      }
+    };
+    auto store_lse = [&](float M, float L) {
+      if (row_valid && p.lse)
+        p.lse[(int64_t)hh * p.k_total + row0 + r] = (M + log2f(L)) * 0.69314718055994531f;
+    };
+    // after every thread has put its chunks: the staged tile goes out by TMA
+    auto flush_out = [&]() {
+      fence_proxy_async_smem();
+      named_bar_sync(1, 256);
+      if (full_tile && elected) {
+        for (int h = 0; h < 2; ++h)
+          for (int bx = 0; bx < 2; ++bx)
+            tma_store_2d(&tmO, (h0 + h) * kD + 64 * bx, (int32_t)(row0 + q0),
+                         smem + kEpiOut + (h * 2 + bx) * kBoxBytes);
+        bulk_commit_group();
+      }
+    };
+    auto own_chunk = [&](int c, float (&x)[32]) {
+      uint32_t ro[32];
+      tmem_ld32(o_t + c * 32, ro);
+      tmem_wait_ld();
+#pragma unroll
+      for (int e = 0; e < 32; ++e) x[e] = __uint_as_float(ro[e]);
+    };
 
-      // Output rows go straight from registers to global memory (one 256-byte row per
-      // thread and head); the Q/K/V shared memory already holds the next item's tiles.
-      auto put_chunk = [&](int c, const float (&acc)[32], float inv) {
-        if (!row_valid) return;
-        uint32_t wv[16];
-#pragma unroll
-        for (int e = 0; e < 16; ++e) wv[e] = pack_bf16x2(acc[2 * e] * inv, acc[2 * e + 1] * inv);
-        uint4* dst = reinterpret_cast<uint4*>(p.o + (it.row0 + r) * p.ld_o + (int64_t)hh * kD + c * 32);
-#pragma unroll
-        for (int u = 0; u < 4; ++u) dst[u] = make_uint4(wv[4 * u], wv[4 * u + 1], wv[4 * u + 2], wv[4 * u + 3]);
-      };
-      auto store_lse = [&](float M, float L) {
-        if (row_valid && p.lse)
-          p.lse[(int64_t)hh * p.k_total + it.row0 + r] = (M + log2f(L)) * 0.69314718055994531f;
-      };
-      auto own_chunk = [&](int c, float (&x)[32]) {
-        uint32_t ro[32];
-        tmem_ld32(o_t + c * 32, ro);
-        tmem_wait_ld();
-#pragma unroll
-        for (int e = 0; e < 32; ++e) x[e] = __uint_as_float(ro[e]);
-      };
-
-      if (it.nparts == 1) {
+    if (nparts == 1) {
+      if (all_done) {
         const float inv = 1.0f / l_sum;
 #pragma unroll 1
         for (int c = 0; c < kD / 32; ++c) {
@@ -641,139 +576,199 @@ __global__ void __launch_bounds__(kThreads, 1)
           put_chunk(c, acc, inv);
         }
         store_lse(m_run, l_sum);
-      } else {
-        // Split query tile.  Each part counts its arrival; every part but the last to
-        // arrive publishes its partial result (unnormalised O, row max, row sum) and
-        // raises its ready flag; the last one merges all parts, summing in part order
-        // whichever part it is (so every run rounds alike):
-        //   M = max_i m_i, L = sum_i 2^(m_i - M) l_i, o = sum_i 2^(m_i - M) O_i / L.
-        // It waits only for parts that have already arrived and are just storing, so the
-        // wait always ends.
-        int* cnt = p.part_count + (int64_t)(it.item - it.part) * hg + it.head_grp;
+        flush_out();
+      }
+    } else if (all_done) {
+      // Split query tile.  Each part counts its arrival; every part but the last to
+      // arrive publishes its partial result (unnormalised O, row max, row sum) with bulk
+      // stores and raises its ready flag; the last one merges all parts, summing in part
+      // order whichever part it is (so every run rounds alike):
+      //   M = max_i m_i, L = sum_i 2^(m_i - M) l_i, o = sum_i 2^(m_i - M) O_i / L.
+      // It waits only for parts that have already arrived and are just storing, so the
+      // wait always ends.
+      int* cnt = p.part_count + (int64_t)(item - part) * hg + head_grp;
+      if (elected) {
+        const int before = atomicAdd(cnt, 1);
+        if (before < 0 || before >= nparts) {
+          // the counter did not start at zero: the workspace was not zero-filled
+          if (p.status) atomicOr(p.status, TG_STATUS_WORKSPACE);
+          *last_part = 2;  // neither publish nor merge
+        } else {
+          *last_part = before == nparts - 1 ? 1 : 0;
+        }
+      }
+      named_bar_sync(1, 256);
+      float* blk_smem = reinterpret_cast<float*>(smem) + wg * kPartFloats;  // this head's block
+      auto blk = [&](int i, int h) {
+        return p.part_ws + ((int64_t)(item - part + i) * p.n_q_heads + h) * kPartFloats;
+      };
+      if (*last_part == 2) {
+        // corrupt workspace: nothing to do (status set above)
+      } else if (!*last_part) {
+        float4* ocol = reinterpret_cast<float4*>(blk_smem) + rit;
+#pragma unroll 1
+        for (int c = 0; c < kD / 32; ++c) {
+          float x[32];
+          own_chunk(c, x);
+#pragma unroll
+          for (int u = 0; u < 8; ++u)
+            ocol[(c * 8 + u) * kBM] = make_float4(x[4 * u], x[4 * u + 1], x[4 * u + 2], x[4 * u + 3]);
+        }
+        blk_smem[kBM * kD + rit] = m_run;
+        blk_smem[kBM * kD + kBM + rit] = l_sum;
+        fence_proxy_async_smem();
+        named_bar_sync(1, 256);
         if (elected) {
-          const int before = atomicAdd(cnt, 1);
-          if (before < 0 || before >= it.nparts) {
-            // the counter did not start at zero: the workspace was not zero-filled
-            if (p.status) atomicOr(p.status, TG_STATUS_WORKSPACE);
-            *last_part = 2;  // neither publish nor merge
-          } else {
-            *last_part = before == it.nparts - 1 ? 1 : 0;
-          }
+          bulk_store(blk(part, h0), smem, kPartFloats * 4);
+          bulk_store(blk(part, h0 + 1), smem + kPartFloats * 4, kPartFloats * 4);
+          bulk_commit_group();
+          bulk_wait_all();          // the partial is in global memory
+          fence_proxy_async_global();
+          st_release_gpu(p.part_ready + (int64_t)item * hg + head_grp, 1);
+        }
+      } else {
+        if (elected) {
+          bool ready = true;
+          for (int i = 0; i < nparts && ready; ++i)
+            if (i != part)
+              ready = wait_flag_gpu(p.part_ready + (int64_t)(item - part + i) * hg + head_grp,
+                                    abort_flag, p.status);
+          fence_proxy_async_global();  // the partials are read by bulk copies next
+          *parts_ready = ready ? 1 : 0;
         }
         named_bar_sync(1, 256);
-        auto blk = [&](int i, int h) {
-          return p.part_ws + ((int64_t)(it.item - it.part + i) * p.n_q_heads + h) * kPartFloats;
-        };
-        const int lp = *last_part;
-        if (lp == 0) {
-          // publish: coalesced float4 columns (group f of row r at f * 128 + r)
-          float4* ocol = reinterpret_cast<float4*>(blk(it.part, hh)) + rit;
-#pragma unroll 1
-          for (int c = 0; c < kD / 32; ++c) {
-            float x[32];
-            own_chunk(c, x);
-#pragma unroll
-            for (int u = 0; u < 8; ++u)
-              ocol[(c * 8 + u) * kBM] = make_float4(x[4 * u], x[4 * u + 1], x[4 * u + 2], x[4 * u + 3]);
-          }
-          blk(it.part, hh)[kBM * kD + rit] = m_run;
-          blk(it.part, hh)[kBM * kD + kBM + rit] = l_sum;
-          __threadfence();  // this thread's partial is visible GPU-wide before the flag
-          named_bar_sync(1, 256);
-          if (elected)
-            st_release_gpu(p.part_ready + (int64_t)it.item * hg + it.head_grp, 1);
-        } else if (lp == 1) {
+        const int np = nparts;
+        int copies = 0;
+        // stage part i's block (both heads) in shared memory; CTA-uniform outcome
+        auto stage = [&](int i) {
+          named_bar_sync(1, 256);  // nobody still reads the previous staged part
           if (elected) {
-            bool ready = true;
-            for (int i = 0; i < it.nparts && ready; ++i)
-              if (i != it.part)
-                ready = wait_flag_gpu(p.part_ready + (int64_t)(it.item - it.part + i) * hg +
-                                          it.head_grp,
-                                      abort_flag, p.status);
-            *parts_ready = ready ? 1 : 0;
+            fence_proxy_async_smem();
+            mbar_arrive_expect_tx(merge_full, 2 * kPartFloats * 4);
+            bulk_load(smem, blk(i, h0), kPartFloats * 4, merge_full);
+            bulk_load(smem + kPartFloats * 4, blk(i, h0 + 1), kPartFloats * 4, merge_full);
           }
-          named_bar_sync(1, 256);
-          if (*parts_ready) {
-            const int np = it.nparts;
-            // the parts' row maxima and sums (its own from registers, the others' from
-            // their published blocks; unrolled so the loads of a round are independent);
-            // the weights go to shared memory for the column loop
-            auto m_of = [&](int i) {
-              return i == it.part ? m_run : __ldcg(blk(i, hh) + kBM * kD + rit);
-            };
-            auto l_of = [&](int i) {
-              return i == it.part ? l_sum : __ldcg(blk(i, hh) + kBM * kD + kBM + rit);
-            };
-            float M = -INFINITY;
-#pragma unroll
-            for (int i = 0; i < kMaxParts; ++i)
-              if (i < np) M = fmaxf(M, m_of(i));
-            float* wts = reinterpret_cast<float*>(smem + AttnSmem::WTS) + wg * 128 + rit;
-            float L = 0.f;
-#pragma unroll
-            for (int i = 0; i < kMaxParts; ++i) {
-              if (i < np) {
-                const float wi = ex2_approx(m_of(i) - M);  // the part's weight
-                wts[i * 256] = wi;
-                L = i == 0 ? wi * l_of(i) : fmaf(wi, l_of(i), L);
-              }
-            }
+          const bool got = named_bar_and(
+              1, 256, mbar_wait(merge_full, (uint32_t)copies & 1u, abort_flag, p.status));
+          ++copies;
+          return got;
+        };
+        bool ok_m = *parts_ready != 0;
+        if (ok_m && np == 2) {
+          // one other part: stage it, then a single pass
+          const int other = 1 - part;
+          ok_m = stage(other);
+          if (ok_m) {
+            const float m_o = blk_smem[kBM * kD + rit], l_o = blk_smem[kBM * kD + kBM + rit];
+            const float M = fmaxf(m_run, m_o);
+            const float w_own = ex2_approx(m_run - M), w_o = ex2_approx(m_o - M);
+            const float w0 = part == 0 ? w_own : w_o, w1 = part == 0 ? w_o : w_own;
+            const float L = fmaf(w1, part == 0 ? l_o : l_sum, w0 * (part == 0 ? l_sum : l_o));
             const float inv = 1.0f / L;
-            // 16 columns at a time, the parts in order (small enough to keep the merge
-            // from taking registers the softmax loop needs)
+            const float4* g = reinterpret_cast<const float4*>(blk_smem) + rit;
 #pragma unroll 1
-            for (int c = 0; c < kD / 16; ++c) {
-              float acc[16];
-#pragma unroll 1
-              for (int i = 0; i < np; ++i) {
-                const float wgt = wts[i * 256];
-                float x[16];
-                if (i == it.part) {
-                  uint32_t ro[16];
-                  tmem_ld16(o_t + c * 16, ro);
-                  tmem_wait_ld();
+            for (int c = 0; c < kD / 32; ++c) {
+              float own[32], acc[32];
+              own_chunk(c, own);
 #pragma unroll
-                  for (int e = 0; e < 16; ++e) x[e] = __uint_as_float(ro[e]);
-                } else {
-                  const float4* g4 = reinterpret_cast<const float4*>(blk(i, hh)) + rit;
+              for (int u = 0; u < 8; ++u) {
+                const float4 x = g[(c * 8 + u) * kBM];
+                const float xs[4] = {x.x, x.y, x.z, x.w};
 #pragma unroll
-                  for (int u = 0; u < 4; ++u) {
-                    const float4 v4 = __ldcg(g4 + (c * 4 + u) * kBM);
-                    x[4 * u] = v4.x;
-                    x[4 * u + 1] = v4.y;
-                    x[4 * u + 2] = v4.z;
-                    x[4 * u + 3] = v4.w;
-                  }
+                for (int e = 0; e < 4; ++e) {
+                  const float a0 = part == 0 ? own[4 * u + e] : xs[e];
+                  const float a1 = part == 0 ? xs[e] : own[4 * u + e];
+                  acc[4 * u + e] = fmaf(w1, a1, w0 * a0);
                 }
-#pragma unroll
-                for (int e = 0; e < 16; ++e) acc[e] = i == 0 ? wgt * x[e] : fmaf(wgt, x[e], acc[e]);
               }
-              if (row_valid) {
-                uint32_t wv[8];
-#pragma unroll
-                for (int e = 0; e < 8; ++e) wv[e] = pack_bf16x2(acc[2 * e] * inv, acc[2 * e + 1] * inv);
-                uint4* dst = reinterpret_cast<uint4*>(p.o + (it.row0 + r) * p.ld_o + (int64_t)hh * kD + c * 16);
-                dst[0] = make_uint4(wv[0], wv[1], wv[2], wv[3]);
-                dst[1] = make_uint4(wv[4], wv[5], wv[6], wv[7]);
-              }
+              put_chunk(c, acc, inv);
             }
             store_lse(M, L);
           }
-          named_bar_sync(1, 256);  // every read of the partials is done
-          if (elected) {  // leave the counters zeroed for the next call
-            for (int i = 0; i < it.nparts; ++i)
-              p.part_ready[(int64_t)(it.item - it.part + i) * hg + it.head_grp] = 0;
-            *cnt = 0;
+        } else if (ok_m) {
+          // several other parts: batch-load every row max and sum, then one pass per
+          // part in part order with the running sum kept in the TMEM columns S used
+          float mi[kMaxParts], li[kMaxParts];
+#pragma unroll
+          for (int i = 0; i < kMaxParts; ++i) {
+            if (i < np) {
+              mi[i] = i == part ? m_run : __ldcg(blk(i, hh) + kBM * kD + rit);
+              li[i] = i == part ? l_sum : __ldcg(blk(i, hh) + kBM * kD + kBM + rit);
+            }
           }
+          float M = -INFINITY;
+#pragma unroll
+          for (int i = 0; i < kMaxParts; ++i)
+            if (i < np) M = fmaxf(M, mi[i]);
+          float L = 0.f;
+#pragma unroll
+          for (int i = 0; i < kMaxParts; ++i) {
+            if (i < np) {
+              mi[i] = ex2_approx(mi[i] - M);  // from here on: the part's weight
+              L = i == 0 ? mi[i] * li[i] : fmaf(mi[i], li[i], L);
+            }
+          }
+          const float inv = 1.0f / L;
+#pragma unroll 1
+          for (int i = 0; i < np && ok_m; ++i) {
+            float w = mi[0];
+#pragma unroll
+            for (int t = 1; t < kMaxParts; ++t)
+              if (t == i) w = mi[t];
+            if (i != part && !(ok_m = stage(i))) break;
+            const float4* g = reinterpret_cast<const float4*>(blk_smem) + rit;
+#pragma unroll 1
+            for (int c = 0; c < kD / 32; ++c) {
+              float acc[32];
+              if (i > 0) {
+                uint32_t ra[32];
+                tmem_ld32(s_t + c * 32, ra);
+                tmem_wait_ld();
+#pragma unroll
+                for (int e = 0; e < 32; ++e) acc[e] = __uint_as_float(ra[e]);
+              }
+              float x[32];
+              if (i == part) {
+                own_chunk(c, x);
+              } else {
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                  const float4 v4 = g[(c * 8 + u) * kBM];
+                  x[4 * u] = v4.x;
+                  x[4 * u + 1] = v4.y;
+                  x[4 * u + 2] = v4.z;
+                  x[4 * u + 3] = v4.w;
+                }
+              }
+#pragma unroll
+              for (int e = 0; e < 32; ++e) acc[e] = i == 0 ? w * x[e] : fmaf(w, x[e], acc[e]);
+              if (i == np - 1) {
+                put_chunk(c, acc, inv);
+              } else {
+                uint32_t wa[32];
+#pragma unroll
+                for (int e = 0; e < 32; ++e) wa[e] = __float_as_uint(acc[e]);
+                tmem_st32(s_t + c * 32, wa);
+                tmem_wait_st();
+              }
+            }
+          }
+          if (ok_m) store_lse(M, L);
         }
-        // lp == 2: corrupt workspace, nothing to do (status set above)
+        // after an abort: the last staged copy may still be landing in shared memory
+        if (!ok_m && copies > 0 && elected)
+          mbar_wait(merge_full, (uint32_t)(copies - 1) & 1u, nullptr, p.status);
+        const int ok_all = named_bar_and(1, 256, ok_m);
+        if (ok_all) flush_out();
+        named_bar_sync(1, 256);  // every read of the partials is done
+        if (elected) {  // leave the counters zeroed for the next call
+          for (int i = 0; i < nparts; ++i)
+            p.part_ready[(int64_t)(item - part + i) * hg + head_grp] = 0;
+          *cnt = 0;
+        }
       }
-      // this head's O has been read: the next item's first PV may overwrite it
-      tc_fence_before();
-      mbar_arrive(&o_empty[wg]);
-      jt += nt;
-      ++ic;
     }
+    if (elected) bulk_wait_all();  // TMA/bulk stores have read shared memory and landed
     tc_fence_before();
   }
   __syncthreads();
@@ -781,40 +776,24 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
-  // the last CTA to finish leaves the work counter at zero for the next call
-  if (tid == 0 && p.sched) {
-    __threadfence();
-    if (atomicAdd(p.sched + 1, 1) == (int)gridDim.x - 1) {
-      p.sched[0] = 0;
-      p.sched[1] = 0;
-    }
-  }
 }
 
 // Work plan: the key-tile chunk per item and the item count per request, chosen to
-// minimise the estimated makespan of the persistent kernel.
+// minimise the estimated makespan over the SMs (one CTA per SM at a time).
 struct AttnPlan {
   int chunk;
   int n_items;
   bool split;
 };
 
-// Makespan (in key-tile units) of the work items of `chunk` handed out in order to the
-// CTAs as they free up (the persistent kernel's work counter): list scheduling, heaviest
-// items first within a request.  An item costs its key tiles plus a fixed kItemOverhead
-// (the softmax start and the output of its rows), a part of a split tile kPartOverhead
-// more (publishing or merging partial results).
-constexpr double kItemOverhead = 0.4;
-constexpr double kPartOverhead = 0.8;
+// Makespan (in key-tile units) of launching the items of `chunk` in launch order on
+// `sms` SMs, one CTA per SM at a time: the block scheduler hands each CTA to the first
+// SM that frees up, which is list scheduling in launch order (heaviest first within a
+// request).  Each CTA also pays a fixed prologue/epilogue cost of kCtaOverhead tiles.
+constexpr double kCtaOverhead = 1.5;
 double simulate_makespan(const int32_t* cu_kept_host, int batch, int head_groups, int sms,
                          int chunk) {
-  int64_t n_work = 0;
-  for (int b = 0; b < batch; ++b) {
-    const int nt = ceil_div(cu_kept_host[b + 1] - cu_kept_host[b], kBM);
-    for (int qt = 0; qt < nt; ++qt) n_work += (int64_t)ceil_div(qt + 1, chunk) * head_groups;
-  }
-  const int ctas = (int)std::min<int64_t>(sms, std::max<int64_t>(n_work, 1));
-  std::vector<double> busy((size_t)ctas, 0.0);  // min-heap of CTA finish times
+  std::vector<double> busy((size_t)sms, 0.0);  // min-heap of SM finish times
   std::make_heap(busy.begin(), busy.end(), std::greater<double>());
   double makespan = 0.0;
   for (int b = 0; b < batch; ++b) {
@@ -823,10 +802,9 @@ double simulate_makespan(const int32_t* cu_kept_host, int batch, int head_groups
       const int np = ceil_div(qt + 1, chunk);
       for (int part = 0; part < np; ++part) {
         const int units = std::min(qt + 1, (part + 1) * chunk) - part * chunk;
-        const double cost = units + kItemOverhead + (np > 1 ? kPartOverhead : 0.0);
         for (int h = 0; h < head_groups; ++h) {
           std::pop_heap(busy.begin(), busy.end(), std::greater<double>());
-          busy.back() += cost;
+          busy.back() += units + kCtaOverhead;
           makespan = std::max(makespan, busy.back());
           std::push_heap(busy.begin(), busy.end(), std::greater<double>());
         }
@@ -855,17 +833,14 @@ int make_plan(const int32_t* cu_kept_host, int batch, int head_groups, int sms, 
   if (layout == cached_layout && cached_hg == head_groups && cached_sms == sms) {
     plan = cached_plan;
   } else {
-    // Candidates: no split, and every chunk up to a few times the balanced share of one
-    // CTA (at most kMaxParts parts per tile).
+    // Candidates: no split, and chunks near the balanced share of one SM.
     const double share = (double)units * head_groups / sms;
     int best = std::max(max_tiles, 1);
-    const double unsplit = simulate_makespan(cu_kept_host, batch, head_groups, sms, best);
-    // a split must shorten the estimate by a tenth to pay for its partials' traffic
-    double best_cost = 0.9 * unsplit;
-    const int c_hi = std::min(max_tiles - 1, (int)std::ceil(3.0 * share) + 1);
-    for (int c = 2; c <= c_hi; ++c) {
-      if (ceil_div(max_tiles, c) > kMaxParts) continue;
-      const double cost = simulate_makespan(cu_kept_host, batch, head_groups, sms, c);
+    double best_cost = simulate_makespan(cu_kept_host, batch, head_groups, sms, best);
+    for (double f : {0.5, 0.75, 1.0, 1.25, 1.5, 2.0, 3.0}) {
+      const int c = (int)std::ceil(share * f);
+      if (c < 2 || c >= max_tiles || ceil_div(max_tiles, c) > kMaxParts) continue;
+      const double cost = simulate_makespan(cu_kept_host, batch, head_groups, sms, c) + 1.0;
       if (cost < best_cost) {
         best_cost = cost;
         best = c;
@@ -890,10 +865,9 @@ int make_plan(const int32_t* cu_kept_host, int batch, int head_groups, int sms, 
   return TG_OK;
 }
 
-// Workspace: the persistent kernel's work counters (256 bytes), then, for a split plan,
-// the parts' partial results and at a 256-byte boundary two int32 arrays indexed by
-// (work item, head group): arrival counters (used at a tile's first item) and ready flags.
-constexpr size_t kSchedBytes = 256;
+// Split workspace: the parts' partial results, then at a 256-byte boundary two int32
+// arrays indexed by (work item, head group): arrival counters (used at a tile's first
+// item) and ready flags.
 size_t part_bytes(int64_t n_items, int n_q_heads) {
   return ((size_t)n_items * n_q_heads * kPartFloats * sizeof(float) + 255) & ~size_t(255);
 }
@@ -931,9 +905,10 @@ extern "C" size_t tg_gated_attention_workspace_size(const int32_t* cu_kept_host,
     return 0;
   AttnPlan plan;
   static thread_local int32_t prefix[kMaxBatch + 1];
-  if (make_plan(cu_kept_host, batch, n_q_heads / 2, sm_count(), plan, prefix) != TG_OK) return 0;
-  return kSchedBytes + (plan.split ? split_workspace_bytes(plan.n_items, n_q_heads, n_q_heads / 2)
-                                   : 0);
+  if (make_plan(cu_kept_host, batch, n_q_heads / 2, sm_count(), plan, prefix) != TG_OK ||
+      !plan.split)
+    return 0;
+  return split_workspace_bytes(plan.n_items, n_q_heads, n_q_heads / 2);
 }
 
 extern "C" int tg_gated_attention(const tg_bf16* q, int64_t ld_q, const tg_bf16* k, int64_t ld_k,
@@ -972,17 +947,13 @@ extern "C" int tg_gated_attention(const tg_bf16* q, int64_t ld_q, const tg_bf16*
   const int head_groups = n_kv_heads * (group / 2);
   AttnPlan plan;
   TG_TRY(make_plan(cu_kept_host, batch, head_groups, sm_count(), plan, prm.item_prefix));
-  // With room for the work counters the kernel is persistent; with room for the partial
-  // results too, long query tiles are split as planned.
-  const bool persistent = workspace && workspace_bytes >= kSchedBytes;
-  const bool split = plan.split && persistent &&
-                     workspace_bytes >= kSchedBytes + split_workspace_bytes(plan.n_items, n_q_heads,
-                                                                            head_groups);
-  if (plan.split && !split) {
+  const size_t need = split_workspace_bytes(plan.n_items, n_q_heads, head_groups);
+  if (plan.split && (!workspace || workspace_bytes < need)) {
     // no room for partial results: one item per query tile
     int max_tiles = 1;
     for (int b = 0; b < batch; ++b)
       max_tiles = std::max(max_tiles, ceil_div(cu_kept_host[b + 1] - cu_kept_host[b], kBM));
+    plan.split = false;
     plan.chunk = max_tiles;
     int items = 0;
     for (int b = 0; b < batch; ++b) {
@@ -991,12 +962,12 @@ extern "C" int tg_gated_attention(const tg_bf16* q, int64_t ld_q, const tg_bf16*
     }
     plan.n_items = items;
   }
-  plan.split = split;
 
-  CUtensorMap tq, tk, tv;
+  CUtensorMap tq, tk, tv, to;
   TG_TRY(make_tmap_bf16_2d(&tq, q, (uint64_t)k_total, (uint64_t)n_q_heads * kD, (uint64_t)ld_q, 64, kBM));
   TG_TRY(make_tmap_bf16_2d(&tk, k, (uint64_t)k_total, (uint64_t)n_kv_heads * kD, (uint64_t)ld_k, 64, kBN));
   TG_TRY(make_tmap_bf16_2d(&tv, v, (uint64_t)k_total, (uint64_t)n_kv_heads * kD, (uint64_t)ld_v, 64, kBN));
+  TG_TRY(make_tmap_bf16_2d(&to, o, (uint64_t)k_total, (uint64_t)n_q_heads * kD, (uint64_t)ld_o, 64, kBM));
   prm.cu_kept = cu_kept;
   prm.kept_pos = kept_pos;
   prm.kept_bias = kept_bias;
@@ -1013,19 +984,15 @@ extern "C" int tg_gated_attention(const tg_bf16* q, int64_t ld_q, const tg_bf16*
   prm.batch = batch;
   prm.status = status;
   prm.chunk = plan.chunk;
-  unsigned char* ws = static_cast<unsigned char*>(workspace);
-  prm.sched = persistent ? reinterpret_cast<int*>(ws) : nullptr;
-  prm.part_ws = split ? reinterpret_cast<float*>(ws + kSchedBytes) : nullptr;
-  prm.part_count = split ? reinterpret_cast<int*>(ws + kSchedBytes +
-                                                  part_bytes(plan.n_items, n_q_heads))
-                         : nullptr;
-  prm.part_ready = split ? prm.part_count + (int64_t)plan.n_items * head_groups : nullptr;
+  prm.part_ws = plan.split ? static_cast<float*>(workspace) : nullptr;
+  prm.part_count = plan.split ? reinterpret_cast<int*>(static_cast<unsigned char*>(workspace) +
+                                                       part_bytes(plan.n_items, n_q_heads))
+                              : nullptr;
+  prm.part_ready = plan.split ? prm.part_count + (int64_t)plan.n_items * head_groups : nullptr;
 
-  const int64_t n_work = (int64_t)plan.n_items * head_groups;
-  if (n_work > 0x7FFFFFFF) return TG_ERR_UNSUPPORTED_SHAPE;
-  prm.n_work = (int)n_work;
-  const int64_t grid = persistent ? std::min<int64_t>(n_work, sm_count()) : n_work;
+  const int64_t grid = (int64_t)plan.n_items * head_groups;
+  if (grid > 0x7FFFFFFF) return TG_ERR_UNSUPPORTED_SHAPE;
   TG_TRY(launch(gated_attention_kernel, dim3((unsigned)grid), dim3(kThreads), AttnSmem::BYTES,
-                (cudaStream_t)stream, tq, tk, tv, prm));
+                (cudaStream_t)stream, tq, tk, tv, to, prm));
   return TG_OK;
 }
