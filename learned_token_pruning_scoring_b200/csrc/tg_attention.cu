@@ -833,13 +833,16 @@ int make_plan(const int32_t* cu_kept_host, int batch, int head_groups, int sms, 
   if (layout == cached_layout && cached_hg == head_groups && cached_sms == sms) {
     plan = cached_plan;
   } else {
-    // Candidates: no split, and chunks near the balanced share of one SM.
+    // Candidates: no split, and every chunk up to three times the balanced share of one
+    // SM (a split pays one more tile's worth for its merge, and must shorten the estimate
+    // by a twentieth).
     const double share = (double)units * head_groups / sms;
     int best = std::max(max_tiles, 1);
-    double best_cost = simulate_makespan(cu_kept_host, batch, head_groups, sms, best);
-    for (double f : {0.5, 0.75, 1.0, 1.25, 1.5, 2.0, 3.0}) {
-      const int c = (int)std::ceil(share * f);
-      if (c < 2 || c >= max_tiles || ceil_div(max_tiles, c) > kMaxParts) continue;
+    // a split must also shorten the estimate by a twentieth (its partials' traffic)
+    double best_cost = 0.95 * simulate_makespan(cu_kept_host, batch, head_groups, sms, best);
+    const int c_hi = std::min(max_tiles - 1, (int)std::ceil(3.0 * share));
+    for (int c = 2; c <= c_hi; ++c) {
+      if (ceil_div(max_tiles, c) > kMaxParts) continue;
       const double cost = simulate_makespan(cu_kept_host, batch, head_groups, sms, c) + 1.0;
       if (cost < best_cost) {
         best_cost = cost;
