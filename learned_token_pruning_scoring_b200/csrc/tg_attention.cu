@@ -768,7 +768,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     }
-    if (elected) bulk_wait_all();  // TMA/bulk stores have read shared memory and landed
+    // TMA/bulk stores have read shared memory before the CTA exits (their global writes
+    // are complete, like every other write of the grid, when the kernel is)
+    if (elected) bulk_wait_read_all();
     tc_fence_before();
   }
   __syncthreads();

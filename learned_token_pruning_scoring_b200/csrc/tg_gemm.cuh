@@ -417,27 +417,36 @@ __device__ __forceinline__ void add_partials(uint32_t (&r)[32], int chunk,
   }
 }
 
+// Per-row inputs of the pair epilogue that do not depend on the accumulator; the
+// epilogue warps read them while the tile's MMAs run.
+__device__ __forceinline__ float pair_row_rscale(const GemmParams& p, int64_t grow) {
+  return (p.rmsnorm && p.row_ssq_in && grow < p.M) ? rscale_from_ssq(p, grow) : 1.0f;
+}
+template <int EPI>
+__device__ __forceinline__ int pair_row_pos(const GemmParams& p, int64_t grow, int n0) {
+  if (EPI != EpiQKV && EPI != EpiQKVNorm) return 0;
+  const bool live = grow < p.M;
+  int pos = (live && n0 < p.q_cols + p.k_cols) ? p.pos[grow] : 0;
+  if (pos < 0 || pos >= p.max_pos) {
+    if (live && p.status) atomicOr(p.status, TG_STATUS_BOUNDS);
+    pos = 0;
+  }
+  return pos;
+}
+
 // Columns [128 h, 128 h + 128) of one 256 x 256 output tile of the pair (each CTA: 128
 // rows, staged in shared memory as four swizzled 64-column boxes); `row` is the thread's
 // row in the CTA's half, `tacc` the TMEM address of the row's accumulator (lane quarter
-// and buffer included).
+// and buffer included); `rscale` and `pos` come from pair_row_rscale / pair_row_pos.
 template <int EPI, int MAXADD>
 __device__ __forceinline__ void pair_epilogue_half(const GemmParams& p, unsigned char* out_s,
                                                    uint32_t tacc, int row, int64_t grow, int n0,
-                                                   int h, bool has_res,
+                                                   int h, bool has_res, float rscale, int pos,
                                                    const float4* const (&adds)[MAXADD],
                                                    int n_add) {
   const bool live = grow < p.M;
-  const float rscale =
-      (p.rmsnorm && p.row_ssq_in && live) ? rscale_from_ssq(p, grow) : 1.0f;
   if (EPI == EpiQKV || EPI == EpiQKVNorm) {
     const bool rope = n0 < p.q_cols + p.k_cols;
-    int pos = (rope && live) ? p.pos[grow] : 0;
-    if (pos < 0 || pos >= p.max_pos) {
-      if (live && p.status) atomicOr(p.status, TG_STATUS_BOUNDS);
-      pos = 0;
-    }
-    const float4* cs_row = reinterpret_cast<const float4*>(p.cos_sin + (int64_t)pos * 128);
     // QK-norm: this group's 128 columns are one Q or K head of the row; a first pass
     // over them gives the head's RMS
     float qk = 1.f;
@@ -460,6 +469,7 @@ __device__ __forceinline__ void pair_epilogue_half(const GemmParams& p, unsigned
       qk = rsqrtf(ss * rscale * rscale * (1.0f / 128.0f) + p.qk_eps);
     }
     const float scale = rscale * qk;
+    const float4* cs_row = reinterpret_cast<const float4*>(p.cos_sin + (int64_t)pos * 128);
 #pragma unroll 1
     for (int pr = 0; pr < 2; ++pr) {
       // 32-column pieces ca and ca + 2 hold columns i and i + 64 of one 128-column head
@@ -875,6 +885,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(320, 1)
       const PairJob& jb = job ? job1 : job0;
       const bool with_res = pc.kind != 2 && has_res(job);
       const int64_t m0 = (int64_t)rp * 256 + rank * 128;
+      // job 1 of a chain reads job 0's row sums of squares only after the wait below
+      const bool late_ssq = job && chain.ready;
+      float rscale = (pc.kind != 2 && !late_ssq) ? pair_row_rscale(jb.p, m0 + row) : 1.0f;
+      const int pos = pc.kind == 2 ? 0
+                      : job        ? pair_row_pos<EPI1>(jb.p, m0 + row, n0)
+                                   : pair_row_pos<EPI0>(jb.p, m0 + row, n0);
       bool ok = mbar_wait(&acc_full[b], (uint32_t)(i >> 1) & 1u, abort_flag, status);
       if (ok && with_res) ok = mbar_wait(&res_full[g], (uint32_t)res_used & 1u, abort_flag, status);
       if (with_res) ++res_used;
@@ -900,7 +916,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(320, 1)
       // job 1 reads job 0's row sums of squares: its producer acquired job 0's release
       // before the loads behind this accumulator; a device fence orders this thread's
       // reads after it too (the counter itself may already be reset by then)
-      if (job && chain.ready) __threadfence();
+      if (late_ssq) __threadfence();
       // one decision for the group's four warps (they meet at named barriers below)
       if (!named_bar_and(bar_id, 128, ok)) break;
       tc_fence_after();
@@ -934,12 +950,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(320, 1)
         named_bar_sync(bar_id, 128);
         continue;
       }
+      if (late_ssq) rscale = pair_row_rscale(jb.p, m0 + row);
       if (job)
         pair_epilogue_half<EPI1, kMaxPieces>(jb.p, out_s, tacc, row, m0 + row, n0, g, with_res,
-                                             adds, n_add);
+                                             rscale, pos, adds, n_add);
       else
         pair_epilogue_half<EPI0, kMaxPieces>(jb.p, out_s, tacc, row, m0 + row, n0, g, with_res,
-                                             adds, n_add);
+                                             rscale, pos, adds, n_add);
       const bool publish = !job && chain.ready;  // job 1 waits for these rows
       if (publish) __threadfence();  // row sums of squares visible before the count
       tc_fence_before();
@@ -981,12 +998,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(320, 1)
       named_bar_sync(bar_id, 128);
     }
     if (elected) {
-      bulk_wait_all();
+      // the staging boxes are read before the CTA exits; the stores' global writes are
+      // complete, like every other write of the grid, when the kernel is
+      bulk_wait_read_all();
       // after an abort: a residual load may still be landing in the staging boxes
       if (res_loads > res_used)
         mbar_wait(&res_full[g], (uint32_t)(res_loads - 1) & 1u, nullptr, status);
     }
   }
+  __syncwarp();  // the role branches above diverge inside warps 0 and 1
   __syncthreads();
   cluster_sync_all();  // no CTA leaves while the pair's MMAs or arrives may touch it
   if (warp == 1) {
