@@ -605,25 +605,25 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (*last_part == 2) {
         // corrupt workspace: nothing to do (status set above)
       } else if (!*last_part) {
-        float4* ocol = reinterpret_cast<float4*>(blk_smem) + rit;
+        // straight from TMEM to this head's block, one row per thread (a warp's stores
+        // of one 4-column group are 512 contiguous bytes)
+        float* dst = blk(part, hh);
+        float4* ocol = reinterpret_cast<float4*>(dst) + rit;
 #pragma unroll 1
         for (int c = 0; c < kD / 32; ++c) {
           float x[32];
           own_chunk(c, x);
 #pragma unroll
           for (int u = 0; u < 8; ++u)
-            ocol[(c * 8 + u) * kBM] = make_float4(x[4 * u], x[4 * u + 1], x[4 * u + 2], x[4 * u + 3]);
+            __stcg(ocol + (c * 8 + u) * kBM,
+                   make_float4(x[4 * u], x[4 * u + 1], x[4 * u + 2], x[4 * u + 3]));
         }
-        blk_smem[kBM * kD + rit] = m_run;
-        blk_smem[kBM * kD + kBM + rit] = l_sum;
-        fence_proxy_async_smem();
+        __stcg(dst + kBM * kD + rit, m_run);
+        __stcg(dst + kBM * kD + kBM + rit, l_sum);
+        __threadfence();  // this thread's rows are visible GPU-wide before the flag
         named_bar_sync(1, 256);
         if (elected) {
-          bulk_store(blk(part, h0), smem, kPartFloats * 4);
-          bulk_store(blk(part, h0 + 1), smem + kPartFloats * 4, kPartFloats * 4);
-          bulk_commit_group();
-          bulk_wait_all();          // the partial is in global memory
-          fence_proxy_async_global();
+          fence_proxy_async_global();  // the merging part reads the block by bulk copies
           st_release_gpu(p.part_ready + (int64_t)item * hg + head_grp, 1);
         }
       } else {
@@ -791,29 +791,50 @@ struct AttnPlan {
 // Makespan (in key-tile units) of launching the items of `chunk` in launch order on
 // `sms` SMs, one CTA per SM at a time: the block scheduler hands each CTA to the first
 // SM that frees up, which is list scheduling in launch order (heaviest first within a
-// request).  Each CTA also pays a fixed prologue/epilogue cost of kCtaOverhead tiles.
-constexpr double kCtaOverhead = 1.5;
+// request).  Costs, measured with a global-timer trace of every CTA on a B200 (one key
+// tile of both heads ~2.2 us): every CTA pays kCtaOverhead for its prologue (first MMA
+// ~4.5 us after the start) and output; a part of a split tile that publishes its partial
+// pays kPublish; the part that arrives last waits for the others' partials and pays
+// kMergePart per other part before the tile is done.
+constexpr double kCtaOverhead = 3.0;
+constexpr double kPublish = 1.0;
+constexpr double kMergePart = 1.3;
 double simulate_makespan(const int32_t* cu_kept_host, int batch, int head_groups, int sms,
                          int chunk) {
-  std::vector<double> busy((size_t)sms, 0.0);  // min-heap of SM finish times
-  std::make_heap(busy.begin(), busy.end(), std::greater<double>());
-  double makespan = 0.0;
+  std::vector<double> busy((size_t)sms, 0.0);  // finish time of each SM's last CTA
+  auto first_free = [&]() {
+    return (int)(std::min_element(busy.begin(), busy.end()) - busy.begin());
+  };
+  std::vector<double> fin;
+  std::vector<int> sm_of;
   for (int b = 0; b < batch; ++b) {
     const int nt = ceil_div(cu_kept_host[b + 1] - cu_kept_host[b], kBM);
     for (int qt = nt - 1; qt >= 0; --qt) {
       const int np = ceil_div(qt + 1, chunk);
+      fin.assign((size_t)np * head_groups, 0.0);
+      sm_of.assign((size_t)np * head_groups, 0);
       for (int part = 0; part < np; ++part) {
         const int units = std::min(qt + 1, (part + 1) * chunk) - part * chunk;
         for (int h = 0; h < head_groups; ++h) {
-          std::pop_heap(busy.begin(), busy.end(), std::greater<double>());
-          busy.back() += units + kCtaOverhead;
-          makespan = std::max(makespan, busy.back());
-          std::push_heap(busy.begin(), busy.end(), std::greater<double>());
+          const int s = first_free();
+          busy[s] += units + kCtaOverhead + (np > 1 ? kPublish : 0.0);
+          fin[(size_t)part * head_groups + h] = busy[s];
+          sm_of[(size_t)part * head_groups + h] = s;
+        }
+      }
+      if (np > 1) {
+        for (int h = 0; h < head_groups; ++h) {
+          int last = 0;
+          for (int part = 1; part < np; ++part)
+            if (fin[(size_t)part * head_groups + h] > fin[(size_t)last * head_groups + h])
+              last = part;
+          busy[sm_of[(size_t)last * head_groups + h]] =
+              fin[(size_t)last * head_groups + h] + kMergePart * (np - 1);
         }
       }
     }
   }
-  return makespan;
+  return *std::max_element(busy.begin(), busy.end());
 }
 
 int make_plan(const int32_t* cu_kept_host, int batch, int head_groups, int sms, AttnPlan& plan,
@@ -836,16 +857,14 @@ int make_plan(const int32_t* cu_kept_host, int batch, int head_groups, int sms, 
     plan = cached_plan;
   } else {
     // Candidates: no split, and every chunk up to three times the balanced share of one
-    // SM (a split pays one more tile's worth for its merge, and must shorten the estimate
-    // by a twentieth).
+    // SM; a split must shorten the estimate by a fiftieth.
     const double share = (double)units * head_groups / sms;
     int best = std::max(max_tiles, 1);
-    // a split must also shorten the estimate by a twentieth (its partials' traffic)
-    double best_cost = 0.95 * simulate_makespan(cu_kept_host, batch, head_groups, sms, best);
+    double best_cost = 0.98 * simulate_makespan(cu_kept_host, batch, head_groups, sms, best);
     const int c_hi = std::min(max_tiles - 1, (int)std::ceil(3.0 * share));
     for (int c = 2; c <= c_hi; ++c) {
       if (ceil_div(max_tiles, c) > kMaxParts) continue;
-      const double cost = simulate_makespan(cu_kept_host, batch, head_groups, sms, c) + 1.0;
+      const double cost = simulate_makespan(cu_kept_host, batch, head_groups, sms, c);
       if (cost < best_cost) {
         best_cost = cost;
         best = c;

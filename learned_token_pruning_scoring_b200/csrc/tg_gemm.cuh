@@ -614,8 +614,9 @@ struct PairChain {
 // shared out evenly, in tile order, as one contiguous range of tail_units per cluster
 // ("pieces").  A piece holding a tile's first k-block finishes that tile: it runs last
 // in its cluster, waits for the tile's other pieces (each the first piece of a later
-// cluster, run first there), adds their fp32 partial sums in k order to its own
-// accumulator and runs the epilogue; the other pieces only publish their partial sums.
+// cluster's range, run before that cluster's whole tiles), adds their fp32 partial sums
+// in k order to its own accumulator and runs the epilogue; the other pieces only
+// publish their partial sums.
 // A cluster has at most one such contributing piece, so partials and ready flags are
 // indexed by cluster: part[((c * 2 + rank) * 2 + group) * 32 * 128 + f * 128 + row]
 // (float4, f = 4-column group within the epilogue group's 128 columns) and
@@ -634,29 +635,26 @@ struct Piece {
   int kind;  // 0: whole tile, 1: finisher (first k-blocks), 2: contributor
 };
 
-// The pieces of cluster c in the order the cluster runs them.
+// The pieces of cluster c in the order the cluster runs them: a tail range that starts
+// inside a tile begins with a contributing piece, which runs first (its partial sums are
+// then published before the cluster's first epilogue, and the finisher that waits for
+// them does not wait behind that epilogue); then the whole tiles; then the rest of the
+// range, whose last piece may be a finisher.
 struct PieceIter {
   int c, C, n_tiles, nk, dp_tiles;
   int64_t u, u1;
   int i;
-  bool split;
+  bool split, lead_done;
   __device__ PieceIter(int c_, int C_, int n_tiles_, int nk_, const PairSplit& sp)
       : c(c_), C(C_), n_tiles(n_tiles_), nk(nk_), dp_tiles(0), u(0), u1(0), i(0),
-        split(sp.part != nullptr) {
+        split(sp.part != nullptr), lead_done(false) {
     if (split) {
       dp_tiles = sp.dp_tiles;
       u = sp.tail_units * c / C;
       u1 = sp.tail_units * (c + 1) / C;
     }
   }
-  __device__ bool next(Piece& pc) {
-    const int t = c + i * C;
-    if (!split ? t < n_tiles : t < dp_tiles) {
-      pc = {t, 0, nk, 0};
-      ++i;
-      return true;
-    }
-    if (!split || u >= u1) return false;
+  __device__ bool tail_piece(Piece& pc) {
     const int tt = (int)(u / nk);
     const int kb0 = (int)(u % nk);
     const int64_t left = u1 - u;
@@ -664,6 +662,20 @@ struct PieceIter {
     pc = {dp_tiles + tt, kb0, kb1, kb0 == 0 ? (kb1 == nk ? 0 : 1) : 2};
     u += kb1 - kb0;
     return true;
+  }
+  __device__ bool next(Piece& pc) {
+    if (split && !lead_done) {
+      lead_done = true;
+      if (u < u1 && u % nk != 0) return tail_piece(pc);
+    }
+    const int t = c + i * C;
+    if (!split ? t < n_tiles : t < dp_tiles) {
+      pc = {t, 0, nk, 0};
+      ++i;
+      return true;
+    }
+    if (!split || u >= u1) return false;
+    return tail_piece(pc);
   }
 };
 

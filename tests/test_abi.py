@@ -200,3 +200,30 @@ def test_scorer_backward_argument_checks(lib):
     big = lib.tg_gate_score_backward_workspace_size(50000, 2048, 256, 2)
     # du' alone is 512 bytes per token
     assert small > 500 * 512 and big - small >= (50000 - 500) * 512
+
+
+def test_attention_split_plan(lib):
+    # The split plan is host logic: tg_gated_attention_workspace_size is the number of
+    # work items times the per-item bytes (partials of every q head, counter and flag
+    # per head group), 0 when no query tile is split.
+    def items(lengths, hq, hkv):
+        cu = np.concatenate([[0], np.cumsum(lengths)]).astype(np.int32)
+        ws = lib.tg_gated_attention_workspace_size(cu.ctypes.data_as(C.c_void_p), len(lengths),
+                                                   hq, hkv, 128)
+        return ws // (hq * (128 * 128 + 2 * 128) * 4 + 8 * (hq // 2))
+
+    def chunk_of(lengths, n_items):
+        tiles = [-(-n // 128) for n in lengths]
+        return [c for c in range(1, max(tiles) + 1)
+                if sum(-(-(qt + 1) // c) for t in tiles for qt in range(t)) == n_items]
+
+    # 16 q / 8 kv heads, one 1638-row request: the six heaviest query tiles in two parts
+    n = items([1638], 16, 8)
+    assert n == 19 and chunk_of([1638], n) == [7]
+    # long single requests and the eight-request ragged batch balance without splitting
+    assert items([13107], 16, 8) == 0
+    assert items([8192], 16, 8) == 0
+    assert items([1638, 819, 410, 1229, 205, 1024, 614, 1433], 16, 8) == 0
+    # one head group: most tiles split, the longest into six parts
+    n = items([2000], 2, 1)
+    assert chunk_of([2000], n) == [3]

@@ -542,6 +542,25 @@ def test_attention_split_varlen_requests(tg):
     assert (lse - lse2).abs().max() <= 1e-4
 
 
+def test_attention_split_many_parts(tg):
+    # One head group (2 q heads, 1 kv head): the plan cuts the request's 16 query tiles
+    # into several key-range parts each, which the last-arriving part merges in part
+    # order.  The chunk is read back from the workspace size (items x per-item bytes).
+    n, Hq, Hkv = 2000, 2, 1
+    q, k, v, pos, bias, gamma, cu = _attn_inputs([n], Hq, Hkv, seed=n, pos_spread=5)
+    per_item = Hq * (128 * 128 + 2 * 128) * 4 + 8 * (Hq // 2)
+    items = tg.tg_gated_attention_workspace_size(cu, Hq, Hkv) // per_item
+    tiles = -(-n // 128)
+    chunks = [c for c in range(1, tiles + 1)
+              if sum(-(-(qt + 1) // c) for qt in range(tiles)) == items]
+    assert chunks and -(-tiles // chunks[-1]) > 2, (items, chunks)
+    o, lse = _run_attention(tg, q, k, v, pos, bias, gamma, 1.0, cu, Hq, Hkv)
+    _check_attention(o, lse, q, k, v, pos, bias, gamma, 1.0, cu, Hq, Hkv)
+    o2, lse2 = _run_attention(tg, q, k, v, pos, bias, gamma, 1.0, cu, Hq, Hkv, split=False)
+    assert (o.double() - o2.double()).abs().max() <= 2 ** -7
+    assert (lse - lse2).abs().max() <= 1e-4
+
+
 def test_attention_n128k_kept_13107_sampled_rows(tg):
     q, k, v, pos, bias, gamma, cu = _attn_inputs([13107], 16, 8, seed=13107, pos_spread=10)
     o, lse = _run_attention(tg, q, k, v, pos, bias, gamma, 1.0, cu, 16, 8)
