@@ -140,6 +140,7 @@ def stage_work(wl, kept_counts, ffn=0):
         "seq_rmsnorm": {"bound": "hbm", "bytes": T * 13},
         "topk_compact": {"bound": "hbm", "bytes": T * 5 + K * 12},
         "gather": {"bound": "hbm", "bytes": 2 * K * H * 2 + K * 4},
+        "rope_rows": {"bound": "hbm", "bytes": 2 * K * d * 4 + K * 4},
         "qkv_rope_cache": {"bound": "tensor", "flops": 2 * K * H * nqkv,
                            "bytes": K * H * 2 + nqkv * H * 2 + K * nqkv * 2 + K * 4
                            + K * (H // 128) * 4},

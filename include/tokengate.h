@@ -134,6 +134,24 @@ int tg_rope_table(float* cos_sin, int max_pos, int head_dim, double theta,
                   tg_stream_t stream);
 
 /*
+ * Per-row rotary table (same source: every kept row rotates by its original position).
+ * Copies each row's row of the tg_rope_table table, transposed in 16-byte blocks so that
+ * block j of consecutive rows is contiguous:
+ *   rot[(j * ld_rot + r) * 4 + e] = cos_sin[pos[r] * head_dim + 4 j + e],  e < 4,
+ * for r < n_rows, j < head_dim / 4 (block j holds cos, sin of rotation pairs 2j, 2j + 1).
+ * Passed to the QKV entry points with pos = NULL (cos_sin = rot, max_pos = ld_rot), it
+ * gives the same results as (pos, cos_sin) with contiguous table reads in the GEMM
+ * epilogue; the kept positions are the same in every gated layer, so one call per step
+ * serves all of them.  pos: int32 [n_rows] (values < max_pos, else TG_STATUS_BOUNDS and
+ * the row takes position 0); cos_sin: float32 [max_pos, head_dim] (16-byte aligned);
+ * rot: float32 [head_dim / 4, ld_rot, 4] (16-byte aligned), ld_rot >= n_rows; head_dim a
+ * multiple of 4 (>= 8).  status may be NULL.  Not a step of the method: a layout change.
+ */
+int tg_rope_rows(const int32_t* pos, int64_t n_rows, const float* cos_sin, int max_pos,
+                 int head_dim, float* rot, int64_t ld_rot, uint32_t* status,
+                 tg_stream_t stream);
+
+/*
  * Host-only planning of the kept counts from per-request budgets (no GPU work).
  * ([farwalk] How do you deploy TokenGate?: generation takes a budget of kept prefill
  *  tokens; [farwalk] How does TokenGate learned token pruning work?: the question is
@@ -469,7 +487,9 @@ size_t tg_gemm_workspace_size(void);
  * followed by tg_gather_rope (rope mode) and tg_kv_compact, in one kernel.
  * x: bf16 [M, hidden] (ld_x); w_qkv: bf16 [(n_q_heads + 2 n_kv_heads) * head_dim, hidden]
  * (rows: Wq, Wk, Wv); pos: int32 [M] (values < max_pos, else TG_STATUS_BOUNDS and the
- * row uses position 0); q_out: bf16 [M, n_q_heads * head_dim] (ld_q); cache_k/cache_v:
+ * row uses position 0), or NULL: then cos_sin is the per-row table of tg_rope_rows for
+ * these M rows and max_pos its row stride ld_rot (>= M, else TG_ERR_INVALID_ARGUMENT);
+ * q_out: bf16 [M, n_q_heads * head_dim] (ld_q); cache_k/cache_v:
  * bf16 rows of n_kv_heads * head_dim (ld_cache).  head_dim = 128, hidden multiple of 64.
  * row_ssq_in (may be NULL): float32 [M, hidden/128] (row stride ld_ssq_in) holding the
  * sums of squares of x per 128 columns (from tg_gather_rope or tg_linear row_ssq_out);

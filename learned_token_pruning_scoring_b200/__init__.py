@@ -23,7 +23,7 @@ from . import _lib
 
 __all__ = [
     "TokenGateError", "lib", "tg_version", "tg_device_supported", "tg_plan_kept",
-    "tg_rope_table", "tg_gate_score_workspace_size", "tg_gate_score", "tg_topk_compact",
+    "tg_rope_table", "tg_rope_rows", "tg_gate_score_workspace_size", "tg_gate_score", "tg_topk_compact",
     "tg_gate_score_noalloc", "tg_seq_rmsnorm", "tg_gather_rope", "tg_kv_compact", "tg_gated_attention", "tg_linear",
     "tg_status_clear", "tg_status_read", "tg_set_launch_overlap", "tg_get_launch_overlap",
     "tg_set_gather_tma", "tg_get_gather_tma", "tg_set_scorer_pair", "tg_get_scorer_pair",
@@ -164,6 +164,24 @@ def tg_rope_table(max_pos: int, head_dim: int, theta: float, out=None, device=No
            "tg_rope_table")
     _count()
     return out
+
+
+def tg_rope_rows(pos, cos_sin, out=None, status=None, stream=None) -> torch.Tensor:
+    """Per-row rotary table [head_dim/4, ld_rot, 4] of the rows' positions (cos_sin from
+    tg_rope_table); pass it as cos_sin with pos=None to the QKV entry points."""
+    n = pos.numel()
+    head_dim = cos_sin.shape[1] * cos_sin.shape[2] if cos_sin.dim() == 3 else cos_sin.shape[1]
+    if out is None:
+        out = torch.empty((head_dim // 4, max(n, 1), 4), dtype=torch.float32, device=pos.device)
+    _check(lib.tg_rope_rows(_ptr(pos), n, _ptr(cos_sin), cos_sin.shape[0], head_dim, _ptr(out),
+                            out.shape[1], _ptr(status), _stream(stream)), "tg_rope_rows")
+    _count()
+    return out
+
+
+def _rope_rows_arg(pos, cos_sin):
+    """max_pos argument of the QKV entry points: table rows, or the per-row table's stride."""
+    return cos_sin.shape[0] if pos is not None else cos_sin.shape[1]
 
 
 def tg_gate_score_workspace_size(total_tokens: int, hidden: int, width: int, batch: int) -> int:
@@ -426,7 +444,8 @@ def tg_linear(a, w, c=None, rmsnorm=False, eps=1e-6, residual=None, row_ssq=None
 def tg_qkv_rope_cache(x, w_qkv, pos, cos_sin, cache_k, cache_v, n_q_heads, n_kv_heads,
                       q_out=None, head_dim=128, eps=1e-6, slot_offset=0, row_ssq=None,
                       status=None, stream=None, q_norm_w=None, k_norm_w=None, workspace=None):
-    """Fused QKV projection (RMSNorm folded) + RoPE at `pos` + compacted KV-cache write;
+    """Fused QKV projection (RMSNorm folded) + RoPE at `pos` + compacted KV-cache write
+    (pos=None: cos_sin is the per-row table of tg_rope_rows);
     with q_norm_w / k_norm_w (float32 [head_dim]) also QK-norm before RoPE
     (tg_qkv_qknorm_rope_cache)."""
     ld_x, ld_w = _mat(x, "x"), _mat(w_qkv, "w_qkv")
@@ -443,7 +462,8 @@ def tg_qkv_rope_cache(x, w_qkv, pos, cos_sin, cache_k, cache_v, n_q_heads, n_kv_
         rc = lib.tg_qkv_qknorm_rope_cache(_ptr(x), ld_x, _ptr(w_qkv), ld_w, M, hidden, n_q_heads,
                                           n_kv_heads, head_dim, float(eps), _ptr(q_norm_w),
                                           _ptr(k_norm_w), _ptr(pos), _ptr(cos_sin),
-                                          cos_sin.shape[0], _ptr(q_out), ld_q, _ptr(cache_k),
+                                          _rope_rows_arg(pos, cos_sin), _ptr(q_out), ld_q,
+                                          _ptr(cache_k),
                                           _ptr(cache_v), ld_c, int(slot_offset), _ptr(row_ssq),
                                           ld_ssq, ws_ptr, ws_bytes, _ptr(status),
                                           _stream(stream))
@@ -451,7 +471,8 @@ def tg_qkv_rope_cache(x, w_qkv, pos, cos_sin, cache_k, cache_v, n_q_heads, n_kv_
     else:
         rc = lib.tg_qkv_rope_cache(_ptr(x), ld_x, _ptr(w_qkv), ld_w, M, hidden, n_q_heads,
                                    n_kv_heads, head_dim, float(eps), _ptr(pos), _ptr(cos_sin),
-                                   cos_sin.shape[0], _ptr(q_out), ld_q, _ptr(cache_k),
+                                   _rope_rows_arg(pos, cos_sin), _ptr(q_out), ld_q,
+                                   _ptr(cache_k),
                                    _ptr(cache_v), ld_c, int(slot_offset), _ptr(row_ssq), ld_ssq,
                                    ws_ptr, ws_bytes, _ptr(status), _stream(stream))
         _check(rc, "tg_qkv_rope_cache")
@@ -520,7 +541,8 @@ def tg_out_proj_qkv_next(o, w_o, x, row_ssq, w_qkv, pos, cos_sin, cache_k, cache
     rc = lib.tg_out_proj_qkv_next(_ptr(o), ld_o, _ptr(w_o), ld_wo, _ptr(x), ld_x, _ptr(row_ssq),
                                   ld_ssq, M, hidden, o.shape[1], _ptr(w_qkv), ld_wqkv, n_q_heads,
                                   n_kv_heads, head_dim, float(eps), _ptr(pos), _ptr(cos_sin),
-                                  cos_sin.shape[0], _ptr(q_out), ld_q, _ptr(cache_k),
+                                  _rope_rows_arg(pos, cos_sin), _ptr(q_out), ld_q,
+                                  _ptr(cache_k),
                                   _ptr(cache_v), ld_c, int(slot_offset), _ptr(workspace),
                                   workspace.numel(), _ptr(status), _stream(stream))
     _check(rc, "tg_out_proj_qkv_next")
@@ -734,6 +756,11 @@ class GatedPrefill:
         # measured slower at the 16k kept count (QKV 45 -> 53 us, output projection 29 ->
         # 39 us), so off by default
         self.split_gemm = False
+        # optional: RoPE in the QKV epilogue from a per-row table built once per step
+        # (tg_rope_rows), whose blocks are contiguous across a warp's rows.  Same bits and,
+        # measured at 16k and 128k, the same time as the position table (the epilogue
+        # waits on the loads' latency, not on their cache lines): off by default
+        self.rope_rows = False
         self._qkv_done = -1  # index of the layer whose QKV already ran in a fused launch
 
     def _mark(self, name):
@@ -765,6 +792,7 @@ class GatedPrefill:
             kept_idx=torch.empty(K, dtype=torch.int32, device=dev),
             kept_pos=torch.empty(K, dtype=torch.int32, device=dev),
             kept_bias=torch.empty(K, **f32),
+            rot=torch.empty((self.d // 4, max(K, 1), 4), **f32),
             x=torch.empty((K, self.hidden), **bf),
             ssq=torch.empty((K, self.hidden // 128), **f32),
             qkv=torch.empty((K, nqkv), **bf),
@@ -810,6 +838,15 @@ class GatedPrefill:
             tg_gather_rope(h, P["x"], row_idx=P["kept_idx"], row_ssq=P["ssq"], status=self.status,
                            stream=stream)
             self._mark("gather")
+            if self.rope_rows:
+                tg_rope_rows(P["kept_pos"], self.cos_sin, out=P["rot"], status=self.status,
+                             stream=stream)
+                self._mark("rope_rows")
+
+    def _rope(self):
+        """(pos, table) arguments of the QKV entry points for the kept rows."""
+        P = self.planned
+        return (None, P["rot"]) if self.rope_rows else (P["kept_pos"], self.cos_sin)
 
     def _fusable(self):
         nq, nkv = self.hq * self.d, self.hkv * self.d
@@ -831,7 +868,8 @@ class GatedPrefill:
         if self._qkv_done == i:
             pass  # ran with the previous layer's output projection
         elif self.fused_qkv or L.q_norm is not None:
-            tg_qkv_rope_cache(x, L.Wqkv, P["kept_pos"], self.cos_sin, ck, cv, self.hq, self.hkv,
+            rpos, rtab = self._rope()
+            tg_qkv_rope_cache(x, L.Wqkv, rpos, rtab, ck, cv, self.hq, self.hkv,
                               q_out=qkv[:, :nq], head_dim=self.d, eps=self.norm_eps,
                               row_ssq=P["ssq"], status=self.status, stream=stream,
                               q_norm_w=L.q_norm, k_norm_w=L.k_norm, workspace=P["gemm_ws"])
@@ -863,7 +901,8 @@ class GatedPrefill:
         if fuse_next and i + 1 < len(self.layers) and self._fusable():
             Ln = self.layers[i + 1]
             ckn, cvn = P["caches"][i + 1]
-            tg_out_proj_qkv_next(o, L.Wo, x, P["ssq"], Ln.Wqkv, P["kept_pos"], self.cos_sin, ckn,
+            rpos, rtab = self._rope()
+            tg_out_proj_qkv_next(o, L.Wo, x, P["ssq"], Ln.Wqkv, rpos, rtab, ckn,
                                  cvn, self.hq, self.hkv, qkv[:, :nq], P["chain_ws"],
                                  head_dim=self.d, eps=self.norm_eps, status=self.status,
                                  stream=stream)

@@ -33,6 +33,7 @@ SIGNATURES = {
     "tg_get_scorer_pair": (_i32, []),
     "tg_prefetch_l2": (_i32, [_p, _sz, _p]),
     "tg_rope_table": (_i32, [_p, _i32, _i32, _f64, _p]),
+    "tg_rope_rows": (_i32, [_p, _i64, _p, _i32, _i32, _p, _i64, _p, _p]),
     "tg_plan_kept": (_i32, [_p, _p, _p, _i32, _p]),
     "tg_gate_score_workspace_size": (_sz, [_i64, _i32, _i32, _i32]),
     "tg_gate_score": (_i32, [_p, _i64, _i64, _i32, _p, _p, _i32, _p, _f32, _p, _p, _i32, _f32,

@@ -37,6 +37,28 @@ __global__ void rope_table_kernel(float2* __restrict__ table, int max_pos, int h
   }
 }
 
+// Per-row rotation table: the (cos, sin) row of each row's position, transposed so that
+// block j (rotation pairs 2j, 2j + 1) of consecutive rows is contiguous:
+// rot[j * ld_rot + r] = table[pos[r]][j] (float4).  One thread per (j, r), r fastest:
+// the stores are coalesced, the table reads are gathers (once per step, not per layer).
+__global__ void rope_rows_kernel(const int32_t* __restrict__ pos, int64_t n_rows,
+                                 const float4* __restrict__ table, int max_pos, int blocks,
+                                 float4* __restrict__ rot, int64_t ld_rot, uint32_t* status) {
+  griddep_wait();
+  const int64_t n = n_rows * blocks;
+  for (int64_t t = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; t < n;
+       t += (int64_t)gridDim.x * blockDim.x) {
+    const int j = (int)(t / n_rows);
+    const int64_t r = t % n_rows;
+    int p = pos[r];
+    if (p < 0 || p >= max_pos) {
+      if (status) atomicOr(status, TG_STATUS_BOUNDS);
+      p = 0;
+    }
+    rot[(int64_t)j * ld_rot + r] = table[(int64_t)p * blocks + j];
+  }
+}
+
 // Plain row copy of `nvec` 16-byte vectors (lane-strided), all loads before stores.
 __device__ __forceinline__ void copy_row(const uint4* __restrict__ s, uint4* __restrict__ d,
                                          int vbegin, int vend, int lane) {
@@ -442,6 +464,24 @@ extern "C" int tg_rope_table(float* cos_sin, int max_pos, int head_dim, double t
   if (grid > sm_count() * 16) grid = sm_count() * 16;
   return launch(rope_table_kernel, dim3(grid), dim3(256), 0, (cudaStream_t)stream,
                 reinterpret_cast<float2*>(cos_sin), max_pos, half, theta, head_dim);
+}
+
+extern "C" int tg_rope_rows(const int32_t* pos, int64_t n_rows, const float* cos_sin,
+                            int max_pos, int head_dim, float* rot, int64_t ld_rot,
+                            uint32_t* status, tg_stream_t stream) {
+  if (n_rows < 0 || max_pos <= 0 || ld_rot < n_rows) return TG_ERR_INVALID_ARGUMENT;
+  if (head_dim < 8 || (head_dim & 3)) return TG_ERR_UNSUPPORTED_SHAPE;
+  if (n_rows == 0) return TG_OK;
+  if (!pos || !cos_sin || !rot) return TG_ERR_INVALID_ARGUMENT;
+  if (!aligned16(cos_sin) || !aligned16(rot)) return TG_ERR_MISALIGNED;
+  TG_TRY(check_device());
+  const int blocks = head_dim / 4;
+  const int64_t n = n_rows * blocks;
+  int grid = (int)((n + 255) / 256);
+  if (grid > sm_count() * 16) grid = sm_count() * 16;
+  return launch(rope_rows_kernel, dim3(grid), dim3(256), 0, (cudaStream_t)stream, pos, n_rows,
+                reinterpret_cast<const float4*>(cos_sin), max_pos, blocks,
+                reinterpret_cast<float4*>(rot), ld_rot, status);
 }
 
 extern "C" int tg_gather_rope(const tg_bf16* src, int64_t ld_src, int64_t src_rows,

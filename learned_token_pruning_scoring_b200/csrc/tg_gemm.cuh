@@ -54,9 +54,9 @@ struct GemmParams {
   float* s_out;
   float* partial;  // [ceil(M / 32)]
   // EpiQKV
-  const int32_t* pos;     // [M] rotary position of each row
-  const float* cos_sin;   // [max_pos, head_dim / 2, 2]
-  int max_pos;
+  const int32_t* pos;     // [M] rotary position of each row, or null (see rope_row)
+  const float* cos_sin;   // [max_pos, head_dim / 2, 2], or the per-row table if pos is null
+  int max_pos;            // table rows, or the per-row table's row stride
   int q_cols, k_cols;     // Q heads in [0, q_cols), K heads in [q_cols, q_cols + k_cols)
   uint16_t* k_out;        // K rows: k_out + row * ld_kv (columns relative to q_cols)
   uint16_t* v_out;        // V rows: v_out + row * ld_kv (columns relative to q_cols + k_cols)
@@ -90,6 +90,20 @@ __device__ __forceinline__ float rscale_from_ssq(const GemmParams& p, int64_t gr
   return rsqrtf(t / (float)p.K + p.eps);
 }
 
+// (cos, sin) of rotation pairs 2j and 2j + 1 of one row is base[j * stride]: from the
+// position table at the row's position (pos given), or, with pos == nullptr, from the
+// per-row table of tg_rope_rows (block j of consecutive rows contiguous, row stride
+// max_pos), where a warp's loads of one block are contiguous.
+struct RopeRow {
+  const float4* base;
+  int64_t stride;
+};
+__device__ __forceinline__ RopeRow rope_row(const GemmParams& p, int64_t grow, int pos) {
+  const float4* t = reinterpret_cast<const float4*>(p.cos_sin);
+  if (p.pos) return {t + (int64_t)pos * 32, 1};
+  return {t + (grow < p.M ? grow : 0), (int64_t)p.max_pos};
+}
+
 // Epilogue of one output row held by this thread: BN accumulator columns at TMEM
 // address `tbase` (the warp's lane quarter), output columns n0 .. n0 + BN.  All lanes
 // of the warp must call it (tcgen05.ld is warp-collective).  Returns the row's score
@@ -114,12 +128,12 @@ __device__ __forceinline__ float epilogue_row(const GemmParams& p, uint32_t tbas
       dcol = n0 - p.q_cols - p.k_cols;
     }
     const bool rope = n0 < p.q_cols + p.k_cols;
-    int pos = (rope && live) ? p.pos[grow] : 0;
-    if (pos < 0 || pos >= p.max_pos) {
+    int pos = (rope && live && p.pos) ? p.pos[grow] : 0;
+    if (p.pos && (pos < 0 || pos >= p.max_pos)) {
       if (live && p.status) atomicOr(p.status, TG_STATUS_BOUNDS);
       pos = 0;
     }
-    const float4* cs_row = reinterpret_cast<const float4*>(p.cos_sin + (int64_t)pos * 128);
+    const RopeRow rr = rope_row(p, grow, pos);
 #pragma unroll 1
     for (int pr = 0; pr < BN / 64; ++pr) {
       // chunk pairs (0,2), (1,3), (4,6), (5,7): columns i and i + 64 of one head
@@ -131,7 +145,7 @@ __device__ __forceinline__ float epilogue_row(const GemmParams& p, uint32_t tbas
       if (live) {
         uint4* da = reinterpret_cast<uint4*>(dst + dcol + ca * 32);
         uint4* db = reinterpret_cast<uint4*>(dst + dcol + cb * 32);
-        const float4* cs = cs_row + (ca & 3) * 16;  // (cos, sin) pairs of i = (ca&3)*32 ..
+        const float4* cs = rr.base + (ca & 3) * 16 * rr.stride;  // pairs i = (ca&3)*32 ..
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
           uint32_t wa[4], wb[4];
@@ -141,7 +155,7 @@ __device__ __forceinline__ float epilogue_row(const GemmParams& p, uint32_t tbas
             float x1a = __uint_as_float(ra[i]) * rscale, x1b = __uint_as_float(ra[i + 1]) * rscale;
             float x2a = __uint_as_float(rb[i]) * rscale, x2b = __uint_as_float(rb[i + 1]) * rscale;
             if (rope) {
-              const float4 t = cs[i >> 1];  // (cos_i, sin_i, cos_i+1, sin_i+1)
+              const float4 t = cs[(i >> 1) * rr.stride];  // (cos_i, sin_i, cos_i+1, sin_i+1)
               const float y1a = x1a * t.x - x2a * t.y, y2a = x2a * t.x + x1a * t.y;
               const float y1b = x1b * t.z - x2b * t.w, y2b = x2b * t.z + x1b * t.w;
               x1a = y1a;
@@ -426,6 +440,7 @@ template <int EPI>
 __device__ __forceinline__ int pair_row_pos(const GemmParams& p, int64_t grow, int n0) {
   if (EPI != EpiQKV && EPI != EpiQKVNorm) return 0;
   const bool live = grow < p.M;
+  if (!p.pos) return 0;  // per-row table: no position lookup
   int pos = (live && n0 < p.q_cols + p.k_cols) ? p.pos[grow] : 0;
   if (pos < 0 || pos >= p.max_pos) {
     if (live && p.status) atomicOr(p.status, TG_STATUS_BOUNDS);
@@ -469,7 +484,7 @@ __device__ __forceinline__ void pair_epilogue_half(const GemmParams& p, unsigned
       qk = rsqrtf(ss * rscale * rscale * (1.0f / 128.0f) + p.qk_eps);
     }
     const float scale = rscale * qk;
-    const float4* cs_row = reinterpret_cast<const float4*>(p.cos_sin + (int64_t)pos * 128);
+    const RopeRow rr = rope_row(p, grow, pos);
 #pragma unroll 1
     for (int pr = 0; pr < 2; ++pr) {
       // 32-column pieces ca and ca + 2 hold columns i and i + 64 of one 128-column head
@@ -482,7 +497,7 @@ __device__ __forceinline__ void pair_epilogue_half(const GemmParams& p, unsigned
       add_partials(rb, pr + 2, adds, n_add);
       unsigned char* box_a = out_s + (ca >> 1) * PairCfg<1>::BOX_BYTES;
       unsigned char* box_b = out_s + (cb >> 1) * PairCfg<1>::BOX_BYTES;
-      const float4* cs = cs_row + (ca & 3) * 16;  // (cos, sin) pairs of i = (ca & 3) * 32 ..
+      const float4* cs = rr.base + (ca & 3) * 16 * rr.stride;  // pairs i = (ca & 3) * 32 ..
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
         uint32_t wa[4], wb[4];
@@ -499,7 +514,7 @@ __device__ __forceinline__ void pair_epilogue_half(const GemmParams& p, unsigned
             x2b *= __ldg(nw + c + 65);
           }
           if (rope) {
-            const float4 t = cs[i >> 1];  // (cos_i, sin_i, cos_i+1, sin_i+1)
+            const float4 t = cs[(i >> 1) * rr.stride];  // (cos_i, sin_i, cos_i+1, sin_i+1)
             const float y1a = x1a * t.x - x2a * t.y, y2a = x2a * t.x + x1a * t.y;
             const float y1b = x1b * t.z - x2b * t.w, y2b = x2b * t.z + x1b * t.w;
             x1a = y1a;

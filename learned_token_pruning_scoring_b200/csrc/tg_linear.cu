@@ -363,10 +363,11 @@ static int qkv_rope_cache_impl(const tg_bf16* x, int64_t ld_x, const tg_bf16* w_
   if (head_dim != 128 || n_q_heads <= 0 || n_kv_heads <= 0 || hidden <= 0 || (hidden % 64))
     return TG_ERR_UNSUPPORTED_SHAPE;
   if (M < 0 || slot_offset < 0 || max_pos <= 0) return TG_ERR_INVALID_ARGUMENT;
+  if (!pos && max_pos < M) return TG_ERR_INVALID_ARGUMENT;  // per-row table: row stride
   if (M == 0) return TG_OK;
   const int q_cols = n_q_heads * head_dim, kv_cols = n_kv_heads * head_dim;
   const int N = q_cols + 2 * kv_cols;
-  if (!x || !w_qkv || !pos || !cos_sin || !q_out || !cache_k || !cache_v)
+  if (!x || !w_qkv || !cos_sin || !q_out || !cache_k || !cache_v)
     return TG_ERR_INVALID_ARGUMENT;
   if (ld_x < hidden || ld_w < hidden || ld_q < q_cols || ld_cache < kv_cols)
     return TG_ERR_INVALID_ARGUMENT;
@@ -517,8 +518,9 @@ extern "C" int tg_out_proj_qkv_next(
   const int q_cols = n_q_heads * head_dim, kv_cols = n_kv_heads * head_dim;
   if ((q_cols % 256) || (kv_cols % 256)) return TG_ERR_UNSUPPORTED_SHAPE;
   if (M < 0 || slot_offset < 0 || max_pos <= 0 || !(eps >= 0.f)) return TG_ERR_INVALID_ARGUMENT;
+  if (!pos && max_pos < M) return TG_ERR_INVALID_ARGUMENT;  // per-row table: row stride
   if (M == 0) return TG_OK;
-  if (!o || !w_o || !x || !row_ssq || !w_qkv || !pos || !cos_sin || !q_out || !cache_k ||
+  if (!o || !w_o || !x || !row_ssq || !w_qkv || !cos_sin || !q_out || !cache_k ||
       !cache_v)
     return TG_ERR_INVALID_ARGUMENT;
   if (ld_o < o_cols || ld_wo < o_cols || ld_x < hidden || ld_ssq < hidden / 128 ||

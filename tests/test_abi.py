@@ -227,3 +227,15 @@ def test_attention_split_plan(lib):
     # one head group: most tiles split, the longest into six parts
     n = items([2000], 2, 1)
     assert chunk_of([2000], n) == [3]
+
+
+def test_rope_rows_argument_checks(lib):
+    p = C.c_void_p(0x10000)
+    # per-row table: row stride below the row count; head_dim not a multiple of 4
+    assert lib.tg_rope_rows(p, 10, p, 100, 128, p, 9, None, None) == -1
+    assert lib.tg_rope_rows(p, 10, p, 100, 126, p, 10, None, None) == -6
+    assert lib.tg_rope_rows(p, 10, C.c_void_p(0x10004), 100, 128, p, 10, None, None) == -2
+    assert lib.tg_rope_rows(p, 0, p, 100, 128, p, 0, None, None) == 0
+    # QKV with pos = NULL reads a per-row table whose row stride (max_pos) must cover M
+    assert lib.tg_qkv_rope_cache(p, 2048, p, 2048, 300, 2048, 16, 8, 128, 1e-6, None, p, 299,
+                                 p, 2048, p, p, 1024, 0, p, 16, None, 0, None, None) == -1

@@ -1005,3 +1005,66 @@ def test_gate_score_backward_without_norm_weight(tg):
         want = ref[name]
         err = np.abs(got.cpu().double().numpy() - want)
         assert err.max() <= 1e-2 * np.abs(want).max(), (name, err.max())
+
+
+def test_rope_rows_copies_the_position_rows(tg):
+    """tg_rope_rows is a transposed gather of tg_rope_table rows: bit-exact, and a
+    position outside the table raises TG_STATUS_BOUNDS and takes row 0."""
+    d, n = 128, 1000
+    g = torch.Generator().manual_seed(5)
+    pos = torch.sort(torch.randperm(8000, generator=g)[:n])[0].to(torch.int32)
+    cs = tg.tg_rope_table(8000, d, 1.0e6)
+    st = _status()
+    rot = tg.tg_rope_rows(_dev(pos), cs, status=st)
+    assert tg.tg_status_read(st) == 0
+    want = cs.view(8000, d // 4, 4)[pos.long().cuda()].permute(1, 0, 2)
+    assert torch.equal(rot, want)
+    bad = pos.clone()
+    bad[7] = 8000
+    st = _status()
+    rot = tg.tg_rope_rows(_dev(bad), cs, status=st)
+    assert tg.tg_status_read(st) & 4  # TG_STATUS_BOUNDS
+    assert torch.equal(rot[:, 7], cs.view(8000, d // 4, 4)[0])
+
+
+@pytest.mark.parametrize("M", [1, 300, 1638])
+def test_qkv_per_row_table_matches_positions(tg, M):
+    """pos = NULL with the per-row table gives the same bits as (pos, table) on the
+    CTA-pair kernel (row sums given), the one-CTA kernel (none), QK-norm, and the fused
+    output projection + next QKV."""
+    Hq, Hkv, d, H = 16, 8, 128, 2048
+    x = _dev(S.uniform_rows(M, H, seed=M + 90))
+    w = _dev(S.uniform_rows((Hq + 2 * Hkv) * d, H, seed=M + 91, scale=0.02))
+    g = torch.Generator().manual_seed(M + 92)
+    pos = _dev(torch.sort(torch.randperm(10 * M + 1, generator=g)[:M])[0].to(torch.int32))
+    cs = tg.tg_rope_table(10 * M + 1, d, 1.0e6)
+    rot = tg.tg_rope_rows(pos, cs)
+    ssq = _dev(_ssq_rows(x.cpu(), H))
+    qn = _dev((0.8 + 0.4 * torch.rand(d, generator=g)).float())
+    kn = _dev((0.8 + 0.4 * torch.rand(d, generator=g)).float())
+
+    def run(p, table, **kw):
+        ck = torch.zeros((M, Hkv * d), dtype=torch.bfloat16, device="cuda")
+        cv = torch.zeros_like(ck)
+        st = _status()
+        q = tg.tg_qkv_rope_cache(x, w, p, table, ck, cv, Hq, Hkv, status=st, **kw)
+        assert tg.tg_status_read(st) == 0
+        return q, ck, cv
+
+    for kw in ({"row_ssq": ssq}, {}, {"row_ssq": ssq, "q_norm_w": qn, "k_norm_w": kn}):
+        for a, b in zip(run(pos, cs, **kw), run(None, rot, **kw)):
+            assert torch.equal(a, b)
+    o = _dev(S.uniform_rows(M, Hq * d, seed=M + 93))
+    wo = _dev(S.uniform_rows(H, Hq * d, seed=M + 94, scale=0.02))
+    outs = []
+    for p, table in ((pos, cs), (None, rot)):
+        xx, ss = x.clone(), torch.empty((M, H // 128), device="cuda")
+        ck = torch.zeros((M, Hkv * d), dtype=torch.bfloat16, device="cuda")
+        cv = torch.zeros_like(ck)
+        q = torch.empty((M, Hq * d), dtype=torch.bfloat16, device="cuda")
+        ws = torch.zeros(max(16, tg.tg_out_proj_qkv_workspace_size(M)), dtype=torch.uint8,
+                         device="cuda")
+        tg.tg_out_proj_qkv_next(o, wo, xx, ss, w, p, table, ck, cv, Hq, Hkv, q, ws)
+        outs.append((xx, q, ck, cv))
+    for a, b in zip(*outs):
+        assert torch.equal(a, b)
