@@ -75,6 +75,9 @@ def parse_args():
     ap.add_argument("--also", default="n128k",
                     help="comma-separated workloads measured after the main one and "
                          "reported as sub-records of the same line ('' for none)")
+    ap.add_argument("--rope-rows", choices=("on", "off"), default=None,
+                    help="QKV RoPE from the per-row table of tg_rope_rows (default: the "
+                         "library's choice)")
     ap.add_argument("--dense-steps", type=int, default=3,
                     help="timed steps of the full-context reference (0 skips it)")
     return ap.parse_args()
@@ -341,6 +344,8 @@ def measure(args, wl_name, rank, world, extras):
                                      device=dev)
     pipe = tg.GatedPrefill(gate, layers, wl.n_q_heads, wl.n_kv_heads, wl.head_dim,
                            wl.rope_theta, device=dev, lower=lower)
+    if args.rope_rows is not None:
+        pipe.rope_rows = args.rope_rows == "on"
     P = pipe.plan(wl.lengths, wl.questions, wl.budgets)
     h_dev = h.to(dev)
     pr_dev = pr.to(dev)

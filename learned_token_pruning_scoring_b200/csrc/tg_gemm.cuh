@@ -399,7 +399,12 @@ struct PairCfg {
   static constexpr int OUT_BYTES = 4 * BOX_BYTES;      // staging of one 128 x 256 output tile
   static constexpr int BAR_BYTES = 256;
   static constexpr int SMEM = 1024 + TILE_BYTES + OUT_BYTES + BAR_BYTES;
-  static constexpr int THREADS = 320;
+  static constexpr int THREADS = 384;                  // three warpgroups
+  // Registers per thread after setmaxnreg: warpgroup 0 (producer, MMA issuer and two
+  // idle warps) gives up what the epilogue warpgroups take.  The split needs a launch
+  // allocation of at least (128 * LOW + 256 * HIGH) / 384 = 160 registers per thread.
+  static constexpr int REGS_LOW = 80, REGS_HIGH = 200;
+  static constexpr int REGS_LAUNCH_MIN = (128 * REGS_LOW + 256 * REGS_HIGH) / 384;
   static constexpr int TMEM_COLS = 2 * BN;             // two accumulators (double buffer)
 };
 
@@ -449,6 +454,20 @@ __device__ __forceinline__ int pair_row_pos(const GemmParams& p, int64_t grow, i
   return pos;
 }
 
+// The 16 (cos, sin) blocks (32 rotation pairs) of one half of a RoPE head, from block j0.
+__device__ __forceinline__ void pair_rope_load(const RopeRow& rr, int j0, float4 (&rt)[16]) {
+#pragma unroll
+  for (int j = 0; j < 16; ++j) rt[j] = rr.base[(int64_t)(j0 + j) * rr.stride];
+}
+// Before the accumulator wait: the first half's blocks of a RoPE tile (Q or K columns of
+// the QKV epilogues), whose latency then hides under the tile's MMAs.
+template <int EPI>
+__device__ __forceinline__ void pair_rope_prefetch(const GemmParams& p, int64_t grow, int n0,
+                                                   int pos, float4 (&rt)[16]) {
+  if ((EPI == EpiQKV || EPI == EpiQKVNorm) && n0 < p.q_cols + p.k_cols)
+    pair_rope_load(rope_row(p, grow, pos), 0, rt);
+}
+
 // Columns [128 h, 128 h + 128) of one 256 x 256 output tile of the pair (each CTA: 128
 // rows, staged in shared memory as four swizzled 64-column boxes); `row` is the thread's
 // row in the CTA's half, `tacc` the TMEM address of the row's accumulator (lane quarter
@@ -457,6 +476,7 @@ template <int EPI, int MAXADD>
 __device__ __forceinline__ void pair_epilogue_half(const GemmParams& p, unsigned char* out_s,
                                                    uint32_t tacc, int row, int64_t grow, int n0,
                                                    int h, bool has_res, float rscale, int pos,
+                                                   float4 (&rt)[16],
                                                    const float4* const (&adds)[MAXADD],
                                                    int n_add) {
   const bool live = grow < p.M;
@@ -489,6 +509,10 @@ __device__ __forceinline__ void pair_epilogue_half(const GemmParams& p, unsigned
     for (int pr = 0; pr < 2; ++pr) {
       // 32-column pieces ca and ca + 2 hold columns i and i + 64 of one 128-column head
       const int ca = 4 * h + pr, cb = ca + 2;
+      // (cos, sin) blocks of this half: the first half's were loaded while the tile's
+      // MMAs ran (pair_rope_prefetch); the second half's are requested here together,
+      // ahead of the TMEM loads
+      if (rope && pr == 1) pair_rope_load(rr, 16, rt);
       uint32_t ra[32], rb[32];
       tmem_ld32(tacc + ca * 32, ra);
       tmem_ld32(tacc + cb * 32, rb);
@@ -497,7 +521,6 @@ __device__ __forceinline__ void pair_epilogue_half(const GemmParams& p, unsigned
       add_partials(rb, pr + 2, adds, n_add);
       unsigned char* box_a = out_s + (ca >> 1) * PairCfg<1>::BOX_BYTES;
       unsigned char* box_b = out_s + (cb >> 1) * PairCfg<1>::BOX_BYTES;
-      const float4* cs = rr.base + (ca & 3) * 16 * rr.stride;  // pairs i = (ca & 3) * 32 ..
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
         uint32_t wa[4], wb[4];
@@ -514,7 +537,7 @@ __device__ __forceinline__ void pair_epilogue_half(const GemmParams& p, unsigned
             x2b *= __ldg(nw + c + 65);
           }
           if (rope) {
-            const float4 t = cs[(i >> 1) * rr.stride];  // (cos_i, sin_i, cos_i+1, sin_i+1)
+            const float4 t = rt[i >> 1];  // (cos_i, sin_i, cos_i+1, sin_i+1), i in the half
             const float y1a = x1a * t.x - x2a * t.y, y2a = x2a * t.x + x1a * t.y;
             const float y1b = x1b * t.z - x2b * t.w, y2b = x2b * t.z + x1b * t.w;
             x1a = y1a;
@@ -650,11 +673,13 @@ struct Piece {
   int kind;  // 0: whole tile, 1: finisher (first k-blocks), 2: contributor
 };
 
-// The pieces of cluster c in the order the cluster runs them: a tail range that starts
+// The pieces of cluster c in the order the cluster runs them (SPLIT = false: the plain
+// tile loop, everything below it compiled out): a tail range that starts
 // inside a tile begins with a contributing piece, which runs first (its partial sums are
 // then published before the cluster's first epilogue, and the finisher that waits for
 // them does not wait behind that epilogue); then the whole tiles; then the rest of the
 // range, whose last piece may be a finisher.
+template <bool SPLIT>
 struct PieceIter {
   int c, C, n_tiles, nk, dp_tiles;
   int64_t u, u1;
@@ -662,8 +687,8 @@ struct PieceIter {
   bool split, lead_done;
   __device__ PieceIter(int c_, int C_, int n_tiles_, int nk_, const PairSplit& sp)
       : c(c_), C(C_), n_tiles(n_tiles_), nk(nk_), dp_tiles(0), u(0), u1(0), i(0),
-        split(sp.part != nullptr), lead_done(false) {
-    if (split) {
+        split(SPLIT && sp.part != nullptr), lead_done(false) {
+    if (SPLIT && split) {
       dp_tiles = sp.dp_tiles;
       u = sp.tail_units * c / C;
       u1 = sp.tail_units * (c + 1) / C;
@@ -679,17 +704,17 @@ struct PieceIter {
     return true;
   }
   __device__ bool next(Piece& pc) {
-    if (split && !lead_done) {
+    if (SPLIT && split && !lead_done) {
       lead_done = true;
       if (u < u1 && u % nk != 0) return tail_piece(pc);
     }
     const int t = c + i * C;
-    if (!split ? t < n_tiles : t < dp_tiles) {
+    if (!(SPLIT && split) ? t < n_tiles : t < dp_tiles) {
       pc = {t, 0, nk, 0};
       ++i;
       return true;
     }
-    if (!split || u >= u1) return false;
+    if (!(SPLIT && split) || u >= u1) return false;
     return tail_piece(pc);
   }
 };
@@ -701,17 +726,19 @@ struct PieceIter {
 //   warp 0     one thread streams A and W k-blocks of every tile through the ring;
 //   warp 1     TMEM owner; in the even CTA one thread issues the M=256 MMAs into
 //              accumulator buffer (tile index & 1);
-//   warps 2-9  epilogue of the previous tile while the next one accumulates, as two
-//              independent groups of four warps (one per TMEM lane quarter), group g
-//              owning tile columns [128 g, 128 g + 128): TMEM -> registers -> bf16 in
-//              swizzled staging boxes -> TMA stores.  For EpiStore with a residual, the
-//              group's boxes are first filled with the residual rows by a TMA load
-//              issued one tile ahead.
+//   warps 2-3  idle (warpgroup 0 lowers its registers for the epilogue warpgroups);
+//   warps 4-11 epilogue of the previous tile while the next one accumulates, as two
+//              independent groups of four warps (one per TMEM lane quarter, one per
+//              warpgroup), group g owning tile columns [128 g, 128 g + 128): TMEM ->
+//              registers -> bf16 in swizzled staging boxes -> TMA stores.  For EpiStore
+//              with a residual, the group's boxes are first filled with the residual
+//              rows by a TMA load issued one tile ahead; a RoPE head's first (cos, sin)
+//              blocks are loaded before the accumulator wait.
 // Barriers: full/empty per ring stage (full lives in the even CTA and counts both CTAs'
 // bytes); acc_full[b] (the even CTA's commit, in both CTAs); acc_empty[b] (even CTA,
 // one arrive per epilogue group of each CTA once it has read buffer b); res_full[g].
-template <int STAGES, int EPI0, int EPI1>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(320, 1)
+template <int STAGES, int EPI0, int EPI1, bool SPLIT>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
     gemm_pair_kernel(const __grid_constant__ PairJob job0, const __grid_constant__ PairJob job1,
                      PairChain chain, PairSplit split) {
   using Cfg = PairCfg<STAGES>;
@@ -776,105 +803,108 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(320, 1)
   cluster_sync_all();  // barriers of both CTAs initialised before any remote arrive
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-
-  if (warp == 0) {
-    if (lane == 0) {
-      // The odd CTA's bytes may reach the even CTA's barrier before the even CTA's
-      // expect_tx: the phase cannot complete early, as it still waits for that arrive.
-      // A stage is reloaded only after the even CTA's commit freed it, which follows
-      // the completion of that barrier's previous phase.
-      const uint32_t full_lead0 = mapa_shared(smem_u32(&full[0]), 0);
-      griddep_wait();
-      int kg = 0;
-      bool ok = true;
-      PieceIter pit(cluster, n_clusters, n_tiles, job0.p.K / Cfg::BK, split);
-      Piece pc;
-      while (ok && pit.next(pc)) {
-        const int t = pc.t;
-        int job, rp, n0;
-        decode(t, job, rp, n0);
-        const PairJob& jb = job ? job1 : job0;
-        if (job && chain.ready) {
-          // job 0 must have finished every column of these rows
-          if (!wait_count_gpu(chain.ready + rp, chain.target, abort_flag, status)) break;
-          fence_proxy_async_global();  // the rows are read by TMA next
-          if (atomicAdd(chain.consumed + rp, 1) == 2 * tn1 - 1) {
-            chain.ready[rp] = 0;  // every producer of these rows has passed its wait
-            chain.consumed[rp] = 0;
+  if (warp < 4) {
+    regs_dec<Cfg::REGS_LOW>();  // warpgroup 0: producer, MMA issuer, two idle warps
+    if (warp == 0) {
+      if (lane == 0) {
+        // The odd CTA's bytes may reach the even CTA's barrier before the even CTA's
+        // expect_tx: the phase cannot complete early, as it still waits for that arrive.
+        // A stage is reloaded only after the even CTA's commit freed it, which follows
+        // the completion of that barrier's previous phase.
+        const uint32_t full_lead0 = mapa_shared(smem_u32(&full[0]), 0);
+        griddep_wait();
+        int kg = 0;
+        bool ok = true;
+        PieceIter<SPLIT> pit(cluster, n_clusters, n_tiles, job0.p.K / Cfg::BK, split);
+        Piece pc;
+        while (ok && pit.next(pc)) {
+          const int t = pc.t;
+          int job, rp, n0;
+          decode(t, job, rp, n0);
+          const PairJob& jb = job ? job1 : job0;
+          if (job && chain.ready) {
+            // job 0 must have finished every column of these rows
+            if (!wait_count_gpu(chain.ready + rp, chain.target, abort_flag, status)) break;
+            fence_proxy_async_global();  // the rows are read by TMA next
+            if (atomicAdd(chain.consumed + rp, 1) == 2 * tn1 - 1) {
+              chain.ready[rp] = 0;  // every producer of these rows has passed its wait
+              chain.consumed[rp] = 0;
+            }
+          }
+          const int64_t m0 = (int64_t)rp * 256 + rank * 128;
+          const int nb = n0 + (int)rank * (Cfg::BN / 2);
+          const int nk = jb.p.K / Cfg::BK;
+          const int kb_end = job ? nk : pc.kb1;
+          for (int kb = job ? 0 : pc.kb0; kb < kb_end; ++kb, ++kg) {
+            const int s = kg % STAGES;
+            const uint32_t ph = (uint32_t)(kg / STAGES) & 1u;
+            if (!mbar_wait(&empty[s], ph ^ 1u, abort_flag, status)) {
+              ok = false;
+              break;
+            }
+            unsigned char* a_s = tiles + s * Cfg::STAGE_BYTES;
+            if (rank == 0) mbar_arrive_expect_tx(&full[s], 2 * Cfg::STAGE_BYTES);
+            tma_load_2d_pair(a_s, &jb.maps.a, kb * Cfg::BK, (int32_t)m0, full_lead0 + s * 8);
+            tma_load_2d_pair(a_s + Cfg::A_BYTES, &jb.maps.b, kb * Cfg::BK, nb, full_lead0 + s * 8);
           }
         }
-        const int64_t m0 = (int64_t)rp * 256 + rank * 128;
-        const int nb = n0 + (int)rank * (Cfg::BN / 2);
-        const int nk = jb.p.K / Cfg::BK;
-        const int kb_end = job ? nk : pc.kb1;
-        for (int kb = job ? 0 : pc.kb0; kb < kb_end; ++kb, ++kg) {
-          const int s = kg % STAGES;
-          const uint32_t ph = (uint32_t)(kg / STAGES) & 1u;
-          if (!mbar_wait(&empty[s], ph ^ 1u, abort_flag, status)) {
-            ok = false;
-            break;
-          }
-          unsigned char* a_s = tiles + s * Cfg::STAGE_BYTES;
-          if (rank == 0) mbar_arrive_expect_tx(&full[s], 2 * Cfg::STAGE_BYTES);
-          tma_load_2d_pair(a_s, &jb.maps.a, kb * Cfg::BK, (int32_t)m0, full_lead0 + s * 8);
-          tma_load_2d_pair(a_s + Cfg::A_BYTES, &jb.maps.b, kb * Cfg::BK, nb, full_lead0 + s * 8);
-        }
+        // The even CTA waits until the last stages' bytes (both CTAs') have landed; the odd
+        // CTA is held by the closing cluster barrier until then.
+        if (rank == 0)
+          for (int g = kg - STAGES < 0 ? 0 : kg - STAGES; g < kg; ++g)
+            mbar_wait(&full[g % STAGES], (uint32_t)(g / STAGES) & 1u, nullptr, status);
       }
-      // The even CTA waits until the last stages' bytes (both CTAs') have landed; the odd
-      // CTA is held by the closing cluster barrier until then.
-      if (rank == 0)
-        for (int g = kg - STAGES < 0 ? 0 : kg - STAGES; g < kg; ++g)
-          mbar_wait(&full[g % STAGES], (uint32_t)(g / STAGES) & 1u, nullptr, status);
-    }
-  } else if (warp == 1) {
-    if (lane == 0 && rank == 0) {
-      constexpr uint32_t idesc = idesc_bf16_f32(256, Cfg::BN, false, false);
-      const uint32_t empty_peer0 = mapa_shared(smem_u32(&empty[0]), 1);
-      const uint32_t acc_full_peer0 = mapa_shared(smem_u32(&acc_full[0]), 1);
-      int kg = 0, i = 0;
-      bool ok = true;
-      PieceIter pit(cluster, n_clusters, n_tiles, job0.p.K / Cfg::BK, split);
-      Piece pc;
-      for (; ok && pit.next(pc); ++i) {
-        const int t = pc.t;
-        const int b = i & 1;
-        const bool j1 = t >= n_tiles0;
-        const int kb_begin = j1 ? 0 : pc.kb0;
-        const int kb_end = j1 ? job1.p.K / Cfg::BK : pc.kb1;
-        // both CTAs' epilogues are done with this buffer (first use passes at once)
-        if (!mbar_wait(&acc_empty[b], ((uint32_t)(i >> 1) & 1u) ^ 1u, abort_flag, status)) break;
-        tc_fence_after();
-        const uint32_t d = tmem + (uint32_t)(b * Cfg::BN);
-        for (int kb = kb_begin; kb < kb_end; ++kb, ++kg) {
-          const int s = kg % STAGES;
-          const uint32_t ph = (uint32_t)(kg / STAGES) & 1u;
-          if (!mbar_wait(&full[s], ph, abort_flag, status)) {
-            ok = false;
-            break;
-          }
+    } else if (warp == 1) {
+      if (lane == 0 && rank == 0) {
+        constexpr uint32_t idesc = idesc_bf16_f32(256, Cfg::BN, false, false);
+        const uint32_t empty_peer0 = mapa_shared(smem_u32(&empty[0]), 1);
+        const uint32_t acc_full_peer0 = mapa_shared(smem_u32(&acc_full[0]), 1);
+        int kg = 0, i = 0;
+        bool ok = true;
+        PieceIter<SPLIT> pit(cluster, n_clusters, n_tiles, job0.p.K / Cfg::BK, split);
+        Piece pc;
+        for (; ok && pit.next(pc); ++i) {
+          const int t = pc.t;
+          const int b = i & 1;
+          const bool j1 = t >= n_tiles0;
+          const int kb_begin = j1 ? 0 : pc.kb0;
+          const int kb_end = j1 ? job1.p.K / Cfg::BK : pc.kb1;
+          // both CTAs' epilogues are done with this buffer (first use passes at once)
+          if (!mbar_wait(&acc_empty[b], ((uint32_t)(i >> 1) & 1u) ^ 1u, abort_flag, status)) break;
           tc_fence_after();
-          const uint32_t a_addr = smem_u32(tiles + s * Cfg::STAGE_BYTES);
-          const uint32_t b_addr = a_addr + Cfg::A_BYTES;
-#pragma unroll
-          for (int k = 0; k < Cfg::BK / 16; ++k)
-            mma_ss_pair(d, sw128_desc(a_addr + k * 32, 16, 1024),
-                        sw128_desc(b_addr + k * 32, 16, 1024), idesc,
-                        (kb != kb_begin || k != 0) ? 1u : 0u);
-          mma_commit_pair(smem_u32(&empty[s]));
-          mma_commit_pair(empty_peer0 + s * 8);
+          const uint32_t d = tmem + (uint32_t)(b * Cfg::BN);
+          for (int kb = kb_begin; kb < kb_end; ++kb, ++kg) {
+            const int s = kg % STAGES;
+            const uint32_t ph = (uint32_t)(kg / STAGES) & 1u;
+            if (!mbar_wait(&full[s], ph, abort_flag, status)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t a_addr = smem_u32(tiles + s * Cfg::STAGE_BYTES);
+            const uint32_t b_addr = a_addr + Cfg::A_BYTES;
+  #pragma unroll
+            for (int k = 0; k < Cfg::BK / 16; ++k)
+              mma_ss_pair(d, sw128_desc(a_addr + k * 32, 16, 1024),
+                          sw128_desc(b_addr + k * 32, 16, 1024), idesc,
+                          (kb != kb_begin || k != 0) ? 1u : 0u);
+            mma_commit_pair(smem_u32(&empty[s]));
+            mma_commit_pair(empty_peer0 + s * 8);
+          }
+          if (!ok) break;
+          mma_commit_pair(smem_u32(&acc_full[b]));
+          mma_commit_pair(acc_full_peer0 + b * 8);
         }
-        if (!ok) break;
-        mma_commit_pair(smem_u32(&acc_full[b]));
-        mma_commit_pair(acc_full_peer0 + b * 8);
+        mma_commit_pair(smem_u32(drain));
+        mbar_wait(drain, 0, nullptr, status);  // all MMAs (and their arrives) done
       }
-      mma_commit_pair(smem_u32(drain));
-      mbar_wait(drain, 0, nullptr, status);  // all MMAs (and their arrives) done
     }
   } else {
+    regs_inc<Cfg::REGS_HIGH>();  // the two epilogue warpgroups
     const int q = warp & 3;        // TMEM lane quarter this warp may access
-    const int g = (warp - 2) >> 2;  // epilogue group: tile columns [128 g, 128 g + 128)
+    const int g = (warp - 4) >> 2;  // epilogue group: tile columns [128 g, 128 g + 128)
     const int row = q * 32 + lane;
-    const bool elected = (warp & 3) == 2 && lane == 0;  // warps 2 and 6
+    const bool elected = (warp & 3) == 0 && lane == 0;  // warps 4 and 8
     const uint32_t bar_id = 1 + (uint32_t)g;
     const uint32_t acc_empty_lead0 = mapa_shared(smem_u32(&acc_empty[0]), 0);
     griddep_wait();
@@ -895,8 +925,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(320, 1)
       decode(t, job, rp, n0);
       return has_res(job);
     };
-    PieceIter pit(cluster, n_clusters, n_tiles, job0.p.K / Cfg::BK, split);
-    PieceIter peek = pit;  // one piece ahead: the residual of the next piece loads early
+    PieceIter<SPLIT> pit(cluster, n_clusters, n_tiles, job0.p.K / Cfg::BK, split);
+    PieceIter<SPLIT> peek = pit;  // one piece ahead: the residual of the next piece loads early
     Piece pc, nx;
     bool has_next = peek.next(nx);
     auto needs_res = [&](const Piece& q) { return q.kind != 2 && res_of(q.t); };
@@ -918,17 +948,25 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(320, 1)
       const int pos = pc.kind == 2 ? 0
                       : job        ? pair_row_pos<EPI1>(jb.p, m0 + row, n0)
                                    : pair_row_pos<EPI0>(jb.p, m0 + row, n0);
+      float4 rt[16];  // first half of a RoPE head's (cos, sin) blocks
+      if (pc.kind != 2) {
+        if (job)
+          pair_rope_prefetch<EPI1>(jb.p, m0 + row, n0, pos, rt);
+        else
+          pair_rope_prefetch<EPI0>(jb.p, m0 + row, n0, pos, rt);
+      }
       bool ok = mbar_wait(&acc_full[b], (uint32_t)(i >> 1) & 1u, abort_flag, status);
       if (ok && with_res) ok = mbar_wait(&res_full[g], (uint32_t)res_used & 1u, abort_flag, status);
       if (with_res) ++res_used;
       // a finisher adds the partial sums of the tile's other pieces: the clusters whose
       // tail ranges start inside this tile, in k order
-      const float4* adds[kMaxPieces];
-      int add_cl[kMaxPieces];
+      constexpr int kAdd = SPLIT ? kMaxPieces : 1;
+      const float4* adds[kAdd];
+      int add_cl[kAdd];
       int n_add = 0;
-      if (pc.kind == 1) {
+      if (SPLIT && pc.kind == 1) {
         const int64_t lo = (int64_t)(t - split.dp_tiles) * nk0, hi = lo + nk0;
-        for (int c2 = cluster + 1; c2 < n_clusters && n_add < kMaxPieces; ++c2) {
+        for (int c2 = cluster + 1; c2 < n_clusters && n_add < kAdd; ++c2) {
           const int64_t b2 = split.tail_units * c2 / n_clusters;
           if (b2 >= hi) break;
           if (b2 > lo) {
@@ -948,7 +986,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(320, 1)
       if (!named_bar_and(bar_id, 128, ok)) break;
       tc_fence_after();
       const uint32_t tacc = tmem + (uint32_t)(b * Cfg::BN) + ((uint32_t)(q * 32) << 16);
-      if (pc.kind == 2) {
+      if (SPLIT && pc.kind == 2) {
         // contributor: the group's 128 raw accumulator columns go to this cluster's
         // partial block (float4 per 4 columns, row-contiguous: coalesced)
         float4* dst = split.part + (int64_t)((cluster * 2 + (int)rank) * 2 + g) * 32 * 128 + row;
@@ -979,11 +1017,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(320, 1)
       }
       if (late_ssq) rscale = pair_row_rscale(jb.p, m0 + row);
       if (job)
-        pair_epilogue_half<EPI1, kMaxPieces>(jb.p, out_s, tacc, row, m0 + row, n0, g, with_res,
-                                             rscale, pos, adds, n_add);
+        pair_epilogue_half<EPI1, kAdd>(jb.p, out_s, tacc, row, m0 + row, n0, g, with_res,
+                                             rscale, pos, rt, adds, n_add);
       else
-        pair_epilogue_half<EPI0, kMaxPieces>(jb.p, out_s, tacc, row, m0 + row, n0, g, with_res,
-                                             rscale, pos, adds, n_add);
+        pair_epilogue_half<EPI0, kAdd>(jb.p, out_s, tacc, row, m0 + row, n0, g, with_res,
+                                             rscale, pos, rt, adds, n_add);
       const bool publish = !job && chain.ready;  // job 1 waits for these rows
       if (publish) __threadfence();  // row sums of squares visible before the count
       tc_fence_before();

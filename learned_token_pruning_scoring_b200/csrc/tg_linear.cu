@@ -60,16 +60,38 @@ PairSplit plan_split(int64_t tiles, int nk, int clusters, void* ws, size_t ws_by
   return sp;
 }
 
+// The pair kernel's setmaxnreg split (PairCfg::REGS_LOW / REGS_HIGH) needs a launch
+// allocation of at least PairCfg::REGS_LAUNCH_MIN registers per thread; with fewer,
+// setmaxnreg.inc would wait forever, so such a build is refused before any launch.
+template <typename K>
+int pair_register_check(K kern, int& checked_dev) {
+  int dev = 0;
+  TG_CUDA_TRY(cudaGetDevice(&dev));
+  if (checked_dev == dev) return TG_OK;
+  cudaFuncAttributes fa;
+  TG_CUDA_TRY(cudaFuncGetAttributes(&fa, kern));
+  if (fa.numRegs < PairCfg<1>::REGS_LAUNCH_MIN || fa.maxThreadsPerBlock < PairCfg<1>::THREADS)
+    return TG_ERR_UNSUPPORTED_SHAPE;
+  checked_dev = dev;
+  return TG_OK;
+}
+
 template <int STAGES, int EPI>
 int launch_pair(const PairMaps& maps, const GemmParams& p, cudaStream_t stream,
                 void* ws = nullptr, size_t ws_bytes = 0) {
   using Cfg = PairCfg<STAGES>;
-  auto kern = gemm_pair_kernel<STAGES, EPI, EPI>;
+  auto kern = gemm_pair_kernel<STAGES, EPI, EPI, false>;
+  auto kern_split = gemm_pair_kernel<STAGES, EPI, EPI, true>;
+  static int regs_dev = -1, regs_dev_split = -1;
+  TG_TRY(pair_register_check(kern, regs_dev));
+  TG_TRY(pair_register_check(kern_split, regs_dev_split));
   static int attr_dev = -1;
   int dev = 0;
   TG_CUDA_TRY(cudaGetDevice(&dev));
   if (attr_dev != dev) {
     TG_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM));
+    TG_CUDA_TRY(cudaFuncSetAttribute(kern_split, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     Cfg::SMEM));
     attr_dev = dev;
   }
   PairJob j0{maps, p}, j1{};
@@ -97,7 +119,7 @@ int launch_pair(const PairMaps& maps, const GemmParams& p, cudaStream_t stream,
   cfg.attrs = attr;
   cfg.numAttrs = 2;
   const cudaError_t e =
-      cudaLaunchKernelEx(&cfg, kern, j0, j1, PairChain{nullptr, nullptr, 0}, sp);
+      cudaLaunchKernelEx(&cfg, kern_split, j0, j1, PairChain{nullptr, nullptr, 0}, sp);
   if (e != cudaSuccess) {
     set_cuda_error(e);
     return TG_ERR_CUDA;
@@ -112,7 +134,9 @@ template <int STAGES, int EPI0, int EPI1>
 int launch_pair_chain(const PairJob& j0, const PairJob& j1, const PairChain& chain,
                       cudaStream_t stream) {
   using Cfg = PairCfg<STAGES>;
-  auto kern = gemm_pair_kernel<STAGES, EPI0, EPI1>;
+  auto kern = gemm_pair_kernel<STAGES, EPI0, EPI1, false>;
+  static int regs_dev = -1;
+  TG_TRY(pair_register_check(kern, regs_dev));
   static int attr_dev = -1;
   int dev = 0;
   TG_CUDA_TRY(cudaGetDevice(&dev));
