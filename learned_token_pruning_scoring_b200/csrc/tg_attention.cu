@@ -199,7 +199,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* s_full = ax_ready + 2;         // [2]
   uint64_t* p_full = s_full + 2;           // [2]
   uint64_t* pv_done = p_full + 2;          // [2]
-  uint64_t* drain = pv_done + 2;
+  uint64_t* p_half = pv_done + 2;          // [2] P of the tile's first 64 keys stored
+  uint64_t* drain = p_half + 2;
   uint64_t* merge_full = drain + 1;        // a split tile's other part staged for the merge
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(merge_full + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -221,6 +222,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&ax_ready[h], 128);
       mbar_init(&s_full[h], 1);
       mbar_init(&p_full[h], 128);
+      mbar_init(&p_half[h], 128);
       mbar_init(&pv_done[h], 1);
     }
     mbar_init(drain, 1);
@@ -364,15 +366,18 @@ __global__ void __launch_bounds__(kThreads, 1)
                  bx_desc0 + (uint64_t)(((j % kStages) * kExBytes) >> 4), idesc_s, 1u);
           mma_commit(&s_full[hh]);
         };
-        auto issue_pv = [&](int hh, int j) {
+        // O += P V over the tile's keys [64 half, 64 half + 64): the first half as soon
+        // as the softmax has stored its P, while it computes the second
+        auto issue_pv = [&](int hh, int j, int half) {
           const uint64_t vd = v_desc0 + (uint64_t)(((j % kStages) * kTileBytes) >> 4);
 #pragma unroll
-          for (int kk = 0; kk < kBN / 16; ++kk) {
+          for (int q = 0; q < kBN / 32; ++q) {
+            const int kk = half * (kBN / 32) + q;
             // A = P (bf16 pairs in TMEM, 8 columns per 16 keys); B = V rows kk*16.. (MN-major)
             mma_ts(tmem + o_col[hh], tmem + s_col[hh] + kk * 8, vd + (uint64_t)((kk * 16 * 128) >> 4),
                    idesc_o, (j | kk) != 0);
           }
-          mma_commit(&pv_done[hh]);
+          if (half) mma_commit(&pv_done[hh]);
         };
         bool ok = mbar_wait(q_full, 0, abort_flag, p.status) &&
                   mbar_wait(&ax_ready[0], 0, abort_flag, p.status) &&
@@ -389,10 +394,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t ph = (uint32_t)(j / kStages) & 1u;
             const uint32_t pj = (uint32_t)j & 1u;
             ok = mbar_wait(&v_full[s], ph, abort_flag, p.status) &&
-                 mbar_wait(&p_full[0], pj, abort_flag, p.status);
+                 mbar_wait(&p_half[0], pj, abort_flag, p.status);
             if (!ok) break;
             tc_fence_after();
-            issue_pv(0, j);
+            issue_pv(0, j, 0);
+            if (!(ok = mbar_wait(&p_full[0], pj, abort_flag, p.status))) break;
+            tc_fence_after();
+            issue_pv(0, j, 1);
             const bool more = j + 1 < nt;
             if (more) {
               const int s2 = (j + 1) % kStages;
@@ -403,9 +411,12 @@ __global__ void __launch_bounds__(kThreads, 1)
               tc_fence_after();
               issue_s(0, j + 1);
             }
+            if (!(ok = mbar_wait(&p_half[1], pj, abort_flag, p.status))) break;
+            tc_fence_after();
+            issue_pv(1, j, 0);
             if (!(ok = mbar_wait(&p_full[1], pj, abort_flag, p.status))) break;
             tc_fence_after();
-            issue_pv(1, j);
+            issue_pv(1, j, 1);
             mma_commit(&v_empty[s]);
             if (more) {
               issue_s(1, j + 1);
@@ -467,6 +478,24 @@ __global__ void __launch_bounds__(kThreads, 1)
         m_run = mx;
         rescale = true;
       }
+      // O rescale, warp-uniform (tcgen05.ld/st are warp-collective; alpha = 1 on rows
+      // that keep their max), before any of this tile's P is released to the PV MMAs.
+      // PV(j-1) has retired: S(j) was committed after it.
+      if (__any_sync(0xFFFFFFFFu, rescale)) {
+        if (!(ok = warp_all(mbar_wait(&pv_done[wg], (uint32_t)(j - 1) & 1u, abort_flag,
+                                      p.status))))
+          break;
+        tc_fence_after();
+#pragma unroll 1
+        for (int c = 0; c < kD / 32; ++c) {
+          uint32_t ro[32];
+          tmem_ld32(o_t + c * 32, ro);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) ro[i] = __float_as_uint(__uint_as_float(ro[i]) * alpha);
+          tmem_st32(o_t + c * 32, ro);
+        }
+      }
       const uint64_t negm = f2pack(-m_run, -m_run);
       const uint64_t t2p = f2pack(t2, t2);
       uint64_t acc0 = f2pack(0.f, 0.f), acc1 = acc0;
@@ -485,28 +514,16 @@ __global__ void __launch_bounds__(kThreads, 1)
           pk[i] = pack_bf16x2(p0, p1);
         }
         tmem_st32(s_t + 32 * hf, pk);
+        if (hf == 0) {  // keys 0..63 (and any O rescale) are in TMEM: their PV may start
+          tmem_wait_st();
+          tc_fence_before();
+          mbar_arrive(&p_half[wg]);
+        }
       }
       float a0, a1, a2, a3;
       f2unpack(acc0, a0, a1);
       f2unpack(acc1, a2, a3);
       l_sum = l_sum * alpha + ((a0 + a1) + (a2 + a3));
-      // O rescale, warp-uniform (tcgen05.ld/st are warp-collective; alpha = 1 on rows
-      // that keep their max).  PV(j-1) has retired: S(j) was committed after it.
-      if (__any_sync(0xFFFFFFFFu, rescale)) {
-        if (!(ok = warp_all(mbar_wait(&pv_done[wg], (uint32_t)(j - 1) & 1u, abort_flag,
-                                      p.status))))
-          break;
-        tc_fence_after();
-#pragma unroll 1
-        for (int c = 0; c < kD / 32; ++c) {
-          uint32_t ro[32];
-          tmem_ld32(o_t + c * 32, ro);
-          tmem_wait_ld();
-#pragma unroll
-          for (int i = 0; i < 32; ++i) ro[i] = __float_as_uint(__uint_as_float(ro[i]) * alpha);
-          tmem_st32(o_t + c * 32, ro);
-        }
-      }
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&p_full[wg]);
