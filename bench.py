@@ -75,6 +75,9 @@ def parse_args():
     ap.add_argument("--also", default="n128k",
                     help="comma-separated workloads measured after the main one and "
                          "reported as sub-records of the same line ('' for none)")
+    ap.add_argument("--fuse-boundaries", choices=("on", "off"), default=None,
+                    help="one launch per layer boundary, the output projection and the next "
+                         "layer's QKV (tg_out_proj_qkv_next; default: the library's choice)")
     ap.add_argument("--rope-rows", choices=("on", "off"), default=None,
                     help="QKV RoPE from the per-row table of tg_rope_rows (default: the "
                          "library's choice)")
@@ -346,6 +349,8 @@ def measure(args, wl_name, rank, world, extras):
                            wl.rope_theta, device=dev, lower=lower)
     if args.rope_rows is not None:
         pipe.rope_rows = args.rope_rows == "on"
+    if args.fuse_boundaries is not None:
+        pipe.fuse_boundaries = args.fuse_boundaries == "on"
     P = pipe.plan(wl.lengths, wl.questions, wl.budgets)
     h_dev = h.to(dev)
     pr_dev = pr.to(dev)
