@@ -81,6 +81,11 @@ def parse_args():
     ap.add_argument("--rope-rows", choices=("on", "off"), default=None,
                     help="QKV RoPE from the per-row table of tg_rope_rows (default: the "
                          "library's choice)")
+    ap.add_argument("--k-pad", default=None,
+                    help="run the layers above the gate on a padded row count: an integer, "
+                         "or 'bucket' for the kept total rounded up to a multiple of 256 "
+                         "(the fixed-padding graph form; tokens/s still counts the input "
+                         "tokens, the padding rows are extra work)")
     ap.add_argument("--dense-steps", type=int, default=3,
                     help="timed steps of the full-context reference (0 skips it)")
     return ap.parse_args()
@@ -183,9 +188,18 @@ def kept_total(wl):
     return k
 
 
+def k_pad_rows(tg, wl, args):
+    """Padded row count of the layers above the gate (--k-pad), or None."""
+    if args.k_pad is None:
+        return None
+    if args.k_pad == "bucket":
+        return tg.k_bucket(kept_total(wl), 256)
+    return int(args.k_pad)
+
+
 def config_dict(wl, args, world):
     """The `config` of the JSON line, the same for both arms."""
-    return {"workload": wl.name, "batch": wl.batch,
+    out = {"workload": wl.name, "batch": wl.batch,
             "tokens_per_request": list(wl.lengths) if wl.batch <= 8 else None,
             "question_tokens": list(wl.questions) if wl.batch <= 8 else None,
             "kept": kept_total(wl), "gated_layers": wl.n_layers,
@@ -196,6 +210,11 @@ def config_dict(wl, args, world):
             "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
             "l2": "flushed before every timed step (512 MiB write, outside the timing)",
             "launch": "cuda_graph" if args.launch == "graph" else "eager"}
+    if getattr(args, "k_pad", None) is not None:
+        kp = args.k_pad
+        out["k_pad"] = (max(256, -(-kept_total(wl) // 256) * 256) if kp == "bucket"
+                        else int(kp))
+    return out
 
 
 def topk_latency_floor(tg, dev, stream, flush, reps=20):
@@ -351,7 +370,7 @@ def measure(args, wl_name, rank, world, extras):
         pipe.rope_rows = args.rope_rows == "on"
     if args.fuse_boundaries is not None:
         pipe.fuse_boundaries = args.fuse_boundaries == "on"
-    P = pipe.plan(wl.lengths, wl.questions, wl.budgets)
+    P = pipe.plan(wl.lengths, wl.questions, wl.budgets, k_pad=k_pad_rows(tg, wl, args))
     h_dev = h.to(dev)
     pr_dev = pr.to(dev)
     stream = torch.cuda.current_stream()

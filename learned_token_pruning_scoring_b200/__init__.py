@@ -32,7 +32,7 @@ __all__ = [
     "tg_swiglu", "tg_fold_norm_weight", "tg_pack_gate_up", "prepare_layer",
     "tg_gated_attention_bias_grad", "tg_gated_attention_bias_grad_workspace_size",
     "tg_gate_score_backward", "tg_gate_score_backward_workspace_size",
-    "GatedPrefill", "FullContextLayers", "LayerWeights", "STATUS_TIMEOUT", "STATUS_BUDGET",
+    "GatedPrefill", "FullContextLayers", "padded_layout", "k_bucket", "LayerWeights", "STATUS_TIMEOUT", "STATUS_BUDGET",
     "STATUS_BOUNDS", "STATUS_WORKSPACE",
 ]
 
@@ -153,6 +153,43 @@ def tg_plan_kept(cu_seqlens_host, n_question_host, budgets_host) -> torch.Tensor
     out = torch.zeros(batch + 1, dtype=torch.int32)
     _check(lib.tg_plan_kept(_ptr(cu), _ptr(nq), _ptr(bud), batch, _ptr(out)), "tg_plan_kept")
     return out
+
+
+def padded_layout(cu_kept_host, k_pad=None) -> torch.Tensor:
+    """Row layout of the layers above the gate (host int32 [B + 1]).
+
+    Without `k_pad` it is the kept layout itself.  With `k_pad` >= K (the kept total)
+    the last request takes k_pad - K extra trailing rows, so the layers always run on
+    k_pad rows and one CUDA graph of them serves every later call with the same layout
+    (for a single request: every kept total up to k_pad).  The pruned forward is
+    captured as a CUDA graph over a fixed padded size in "TokenGate: Adapting LLMs for
+    Fast and Memory-Efficient Prefill with Learned Token Pruning" (paper digest),
+    sections 方法关键点 and 工作参考价值.
+
+    Each kept row keeps its index, and as attention is causal within a request and the
+    padding rows follow every kept row of theirs, no kept row's keys include a padding
+    row.  Kept rows therefore get the unpadded results, up to the fp32 summation order
+    of the attention when the longer layout splits the key range differently."""
+    ckh = _host_i32(cu_kept_host).clone()
+    if k_pad is None:
+        return ckh
+    K = int(ckh[-1])
+    k_pad = int(k_pad)
+    if ckh.numel() < 2:
+        raise ValueError("padded_layout: the layout needs at least one request")
+    if k_pad < K:
+        raise ValueError(f"padded_layout: k_pad={k_pad} is below the kept total {K}")
+    ckh[-1] = k_pad
+    return ckh
+
+
+def k_bucket(K: int, granule: int = 256) -> int:
+    """The padded row count of a kept total: K rounded up to a multiple of `granule`
+    (at least one granule), so calls whose kept totals round to the same bucket share
+    one captured graph of the layers above the gate."""
+    if granule <= 0:
+        raise ValueError("k_bucket: granule must be positive")
+    return max(granule, -(-int(K) // granule) * granule)
 
 
 def tg_rope_table(max_pos: int, head_dim: int, theta: float, out=None, device=None,
@@ -762,12 +799,24 @@ class GatedPrefill:
         # accumulator wait, the 16k step takes 2.27 instead of 2.34 ms (one more launch)
         self.rope_rows = True
         self._qkv_done = -1  # index of the layer whose QKV already ran in a fused launch
+        self._graph = None   # CUDA graph of the layers above the gate (upper_layers(graph=True))
+        self._graph_key_cur = None
+        self.graph_captures = 0  # graphs captured by upper_layers(graph=True)
+        self._upper_gen = 0
 
     def _mark(self, name):
         if self.marker is not None:
             self.marker(name)
 
-    def plan(self, lengths, n_question, budgets):
+    def plan(self, lengths, n_question, budgets, k_pad=None):
+        """Fix the request layout and allocate the step's buffers.
+
+        `k_pad`: rows of the layers above the gate (>= the kept total K).  The layers then
+        run on a fixed row count whatever K a call keeps: rows [K, k_pad) are padding that
+        the last request takes as extra trailing rows (see `padded_layout`), so one CUDA
+        graph of those layers (`upper_layers(..., graph=True)`) serves every later plan
+        with the same padded layout.  A re-plan with the same padded layout keeps the
+        upper buffers (and the graph); only the gate's buffers follow the new lengths."""
         lengths = [int(x) for x in lengths]
         cu = [0]
         for n in lengths:
@@ -775,46 +824,75 @@ class GatedPrefill:
         cu_h = _host_i32(cu)
         ck_h = tg_plan_kept(cu_h, n_question, budgets)
         T, K = cu[-1], int(ck_h[-1])
+        up_h = padded_layout(ck_h, k_pad)
+        R = int(up_h[-1])
         dev = self.device
         max_pos = max(lengths) if lengths else 1
         if self.cos_sin is None or self.cos_sin.shape[0] < max_pos:
             self.cos_sin = tg_rope_table(max_pos, self.d, self.theta, device=dev)
         f32 = dict(dtype=torch.float32, device=dev)
-        bf = dict(dtype=torch.bfloat16, device=dev)
-        nqkv = (self.hq + 2 * self.hkv) * self.d
+        up_key = (tuple(up_h.tolist()), k_pad is not None)
+        prev = self.planned
+        if k_pad is not None and prev is not None and prev.get("up_key") == up_key:
+            upper = {k: prev[k] for k in self._UPPER_KEYS}
+        else:
+            upper = self._upper_buffers(up_h)
+        upper["up_key"] = up_key
+        if R > K:  # padding rows: h row 0 at position 0 with zero bias (finite, unused)
+            for k in ("kept_idx", "kept_pos", "kept_bias"):
+                upper[k][K:].zero_()
         self.planned = dict(
-            T=T, K=K, cu_h=cu_h, ck_h=ck_h,
+            T=T, K=K, R=R, cu_h=cu_h, ck_h=ck_h,
             cu=cu_h.to(dev), ck=ck_h.to(dev),
             s=torch.empty(T, **f32), z=torch.empty(T, **f32), bias=torch.empty(T, **f32),
             ws=torch.empty(tg_gate_score_workspace_size(T, self.hidden, self.width,
                                                         len(lengths)), dtype=torch.uint8,
                            device=dev),
-            kept_idx=torch.empty(K, dtype=torch.int32, device=dev),
-            kept_pos=torch.empty(K, dtype=torch.int32, device=dev),
-            kept_bias=torch.empty(K, **f32),
-            rot=torch.empty((self.d // 4, max(K, 1), 4), **f32),
-            x=torch.empty((K, self.hidden), **bf),
-            ssq=torch.empty((K, self.hidden // 128), **f32),
-            qkv=torch.empty((K, nqkv), **bf),
-            o=torch.empty((K, self.hq * self.d), **bf),
-            attn_ws=torch.zeros(tg_gated_attention_workspace_size(ck_h, self.hq, self.hkv, self.d),
-                                dtype=torch.uint8, device=dev),
-            caches=[(torch.empty((K, self.hkv * self.d), **bf),
-                     torch.empty((K, self.hkv * self.d), **bf)) for _ in self.layers],
-            chain_ws=torch.zeros(max(16, tg_out_proj_qkv_workspace_size(K)), dtype=torch.uint8,
-                                 device=dev),
-            # stream-K tail of the projections (zero-filled; empty = unsplit)
-            gemm_ws=torch.zeros(tg_gemm_workspace_size() if self.split_gemm else 0,
-                                dtype=torch.uint8, device=dev),
-            ffn=torch.empty((K, max([L.ffn for L in self.layers] + [0])), **bf),
+            **upper,
         )
         if self.lower is not None:
+            bf = dict(dtype=torch.bfloat16, device=dev)
             self.lower.plan(lengths, self.hidden)
             if self.trim_lower_kv:
                 self.planned["lower_caches"] = [
                     (torch.empty((K, self.hkv * self.d), **bf),
                      torch.empty((K, self.hkv * self.d), **bf)) for _ in self.lower.layers]
         return self.planned
+
+    _UPPER_KEYS = ("up_gen", "up_h", "up", "kept_idx", "kept_pos", "kept_bias", "rot", "x",
+                   "ssq", "qkv", "o", "attn_ws", "caches", "chain_ws", "gemm_ws", "ffn")
+
+    def _upper_buffers(self, up_h):
+        """Buffers of the layers above the gate for the row layout `up_h` (R rows)."""
+        R = int(up_h[-1])
+        dev = self.device
+        f32 = dict(dtype=torch.float32, device=dev)
+        bf = dict(dtype=torch.bfloat16, device=dev)
+        nqkv = (self.hq + 2 * self.hkv) * self.d
+        self._upper_gen += 1
+        return dict(
+            up_gen=self._upper_gen,  # which allocation these are (a graph is tied to one)
+            up_h=up_h, up=up_h.to(dev),
+            kept_idx=torch.zeros(R, dtype=torch.int32, device=dev),
+            kept_pos=torch.zeros(R, dtype=torch.int32, device=dev),
+            kept_bias=torch.zeros(R, **f32),
+            rot=torch.empty((self.d // 4, max(R, 1), 4), **f32),
+            x=torch.empty((R, self.hidden), **bf),
+            ssq=torch.empty((R, self.hidden // 128), **f32),
+            qkv=torch.empty((R, nqkv), **bf),
+            o=torch.empty((R, self.hq * self.d), **bf),
+            attn_ws=torch.zeros(tg_gated_attention_workspace_size(up_h, self.hq, self.hkv,
+                                                                  self.d),
+                                dtype=torch.uint8, device=dev),
+            caches=[(torch.empty((R, self.hkv * self.d), **bf),
+                     torch.empty((R, self.hkv * self.d), **bf)) for _ in self.layers],
+            chain_ws=torch.zeros(max(16, tg_out_proj_qkv_workspace_size(R)), dtype=torch.uint8,
+                                 device=dev),
+            # stream-K tail of the projections (zero-filled; empty = unsplit)
+            gemm_ws=torch.zeros(tg_gemm_workspace_size() if self.split_gemm else 0,
+                                dtype=torch.uint8, device=dev),
+            ffn=torch.empty((R, max([L.ffn for L in self.layers] + [0])), **bf),
+        )
 
     def score(self, h, prunable, stream=None):
         P = self.planned
@@ -893,7 +971,7 @@ class GatedPrefill:
             tg_prefetch_l2(L.Wo, stream=self._side)
             if i + 1 < len(self.layers):
                 tg_prefetch_l2(self.layers[i + 1].Wqkv, stream=self._side)
-        tg_gated_attention(qkv[:, :nq], ck, cv, P["ck"], P["ck_h"], self.hq, self.hkv,
+        tg_gated_attention(qkv[:, :nq], ck, cv, P["up"], P["up_h"], self.hq, self.hkv,
                            P["kept_pos"], P["kept_bias"], L.gamma, L.beta, o=o,
                            head_dim=self.d, workspace=P["attn_ws"], status=self.status,
                            stream=stream)
@@ -914,8 +992,7 @@ class GatedPrefill:
             self._mark("out_proj")
         _mlp(L, x, P, self.norm_eps, self.status, stream, self._mark)
 
-    def upper_layers(self, h, stream=None):
-        self.gather(h, stream=stream)
+    def _layers(self, stream=None):
         self._qkv_done = -1
         for i in range(len(self.layers)):
             self.layer(i, stream=stream, fuse_next=self.fuse_boundaries)
@@ -924,7 +1001,42 @@ class GatedPrefill:
             main = stream if stream is not None else torch.cuda.current_stream(self.device)
             main.wait_stream(self._side)
 
-    def run(self, h, prunable, scores=None, stream=None):
+    def _graph_key(self):
+        P = self.planned
+        # the position table is read inside the layers only without the per-row table
+        table = 0 if self.rope_rows else self.cos_sin.data_ptr()
+        return (P["up_key"], P["up_gen"], table, self.rope_rows, self.fuse_boundaries,
+                self.fused_qkv, self.prefetch_weights, tg_get_launch_overlap())
+
+    def upper_layers(self, h, stream=None, graph=False):
+        """The kept rows' way up: the gather, then every layer above the gate.
+
+        With `graph`, the layers (not the gather, whose source rows change from call to
+        call) run as one CUDA graph captured for the planned row layout.  The first such
+        call runs them eagerly and captures the graph; later calls with the same layout
+        (the same `k_pad` bucket and the same buffers) replay it."""
+        self.gather(h, stream=stream)
+        if not graph or self.planned["K"] == 0:
+            self._layers(stream)
+            return
+        main = stream if stream is not None else torch.cuda.current_stream(self.device)
+        key = self._graph_key()
+        if self._graph is not None and self._graph_key_cur == key:
+            with torch.cuda.stream(main):
+                self._graph.replay()
+            return
+        self._graph = None
+        self._layers(main)  # this call's result, and the kernels' one-time set-up
+        side = torch.cuda.Stream(device=self.device)
+        side.wait_stream(main)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=side):
+            self._layers(side)
+        main.wait_stream(side)
+        self._graph, self._graph_key_cur = g, key
+        self.graph_captures += 1
+
+    def run(self, h, prunable, scores=None, stream=None, graph=False):
         """One gated prefill step.  With lower layers, h is the model's input rows and
         the lower layers run first on all of them.  The scorer always runs on the
         gate layer's residual; with `scores` (raw per-token scores, fp32 [T]) selection
@@ -943,7 +1055,7 @@ class GatedPrefill:
         self.select(prunable, stream=stream)
         if self.lower is not None and self.trim_lower_kv:
             P = self.planned
-            self.lower.trim(P["kept_idx"], out=P["lower_caches"], stream=stream)
+            self.lower.trim(P["kept_idx"][:P["K"]], out=P["lower_caches"], stream=stream)
             self._mark("lower_kv_trim")
-        self.upper_layers(h, stream=stream)
+        self.upper_layers(h, stream=stream, graph=graph)
         return self.planned

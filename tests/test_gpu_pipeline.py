@@ -140,9 +140,11 @@ def _select_oracle_z(pipe, prd, z_ref, pr, cu, ck):
     z32 = z_ref.astype(np.float32)
     pipe.select(prd, z=torch.from_numpy(z32).to(prd.device))
     idx_ref, pos_ref, bias_ref = O.select_topk(z32, pr, cu, ck)
-    assert np.array_equal(P["kept_idx"].cpu().numpy(), idx_ref)
-    assert np.array_equal(P["kept_pos"].cpu().numpy(), pos_ref)
-    assert np.array_equal(P["kept_bias"].cpu().numpy().view(np.int32), bias_ref.view(np.int32))
+    K = P["K"]  # the buffers hold R >= K rows when the layers run on a padded layout
+    assert np.array_equal(P["kept_idx"][:K].cpu().numpy(), idx_ref)
+    assert np.array_equal(P["kept_pos"][:K].cpu().numpy(), pos_ref)
+    assert np.array_equal(P["kept_bias"][:K].cpu().numpy().view(np.int32),
+                          bias_ref.view(np.int32))
     return idx_ref, pos_ref, bias_ref
 
 
@@ -369,6 +371,63 @@ def test_launch_overlap_gives_identical_results(tg):
             assert torch.equal(got[k], ref[k]), k
         for (k0, v0), (k1, v1) in zip(got["caches"], ref["caches"]):
             assert torch.equal(k0, k1) and torch.equal(v0, v1)
+    assert tg.tg_status_read(pipe.status) == 0
+
+
+def test_padded_graph_serves_several_kept_totals(tg):
+    """The layers above the gate on a padded row count (k_pad = 1024), captured once as
+    a CUDA graph and replayed for three plans: kept totals 700, 1000 and 450, prompt
+    lengths 3000 and 2000.  Each plan's kept rows match the oracle run unpadded on that
+    plan (x after two layers, the first layer's K cache); the padding rows stay finite;
+    the graph is captured once."""
+    k_pad = 1024
+    plans = [S.custom([3000], [32], [700], n_layers=2, name="pad_a"),
+             S.custom([2000], [32], [1000], n_layers=2, seeds=[5], name="pad_b"),
+             S.custom([3000], [32], [450], n_layers=2, seeds=[9], name="pad_c")]
+    _, gate, layers, _, pipe = _setup(tg, plans[0])
+    for wl in plans:
+        h, pr = S.hidden_rows(wl), S.prunable_mask(wl)
+        hd, prd = h.cuda(), pr.cuda()
+        P = pipe.plan(wl.lengths, wl.questions, wl.budgets, k_pad=k_pad)
+        K = P["K"]
+        assert P["R"] == k_pad and P["up_h"].tolist() == [0, k_pad]
+        cu = wl.cu_seqlens()
+        ref = O.prefill(h, pr, cu, wl.budgets, gate, layers, wl.n_q_heads, wl.n_kv_heads,
+                        wl.head_dim, wl.rope_theta)
+        pipe.score(hd, prd)
+        _select_oracle_z(pipe, prd, ref["z"], pr.numpy(), cu, ref["cu_kept"])
+        pipe.upper_layers(hd, graph=True)
+        torch.cuda.synchronize()
+        _check_x(f"{wl.name} K={K} padded to {k_pad}", O.as_f64(P["x"][:K].cpu()), ref["x"],
+                 wl.n_layers)
+        k_ref = ref["caches"][0][0]
+        err = np.abs(O.as_f64(P["caches"][0][0][:K].cpu()).reshape(k_ref.shape) - k_ref)
+        assert err.max() <= 2.0 ** -6 * np.abs(k_ref).max()
+        assert torch.isfinite(P["x"][K:].float()).all()
+    assert pipe.graph_captures == 1
+    assert tg.tg_status_read(pipe.status) == 0
+
+
+def test_padded_layout_ragged_batch(tg):
+    """Two requests, kept totals 400 + 300, padded to 1024 rows (the second request takes
+    the 324 padding rows): eager layers and the graph replay both match the oracle on the
+    kept rows."""
+    wl = S.custom([1500, 900], [16, 8], [400, 300], n_layers=2, name="pad_ragged")
+    h, gate, layers, pr, pipe = _setup(tg, wl)
+    hd, prd = h.cuda(), pr.cuda()
+    P = pipe.plan(wl.lengths, wl.questions, wl.budgets, k_pad=1024)
+    assert P["up_h"].tolist() == [0, 400, 1024] and P["ck_h"].tolist() == [0, 400, 700]
+    cu = wl.cu_seqlens()
+    ref = O.prefill(h, pr, cu, wl.budgets, gate, layers, wl.n_q_heads, wl.n_kv_heads,
+                    wl.head_dim, wl.rope_theta)
+    pipe.score(hd, prd)
+    _select_oracle_z(pipe, prd, ref["z"], pr.numpy(), cu, ref["cu_kept"])
+    for graph in (False, True, True):  # eager; capture (runs eagerly); replay
+        pipe.upper_layers(hd, graph=graph)
+        torch.cuda.synchronize()
+        _check_x(f"ragged padded (graph={graph})", O.as_f64(P["x"][:700].cpu()), ref["x"],
+                 wl.n_layers)
+    assert pipe.graph_captures == 1
     assert tg.tg_status_read(pipe.status) == 0
 
 
