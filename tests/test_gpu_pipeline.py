@@ -473,10 +473,13 @@ def test_full_context_layers_against_oracle(tg, lengths):
     assert tg.tg_status_read(full.status) == 0
 
 
-def test_pipeline_with_lower_layers_and_kv_trim(tg):
+@pytest.mark.parametrize("k_pad", [None, 1536])
+def test_pipeline_with_lower_layers_and_kv_trim(tg, k_pad):
     """Two full-context layers, the gate on their output, selection on drawn scores
     (so that the kept set does not hinge on rounding), one gated layer above; the
-    lower caches trimmed to the kept rows."""
+    lower caches trimmed to the kept rows.  With `k_pad` the gated layer runs on 1536
+    rows (1200 kept) as a captured graph: the step runs twice, eagerly while capturing
+    and then from the graph, with identical results."""
     wl = S.custom([700, 1500, 333], [16, 64, 5], [100, 800, 300], n_layers=1,
                   planted_cluster=True, name="ragged3_lower")
     h = S.hidden_rows(wl)
@@ -487,10 +490,18 @@ def test_pipeline_with_lower_layers_and_kv_trim(tg):
     lower, full = _lower_setup(tg, wl, 2)
     pipe = tg.GatedPrefill(_dev_dict(gate), [_dev_dict(l) for l in upper], wl.n_q_heads,
                            wl.n_kv_heads, wl.head_dim, wl.rope_theta, lower=full)
-    P = pipe.plan(wl.lengths, wl.questions, wl.budgets)
+    P = pipe.plan(wl.lengths, wl.questions, wl.budgets, k_pad=k_pad)
     hd = h.cuda()
-    pipe.run(hd, pr.cuda(), scores=drawn.cuda())
+    graph = k_pad is not None
+    pipe.run(hd, pr.cuda(), scores=drawn.cuda(), graph=graph)
     torch.cuda.synchronize()
+    if graph:
+        first = P["x"].clone()
+        pipe.run(hd, pr.cuda(), scores=drawn.cuda(), graph=True)
+        torch.cuda.synchronize()
+        assert pipe.graph_captures == 1 and torch.equal(P["x"], first)
+        assert P["up_h"].tolist() == [0, 100, 900, k_pad]
+    K = P["K"]
     cu = wl.cu_seqlens()
     ref = O.prefill(h, pr, cu, wl.budgets, gate, upper, wl.n_q_heads, wl.n_kv_heads,
                     wl.head_dim, wl.rope_theta, scores=drawn, lower_layers=lower)
@@ -507,8 +518,8 @@ def test_pipeline_with_lower_layers_and_kv_trim(tg):
     same = _check_selection(wl, pr.numpy(), ref["z"], ref["cu_kept"],
                             P["kept_idx"].cpu().numpy(), P["ck_h"].numpy())
     assert same
-    kept = P["kept_idx"].cpu().numpy()
-    assert np.array_equal(P["kept_pos"].cpu().numpy(), ref["kept_pos"])
+    kept = P["kept_idx"][:K].cpu().numpy()
+    assert np.array_equal(P["kept_pos"][:K].cpu().numpy(), ref["kept_pos"])
     # trimmed lower caches: exactly the kept rows of the full-length ones, and those
     # against the oracle's trimmed caches
     for i, ((tk, tv), (fk, fv)) in enumerate(zip(P["lower_caches"], full.planned["caches"])):
@@ -517,7 +528,7 @@ def test_pipeline_with_lower_layers_and_kv_trim(tg):
         kc = O.as_f64(tk.cpu()).reshape(k_ref.shape)
         assert np.abs(kc - k_ref).max() <= 2.0 ** -6 * np.abs(k_ref).max()
     # one gated layer above: three layers of rounding in the residual stream
-    x = O.as_f64(P["x"].cpu())
+    x = O.as_f64(P["x"][:K].cpu())
     err = np.abs(x - ref["x"])
     tol, tol_mean = _x_tol(ref["x"], 3)
     assert np.all(err <= tol) and err.mean() <= tol_mean, (err.max(), err.mean())
