@@ -74,9 +74,11 @@ def parse_args():
     ap.add_argument("--scorer-bwd-steps", type=int, default=5,
                     help="timed calls of the scorer backward (parameter gradients from a "
                          "seeded d kept_bias; 0 skips it)")
-    ap.add_argument("--also", default="n128k",
+    ap.add_argument("--also", default="n128k,n16k@bucket",
                     help="comma-separated workloads measured after the main one and "
-                         "reported as sub-records of the same line ('' for none)")
+                         "reported as sub-records of the same line ('' for none); "
+                         "'name@bucket' or 'name@ROWS' runs the layers above the gate on a "
+                         "padded row count (the fixed-padding graph form)")
     ap.add_argument("--fuse-boundaries", choices=("on", "off"), default=None,
                     help="one launch per layer boundary, the output projection and the next "
                          "layer's QKV (tg_out_proj_qkv_next; default: the library's choice)")
@@ -193,16 +195,17 @@ def kept_total(wl):
     return k
 
 
-def k_pad_rows(tg, wl, args):
-    """Padded row count of the layers above the gate (--k-pad), or None."""
-    if args.k_pad is None:
+def k_pad_rows(wl, spec):
+    """Padded row count of the layers above the gate for a --k-pad value ('bucket': the
+    kept total rounded up to a multiple of 256, the library's k_bucket), or None."""
+    if spec is None:
         return None
-    if args.k_pad == "bucket":
-        return tg.k_bucket(kept_total(wl), 256)
-    return int(args.k_pad)
+    if spec == "bucket":
+        return max(256, -(-kept_total(wl) // 256) * 256)
+    return int(spec)
 
 
-def config_dict(wl, args, world):
+def config_dict(wl, args, world, k_pad=None):
     """The `config` of the JSON line, the same for both arms."""
     out = {"workload": wl.name, "batch": wl.batch,
             "tokens_per_request": list(wl.lengths) if wl.batch <= 8 else None,
@@ -215,10 +218,9 @@ def config_dict(wl, args, world):
             "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
             "l2": "flushed before every timed step (512 MiB write, outside the timing)",
             "launch": "cuda_graph" if args.launch == "graph" else "eager"}
-    if getattr(args, "k_pad", None) is not None:
-        kp = args.k_pad
-        out["k_pad"] = (max(256, -(-kept_total(wl) // 256) * 256) if kp == "bucket"
-                        else int(kp))
+    rows = k_pad_rows(wl, k_pad if k_pad is not None else getattr(args, "k_pad", None))
+    if rows is not None:
+        out["k_pad"] = rows
     return out
 
 
@@ -325,7 +327,10 @@ def run_ours(args, rank, world):
     for name in [w for w in args.also.split(",") if w and w != args.workload]:
         torch.cuda.empty_cache()
         sub = measure(args, name, rank, world, extras=False)
-        subs[sub["config"]["workload"]] = {k: sub[k] for k in (
+        key = sub["config"]["workload"]
+        if "k_pad" in sub["config"]:
+            key += f"@k_pad{sub['config']['k_pad']}"
+        subs[key] = {k: sub[k] for k in (
             "value", "unit", "ms_per_step", "steps", "warmup", "config", "e2e", "gpu_launches",
             "roofline", "rooflines", "stages", "clocks")}
     if subs:
@@ -343,6 +348,9 @@ def measure(args, wl_name, rank, world, extras):
     import synthetic_inputs as S
 
     dev = torch.device("cuda", torch.cuda.current_device())
+    # "name@pad": the workload with the layers above the gate on a padded row count
+    wl_name, _, pad_spec = wl_name.partition("@")
+    pad_spec = pad_spec or args.k_pad
     wl = workload(wl_name)
     # replicas: rank r draws its own batch (seed offset), same weights
     wl = replica_workload(wl, rank, world)
@@ -375,7 +383,7 @@ def measure(args, wl_name, rank, world, extras):
         pipe.rope_rows = args.rope_rows == "on"
     if args.fuse_boundaries is not None:
         pipe.fuse_boundaries = args.fuse_boundaries == "on"
-    P = pipe.plan(wl.lengths, wl.questions, wl.budgets, k_pad=k_pad_rows(tg, wl, args))
+    P = pipe.plan(wl.lengths, wl.questions, wl.budgets, k_pad=k_pad_rows(wl, pad_spec))
     h_dev = h.to(dev)
     pr_dev = pr.to(dev)
     stream = torch.cuda.current_stream()
@@ -624,7 +632,7 @@ def measure(args, wl_name, rank, world, extras):
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": config_dict(wl, args, world),
+        "config": config_dict(wl, args, world, pad_spec),
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "steps": e2e_steps_done,
                 "copies": "double-buffered: next step's H2D and this step's D2H overlap the "
