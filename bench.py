@@ -82,6 +82,9 @@ def parse_args():
     ap.add_argument("--fuse-boundaries", choices=("on", "off"), default=None,
                     help="one launch per layer boundary, the output projection and the next "
                          "layer's QKV (tg_out_proj_qkv_next; default: the library's choice)")
+    ap.add_argument("--launch-overlap", choices=("on", "off"), default=None,
+                    help="programmatic dependent launch between the library's kernels "
+                         "(tg_set_launch_overlap; default: the library's choice)")
     ap.add_argument("--rope-rows", choices=("on", "off"), default=None,
                     help="QKV RoPE from the per-row table of tg_rope_rows (default: the "
                          "library's choice)")
@@ -381,6 +384,8 @@ def measure(args, wl_name, rank, world, extras):
                            wl.rope_theta, device=dev, lower=lower)
     if args.rope_rows is not None:
         pipe.rope_rows = args.rope_rows == "on"
+    if args.launch_overlap is not None:
+        tg.tg_set_launch_overlap(args.launch_overlap == "on")
     if args.fuse_boundaries is not None:
         pipe.fuse_boundaries = args.fuse_boundaries == "on"
     P = pipe.plan(wl.lengths, wl.questions, wl.budgets, k_pad=k_pad_rows(wl, pad_spec))

@@ -70,7 +70,7 @@ int make_tmap_bf16_2d_swz(CUtensorMap* out, const void* base, uint64_t rows, uin
 }
 
 namespace {
-std::atomic<int> g_launch_overlap{0};
+std::atomic<int> g_launch_overlap{1};
 std::atomic<int> g_gather_tma{0};
 std::atomic<int> g_scorer_pair{1};
 }

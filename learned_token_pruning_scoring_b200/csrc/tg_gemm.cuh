@@ -803,6 +803,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
   cluster_sync_all();  // barriers of both CTAs initialised before any remote arrive
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // Past the previous grid: the next one may be scheduled on the SMs this grid leaves
+  // free (all of its clusters are resident, one wave), to wait there for its completion.
+  griddep_wait();
+  griddep_launch_dependents();
   if (warp < 4) {
     regs_dec<Cfg::REGS_LOW>();  // warpgroup 0: producer, MMA issuer, two idle warps
     if (warp == 0) {

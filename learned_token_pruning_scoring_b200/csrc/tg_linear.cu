@@ -294,6 +294,7 @@ __global__ void pack_rows_kernel(const uint16_t* __restrict__ a, int64_t lda,
                                  const uint16_t* __restrict__ b, int64_t ldb, int64_t rows,
                                  int cols, const float* __restrict__ norm_w,
                                  uint16_t* __restrict__ out, int64_t ld_out, int interleave) {
+  griddep_wait();  // the weights may come from an earlier grid
   const int64_t n = rows * cols;
   for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n;
        i += (int64_t)gridDim.x * blockDim.x) {

@@ -42,11 +42,21 @@ __device__ __forceinline__ uint32_t lane_id() {
 // thread's generic accesses; the proxy fence after it extends that to the TMA loads
 // (async proxy) the thread issues next, which a kernel boundary would otherwise order.
 // Every kernel of this library calls it before touching global memory that another
-// grid may write.  None of them signals an earlier start
-// (griddepcontrol.launch_dependents): letting the next grid's CTAs occupy SMs while this
-// grid still runs was measured to slow the attention kernels.
+// grid may write.
 __device__ __forceinline__ void griddep_wait() {
   asm volatile("griddepcontrol.wait;\n\tfence.proxy.async.global;" ::: "memory");
+}
+
+// Lets the next grid in the stream (if launched with programmatic stream serialisation)
+// be scheduled once every CTA of this grid has signalled or exited; its CTAs then take
+// only SMs this grid leaves free and wait in griddep_wait() until this grid completes.
+// Signalled only by the persistent CTA-pair GEMM, whose grid never exceeds one wave of
+// clusters: a grid with CTAs still to launch must not signal, or the next grid's waiting
+// CTAs could take the SMs those CTAs need.  The attention kernel (a second wave when the
+// key range is split) does not signal: letting the next grid in early was measured to
+// slow it.
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
 // ------------------------------------------------------------------ mbarrier
