@@ -431,6 +431,35 @@ def test_padded_layout_ragged_batch(tg):
     assert tg.tg_status_read(pipe.status) == 0
 
 
+def test_padded_layout_edge_cases(tg):
+    """k_pad equal to the kept total (no padding rows: the layout is the kept layout and
+    the graph run matches the oracle), and a plan that keeps nothing (K = 0 with 256
+    padded rows: the step launches no layer and reports no error)."""
+    wl = S.custom([600], [8], [150], n_layers=2, name="pad_exact")
+    h, gate, layers, pr, pipe = _setup(tg, wl)
+    hd, prd = h.cuda(), pr.cuda()
+    P = pipe.plan(wl.lengths, wl.questions, wl.budgets, k_pad=150)
+    assert P["K"] == P["R"] == 150 and P["up_h"].tolist() == P["ck_h"].tolist()
+    cu = wl.cu_seqlens()
+    ref = O.prefill(h, pr, cu, wl.budgets, gate, layers, wl.n_q_heads, wl.n_kv_heads,
+                    wl.head_dim, wl.rope_theta)
+    pipe.score(hd, prd)
+    _select_oracle_z(pipe, prd, ref["z"], pr.numpy(), cu, ref["cu_kept"])
+    pipe.upper_layers(hd, graph=True)
+    torch.cuda.synchronize()
+    _check_x("k_pad = K", O.as_f64(P["x"].cpu()), ref["x"], wl.n_layers)
+    assert pipe.graph_captures == 1
+
+    wl0 = S.custom([300], [0], [0], n_layers=2, name="pad_none_kept")
+    h0 = S.hidden_rows(wl0)
+    P = pipe.plan(wl0.lengths, wl0.questions, wl0.budgets, k_pad=256)
+    assert P["K"] == 0 and P["R"] == 256
+    pipe.run(h0.cuda(), S.prunable_mask(wl0).cuda(), graph=True)
+    torch.cuda.synchronize()
+    assert pipe.graph_captures == 1  # nothing to capture
+    assert tg.tg_status_read(pipe.status) == 0
+
+
 # ------------------------------------------------------------------ layers below the gate
 #
 # Tolerances for the full-context layers, derived by `tests/tolerance_study.py lower`
